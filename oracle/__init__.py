@@ -1,0 +1,181 @@
+"""fp64 CPU oracle for chunkwise Gated DeltaNet — TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py`` (its CPU-baseline
+and reference legs) may import this package. It shares no code with the CUDA
+library: the arithmetic lives in ``gdn_oracle.c`` (plain C, IEEE double, no
+fast-math), compiled here with gcc and called through ctypes.
+
+Functions (each cites the passages it follows in ``gdn_oracle.c``):
+  recurrent_fwd  token-by-token recurrence, the definition of the operator
+  decode_step    one token for many independent heads, state in place
+  chunked_fwd    fp64 chunkwise re-derivation (UT/WY form) for invariance tests
+  ut_transform   the per-chunk T = (I + A)^-1 factor
+
+Pins (tests/test_oracle_pins.py) tie these to what the pages fix: the masked
+parallel form, the positions 1-4 cumulative-sum example, the delta rule as one
+gradient step, exact key->value recall, the Householder reflection, brute-force
+transition products, the WY product form and chunk-size invariance.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+from typing import Optional
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gdn_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def compile_c(src: str, out: str) -> str:
+    """gcc -O2 (no fast-math, no FMA contraction) of one C file into a shared library."""
+    tmp = out + f".tmp{os.getpid()}"
+    subprocess.check_call(["gcc", "-O2", "-fno-fast-math", "-ffp-contract=off", "-std=c11",
+                           "-fPIC", "-shared", "-o", tmp, src, "-lm", "-lpthread"])
+    os.replace(tmp, out)
+    return out
+
+
+def build(force: bool = False) -> str:
+    """Compile gdn_oracle.c into liboracle.so when missing or stale."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        compile_c(_SRC, _LIB_PATH)
+    return _LIB_PATH
+
+
+def load_variant(path: str):
+    """Bind a separately compiled copy of the oracle (used to plant mistakes in tests)."""
+    return _bind(path)
+
+
+def _bind(path: str):
+    lib = ctypes.CDLL(path)
+    P = ctypes.c_void_p
+    l, d, i = ctypes.c_long, ctypes.c_double, ctypes.c_int
+    lib.oracle_recurrent_fwd.argtypes = [P, P, P, P, P, P, P, P, l, l, l, l, d, i]
+    lib.oracle_decode_step.argtypes = [P, P, P, P, P, P, P, l, l, l, d, i]
+    lib.oracle_chunked_fwd.argtypes = [P, P, P, P, P, P, P, P, l, l, l, l, l, d, i]
+    lib.oracle_ut_transform.argtypes = [P, P, P, P, l, l]
+    for f in (lib.oracle_recurrent_fwd, lib.oracle_decode_step, lib.oracle_chunked_fwd,
+              lib.oracle_ut_transform):
+        f.restype = ctypes.c_int
+    return lib
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            _lib = _bind(build())
+    return _lib
+
+
+def default_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def _f64(x) -> Optional[np.ndarray]:
+    """Exact upcast of a torch tensor / array (bf16, fp32, fp64) to C-contiguous fp64."""
+    if x is None:
+        return None
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            x = x.detach().to("cpu", torch.float64).numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def recurrent_fwd(q, k, v, beta=None, g=None, s0=None, scale: float = 1.0,
+                  nthreads: Optional[int] = None, lib=None):
+    """Token-by-token fp64 recurrence.
+
+    q, k: (..., L, dk); v: (..., L, dv); beta, g: (..., L) or None; s0: (..., dk, dv)
+    or None. Returns (o (..., L, dv), S_final (..., dk, dv)) as float64 arrays.
+    """
+    q, k, v, beta, g, s0 = map(_f64, (q, k, v, beta, g, s0))
+    lead = q.shape[:-2]
+    L, dk = q.shape[-2:]
+    dv = v.shape[-1]
+    BH = int(np.prod(lead)) if lead else 1
+    o = np.zeros(lead + (L, dv), np.float64)
+    sf = np.zeros(lead + (dk, dv), np.float64)
+    rc = (lib or _load()).oracle_recurrent_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(s0),
+                                      _ptr(o), _ptr(sf), BH, L, dk, dv, float(scale),
+                                      nthreads or default_threads())
+    if rc:
+        raise ValueError("oracle_recurrent_fwd: bad sizes")
+    return o, sf
+
+
+def decode_step(q, k, v, beta, g, state: np.ndarray, scale: float = 1.0,
+                nthreads: Optional[int] = None, lib=None):
+    """One decode token for every head; ``state`` (fp64, (..., dk, dv)) is updated in place.
+
+    q, k: (..., dk); v: (..., dv); beta, g: (...) or None. Returns o (..., dv).
+    """
+    q, k, v, beta, g = map(_f64, (q, k, v, beta, g))
+    assert state.dtype == np.float64 and state.flags.c_contiguous
+    lead = q.shape[:-1]
+    dk, dv = state.shape[-2:]
+    NH = int(np.prod(lead)) if lead else 1
+    o = np.zeros(lead + (dv,), np.float64)
+    rc = (lib or _load()).oracle_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(state),
+                                    _ptr(o), NH, dk, dv, float(scale), nthreads or default_threads())
+    if rc:
+        raise ValueError("oracle_decode_step: bad sizes")
+    return o
+
+
+def chunked_fwd(q, k, v, beta=None, g=None, s0=None, chunk: int = 64, scale: float = 1.0,
+                nthreads: Optional[int] = None, lib=None):
+    """fp64 chunkwise (UT/WY) form; same contract as :func:`recurrent_fwd`."""
+    q, k, v, beta, g, s0 = map(_f64, (q, k, v, beta, g, s0))
+    lead = q.shape[:-2]
+    L, dk = q.shape[-2:]
+    dv = v.shape[-1]
+    BH = int(np.prod(lead)) if lead else 1
+    o = np.zeros(lead + (L, dv), np.float64)
+    sf = np.zeros(lead + (dk, dv), np.float64)
+    rc = (lib or _load()).oracle_chunked_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(s0),
+                                    _ptr(o), _ptr(sf), BH, L, dk, dv, int(chunk), float(scale),
+                                    nthreads or default_threads())
+    if rc:
+        raise ValueError("oracle_chunked_fwd: bad sizes")
+    return o, sf
+
+
+def ut_transform(K, beta, g=None, lib=None):
+    """T = (I + A)^-1 for one chunk (K: n x dk, beta: n, g: n or None)."""
+    K, beta, g = map(_f64, (K, beta, g))
+    n, dk = K.shape
+    T = np.zeros((n, n), np.float64)
+    rc = (lib or _load()).oracle_ut_transform(_ptr(K), _ptr(beta), _ptr(g), _ptr(T), n, dk)
+    if rc:
+        raise ValueError("oracle_ut_transform: bad sizes")
+    return T
+
+
+def max_norm_err(x, ref) -> float:
+    """max|x - ref| / max|ref| over the whole tensor (0 when both are all-zero)."""
+    x = _f64(x)
+    ref = _f64(ref)
+    den = float(np.max(np.abs(ref))) if ref.size else 0.0
+    num = float(np.max(np.abs(x - ref))) if ref.size else 0.0
+    if den == 0.0:
+        return num
+    return num / den

@@ -1,0 +1,171 @@
+"""ctypes binding of libgdn.so (the C ABI declared in include/gdn.h).
+
+Argument marshalling only: tensors are checked for dtype, shape, device and
+contiguity, their data pointers and sizes are passed to the C entry points, and a
+non-OK status raises. Every step of the computation runs in the library's CUDA
+kernels; there is no other code path. The library must be built
+(``python -m gated_deltanet_sequence_b200.build``); if it is missing, importing this
+module raises ImportError.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgdn.so")
+
+GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_TIMEOUT = range(5)
+GDN_F32, GDN_BF16 = 0, 1
+
+EXPORTS = ("lin_attn_chunk_fwd", "gdn_chunk_fwd", "gdn_decode_step", "gdn_status_str",
+           "gdn_sync_status", "gdn_version")
+
+
+class GdnError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {status_str(status)} ({status})")
+        self.status = status
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libgdn.so is not built ({LIB_PATH}); run "
+                          "`python -m gated_deltanet_sequence_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.lin_attn_chunk_fwd.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
+    lib.gdn_chunk_fwd.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
+    lib.gdn_decode_step.argtypes = [P, P, P, P, P, P, P, I, I, I, I, F, I, P]
+    lib.gdn_status_str.argtypes = [I]
+    lib.gdn_status_str.restype = ctypes.c_char_p
+    lib.gdn_sync_status.argtypes = [P]
+    lib.gdn_version.argtypes = []
+    for f in (lib.lin_attn_chunk_fwd, lib.gdn_chunk_fwd, lib.gdn_decode_step, lib.gdn_sync_status,
+              lib.gdn_version):
+        f.restype = ctypes.c_int
+    return lib
+
+
+lib = _load()
+
+
+def status_str(status: int) -> str:
+    return lib.gdn_status_str(int(status)).decode()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return GDN_BF16
+    if t.dtype == torch.float32:
+        return GDN_F32
+    raise TypeError(f"q/k/v must be bfloat16 or float32, got {t.dtype}")
+
+
+def _check(name: str, t: Optional[torch.Tensor], shape, dtype=None, device=None, required=True):
+    if t is None:
+        if required:
+            raise ValueError(f"{name} is required")
+        return
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
+
+
+def _raise(fn: str, st: int):
+    if st != GDN_OK:
+        raise GdnError(fn, st)
+
+
+def lin_attn_chunk_fwd(q, k, v, g=None, o=None, s0=None, s_final=None, chunk: int = 64,
+                       scale: float = 1.0, stream=None):
+    """Plain (g None) or gated causal linear attention. Returns (o, s_final)."""
+    B, H, L, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    _check("q", q, (B, H, L, dk), device=dev)
+    _check("k", k, (B, H, L, dk), q.dtype, dev)
+    _check("v", v, (B, H, L, dv), q.dtype, dev)
+    _check("g", g, (B, H, L), torch.float32, dev, required=False)
+    _check("s0", s0, (B, H, dk, dv), torch.float32, dev, required=False)
+    if o is None:
+        o = torch.empty(B, H, L, dv, dtype=torch.float32, device=dev)
+    _check("o", o, (B, H, L, dv), torch.float32, dev)
+    _check("s_final", s_final, (B, H, dk, dv), torch.float32, dev, required=False)
+    st = lib.lin_attn_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(o), _ptr(s0),
+                                _ptr(s_final), B, H, L, dk, dv, int(chunk), float(scale),
+                                _dtype_code(q), _stream(stream))
+    _raise("lin_attn_chunk_fwd", st)
+    return o, s_final
+
+
+def gdn_chunk_fwd(q, k, v, beta, g=None, o=None, s0=None, s_final=None, chunk: int = 64,
+                  scale: float = 1.0, stream=None):
+    """DeltaNet (g None) or Gated DeltaNet chunkwise prefill. Returns (o, s_final)."""
+    B, H, L, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    _check("q", q, (B, H, L, dk), device=dev)
+    _check("k", k, (B, H, L, dk), q.dtype, dev)
+    _check("v", v, (B, H, L, dv), q.dtype, dev)
+    _check("beta", beta, (B, H, L), torch.float32, dev, required=L > 0)
+    _check("g", g, (B, H, L), torch.float32, dev, required=False)
+    _check("s0", s0, (B, H, dk, dv), torch.float32, dev, required=False)
+    if o is None:
+        o = torch.empty(B, H, L, dv, dtype=torch.float32, device=dev)
+    _check("o", o, (B, H, L, dv), torch.float32, dev)
+    _check("s_final", s_final, (B, H, dk, dv), torch.float32, dev, required=False)
+    st = lib.gdn_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(o), _ptr(s0),
+                           _ptr(s_final), B, H, L, dk, dv, int(chunk), float(scale),
+                           _dtype_code(q), _stream(stream))
+    _raise("gdn_chunk_fwd", st)
+    return o, s_final
+
+
+def gdn_decode_step(q, k, v, beta, g, state, o=None, scale: float = 1.0, stream=None):
+    """One decode token for (N, H) heads; ``state`` (N, H, dk, dv) fp32 is updated in place."""
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    _check("q", q, (N, H, dk), device=dev)
+    _check("k", k, (N, H, dk), q.dtype, dev)
+    _check("v", v, (N, H, dv), q.dtype, dev)
+    _check("beta", beta, (N, H), torch.float32, dev, required=False)
+    _check("g", g, (N, H), torch.float32, dev, required=False)
+    _check("state", state, (N, H, dk, dv), torch.float32, dev)
+    if o is None:
+        o = torch.empty(N, H, dv, dtype=torch.float32, device=dev)
+    _check("o", o, (N, H, dv), torch.float32, dev)
+    st = lib.gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(state),
+                             _ptr(o), N, H, dk, dv, float(scale), _dtype_code(q), _stream(stream))
+    _raise("gdn_decode_step", st)
+    return o
+
+
+def gdn_sync_status(stream=None) -> int:
+    """Synchronise the stream; return the library's status word (GDN_OK / GDN_ERR_TIMEOUT / ...)."""
+    return lib.gdn_sync_status(_stream(stream))
+
+
+def gdn_version() -> int:
+    return lib.gdn_version()

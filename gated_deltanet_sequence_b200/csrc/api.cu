@@ -1,0 +1,101 @@
+// C-ABI entry points of libgdn.so: argument validation and kernel dispatch.
+// Every launch goes on the caller's stream; nothing here allocates memory.
+#include <math.h>
+
+#include "common.cuh"
+#include "tc_kernels.cuh"
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool opt_aligned16(const void *p) { return p == nullptr || aligned16(p); }
+bool head_dim_ok(int d) { return d == 64 || d == 128; }
+
+gdn_status_t check_prefill(const void *q, const void *k, const void *v, const float *g, float *o,
+                           const float *s0, float *s_final, int B, int H, int L, int dk, int dv,
+                           int chunk, float scale, gdn_dtype_t in_dtype) {
+    if (B < 1 || H < 1 || L < 0 || !isfinite(scale)) return GDN_ERR_INVALID_ARG;
+    if (in_dtype != GDN_F32 && in_dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (L > 0 && (!q || !k || !v || !o)) return GDN_ERR_INVALID_ARG;
+    if (!opt_aligned16(q) || !opt_aligned16(k) || !opt_aligned16(v) || !opt_aligned16(o) ||
+        !opt_aligned16(g) || !opt_aligned16(s0) || !opt_aligned16(s_final))
+        return GDN_ERR_INVALID_ARG;
+    if (chunk < 1) return GDN_ERR_INVALID_ARG;
+    if (!head_dim_ok(dk) || !head_dim_ok(dv) || chunk > 64) return GDN_ERR_UNSUPPORTED;
+    // every element offset must fit the kernels' 64-bit index arithmetic and the
+    // per-head length must fit a 32-bit token index
+    const double elems = (double)B * H * (double)L * (dk > dv ? dk : dv);
+    if (elems > 9.0e18 || (double)B * H > 2147483647.0) return GDN_ERR_INVALID_ARG;
+    return GDN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *gdn_status_str(gdn_status_t s) {
+    switch (s) {
+        case GDN_OK: return "GDN_OK";
+        case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG";
+        case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED";
+        case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
+        case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT";
+    }
+    return "GDN_ERR_UNKNOWN";
+}
+
+int gdn_version(void) { return 100; }
+
+gdn_status_t lin_attn_chunk_fwd(const void *q, const void *k, const void *v, const float *g,
+                                float *o, const float *s0, float *s_final, int B, int H, int L,
+                                int dk, int dv, int chunk, float scale, gdn_dtype_t in_dtype,
+                                void *cuda_stream) {
+    gdn_status_t st = check_prefill(q, k, v, g, o, s0, s_final, B, H, L, dk, dv, chunk, scale, in_dtype);
+    if (st != GDN_OK) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+    if (gdn::tc_supported(in_dtype, dk, dv, chunk) && L > 0)
+        return gdn::launch_tc_la(q, k, v, g, o, s0, s_final, B, H, L, scale, stream);
+    return gdn::launch_simt_fwd(q, k, v, nullptr, g, o, s0, s_final, B, H, L, dk, dv, chunk, scale,
+                                in_dtype, stream);
+}
+
+gdn_status_t gdn_chunk_fwd(const void *q, const void *k, const void *v, const float *beta,
+                           const float *g, float *o, const float *s0, float *s_final, int B, int H,
+                           int L, int dk, int dv, int chunk, float scale, gdn_dtype_t in_dtype,
+                           void *cuda_stream) {
+    gdn_status_t st = check_prefill(q, k, v, g, o, s0, s_final, B, H, L, dk, dv, chunk, scale, in_dtype);
+    if (st != GDN_OK) return st;
+    if (L > 0 && !beta) return GDN_ERR_INVALID_ARG;
+    if (!opt_aligned16(beta)) return GDN_ERR_INVALID_ARG;
+    cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+    if (gdn::tc_supported(in_dtype, dk, dv, chunk) && L > 0)
+        return gdn::launch_tc_gdn(q, k, v, beta, g, o, s0, s_final, B, H, L, scale, stream);
+    // with L == 0 beta may be NULL: the kernel then only writes s0 (or zeros) to s_final
+    return gdn::launch_simt_fwd(q, k, v, beta, g, o, s0, s_final, B, H, L, dk, dv, chunk, scale,
+                                in_dtype, stream);
+}
+
+gdn_status_t gdn_decode_step(const void *q, const void *k, const void *v, const float *beta,
+                             const float *g, float *state, float *o, int N, int H, int dk, int dv,
+                             float scale, gdn_dtype_t in_dtype, void *cuda_stream) {
+    if (N < 1 || H < 1 || !isfinite(scale)) return GDN_ERR_INVALID_ARG;
+    if (in_dtype != GDN_F32 && in_dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (!q || !k || !v || !state || !o) return GDN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(state) || !aligned16(o) ||
+        !opt_aligned16(beta) || !opt_aligned16(g))
+        return GDN_ERR_INVALID_ARG;
+    if (!head_dim_ok(dk) || !head_dim_ok(dv)) return GDN_ERR_UNSUPPORTED;
+    if ((double)N * H > 2147483647.0) return GDN_ERR_INVALID_ARG;
+    return gdn::launch_decode(q, k, v, beta, g, state, o, N, H, dk, dv, scale, in_dtype,
+                              static_cast<cudaStream_t>(cuda_stream));
+}
+
+gdn_status_t gdn_sync_status(void *cuda_stream) {
+    cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return GDN_ERR_CUDA;
+    unsigned err = 0u;
+    if (!gdn::read_and_clear_device_error(&err)) return GDN_ERR_CUDA;
+    return err ? GDN_ERR_TIMEOUT : GDN_OK;
+}
+
+}  // extern "C"

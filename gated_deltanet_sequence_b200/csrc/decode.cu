@@ -1,0 +1,151 @@
+// One-token recurrent decode step, state updated in place (HBM-streaming).
+//
+// Page "【CS336】lecture4 线性注意力|Mamba|GDN|DSA", sections "朴素线性注意力" and
+// "继续改进：GDN": a decoded token costs O(d^2) because k^T S is formed first and
+// the erase term (I - beta k k^T) is never materialised. With q' = scale q:
+//   sk = S^T k,  sq = S^T q'                       (one pass over S)
+//   u  = beta (v - alpha sk)    (u = v without the delta term)
+//   o  = alpha sq + (q'.k) u    (= S_new^T q')
+//   S <- alpha S + k u^T        (written back from registers)
+// The state is read once and written once; everything else is O(d).
+//
+// Layout: one CTA per (sequence, head); thread t owns 4 consecutive value
+// columns (float4) of RPT rows strided by the number of row groups, so every
+// warp-wide access is a contiguous 256-512 B run of one or two state rows.
+#include "common.cuh"
+
+namespace gdn {
+namespace {
+
+constexpr int kDecThreads = 256;
+
+template <int DK, int DV, typename IT, bool DELTA>
+__global__ void __launch_bounds__(kDecThreads)
+decode_step_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT *__restrict__ v,
+                   const float *__restrict__ beta, const float *__restrict__ g,
+                   float *__restrict__ state, float *__restrict__ o, float scale) {
+    constexpr int CG = DV / 4;               // float4 column groups
+    constexpr int RG = kDecThreads / CG;     // row groups
+    constexpr int RPT = DK / RG;             // rows per thread
+    static_assert(RPT >= 1 && RG * RPT == DK, "bad decode tiling");
+    __shared__ float s_k[DK], s_q[DK], s_v[DV];
+    __shared__ float red_k[DELTA ? RG : 1][DV];
+    __shared__ float red_q[RG][DV];
+    __shared__ float s_qk;
+
+    const long head = blockIdx.x;
+    const int tid = threadIdx.x;
+    const int cg = tid % CG, rg = tid / CG;
+    float *S = state + head * (long)DK * DV;
+
+    // stream the state rows into registers first (independent 16 B loads)
+    float4 sreg[RPT];
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) sreg[i] = ld_global4(S + (long)(rg + RG * i) * DV + 4 * cg);
+
+    for (int i = tid; i < DK; i += kDecThreads) {
+        s_k[i] = ld_in(k + head * DK + i);
+        s_q[i] = scale * ld_in(q + head * DK + i);
+    }
+    for (int i = tid; i < DV; i += kDecThreads) s_v[i] = ld_in(v + head * DV + i);
+    const float alpha = g ? expf(g[head]) : 1.f;
+    const float bt = DELTA ? beta[head] : 0.f;
+    __syncthreads();
+
+    // partial S^T k and S^T q' over this thread's rows
+    float4 pk = make_float4(0.f, 0.f, 0.f, 0.f), pq = pk;
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) {
+        const int j = rg + RG * i;
+        const float kj = s_k[j], qj = s_q[j];
+        if (DELTA) {
+            pk.x = fmaf(sreg[i].x, kj, pk.x); pk.y = fmaf(sreg[i].y, kj, pk.y);
+            pk.z = fmaf(sreg[i].z, kj, pk.z); pk.w = fmaf(sreg[i].w, kj, pk.w);
+        }
+        pq.x = fmaf(sreg[i].x, qj, pq.x); pq.y = fmaf(sreg[i].y, qj, pq.y);
+        pq.z = fmaf(sreg[i].z, qj, pq.z); pq.w = fmaf(sreg[i].w, qj, pq.w);
+    }
+    if (DELTA) *reinterpret_cast<float4 *>(&red_k[rg][4 * cg]) = pk;
+    *reinterpret_cast<float4 *>(&red_q[rg][4 * cg]) = pq;
+    if (tid < 32) {
+        float x = 0.f;
+        for (int j = tid; j < DK; j += 32) x = fmaf(s_q[j], s_k[j], x);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+        if (tid == 0) s_qk = x;
+    }
+    __syncthreads();
+
+    float sk[4] = {0.f, 0.f, 0.f, 0.f}, sq[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int r = 0; r < RG; ++r) {
+        const float4 b = *reinterpret_cast<const float4 *>(&red_q[r][4 * cg]);
+        sq[0] += b.x; sq[1] += b.y; sq[2] += b.z; sq[3] += b.w;
+        if (DELTA) {
+            const float4 a = *reinterpret_cast<const float4 *>(&red_k[r][4 * cg]);
+            sk[0] += a.x; sk[1] += a.y; sk[2] += a.z; sk[3] += a.w;
+        }
+    }
+    float u[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const float vc = s_v[4 * cg + c];
+        u[c] = DELTA ? bt * (vc - alpha * sk[c]) : vc;
+    }
+    if (rg == 0) {
+        const float qk = s_qk;
+        float4 ov;
+        ov.x = fmaf(alpha, sq[0], qk * u[0]);
+        ov.y = fmaf(alpha, sq[1], qk * u[1]);
+        ov.z = fmaf(alpha, sq[2], qk * u[2]);
+        ov.w = fmaf(alpha, sq[3], qk * u[3]);
+        st_global4(o + head * DV + 4 * cg, ov);
+    }
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) {
+        const int j = rg + RG * i;
+        const float kj = s_k[j];
+        float4 s = sreg[i];
+        s.x = fmaf(alpha, s.x, kj * u[0]);
+        s.y = fmaf(alpha, s.y, kj * u[1]);
+        s.z = fmaf(alpha, s.z, kj * u[2]);
+        s.w = fmaf(alpha, s.w, kj * u[3]);
+        st_global4(S + (long)j * DV + 4 * cg, s);
+    }
+}
+
+template <int DK, int DV, typename IT>
+gdn_status_t launch_dec_t(const void *q, const void *k, const void *v, const float *beta,
+                          const float *g, float *state, float *o, long NH, float scale,
+                          cudaStream_t stream) {
+    if (beta)
+        decode_step_kernel<DK, DV, IT, true><<<(unsigned)NH, kDecThreads, 0, stream>>>(
+            (const IT *)q, (const IT *)k, (const IT *)v, beta, g, state, o, scale);
+    else
+        decode_step_kernel<DK, DV, IT, false><<<(unsigned)NH, kDecThreads, 0, stream>>>(
+            (const IT *)q, (const IT *)k, (const IT *)v, beta, g, state, o, scale);
+    return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+template <typename IT>
+gdn_status_t launch_dec_dt(const void *q, const void *k, const void *v, const float *beta,
+                           const float *g, float *state, float *o, long NH, int dk, int dv,
+                           float scale, cudaStream_t stream) {
+    if (dk == 128 && dv == 128) return launch_dec_t<128, 128, IT>(q, k, v, beta, g, state, o, NH, scale, stream);
+    if (dk == 128 && dv == 64) return launch_dec_t<128, 64, IT>(q, k, v, beta, g, state, o, NH, scale, stream);
+    if (dk == 64 && dv == 128) return launch_dec_t<64, 128, IT>(q, k, v, beta, g, state, o, NH, scale, stream);
+    return launch_dec_t<64, 64, IT>(q, k, v, beta, g, state, o, NH, scale, stream);
+}
+
+}  // namespace
+
+gdn_status_t launch_decode(const void *q, const void *k, const void *v, const float *beta,
+                           const float *g, float *state, float *o, int N, int H, int dk, int dv,
+                           float scale, gdn_dtype_t in_dtype, cudaStream_t stream) {
+    const long NH = (long)N * H;
+    if (in_dtype == GDN_F32)
+        return launch_dec_dt<float>(q, k, v, beta, g, state, o, NH, dk, dv, scale, stream);
+    return launch_dec_dt<__nv_bfloat16>(q, k, v, beta, g, state, o, NH, dk, dv, scale, stream);
+}
+
+}  // namespace gdn

@@ -1,0 +1,222 @@
+// SIMT (fp32 CUDA-core) chunkwise prefill for plain / gated linear attention,
+// DeltaNet and Gated DeltaNet. It serves fp32 inputs (where fp32 arithmetic is
+// needed to meet a 1e-5 tolerance), head sizes 64, and chunk sizes other than
+// 64; bf16 inputs with dk = dv = 128 and chunk 64 take the tcgen05 kernel.
+//
+// One CTA owns one (batch, head) and a 32-wide slice of the value columns:
+// the state's value columns evolve independently (column c of S only ever
+// mixes with column c of V), so slices need no communication. Per chunk of n
+// rows (page "混合注意力学习(1)", sections "FWP分块并行机制" and "DeltaNet 分块并行机制";
+// page "LinearAttention 概述", section "FLASH": the chunk form is exact):
+//   G = within-chunk cumsum(g); gamma = exp(G); Gamma_rs = exp(G_r - G_s), s <= r
+//   A_rs = beta_r Gamma_rs k_r.k_s (s < r);  T = (I + A)^-1 (forward substitution)
+//   W = T diag(beta gamma) K;  Ut = T diag(beta) V - W S    (Ut = V without delta)
+//   O = diag(gamma) Q S + (Q K^T o Gamma) Ut
+//   S <- gamma_n S + sum_s exp(G_n - G_s) k_s Ut_s^T
+#include "common.cuh"
+
+namespace gdn {
+namespace {
+
+constexpr int kSimtThreads = 256;
+constexpr int kDvs = 32;      // value columns per CTA
+constexpr int kCmax = 64;     // largest supported chunk
+
+template <int DK>
+struct SimtSmem {
+    static constexpr int KP = DK + 1;            // padded row pitch for K, Q, W
+    static constexpr int CP = kCmax + 1;         // padded row pitch for A, T, P
+    float K[kCmax * KP];
+    float Q[kCmax * KP];
+    float W[kCmax * KP];
+    float V[kCmax * kDvs];
+    float U[kCmax * kDvs];
+    float S[DK * kDvs];
+    float A[kCmax * CP];
+    float T[kCmax * CP];
+    float P[kCmax * CP];
+    float G[kCmax];
+    float bt[kCmax];
+};
+
+template <int DK, typename IT, bool DELTA>
+__global__ void __launch_bounds__(kSimtThreads)
+simt_chunk_fwd_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT *__restrict__ v,
+                      const float *__restrict__ beta, const float *__restrict__ g,
+                      float *__restrict__ o, const float *__restrict__ s0,
+                      float *__restrict__ s_final, int L, int dv, int C, float scale) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    using Sm = SimtSmem<DK>;
+    Sm &sm = *reinterpret_cast<Sm *>(smem_raw);
+    constexpr int KP = Sm::KP, CP = Sm::CP;
+    const int tid = threadIdx.x;
+    const long bh = blockIdx.x;
+    const int c0 = blockIdx.y * kDvs;            // first value column of this CTA
+
+    const IT *qh = q + bh * (long)L * DK;
+    const IT *kh = k + bh * (long)L * DK;
+    const IT *vh = v + bh * (long)L * dv;
+    const float *bh_beta = DELTA ? beta + bh * (long)L : nullptr;
+    const float *bh_g = g ? g + bh * (long)L : nullptr;
+    float *oh = o + bh * (long)L * dv;
+
+    for (int i = tid; i < DK * kDvs; i += kSimtThreads) {
+        const int j = i / kDvs, c = i % kDvs;
+        sm.S[i] = s0 ? s0[(bh * DK + j) * dv + c0 + c] : 0.f;
+    }
+
+    for (int t0 = 0; t0 < L; t0 += C) {
+        const int n = min(C, L - t0);
+        __syncthreads();
+        // ---- load the chunk ------------------------------------------------
+        for (int i = tid; i < n * DK; i += kSimtThreads) {
+            const int r = i / DK, j = i % DK;
+            sm.K[r * KP + j] = ld_in(kh + (long)(t0 + r) * DK + j);
+            sm.Q[r * KP + j] = scale * ld_in(qh + (long)(t0 + r) * DK + j);
+        }
+        for (int i = tid; i < n * kDvs; i += kSimtThreads) {
+            const int r = i / kDvs, c = i % kDvs;
+            sm.V[i] = ld_in(vh + (long)(t0 + r) * dv + c0 + c);
+        }
+        if (tid < 32) {
+            // inclusive within-chunk cumulative sum of g (warp scan, two passes of 32)
+            float carry = 0.f;
+            for (int base = 0; base < n; base += 32) {
+                const int r = base + tid;
+                float x = (bh_g && r < n) ? bh_g[t0 + r] : 0.f;
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, x, off);
+                    if (tid >= off) x += y;
+                }
+                if (r < n) sm.G[r] = carry + x;
+                carry += __shfl_sync(0xffffffffu, x, 31);
+            }
+        } else if (DELTA && tid >= 64 && tid < 64 + kCmax) {
+            const int r = tid - 64;
+            if (r < n) sm.bt[r] = bh_beta[t0 + r];
+        }
+        __syncthreads();
+        // ---- Gram products with the decay mask ---------------------------------
+        for (int i = tid; i < n * n; i += kSimtThreads) {
+            const int r = i / n, s = i % n;
+            float p = 0.f, a = 0.f;
+            if (s <= r) {
+                const float dec = expf(sm.G[r] - sm.G[s]);
+#pragma unroll 8
+                for (int j = 0; j < DK; ++j) {
+                    p = fmaf(sm.Q[r * KP + j], sm.K[s * KP + j], p);
+                    if (DELTA) a = fmaf(sm.K[r * KP + j], sm.K[s * KP + j], a);
+                }
+                p *= dec;
+                if (DELTA) a = (s < r) ? sm.bt[r] * dec * a : 0.f;
+            }
+            sm.P[r * CP + s] = p;
+            if (DELTA) sm.A[r * CP + s] = a;
+        }
+        __syncthreads();
+        if (DELTA) {
+            // ---- T = (I + A)^-1: thread j solves column j by forward substitution
+            if (tid < n) {
+                const int jc = tid;
+                for (int r = 0; r < n; ++r) {
+                    float x = (r == jc) ? 1.f : 0.f;
+                    for (int s = jc; s < r; ++s) x = fmaf(-sm.A[r * CP + s], sm.T[s * CP + jc], x);
+                    sm.T[r * CP + jc] = (r < jc) ? 0.f : x;
+                }
+            }
+            __syncthreads();
+            // ---- W = T diag(beta gamma) K ;  U = T diag(beta) V ----------------------
+            for (int i = tid; i < n * DK; i += kSimtThreads) {
+                const int r = i / DK, j = i % DK;
+                float w = 0.f;
+                for (int s = 0; s <= r; ++s)
+                    w = fmaf(sm.T[r * CP + s] * sm.bt[s] * expf(sm.G[s]), sm.K[s * KP + j], w);
+                sm.W[r * KP + j] = w;
+            }
+            for (int i = tid; i < n * kDvs; i += kSimtThreads) {
+                const int r = i / kDvs, c = i % kDvs;
+                float u = 0.f;
+                for (int s = 0; s <= r; ++s) u = fmaf(sm.T[r * CP + s] * sm.bt[s], sm.V[s * kDvs + c], u);
+                sm.U[i] = u;
+            }
+            __syncthreads();
+            // ---- Ut = U - W S ----------------------------------------------------------
+            for (int i = tid; i < n * kDvs; i += kSimtThreads) {
+                const int r = i / kDvs, c = i % kDvs;
+                float ws = 0.f;
+#pragma unroll 8
+                for (int j = 0; j < DK; ++j) ws = fmaf(sm.W[r * KP + j], sm.S[j * kDvs + c], ws);
+                sm.U[i] -= ws;
+            }
+            __syncthreads();
+        }
+        const float *Ut = DELTA ? sm.U : sm.V;
+        // ---- O = diag(gamma) Q S + P Ut ---------------------------------------------
+        for (int i = tid; i < n * kDvs; i += kSimtThreads) {
+            const int r = i / kDvs, c = i % kDvs;
+            float qs = 0.f;
+#pragma unroll 8
+            for (int j = 0; j < DK; ++j) qs = fmaf(sm.Q[r * KP + j], sm.S[j * kDvs + c], qs);
+            float pu = 0.f;
+            for (int s = 0; s <= r; ++s) pu = fmaf(sm.P[r * CP + s], Ut[s * kDvs + c], pu);
+            oh[(long)(t0 + r) * dv + c0 + c] = expf(sm.G[r]) * qs + pu;
+        }
+        __syncthreads();
+        // ---- S <- gamma_n S + sum_s exp(G_n - G_s) k_s Ut_s^T ----------------------
+        {
+            const float Gn = sm.G[n - 1];
+            for (int i = tid; i < DK * kDvs; i += kSimtThreads) {
+                const int j = i / kDvs, c = i % kDvs;
+                float x = expf(Gn) * sm.S[i];
+                for (int s = 0; s < n; ++s)
+                    x = fmaf(expf(Gn - sm.G[s]) * sm.K[s * KP + j], Ut[s * kDvs + c], x);
+                sm.S[i] = x;
+            }
+        }
+    }
+    __syncthreads();
+    if (s_final) {
+        for (int i = tid; i < DK * kDvs; i += kSimtThreads) {
+            const int j = i / kDvs, c = i % kDvs;
+            s_final[(bh * DK + j) * dv + c0 + c] = sm.S[i];
+        }
+    }
+}
+
+template <int DK, typename IT, bool DELTA>
+gdn_status_t launch_simt_t(const void *q, const void *k, const void *v, const float *beta,
+                           const float *g, float *o, const float *s0, float *s_final, int BH,
+                           int L, int dv, int chunk, float scale, cudaStream_t stream) {
+    auto kern = simt_chunk_fwd_kernel<DK, IT, DELTA>;
+    const int smem = (int)sizeof(SimtSmem<DK>);
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    dim3 grid(BH, dv / kDvs);
+    kern<<<grid, kSimtThreads, smem, stream>>>((const IT *)q, (const IT *)k, (const IT *)v, beta, g,
+                                               o, s0, s_final, L, dv, chunk, scale);
+    return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+}  // namespace
+
+gdn_status_t launch_simt_fwd(const void *q, const void *k, const void *v, const float *beta,
+                             const float *g, float *o, const float *s0, float *s_final, int B,
+                             int H, int L, int dk, int dv, int chunk, float scale,
+                             gdn_dtype_t in_dtype, cudaStream_t stream) {
+    const int BH = B * H;
+    const bool delta = beta != nullptr;
+#define GDN_SIMT_CASE(DKV, IT)                                                                     \
+    return delta ? launch_simt_t<DKV, IT, true>(q, k, v, beta, g, o, s0, s_final, BH, L, dv, chunk, \
+                                                scale, stream)                                     \
+                 : launch_simt_t<DKV, IT, false>(q, k, v, beta, g, o, s0, s_final, BH, L, dv,     \
+                                                 chunk, scale, stream)
+    if (in_dtype == GDN_F32) {
+        if (dk == 64) { GDN_SIMT_CASE(64, float); }
+        GDN_SIMT_CASE(128, float);
+    }
+    if (dk == 64) { GDN_SIMT_CASE(64, __nv_bfloat16); }
+    GDN_SIMT_CASE(128, __nv_bfloat16);
+#undef GDN_SIMT_CASE
+}
+
+}  // namespace gdn

@@ -1,0 +1,126 @@
+/*
+ * gdn.h — C ABI of libgdn.so: chunkwise causal linear attention (plain, gated),
+ * DeltaNet and Gated DeltaNet prefill, plus the one-token recurrent decode step,
+ * as hand-written CUDA kernels for NVIDIA B200 (sm_100a).
+ *
+ * The operator (per head; dk x dv state S stored key-rows by value-columns):
+ *     alpha_t = exp(g_t)                    (alpha_t = 1 when g is NULL)
+ *     u_t     = beta_t (v_t - alpha_t S^T k_t)   (u_t = v_t when beta is NULL)
+ *     S_t     = alpha_t S_{t-1} + k_t u_t^T
+ *     o_t     = S_t^T (scale * q_t)
+ * This is the Gated DeltaNet recurrence S_t = alpha_t S_{t-1}(I - beta_t k k^T)
+ * + beta_t v k^T written in the transposed (dk, dv) storage layout.
+ * Sources: "混合注意力学习(1): 线性注意力" (sections "Fast Weight Programmers与DeltaNet",
+ * "Gated DeltaNet", "FWP分块并行机制", "DeltaNet 分块并行机制", "HouseHolder变换和WY表示");
+ * "LinearAttention 概述" (sections "FLASH", "Lightning Attention": the chunkwise
+ * form is exact and position t sees 1..t inclusive); "【CS336】lecture4 线性注意力|
+ * Mamba|GDN|DSA" (sections "朴素线性注意力", "继续改进：Mamba", "继续改进：GDN").
+ *
+ * Conventions for every entry point
+ *  - Ownership: the caller allocates and owns every buffer (device memory unless
+ *    stated). The library allocates no memory and keeps no per-call state.
+ *  - Layout: dense, contiguous, row-major, as annotated. Device pointers must be
+ *    16-byte aligned.
+ *  - Asynchrony: work is enqueued on `cuda_stream` (a cudaStream_t; NULL = the
+ *    legacy default stream) and the call returns without synchronising. The
+ *    return value reports argument validation and launch errors only; a kernel
+ *    that gave up on a bounded wait records it in a device-side word that
+ *    gdn_sync_status() reads.
+ *  - Errors: on any non-OK return nothing was enqueued (validation) or the
+ *    launch failed (GDN_ERR_CUDA). No exceptions cross this boundary.
+ *  - Aliasing: s_final may alias s0. q, k, v, beta, g must not alias o.
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1,   /* NULL required pointer, bad size, misaligned pointer */
+    GDN_ERR_UNSUPPORTED = 2,   /* valid but not implemented (head dim, chunk, dtype)  */
+    GDN_ERR_CUDA = 3,          /* a CUDA runtime/driver call or launch failed          */
+    GDN_ERR_TIMEOUT = 4        /* a kernel gave up on a bounded wait (see sync_status) */
+} gdn_status_t;
+
+typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype_t;
+
+/*
+ * lin_attn_chunk_fwd — causal linear attention without normaliser, plain
+ * (g == NULL: alpha = 1) or with a scalar per-token decay (g != NULL).
+ * Page "混合注意力学习(1)" section "FWP分块并行机制" (chunk-mixed intra/inter form);
+ * page "LinearAttention 概述" sections "快速预览" (O = (QK^T o M)V) and "Lightning
+ * Attention" (positions 1..t inclusive); page "【CS336】lecture4" section
+ * "继续改进：Mamba" (gated state decay).
+ *
+ *  q, k     (B, H, L, dk) in_dtype            device, read
+ *  v        (B, H, L, dv) in_dtype            device, read
+ *  g        (B, H, L) fp32 log-alpha (<= 0 expected), nullable
+ *  o        (B, H, L, dv) fp32                device, written
+ *  s0       (B, H, dk, dv) fp32 initial state, nullable (zero state)
+ *  s_final  (B, H, dk, dv) fp32 final state,   nullable (not written)
+ *  B, H >= 1; L >= 0 (L == 0: only s_final is written, = s0 or 0)
+ *  dk, dv in {64, 128}; chunk: 1..64 (bf16 with dk = dv = 128 requires 64).
+ *  scale multiplies q.  in_dtype: GDN_BF16 or GDN_F32 (q, k, v share it).
+ */
+gdn_status_t lin_attn_chunk_fwd(const void *q, const void *k, const void *v, const float *g,
+                                float *o, const float *s0, float *s_final,
+                                int B, int H, int L, int dk, int dv, int chunk, float scale,
+                                gdn_dtype_t in_dtype, void *cuda_stream);
+
+/*
+ * gdn_chunk_fwd — DeltaNet (g == NULL) or Gated DeltaNet (g != NULL), chunkwise:
+ * per chunk the UT transform T = (I + tril(diag(beta) K K^T o Gamma, -1))^-1 by
+ * forward substitution, W = T diag(beta gamma) K, U = T diag(beta) V, the
+ * state-dependent pseudo-values U - W S_c, the output diag(gamma) Q S_c +
+ * tril(Q K^T o Gamma)(U - W S_c) and the state scan
+ * S_{c+1} = gamma_C S_c + K~^T (U - W S_c).
+ * Page "混合注意力学习(1)" sections "DeltaNet 分块并行机制", "重新定义降低内存占用",
+ * "HouseHolder变换和WY表示"; page "LinearAttention 概述" section "FLASH".
+ *
+ *  beta     (B, H, L) fp32, required (the delta term's learning rate)
+ *  other arguments as for lin_attn_chunk_fwd.
+ */
+gdn_status_t gdn_chunk_fwd(const void *q, const void *k, const void *v, const float *beta,
+                           const float *g, float *o, const float *s0, float *s_final,
+                           int B, int H, int L, int dk, int dv, int chunk, float scale,
+                           gdn_dtype_t in_dtype, void *cuda_stream);
+
+/*
+ * gdn_decode_step — one token for N independent sequences, state updated in place:
+ *   u = beta (v - alpha S^T k);  o = alpha S^T q' + (q'.k) u;  S <- alpha S + k u^T
+ * with q' = scale q (o equals S_new^T q'). The state is read once and written
+ * once. Page "【CS336】lecture4" sections "朴素线性注意力" (O(d^2) per decoded token)
+ * and "继续改进：GDN" (k^T S first keeps the erase term O(d^2)).
+ *
+ *  q, k   (N, H, dk) in_dtype; v (N, H, dv) in_dtype
+ *  beta   (N, H) fp32, nullable (NULL: no delta term, u = v)
+ *  g      (N, H) fp32 log-alpha, nullable (alpha = 1)
+ *  state  (N, H, dk, dv) fp32, read and written in place
+ *  o      (N, H, dv) fp32, written
+ *  N, H >= 1; dk, dv in {64, 128}.
+ */
+gdn_status_t gdn_decode_step(const void *q, const void *k, const void *v, const float *beta,
+                             const float *g, float *state, float *o, int N, int H, int dk,
+                             int dv, float scale, gdn_dtype_t in_dtype, void *cuda_stream);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char *gdn_status_str(gdn_status_t status);
+
+/*
+ * gdn_sync_status — synchronise `cuda_stream`, then report (and clear) whether any
+ * kernel of this library on the current device gave up on a bounded wait since
+ * the last call: GDN_ERR_TIMEOUT in that case, GDN_ERR_CUDA if the stream
+ * reported an error, GDN_OK otherwise.
+ */
+gdn_status_t gdn_sync_status(void *cuda_stream);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int gdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GDN_H_ */

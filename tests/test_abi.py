@@ -1,0 +1,97 @@
+"""The C-ABI library loads, exports what include/gdn.h declares, and validates
+arguments on the host (these calls return before any CUDA work, so no GPU is needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from gated_deltanet_sequence_b200 import build
+    build.build()
+    from gated_deltanet_sequence_b200 import _lib
+    return _lib
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for want in ("lin_attn_chunk_fwd", "gdn_chunk_fwd", "gdn_decode_step", "gdn_status_str",
+                 "gdn_sync_status", "gdn_version"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    raw = ctypes.CDLL(lib.LIB_PATH)
+    for name in _declared_functions():
+        assert hasattr(raw, name), f"libgdn.so does not export {name}"
+
+
+def test_status_strings_and_version(lib):
+    assert lib.status_str(0) == "GDN_OK"
+    assert lib.status_str(4) == "GDN_ERR_TIMEOUT"
+    assert lib.status_str(99) == "GDN_ERR_UNKNOWN"
+    assert lib.gdn_version() >= 100
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails first
+
+
+def _prefill(lib, fn, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, beta=FAKE, g=None, o=FAKE, s0=None, s_final=None,
+             B=1, H=1, L=8, dk=64, dv=64, chunk=64, scale=1.0, dt=1)
+    a.update(kw)
+    P = ctypes.c_void_p
+    if fn == "gdn":
+        return lib.lib.gdn_chunk_fwd(P(a["q"]), P(a["k"]), P(a["v"]), P(a["beta"]), P(a["g"]),
+                                     P(a["o"]), P(a["s0"]), P(a["s_final"]), a["B"], a["H"],
+                                     a["L"], a["dk"], a["dv"], a["chunk"], a["scale"], a["dt"], None)
+    return lib.lib.lin_attn_chunk_fwd(P(a["q"]), P(a["k"]), P(a["v"]), P(a["g"]), P(a["o"]),
+                                      P(a["s0"]), P(a["s_final"]), a["B"], a["H"], a["L"],
+                                      a["dk"], a["dv"], a["chunk"], a["scale"], a["dt"], None)
+
+
+@pytest.mark.parametrize("fn", ["gdn", "la"])
+@pytest.mark.parametrize("kw,want", [
+    (dict(B=0), 1), (dict(H=0), 1), (dict(L=-1), 1), (dict(q=None), 1), (dict(o=None), 1),
+    (dict(q=FAKE + 2), 1), (dict(o=FAKE + 8), 1), (dict(s0=FAKE + 4), 1), (dict(chunk=0), 1),
+    (dict(dt=7), 1), (dict(scale=float("nan")), 1),
+    (dict(dk=96), 2), (dict(dv=32), 2), (dict(chunk=65), 2),
+])
+def test_prefill_rejects_bad_arguments(lib, fn, kw, want):
+    assert _prefill(lib, fn, **kw) == want
+
+
+def test_gdn_requires_beta(lib):
+    assert _prefill(lib, "gdn", beta=None) == 1
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(N=0), 1), (dict(q=None), 1), (dict(state=FAKE + 4), 1), (dict(dk=32), 2), (dict(dt=3), 1),
+])
+def test_decode_rejects_bad_arguments(lib, kw, want):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, beta=None, g=None, state=FAKE, o=FAKE, N=1, H=1, dk=64,
+             dv=64, scale=1.0, dt=1)
+    a.update(kw)
+    P = ctypes.c_void_p
+    st = lib.lib.gdn_decode_step(P(a["q"]), P(a["k"]), P(a["v"]), P(a["beta"]), P(a["g"]),
+                                 P(a["state"]), P(a["o"]), a["N"], a["H"], a["dk"], a["dv"],
+                                 a["scale"], a["dt"], None)
+    assert st == want
+
+
+def test_binding_raises_on_bad_shapes(lib):
+    import torch
+    q = torch.zeros(1, 1, 4, 64)
+    with pytest.raises(ValueError):
+        lib.gdn_chunk_fwd(q, q, torch.zeros(1, 1, 5, 64), torch.zeros(1, 1, 4))

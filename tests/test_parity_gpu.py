@@ -1,0 +1,251 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Error metric: max|x_gpu - x_ref| / max|x_ref| over the compared tensor, for the
+output o and separately for the final state. Bounds: 2e-3 for bf16 inputs (fp32
+accumulation), 1e-5 for fp32 inputs. Small cases span several 64-row chunks and a
+ragged tail; the full-size workloads are checked on sampled heads (the oracle
+recomputes those heads token by token) in the launch configuration the benchmark
+times.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gated_deltanet_sequence_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+TOL = {torch.bfloat16: 2e-3, torch.float32: 1e-5}
+MODES = {"plain": (False, False), "gated": (False, True), "delta": (True, False), "gdn": (True, True)}
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from gated_deltanet_sequence_b200 import _lib
+    return _lib
+
+
+def _inputs(B, H, L, dk, dv, mode, dtype, s0, seed):
+    delta, gated = MODES[mode]
+    inp = W.make_prefill_inputs(B, H, L, dk, dv, mode="gdn", in_dtype=dtype, s0=s0, seed=seed)
+    if not delta:
+        inp["beta"] = None
+    if not gated:
+        inp["g"] = None
+    return inp
+
+
+def _to(x, dev="cuda"):
+    return None if x is None else x.to(dev)
+
+
+def gpu_prefill(lib, inp, chunk=64, scale=1.0):
+    q, k, v, beta, g, s0 = (_to(inp[n]) for n in ("q", "k", "v", "beta", "g", "s0"))
+    B, H, L, dk = q.shape
+    dv = v.shape[-1]
+    sf = torch.full((B, H, dk, dv), float("nan"), device="cuda")
+    o = torch.full((B, H, L, dv), float("nan"), device="cuda")
+    if beta is not None:
+        lib.gdn_chunk_fwd(q, k, v, beta, g, o=o, s0=s0, s_final=sf, chunk=chunk, scale=scale)
+    else:
+        lib.lin_attn_chunk_fwd(q, k, v, g, o=o, s0=s0, s_final=sf, chunk=chunk, scale=scale)
+    assert lib.gdn_sync_status() == 0
+    return o.cpu(), sf.cpu()
+
+
+def check(x, ref, tol, what):
+    err = oracle.max_norm_err(x, ref)
+    assert np.isfinite(err) and err <= tol, f"{what}: max-normalised error {err:.3e} > {tol:.1e}"
+    return err
+
+
+# --------------------------------------------------------------------------------------
+@pytest.mark.parametrize("mode", list(MODES))
+@pytest.mark.parametrize("L", [1, 63, 64, 65, 130, 300])
+def test_bf16_d128_chunk64_small(lib, mode, L):
+    inp = _inputs(2, 3, L, 128, 128, mode, torch.bfloat16, s0=(L % 2 == 1), seed=10 + L)
+    o, sf = gpu_prefill(lib, inp)
+    o_ref, s_ref = oracle.recurrent_fwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["g"], inp["s0"])
+    check(o, o_ref, 2e-3, f"o {mode} L={L}")
+    check(sf, s_ref, 2e-3, f"S {mode} L={L}")
+
+
+@pytest.mark.parametrize("mode", list(MODES))
+@pytest.mark.parametrize("dk,dv,chunk,L,dtype", [
+    (64, 64, 64, 200, torch.float32), (128, 64, 32, 97, torch.float32),
+    (64, 128, 7, 50, torch.float32), (128, 128, 64, 129, torch.float32),
+    (64, 64, 1, 20, torch.float32), (64, 64, 64, 150, torch.bfloat16),
+    (128, 128, 16, 77, torch.bfloat16),
+])
+def test_general_sizes(lib, mode, dk, dv, chunk, L, dtype):
+    inp = _inputs(1, 2, L, dk, dv, mode, dtype, s0=True, seed=20 + L + dk)
+    o, sf = gpu_prefill(lib, inp, chunk=chunk, scale=0.6)
+    o_ref, s_ref = oracle.recurrent_fwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["g"],
+                                        inp["s0"], scale=0.6)
+    check(o, o_ref, TOL[dtype], f"o {mode} {dk}x{dv} C={chunk} L={L} {dtype}")
+    check(sf, s_ref, TOL[dtype], f"S {mode}")
+
+
+def test_workload0_gdn_fp32_full(lib):
+    w = W.WORKLOADS[0]
+    inp = W.make_workload_inputs(w)
+    o, sf = gpu_prefill(lib, inp, chunk=w.chunk)
+    o_ref, s_ref = oracle.recurrent_fwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["g"], None)
+    check(o, o_ref, 1e-5, "o workload 0")
+    check(sf, s_ref, 1e-5, "S workload 0")
+
+
+def _sampled_full(lib, idx, heads):
+    """Run a full-size workload on the GPU, compare the listed (b, h) heads with the oracle."""
+    w = W.WORKLOADS[idx]
+    inp = W.make_workload_inputs(w, device="cuda")
+    o, sf = gpu_prefill(lib, inp, chunk=w.chunk)
+    assert torch.isfinite(o).all() and torch.isfinite(sf).all()
+    sel = lambda x: None if x is None else torch.stack([x[b, h] for b, h in heads]).cpu()
+    o_ref, s_ref = oracle.recurrent_fwd(sel(inp["q"]), sel(inp["k"]), sel(inp["v"]),
+                                        sel(inp["beta"]), sel(inp["g"]), sel(inp["s0"]))
+    check(sel(o), o_ref, 2e-3, f"o workload {idx}")
+    check(sel(sf), s_ref, 2e-3, f"S workload {idx}")
+
+
+def test_workload1_plain_la_full_sampled(lib):
+    _sampled_full(lib, 1, [(0, 0), (1, 7), (3, 15)])
+
+
+def test_workload2_gdn_full_sampled(lib):
+    _sampled_full(lib, 2, [(0, 0), (3, 9), (7, 15)])
+
+
+def test_workload3_long_gdn_full_sampled(lib):
+    _sampled_full(lib, 3, [(0, 0), (0, 31)])
+
+
+# --------------------------------------------------------------------------------------
+def test_decode_workload4_full_state(lib):
+    w = W.WORKLOADS[4]
+    steps = 3
+    inp = W.make_workload_inputs(w, device="cuda", steps=steps)
+    state = inp["state"].clone()
+    ref_state = inp["state"].cpu().double().numpy().copy()
+    for t in range(steps):
+        o = lib.gdn_decode_step(inp["q"][t], inp["k"][t], inp["v"][t], inp["beta"][t], inp["g"][t], state)
+        o_ref = oracle.decode_step(inp["q"][t].cpu(), inp["k"][t].cpu(), inp["v"][t].cpu(),
+                                   inp["beta"][t].cpu(), inp["g"][t].cpu(), ref_state)
+        check(o.cpu(), o_ref, 2e-3, f"decode o step {t}")
+    assert lib.gdn_sync_status() == 0
+    check(state.cpu(), ref_state, 2e-3, "decode final state")
+
+
+def test_decode_workload4_sampled_many_steps(lib):
+    w = W.WORKLOADS[4]
+    steps = 24
+    inp = W.make_workload_inputs(w, device="cuda", steps=steps)
+    state = inp["state"].clone()
+    ns = [0, 37, 101, 128, 170, 200, 231, 255]
+    ref_state = np.ascontiguousarray(inp["state"][ns].cpu().double().numpy())
+    for t in range(steps):
+        o = lib.gdn_decode_step(inp["q"][t], inp["k"][t], inp["v"][t], inp["beta"][t], inp["g"][t], state)
+        o_ref = oracle.decode_step(inp["q"][t][ns].cpu(), inp["k"][t][ns].cpu(), inp["v"][t][ns].cpu(),
+                                   inp["beta"][t][ns].cpu(), inp["g"][t][ns].cpu(), ref_state)
+        check(o[ns].cpu(), o_ref, 2e-3, f"decode o step {t}")
+    check(state[ns].cpu(), ref_state, 2e-3, "decode state")
+
+
+@pytest.mark.parametrize("delta,gated", [(False, False), (True, False), (False, True), (True, True)])
+@pytest.mark.parametrize("dk,dv,dtype", [(128, 128, torch.bfloat16), (64, 128, torch.float32),
+                                         (128, 64, torch.bfloat16), (64, 64, torch.float32)])
+def test_decode_modes_and_sizes(lib, delta, gated, dk, dv, dtype):
+    inp = W.make_decode_inputs(3, 5, dk, dv, 4, in_dtype=dtype, seed=77, device="cuda",
+                               delta=delta, gated=gated)
+    state = inp["state"].clone()
+    ref_state = inp["state"].cpu().double().numpy().copy()
+    for t in range(4):
+        b = inp["beta"][t] if delta else None
+        g = inp["g"][t] if gated else None
+        o = lib.gdn_decode_step(inp["q"][t], inp["k"][t], inp["v"][t], b, g, state, scale=0.9)
+        o_ref = oracle.decode_step(inp["q"][t].cpu(), inp["k"][t].cpu(), inp["v"][t].cpu(),
+                                   None if b is None else b.cpu(), None if g is None else g.cpu(),
+                                   ref_state, scale=0.9)
+        check(o.cpu(), o_ref, TOL[dtype], f"decode o t={t}")
+    check(state.cpu(), ref_state, TOL[dtype], "decode state")
+
+
+def test_decode_steps_equal_prefill(lib):
+    B, H, L, d = 2, 4, 70, 128
+    inp = _inputs(B, H, L, d, d, "gdn", torch.bfloat16, s0=True, seed=5)
+    o_pre, s_pre = gpu_prefill(lib, inp)
+    state = inp["s0"].cuda().clone()
+    outs = []
+    for t in range(L):
+        outs.append(lib.gdn_decode_step(inp["q"][:, :, t].cuda().contiguous(),
+                                        inp["k"][:, :, t].cuda().contiguous(),
+                                        inp["v"][:, :, t].cuda().contiguous(),
+                                        inp["beta"][:, :, t].cuda().contiguous(),
+                                        inp["g"][:, :, t].cuda().contiguous(), state))
+    o_dec = torch.stack(outs, 2).cpu()
+    check(o_dec, o_pre, 4e-3, "decode vs prefill o")
+    check(state.cpu(), s_pre, 4e-3, "decode vs prefill S")
+
+
+# --------------------------------------------------------------------------------------
+def test_empty_sequence_copies_state(lib):
+    inp = _inputs(2, 2, 0, 128, 128, "gdn", torch.bfloat16, s0=True, seed=3)
+    q, k, v = (inp[n].cuda() for n in "qkv")
+    s0 = inp["s0"].cuda()
+    sf = torch.full_like(s0, float("nan"))
+    lib.gdn_chunk_fwd(q, k, v, None, None, s0=s0, s_final=sf)
+    assert torch.equal(sf, s0)
+    sf2 = torch.full_like(s0, float("nan"))
+    lib.lin_attn_chunk_fwd(q, k, v, None, s0=None, s_final=sf2)
+    assert torch.count_nonzero(sf2) == 0
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_exact_recall_with_basis_keys(lib, dtype):
+    # alpha = beta = 1, distinct basis keys: querying key j returns v_j exactly
+    d, m, L = 128, 90, 180
+    rng = np.random.default_rng(0)
+    perm = rng.permutation(d)
+    keys = np.eye(d)[perm[:m]]
+    vals = rng.integers(-8, 8, size=(m, d)).astype(np.float32)
+    spare = np.eye(d)[perm[m]]
+    q = np.vstack([np.zeros((m, d)), keys])
+    k = np.vstack([keys, np.tile(spare, (m, 1))])
+    v = np.vstack([vals, np.zeros((m, d))])
+    t = lambda x: torch.tensor(x, dtype=dtype).reshape(1, 1, L, d).contiguous()
+    inp = dict(q=t(q), k=t(k), v=t(v), beta=torch.ones(1, 1, L), g=None, s0=None)
+    o, _ = gpu_prefill(lib, inp)
+    assert torch.equal(o[0, 0, m:], torch.tensor(vals)), "recall is not exact"
+
+
+def test_deterministic_bitwise(lib):
+    inp = _inputs(2, 4, 333, 128, 128, "gdn", torch.bfloat16, s0=True, seed=8)
+    a = gpu_prefill(lib, inp)
+    b = gpu_prefill(lib, inp)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_state_passing_chunk_aligned_is_bitwise(lib):
+    B, H, L1, L2, d = 2, 3, 128, 75, 128
+    inp = _inputs(B, H, L1 + L2, d, d, "gdn", torch.bfloat16, s0=True, seed=9)
+    o_all, s_all = gpu_prefill(lib, inp)
+    first = {n: (None if inp[n] is None else inp[n][:, :, :L1].contiguous()) for n in ("q", "k", "v", "beta", "g")}
+    first["s0"] = inp["s0"]
+    o1, s1 = gpu_prefill(lib, first)
+    second = {n: (None if inp[n] is None else inp[n][:, :, L1:].contiguous()) for n in ("q", "k", "v", "beta", "g")}
+    second["s0"] = s1
+    o2, s2 = gpu_prefill(lib, second)
+    assert torch.equal(torch.cat([o1, o2], 2), o_all)
+    assert torch.equal(s2, s_all)
+
+
+def test_nan_free_with_strong_decay(lib):
+    # very negative log-alpha: every exponent is of a difference inside one chunk, so
+    # nothing overflows; the state forgets almost everything
+    inp = _inputs(1, 2, 200, 128, 128, "gdn", torch.bfloat16, s0=True, seed=12)
+    inp["g"] = torch.full_like(inp["g"], -30.0)
+    o, sf = gpu_prefill(lib, inp)
+    o_ref, s_ref = oracle.recurrent_fwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["g"], inp["s0"])
+    check(o, o_ref, 2e-3, "o strong decay")
+    check(sf, s_ref, 2e-3, "S strong decay")

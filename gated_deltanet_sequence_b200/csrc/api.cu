@@ -9,6 +9,7 @@ namespace {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool opt_aligned16(const void *p) { return p == nullptr || aligned16(p); }
+bool opt_aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 bool head_dim_ok(int d) { return d == 64 || d == 128; }
 
 gdn_status_t check_prefill(const void *q, const void *k, const void *v, const float *g, float *o,
@@ -18,7 +19,7 @@ gdn_status_t check_prefill(const void *q, const void *k, const void *v, const fl
     if (in_dtype != GDN_F32 && in_dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
     if (L > 0 && (!q || !k || !v || !o)) return GDN_ERR_INVALID_ARG;
     if (!opt_aligned16(q) || !opt_aligned16(k) || !opt_aligned16(v) || !opt_aligned16(o) ||
-        !opt_aligned16(g) || !opt_aligned16(s0) || !opt_aligned16(s_final))
+        !opt_aligned4(g) || !opt_aligned16(s0) || !opt_aligned16(s_final))
         return GDN_ERR_INVALID_ARG;
     if (chunk < 1) return GDN_ERR_INVALID_ARG;
     if (!head_dim_ok(dk) || !head_dim_ok(dv) || chunk > 64) return GDN_ERR_UNSUPPORTED;
@@ -66,7 +67,7 @@ gdn_status_t gdn_chunk_fwd(const void *q, const void *k, const void *v, const fl
     gdn_status_t st = check_prefill(q, k, v, g, o, s0, s_final, B, H, L, dk, dv, chunk, scale, in_dtype);
     if (st != GDN_OK) return st;
     if (L > 0 && !beta) return GDN_ERR_INVALID_ARG;
-    if (!opt_aligned16(beta)) return GDN_ERR_INVALID_ARG;
+    if (!opt_aligned4(beta)) return GDN_ERR_INVALID_ARG;
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
     if (gdn::tc_supported(in_dtype, dk, dv, chunk) && L > 0)
         return gdn::launch_tc_gdn(q, k, v, beta, g, o, s0, s_final, B, H, L, scale, stream);
@@ -82,7 +83,7 @@ gdn_status_t gdn_decode_step(const void *q, const void *k, const void *v, const 
     if (in_dtype != GDN_F32 && in_dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
     if (!q || !k || !v || !state || !o) return GDN_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(state) || !aligned16(o) ||
-        !opt_aligned16(beta) || !opt_aligned16(g))
+        !opt_aligned4(beta) || !opt_aligned4(g))
         return GDN_ERR_INVALID_ARG;
     if (!head_dim_ok(dk) || !head_dim_ok(dv)) return GDN_ERR_UNSUPPORTED;
     if ((double)N * H > 2147483647.0) return GDN_ERR_INVALID_ARG;

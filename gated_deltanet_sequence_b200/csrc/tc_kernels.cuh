@@ -13,4 +13,16 @@ gdn_status_t launch_tc_la(const void *q, const void *k, const void *v, const flo
                           cudaStream_t stream);
 // Reads and clears the device-side error word of the current device.
 bool read_and_clear_device_error(unsigned *err);
+// Device address of that word on the current device (looked up once per device),
+// handed to kernels that may record a bounded-wait timeout; nullptr on failure.
+unsigned *device_error_word();
+// Bounded-wait limit handed to the tensor-core kernels (clock cycles, ~2 s at 2 GHz).
+constexpr long long kWaitLimitCycles = 4000000000LL;
+}  // namespace gdn
+
+#include <cuda.h>
+namespace gdn {
+// 3-D TMA map over a (BH, L, 128) bf16 tensor: 64 x 64 boxes, 128-byte swizzle,
+// zero fill outside the tensor (rows past L read as zeros).
+bool make_qkv_map(CUtensorMap *m, const void *ptr, int L, int BH);
 }  // namespace gdn

@@ -20,7 +20,7 @@
  *  - Ownership: the caller allocates and owns every buffer (device memory unless
  *    stated). The library allocates no memory and keeps no per-call state.
  *  - Layout: dense, contiguous, row-major, as annotated. Device pointers must be
- *    16-byte aligned.
+ *    16-byte aligned, except beta and g, which need 4-byte alignment.
  *  - Asynchrony: work is enqueued on `cuda_stream` (a cudaStream_t; NULL = the
  *    legacy default stream) and the call returns without synchronising. The
  *    return value reports argument validation and launch errors only; a kernel

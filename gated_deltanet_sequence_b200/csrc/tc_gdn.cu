@@ -2,8 +2,8 @@
 // (bf16 inputs, dk = dv = 128, chunk C = 64; fp32 accumulation, output and state).
 //
 // One CTA per (batch, head) walks the chunks in order; the fp32 state S (dk x dv)
-// lives in tensor memory for the whole sequence and never goes to HBM until the
-// end. Per chunk of C rows (page "混合注意力学习(1)", sections "DeltaNet 分块并行机制",
+// lives in tensor memory for the whole sequence and goes to HBM only at the end.
+// Per chunk of C rows (page "混合注意力学习(1)", sections "DeltaNet 分块并行机制",
 // "重新定义降低内存占用", "HouseHolder变换和WY表示"; page "LinearAttention 概述", section
 // "FLASH"), with G the within-chunk cumulative sum of g, gamma = exp(G),
 // Gamma_rs = exp(G_r - G_s) (s <= r) and d_s = exp(G_last - G_s):
@@ -11,18 +11,28 @@
 //   UT     A = tril(diag(beta) KK^T o Gamma, -1), T = (I + A)^-1   (forward subst.)
 //   W, U   W^T = K^T (T diag(beta gamma))^T, U^T = V^T (T diag(beta))^T
 //   Ut     Ut^T = U^T - S^T W^T   (accumulated onto U^T with a negated operand)
-//   QS     (Q S)^T = S^T Q^T
+//   out    O^T = S^T Q'^T + Ut^T (scale Q K^T o Gamma)^T,  Q' = diag(scale gamma) Q
 //   state  S <- gamma_last S + K^T (diag(d) Ut)
-//   out    O^T = Ut^T (scale Q K^T o Gamma)^T;  o = scale gamma (QS) + O
-// Every product is written with dk or dv (= 128) as the UMMA M dimension so each
-// tcgen05.mma is a full 128-lane M=128 instruction; TMEM lane = row of the result.
+// Every product has dk or dv (= 128) as the UMMA M dimension, so each tcgen05.mma
+// is a full 128-lane instruction and TMEM lane = row of the result.
 //
-// Shared-memory operands use the 128-byte swizzled canonical layouts (TMA writes
-// Q, K, V that way; the epilogue threads write T, P, W, S and Ut the same way).
-// All UMMA operands are fp16 (10-bit mantissa): the bf16 input tiles are converted
-// in place (exact within the fp16 range) and every computed operand (T, P, W, S,
-// Ut) is rounded to fp16, which keeps the rounding of the chunk intermediates ~8x
-// below what bf16 operands give; accumulation is fp32 throughout.
+// Warp roles (384 threads):
+//   warp 0      TMA producer (2-stage ring of Q, K, V tiles)
+//   warp 1      issues the state-independent UMMAs of a chunk (Gram, W/U)
+//   warp 2      issues the state-dependent UMMAs of a chunk (U - W S, output, state)
+//   warps 4-7   "state" group: S -> fp16 operand, Ut epilogue, output stores, and
+//               the W epilogue of the next chunk (in its idle slot)
+//   warps 8-11  "prep" group, one chunk ahead of the state chain: gate scan, A / P
+//               masks, tile conversion with the Q scaling, blocked UT solve
+// so the state-independent work of chunk c+1 overlaps the serial state chain of
+// chunk c. Hand-offs are mbarriers with one arrival each.
+//
+// Precision: the Gram product runs on the bf16 input tiles (exact products, fp32
+// sums). Every other UMMA takes fp16 operands (10-bit mantissa): K, V are converted
+// in place after the Gram has read them, Q is replaced by Q' in fp16, and every
+// computed operand (T, P, W, S, Ut) is rounded to fp16, which keeps the rounding of
+// the chunk intermediates ~8x below what bf16 operands give. Shared-memory
+// operands use the 128-byte swizzled canonical layouts.
 #include <mutex>
 
 #include "tc_kernels.cuh"
@@ -58,51 +68,145 @@ bool read_and_clear_device_error(unsigned *err) {
 namespace {
 using namespace ptx;
 
-constexpr int kC = 64;          // chunk rows
-constexpr int kD = 128;         // dk = dv
-constexpr int kThreads = 128;   // 4 warps: warp w owns TMEM lanes 32w..32w+31
+constexpr int kC = 64;           // chunk rows
+constexpr int kD = 128;          // dk = dv
+constexpr int kThreads = 384;
+constexpr int kGroupS = 4;       // first warp of the state group
+constexpr int kGroupP = 8;       // first warp of the prep group
+constexpr int kBarS = 1, kBarP = 2;   // named barriers of the two 128-thread groups
 
 // ---- shared memory map (byte offsets from a 1024-aligned base) ------------------
-constexpr uint32_t kStageBytes = 49152;  // one chunk of K, Q, V (bf16, swizzled)
-constexpr uint32_t ST_K0 = 0;            // K, key columns 0-63   (64 rows x 128 B)
-constexpr uint32_t ST_Q0 = 8192;         // Q, key columns 0-63   (directly after K: [K;Q])
-constexpr uint32_t ST_K1 = 16384;        // K, key columns 64-127
-constexpr uint32_t ST_Q1 = 24576;        // Q, key columns 64-127
-constexpr uint32_t ST_V0 = 32768;        // V, value columns 0-63
-constexpr uint32_t ST_V1 = 40960;        // V, value columns 64-127
-constexpr uint32_t OFF_T1 = 2 * kStageBytes;       // T diag(beta gamma), K-major 64 x 64
-constexpr uint32_t OFF_T2 = OFF_T1 + 8192;         // T diag(beta)
-constexpr uint32_t OFF_PG = OFF_T2 + 8192;         // scale (Q K^T o Gamma), K-major 64 x 64
-constexpr uint32_t OFF_W = OFF_PG + 8192;          // W as MN-major B: 128 key rows x 64 r
-constexpr uint32_t OFF_S = OFF_W + 16384;          // S as MN-major A: 2 x (128 key rows x 64 v)
-constexpr uint32_t OFF_UB = OFF_S + 32768;         // Ut, K-major: 128 value rows x 64 s
-constexpr uint32_t OFF_UD = OFF_UB + 16384;        // diag(d) Ut, K-major
-constexpr uint32_t OFF_A = OFF_UD + 16384;         // A fp32 64 x 64 (float4 groups swizzled)
-constexpr uint32_t OFF_VEC = OFF_A + kC * kC * 4;  // G, beta, gamma, d: 4 x 64 fp32
-constexpr uint32_t OFF_BAR = OFF_VEC + 1024;       // 3 mbarriers, TMEM base, abort flag
-constexpr uint32_t kSmemBytes = OFF_BAR + 64;
+constexpr uint32_t kStageBytes = 49152;   // one chunk of K, Q, V
+constexpr uint32_t ST_K0 = 0;             // K, key columns 0-63   (64 rows x 128 B)
+constexpr uint32_t ST_Q0 = 8192;          // Q, key columns 0-63   (directly after K: [K;Q])
+constexpr uint32_t ST_K1 = 16384;         // K, key columns 64-127
+constexpr uint32_t ST_Q1 = 24576;         // Q, key columns 64-127
+constexpr uint32_t ST_V0 = 32768;         // V, value columns 0-63; holds W (MN-major, 128 key
+constexpr uint32_t ST_V1 = 40960;         //   rows x 64 r) once U has been formed
+constexpr uint32_t ST_W = ST_V0;
+constexpr uint32_t OFF_AT = 2 * kStageBytes;        // UT-solve workspace, reused in turn by:
+                                                    //   A^T fp32 64 x 64 (solve input),
+constexpr uint32_t OFF_X = OFF_AT;                  //   A_10 T_00 fp32 32 x 36 (after A^T is read),
+constexpr int kXP = 36;
+constexpr uint32_t OFF_T1 = OFF_AT;                 //   T diag(beta gamma), K-major 64 x 64 fp16,
+constexpr uint32_t OFF_T2 = OFF_AT + 8192;          //   T diag(beta)
+constexpr uint32_t OFF_TF = OFF_AT + 16384;         // T fp32 64 x 68 (pitch 68)
+constexpr int kTP = 68;
+constexpr uint32_t OFF_PG = OFF_TF + 64 * kTP * 4;  // 2 x scale (Q K^T o Gamma), K-major 64 x 64
+constexpr uint32_t OFF_S = OFF_PG + 16384;          // S as MN-major A: 2 x (128 key rows x 64 v)
+constexpr uint32_t OFF_UB = OFF_S + 32768;          // Ut, K-major: 128 value rows x 64 s
+constexpr uint32_t OFF_UD = OFF_UB + 16384;         // diag(d) Ut, K-major
+constexpr uint32_t OFF_VEC = OFF_UD + 16384;        // 2 x {G, beta, gamma, d} (64 fp32 each)
+constexpr uint32_t OFF_BAR = OFF_VEC + 2048;        // mbarriers, TMEM base, abort flag
+constexpr uint32_t kSmemBytes = OFF_BAR + 256;
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;  // slack to align the base to 1024 B
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
+static_assert(OFF_T1 % 1024 == 0 && OFF_PG % 1024 == 0 && OFF_S % 1024 == 0, "UMMA tiles need 1024-B alignment");
 
 // ---- tensor memory columns (512 allocated) ----------------------------------------
-constexpr uint32_t TM_S = 0;     // state S: lane = key row j, 128 value columns
-constexpr uint32_t TM_G = 128;   // [K;Q] K^T: lanes 0-63 K K^T, 64-127 Q K^T; 64 columns s
-constexpr uint32_t TM_W = 192;   // W^T: lane = key j, 64 columns r
-constexpr uint32_t TM_U = 256;   // U^T then Ut^T: lane = value v, 64 columns r
-constexpr uint32_t TM_QS = 320;  // (Q S)^T: lane = value v, 64 columns r
-constexpr uint32_t TM_O = 384;   // Ut^T P^T: lane = value v, 64 columns r
+constexpr uint32_t TM_S = 0;      // state S: lane = key row j, 128 value columns
+constexpr uint32_t TM_X = 128;    // [K;Q] K^T (64 cols s), later W^T (lane = key j, cols r)
+constexpr uint32_t TM_U = 192;    // 2 x U^T then Ut^T: lane = value v, 64 columns r
+constexpr uint32_t TM_O = 320;    // 2 x O^T: lane = value v, 64 columns r
 
-constexpr uint32_t ID_GRAM = idesc_f16(128, 64, false, false);
+constexpr uint32_t ID_GRAM = idesc_f16(128, 64, false, false, false, /*bf16=*/true);
 constexpr uint32_t ID_WU = idesc_f16(128, 64, true, false);
 constexpr uint32_t ID_SW = idesc_f16(128, 64, true, true, /*neg_a=*/true);
 constexpr uint32_t ID_SQ = idesc_f16(128, 64, true, false);
 constexpr uint32_t ID_ST = idesc_f16(128, 128, true, false);
 constexpr uint32_t ID_O = idesc_f16(128, 64, false, false);
 
-__device__ __forceinline__ void record_timeout(unsigned *err, int *abort_flag) {
-    atomicOr(err, kErrWaitTimeout);
-    *abort_flag = 1;
+// mbarriers (index into the barrier array). A parity wait for phase k is only
+// correct while the producer cannot complete phase k+1 first; hand-offs whose
+// producer may run two chunks ahead of the consumer use one barrier per chunk
+// parity (waited with parity (c >> 1) & 1).
+enum : int {
+    B_FULL = 0,      // [2] TMA -> prep issuer (Gram) and prep group
+    B_CDONE = 2,     // [2] state-update UMMAs of chunk c done (frees stage, U, PG, vec of parity c)
+    B_GATE = 4,      // [2] prep: G, beta, gamma, d ready   -> state group
+    B_PREP = 6,      // [2] prep: P, Q' ready               -> state issuer
+    B_GRAM = 8,      // Gram done                          -> prep group
+    B_TRDY = 9,      // prep: T1/T2, K/V fp16 written      -> prep issuer (W/U)
+    B_WU = 10,       // W/U done                           -> state group (W epilogue)
+    B_XFREE = 11,    // state group has read W^T from TM_X -> prep issuer (next Gram)
+    B_WRDY = 12,     // state group: W operand written     -> state issuer
+    B_SRDY = 13,     // state group: S operand written, S scaled -> state issuer
+    B_ADONE = 14,    // U - W S and S Q' done              -> state group (Ut epilogue)
+    B_URDY = 15,     // state group: Ut operands ready     -> state issuer
+    kNumBars = 16
+};
+
+struct Ctl {
+    uint64_t *bar;
+    int *abort_flag;     // CTA-wide: set by the first wait that gives up
+    unsigned *err;
+    long long limit;
+    // Bounded wait. After any timeout in the CTA every later wait fails at once; a
+    // role whose wait fails stops issuing (no further arrivals, copies or UMMAs)
+    // and leaves its loop, so the CTA winds down within a few wait limits.
+    __device__ __forceinline__ bool wait(int b, uint32_t parity) const {
+        if (*reinterpret_cast<volatile int *>(abort_flag)) return false;
+        if (mbar_wait(&bar[b], parity, limit)) return true;
+        atomicOr(err, kErrWaitTimeout);
+        *reinterpret_cast<volatile int *>(abort_flag) = 1;
+        return false;
+    }
+    // bounded wait that ignores the abort flag (final drain of in-flight operations)
+    __device__ __forceinline__ void drain(int b, uint32_t parity) const { mbar_wait(&bar[b], parity, limit); }
+    // Group-uniform wait for a 128-thread group: the leader polls, the group meets on
+    // its named barrier and every thread reads the same verdict (a sticky flag), so
+    // the whole group leaves its loop together.
+    __device__ __forceinline__ bool group_wait(int b, uint32_t parity, int bar_id, int *group_abort,
+                                               bool leader) const {
+        if (leader && !wait(b, parity)) *reinterpret_cast<volatile int *>(group_abort) = 1;
+        named_bar(bar_id, 128);
+        return *reinterpret_cast<volatile int *>(group_abort) == 0;
+    }
+};
+
+template <int N>
+__device__ __forceinline__ void ld_cols(uint32_t taddr, float (&v)[N]) {
+    static_assert(N % 16 == 0, "16-column pieces");
+#pragma unroll
+    for (int cc = 0; cc < N / 16; ++cc) {
+        float t[16];
+        tmem_ld16(taddr + cc * 16, t);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) v[cc * 16 + e] = t[e];
+    }
+    tmem_wait_ld();
 }
+
+// 16 fp32 values -> two swizzled 16-byte chunks (ch, ch+1) of row `row` in a 128-byte-row tile
+__device__ __forceinline__ void st_row16_h(uint32_t tile, uint32_t row, int ch, const float *x) {
+    st_shared_v4(tile + sw128(row, ch), pack_h2(x[0], x[1]), pack_h2(x[2], x[3]), pack_h2(x[4], x[5]),
+                 pack_h2(x[6], x[7]));
+    st_shared_v4(tile + sw128(row, ch + 1), pack_h2(x[8], x[9]), pack_h2(x[10], x[11]), pack_h2(x[12], x[13]),
+                 pack_h2(x[14], x[15]));
+}
+
+// 64 output rows of one value column from TMEM to HBM (rows >= n are padding)
+__device__ __forceinline__ void store_out_col(uint32_t taddr, float *ocol, int n) {
+    float ov[64];
+    ld_cols<64>(taddr, ov);
+#pragma unroll
+    for (int r = 0; r < 64; ++r)
+        if (r < n) ocol[static_cast<size_t>(r) * kD] = ov[r];
+}
+
+// W^T row j (TMEM) -> fp16 MN-major W operand in a stage's V slot
+__device__ __forceinline__ void store_w_row(uint32_t trow_x, uint32_t wtile, int j) {
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+        float w[16];
+        tmem_ld16(trow_x + cc * 16, w);
+        tmem_wait_ld();
+        st_row16_h(wtile, j, 2 * cc, w);
+    }
+}
+
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 template <bool GATED>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -111,16 +215,16 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
               const float *__restrict__ g, float *__restrict__ o, const float *__restrict__ s0,
               float *__restrict__ s_final, int L, float scale, long long wait_limit,
               unsigned *__restrict__ err_word) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // 1024-byte aligned base derived by pointer arithmetic on the shared array, so the
+    // compiler keeps every access below in the shared address space (LDS/STS)
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sb = smem_u32(smem);
-    float *Gs = reinterpret_cast<float *>(smem + OFF_VEC);
-    float *bts = Gs + 64, *gms = Gs + 128, *dss = Gs + 192;
-    float *Am = reinterpret_cast<float *>(smem + OFF_A);
-    uint64_t *bar_tma = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
-    uint64_t *bar_mma = bar_tma + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_mma + 1);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kNumBars);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
+    int *abort_s = abort_flag + 1, *abort_p = abort_flag + 2;   // state / prep group verdicts
+    const Ctl ctl{bars, abort_flag, err_word, wait_limit};
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int bh = blockIdx.x;
@@ -128,10 +232,8 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const size_t row0 = static_cast<size_t>(bh) * L;   // first token row of this head
 
     if (tid == 0) {
-        mbar_init(&bar_tma[0], 1);
-        mbar_init(&bar_tma[1], 1);
-        mbar_init(bar_mma, 1);
-        *abort_flag = 0;
+        for (int b = 0; b < kNumBars; ++b) mbar_init(&bars[b], 1);
+        abort_flag[0] = abort_flag[1] = abort_flag[2] = 0;
         fence_mbar_init();
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
@@ -145,323 +247,456 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);  // this warp's lanes
 
-    auto issue_tma = [&](int c) {
-        const int s = c & 1;
-        uint8_t *st = smem + s * kStageBytes;
-        mbar_arrive_expect_tx(&bar_tma[s], kStageBytes);
-        tma_load_3d(st + ST_K0, &tm_k, &bar_tma[s], 0, c * kC, bh);
-        tma_load_3d(st + ST_K1, &tm_k, &bar_tma[s], 64, c * kC, bh);
-        tma_load_3d(st + ST_Q0, &tm_q, &bar_tma[s], 0, c * kC, bh);
-        tma_load_3d(st + ST_Q1, &tm_q, &bar_tma[s], 64, c * kC, bh);
-        tma_load_3d(st + ST_V0, &tm_v, &bar_tma[s], 0, c * kC, bh);
-        tma_load_3d(st + ST_V1, &tm_v, &bar_tma[s], 64, c * kC, bh);
-    };
-    if (tid == 0) {
-        issue_tma(0);
-        if (nchunks > 1) issue_tma(1);
-    }
-
-    // initial state -> TMEM (thread t holds key row j = t)
-    {
-        const float *src = s0 ? s0 + (static_cast<size_t>(bh) * kD + tid) * kD : nullptr;
-#pragma unroll 1
-        for (int cc = 0; cc < 8; ++cc) {
-            float r[16];
-#pragma unroll
-            for (int e = 0; e < 16; e += 4) {
-                float4 x = src ? *reinterpret_cast<const float4 *>(src + cc * 16 + e) : make_float4(0.f, 0.f, 0.f, 0.f);
-                r[e] = x.x; r[e + 1] = x.y; r[e + 2] = x.z; r[e + 3] = x.w;
+    if (warp == 0) {
+        // ================================================================ TMA producer
+        if (lane == 0) {
+            int last[2] = {-1, -1};   // last chunk loaded into each stage
+            for (int c = 0; c < nchunks; ++c) {
+                const int s = c & 1;
+                if (c >= 2 && !ctl.wait(B_CDONE + s, ((c - 2) >> 1) & 1)) break;
+                uint8_t *st = smem + s * kStageBytes;
+                uint64_t *fb = &bars[B_FULL + s];
+                mbar_arrive_expect_tx(fb, kStageBytes);
+                tma_load_3d(st + ST_K0, &tm_k, fb, 0, c * kC, bh);
+                tma_load_3d(st + ST_Q0, &tm_q, fb, 0, c * kC, bh);
+                tma_load_3d(st + ST_K1, &tm_k, fb, 64, c * kC, bh);
+                tma_load_3d(st + ST_Q1, &tm_q, fb, 64, c * kC, bh);
+                tma_load_3d(st + ST_V0, &tm_v, fb, 0, c * kC, bh);
+                tma_load_3d(st + ST_V1, &tm_v, fb, 64, c * kC, bh);
+                last[s] = c;
             }
-            tmem_st16(trow + TM_S + cc * 16, r);
+            // never leave a copy in flight past the end of the CTA
+            for (int s = 0; s < 2; ++s)
+                if (last[s] >= 0) ctl.drain(B_FULL + s, (last[s] >> 1) & 1);
         }
-        tmem_wait_st();
-    }
-
-    uint32_t mma_phase = 0;
-#pragma unroll 1
-    for (int c = 0; c < nchunks; ++c) {
-        const int t0 = c * kC;
-        const int n = min(kC, L - t0);
-        const uint32_t stg = sb + (c & 1) * kStageBytes;
-
-        // ---- gate cumulative sum and beta for the 64 rows (rows >= n padded: g = beta = 0)
-        if (tid < 64) {
-            float x = (GATED && tid < n) ? g[row0 + t0 + tid] : 0.f;
-            bts[tid] = (tid < n) ? beta[row0 + t0 + tid] : 0.f;
+    } else if (warp == 1) {
+        // ================================================================ prep UMMA issuer
+        if (lane == 0) {
+            int gram_last = -1, wu_last = -1;
+            for (int c = 0; c < nchunks; ++c) {
+                const int s = c & 1;
+                const uint32_t stg = sb + s * kStageBytes;
+                if (!ctl.wait(B_FULL + s, (c >> 1) & 1)) break;
+                if (c >= 1 && !ctl.wait(B_XFREE, (c - 1) & 1)) break;   // W^T of chunk c-1 has left TM_X
+                tc_fence_after();
+                // [K;Q] K^T on the bf16 tiles
 #pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, x, off);
-                if (lane >= off) x += y;
-            }
-            Gs[tid] = x;
-        }
-        __syncthreads();
-        if (tid >= 32 && tid < 64) Gs[tid] += Gs[31];
-        __syncthreads();
-        if (tid < 64) {
-            gms[tid] = GATED ? __expf(Gs[tid]) : 1.f;
-            dss[tid] = GATED ? __expf(Gs[63] - Gs[tid]) : 1.f;
-        }
-        // ---- wait for this chunk's Q, K, V tiles
-        if (!mbar_wait(&bar_tma[c & 1], (c >> 1) & 1, wait_limit)) record_timeout(err_word, abort_flag);
-        tc_fence_before();
-        __syncthreads();
-        if (*abort_flag) break;
-        // the tensor-core operands are fp16: convert this chunk's bf16 tiles in place
-        convert_tile_bf16_to_f16(smem + (c & 1) * kStageBytes, kStageBytes, tid, kThreads);
-        fence_proxy_async();
-        __syncthreads();
-
-        // ---- (1) Gram [K;Q] K^T -> TM_G
-        if (tid == 0) {
-            tc_fence_after();
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
+                    mma_f16(tmem + TM_X, sdesc_sw128(stg + ST_K0 + off, 16, 1024),
+                            sdesc_sw128(stg + ST_K0 + off, 16, 1024), ID_GRAM, kk > 0);
+                }
+                mma_commit(&bars[B_GRAM]);
+                gram_last = c;
+                if (!ctl.wait(B_TRDY, c & 1)) break;
+                if (c >= 2 && !ctl.wait(B_CDONE + s, ((c - 2) >> 1) & 1)) break;   // U buffer s is free
+                tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
-                mma_f16(tmem + TM_G, sdesc_sw128(stg + ST_K0 + off, 16, 1024),
-                         sdesc_sw128(stg + ST_K0 + off, 16, 1024), ID_GRAM, kk > 0);
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_f16(tmem + TM_X, sdesc_sw128(stg + ST_K0 + kk * 2048, 16384, 1024),
+                            sdesc_sw128(sb + OFF_T1 + kk * 32, 16, 1024), ID_WU, kk > 0);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_f16(tmem + TM_U + s * 64, sdesc_sw128(stg + ST_V0 + kk * 2048, 8192, 1024),
+                            sdesc_sw128(sb + OFF_T2 + kk * 32, 16, 1024), ID_WU, kk > 0);
+                mma_commit(&bars[B_WU]);
+                wu_last = c;
             }
-            mma_commit(bar_mma);
+            // UMMAs complete in issue order: the last commit covers everything issued
+            if (wu_last == gram_last && wu_last >= 0) ctl.drain(B_WU, wu_last & 1);
+            else if (gram_last >= 0) ctl.drain(B_GRAM, gram_last & 1);
         }
-        if (!mbar_wait(bar_mma, mma_phase, wait_limit)) record_timeout(err_word, abort_flag);
-        mma_phase ^= 1;
-        tc_fence_after();
-
-        // ---- (E1) rows 0-63: A = beta_r Gamma_rs k_r.k_s (s < r), fp32, float4 groups
-        //      swizzled by row; rows 64-127: scale Gamma_rs q_r.k_s (s <= r), bf16 -> PG
+    } else if (warp == 2) {
+        // ================================================================ state UMMA issuer
+        if (lane == 0) {
+            int a_last = -1, c_last = -1;
+            for (int c = 0; c < nchunks; ++c) {
+                const int s = c & 1;
+                const uint32_t stg = sb + s * kStageBytes;
+                if (!ctl.wait(B_PREP + s, (c >> 1) & 1)) break;
+                if (!ctl.wait(B_WRDY, c & 1)) break;
+                if (!ctl.wait(B_SRDY, c & 1)) break;
+                tc_fence_after();
+                // Ut^T = U^T - S^T W^T ;  O^T = S^T Q'^T
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_f16(tmem + TM_U + s * 64, sdesc_sw128(sb + OFF_S + kk * 2048, 16384, 1024),
+                            sdesc_sw128(stg + ST_W + kk * 2048, 8192, 1024), ID_SW, 1u);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
+                    mma_f16(tmem + TM_O + s * 64, sdesc_sw128(sb + OFF_S + kk * 2048, 16384, 1024),
+                            sdesc_sw128(stg + ST_Q0 + off, 16, 1024), ID_SQ, kk > 0);
+                }
+                mma_commit(&bars[B_ADONE]);
+                a_last = c;
+                if (!ctl.wait(B_URDY, c & 1)) break;
+                tc_fence_after();
+                // S += K^T diag(d) Ut ;  O^T += Ut^T PG^T
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_f16(tmem + TM_S, sdesc_sw128(stg + ST_K0 + kk * 2048, 16384, 1024),
+                            sdesc_sw128(sb + OFF_UD + kk * 32, 16, 1024), ID_ST, 1u);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_f16(tmem + TM_O + s * 64, sdesc_sw128(sb + OFF_UB + kk * 32, 16, 1024),
+                            sdesc_sw128(sb + OFF_PG + s * 8192 + kk * 32, 16, 1024), ID_O, 1u);
+                mma_commit(&bars[B_CDONE + s]);
+                c_last = c;
+            }
+            if (c_last == a_last && c_last >= 0) ctl.drain(B_CDONE + (c_last & 1), (c_last >> 1) & 1);
+            else if (a_last >= 0) ctl.drain(B_ADONE, a_last & 1);
+        }
+    } else if (warp >= kGroupS && warp < kGroupS + 4) {
+        // ================================================================ state group
+        const int j = tid - kGroupS * 32;                // = TMEM lane (key row j / value column v)
+        const bool lead = (j == 0);
+        const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
         {
-            float v[64];
+            const float *src = s0 ? s0 + (static_cast<size_t>(bh) * kD + j) * kD : nullptr;
+#pragma unroll 1
+            for (int cc = 0; cc < 8; ++cc) {
+                float r[16];
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                float t16[16];
-                tmem_ld16(trow + TM_G + cc * 16, t16);
-#pragma unroll
-                for (int e = 0; e < 16; ++e) v[cc * 16 + e] = t16[e];
+                for (int e = 0; e < 16; e += 4) {
+                    const float4 x = src ? *reinterpret_cast<const float4 *>(src + cc * 16 + e)
+                                         : make_float4(0.f, 0.f, 0.f, 0.f);
+                    r[e] = x.x; r[e + 1] = x.y; r[e + 2] = x.z; r[e + 3] = x.w;
+                }
+                tmem_st16(trow + TM_S + cc * 16, r);
             }
-            tmem_wait_ld();
-            if (warp < 2) {
-                const int r = tid;
-                const float br = bts[r], Gr = Gs[r];
-                float *Arow = Am + r * kC;
-#pragma unroll
-                for (int qg = 0; qg < 16; ++qg) {
-                    float a[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int s = qg * 4 + e;
-                        a[e] = (s < r) ? br * __expf(Gr - Gs[s]) * v[s] : 0.f;
-                    }
-                    *reinterpret_cast<float4 *>(Arow + ((qg ^ (r & 15)) << 2)) = make_float4(a[0], a[1], a[2], a[3]);
-                }
-            } else {
-                const int r = tid - 64;
-                const float Gr = Gs[r];
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    uint32_t pk[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int s0i = ch * 8 + 2 * e;
-                        const float p0 = (s0i <= r) ? scale * __expf(Gr - Gs[s0i]) * v[s0i] : 0.f;
-                        const float p1 = (s0i + 1 <= r) ? scale * __expf(Gr - Gs[s0i + 1]) * v[s0i + 1] : 0.f;
-                        pk[e] = pack_h2(p0, p1);
-                    }
-                    st_shared_v4(sb + OFF_PG + sw128(r, ch), pk[0], pk[1], pk[2], pk[3]);
-                }
+            tmem_wait_st();
+        }
+        int done = 0;   // chunks whose output tile has been stored
+        bool ok = true;
+        // W operand of chunk 0
+        if (nchunks > 0) {
+            ok = ctl.group_wait(B_WU, 0, kBarS, abort_s, lead);
+            if (ok) {
+                tc_fence_after();
+                store_w_row(trow + TM_X, sb + ST_W, j);
                 fence_proxy_async();
+                tc_fence_before();
+                named_bar(kBarS, 128);
+                if (lead) {
+                    mbar_arrive(&bars[B_WRDY]);
+                    mbar_arrive(&bars[B_XFREE]);
+                }
             }
         }
-        __syncthreads();
-
-        // ---- (UT) T = (I + A)^-1: thread j (< 64) solves column j by forward substitution,
-        //      then writes T diag(beta gamma) and T diag(beta) (bf16, K-major rows r)
-        if (warp < 2) {
-            const int j = tid;
-            float x[64];
+#pragma unroll 1
+        for (int c = 0; ok && c < nchunks; ++c) {
+            const int s = c & 1;
+            const float *vec = reinterpret_cast<const float *>(smem + OFF_VEC + s * 1024);
+            // S(c) complete, and this chunk's gate values
+            if (c >= 1 && !ctl.group_wait(B_CDONE + ((c - 1) & 1), ((c - 1) >> 1) & 1, kBarS, abort_s, lead)) break;
+            if (!ctl.group_wait(B_GATE + s, (c >> 1) & 1, kBarS, abort_s, lead)) break;
+            tc_fence_after();
+            // ---- S row j -> fp16 MN-major operand; S <- gamma_last S (ahead of the update)
+            {
+                const float gl = GATED ? vec[128 + 63] : 1.f;
 #pragma unroll
-            for (int r = 0; r < 64; ++r) x[r] = 0.f;
+                for (int cc = 0; cc < 8; ++cc) {
+                    float sv[16];
+                    tmem_ld16(trow + TM_S + cc * 16, sv);
+                    tmem_wait_ld();
+                    st_row16_h(sb + OFF_S + (cc >> 2) * 16384u, j, (cc & 3) * 2, sv);
+                    if (GATED) {
 #pragma unroll
-            for (int r = 0; r < 64; ++r) {
-                float a0 = (r == j) ? 1.f : 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-                const float *Ar = Am + r * kC;
-#pragma unroll
-                for (int qg = 0; qg < (r + 3) / 4; ++qg) {
-                    const float4 av = *reinterpret_cast<const float4 *>(Ar + ((qg ^ (r & 15)) << 2));
-                    a0 = fmaf(-av.x, x[4 * qg], a0);
-                    a1 = fmaf(-av.y, x[4 * qg + 1], a1);
-                    a2 = fmaf(-av.z, x[4 * qg + 2], a2);
-                    a3 = fmaf(-av.w, x[4 * qg + 3], a3);
+                        for (int e = 0; e < 16; ++e) sv[e] *= gl;
+                        tmem_st16(trow + TM_S + cc * 16, sv);
+                    }
                 }
-                x[r] = (a0 + a1) + (a2 + a3);
-            }
-            const float bj = bts[j], bgj = bj * gms[j];
-            uint8_t *t1 = smem + OFF_T1, *t2 = smem + OFF_T2;
-#pragma unroll
-            for (int r = 0; r < 64; ++r) {
-                const uint32_t off = sw128(r, j >> 3) + (j & 7) * 2;
-                *reinterpret_cast<__half *>(t1 + off) = __float2half_rn(x[r] * bgj);
-                *reinterpret_cast<__half *>(t2 + off) = __float2half_rn(x[r] * bj);
+                if (GATED) tmem_wait_st();
             }
             fence_proxy_async();
-        }
-        __syncthreads();
-
-        // ---- (2) W^T = K^T T1^T -> TM_W ; U^T = V^T T2^T -> TM_U
-        if (tid == 0) {
+            tc_fence_before();
+            named_bar(kBarS, 128);
+            if (lead) mbar_arrive(&bars[B_SRDY]);
+            // ---- output of the previous chunk (its O tile is complete)
+            if (c >= 1) {
+                const int cp = c - 1;
+                store_out_col(trow + TM_O + (cp & 1) * 64, o + (row0 + static_cast<size_t>(cp) * kC) * kD + j, kC);
+                done = c;
+            }
+            // ---- Ut^T row v -> Ut and diag(d) Ut operands (K-major, rows v)
+            if (!ctl.group_wait(B_ADONE, c & 1, kBarS, abort_s, lead)) break;
             tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_f16(tmem + TM_W, sdesc_sw128(stg + ST_K0 + kk * 2048, 16384, 1024),
-                         sdesc_sw128(sb + OFF_T1 + kk * 32, 16, 1024), ID_WU, kk > 0);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_f16(tmem + TM_U, sdesc_sw128(stg + ST_V0 + kk * 2048, 8192, 1024),
-                         sdesc_sw128(sb + OFF_T2 + kk * 32, 16, 1024), ID_WU, kk > 0);
-            mma_commit(bar_mma);
-        }
-        if (!mbar_wait(bar_mma, mma_phase, wait_limit)) record_timeout(err_word, abort_flag);
-        mma_phase ^= 1;
-        tc_fence_after();
-
-        // ---- (E3) W^T row j -> W tile (MN-major B); S row j -> S tile (MN-major A), and
-        //      S <- gamma_last S in TMEM ahead of the state update
-        {
-            const int j = tid;
-#pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
-                float w[16];
-                tmem_ld16(trow + TM_W + cc * 16, w);
+                float u[16];
+                tmem_ld16(trow + TM_U + s * 64 + cc * 16, u);
                 tmem_wait_ld();
-                st_shared_v4(sb + OFF_W + sw128(j, 2 * cc), pack_h2(w[0], w[1]), pack_h2(w[2], w[3]),
-                             pack_h2(w[4], w[5]), pack_h2(w[6], w[7]));
-                st_shared_v4(sb + OFF_W + sw128(j, 2 * cc + 1), pack_h2(w[8], w[9]),
-                             pack_h2(w[10], w[11]), pack_h2(w[12], w[13]), pack_h2(w[14], w[15]));
-            }
-            const float gl = gms[63];
+                st_row16_h(sb + OFF_UB, j, 2 * cc, u);
+                if (GATED) {
 #pragma unroll
+                    for (int e = 0; e < 16; ++e) u[e] *= vec[192 + cc * 16 + e];
+                }
+                st_row16_h(sb + OFF_UD, j, 2 * cc, u);
+            }
+            fence_proxy_async();
+            tc_fence_before();
+            named_bar(kBarS, 128);
+            if (lead) mbar_arrive(&bars[B_URDY]);
+            // ---- W operand of the next chunk (V of that stage is consumed by then)
+            if (c + 1 < nchunks) {
+                if (!ctl.group_wait(B_WU, (c + 1) & 1, kBarS, abort_s, lead)) break;
+                tc_fence_after();
+                store_w_row(trow + TM_X, sb + ((c + 1) & 1) * kStageBytes + ST_W, j);
+                fence_proxy_async();
+                tc_fence_before();
+                named_bar(kBarS, 128);
+                if (lead) {
+                    mbar_arrive(&bars[B_WRDY]);
+                    mbar_arrive(&bars[B_XFREE]);
+                }
+            }
+        }
+        // ---- last output tile and the final state
+        if (nchunks > 0 && done == nchunks - 1) {
+            const int cp = nchunks - 1;
+            if (ctl.group_wait(B_CDONE + (cp & 1), (cp >> 1) & 1, kBarS, abort_s, lead)) {
+                tc_fence_after();
+                store_out_col(trow + TM_O + (cp & 1) * 64, o + (row0 + static_cast<size_t>(cp) * kC) * kD + j,
+                              L - cp * kC);
+                done = nchunks;
+            }
+        }
+        if (s_final && done == nchunks) {
+            float *dst = s_final + (static_cast<size_t>(bh) * kD + j) * kD;
+#pragma unroll 1
             for (int cc = 0; cc < 8; ++cc) {
                 float sv[16];
                 tmem_ld16(trow + TM_S + cc * 16, sv);
                 tmem_wait_ld();
-                const uint32_t base = sb + OFF_S + (cc >> 2) * 16384u;
-                const int ch = (cc & 3) * 2;
-                st_shared_v4(base + sw128(j, ch), pack_h2(sv[0], sv[1]), pack_h2(sv[2], sv[3]),
-                             pack_h2(sv[4], sv[5]), pack_h2(sv[6], sv[7]));
-                st_shared_v4(base + sw128(j, ch + 1), pack_h2(sv[8], sv[9]), pack_h2(sv[10], sv[11]),
-                             pack_h2(sv[12], sv[13]), pack_h2(sv[14], sv[15]));
-                if (GATED) {
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) sv[e] *= gl;
-                    tmem_st16(trow + TM_S + cc * 16, sv);
-                }
-            }
-            if (GATED) tmem_wait_st();
-            fence_proxy_async();
-        }
-        tc_fence_before();
-        __syncthreads();
-
-        // ---- (3) Ut^T = U^T - S^T W^T (into TM_U) ; (Q S)^T = S^T Q^T -> TM_QS
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-                mma_f16(tmem + TM_U, sdesc_sw128(sb + OFF_S + kk * 2048, 16384, 1024),
-                         sdesc_sw128(sb + OFF_W + kk * 2048, 8192, 1024), ID_SW, 1u);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
-                mma_f16(tmem + TM_QS, sdesc_sw128(sb + OFF_S + kk * 2048, 16384, 1024),
-                         sdesc_sw128(stg + ST_Q0 + off, 16, 1024), ID_SQ, kk > 0);
-            }
-            mma_commit(bar_mma);
-        }
-        if (!mbar_wait(bar_mma, mma_phase, wait_limit)) record_timeout(err_word, abort_flag);
-        mma_phase ^= 1;
-        tc_fence_after();
-
-        // ---- (E4) Ut^T row v -> Ut tile and diag(d) Ut tile (K-major, rows v)
-        {
-            const int vrow = tid;
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                float u[16];
-                tmem_ld16(trow + TM_U + cc * 16, u);
-                tmem_wait_ld();
-                st_shared_v4(sb + OFF_UB + sw128(vrow, 2 * cc), pack_h2(u[0], u[1]), pack_h2(u[2], u[3]),
-                             pack_h2(u[4], u[5]), pack_h2(u[6], u[7]));
-                st_shared_v4(sb + OFF_UB + sw128(vrow, 2 * cc + 1), pack_h2(u[8], u[9]),
-                             pack_h2(u[10], u[11]), pack_h2(u[12], u[13]), pack_h2(u[14], u[15]));
-                float ud[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) ud[e] = GATED ? u[e] * dss[cc * 16 + e] : u[e];
-                st_shared_v4(sb + OFF_UD + sw128(vrow, 2 * cc), pack_h2(ud[0], ud[1]), pack_h2(ud[2], ud[3]),
-                             pack_h2(ud[4], ud[5]), pack_h2(ud[6], ud[7]));
-                st_shared_v4(sb + OFF_UD + sw128(vrow, 2 * cc + 1), pack_h2(ud[8], ud[9]),
-                             pack_h2(ud[10], ud[11]), pack_h2(ud[12], ud[13]), pack_h2(ud[14], ud[15]));
-            }
-            fence_proxy_async();
-        }
-        tc_fence_before();
-        __syncthreads();
-
-        // ---- (4) S += K^T (diag(d) Ut) -> TM_S ; O^T = Ut^T PG^T -> TM_O
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_f16(tmem + TM_S, sdesc_sw128(stg + ST_K0 + kk * 2048, 16384, 1024),
-                         sdesc_sw128(sb + OFF_UD + kk * 32, 16, 1024), ID_ST, 1u);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_f16(tmem + TM_O, sdesc_sw128(sb + OFF_UB + kk * 32, 16, 1024),
-                         sdesc_sw128(sb + OFF_PG + kk * 32, 16, 1024), ID_O, kk > 0);
-            mma_commit(bar_mma);
-        }
-        if (!mbar_wait(bar_mma, mma_phase, wait_limit)) record_timeout(err_word, abort_flag);
-        mma_phase ^= 1;
-        tc_fence_after();
-        // this stage's tiles are consumed: prefetch chunk c + 2 into it
-        if (tid == 0 && c + 2 < nchunks) issue_tma(c + 2);
-
-        // ---- (E5) o[r][v] = scale gamma_r (Q S)[r][v] + O[r][v]   (thread = value column v)
-        {
-            const int vcol = tid;
-            float *orow = o + (row0 + t0) * kD + vcol;
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                float qs[16], ov[16];
-                tmem_ld16(trow + TM_QS + cc * 16, qs);
-                tmem_ld16(trow + TM_O + cc * 16, ov);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int r = cc * 16 + e;
-                    if (r < n) orow[static_cast<size_t>(r) * kD] = fmaf(scale * gms[r], qs[e], ov[e]);
-                }
+                for (int e = 0; e < 16; e += 4)
+                    *reinterpret_cast<float4 *>(dst + cc * 16 + e) = make_float4(sv[e], sv[e + 1], sv[e + 2], sv[e + 3]);
             }
         }
-        tc_fence_before();
-        __syncthreads();
-        if (*abort_flag) break;
-    }
-
-    // ---- final state TMEM -> HBM
-    if (!*abort_flag && s_final) {
-        tc_fence_after();
-        float *dst = s_final + (static_cast<size_t>(bh) * kD + tid) * kD;
+    } else if (warp >= kGroupP && warp < kGroupP + 4) {
+        // ================================================================ prep group
+        const int p = tid - kGroupP * 32;                // 0..127 = TMEM lane
+        const int w4 = warp & 3;
+        const uint32_t trow = tmem + (static_cast<uint32_t>(w4 * 32) << 16);
+        float *__restrict__ At = reinterpret_cast<float *>(smem + OFF_AT);   // At[s * 64 + r] = A[r][s]
+        float *__restrict__ Tf = reinterpret_cast<float *>(smem + OFF_TF);   // Tf[r * kTP + c] = T[r][c]
+        float *__restrict__ Xs = reinterpret_cast<float *>(smem + OFF_X);
+        // gate and beta of the next chunk are fetched one chunk ahead (hides HBM latency)
+        float g_next = 0.f, b_next = 0.f;
+        if (p < 64 && p < L) {
+            if (GATED) g_next = g[row0 + p];
+            b_next = beta[row0 + p];
+        }
 #pragma unroll 1
-        for (int cc = 0; cc < 8; ++cc) {
-            float sv[16];
-            tmem_ld16(trow + TM_S + cc * 16, sv);
-            tmem_wait_ld();
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c & 1;
+            const int t0 = c * kC;
+            const int n = min(kC, L - t0);
+            float *__restrict__ vec = reinterpret_cast<float *>(smem + OFF_VEC + s * 1024);   // G|beta|gamma|d
+            uint8_t *st = smem + s * kStageBytes;
+            // vec, PG and the stage of parity s are free once chunk c-2 is complete
+            if (c >= 2 && !ctl.group_wait(B_CDONE + s, ((c - 2) >> 1) & 1, kBarP, abort_p, p == 0)) break;
+            // ---- gate cumulative sum and beta (rows >= n padded: g = beta = 0)
+            if (p < 64) {
+                float x = g_next;
+                vec[64 + p] = b_next;
+                const int tn = t0 + kC + p;                          // prefetch chunk c + 1
+                g_next = (GATED && c + 1 < nchunks && tn < L) ? g[row0 + tn] : 0.f;
+                b_next = (c + 1 < nchunks && tn < L) ? beta[row0 + tn] : 0.f;
 #pragma unroll
-            for (int e = 0; e < 16; e += 4)
-                *reinterpret_cast<float4 *>(dst + cc * 16 + e) = make_float4(sv[e], sv[e + 1], sv[e + 2], sv[e + 3]);
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, x, off);
+                    if (lane >= off) x += y;
+                }
+                vec[p] = x;
+            }
+            named_bar(kBarP, 128);
+            if (p >= 32 && p < 64) vec[p] += vec[31];
+            named_bar(kBarP, 128);
+            if (p < 64) {
+                vec[128 + p] = GATED ? __expf(vec[p]) : 1.f;
+                vec[192 + p] = GATED ? __expf(vec[63] - vec[p]) : 1.f;
+            }
+            named_bar(kBarP, 128);
+            if (p == 0) mbar_arrive(&bars[B_GATE + s]);
+            // ---- Gram rows: A^T (fp32, UT-solve input) and scale Gamma o Q K^T (fp16)
+            if (!ctl.group_wait(B_FULL + s, (c >> 1) & 1, kBarP, abort_p, p == 0)) break;
+            if (!ctl.group_wait(B_GRAM, c & 1, kBarP, abort_p, p == 0)) break;
+            tc_fence_after();
+            {
+                float v[64];
+                ld_cols<64>(trow + TM_X, v);
+                tc_fence_before();
+                if (p < 64) {
+                    const int r = p;
+                    const float br = vec[64 + r], Gr = vec[r];
+#pragma unroll
+                    for (int hf = 0; hf < 2; ++hf) {
+                        float Gs[32];   // load first, then store: no load waits on a store
+#pragma unroll
+                        for (int q4 = 0; q4 < 8; ++q4) {
+                            const float4 G4 = *reinterpret_cast<const float4 *>(vec + 32 * hf + 4 * q4);
+                            Gs[4 * q4] = G4.x; Gs[4 * q4 + 1] = G4.y; Gs[4 * q4 + 2] = G4.z; Gs[4 * q4 + 3] = G4.w;
+                        }
+                        float av[32];
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const int a = 32 * hf + e;
+                            const float dec = GATED ? __expf(Gr - Gs[e]) : 1.f;
+                            av[e] = (a < r) ? br * dec * v[a] : 0.f;
+                        }
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) At[(32 * hf + e) * 64 + r] = av[e];
+                    }
+                } else {
+                    const int r = p - 64;
+                    const float Gr = vec[r];
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) {
+                        const float4 Ga = *reinterpret_cast<const float4 *>(vec + 8 * ch);
+                        const float4 Gb = *reinterpret_cast<const float4 *>(vec + 8 * ch + 4);
+                        const float Gs[8] = {Ga.x, Ga.y, Ga.z, Ga.w, Gb.x, Gb.y, Gb.z, Gb.w};
+                        float pv[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int a = ch * 8 + e;
+                            const float dec = GATED ? __expf(Gr - Gs[e]) : 1.f;
+                            pv[e] = (a <= r) ? scale * dec * v[a] : 0.f;
+                        }
+                        st_shared_v4(sb + OFF_PG + s * 8192 + sw128(r, ch), pack_h2(pv[0], pv[1]),
+                                     pack_h2(pv[2], pv[3]), pack_h2(pv[4], pv[5]), pack_h2(pv[6], pv[7]));
+                    }
+                }
+            }
+            // ---- tiles (the Gram has read them): K, V bf16 -> fp16, Q -> Q' = fp16(scale gamma q)
+            {
+#pragma unroll
+                for (int half = 0; half < 3; ++half) {
+                    uint4 x[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        x[i] = *reinterpret_cast<const uint4 *>(st + ((half * 8 + i) * 128 + p) * 16);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const uint32_t off = ((half * 8 + i) * 128 + p) * 16;
+                        const bool isq = off < 32768u && (off & 8192u);
+                        const float f = isq ? scale * vec[128 + ((off & 8191u) >> 7)] : 1.f;
+                        x[i].x = pack_h2(f * bf_lo(x[i].x), f * bf_hi(x[i].x));
+                        x[i].y = pack_h2(f * bf_lo(x[i].y), f * bf_hi(x[i].y));
+                        x[i].z = pack_h2(f * bf_lo(x[i].z), f * bf_hi(x[i].z));
+                        x[i].w = pack_h2(f * bf_lo(x[i].w), f * bf_hi(x[i].w));
+                        *reinterpret_cast<uint4 *>(st + off) = x[i];
+                    }
+                }
+            }
+            fence_proxy_async();
+            named_bar(kBarP, 128);
+            // ---- UT solve, 2 x 2 blocks of 32: T_bb = (I + A_bb)^-1 by right-looking
+            //      substitution (warp b, lane = column), then T_10 = -T_11 (A_10 T_00)
+            if (w4 < 2) {
+                const int b = w4, col = 32 * b + lane;
+                float acc[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) acc[i] = (i == lane) ? 1.f : 0.f;
+#pragma unroll
+                for (int s2 = 0; s2 < 31; ++s2) {
+                    const float xs = acc[s2];
+                    const float *arow = At + (32 * b + s2) * 64 + 32 * b;
+#pragma unroll
+                    for (int k4 = 0; k4 < 8; ++k4) {
+                        if (4 * k4 + 3 <= s2) continue;              // rows of this group are not below s2
+                        const float4 a = *reinterpret_cast<const float4 *>(arow + 4 * k4);
+                        acc[4 * k4 + 0] = fmaf(-a.x, xs, acc[4 * k4 + 0]);
+                        acc[4 * k4 + 1] = fmaf(-a.y, xs, acc[4 * k4 + 1]);
+                        acc[4 * k4 + 2] = fmaf(-a.z, xs, acc[4 * k4 + 2]);
+                        acc[4 * k4 + 3] = fmaf(-a.w, xs, acc[4 * k4 + 3]);
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < 32; ++i) Tf[(32 * b + i) * kTP + col] = acc[i];
+                if (b == 0) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) Tf[i * kTP + 32 + lane] = 0.f;   // upper-right block
+                }
+            }
+            named_bar(kBarP, 128);
+            {
+                // X = A_10 T_00: thread -> row r (0..31), columns 8q .. 8q+7
+                const int r = p >> 2, q = p & 3;
+                float x8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+                for (int k = 0; k < 32; ++k) {
+                    const float a = At[k * 64 + 32 + r];
+                    const float4 t0v = *reinterpret_cast<const float4 *>(Tf + k * kTP + 8 * q);
+                    const float4 t1v = *reinterpret_cast<const float4 *>(Tf + k * kTP + 8 * q + 4);
+                    x8[0] = fmaf(a, t0v.x, x8[0]); x8[1] = fmaf(a, t0v.y, x8[1]);
+                    x8[2] = fmaf(a, t0v.z, x8[2]); x8[3] = fmaf(a, t0v.w, x8[3]);
+                    x8[4] = fmaf(a, t1v.x, x8[4]); x8[5] = fmaf(a, t1v.y, x8[5]);
+                    x8[6] = fmaf(a, t1v.z, x8[6]); x8[7] = fmaf(a, t1v.w, x8[7]);
+                }
+                named_bar(kBarP, 128);   // A^T fully read: X overwrites it
+                *reinterpret_cast<float4 *>(Xs + r * kXP + 8 * q) = make_float4(x8[0], x8[1], x8[2], x8[3]);
+                *reinterpret_cast<float4 *>(Xs + r * kXP + 8 * q + 4) = make_float4(x8[4], x8[5], x8[6], x8[7]);
+                named_bar(kBarP, 128);
+                // T_10 = -T_11 X
+                float y8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+                for (int k = 0; k < 32; ++k) {
+                    const float a = Tf[(32 + r) * kTP + 32 + k];
+                    const float4 x0 = *reinterpret_cast<const float4 *>(Xs + k * kXP + 8 * q);
+                    const float4 x1 = *reinterpret_cast<const float4 *>(Xs + k * kXP + 8 * q + 4);
+                    y8[0] = fmaf(a, x0.x, y8[0]); y8[1] = fmaf(a, x0.y, y8[1]);
+                    y8[2] = fmaf(a, x0.z, y8[2]); y8[3] = fmaf(a, x0.w, y8[3]);
+                    y8[4] = fmaf(a, x1.x, y8[4]); y8[5] = fmaf(a, x1.y, y8[5]);
+                    y8[6] = fmaf(a, x1.z, y8[6]); y8[7] = fmaf(a, x1.w, y8[7]);
+                }
+                *reinterpret_cast<float4 *>(Tf + (32 + r) * kTP + 8 * q) = make_float4(-y8[0], -y8[1], -y8[2], -y8[3]);
+                *reinterpret_cast<float4 *>(Tf + (32 + r) * kTP + 8 * q + 4) = make_float4(-y8[4], -y8[5], -y8[6], -y8[7]);
+            }
+            named_bar(kBarP, 128);
+            // ---- T1 = T diag(beta gamma), T2 = T diag(beta): fp16, K-major rows r (over X)
+            {
+                const int r = p >> 1, hc = p & 1;
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {
+                    const int c0 = 32 * hc + 8 * ch;
+                    const float4 ta = *reinterpret_cast<const float4 *>(Tf + r * kTP + c0);
+                    const float4 tb = *reinterpret_cast<const float4 *>(Tf + r * kTP + c0 + 4);
+                    const float4 ba = *reinterpret_cast<const float4 *>(vec + 64 + c0);
+                    const float4 bb = *reinterpret_cast<const float4 *>(vec + 64 + c0 + 4);
+                    float ga[8] = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f};
+                    if (GATED) {
+                        const float4 g0 = *reinterpret_cast<const float4 *>(vec + 128 + c0);
+                        const float4 g1 = *reinterpret_cast<const float4 *>(vec + 128 + c0 + 4);
+                        ga[0] = g0.x; ga[1] = g0.y; ga[2] = g0.z; ga[3] = g0.w;
+                        ga[4] = g1.x; ga[5] = g1.y; ga[6] = g1.z; ga[7] = g1.w;
+                    }
+                    const float t8[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
+                    const float b8[8] = {ba.x, ba.y, ba.z, ba.w, bb.x, bb.y, bb.z, bb.w};
+                    float t1[8], t2[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        t2[e] = t8[e] * b8[e];
+                        t1[e] = t2[e] * ga[e];
+                    }
+                    const int chunk = 4 * hc + ch;
+                    st_shared_v4(sb + OFF_T1 + sw128(r, chunk), pack_h2(t1[0], t1[1]), pack_h2(t1[2], t1[3]),
+                                 pack_h2(t1[4], t1[5]), pack_h2(t1[6], t1[7]));
+                    st_shared_v4(sb + OFF_T2 + sw128(r, chunk), pack_h2(t2[0], t2[1]), pack_h2(t2[2], t2[3]),
+                                 pack_h2(t2[4], t2[5]), pack_h2(t2[6], t2[7]));
+                }
+            }
+            fence_proxy_async();
+            named_bar(kBarP, 128);
+            if (p == 0) {
+                mbar_arrive(&bars[B_TRDY]);
+                mbar_arrive(&bars[B_PREP + s]);
+            }
         }
     }
+
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {

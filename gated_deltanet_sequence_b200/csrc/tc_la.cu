@@ -55,8 +55,10 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
              const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ g, float *__restrict__ o,
              const float *__restrict__ s0, float *__restrict__ s_final, int L, float scale,
              long long wait_limit, unsigned *__restrict__ err_word) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // 1024-byte aligned base derived by pointer arithmetic on the shared array, so the
+    // compiler keeps every access below in the shared address space (LDS/STS)
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sb = smem_u32(smem);
     float *Gs = reinterpret_cast<float *>(smem + OFF_VEC);
     float *gms = Gs + 64, *dss = Gs + 128;

@@ -36,6 +36,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// Named barrier over `nthreads` threads (a multiple of 32) of this CTA.
+__device__ __forceinline__ void named_bar(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
 // Wait for phase `parity` of the barrier to complete; give up after `limit` clock
 // cycles and return false (the caller records the timeout and unwinds).
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, long long limit) {
@@ -143,12 +150,13 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
     return d;
 }
 
-// Instruction descriptor of tcgen05.mma kind::f16 with fp16 A/B and fp32 D.
+// Instruction descriptor of tcgen05.mma kind::f16 with fp16 (or bf16) A/B and fp32 D.
 // a_mn / b_mn select MN-major (transposed) operands; neg_a negates A.
-__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool a_mn, bool b_mn, bool neg_a = false) {
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool a_mn, bool b_mn, bool neg_a = false,
+                                                 bool bf16 = false) {
     return (1u << 4)                                   // D format: f32
-           | (0u << 7)                                 // A format: f16
-           | (0u << 10)                                // B format: f16
+           | ((bf16 ? 1u : 0u) << 7)                   // A format: f16 / bf16
+           | ((bf16 ? 1u : 0u) << 10)                  // B format: f16 / bf16
            | ((neg_a ? 1u : 0u) << 13)                 // negate A
            | ((a_mn ? 1u : 0u) << 15)                  // A major
            | ((b_mn ? 1u : 0u) << 16)                  // B major

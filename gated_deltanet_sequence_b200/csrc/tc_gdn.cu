@@ -12,20 +12,27 @@
 //   W, U   W^T = K^T (T diag(beta gamma))^T, U^T = V^T (T diag(beta))^T
 //   Ut     Ut^T = U^T - S^T W^T   (accumulated onto U^T with a negated operand)
 //   out    O^T = S^T Q'^T + Ut^T (scale Q K^T o Gamma)^T,  Q' = diag(scale gamma) Q
-//   state  S <- gamma_last S + K^T (diag(d) Ut)
+//   state  S <- gamma_last S + (diag(d) K)^T Ut   (K scaled in place once W/U has read it)
 // Every product has dk or dv (= 128) as the UMMA M dimension, so each tcgen05.mma
 // is a full 128-lane instruction and TMEM lane = row of the result.
 //
-// Warp roles (384 threads):
+// Warp roles (512 threads):
 //   warp 0      TMA producer (2-stage ring of Q, K, V tiles)
-//   warp 1      issues the state-independent UMMAs of a chunk (Gram, W/U)
-//   warp 2      issues the state-dependent UMMAs of a chunk (U - W S, output, state)
+//   warp 1      issues the Gram UMMA of each chunk as soon as its tiles land
+//   warp 2      issues the chain UMMAs (U - W S, output, state) and the next W/U
+//   warp 3      gate warp: cumulative log-decay G, gamma = exp(G), d, exp(-G), beta
 //   warps 4-7   "state" group: S -> fp16 operand, Ut epilogue, output stores, and
 //               the W epilogue of the next chunk (in its idle slot)
-//   warps 8-11  "prep" group, one chunk ahead of the state chain: gate scan, A / P
-//               masks, tile conversion with the Q scaling, blocked UT solve
+//   warps 8-15  "prep" group, one chunk ahead of the state chain: A / P masks, the
+//               blocked UT solve on warps 8-11 (16 x 16 diagonal blocks by substitution,
+//               off-diagonal blocks by warp-level tf32 MMA) while warps 12-15 convert the
+//               tiles with the Q scaling, then the fp16 T factors
 // so the state-independent work of chunk c+1 overlaps the serial state chain of
 // chunk c. Hand-offs are mbarriers with one arrival each.
+//
+// Decay factors: Gamma_rs = exp(G_r - G_s) is formed as gamma_r * exp(-G_s) when the
+// chunk's total log-decay G_last >= -60 (both factors then stay far inside fp32
+// range); chunks with stronger decay take one exp per element instead.
 //
 // Precision: the Gram product runs on the bf16 input tiles (exact products, fp32
 // sums). Every other UMMA takes fp16 operands (10-bit mantissa): K, V are converted
@@ -70,10 +77,12 @@ using namespace ptx;
 
 constexpr int kC = 64;           // chunk rows
 constexpr int kD = 128;          // dk = dv
-constexpr int kThreads = 384;
-constexpr int kGroupS = 4;       // first warp of the state group
-constexpr int kGroupP = 8;       // first warp of the prep group
-constexpr int kBarS = 1, kBarP = 2;   // named barriers of the two 128-thread groups
+constexpr int kThreads = 512;
+constexpr int kGroupS = 4;       // first warp of the state group (4 warps)
+constexpr int kGroupP = 8;       // first warp of the prep group (8 warps)
+constexpr int kNP = 256;         // prep group threads
+constexpr int kBarS = 1, kBarP = 2;   // named barriers of the state (128) and prep (256) groups
+constexpr float kFastDecayLimit = -60.f;   // G_last >= this: Gamma = gamma_r * exp(-G_s)
 
 // ---- shared memory map (byte offsets from a 1024-aligned base) ------------------
 constexpr uint32_t kStageBytes = 49152;   // one chunk of K, Q, V
@@ -84,29 +93,30 @@ constexpr uint32_t ST_Q1 = 24576;         // Q, key columns 64-127
 constexpr uint32_t ST_V0 = 32768;         // V, value columns 0-63; holds W (MN-major, 128 key
 constexpr uint32_t ST_V1 = 40960;         //   rows x 64 r) once U has been formed
 constexpr uint32_t ST_W = ST_V0;
-constexpr uint32_t OFF_AT = 2 * kStageBytes;        // UT-solve workspace, reused in turn by:
-                                                    //   A^T fp32 64 x 64 (solve input),
-constexpr uint32_t OFF_X = OFF_AT;                  //   A_10 T_00 fp32 32 x 36 (after A^T is read),
-constexpr int kXP = 36;
-constexpr uint32_t OFF_T1 = OFF_AT;                 //   T diag(beta gamma), K-major 64 x 64 fp16,
-constexpr uint32_t OFF_T2 = OFF_AT + 8192;          //   T diag(beta)
+constexpr uint32_t OFF_AT = 2 * kStageBytes;        // A^T fp32 64 x 64 (UT-solve input)
 constexpr uint32_t OFF_TF = OFF_AT + 16384;         // T fp32 64 x 68 (pitch 68)
 constexpr int kTP = 68;
-constexpr uint32_t OFF_PG = OFF_TF + 64 * kTP * 4;  // 2 x scale (Q K^T o Gamma), K-major 64 x 64
+constexpr uint32_t OFF_R = OFF_TF + 64 * kTP * 4;   // 4 x 16 x 16 fp32 per-warp block scratch
+constexpr uint32_t OFF_PG = OFF_R + 4096;           // 2 x scale (Q K^T o Gamma), K-major 64 x 64
 constexpr uint32_t OFF_S = OFF_PG + 16384;          // S as MN-major A: 2 x (128 key rows x 64 v)
 constexpr uint32_t OFF_UB = OFF_S + 32768;          // Ut, K-major: 128 value rows x 64 s
-constexpr uint32_t OFF_UD = OFF_UB + 16384;         // diag(d) Ut, K-major
-constexpr uint32_t OFF_VEC = OFF_UD + 16384;        // 2 x {G, beta, gamma, d} (64 fp32 each)
-constexpr uint32_t OFF_BAR = OFF_VEC + 2048;        // mbarriers, TMEM base, abort flag
-constexpr uint32_t kSmemBytes = OFF_BAR + 256;
+constexpr uint32_t OFF_T1 = OFF_UB + 16384;         // T diag(beta gamma), K-major 64 x 64 fp16
+constexpr uint32_t OFF_T2 = OFF_T1 + 8192;          // T diag(beta)
+constexpr uint32_t OFF_VEC = OFF_T2 + 8192;        // 2 x {G, beta, gamma, d, exp(-G), flag}
+constexpr uint32_t kVecBytes = 1536;                //   (64 fp32 each; flag = fast decay path)
+constexpr int V_G = 0, V_B = 64, V_GAM = 128, V_D = 192, V_IG = 256, V_FAST = 320;
+constexpr uint32_t OFF_BAR = OFF_VEC + 2 * kVecBytes;   // mbarriers, TMEM base, abort flags
+constexpr uint32_t kSmemBytes = OFF_BAR + 512;
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;  // slack to align the base to 1024 B
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
-static_assert(OFF_T1 % 1024 == 0 && OFF_PG % 1024 == 0 && OFF_S % 1024 == 0, "UMMA tiles need 1024-B alignment");
+static_assert(OFF_T1 % 1024 == 0 && OFF_PG % 1024 == 0 && OFF_S % 1024 == 0 && OFF_UB % 1024 == 0,
+              "UMMA tiles need 1024-B alignment");
 
 // ---- tensor memory columns (512 allocated) ----------------------------------------
 constexpr uint32_t TM_S = 0;      // state S: lane = key row j, 128 value columns
-constexpr uint32_t TM_X = 128;    // [K;Q] K^T (64 cols s), later W^T (lane = key j, cols r)
-constexpr uint32_t TM_U = 192;    // 2 x U^T then Ut^T: lane = value v, 64 columns r
+constexpr uint32_t TM_G = 128;    // [K;Q] K^T: lanes 0-63 K K^T, 64-127 Q K^T; 64 columns s
+constexpr uint32_t TM_W = 192;    // W^T: lane = key j, 64 columns r
+constexpr uint32_t TM_U = 256;    // U^T then Ut^T: lane = value v, 64 columns r
 constexpr uint32_t TM_O = 320;    // 2 x O^T: lane = value v, 64 columns r
 
 constexpr uint32_t ID_GRAM = idesc_f16(128, 64, false, false, false, /*bf16=*/true);
@@ -122,18 +132,20 @@ constexpr uint32_t ID_O = idesc_f16(128, 64, false, false);
 // parity (waited with parity (c >> 1) & 1).
 enum : int {
     B_FULL = 0,      // [2] TMA -> prep issuer (Gram) and prep group
-    B_CDONE = 2,     // [2] state-update UMMAs of chunk c done (frees stage, U, PG, vec of parity c)
-    B_GATE = 4,      // [2] prep: G, beta, gamma, d ready   -> state group
-    B_PREP = 6,      // [2] prep: P, Q' ready               -> state issuer
-    B_GRAM = 8,      // Gram done                          -> prep group
-    B_TRDY = 9,      // prep: T1/T2, K/V fp16 written      -> prep issuer (W/U)
-    B_WU = 10,       // W/U done                           -> state group (W epilogue)
-    B_XFREE = 11,    // state group has read W^T from TM_X -> prep issuer (next Gram)
-    B_WRDY = 12,     // state group: W operand written     -> state issuer
-    B_SRDY = 13,     // state group: S operand written, S scaled -> state issuer
-    B_ADONE = 14,    // U - W S and S Q' done              -> state group (Ut epilogue)
-    B_URDY = 15,     // state group: Ut operands ready     -> state issuer
-    kNumBars = 16
+    B_CDONE = 2,     // [2] state-update UMMAs of chunk c done (frees stage, PG, vec of parity c)
+    B_GATE = 4,      // [2] gate warp: vec ready           -> state group
+    B_GATEP = 6,     // [2] gate warp: vec ready           -> prep group
+    B_PREP = 8,      // [2] prep: P, Q' ready               -> state issuer
+    B_TRDY = 10,     // [2] prep: T1/T2, K/V fp16 written  -> prep issuer (W/U)
+    B_GRAM = 12,     // Gram done                          -> prep group
+    B_GFREE = 13,    // prep group has read the Gram       -> prep issuer (next Gram)
+    B_WU = 14,       // W/U done                           -> state group (W epilogue)
+    B_XFREE = 15,    // state group has read W^T           -> prep issuer (next W/U)
+    B_WRDY = 16,     // state group: W operand written     -> state issuer
+    B_SRDY = 17,     // state group: S operand written, S scaled -> state issuer
+    B_ADONE = 18,    // U - W S and S Q' done              -> state group (Ut epilogue)
+    B_URDY = 19,     // state group: Ut operand ready (U^T read) -> chain issuer
+    kNumBars = 20
 };
 
 struct Ctl {
@@ -153,13 +165,13 @@ struct Ctl {
     }
     // bounded wait that ignores the abort flag (final drain of in-flight operations)
     __device__ __forceinline__ void drain(int b, uint32_t parity) const { mbar_wait(&bar[b], parity, limit); }
-    // Group-uniform wait for a 128-thread group: the leader polls, the group meets on
+    // Group-uniform wait for a group of warps: the leader polls, the group meets on
     // its named barrier and every thread reads the same verdict (a sticky flag), so
     // the whole group leaves its loop together.
     __device__ __forceinline__ bool group_wait(int b, uint32_t parity, int bar_id, int *group_abort,
-                                               bool leader) const {
+                                               bool leader, int nthreads = 128) const {
         if (leader && !wait(b, parity)) *reinterpret_cast<volatile int *>(group_abort) = 1;
-        named_bar(bar_id, 128);
+        named_bar(bar_id, nthreads);
         return *reinterpret_cast<volatile int *>(group_abort) == 0;
     }
 };
@@ -202,6 +214,48 @@ __device__ __forceinline__ void store_w_row(uint32_t trow_x, uint32_t wtile, int
         tmem_ld16(trow_x + cc * 16, w);
         tmem_wait_ld();
         st_row16_h(wtile, j, 2 * cc, w);
+    }
+}
+
+// warp-level tensor-core product for the small blocks of the UT solve (tf32 inputs,
+// fp32 accumulation): d += a (16 x 8, row-major) * b (8 x 8)
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t u;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(u) : "f"(x));
+    return u;
+}
+__device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// acc (16 x 16, two 16 x 8 tiles) += X (16 x 8KS) * Z (8KS x 16), both read from shared
+// memory through the accessors; lane layout of the m16n8k8 fragments (g = lane / 4,
+// t = lane % 4): A (g|g+8, t|t+4), B (t|t+4, g), D (g|g+8, 2t|2t+1)
+template <int KS, typename XF, typename ZF>
+__device__ __forceinline__ void block_mm(float (&acc)[2][4], XF xget, ZF zget, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+        const uint32_t a[4] = {to_tf32(xget(g, 8 * ks + t)), to_tf32(xget(g + 8, 8 * ks + t)),
+                               to_tf32(xget(g, 8 * ks + t + 4)), to_tf32(xget(g + 8, 8 * ks + t + 4))};
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const uint32_t b[2] = {to_tf32(zget(8 * ks + t, 8 * nt + g)), to_tf32(zget(8 * ks + t + 4, 8 * nt + g))};
+            mma_tf32_16x8x8(acc[nt], a, b);
+        }
+    }
+}
+// write a block_mm result (optionally negated) through an accessor
+template <typename WF>
+__device__ __forceinline__ void block_store(const float (&acc)[2][4], WF wput, int lane, float sgn) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        wput(g, 8 * nt + 2 * t, sgn * acc[nt][0]);
+        wput(g, 8 * nt + 2 * t + 1, sgn * acc[nt][1]);
+        wput(g + 8, 8 * nt + 2 * t, sgn * acc[nt][2]);
+        wput(g + 8, 8 * nt + 2 * t + 1, sgn * acc[nt][3]);
     }
 }
 
@@ -271,47 +325,52 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 if (last[s] >= 0) ctl.drain(B_FULL + s, (last[s] >> 1) & 1);
         }
     } else if (warp == 1) {
-        // ================================================================ prep UMMA issuer
+        // ================================================================ Gram issuer
+        // [K;Q] K^T of each chunk on its bf16 tiles, as soon as the tiles have landed and
+        // the previous Gram has been read
         if (lane == 0) {
-            int gram_last = -1, wu_last = -1;
+            int gram_last = -1;
             for (int c = 0; c < nchunks; ++c) {
                 const int s = c & 1;
                 const uint32_t stg = sb + s * kStageBytes;
                 if (!ctl.wait(B_FULL + s, (c >> 1) & 1)) break;
-                if (c >= 1 && !ctl.wait(B_XFREE, (c - 1) & 1)) break;   // W^T of chunk c-1 has left TM_X
+                if (c >= 1 && !ctl.wait(B_GFREE, (c - 1) & 1)) break;
                 tc_fence_after();
-                // [K;Q] K^T on the bf16 tiles
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
-                    mma_f16(tmem + TM_X, sdesc_sw128(stg + ST_K0 + off, 16, 1024),
+                    mma_f16(tmem + TM_G, sdesc_sw128(stg + ST_K0 + off, 16, 1024),
                             sdesc_sw128(stg + ST_K0 + off, 16, 1024), ID_GRAM, kk > 0);
                 }
                 mma_commit(&bars[B_GRAM]);
                 gram_last = c;
-                if (!ctl.wait(B_TRDY, c & 1)) break;
-                if (c >= 2 && !ctl.wait(B_CDONE + s, ((c - 2) >> 1) & 1)) break;   // U buffer s is free
+            }
+            if (gram_last >= 0) ctl.drain(B_GRAM, gram_last & 1);
+        }
+    } else if (warp == 2) {
+        // ================================================================ chain UMMA issuer
+        // per chunk: U - W S and S Q' ; state update and P Ut ; then W/U of the next chunk
+        if (lane == 0) {
+            auto wu = [&](int c) {
+                const uint32_t stg = sb + (c & 1) * kStageBytes;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_f16(tmem + TM_X, sdesc_sw128(stg + ST_K0 + kk * 2048, 16384, 1024),
+                    mma_f16(tmem + TM_W, sdesc_sw128(stg + ST_K0 + kk * 2048, 16384, 1024),
                             sdesc_sw128(sb + OFF_T1 + kk * 32, 16, 1024), ID_WU, kk > 0);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_f16(tmem + TM_U + s * 64, sdesc_sw128(stg + ST_V0 + kk * 2048, 8192, 1024),
+                    mma_f16(tmem + TM_U, sdesc_sw128(stg + ST_V0 + kk * 2048, 8192, 1024),
                             sdesc_sw128(sb + OFF_T2 + kk * 32, 16, 1024), ID_WU, kk > 0);
                 mma_commit(&bars[B_WU]);
-                wu_last = c;
+            };
+            int last_bar = -1, last_par = 0;   // last commit, for the final drain
+            if (nchunks > 0 && ctl.wait(B_TRDY, 0)) {
+                wu(0);
+                last_bar = B_WU;
+                last_par = 0;
             }
-            // UMMAs complete in issue order: the last commit covers everything issued
-            if (wu_last == gram_last && wu_last >= 0) ctl.drain(B_WU, wu_last & 1);
-            else if (gram_last >= 0) ctl.drain(B_GRAM, gram_last & 1);
-        }
-    } else if (warp == 2) {
-        // ================================================================ state UMMA issuer
-        if (lane == 0) {
-            int a_last = -1, c_last = -1;
-            for (int c = 0; c < nchunks; ++c) {
+            for (int c = 0; last_bar >= 0 && c < nchunks; ++c) {
                 const int s = c & 1;
                 const uint32_t stg = sb + s * kStageBytes;
                 if (!ctl.wait(B_PREP + s, (c >> 1) & 1)) break;
@@ -321,7 +380,7 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 // Ut^T = U^T - S^T W^T ;  O^T = S^T Q'^T
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_f16(tmem + TM_U + s * 64, sdesc_sw128(sb + OFF_S + kk * 2048, 16384, 1024),
+                    mma_f16(tmem + TM_U, sdesc_sw128(sb + OFF_S + kk * 2048, 16384, 1024),
                             sdesc_sw128(stg + ST_W + kk * 2048, 8192, 1024), ID_SW, 1u);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
@@ -330,23 +389,33 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                             sdesc_sw128(stg + ST_Q0 + off, 16, 1024), ID_SQ, kk > 0);
                 }
                 mma_commit(&bars[B_ADONE]);
-                a_last = c;
+                last_bar = B_ADONE;
+                last_par = c & 1;
                 if (!ctl.wait(B_URDY, c & 1)) break;
                 tc_fence_after();
-                // S += K^T diag(d) Ut ;  O^T += Ut^T PG^T
+                // S += (diag(d) K)^T Ut ;  O^T += Ut^T PG^T
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     mma_f16(tmem + TM_S, sdesc_sw128(stg + ST_K0 + kk * 2048, 16384, 1024),
-                            sdesc_sw128(sb + OFF_UD + kk * 32, 16, 1024), ID_ST, 1u);
+                            sdesc_sw128(sb + OFF_UB + kk * 32, 16, 1024), ID_ST, 1u);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     mma_f16(tmem + TM_O + s * 64, sdesc_sw128(sb + OFF_UB + kk * 32, 16, 1024),
                             sdesc_sw128(sb + OFF_PG + s * 8192 + kk * 32, 16, 1024), ID_O, 1u);
                 mma_commit(&bars[B_CDONE + s]);
-                c_last = c;
+                last_bar = B_CDONE + s;
+                last_par = (c >> 1) & 1;
+                if (c + 1 < nchunks) {
+                    // W/U of the next chunk: its T factors, and W^T of this chunk read
+                    if (!ctl.wait(B_TRDY + ((c + 1) & 1), ((c + 1) >> 1) & 1)) break;
+                    if (!ctl.wait(B_XFREE, c & 1)) break;
+                    wu(c + 1);
+                    last_bar = B_WU;
+                    last_par = (c + 1) & 1;
+                }
             }
-            if (c_last == a_last && c_last >= 0) ctl.drain(B_CDONE + (c_last & 1), (c_last >> 1) & 1);
-            else if (a_last >= 0) ctl.drain(B_ADONE, a_last & 1);
+            // UMMAs complete in issue order: the last commit covers everything issued
+            if (last_bar >= 0) ctl.drain(last_bar, last_par);
         }
     } else if (warp >= kGroupS && warp < kGroupS + 4) {
         // ================================================================ state group
@@ -369,33 +438,18 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             tmem_wait_st();
         }
         int done = 0;   // chunks whose output tile has been stored
-        bool ok = true;
-        // W operand of chunk 0
-        if (nchunks > 0) {
-            ok = ctl.group_wait(B_WU, 0, kBarS, abort_s, lead);
-            if (ok) {
-                tc_fence_after();
-                store_w_row(trow + TM_X, sb + ST_W, j);
-                fence_proxy_async();
-                tc_fence_before();
-                named_bar(kBarS, 128);
-                if (lead) {
-                    mbar_arrive(&bars[B_WRDY]);
-                    mbar_arrive(&bars[B_XFREE]);
-                }
-            }
-        }
 #pragma unroll 1
-        for (int c = 0; ok && c < nchunks; ++c) {
+        for (int c = 0; c < nchunks; ++c) {
             const int s = c & 1;
-            const float *vec = reinterpret_cast<const float *>(smem + OFF_VEC + s * 1024);
+            const float *vec = reinterpret_cast<const float *>(smem + OFF_VEC + s * kVecBytes);
+            uint8_t *st = smem + s * kStageBytes;
             // S(c) complete, and this chunk's gate values
             if (c >= 1 && !ctl.group_wait(B_CDONE + ((c - 1) & 1), ((c - 1) >> 1) & 1, kBarS, abort_s, lead)) break;
             if (!ctl.group_wait(B_GATE + s, (c >> 1) & 1, kBarS, abort_s, lead)) break;
             tc_fence_after();
             // ---- S row j -> fp16 MN-major operand; S <- gamma_last S (ahead of the update)
             {
-                const float gl = GATED ? vec[128 + 63] : 1.f;
+                const float gl = GATED ? vec[V_GAM + 63] : 1.f;
 #pragma unroll
                 for (int cc = 0; cc < 8; ++cc) {
                     float sv[16];
@@ -414,44 +468,52 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             tc_fence_before();
             named_bar(kBarS, 128);
             if (lead) mbar_arrive(&bars[B_SRDY]);
+            // ---- W operand of this chunk (its V slot is consumed) and K <- diag(d) K
+            //      (K's last reader before the state update was W/U)
+            if (!ctl.group_wait(B_WU, c & 1, kBarS, abort_s, lead)) break;
+            tc_fence_after();
+            store_w_row(trow + TM_W, sb + s * kStageBytes + ST_W, j);
+            if (GATED) {
+                // K tiles: 2 x 8 KB at ST_K0 / ST_K1, 64 rows of 128 B each; 1024 chunks of 16 B
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const uint32_t idx = static_cast<uint32_t>(i * 128 + j);
+                    const uint32_t off = (idx >> 9) * 16384u + ST_K0 + (idx & 511u) * 16u;
+                    const __half2 f = __float2half2_rn(vec[V_D + ((idx & 511u) >> 3)]);
+                    uint4 x = *reinterpret_cast<const uint4 *>(st + off);
+                    __half2 *hh = reinterpret_cast<__half2 *>(&x);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) hh[e] = __hmul2(hh[e], f);
+                    *reinterpret_cast<uint4 *>(st + off) = x;
+                }
+            }
+            fence_proxy_async();
+            tc_fence_before();
+            named_bar(kBarS, 128);
+            if (lead) {
+                mbar_arrive(&bars[B_WRDY]);
+                mbar_arrive(&bars[B_XFREE]);
+            }
             // ---- output of the previous chunk (its O tile is complete)
             if (c >= 1) {
                 const int cp = c - 1;
                 store_out_col(trow + TM_O + (cp & 1) * 64, o + (row0 + static_cast<size_t>(cp) * kC) * kD + j, kC);
                 done = c;
             }
-            // ---- Ut^T row v -> Ut and diag(d) Ut operands (K-major, rows v)
+            // ---- Ut^T row v -> Ut operand (K-major, rows v)
             if (!ctl.group_wait(B_ADONE, c & 1, kBarS, abort_s, lead)) break;
             tc_fence_after();
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
                 float u[16];
-                tmem_ld16(trow + TM_U + s * 64 + cc * 16, u);
+                tmem_ld16(trow + TM_U + cc * 16, u);
                 tmem_wait_ld();
                 st_row16_h(sb + OFF_UB, j, 2 * cc, u);
-                if (GATED) {
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) u[e] *= vec[192 + cc * 16 + e];
-                }
-                st_row16_h(sb + OFF_UD, j, 2 * cc, u);
             }
             fence_proxy_async();
             tc_fence_before();
             named_bar(kBarS, 128);
             if (lead) mbar_arrive(&bars[B_URDY]);
-            // ---- W operand of the next chunk (V of that stage is consumed by then)
-            if (c + 1 < nchunks) {
-                if (!ctl.group_wait(B_WU, (c + 1) & 1, kBarS, abort_s, lead)) break;
-                tc_fence_after();
-                store_w_row(trow + TM_X, sb + ((c + 1) & 1) * kStageBytes + ST_W, j);
-                fence_proxy_async();
-                tc_fence_before();
-                named_bar(kBarS, 128);
-                if (lead) {
-                    mbar_arrive(&bars[B_WRDY]);
-                    mbar_arrive(&bars[B_XFREE]);
-                }
-            }
         }
         // ---- last output tile and the final state
         if (nchunks > 0 && done == nchunks - 1) {
@@ -475,114 +537,149 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     *reinterpret_cast<float4 *>(dst + cc * 16 + e) = make_float4(sv[e], sv[e + 1], sv[e + 2], sv[e + 3]);
             }
         }
-    } else if (warp >= kGroupP && warp < kGroupP + 4) {
+    } else if (warp >= kGroupP) {
         // ================================================================ prep group
-        const int p = tid - kGroupP * 32;                // 0..127 = TMEM lane
-        const int w4 = warp & 3;
-        const uint32_t trow = tmem + (static_cast<uint32_t>(w4 * 32) << 16);
-        float *__restrict__ At = reinterpret_cast<float *>(smem + OFF_AT);   // At[s * 64 + r] = A[r][s]
-        float *__restrict__ Tf = reinterpret_cast<float *>(smem + OFF_TF);   // Tf[r * kTP + c] = T[r][c]
-        float *__restrict__ Xs = reinterpret_cast<float *>(smem + OFF_X);
-        // gate and beta of the next chunk are fetched one chunk ahead (hides HBM latency)
-        float g_next = 0.f, b_next = 0.f;
-        if (p < 64 && p < L) {
-            if (GATED) g_next = g[row0 + p];
-            b_next = beta[row0 + p];
-        }
+        const int p = tid - kGroupP * 32;                // 0..255
+        const int w8 = warp - kGroupP;                   // 0..7
+        const int sub = warp & 3;                        // TMEM lane quarter of this warp
+        const int hh = w8 >> 2;                          // which 32 of the 64 Gram columns
+        const uint32_t trow = tmem + (static_cast<uint32_t>(sub * 32) << 16);
+        float *At = reinterpret_cast<float *>(smem + OFF_AT);   // At[s * 64 + r] = A[r][s]
+        float *Tf = reinterpret_cast<float *>(smem + OFF_TF);   // Tf[r * kTP + c] = T[r][c]
 #pragma unroll 1
         for (int c = 0; c < nchunks; ++c) {
             const int s = c & 1;
-            const int t0 = c * kC;
-            const int n = min(kC, L - t0);
-            float *__restrict__ vec = reinterpret_cast<float *>(smem + OFF_VEC + s * 1024);   // G|beta|gamma|d
+            const float *vec = reinterpret_cast<const float *>(smem + OFF_VEC + s * kVecBytes);
             uint8_t *st = smem + s * kStageBytes;
-            // vec, PG and the stage of parity s are free once chunk c-2 is complete
-            if (c >= 2 && !ctl.group_wait(B_CDONE + s, ((c - 2) >> 1) & 1, kBarP, abort_p, p == 0)) break;
-            // ---- gate cumulative sum and beta (rows >= n padded: g = beta = 0)
-            if (p < 64) {
-                float x = g_next;
-                vec[64 + p] = b_next;
-                const int tn = t0 + kC + p;                          // prefetch chunk c + 1
-                g_next = (GATED && c + 1 < nchunks && tn < L) ? g[row0 + tn] : 0.f;
-                b_next = (c + 1 < nchunks && tn < L) ? beta[row0 + tn] : 0.f;
-#pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const float y = __shfl_up_sync(0xffffffffu, x, off);
-                    if (lane >= off) x += y;
-                }
-                vec[p] = x;
-            }
-            named_bar(kBarP, 128);
-            if (p >= 32 && p < 64) vec[p] += vec[31];
-            named_bar(kBarP, 128);
-            if (p < 64) {
-                vec[128 + p] = GATED ? __expf(vec[p]) : 1.f;
-                vec[192 + p] = GATED ? __expf(vec[63] - vec[p]) : 1.f;
-            }
-            named_bar(kBarP, 128);
-            if (p == 0) mbar_arrive(&bars[B_GATE + s]);
-            // ---- Gram rows: A^T (fp32, UT-solve input) and scale Gamma o Q K^T (fp16)
-            if (!ctl.group_wait(B_FULL + s, (c >> 1) & 1, kBarP, abort_p, p == 0)) break;
-            if (!ctl.group_wait(B_GRAM, c & 1, kBarP, abort_p, p == 0)) break;
+            // PG of parity s is free once chunk c-2 is complete; then this chunk's gate
+            // values, its tiles and its Gram
+            if (c >= 2 && !ctl.group_wait(B_CDONE + s, ((c - 2) >> 1) & 1, kBarP, abort_p, p == 0, kNP)) break;
+            if (!ctl.group_wait(B_GATEP + s, (c >> 1) & 1, kBarP, abort_p, p == 0, kNP)) break;
+            if (!ctl.group_wait(B_FULL + s, (c >> 1) & 1, kBarP, abort_p, p == 0, kNP)) break;
+            if (!ctl.group_wait(B_GRAM, c & 1, kBarP, abort_p, p == 0, kNP)) break;
             tc_fence_after();
+            const bool fast = !GATED || reinterpret_cast<const int *>(vec)[V_FAST] != 0;
+            // ---- Gram rows (lane quarter `sub`, columns 32 hh .. 32 hh + 31):
+            //      rows 0-63 -> A^T (fp32, UT-solve input), rows 64-127 -> scale Gamma o Q K^T
             {
-                float v[64];
-                ld_cols<64>(trow + TM_X, v);
+                float v[32];
+                ld_cols<32>(trow + TM_G + 32 * hh, v);
                 tc_fence_before();
-                if (p < 64) {
-                    const int r = p;
-                    const float br = vec[64 + r], Gr = vec[r];
+                named_bar(kBarP, kNP);                       // every Gram row has been read
+                if (p == 0) mbar_arrive(&bars[B_GFREE]);
+                const int R = sub * 32 + lane;
+                float ig[32];
 #pragma unroll
-                    for (int hf = 0; hf < 2; ++hf) {
-                        float Gs[32];   // load first, then store: no load waits on a store
+                for (int q4 = 0; q4 < 8; ++q4) {
+                    const float4 t = *reinterpret_cast<const float4 *>(vec + V_IG + 32 * hh + 4 * q4);
+                    ig[4 * q4] = t.x; ig[4 * q4 + 1] = t.y; ig[4 * q4 + 2] = t.z; ig[4 * q4 + 3] = t.w;
+                }
+                if (!fast) {
+                    // strong decay: exp(G_r - G_s) per element (ig holds G_s here)
 #pragma unroll
-                        for (int q4 = 0; q4 < 8; ++q4) {
-                            const float4 G4 = *reinterpret_cast<const float4 *>(vec + 32 * hf + 4 * q4);
-                            Gs[4 * q4] = G4.x; Gs[4 * q4 + 1] = G4.y; Gs[4 * q4 + 2] = G4.z; Gs[4 * q4 + 3] = G4.w;
-                        }
-                        float av[32];
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            const int a = 32 * hf + e;
-                            const float dec = GATED ? __expf(Gr - Gs[e]) : 1.f;
-                            av[e] = (a < r) ? br * dec * v[a] : 0.f;
-                        }
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) At[(32 * hf + e) * 64 + r] = av[e];
-                    }
-                } else {
-                    const int r = p - 64;
-                    const float Gr = vec[r];
-#pragma unroll
-                    for (int ch = 0; ch < 8; ++ch) {
-                        const float4 Ga = *reinterpret_cast<const float4 *>(vec + 8 * ch);
-                        const float4 Gb = *reinterpret_cast<const float4 *>(vec + 8 * ch + 4);
-                        const float Gs[8] = {Ga.x, Ga.y, Ga.z, Ga.w, Gb.x, Gb.y, Gb.z, Gb.w};
-                        float pv[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const int a = ch * 8 + e;
-                            const float dec = GATED ? __expf(Gr - Gs[e]) : 1.f;
-                            pv[e] = (a <= r) ? scale * dec * v[a] : 0.f;
-                        }
-                        st_shared_v4(sb + OFF_PG + s * 8192 + sw128(r, ch), pack_h2(pv[0], pv[1]),
-                                     pack_h2(pv[2], pv[3]), pack_h2(pv[4], pv[5]), pack_h2(pv[6], pv[7]));
+                    for (int q4 = 0; q4 < 8; ++q4) {
+                        const float4 t = *reinterpret_cast<const float4 *>(vec + V_G + 32 * hh + 4 * q4);
+                        ig[4 * q4] = t.x; ig[4 * q4 + 1] = t.y; ig[4 * q4 + 2] = t.z; ig[4 * q4 + 3] = t.w;
                     }
                 }
-            }
-            // ---- tiles (the Gram has read them): K, V bf16 -> fp16, Q -> Q' = fp16(scale gamma q)
-            {
+                if (R < 64) {
+                    const int r = R;
+                    float av[32];
+                    if (fast) {
+                        const float lead = vec[V_B + r] * vec[V_GAM + r];
 #pragma unroll
-                for (int half = 0; half < 3; ++half) {
+                        for (int e = 0; e < 32; ++e) av[e] = (32 * hh + e < r) ? lead * ig[e] * v[e] : 0.f;
+                    } else {
+                        const float br = vec[V_B + r], Gr = vec[V_G + r];
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) av[e] = (32 * hh + e < r) ? br * __expf(Gr - ig[e]) * v[e] : 0.f;
+                    }
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) At[(32 * hh + e) * 64 + r] = av[e];
+                } else {
+                    const int r = R - 64;
+                    float pv[32];
+                    if (fast) {
+                        const float lead = scale * vec[V_GAM + r];
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) pv[e] = (32 * hh + e <= r) ? lead * ig[e] * v[e] : 0.f;
+                    } else {
+                        const float Gr = vec[V_G + r];
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) pv[e] = (32 * hh + e <= r) ? scale * __expf(Gr - ig[e]) * v[e] : 0.f;
+                    }
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch)
+                        st_shared_v4(sb + OFF_PG + s * 8192 + sw128(r, 4 * hh + ch), pack_h2(pv[8 * ch], pv[8 * ch + 1]),
+                                     pack_h2(pv[8 * ch + 2], pv[8 * ch + 3]), pack_h2(pv[8 * ch + 4], pv[8 * ch + 5]),
+                                     pack_h2(pv[8 * ch + 6], pv[8 * ch + 7]));
+                }
+            }
+            named_bar(kBarP, kNP);
+            if (w8 < 4) {
+                // ---- UT solve. Diagonal blocks of 16: D_i = (I + A_ii)^-1 by right-looking
+                //      substitution (warp i, lane = column; lanes 16-31 mirror 0-15)
+                const int bi = w8, cl = lane & 15;
+                float acc[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) acc[i] = (i == cl) ? 1.f : 0.f;
+#pragma unroll
+                for (int s2 = 0; s2 < 15; ++s2) {
+                    const float xs = acc[s2];
+                    const float *arow = At + (16 * bi + s2) * 64 + 16 * bi;
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        if (4 * k4 + 3 <= s2) continue;              // rows of this group are not below s2
+                        const float4 a4 = *reinterpret_cast<const float4 *>(arow + 4 * k4);
+                        acc[4 * k4 + 0] = fmaf(-a4.x, xs, acc[4 * k4 + 0]);
+                        acc[4 * k4 + 1] = fmaf(-a4.y, xs, acc[4 * k4 + 1]);
+                        acc[4 * k4 + 2] = fmaf(-a4.z, xs, acc[4 * k4 + 2]);
+                        acc[4 * k4 + 3] = fmaf(-a4.w, xs, acc[4 * k4 + 3]);
+                    }
+                }
+                if (lane < 16) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) Tf[(16 * bi + i) * kTP + 16 * bi + cl] = acc[i];
+                }
+                // ---- off-diagonal blocks, one level (i - j) at a time:
+                //      T_ij = -D_i (A_{i, j..i-1} T_{j..i-1, j})  (contiguous blocks of A and T)
+                float *Rw = reinterpret_cast<float *>(smem + OFF_R) + bi * 256;
+#pragma unroll
+                for (int lev = 1; lev <= 3; ++lev) {
+                    asm volatile("bar.sync 3, 128;" ::: "memory");   // previous level of T complete
+                    const int i = bi + lev, j = bi;
+                    if (i <= 3) {
+                        float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                        auto xa = [&](int r, int k) { return At[(16 * j + k) * 64 + 16 * i + r]; };
+                        auto zt = [&](int k, int n) { return Tf[(16 * j + k) * kTP + 16 * j + n]; };
+                        if (lev == 1) block_mm<2>(acc2, xa, zt, lane);
+                        else if (lev == 2) block_mm<4>(acc2, xa, zt, lane);
+                        else block_mm<6>(acc2, xa, zt, lane);
+                        block_store(acc2, [&](int r, int n, float x) { Rw[r * 16 + n] = x; }, lane, 1.f);
+                        __syncwarp();
+                        float acc3[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                        block_mm<2>(acc3, [&](int r, int k) { return Tf[(16 * i + r) * kTP + 16 * i + k]; },
+                                    [&](int k, int n) { return Rw[k * 16 + n]; }, lane);
+                        block_store(acc3, [&](int r, int n, float x) { Tf[(16 * i + r) * kTP + 16 * j + n] = x; }, lane,
+                                    -1.f);
+                        __syncwarp();
+                    }
+                }
+            } else {
+                // ---- meanwhile (the Gram has read the tiles): K, V bf16 -> fp16 and
+                //      Q -> Q' = fp16(scale gamma q), in place; 3072 chunks of 16 B
+                const int t4 = p - 128;                      // 0..127
+#pragma unroll
+                for (int part = 0; part < 3; ++part) {
                     uint4 x[8];
 #pragma unroll
                     for (int i = 0; i < 8; ++i)
-                        x[i] = *reinterpret_cast<const uint4 *>(st + ((half * 8 + i) * 128 + p) * 16);
+                        x[i] = *reinterpret_cast<const uint4 *>(st + ((part * 8 + i) * 128 + t4) * 16);
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
-                        const uint32_t off = ((half * 8 + i) * 128 + p) * 16;
+                        const uint32_t off = ((part * 8 + i) * 128 + t4) * 16;
                         const bool isq = off < 32768u && (off & 8192u);
-                        const float f = isq ? scale * vec[128 + ((off & 8191u) >> 7)] : 1.f;
+                        const float f = isq ? scale * vec[V_GAM + ((off & 8191u) >> 7)] : 1.f;
                         x[i].x = pack_h2(f * bf_lo(x[i].x), f * bf_hi(x[i].x));
                         x[i].y = pack_h2(f * bf_lo(x[i].y), f * bf_hi(x[i].y));
                         x[i].z = pack_h2(f * bf_lo(x[i].z), f * bf_hi(x[i].z));
@@ -590,86 +687,28 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         *reinterpret_cast<uint4 *>(st + off) = x[i];
                     }
                 }
+                fence_proxy_async();
             }
-            fence_proxy_async();
-            named_bar(kBarP, 128);
-            // ---- UT solve, 2 x 2 blocks of 32: T_bb = (I + A_bb)^-1 by right-looking
-            //      substitution (warp b, lane = column), then T_10 = -T_11 (A_10 T_00)
-            if (w4 < 2) {
-                const int b = w4, col = 32 * b + lane;
-                float acc[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) acc[i] = (i == lane) ? 1.f : 0.f;
-#pragma unroll
-                for (int s2 = 0; s2 < 31; ++s2) {
-                    const float xs = acc[s2];
-                    const float *arow = At + (32 * b + s2) * 64 + 32 * b;
-#pragma unroll
-                    for (int k4 = 0; k4 < 8; ++k4) {
-                        if (4 * k4 + 3 <= s2) continue;              // rows of this group are not below s2
-                        const float4 a = *reinterpret_cast<const float4 *>(arow + 4 * k4);
-                        acc[4 * k4 + 0] = fmaf(-a.x, xs, acc[4 * k4 + 0]);
-                        acc[4 * k4 + 1] = fmaf(-a.y, xs, acc[4 * k4 + 1]);
-                        acc[4 * k4 + 2] = fmaf(-a.z, xs, acc[4 * k4 + 2]);
-                        acc[4 * k4 + 3] = fmaf(-a.w, xs, acc[4 * k4 + 3]);
-                    }
-                }
-#pragma unroll
-                for (int i = 0; i < 32; ++i) Tf[(32 * b + i) * kTP + col] = acc[i];
-                if (b == 0) {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) Tf[i * kTP + 32 + lane] = 0.f;   // upper-right block
-                }
-            }
-            named_bar(kBarP, 128);
+            // T1/T2 of chunk c-1 must have been read by its W/U before they are overwritten
+            if (c >= 1 && !ctl.group_wait(B_WU, (c - 1) & 1, kBarP, abort_p, p == 0, kNP)) break;
+            if (c == 0) named_bar(kBarP, kNP);
+            // ---- T1 = T diag(beta gamma), T2 = T diag(beta): fp16, K-major rows r;
+            //      blocks above the diagonal are zero
             {
-                // X = A_10 T_00: thread -> row r (0..31), columns 8q .. 8q+7
-                const int r = p >> 2, q = p & 3;
-                float x8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-                for (int k = 0; k < 32; ++k) {
-                    const float a = At[k * 64 + 32 + r];
-                    const float4 t0v = *reinterpret_cast<const float4 *>(Tf + k * kTP + 8 * q);
-                    const float4 t1v = *reinterpret_cast<const float4 *>(Tf + k * kTP + 8 * q + 4);
-                    x8[0] = fmaf(a, t0v.x, x8[0]); x8[1] = fmaf(a, t0v.y, x8[1]);
-                    x8[2] = fmaf(a, t0v.z, x8[2]); x8[3] = fmaf(a, t0v.w, x8[3]);
-                    x8[4] = fmaf(a, t1v.x, x8[4]); x8[5] = fmaf(a, t1v.y, x8[5]);
-                    x8[6] = fmaf(a, t1v.z, x8[6]); x8[7] = fmaf(a, t1v.w, x8[7]);
-                }
-                named_bar(kBarP, 128);   // A^T fully read: X overwrites it
-                *reinterpret_cast<float4 *>(Xs + r * kXP + 8 * q) = make_float4(x8[0], x8[1], x8[2], x8[3]);
-                *reinterpret_cast<float4 *>(Xs + r * kXP + 8 * q + 4) = make_float4(x8[4], x8[5], x8[6], x8[7]);
-                named_bar(kBarP, 128);
-                // T_10 = -T_11 X
-                float y8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-                for (int k = 0; k < 32; ++k) {
-                    const float a = Tf[(32 + r) * kTP + 32 + k];
-                    const float4 x0 = *reinterpret_cast<const float4 *>(Xs + k * kXP + 8 * q);
-                    const float4 x1 = *reinterpret_cast<const float4 *>(Xs + k * kXP + 8 * q + 4);
-                    y8[0] = fmaf(a, x0.x, y8[0]); y8[1] = fmaf(a, x0.y, y8[1]);
-                    y8[2] = fmaf(a, x0.z, y8[2]); y8[3] = fmaf(a, x0.w, y8[3]);
-                    y8[4] = fmaf(a, x1.x, y8[4]); y8[5] = fmaf(a, x1.y, y8[5]);
-                    y8[6] = fmaf(a, x1.z, y8[6]); y8[7] = fmaf(a, x1.w, y8[7]);
-                }
-                *reinterpret_cast<float4 *>(Tf + (32 + r) * kTP + 8 * q) = make_float4(-y8[0], -y8[1], -y8[2], -y8[3]);
-                *reinterpret_cast<float4 *>(Tf + (32 + r) * kTP + 8 * q + 4) = make_float4(-y8[4], -y8[5], -y8[6], -y8[7]);
-            }
-            named_bar(kBarP, 128);
-            // ---- T1 = T diag(beta gamma), T2 = T diag(beta): fp16, K-major rows r (over X)
-            {
-                const int r = p >> 1, hc = p & 1;
+                const int r = p >> 2, c0 = (p & 3) * 16;
 #pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    const int c0 = 32 * hc + 8 * ch;
-                    const float4 ta = *reinterpret_cast<const float4 *>(Tf + r * kTP + c0);
-                    const float4 tb = *reinterpret_cast<const float4 *>(Tf + r * kTP + c0 + 4);
-                    const float4 ba = *reinterpret_cast<const float4 *>(vec + 64 + c0);
-                    const float4 bb = *reinterpret_cast<const float4 *>(vec + 64 + c0 + 4);
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const int cb = c0 + 8 * h2;
+                    const bool upper = (cb >> 4) > (r >> 4);
+                    float4 ta = *reinterpret_cast<const float4 *>(Tf + r * kTP + cb);
+                    float4 tb = *reinterpret_cast<const float4 *>(Tf + r * kTP + cb + 4);
+                    if (upper) ta = tb = make_float4(0.f, 0.f, 0.f, 0.f);
+                    const float4 ba = *reinterpret_cast<const float4 *>(vec + V_B + cb);
+                    const float4 bb = *reinterpret_cast<const float4 *>(vec + V_B + cb + 4);
                     float ga[8] = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f};
                     if (GATED) {
-                        const float4 g0 = *reinterpret_cast<const float4 *>(vec + 128 + c0);
-                        const float4 g1 = *reinterpret_cast<const float4 *>(vec + 128 + c0 + 4);
+                        const float4 g0 = *reinterpret_cast<const float4 *>(vec + V_GAM + cb);
+                        const float4 g1 = *reinterpret_cast<const float4 *>(vec + V_GAM + cb + 4);
                         ga[0] = g0.x; ga[1] = g0.y; ga[2] = g0.z; ga[3] = g0.w;
                         ga[4] = g1.x; ga[5] = g1.y; ga[6] = g1.z; ga[7] = g1.w;
                     }
@@ -681,7 +720,7 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         t2[e] = t8[e] * b8[e];
                         t1[e] = t2[e] * ga[e];
                     }
-                    const int chunk = 4 * hc + ch;
+                    const int chunk = cb >> 3;
                     st_shared_v4(sb + OFF_T1 + sw128(r, chunk), pack_h2(t1[0], t1[1]), pack_h2(t1[2], t1[3]),
                                  pack_h2(t1[4], t1[5]), pack_h2(t1[6], t1[7]));
                     st_shared_v4(sb + OFF_T2 + sw128(r, chunk), pack_h2(t2[0], t2[1]), pack_h2(t2[2], t2[3]),
@@ -689,10 +728,69 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 }
             }
             fence_proxy_async();
-            named_bar(kBarP, 128);
+            named_bar(kBarP, kNP);
             if (p == 0) {
-                mbar_arrive(&bars[B_TRDY]);
+                mbar_arrive(&bars[B_TRDY + s]);
                 mbar_arrive(&bars[B_PREP + s]);
+            }
+        }
+    } else if (warp == 3) {
+        // ================================================================ gate warp
+        // lane l owns rows 2l, 2l+1 of each chunk; values of chunk c+1 are fetched one
+        // chunk ahead to hide the HBM latency
+        float g_nx[2] = {0.f, 0.f}, b_nx[2] = {0.f, 0.f};
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int t = 2 * lane + e;
+            if (t < L) {
+                if (GATED) g_nx[e] = g[row0 + t];
+                b_nx[e] = beta[row0 + t];
+            }
+        }
+        bool ok = true;
+#pragma unroll 1
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c & 1;
+            float *vec = reinterpret_cast<float *>(smem + OFF_VEC + s * kVecBytes);
+            // vec of parity s is free once chunk c-2 is complete
+            if (c >= 2) {
+                int w = 1;
+                if (lane == 0) w = ctl.wait(B_CDONE + s, ((c - 2) >> 1) & 1) ? 1 : 0;
+                ok = __shfl_sync(0xffffffffu, w, 0) != 0;
+                if (!ok) break;
+            }
+            const float g0 = g_nx[0], g1 = g_nx[1], b0 = b_nx[0], b1 = b_nx[1];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int t = (c + 1) * kC + 2 * lane + e;
+                g_nx[e] = (GATED && c + 1 < nchunks && t < L) ? g[row0 + t] : 0.f;
+                b_nx[e] = (c + 1 < nchunks && t < L) ? beta[row0 + t] : 0.f;
+            }
+            // inclusive scan of the 64 log-decays (pairs, then a warp scan of pair sums)
+            float x = g0 + g1;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, x, off);
+                if (lane >= off) x += y;
+            }
+            const float G1 = x, G0 = x - g1;
+            const float Glast = __shfl_sync(0xffffffffu, x, 31);
+            const bool fast = Glast >= kFastDecayLimit;
+            vec[V_G + 2 * lane] = G0;
+            vec[V_G + 2 * lane + 1] = G1;
+            vec[V_B + 2 * lane] = b0;
+            vec[V_B + 2 * lane + 1] = b1;
+            vec[V_GAM + 2 * lane] = GATED ? __expf(G0) : 1.f;
+            vec[V_GAM + 2 * lane + 1] = GATED ? __expf(G1) : 1.f;
+            vec[V_D + 2 * lane] = GATED ? __expf(Glast - G0) : 1.f;
+            vec[V_D + 2 * lane + 1] = GATED ? __expf(Glast - G1) : 1.f;
+            vec[V_IG + 2 * lane] = (GATED && fast) ? __expf(-G0) : 1.f;
+            vec[V_IG + 2 * lane + 1] = (GATED && fast) ? __expf(-G1) : 1.f;
+            if (lane == 0) reinterpret_cast<int *>(vec)[V_FAST] = fast ? 1 : 0;
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&bars[B_GATE + s]);
+                mbar_arrive(&bars[B_GATEP + s]);
             }
         }
     }

@@ -367,6 +367,46 @@ def run_reference(args, rank, world):
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+# ------------------------------------------------------------------------- profiling driver
+def run_profile(spec: str):
+    """Run one kernel a few times on one case (for an ncu capture; prints nothing timed).
+    spec: gdn[:B] (GDN bf16, B x 16 x 4096 x 128), la[:B] (plain LA, B x 16 x 4096 x 128),
+    decode[:N] (N x 32 heads, 3 steps), gdn_long (1 x 32 x 65536)."""
+    from gated_deltanet_sequence_b200 import _lib as gdn
+    kind, _, arg = spec.partition(":")
+    torch.cuda.set_device(0)
+    if kind in ("gdn", "la"):
+        B = int(arg or 4)
+        w = W.WORKLOADS[2 if kind == "gdn" else 1]
+        inp = W.make_prefill_inputs(B, w.H, w.L, w.dk, w.dv, mode=w.mode, in_dtype=torch.bfloat16,
+                                    seed=W.SEED_BASE + w.index, device="cuda")
+        o = torch.empty(B, w.H, w.L, w.dv, device="cuda")
+        sf = torch.empty(B, w.H, w.dk, w.dv, device="cuda")
+        for _ in range(3):
+            if kind == "gdn":
+                gdn.gdn_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["g"], o=o, s_final=sf)
+            else:
+                gdn.lin_attn_chunk_fwd(inp["q"], inp["k"], inp["v"], None, o=o, s_final=sf)
+    elif kind == "gdn_long":
+        w = W.WORKLOADS[3]
+        inp = W.make_workload_inputs(w, device="cuda")
+        o = torch.empty(w.B, w.H, w.L, w.dv, device="cuda")
+        sf = torch.empty(w.B, w.H, w.dk, w.dv, device="cuda")
+        for _ in range(2):
+            gdn.gdn_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["g"], o=o, s0=inp["s0"], s_final=sf)
+    elif kind == "decode":
+        N = int(arg or 64)
+        inp = W.make_decode_inputs(N, 32, 128, 128, 3, device="cuda", seed=W.SEED_BASE + 4)
+        for t in range(3):
+            gdn.gdn_decode_step(inp["q"][t], inp["k"][t], inp["v"][t], inp["beta"][t], inp["g"][t], inp["state"])
+    else:
+        raise SystemExit(f"unknown profile case {spec}")
+    torch.cuda.synchronize()
+    if gdn.gdn_sync_status() != 0:
+        raise SystemExit("device-side timeout")
+    print(f"profile case {spec} done")
+
+
 # ------------------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -379,7 +419,12 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--quick", action="store_true", help="shorter decode row (100 steps)")
+    ap.add_argument("--profile", default=None,
+                    help="run one kernel a few times for a profiler capture: gdn[:B] | la[:B] | decode[:N] | gdn_long")
     args = ap.parse_args()
+    if args.profile:
+        run_profile(args.profile)
+        return
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
 

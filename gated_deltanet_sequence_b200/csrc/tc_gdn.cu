@@ -544,6 +544,8 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const int sub = warp & 3;                        // TMEM lane quarter of this warp
         const int hh = w8 >> 2;                          // which 32 of the 64 Gram columns
         const uint32_t trow = tmem + (static_cast<uint32_t>(sub * 32) << 16);
+        for (int i = p; i < 16384 / 16; i += kNP)          // T1/T2: upper blocks stay zero
+            *reinterpret_cast<uint4 *>(smem + OFF_T1 + i * 16) = make_uint4(0u, 0u, 0u, 0u);
         float *At = reinterpret_cast<float *>(smem + OFF_AT);   // At[s * 64 + r] = A[r][s]
         float *Tf = reinterpret_cast<float *>(smem + OFF_TF);   // Tf[r * kTP + c] = T[r][c]
 #pragma unroll 1
@@ -615,120 +617,166 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                                      pack_h2(pv[8 * ch + 6], pv[8 * ch + 7]));
                 }
             }
-            named_bar(kBarP, kNP);
+            named_bar(kBarP, kNP);                           // A^T complete
             if (w8 < 4) {
-                // ---- UT solve. Diagonal blocks of 16: D_i = (I + A_ii)^-1 by right-looking
-                //      substitution (warp i, lane = column; lanes 16-31 mirror 0-15)
+                // ---- UT solve on warps 8-11. Blocks of T are kept in fp32 (Tf) for the
+                //      products that follow and copied, once final, into the fp16 factors
+                //      T1 = T diag(beta gamma), T2 = T diag(beta) (K-major rows r).
+                //      The upper blocks of T1/T2 are zero from the start.
+                const uint32_t sb = smem_u32(smem);
+                // one 16 x 16 block (bi, bj) of Tf -> T1/T2; lane: row lane / 2, 8 columns
+                auto emit = [&](int bi2, int bj2) {
+                    __syncwarp();
+                    const int r = 16 * bi2 + (lane >> 1), c0 = 16 * bj2 + 8 * (lane & 1);
+                    const float4 b0 = *reinterpret_cast<const float4 *>(vec + V_B + c0);
+                    const float4 b1 = *reinterpret_cast<const float4 *>(vec + V_B + c0 + 4);
+                    float4 g0 = make_float4(1.f, 1.f, 1.f, 1.f), g1 = g0;
+                    if (GATED) {
+                        g0 = *reinterpret_cast<const float4 *>(vec + V_GAM + c0);
+                        g1 = *reinterpret_cast<const float4 *>(vec + V_GAM + c0 + 4);
+                    }
+                    const float4 t0 = *reinterpret_cast<const float4 *>(Tf + r * kTP + c0);
+                    const float4 t1v = *reinterpret_cast<const float4 *>(Tf + r * kTP + c0 + 4);
+                    const float u[8] = {t0.x * b0.x, t0.y * b0.y, t0.z * b0.z, t0.w * b0.w,
+                                        t1v.x * b1.x, t1v.y * b1.y, t1v.z * b1.z, t1v.w * b1.w};
+                    const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+                    const uint32_t off = sw128(r, c0 >> 3);
+                    st_shared_v4(sb + OFF_T2 + off, pack_h2(u[0], u[1]), pack_h2(u[2], u[3]), pack_h2(u[4], u[5]),
+                                 pack_h2(u[6], u[7]));
+                    st_shared_v4(sb + OFF_T1 + off, pack_h2(u[0] * gg[0], u[1] * gg[1]),
+                                 pack_h2(u[2] * gg[2], u[3] * gg[3]), pack_h2(u[4] * gg[4], u[5] * gg[5]),
+                                 pack_h2(u[6] * gg[6], u[7] * gg[7]));
+                };
+                // diagonal blocks of 16: D_i = (I + A_ii)^-1 by right-looking substitution
+                // (warp i, lane = column; lanes 16-31 mirror 0-15)
                 const int bi = w8, cl = lane & 15;
-                float acc[16];
+                {
+                    float acc[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) acc[i] = (i == cl) ? 1.f : 0.f;
+                    for (int i = 0; i < 16; ++i) acc[i] = (i == cl) ? 1.f : 0.f;
 #pragma unroll
-                for (int s2 = 0; s2 < 15; ++s2) {
-                    const float xs = acc[s2];
-                    const float *arow = At + (16 * bi + s2) * 64 + 16 * bi;
+                    for (int s2 = 0; s2 < 15; ++s2) {
+                        const float xs = acc[s2];
+                        const float *arow = At + (16 * bi + s2) * 64 + 16 * bi;
 #pragma unroll
-                    for (int k4 = 0; k4 < 4; ++k4) {
-                        if (4 * k4 + 3 <= s2) continue;              // rows of this group are not below s2
-                        const float4 a4 = *reinterpret_cast<const float4 *>(arow + 4 * k4);
-                        acc[4 * k4 + 0] = fmaf(-a4.x, xs, acc[4 * k4 + 0]);
-                        acc[4 * k4 + 1] = fmaf(-a4.y, xs, acc[4 * k4 + 1]);
-                        acc[4 * k4 + 2] = fmaf(-a4.z, xs, acc[4 * k4 + 2]);
-                        acc[4 * k4 + 3] = fmaf(-a4.w, xs, acc[4 * k4 + 3]);
+                        for (int k4 = 0; k4 < 4; ++k4) {
+                            if (4 * k4 + 3 <= s2) continue;          // rows of this group are not below s2
+                            const float4 a4 = *reinterpret_cast<const float4 *>(arow + 4 * k4);
+                            acc[4 * k4 + 0] = fmaf(-a4.x, xs, acc[4 * k4 + 0]);
+                            acc[4 * k4 + 1] = fmaf(-a4.y, xs, acc[4 * k4 + 1]);
+                            acc[4 * k4 + 2] = fmaf(-a4.z, xs, acc[4 * k4 + 2]);
+                            acc[4 * k4 + 3] = fmaf(-a4.w, xs, acc[4 * k4 + 3]);
+                        }
+                    }
+                    if (lane < 16) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) Tf[(16 * bi + i) * kTP + 16 * bi + cl] = acc[i];
                     }
                 }
-                if (lane < 16) {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) Tf[(16 * bi + i) * kTP + 16 * bi + cl] = acc[i];
-                }
-                // ---- off-diagonal blocks, one level (i - j) at a time:
-                //      T_ij = -D_i (A_{i, j..i-1} T_{j..i-1, j})  (contiguous blocks of A and T)
-                float *Rw = reinterpret_cast<float *>(smem + OFF_R) + bi * 256;
-#pragma unroll
-                for (int lev = 1; lev <= 3; ++lev) {
-                    asm volatile("bar.sync 3, 128;" ::: "memory");   // previous level of T complete
-                    const int i = bi + lev, j = bi;
-                    if (i <= 3) {
+                // T1/T2 of chunk c-1 must have been read by its W/U before they are overwritten
+                bool ok = true;
+                if (c >= 1) ok = ctl.group_wait(B_WU, (c - 1) & 1, 3, abort_p, p == 0, 128);
+                else asm volatile("bar.sync 3, 128;" ::: "memory");
+                if (ok) {
+                    emit(bi, bi);
+                    float *Rw = reinterpret_cast<float *>(smem + OFF_R);
+                    // level 1 (warps 0, 1): T_10 = -D_1 (A_10 D_0), T_32 = -D_3 (A_32 D_2)
+                    if (bi < 2) {
+                        const int i = 2 * bi + 1, j = 2 * bi;
+                        float *R = Rw + bi * 256;
                         float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-                        auto xa = [&](int r, int k) { return At[(16 * j + k) * 64 + 16 * i + r]; };
-                        auto zt = [&](int k, int n) { return Tf[(16 * j + k) * kTP + 16 * j + n]; };
-                        if (lev == 1) block_mm<2>(acc2, xa, zt, lane);
-                        else if (lev == 2) block_mm<4>(acc2, xa, zt, lane);
-                        else block_mm<6>(acc2, xa, zt, lane);
-                        block_store(acc2, [&](int r, int n, float x) { Rw[r * 16 + n] = x; }, lane, 1.f);
+                        block_mm<2>(acc2, [&](int r, int k) { return At[(16 * j + k) * 64 + 16 * i + r]; },
+                                    [&](int k, int n) { return Tf[(16 * j + k) * kTP + 16 * j + n]; }, lane);
+                        block_store(acc2, [&](int r, int n, float x) { R[r * 16 + n] = x; }, lane, 1.f);
                         __syncwarp();
                         float acc3[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
                         block_mm<2>(acc3, [&](int r, int k) { return Tf[(16 * i + r) * kTP + 16 * i + k]; },
-                                    [&](int k, int n) { return Rw[k * 16 + n]; }, lane);
-                        block_store(acc3, [&](int r, int n, float x) { Tf[(16 * i + r) * kTP + 16 * j + n] = x; }, lane,
-                                    -1.f);
-                        __syncwarp();
+                                    [&](int k, int n) { return R[k * 16 + n]; }, lane);
+                        block_store(acc3, [&](int r, int n, float x) { Tf[(16 * i + r) * kTP + 16 * j + n] = x; },
+                                    lane, -1.f);
+                        emit(i, j);
+                    }
+                    asm volatile("bar.sync 3, 128;" ::: "memory");
+                    // level 2 (warp w -> block (i, j) = (2 + w / 2, w % 2)): X_ij = A_{i,0..1} T_{0..1,j}
+                    const int ii = 2 + (bi >> 1), jj = bi & 1;
+                    {
+                        float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                        if (jj == 0)
+                            block_mm<4>(acc2, [&](int r, int k) { return At[k * 64 + 16 * ii + r]; },
+                                        [&](int k, int n) { return Tf[k * kTP + n]; }, lane);
+                        else
+                            block_mm<2>(acc2, [&](int r, int k) { return At[(16 + k) * 64 + 16 * ii + r]; },
+                                        [&](int k, int n) { return Tf[(16 + k) * kTP + 16 + n]; }, lane);
+                        float *R = Rw + bi * 256;
+                        block_store(acc2, [&](int r, int n, float x) { R[r * 16 + n] = x; }, lane, 1.f);
+                    }
+                    asm volatile("bar.sync 3, 128;" ::: "memory");
+                    // level 3: T_2j = -D_2 X_2j,  T_3j = -(T_32 X_2j + D_3 X_3j)
+                    {
+                        const float *X2 = Rw + jj * 256, *X3 = Rw + (2 + jj) * 256;
+                        float acc3[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                        if (ii == 2)
+                            block_mm<2>(acc3, [&](int r, int k) { return Tf[(32 + r) * kTP + 32 + k]; },
+                                        [&](int k, int n) { return X2[k * 16 + n]; }, lane);
+                        else
+                            block_mm<4>(acc3, [&](int r, int k) { return Tf[(48 + r) * kTP + 32 + k]; },
+                                        [&](int k, int n) { return k < 16 ? X2[k * 16 + n] : X3[(k - 16) * 16 + n]; },
+                                        lane);
+                        // block (ii, jj) of Tf is read by no other warp at this level
+                        block_store(acc3, [&](int r, int n, float x) { Tf[(16 * ii + r) * kTP + 16 * jj + n] = x; },
+                                    lane, -1.f);
+                        emit(ii, jj);
                     }
                 }
             } else {
                 // ---- meanwhile (the Gram has read the tiles): K, V bf16 -> fp16 and
-                //      Q -> Q' = fp16(scale gamma q), in place; 3072 chunks of 16 B
+                //      Q -> Q' = fp16(scale gamma q), in place (128 threads)
                 const int t4 = p - 128;                      // 0..127
+                // K and V: 2048 chunks of 16 B at [0,8K) [16K,24K) [32K,48K)
 #pragma unroll
-                for (int part = 0; part < 3; ++part) {
+                for (int part = 0; part < 2; ++part) {
                     uint4 x[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        x[i] = *reinterpret_cast<const uint4 *>(st + ((part * 8 + i) * 128 + t4) * 16);
+                    uint32_t offs[8];
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
-                        const uint32_t off = ((part * 8 + i) * 128 + t4) * 16;
-                        const bool isq = off < 32768u && (off & 8192u);
-                        const float f = isq ? scale * vec[V_GAM + ((off & 8191u) >> 7)] : 1.f;
+                        const uint32_t idx = static_cast<uint32_t>((part * 8 + i) * 128 + t4);   // 0..2047
+                        const uint32_t reg = idx >> 9;                                            // 0..3
+                        offs[i] = (reg < 2 ? reg * 16384u : 32768u + (reg - 2) * 8192u) + (idx & 511u) * 16u;
+                        x[i] = *reinterpret_cast<const uint4 *>(st + offs[i]);
+                    }
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        x[i].x = pack_h2(bf_lo(x[i].x), bf_hi(x[i].x));
+                        x[i].y = pack_h2(bf_lo(x[i].y), bf_hi(x[i].y));
+                        x[i].z = pack_h2(bf_lo(x[i].z), bf_hi(x[i].z));
+                        x[i].w = pack_h2(bf_lo(x[i].w), bf_hi(x[i].w));
+                        *reinterpret_cast<uint4 *>(st + offs[i]) = x[i];
+                    }
+                }
+                // Q: 1024 chunks at [8K,16K) [24K,32K), row r = (offset within the box) / 128
+                {
+                    uint4 x[8];
+                    uint32_t offs[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const uint32_t idx = static_cast<uint32_t>(i * 128 + t4);                 // 0..1023
+                        offs[i] = ST_Q0 + (idx >> 9) * 16384u + (idx & 511u) * 16u;
+                        x[i] = *reinterpret_cast<const uint4 *>(st + offs[i]);
+                    }
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float f = scale * vec[V_GAM + ((offs[i] & 8191u) >> 7)];
                         x[i].x = pack_h2(f * bf_lo(x[i].x), f * bf_hi(x[i].x));
                         x[i].y = pack_h2(f * bf_lo(x[i].y), f * bf_hi(x[i].y));
                         x[i].z = pack_h2(f * bf_lo(x[i].z), f * bf_hi(x[i].z));
                         x[i].w = pack_h2(f * bf_lo(x[i].w), f * bf_hi(x[i].w));
-                        *reinterpret_cast<uint4 *>(st + off) = x[i];
+                        *reinterpret_cast<uint4 *>(st + offs[i]) = x[i];
                     }
-                }
-                fence_proxy_async();
-            }
-            // T1/T2 of chunk c-1 must have been read by its W/U before they are overwritten
-            if (c >= 1 && !ctl.group_wait(B_WU, (c - 1) & 1, kBarP, abort_p, p == 0, kNP)) break;
-            if (c == 0) named_bar(kBarP, kNP);
-            // ---- T1 = T diag(beta gamma), T2 = T diag(beta): fp16, K-major rows r;
-            //      blocks above the diagonal are zero
-            {
-                const int r = p >> 2, c0 = (p & 3) * 16;
-#pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    const int cb = c0 + 8 * h2;
-                    const bool upper = (cb >> 4) > (r >> 4);
-                    float4 ta = *reinterpret_cast<const float4 *>(Tf + r * kTP + cb);
-                    float4 tb = *reinterpret_cast<const float4 *>(Tf + r * kTP + cb + 4);
-                    if (upper) ta = tb = make_float4(0.f, 0.f, 0.f, 0.f);
-                    const float4 ba = *reinterpret_cast<const float4 *>(vec + V_B + cb);
-                    const float4 bb = *reinterpret_cast<const float4 *>(vec + V_B + cb + 4);
-                    float ga[8] = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f};
-                    if (GATED) {
-                        const float4 g0 = *reinterpret_cast<const float4 *>(vec + V_GAM + cb);
-                        const float4 g1 = *reinterpret_cast<const float4 *>(vec + V_GAM + cb + 4);
-                        ga[0] = g0.x; ga[1] = g0.y; ga[2] = g0.z; ga[3] = g0.w;
-                        ga[4] = g1.x; ga[5] = g1.y; ga[6] = g1.z; ga[7] = g1.w;
-                    }
-                    const float t8[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
-                    const float b8[8] = {ba.x, ba.y, ba.z, ba.w, bb.x, bb.y, bb.z, bb.w};
-                    float t1[8], t2[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        t2[e] = t8[e] * b8[e];
-                        t1[e] = t2[e] * ga[e];
-                    }
-                    const int chunk = cb >> 3;
-                    st_shared_v4(sb + OFF_T1 + sw128(r, chunk), pack_h2(t1[0], t1[1]), pack_h2(t1[2], t1[3]),
-                                 pack_h2(t1[4], t1[5]), pack_h2(t1[6], t1[7]));
-                    st_shared_v4(sb + OFF_T2 + sw128(r, chunk), pack_h2(t2[0], t2[1]), pack_h2(t2[2], t2[3]),
-                                 pack_h2(t2[4], t2[5]), pack_h2(t2[6], t2[7]));
                 }
             }
             fence_proxy_async();
             named_bar(kBarP, kNP);
+            if (*reinterpret_cast<volatile int *>(abort_p)) break;   // the solve warps gave up waiting
             if (p == 0) {
                 mbar_arrive(&bars[B_TRDY + s]);
                 mbar_arrive(&bars[B_PREP + s]);

@@ -8,14 +8,32 @@
 // "快速预览" / "Lightning Attention": O = (Q K^T o M) V with the diagonal included.
 // Per chunk, with G the within-chunk cumulative sum of g (0 when ungated),
 // gamma = exp(G), Gamma_rs = exp(G_r - G_s) (s <= r), d_s = exp(G_last - G_s):
-//   Gram   [K;Q] K^T (the Q K^T half is used)      M=128 UMMA
-//   QS     (Q S)^T = S^T Q^T                        M=128 (value rows)
-//   out    O^T = V^T (scale Q K^T o Gamma)^T;  o = scale gamma (QS) + O
-//   state  S <- gamma_last S + K^T diag(d) V        M=128 (key rows)
-// One CTA per (batch, head); the fp32 state stays in tensor memory; Q, K, V stream
-// through a 3-stage TMA ring because this kernel is bound by HBM bandwidth. UMMA
-// operands are fp16: the bf16 tiles are converted in place (exact in fp16 range)
-// and the computed operands (S, P, diag(d) V) are rounded to fp16.
+//   Gram   [Q;K] K^T (the Q K^T half is used)           one M=128 UMMA
+//   state  S^T <- gamma_last S^T + V^T (diag(d) K)        M=128 (value rows)
+//   out    O^T = S^T Q'^T + V^T P^T,  Q' = diag(scale gamma) Q,
+//          P = scale (Q K^T o Gamma) (s <= r)
+// One CTA per (batch, head) walks its chunks in order. The fp32 state S^T (lane =
+// value column) and its fp16 copy (the A operand of S^T Q'^T) live in tensor memory
+// for the whole sequence. The state chain per chunk is one fp32 -> fp16 pass over
+// S^T (with the decay) and four state-update UMMAs; everything else (tile loads,
+// the Gram, P, the fp16 operand conversion, the output products and the output
+// stores) is pipelined around it by dedicated warps.
+//
+// Warp roles (512 threads):
+//   warp 0      TMA producer (4-stage ring of Q, K, V tiles)
+//   warp 1      Gram issuer
+//   warp 2      gate warp (gated only): G, gamma, d, exp(-G) per chunk
+//   warp 3      chain issuer: state update, then S^T Q'^T and V^T P^T
+//   warps 4-7   state group: S^T -> fp16 copy, S^T <- gamma_last S^T
+//   warps 8-11  output group: O^T -> o; warps 8-9 also form P from the Gram
+//   warps 12-15 converter: Q -> Q', K -> diag(d) K, V -> fp16, in place
+// Hand-offs are mbarriers with one arrival each; resources used by consecutive
+// chunks (O^T, fp16 S, P, gate values) are double-buffered and their barriers are
+// indexed by chunk parity, per-stage barriers by stage.
+//
+// UMMA operands are fp16: the bf16 tiles are converted in place once the Gram has
+// read them (exact in fp16 range), the computed operands (S, P, Q', diag(d) K) are
+// rounded to fp16. Shared-memory operands use the 128-byte swizzled layouts.
 #include <mutex>
 
 #include "tc_kernels.cuh"
@@ -28,26 +46,99 @@ using namespace ptx;
 
 constexpr int kC = 64;
 constexpr int kD = 128;
-constexpr int kThreads = 128;
-constexpr int kStages = 3;
+constexpr int kThreads = 512;
+constexpr int kStages = 4;
+constexpr float kFastDecayLimit = -60.f;   // G_last >= this: Gamma = gamma_r * exp(-G_s)
 
+// ---- shared memory map (byte offsets from a 1024-aligned base) ------------------
 constexpr uint32_t kStageBytes = 49152;
-constexpr uint32_t ST_K0 = 0, ST_Q0 = 8192, ST_K1 = 16384, ST_Q1 = 24576, ST_V0 = 32768, ST_V1 = 40960;
-constexpr uint32_t OFF_PG = kStages * kStageBytes;   // scale (Q K^T o Gamma), K-major 64 x 64
-constexpr uint32_t OFF_S = OFF_PG + 8192;            // S as MN-major A: 2 x (128 key rows x 64 v)
-constexpr uint32_t OFF_VD = OFF_S + 32768;           // diag(d) V, same layout as the V tiles
-constexpr uint32_t OFF_VEC = OFF_VD + 16384;         // G, gamma, d
-constexpr uint32_t OFF_BAR = OFF_VEC + 1024;
-constexpr uint32_t kSmemBytes = OFF_BAR + 64;
-constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;
+// Each key half holds the 64 Q rows directly followed by the 64 K rows, so [Q;K] is
+// one 128-row operand of the Gram.
+constexpr uint32_t ST_Q0 = 0, ST_K0 = 8192, ST_Q1 = 16384, ST_K1 = 24576, ST_V0 = 32768, ST_V1 = 40960;
+constexpr uint32_t OFF_PG = kStages * kStageBytes;   // 2 x P, K-major 64 x 64 fp16
+constexpr uint32_t OFF_VEC = OFF_PG + 16384;         // 2 x {G, gamma, d, exp(-G), flag}
+constexpr uint32_t kVecBytes = 1536;
+constexpr int V_G = 0, V_GAM = 64, V_D = 128, V_IG = 192, V_FAST = 256;
+constexpr uint32_t OFF_BAR = OFF_VEC + 2 * kVecBytes;
+constexpr uint32_t kSmemBytes = OFF_BAR + 512;
+constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;   // slack to align the base to 1024 B
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
+static_assert(OFF_PG % 1024 == 0, "UMMA tiles need 1024-B alignment");
 
-constexpr uint32_t TM_S = 0, TM_G = 128, TM_QS = 192, TM_O = 256;
+// ---- tensor memory columns (512 allocated) ----------------------------------------
+constexpr uint32_t TM_S = 0;      // S^T fp32: lane = value v, 128 key columns
+constexpr uint32_t TM_G = 128;    // [Q;K] K^T: lanes 0-63 Q K^T (row r, column s)
+constexpr uint32_t TM_SH = 192;   // 2 x S^T fp16 (A operand): 64 columns of key pairs
+constexpr uint32_t TM_O = 320;    // 2 x O^T: lane = value v, 64 columns r
 
-constexpr uint32_t ID_GRAM = idesc_f16(128, 64, false, false);
-constexpr uint32_t ID_SQ = idesc_f16(128, 64, true, false);
-constexpr uint32_t ID_O = idesc_f16(128, 64, true, false);
+constexpr uint32_t ID_GRAM = idesc_f16(128, 64, false, false, false, /*bf16=*/true);
+constexpr uint32_t ID_SQ = idesc_f16(128, 64, false, false);
 constexpr uint32_t ID_ST = idesc_f16(128, 128, true, true);
+constexpr uint32_t ID_PV = idesc_f16(128, 64, true, false);
+
+// mbarriers. A parity wait for phase k is only correct while the producer cannot
+// complete phase k+1 first: per-stage barriers are waited with parity (c / 4) & 1,
+// per-parity ones with (c >> 1) & 1, single ones with c & 1.
+enum : int {
+    B_FULL = 0,      // [4] TMA -> Gram issuer, converter
+    B_GREAD = 4,     // [4] Gram has read the bf16 tiles of the stage -> converter
+    B_CONV = 8,      // [4] fp16 operands of the stage written -> chain issuer
+    B_SFREE = 12,    // [4] last UMMA reading the stage done -> TMA
+    B_GATE = 16,     // [2] gate values of the chunk ready -> converter, P writer, state group
+    B_ODONE = 20,    // [2] O^T of the chunk complete -> output group, gate warp, P writer
+    B_OFREE = 22,    // [2] output group has read O^T -> chain issuer
+    B_PREP = 24,     // [2] P of the chunk written -> chain issuer
+    B_GRAM = 26,     // Gram done -> P writer
+    B_GFREE = 27,    // P writer has read the Gram -> Gram issuer
+    B_SRDY = 28,     // fp16 S written and S decayed -> chain issuer
+    B_SDONE = 29,    // state update done -> state group
+    kNumBars = 30
+};
+constexpr int kBarState = 1, kBarOut = 2, kBarP = 3, kBarConv = 4;   // named barriers
+
+struct Ctl {
+    uint64_t *bar;
+    int *abort_flag;     // CTA-wide: set by the first wait that gives up
+    unsigned *err;
+    long long limit;
+    // Bounded wait; after any timeout in the CTA every later wait fails at once and
+    // each role leaves its loop without issuing further work.
+    __device__ __forceinline__ bool wait(int b, uint32_t parity) const {
+        if (*reinterpret_cast<volatile int *>(abort_flag)) return false;
+        if (mbar_wait(&bar[b], parity, limit)) return true;
+        atomicOr(err, kErrWaitTimeout);
+        *reinterpret_cast<volatile int *>(abort_flag) = 1;
+        return false;
+    }
+    __device__ __forceinline__ void drain(int b, uint32_t parity) const { mbar_wait(&bar[b], parity, limit); }
+    // Group-uniform wait: the leader polls, the group meets on its named barrier and
+    // every thread reads the same sticky verdict.
+    __device__ __forceinline__ bool group_wait(int b, uint32_t parity, int bar_id, int *group_abort, bool leader,
+                                               int nthreads) const {
+        if (leader && !wait(b, parity)) *reinterpret_cast<volatile int *>(group_abort) = 1;
+        named_bar(bar_id, nthreads);
+        return *reinterpret_cast<volatile int *>(group_abort) == 0;
+    }
+};
+
+template <int N>
+__device__ __forceinline__ void ld_cols(uint32_t taddr, float (&v)[N]) {
+    static_assert(N % 16 == 0, "16-column pieces");
+#pragma unroll
+    for (int cc = 0; cc < N / 16; ++cc) tmem_ld16(taddr + cc * 16, *reinterpret_cast<float (*)[16]>(v + cc * 16));
+    tmem_wait_ld();
+}
+
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+// 8 bf16 (one 16-byte chunk) -> 8 fp16 scaled by f
+__device__ __forceinline__ uint4 scale_chunk(uint4 x, float f) {
+    x.x = pack_h2(f * bf_lo(x.x), f * bf_hi(x.x));
+    x.y = pack_h2(f * bf_lo(x.y), f * bf_hi(x.y));
+    x.z = pack_h2(f * bf_lo(x.z), f * bf_hi(x.z));
+    x.w = pack_h2(f * bf_lo(x.w), f * bf_hi(x.w));
+    return x;
+}
 
 template <bool GATED>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -60,12 +151,11 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     // compiler keeps every access below in the shared address space (LDS/STS)
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sb = smem_u32(smem);
-    float *Gs = reinterpret_cast<float *>(smem + OFF_VEC);
-    float *gms = Gs + 64, *dss = Gs + 128;
-    uint64_t *bar_tma = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
-    uint64_t *bar_mma = bar_tma + kStages;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_mma + 1);
-    int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kNumBars);
+    int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);   // [0] CTA, [1..4] group verdicts
+    int *abort_s = abort_flag + 1, *abort_o = abort_flag + 2, *abort_cv = abort_flag + 3;
+    const Ctl ctl{bars, abort_flag, err_word, wait_limit};
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int bh = blockIdx.x;
@@ -73,13 +163,22 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     const size_t row0 = static_cast<size_t>(bh) * L;
 
     if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) mbar_init(&bar_tma[s], 1);
-        mbar_init(bar_mma, 1);
-        *abort_flag = 0;
+        for (int b = 0; b < kNumBars; ++b) mbar_init(&bars[b], 1);
+        for (int i = 0; i < 5; ++i) abort_flag[i] = 0;
         fence_mbar_init();
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
+    }
+    if (!GATED && tid < 128) {
+        // constant gate values of the ungated case, in both buffers
+        float *vec = reinterpret_cast<float *>(smem + OFF_VEC + (tid >> 6) * kVecBytes);
+        const int i = tid & 63;
+        vec[V_G + i] = 0.f;
+        vec[V_GAM + i] = 1.f;
+        vec[V_D + i] = 1.f;
+        vec[V_IG + i] = 1.f;
+        if (i == 0) reinterpret_cast<int *>(vec)[V_FAST] = 1;
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, 512);
@@ -89,231 +188,325 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
 
-    auto issue_tma = [&](int c) {
-        const int s = c % kStages;
-        uint8_t *st = smem + s * kStageBytes;
-        mbar_arrive_expect_tx(&bar_tma[s], kStageBytes);
-        tma_load_3d(st + ST_K0, &tm_k, &bar_tma[s], 0, c * kC, bh);
-        tma_load_3d(st + ST_K1, &tm_k, &bar_tma[s], 64, c * kC, bh);
-        tma_load_3d(st + ST_Q0, &tm_q, &bar_tma[s], 0, c * kC, bh);
-        tma_load_3d(st + ST_Q1, &tm_q, &bar_tma[s], 64, c * kC, bh);
-        tma_load_3d(st + ST_V0, &tm_v, &bar_tma[s], 0, c * kC, bh);
-        tma_load_3d(st + ST_V1, &tm_v, &bar_tma[s], 64, c * kC, bh);
-    };
-    if (tid == 0)
-        for (int c = 0; c < kStages && c < nchunks; ++c) issue_tma(c);
-
-    {
-        const float *src = s0 ? s0 + (static_cast<size_t>(bh) * kD + tid) * kD : nullptr;
-#pragma unroll 1
-        for (int cc = 0; cc < 8; ++cc) {
-            float r[16];
-#pragma unroll
-            for (int e = 0; e < 16; e += 4) {
-                float4 x = src ? *reinterpret_cast<const float4 *>(src + cc * 16 + e) : make_float4(0.f, 0.f, 0.f, 0.f);
-                r[e] = x.x; r[e + 1] = x.y; r[e + 2] = x.z; r[e + 3] = x.w;
+    if (warp == 0) {
+        // ================================================================ TMA producer
+        if (lane == 0) {
+            int last[kStages] = {-1, -1, -1, -1};
+            for (int c = 0; c < nchunks; ++c) {
+                const int s = c % kStages;
+                if (c >= kStages && !ctl.wait(B_SFREE + s, (c / kStages - 1) & 1)) break;
+                uint8_t *st = smem + s * kStageBytes;
+                uint64_t *fb = &bars[B_FULL + s];
+                mbar_arrive_expect_tx(fb, kStageBytes);
+                tma_load_3d(st + ST_Q0, &tm_q, fb, 0, c * kC, bh);
+                tma_load_3d(st + ST_K0, &tm_k, fb, 0, c * kC, bh);
+                tma_load_3d(st + ST_Q1, &tm_q, fb, 64, c * kC, bh);
+                tma_load_3d(st + ST_K1, &tm_k, fb, 64, c * kC, bh);
+                tma_load_3d(st + ST_V0, &tm_v, fb, 0, c * kC, bh);
+                tma_load_3d(st + ST_V1, &tm_v, fb, 64, c * kC, bh);
+                last[s] = c;
             }
-            tmem_st16(trow + TM_S + cc * 16, r);
+            // never leave a copy in flight past the end of the CTA
+            for (int s = 0; s < kStages; ++s)
+                if (last[s] >= 0) ctl.drain(B_FULL + s, (last[s] / kStages) & 1);
         }
-        tmem_wait_st();
-    }
-
-    uint32_t mma_phase = 0;
-#pragma unroll 1
-    for (int c = 0; c < nchunks; ++c) {
-        const int t0 = c * kC;
-        const int n = min(kC, L - t0);
-        const int stage = c % kStages;
-        const uint32_t stg = sb + stage * kStageBytes;
-
+    } else if (warp == 1) {
+        // ================================================================ Gram issuer
+        if (lane == 0) {
+            int last = -1;
+            for (int c = 0; c < nchunks; ++c) {
+                const int s = c % kStages;
+                const uint32_t stg = sb + s * kStageBytes;
+                if (!ctl.wait(B_FULL + s, (c / kStages) & 1)) break;
+                if (c >= 1 && !ctl.wait(B_GFREE, (c - 1) & 1)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
+                    mma_f16(tmem + TM_G, sdesc_sw128(stg + ST_Q0 + off, 16, 1024),
+                            sdesc_sw128(stg + ST_K0 + off, 16, 1024), ID_GRAM, kk > 0);
+                }
+                mma_commit(&bars[B_GRAM]);
+                mma_commit(&bars[B_GREAD + s]);
+                last = c;
+            }
+            if (last >= 0) ctl.drain(B_GREAD + last % kStages, (last / kStages) & 1);
+        }
+    } else if (warp == 2) {
+        // ================================================================ gate warp
+        // lane l owns rows 2l, 2l+1 of each chunk; values of chunk c+1 are fetched one
+        // chunk ahead to hide the HBM latency
         if (GATED) {
-            if (tid < 64) {
-                float x = (tid < n) ? g[row0 + t0 + tid] : 0.f;
+            float g_nx[2] = {0.f, 0.f};
+#pragma unroll
+            for (int e = 0; e < 2; ++e)
+                if (2 * lane + e < L) g_nx[e] = g[row0 + 2 * lane + e];
+#pragma unroll 1
+            for (int c = 0; c < nchunks; ++c) {
+                const int p = c & 1;
+                float *vec = reinterpret_cast<float *>(smem + OFF_VEC + p * kVecBytes);
+                // the gate values of parity p are free once chunk c-2 is complete
+                if (c >= 2) {
+                    int w = 1;
+                    if (lane == 0) w = ctl.wait(B_ODONE + p, ((c - 2) >> 1) & 1) ? 1 : 0;
+                    if (__shfl_sync(0xffffffffu, w, 0) == 0) break;
+                }
+                const float g0 = g_nx[0], g1 = g_nx[1];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int t = (c + 1) * kC + 2 * lane + e;
+                    g_nx[e] = (c + 1 < nchunks && t < L) ? g[row0 + t] : 0.f;
+                }
+                float x = g0 + g1;
 #pragma unroll
                 for (int off = 1; off < 32; off <<= 1) {
                     const float y = __shfl_up_sync(0xffffffffu, x, off);
                     if (lane >= off) x += y;
                 }
-                Gs[tid] = x;
-            }
-            __syncthreads();
-            if (tid >= 32 && tid < 64) Gs[tid] += Gs[31];
-            __syncthreads();
-            if (tid < 64) {
-                gms[tid] = __expf(Gs[tid]);
-                dss[tid] = __expf(Gs[63] - Gs[tid]);
+                const float G1 = x, G0 = x - g1;
+                const float Glast = __shfl_sync(0xffffffffu, x, 31);
+                const bool fast = Glast >= kFastDecayLimit;
+                vec[V_G + 2 * lane] = G0;
+                vec[V_G + 2 * lane + 1] = G1;
+                vec[V_GAM + 2 * lane] = __expf(G0);
+                vec[V_GAM + 2 * lane + 1] = __expf(G1);
+                vec[V_D + 2 * lane] = __expf(Glast - G0);
+                vec[V_D + 2 * lane + 1] = __expf(Glast - G1);
+                vec[V_IG + 2 * lane] = fast ? __expf(-G0) : 1.f;
+                vec[V_IG + 2 * lane + 1] = fast ? __expf(-G1) : 1.f;
+                if (lane == 0) reinterpret_cast<int *>(vec)[V_FAST] = fast ? 1 : 0;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[B_GATE + p]);
             }
         }
-        if (!mbar_wait(&bar_tma[stage], (c / kStages) & 1, wait_limit)) {
-            atomicOr(err_word, kErrWaitTimeout);
-            *abort_flag = 1;
-        }
-        tc_fence_before();
-        __syncthreads();
-        if (*abort_flag) break;
-        // fp16 tensor-core operands: convert this chunk's bf16 tiles in place
-        convert_tile_bf16_to_f16(smem + stage * kStageBytes, kStageBytes, tid, kThreads);
-        fence_proxy_async();
-        __syncthreads();
-
-        // ---- (1) [K;Q] K^T -> TM_G
-        if (tid == 0) {
-            tc_fence_after();
+    } else if (warp == 3) {
+        // ================================================================ chain issuer
+        if (lane == 0) {
+            int last_bar = -1, last_par = 0;
+            for (int c = 0; c < nchunks; ++c) {
+                const int s = c % kStages, p = c & 1;
+                const uint32_t stg = sb + s * kStageBytes;
+                if (!ctl.wait(B_SRDY, c & 1)) break;
+                if (!ctl.wait(B_CONV + s, (c / kStages) & 1)) break;
+                tc_fence_after();
+                // S^T += V^T (diag(d) K): the serial state chain goes first
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
-                mma_f16(tmem + TM_G, sdesc_sw128(stg + ST_K0 + off, 16, 1024),
-                         sdesc_sw128(stg + ST_K0 + off, 16, 1024), ID_GRAM, kk > 0);
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_f16(tmem + TM_S, sdesc_sw128(stg + ST_V0 + kk * 2048, 8192, 1024),
+                            sdesc_sw128(stg + ST_K0 + kk * 2048, 16384, 1024), ID_ST, 1u);
+                mma_commit(&bars[B_SDONE]);
+                last_bar = B_SDONE;
+                last_par = c & 1;
+                // O^T = S^T Q'^T into the O buffer of parity p, once chunk c-2's output was read
+                if (c >= 2 && !ctl.wait(B_OFREE + p, ((c - 2) >> 1) & 1)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
+                    mma_f16_ts(tmem + TM_O + p * 64, tmem + TM_SH + p * 64 + kk * 8,
+                               sdesc_sw128(stg + ST_Q0 + off, 16, 1024), ID_SQ, kk > 0);
+                }
+                if (!ctl.wait(B_PREP + p, (c >> 1) & 1)) {
+                    // cover the UMMAs just issued by a commit, so the final drain waits for them
+                    mma_commit(&bars[B_ODONE + p]);
+                    last_bar = B_ODONE + p;
+                    last_par = (c >> 1) & 1;
+                    break;
+                }
+                tc_fence_after();
+                // O^T += V^T P^T
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_f16(tmem + TM_O + p * 64, sdesc_sw128(stg + ST_V0 + kk * 2048, 8192, 1024),
+                            sdesc_sw128(sb + OFF_PG + p * 8192 + kk * 32, 16, 1024), ID_PV, 1u);
+                mma_commit(&bars[B_ODONE + p]);
+                mma_commit(&bars[B_SFREE + s]);
+                last_bar = B_SFREE + s;
+                last_par = (c / kStages) & 1;
             }
-            mma_commit(bar_mma);
+            // UMMAs complete in issue order: the last commit covers everything issued
+            if (last_bar >= 0) ctl.drain(last_bar, last_par);
         }
-
-        // ---- (E1a, overlapping the Gram MMA) S row j -> S tile; S <- gamma_last S;
-        //      diag(d) V tile for the gated state update
+    } else if (warp < 8) {
+        // ================================================================ state group
+        const int v = tid - 128;                          // TMEM lane = value column
+        const bool lead = (v == 0);
+        const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
         {
-            const int j = tid;
-            const float gl = GATED ? gms[63] : 1.f;
+            // S^T row v = column v of the initial state (a warp reads 32 consecutive floats)
+            const float *src = s0 ? s0 + static_cast<size_t>(bh) * kD * kD + v : nullptr;
+#pragma unroll 1
+            for (int cc = 0; cc < 8; ++cc) {
+                float r[16];
 #pragma unroll
+                for (int e = 0; e < 16; ++e) r[e] = src ? src[static_cast<size_t>(cc * 16 + e) * kD] : 0.f;
+                tmem_st16(trow + TM_S + cc * 16, r);
+            }
+            tmem_wait_st();
+        }
+        int done = -1;   // last chunk whose state update this group has seen issued
+#pragma unroll 1
+        for (int c = 0; c < nchunks; ++c) {
+            const int p = c & 1;
+            const float *vec = reinterpret_cast<const float *>(smem + OFF_VEC + p * kVecBytes);
+            if (c >= 1 && !ctl.group_wait(B_SDONE, (c - 1) & 1, kBarState, abort_s, lead, 128)) break;
+            if (GATED && !ctl.group_wait(B_GATE + p, (c >> 1) & 1, kBarState, abort_s, lead, 128)) break;
+            tc_fence_after();
+            // S^T row v -> fp16 pairs (A operand of S^T Q'^T); S <- gamma_last S
+            const float gl = GATED ? vec[V_GAM + 63] : 1.f;
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                float sv[32];
+                ld_cols<32>(trow + TM_S + h * 32, sv);
+                float hv[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) hv[e] = __uint_as_float(pack_h2(sv[2 * e], sv[2 * e + 1]));
+                tmem_st16(trow + TM_SH + p * 64 + h * 16, hv);
+                if (GATED) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) sv[e] *= gl;
+                    tmem_st16(trow + TM_S + h * 32, *reinterpret_cast<float (*)[16]>(sv));
+                    tmem_st16(trow + TM_S + h * 32 + 16, *reinterpret_cast<float (*)[16]>(sv + 16));
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            named_bar(kBarState, 128);
+            if (lead) mbar_arrive(&bars[B_SRDY]);
+            done = c;
+        }
+        if (s_final && nchunks > 0 && done == nchunks - 1 &&
+            ctl.group_wait(B_SDONE, (nchunks - 1) & 1, kBarState, abort_s, lead, 128)) {
+            tc_fence_after();
+            // column v of the final state (a warp writes 32 consecutive floats)
+            float *dst = s_final + static_cast<size_t>(bh) * kD * kD + v;
+#pragma unroll 1
             for (int cc = 0; cc < 8; ++cc) {
                 float sv[16];
                 tmem_ld16(trow + TM_S + cc * 16, sv);
                 tmem_wait_ld();
-                const uint32_t base = sb + OFF_S + (cc >> 2) * 16384u;
-                const int ch = (cc & 3) * 2;
-                st_shared_v4(base + sw128(j, ch), pack_h2(sv[0], sv[1]), pack_h2(sv[2], sv[3]),
-                             pack_h2(sv[4], sv[5]), pack_h2(sv[6], sv[7]));
-                st_shared_v4(base + sw128(j, ch + 1), pack_h2(sv[8], sv[9]), pack_h2(sv[10], sv[11]),
-                             pack_h2(sv[12], sv[13]), pack_h2(sv[14], sv[15]));
-                if (GATED) {
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) sv[e] *= gl;
-                    tmem_st16(trow + TM_S + cc * 16, sv);
+                for (int e = 0; e < 16; ++e) dst[static_cast<size_t>(cc * 16 + e) * kD] = sv[e];
+            }
+        }
+    } else if (warp < 12) {
+        // ================================================================ output group
+        const int v = tid - 256;                          // TMEM lane = value column
+        const bool lead = (v == 0);
+        const bool pw = warp < 10;                        // P writers: Gram rows 0-63
+        const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+        auto store_out = [&](int c) -> bool {
+            const int p = c & 1;
+            if (!ctl.group_wait(B_ODONE + p, (c >> 1) & 1, kBarOut, abort_o, lead, 128)) return false;
+            tc_fence_after();
+            float ov[64];
+            ld_cols<64>(trow + TM_O + p * 64, ov);
+            tc_fence_before();
+            named_bar(kBarOut, 128);
+            if (lead) mbar_arrive(&bars[B_OFREE + p]);
+            const int n = min(kC, L - c * kC);
+            float *ocol = o + (row0 + static_cast<size_t>(c) * kC) * kD + v;
+#pragma unroll
+            for (int r = 0; r < 64; ++r)
+                if (r < n) ocol[static_cast<size_t>(r) * kD] = ov[r];
+            return true;
+        };
+#pragma unroll 1
+        for (int c = 0; c < nchunks; ++c) {
+            const int p = c & 1;
+            if (pw) {
+                // ---- P = scale (Q K^T o Gamma), s <= r, row r = v (0..63) -> PG (fp16)
+                const float *vec = reinterpret_cast<const float *>(smem + OFF_VEC + p * kVecBytes);
+                const bool pl = (v == 0);
+                bool ok = true;
+                if (c >= 2) ok = ctl.group_wait(B_ODONE + p, ((c - 2) >> 1) & 1, kBarP, abort_o, pl, 64);
+                if (ok && GATED) ok = ctl.group_wait(B_GATE + p, (c >> 1) & 1, kBarP, abort_o, pl, 64);
+                if (ok) ok = ctl.group_wait(B_GRAM, c & 1, kBarP, abort_o, pl, 64);
+                if (ok) {
+                    tc_fence_after();
+                    float x[64];
+                    ld_cols<64>(trow + TM_G, x);
+                    tc_fence_before();
+                    named_bar(kBarP, 64);
+                    if (pl) mbar_arrive(&bars[B_GFREE]);
+                    const int r = v;
+                    const bool fast = !GATED || reinterpret_cast<const int *>(vec)[V_FAST] != 0;
+                    if (fast) {
+                        const float fr = scale * (GATED ? vec[V_GAM + r] : 1.f);
+#pragma unroll
+                        for (int s2 = 0; s2 < 64; ++s2)
+                            x[s2] = (s2 <= r) ? fr * x[s2] * (GATED ? vec[V_IG + s2] : 1.f) : 0.f;
+                    } else {
+                        const float Gr = vec[V_G + r];
+#pragma unroll
+                        for (int s2 = 0; s2 < 64; ++s2)
+                            x[s2] = (s2 <= r) ? scale * x[s2] * __expf(Gr - vec[V_G + s2]) : 0.f;
+                    }
+                    const uint32_t prow = sb + OFF_PG + p * 8192;
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch)
+                        st_shared_v4(prow + sw128(r, ch), pack_h2(x[8 * ch], x[8 * ch + 1]),
+                                     pack_h2(x[8 * ch + 2], x[8 * ch + 3]), pack_h2(x[8 * ch + 4], x[8 * ch + 5]),
+                                     pack_h2(x[8 * ch + 6], x[8 * ch + 7]));
+                    fence_proxy_async();
+                    named_bar(kBarP, 64);
+                    if (pl) mbar_arrive(&bars[B_PREP + p]);
                 }
             }
-            if (GATED) {
-                tmem_wait_st();
-                // 16 KB of V (1024 chunks of 16 B): chunk at byte offset b sits in row (b / 128) % 64
+            // group-uniform checkpoint: the P writers' verdict reaches warps 10-11 too
+            named_bar(kBarOut, 128);
+            if (*reinterpret_cast<volatile int *>(abort_o)) break;
+            // ---- output of the previous chunk
+            if (c >= 1 && !store_out(c - 1)) break;
+        }
+        if (nchunks > 0 && *reinterpret_cast<volatile int *>(abort_o) == 0) store_out(nchunks - 1);
+    } else {
+        // ================================================================ converter
+        // Q -> fp16(scale gamma_r q), K -> fp16(d_s k), V -> fp16, in place, once the Gram
+        // has read the bf16 tiles
+        const int t = tid - 384;                          // 0..127
+        const bool lead = (t == 0);
+#pragma unroll 1
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c % kStages, p = c & 1;
+            const float *vec = reinterpret_cast<const float *>(smem + OFF_VEC + p * kVecBytes);
+            uint8_t *st = smem + s * kStageBytes;
+            if (!ctl.group_wait(B_FULL + s, (c / kStages) & 1, kBarConv, abort_cv, lead, 128)) break;
+            if (GATED && !ctl.group_wait(B_GATE + p, (c >> 1) & 1, kBarConv, abort_cv, lead, 128)) break;
+            if (!ctl.group_wait(B_GREAD + s, (c / kStages) & 1, kBarConv, abort_cv, lead, 128)) break;
+            // 3 x 1024 chunks of 16 B; chunk i of a tensor sits in box i / 512 (key or value
+            // half), row (i % 512) / 8 of that box
+#pragma unroll
+            for (int part = 0; part < 3; ++part) {
+                uint4 x[8];
+                uint32_t off[8];
+                float f[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    const uint32_t b = (i * kThreads + tid) * 16u;
-                    const int row = (b >> 7) & 63;
-                    const uint4 x = *reinterpret_cast<const uint4 *>(smem + stage * kStageBytes + ST_V0 + b);
-                    const float dsc = dss[row];
-                    const __half2 *h = reinterpret_cast<const __half2 *>(&x);
-                    uint32_t y[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 f = __half22float2(h[e]);
-                        y[e] = pack_h2(f.x * dsc, f.y * dsc);
+                    const uint32_t idx = static_cast<uint32_t>(i * 128 + t);     // 0..1023
+                    const uint32_t box = idx >> 9, row = (idx & 511u) >> 3;
+                    if (part == 0) {
+                        off[i] = ST_Q0 + box * 16384u + (idx & 511u) * 16u;
+                        f[i] = scale * (GATED ? vec[V_GAM + row] : 1.f);
+                    } else if (part == 1) {
+                        off[i] = ST_K0 + box * 16384u + (idx & 511u) * 16u;
+                        f[i] = GATED ? vec[V_D + row] : 1.f;
+                    } else {
+                        off[i] = ST_V0 + box * 8192u + (idx & 511u) * 16u;
+                        f[i] = 1.f;
                     }
-                    st_shared_v4(sb + OFF_VD + b, y[0], y[1], y[2], y[3]);
+                    x[i] = *reinterpret_cast<const uint4 *>(st + off[i]);
                 }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) *reinterpret_cast<uint4 *>(st + off[i]) = scale_chunk(x[i], f[i]);
             }
+            fence_proxy_async();
+            named_bar(kBarConv, 128);
+            if (lead) mbar_arrive(&bars[B_CONV + s]);
         }
-        if (!mbar_wait(bar_mma, mma_phase, wait_limit)) {
-            atomicOr(err_word, kErrWaitTimeout);
-            *abort_flag = 1;
-        }
-        mma_phase ^= 1;
-        tc_fence_after();
-        // ---- (E1b) rows 64-127 of the Gram: scale Gamma_rs q_r.k_s (s <= r) -> PG (bf16)
-        if (warp >= 2) {
-            const int r = tid - 64;
-            float v[64];
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                float t16[16];
-                tmem_ld16(trow + TM_G + cc * 16, t16);
-#pragma unroll
-                for (int e = 0; e < 16; ++e) v[cc * 16 + e] = t16[e];
-            }
-            tmem_wait_ld();
-            const float Gr = GATED ? Gs[r] : 0.f;
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-                uint32_t pk[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int s = ch * 8 + 2 * e;
-                    const float w0 = GATED ? __expf(Gr - Gs[s]) : 1.f;
-                    const float w1 = GATED ? __expf(Gr - Gs[s + 1]) : 1.f;
-                    const float p0 = (s <= r) ? scale * w0 * v[s] : 0.f;
-                    const float p1 = (s + 1 <= r) ? scale * w1 * v[s + 1] : 0.f;
-                    pk[e] = pack_h2(p0, p1);
-                }
-                st_shared_v4(sb + OFF_PG + sw128(r, ch), pk[0], pk[1], pk[2], pk[3]);
-            }
-        }
-        fence_proxy_async();
-        tc_fence_before();
-        __syncthreads();
-
-        // ---- (2) (Q S)^T -> TM_QS ; O^T = V^T PG^T -> TM_O ; S += K^T diag(d) V
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
-                mma_f16(tmem + TM_QS, sdesc_sw128(sb + OFF_S + kk * 2048, 16384, 1024),
-                         sdesc_sw128(stg + ST_Q0 + off, 16, 1024), ID_SQ, kk > 0);
-            }
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_f16(tmem + TM_O, sdesc_sw128(stg + ST_V0 + kk * 2048, 8192, 1024),
-                         sdesc_sw128(sb + OFF_PG + kk * 32, 16, 1024), ID_O, kk > 0);
-            const uint32_t vb = GATED ? sb + OFF_VD : stg + ST_V0;
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_f16(tmem + TM_S, sdesc_sw128(stg + ST_K0 + kk * 2048, 16384, 1024),
-                         sdesc_sw128(vb + kk * 2048, 8192, 1024), ID_ST, 1u);
-            mma_commit(bar_mma);
-        }
-        if (!mbar_wait(bar_mma, mma_phase, wait_limit)) {
-            atomicOr(err_word, kErrWaitTimeout);
-            *abort_flag = 1;
-        }
-        mma_phase ^= 1;
-        tc_fence_after();
-        if (tid == 0 && c + kStages < nchunks) issue_tma(c + kStages);
-
-        // ---- (E2) o[r][v] = scale gamma_r (Q S)[r][v] + O[r][v]
-        {
-            const int vcol = tid;
-            float *orow = o + (row0 + t0) * kD + vcol;
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                float qs[16], ov[16];
-                tmem_ld16(trow + TM_QS + cc * 16, qs);
-                tmem_ld16(trow + TM_O + cc * 16, ov);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int r = cc * 16 + e;
-                    const float gr = GATED ? gms[r] : 1.f;
-                    if (r < n) orow[static_cast<size_t>(r) * kD] = fmaf(scale * gr, qs[e], ov[e]);
-                }
-            }
-        }
-        tc_fence_before();
-        __syncthreads();
-        if (*abort_flag) break;
     }
 
-    if (!*abort_flag && s_final) {
-        tc_fence_after();
-        float *dst = s_final + (static_cast<size_t>(bh) * kD + tid) * kD;
-#pragma unroll 1
-        for (int cc = 0; cc < 8; ++cc) {
-            float sv[16];
-            tmem_ld16(trow + TM_S + cc * 16, sv);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 16; e += 4)
-                *reinterpret_cast<float4 *>(dst + cc * 16 + e) = make_float4(sv[e], sv[e + 1], sv[e + 2], sv[e + 3]);
-        }
-    }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {

@@ -8,7 +8,7 @@
 // "快速预览" / "Lightning Attention": O = (Q K^T o M) V with the diagonal included.
 // Per chunk, with G the within-chunk cumulative sum of g (0 when ungated),
 // gamma = exp(G), Gamma_rs = exp(G_r - G_s) (s <= r), d_s = exp(G_last - G_s):
-//   Gram   [Q;K] K^T (the Q K^T half is used)           one M=128 UMMA
+//   Gram   [K;Q] K^T (the Q K^T half is used)           one M=128 UMMA
 //   state  S^T <- gamma_last S^T + V^T (diag(d) K)        M=128 (value rows)
 //   out    O^T = S^T Q'^T + V^T P^T,  Q' = diag(scale gamma) Q,
 //          P = scale (Q K^T o Gamma) (s <= r)
@@ -19,14 +19,16 @@
 // the Gram, P, the fp16 operand conversion, the output products and the output
 // stores) is pipelined around it by dedicated warps.
 //
-// Warp roles (512 threads):
+// Warp roles (640 threads):
 //   warp 0      TMA producer (4-stage ring of Q, K, V tiles)
 //   warp 1      Gram issuer
 //   warp 2      gate warp (gated only): G, gamma, d, exp(-G) per chunk
 //   warp 3      chain issuer: state update, then S^T Q'^T and V^T P^T
 //   warps 4-7   state group: S^T -> fp16 copy, S^T <- gamma_last S^T
-//   warps 8-11  output group: O^T -> o; warps 8-9 also form P from the Gram
-//   warps 12-15 converter: Q -> Q', K -> diag(d) K, V -> fp16, in place
+//   warps 8-11  output group: O^T -> o
+//   warps 12-15 converter: Q -> Q', K -> diag(d) K, in place
+//   warps 16-17 V -> fp16, in place
+//   warps 18-19 P writers (Gram rows 64-127: Q K^T)
 // Hand-offs are mbarriers with one arrival each; resources used by consecutive
 // chunks (O^T, fp16 S, P, gate values) are double-buffered and their barriers are
 // indexed by chunk parity, per-stage barriers by stage.
@@ -46,15 +48,15 @@ using namespace ptx;
 
 constexpr int kC = 64;
 constexpr int kD = 128;
-constexpr int kThreads = 512;
+constexpr int kThreads = 640;
 constexpr int kStages = 4;
 constexpr float kFastDecayLimit = -60.f;   // G_last >= this: Gamma = gamma_r * exp(-G_s)
 
 // ---- shared memory map (byte offsets from a 1024-aligned base) ------------------
 constexpr uint32_t kStageBytes = 49152;
-// Each key half holds the 64 Q rows directly followed by the 64 K rows, so [Q;K] is
+// Each key half holds the 64 K rows directly followed by the 64 Q rows, so [K;Q] is
 // one 128-row operand of the Gram.
-constexpr uint32_t ST_Q0 = 0, ST_K0 = 8192, ST_Q1 = 16384, ST_K1 = 24576, ST_V0 = 32768, ST_V1 = 40960;
+constexpr uint32_t ST_K0 = 0, ST_Q0 = 8192, ST_K1 = 16384, ST_Q1 = 24576, ST_V0 = 32768, ST_V1 = 40960;
 constexpr uint32_t OFF_PG = kStages * kStageBytes;   // 2 x P, K-major 64 x 64 fp16
 constexpr uint32_t OFF_VEC = OFF_PG + 16384;         // 2 x {G, gamma, d, exp(-G), flag}
 constexpr uint32_t kVecBytes = 1536;
@@ -67,9 +69,9 @@ static_assert(OFF_PG % 1024 == 0, "UMMA tiles need 1024-B alignment");
 
 // ---- tensor memory columns (512 allocated) ----------------------------------------
 constexpr uint32_t TM_S = 0;      // S^T fp32: lane = value v, 128 key columns
-constexpr uint32_t TM_G = 128;    // [Q;K] K^T: lanes 0-63 Q K^T (row r, column s)
-constexpr uint32_t TM_SH = 192;   // 2 x S^T fp16 (A operand): 64 columns of key pairs
-constexpr uint32_t TM_O = 320;    // 2 x O^T: lane = value v, 64 columns r
+constexpr uint32_t TM_G = 128;    // 2 x [K;Q] K^T: lanes 64-127 Q K^T (row r, column s)
+constexpr uint32_t TM_SH = 256;   // 2 x S^T fp16 (A operand): 64 columns of key pairs
+constexpr uint32_t TM_O = 384;    // 2 x O^T: lane = value v, 64 columns r
 
 constexpr uint32_t ID_GRAM = idesc_f16(128, 64, false, false, false, /*bf16=*/true);
 constexpr uint32_t ID_SQ = idesc_f16(128, 64, false, false);
@@ -81,20 +83,21 @@ constexpr uint32_t ID_PV = idesc_f16(128, 64, true, false);
 // per-parity ones with (c >> 1) & 1, single ones with c & 1.
 enum : int {
     B_FULL = 0,      // [4] TMA -> Gram issuer, converter
-    B_GREAD = 4,     // [4] Gram has read the bf16 tiles of the stage -> converter
-    B_CONV = 8,      // [4] fp16 operands of the stage written -> chain issuer
+    B_GREAD = 4,     // [4] Gram has read the bf16 Q, K tiles of the stage -> converter
+    B_CONV = 8,      // [4] Q', diag(d) K of the stage written -> chain issuer
     B_SFREE = 12,    // [4] last UMMA reading the stage done -> TMA
-    B_GATE = 16,     // [2] gate values of the chunk ready -> converter, P writer, state group
+    B_GATE = 16,     // [2] gate values of the chunk ready -> converter, P writers, state group
     B_ODONE = 20,    // [2] O^T of the chunk complete -> output group, gate warp, P writer
     B_OFREE = 22,    // [2] output group has read O^T -> chain issuer
     B_PREP = 24,     // [2] P of the chunk written -> chain issuer
-    B_GRAM = 26,     // Gram done -> P writer
-    B_GFREE = 27,    // P writer has read the Gram -> Gram issuer
-    B_SRDY = 28,     // fp16 S written and S decayed -> chain issuer
-    B_SDONE = 29,    // state update done -> state group
-    kNumBars = 30
+    B_GRAM = 26,     // [2] Gram of the chunk done -> P writer
+    B_GFREE = 28,    // [2] P writer has read the Gram -> Gram issuer
+    B_VCONV = 30,    // [4] V of the stage converted to fp16 -> chain issuer
+    B_SRDY = 34,     // fp16 S written and S decayed -> chain issuer
+    B_SDONE = 35,    // state update done -> state group
+    kNumBars = 36
 };
-constexpr int kBarState = 1, kBarOut = 2, kBarP = 3, kBarConv = 4;   // named barriers
+constexpr int kBarState = 1, kBarOut = 2, kBarP = 3, kBarConv = 4, kBarV = 5;   // named barriers
 
 struct Ctl {
     uint64_t *bar;
@@ -155,6 +158,7 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kNumBars);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);   // [0] CTA, [1..4] group verdicts
     int *abort_s = abort_flag + 1, *abort_o = abort_flag + 2, *abort_cv = abort_flag + 3;
+    int *abort_v = abort_flag + 4, *abort_p = abort_flag + 5;
     const Ctl ctl{bars, abort_flag, err_word, wait_limit};
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -164,7 +168,7 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 
     if (tid == 0) {
         for (int b = 0; b < kNumBars; ++b) mbar_init(&bars[b], 1);
-        for (int i = 0; i < 5; ++i) abort_flag[i] = 0;
+        for (int i = 0; i < 6; ++i) abort_flag[i] = 0;
         fence_mbar_init();
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
@@ -218,16 +222,17 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             for (int c = 0; c < nchunks; ++c) {
                 const int s = c % kStages;
                 const uint32_t stg = sb + s * kStageBytes;
+                const int p = c & 1;
                 if (!ctl.wait(B_FULL + s, (c / kStages) & 1)) break;
-                if (c >= 1 && !ctl.wait(B_GFREE, (c - 1) & 1)) break;
+                if (c >= 2 && !ctl.wait(B_GFREE + p, ((c - 2) >> 1) & 1)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
-                    mma_f16(tmem + TM_G, sdesc_sw128(stg + ST_Q0 + off, 16, 1024),
+                    mma_f16(tmem + TM_G + p * 64, sdesc_sw128(stg + ST_K0 + off, 16, 1024),
                             sdesc_sw128(stg + ST_K0 + off, 16, 1024), ID_GRAM, kk > 0);
                 }
-                mma_commit(&bars[B_GRAM]);
+                mma_commit(&bars[B_GRAM + p]);
                 mma_commit(&bars[B_GREAD + s]);
                 last = c;
             }
@@ -289,6 +294,7 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 const uint32_t stg = sb + s * kStageBytes;
                 if (!ctl.wait(B_SRDY, c & 1)) break;
                 if (!ctl.wait(B_CONV + s, (c / kStages) & 1)) break;
+                if (!ctl.wait(B_VCONV + s, (c / kStages) & 1)) break;
                 tc_fence_after();
                 // S^T += V^T (diag(d) K): the serial state chain goes first
 #pragma unroll
@@ -394,11 +400,11 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         // ================================================================ output group
         const int v = tid - 256;                          // TMEM lane = value column
         const bool lead = (v == 0);
-        const bool pw = warp < 10;                        // P writers: Gram rows 0-63
         const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-        auto store_out = [&](int c) -> bool {
+#pragma unroll 1
+        for (int c = 0; c < nchunks; ++c) {
             const int p = c & 1;
-            if (!ctl.group_wait(B_ODONE + p, (c >> 1) & 1, kBarOut, abort_o, lead, 128)) return false;
+            if (!ctl.group_wait(B_ODONE + p, (c >> 1) & 1, kBarOut, abort_o, lead, 128)) break;
             tc_fence_after();
             float ov[64];
             ld_cols<64>(trow + TM_O + p * 64, ov);
@@ -410,62 +416,83 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 #pragma unroll
             for (int r = 0; r < 64; ++r)
                 if (r < n) ocol[static_cast<size_t>(r) * kD] = ov[r];
-            return true;
-        };
+        }
+    } else if (warp >= 18) {
+        // ================================================================ P writers
+        // P = scale (Q K^T o Gamma), s <= r, row r (Gram lane 64 + r) -> PG (fp16)
+        const int r = tid - 576;                          // 0..63
+        const bool pl = (r == 0);
+        const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
 #pragma unroll 1
         for (int c = 0; c < nchunks; ++c) {
             const int p = c & 1;
-            if (pw) {
-                // ---- P = scale (Q K^T o Gamma), s <= r, row r = v (0..63) -> PG (fp16)
-                const float *vec = reinterpret_cast<const float *>(smem + OFF_VEC + p * kVecBytes);
-                const bool pl = (v == 0);
-                bool ok = true;
-                if (c >= 2) ok = ctl.group_wait(B_ODONE + p, ((c - 2) >> 1) & 1, kBarP, abort_o, pl, 64);
-                if (ok && GATED) ok = ctl.group_wait(B_GATE + p, (c >> 1) & 1, kBarP, abort_o, pl, 64);
-                if (ok) ok = ctl.group_wait(B_GRAM, c & 1, kBarP, abort_o, pl, 64);
-                if (ok) {
-                    tc_fence_after();
-                    float x[64];
-                    ld_cols<64>(trow + TM_G, x);
+            const float *vec = reinterpret_cast<const float *>(smem + OFF_VEC + p * kVecBytes);
+            // PG of parity p is free once chunk c-2 is complete
+            if (c >= 2 && !ctl.group_wait(B_ODONE + p, ((c - 2) >> 1) & 1, kBarP, abort_p, pl, 64)) break;
+            if (GATED && !ctl.group_wait(B_GATE + p, (c >> 1) & 1, kBarP, abort_p, pl, 64)) break;
+            if (!ctl.group_wait(B_GRAM + p, (c >> 1) & 1, kBarP, abort_p, pl, 64)) break;
+            tc_fence_after();
+            const bool fast = !GATED || reinterpret_cast<const int *>(vec)[V_FAST] != 0;
+            const float fr = scale * (GATED ? vec[V_GAM + r] : 1.f);
+            const float Gr = GATED ? vec[V_G + r] : 0.f;
+            const uint32_t prow = sb + OFF_PG + p * 8192;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float x[32];
+                ld_cols<32>(trow + TM_G + p * 64 + h * 32, x);
+                if (h == 1) {
+                    // both halves of the Gram row are in registers: release the buffer
                     tc_fence_before();
                     named_bar(kBarP, 64);
-                    if (pl) mbar_arrive(&bars[B_GFREE]);
-                    const int r = v;
-                    const bool fast = !GATED || reinterpret_cast<const int *>(vec)[V_FAST] != 0;
-                    if (fast) {
-                        const float fr = scale * (GATED ? vec[V_GAM + r] : 1.f);
-#pragma unroll
-                        for (int s2 = 0; s2 < 64; ++s2)
-                            x[s2] = (s2 <= r) ? fr * x[s2] * (GATED ? vec[V_IG + s2] : 1.f) : 0.f;
-                    } else {
-                        const float Gr = vec[V_G + r];
-#pragma unroll
-                        for (int s2 = 0; s2 < 64; ++s2)
-                            x[s2] = (s2 <= r) ? scale * x[s2] * __expf(Gr - vec[V_G + s2]) : 0.f;
-                    }
-                    const uint32_t prow = sb + OFF_PG + p * 8192;
-#pragma unroll
-                    for (int ch = 0; ch < 8; ++ch)
-                        st_shared_v4(prow + sw128(r, ch), pack_h2(x[8 * ch], x[8 * ch + 1]),
-                                     pack_h2(x[8 * ch + 2], x[8 * ch + 3]), pack_h2(x[8 * ch + 4], x[8 * ch + 5]),
-                                     pack_h2(x[8 * ch + 6], x[8 * ch + 7]));
-                    fence_proxy_async();
-                    named_bar(kBarP, 64);
-                    if (pl) mbar_arrive(&bars[B_PREP + p]);
+                    if (pl) mbar_arrive(&bars[B_GFREE + p]);
                 }
+                if (fast) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        x[e] = (32 * h + e <= r) ? fr * (GATED ? vec[V_IG + 32 * h + e] : 1.f) * x[e] : 0.f;
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        x[e] = (32 * h + e <= r) ? scale * __expf(Gr - vec[V_G + 32 * h + e]) * x[e] : 0.f;
+                }
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch)
+                    st_shared_v4(prow + sw128(r, 4 * h + ch), pack_h2(x[8 * ch], x[8 * ch + 1]),
+                                 pack_h2(x[8 * ch + 2], x[8 * ch + 3]), pack_h2(x[8 * ch + 4], x[8 * ch + 5]),
+                                 pack_h2(x[8 * ch + 6], x[8 * ch + 7]));
             }
-            // group-uniform checkpoint: the P writers' verdict reaches warps 10-11 too
-            named_bar(kBarOut, 128);
-            if (*reinterpret_cast<volatile int *>(abort_o)) break;
-            // ---- output of the previous chunk
-            if (c >= 1 && !store_out(c - 1)) break;
+            fence_proxy_async();
+            named_bar(kBarP, 64);
+            if (pl) mbar_arrive(&bars[B_PREP + p]);
         }
-        if (nchunks > 0 && *reinterpret_cast<volatile int *>(abort_o) == 0) store_out(nchunks - 1);
+    } else if (warp >= 16) {
+        // ================================================================ V converter
+        // V (2 x 8 KB, 1024 chunks of 16 B) -> fp16 in place once the tiles have landed
+        const int t = tid - 512;                          // 0..63
+        const bool lead = (t == 0);
+#pragma unroll 1
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c % kStages;
+            if (!ctl.group_wait(B_FULL + s, (c / kStages) & 1, kBarV, abort_v, lead, 64)) break;
+            uint8_t *vt = smem + s * kStageBytes + ST_V0;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint4 x[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) x[i] = *reinterpret_cast<const uint4 *>(vt + ((h * 8 + i) * 64 + t) * 16);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    *reinterpret_cast<uint4 *>(vt + ((h * 8 + i) * 64 + t) * 16) = scale_chunk(x[i], 1.f);
+            }
+            fence_proxy_async();
+            named_bar(kBarV, 64);
+            if (lead) mbar_arrive(&bars[B_VCONV + s]);
+        }
     } else {
-        // ================================================================ converter
+        // ================================================================ Q / K converter
         // Q -> fp16(scale gamma_r q), K -> fp16(d_s k), V -> fp16, in place, once the Gram
         // has read the bf16 tiles
-        const int t = tid - 384;                          // 0..127
+        const int t = tid - 384;                          // 0..127 (warps 12-15)
         const bool lead = (t == 0);
 #pragma unroll 1
         for (int c = 0; c < nchunks; ++c) {
@@ -475,10 +502,10 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             if (!ctl.group_wait(B_FULL + s, (c / kStages) & 1, kBarConv, abort_cv, lead, 128)) break;
             if (GATED && !ctl.group_wait(B_GATE + p, (c >> 1) & 1, kBarConv, abort_cv, lead, 128)) break;
             if (!ctl.group_wait(B_GREAD + s, (c / kStages) & 1, kBarConv, abort_cv, lead, 128)) break;
-            // 3 x 1024 chunks of 16 B; chunk i of a tensor sits in box i / 512 (key or value
-            // half), row (i % 512) / 8 of that box
+            // 2 x 1024 chunks of 16 B; chunk i of a tensor sits in box i / 512 (key half),
+            // row (i % 512) / 8 of that box (V is converted by the state group)
 #pragma unroll
-            for (int part = 0; part < 3; ++part) {
+            for (int part = 0; part < 2; ++part) {
                 uint4 x[8];
                 uint32_t off[8];
                 float f[8];
@@ -489,12 +516,9 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     if (part == 0) {
                         off[i] = ST_Q0 + box * 16384u + (idx & 511u) * 16u;
                         f[i] = scale * (GATED ? vec[V_GAM + row] : 1.f);
-                    } else if (part == 1) {
+                    } else {
                         off[i] = ST_K0 + box * 16384u + (idx & 511u) * 16u;
                         f[i] = GATED ? vec[V_D + row] : 1.f;
-                    } else {
-                        off[i] = ST_V0 + box * 8192u + (idx & 511u) * 16u;
-                        f[i] = 1.f;
                     }
                     x[i] = *reinterpret_cast<const uint4 *>(st + off[i]);
                 }

@@ -259,7 +259,7 @@ def measure_rows(gdn, peaks, peak_src, args):
     ms = timed(fn, max(5, args.steps), 3)
     nb = prefill_bytes(w.B, w.H, w.L, w.dk, w.dv, 2, False, False, False, False)
     fl = flops_per_head_token("la", w.dk, w.dv, w.chunk) * w.B * w.H * w.L
-    rows["la_prefill"] = _row(w, ms, nb, fl, peaks, peak_src, "hbm", w.B * w.L)
+    rows["la_prefill"] = _row(w, ms, nb, fl, peaks, peak_src, "hbm", w.B * w.L, "lin_attn_tc")
     del inp, o
     # long-context Gated DeltaNet, 1 x 32 x 65536 x 128, S0 != 0
     w = W.WORKLOADS[3]
@@ -302,12 +302,13 @@ def measure_rows(gdn, peaks, peak_src, args):
     return rows
 
 
-def _row(w, ms, nbytes, flop, peaks, peak_src, bound, tokens):
+def _row(w, ms, nbytes, flop, peaks, peak_src, bound, tokens, traffic_key=None):
     gbs = nbytes / (ms * 1e-3) / 1e9
     tfs = flop / (ms * 1e-3) / 1e12
     return {"workload": w.name, "ms_per_launch": round(ms, 4), "tokens_per_s": round(tokens / (ms * 1e-3), 1),
             "roofline": {"bound": bound, "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_source": peak_src,
+                         "traffic": traffic_from_profiles(traffic_key) if traffic_key else None,
                          "algorithmic_bytes_per_launch": nbytes},
             "tensor": {"achieved": round(tfs, 1), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                        "frac": round(tfs / peaks["bf16_tflops"], 4)}}

@@ -274,6 +274,26 @@ def measure_rows(gdn, peaks, peak_src, args):
     rows["gdn_prefill_long"] = _row(w, ms, nb, fl, peaks, peak_src, "hbm", w.B * w.L)
     del inp, o, sf
     torch.cuda.empty_cache()
+    # packed variable-length Gated DeltaNet: 24 sequences (log-uniform length mix), 16 heads
+    wv = W.VARLEN_WORKLOAD
+    lens = W.draw_seqlens(wv["N"], wv["T"], seed=wv["seed"], min_len=wv["min_len"])
+    inp = W.make_varlen_inputs(lens, wv["H"], 128, 128, mode="gdn", in_dtype=torch.bfloat16,
+                               seed=wv["seed"], device="cuda")
+    T, H, N = wv["T"], wv["H"], wv["N"]
+    o = torch.empty(H, T, 128, device="cuda")
+    sf = torch.empty(N, H, 128, 128, device="cuda")
+    fn = lambda: gdn.gdn_chunk_fwd_varlen(inp["q"], inp["k"], inp["v"], inp["beta"], inp["cu_seqlens"],
+                                          inp["g"], o=o, s_final=sf)
+    ms = timed(fn, max(5, args.steps), 3)
+    # per-token bytes as a (1, H, T) batch, plus one final state per (sequence, head)
+    nb = prefill_bytes(1, H, T, 128, 128, 2, True, True, False, False) + N * H * 128 * 128 * 4
+    fl = flops_per_head_token("gdn", 128, 128, 64) * H * T
+    row = _row(w, ms, nb, fl, peaks, peak_src, "hbm", T)
+    row["workload"] = wv["name"]
+    row["seqlens"] = {"n": N, "min": min(lens), "max": max(lens), "total": T}
+    rows["gdn_prefill_varlen"] = row
+    del inp, o, sf
+    torch.cuda.empty_cache()
     # decode: 256 sequences x 32 heads, 1000 consecutive steps, state in place
     w = W.WORKLOADS[4]
     steps = w.L if not args.quick else 100

@@ -21,8 +21,8 @@ LIB_PATH = os.path.join(_HERE, "libgdn.so")
 GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_TIMEOUT = range(5)
 GDN_F32, GDN_BF16 = 0, 1
 
-EXPORTS = ("lin_attn_chunk_fwd", "gdn_chunk_fwd", "gdn_decode_step", "gdn_status_str",
-           "gdn_sync_status", "gdn_version")
+EXPORTS = ("lin_attn_chunk_fwd", "gdn_chunk_fwd", "lin_attn_chunk_fwd_varlen", "gdn_chunk_fwd_varlen",
+           "gdn_decode_step", "gdn_status_str", "gdn_sync_status", "gdn_version")
 
 
 class GdnError(RuntimeError):
@@ -39,13 +39,15 @@ def _load() -> ctypes.CDLL:
     P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
     lib.lin_attn_chunk_fwd.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
     lib.gdn_chunk_fwd.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
+    lib.lin_attn_chunk_fwd_varlen.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
+    lib.gdn_chunk_fwd_varlen.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
     lib.gdn_decode_step.argtypes = [P, P, P, P, P, P, P, I, I, I, I, F, I, P]
     lib.gdn_status_str.argtypes = [I]
     lib.gdn_status_str.restype = ctypes.c_char_p
     lib.gdn_sync_status.argtypes = [P]
     lib.gdn_version.argtypes = []
-    for f in (lib.lin_attn_chunk_fwd, lib.gdn_chunk_fwd, lib.gdn_decode_step, lib.gdn_sync_status,
-              lib.gdn_version):
+    for f in (lib.lin_attn_chunk_fwd, lib.gdn_chunk_fwd, lib.lin_attn_chunk_fwd_varlen,
+              lib.gdn_chunk_fwd_varlen, lib.gdn_decode_step, lib.gdn_sync_status, lib.gdn_version):
         f.restype = ctypes.c_int
     return lib
 
@@ -139,6 +141,60 @@ def gdn_chunk_fwd(q, k, v, beta, g=None, o=None, s0=None, s_final=None, chunk: i
                            _ptr(s_final), B, H, L, dk, dv, int(chunk), float(scale),
                            _dtype_code(q), _stream(stream))
     _raise("gdn_chunk_fwd", st)
+    return o, s_final
+
+
+def _check_varlen(q, k, v, cu_seqlens, s0, s_final):
+    if q.dim() != 3:
+        raise ValueError(f"q: expected (H, T, dk), got shape {tuple(q.shape)}")
+    H, T, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    _check("q", q, (H, T, dk), device=dev)
+    _check("k", k, (H, T, dk), q.dtype, dev)
+    _check("v", v, (H, T, dv), q.dtype, dev)
+    if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2:
+        raise ValueError("cu_seqlens: expected (N + 1,) with N >= 1")
+    _check("cu_seqlens", cu_seqlens, (cu_seqlens.numel(),), torch.int32, dev)
+    N = cu_seqlens.numel() - 1
+    _check("s0", s0, (N, H, dk, dv), torch.float32, dev, required=False)
+    _check("s_final", s_final, (N, H, dk, dv), torch.float32, dev, required=False)
+    return N, H, T, dk, dv, dev
+
+
+def lin_attn_chunk_fwd_varlen(q, k, v, cu_seqlens, g=None, o=None, s0=None, s_final=None,
+                              chunk: int = 64, scale: float = 1.0, stream=None):
+    """Packed variable-length batch of plain / gated linear attention.
+
+    q, k (H, T, dk); v (H, T, dv); g (H, T) or None; cu_seqlens (N + 1,) int32 on the device
+    (sequence n is tokens cu[n] .. cu[n+1]-1 of every head). s0, s_final (N, H, dk, dv).
+    Returns (o, s_final); rows outside every sequence are left as they were in ``o``."""
+    N, H, T, dk, dv, dev = _check_varlen(q, k, v, cu_seqlens, s0, s_final)
+    _check("g", g, (H, T), torch.float32, dev, required=False)
+    if o is None:
+        o = torch.zeros(H, T, dv, dtype=torch.float32, device=dev)
+    _check("o", o, (H, T, dv), torch.float32, dev)
+    st = lib.lin_attn_chunk_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(o), _ptr(s0),
+                                       _ptr(s_final), _ptr(cu_seqlens), N, H, T, dk, dv, int(chunk),
+                                       float(scale), _dtype_code(q), _stream(stream))
+    _raise("lin_attn_chunk_fwd_varlen", st)
+    return o, s_final
+
+
+def gdn_chunk_fwd_varlen(q, k, v, beta, cu_seqlens, g=None, o=None, s0=None, s_final=None,
+                         chunk: int = 64, scale: float = 1.0, stream=None):
+    """Packed variable-length batch of DeltaNet / Gated DeltaNet (see lin_attn_chunk_fwd_varlen);
+    beta (H, T) fp32."""
+    N, H, T, dk, dv, dev = _check_varlen(q, k, v, cu_seqlens, s0, s_final)
+    _check("beta", beta, (H, T), torch.float32, dev, required=T > 0)
+    _check("g", g, (H, T), torch.float32, dev, required=False)
+    if o is None:
+        o = torch.zeros(H, T, dv, dtype=torch.float32, device=dev)
+    _check("o", o, (H, T, dv), torch.float32, dev)
+    st = lib.gdn_chunk_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(o), _ptr(s0),
+                                  _ptr(s_final), _ptr(cu_seqlens), N, H, T, dk, dv, int(chunk),
+                                  float(scale), _dtype_code(q), _stream(stream))
+    _raise("gdn_chunk_fwd_varlen", st)
     return o, s_final
 
 

@@ -55,9 +55,9 @@ gdn_status_t lin_attn_chunk_fwd(const void *q, const void *k, const void *v, con
     if (st != GDN_OK) return st;
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
     if (gdn::tc_supported(in_dtype, dk, dv, chunk) && L > 0)
-        return gdn::launch_tc_la(q, k, v, g, o, s0, s_final, B, H, L, scale, stream);
-    return gdn::launch_simt_fwd(q, k, v, nullptr, g, o, s0, s_final, B, H, L, dk, dv, chunk, scale,
-                                in_dtype, stream);
+        return gdn::launch_tc_la(q, k, v, g, o, s0, s_final, nullptr, B, H, L, scale, stream);
+    return gdn::launch_simt_fwd(q, k, v, nullptr, g, o, s0, s_final, nullptr, B, H, L, dk, dv, chunk,
+                                scale, in_dtype, stream);
 }
 
 gdn_status_t gdn_chunk_fwd(const void *q, const void *k, const void *v, const float *beta,
@@ -70,10 +70,43 @@ gdn_status_t gdn_chunk_fwd(const void *q, const void *k, const void *v, const fl
     if (!opt_aligned4(beta)) return GDN_ERR_INVALID_ARG;
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
     if (gdn::tc_supported(in_dtype, dk, dv, chunk) && L > 0)
-        return gdn::launch_tc_gdn(q, k, v, beta, g, o, s0, s_final, B, H, L, scale, stream);
+        return gdn::launch_tc_gdn(q, k, v, beta, g, o, s0, s_final, nullptr, B, H, L, scale, stream);
     // with L == 0 beta may be NULL: the kernel then only writes s0 (or zeros) to s_final
-    return gdn::launch_simt_fwd(q, k, v, beta, g, o, s0, s_final, B, H, L, dk, dv, chunk, scale,
-                                in_dtype, stream);
+    return gdn::launch_simt_fwd(q, k, v, beta, g, o, s0, s_final, nullptr, B, H, L, dk, dv, chunk,
+                                scale, in_dtype, stream);
+}
+
+gdn_status_t lin_attn_chunk_fwd_varlen(const void *q, const void *k, const void *v, const float *g,
+                                       float *o, const float *s0, float *s_final,
+                                       const int *cu_seqlens, int N, int H, int T, int dk, int dv,
+                                       int chunk, float scale, gdn_dtype_t in_dtype,
+                                       void *cuda_stream) {
+    if (N < 1 || !cu_seqlens || !opt_aligned4(cu_seqlens)) return GDN_ERR_INVALID_ARG;
+    gdn_status_t st = check_prefill(q, k, v, g, o, s0, s_final, 1, H, T, dk, dv, chunk, scale, in_dtype);
+    if (st != GDN_OK) return st;
+    if ((double)N * H > 2147483647.0) return GDN_ERR_INVALID_ARG;
+    cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+    if (gdn::tc_supported(in_dtype, dk, dv, chunk) && T > 0)
+        return gdn::launch_tc_la(q, k, v, g, o, s0, s_final, cu_seqlens, N, H, T, scale, stream);
+    return gdn::launch_simt_fwd(q, k, v, nullptr, g, o, s0, s_final, cu_seqlens, N, H, T, dk, dv, chunk,
+                                scale, in_dtype, stream);
+}
+
+gdn_status_t gdn_chunk_fwd_varlen(const void *q, const void *k, const void *v, const float *beta,
+                                  const float *g, float *o, const float *s0, float *s_final,
+                                  const int *cu_seqlens, int N, int H, int T, int dk, int dv, int chunk,
+                                  float scale, gdn_dtype_t in_dtype, void *cuda_stream) {
+    if (N < 1 || !cu_seqlens || !opt_aligned4(cu_seqlens)) return GDN_ERR_INVALID_ARG;
+    gdn_status_t st = check_prefill(q, k, v, g, o, s0, s_final, 1, H, T, dk, dv, chunk, scale, in_dtype);
+    if (st != GDN_OK) return st;
+    if ((double)N * H > 2147483647.0) return GDN_ERR_INVALID_ARG;
+    if (T > 0 && !beta) return GDN_ERR_INVALID_ARG;
+    if (!opt_aligned4(beta)) return GDN_ERR_INVALID_ARG;
+    cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+    if (gdn::tc_supported(in_dtype, dk, dv, chunk) && T > 0)
+        return gdn::launch_tc_gdn(q, k, v, beta, g, o, s0, s_final, cu_seqlens, N, H, T, scale, stream);
+    return gdn::launch_simt_fwd(q, k, v, beta, g, o, s0, s_final, cu_seqlens, N, H, T, dk, dv, chunk,
+                                scale, in_dtype, stream);
 }
 
 gdn_status_t gdn_decode_step(const void *q, const void *k, const void *v, const float *beta,
@@ -96,6 +129,7 @@ gdn_status_t gdn_sync_status(void *cuda_stream) {
     if (cudaStreamSynchronize(stream) != cudaSuccess) return GDN_ERR_CUDA;
     unsigned err = 0u;
     if (!gdn::read_and_clear_device_error(&err)) return GDN_ERR_CUDA;
+    if (err & gdn::kErrBadSeqlens) return GDN_ERR_INVALID_ARG;
     return err ? GDN_ERR_TIMEOUT : GDN_OK;
 }
 

@@ -8,9 +8,31 @@
 
 namespace gdn {
 
-// Codes a kernel ORs into the device-side error word when it gives up on a
-// bounded wait (the word lives in the tensor-core translation unit).
-enum : unsigned { kErrWaitTimeout = 1u };
+// Codes a kernel ORs into the device-side error word (the word lives in the
+// tensor-core translation unit): a bounded wait gave up, or a packed batch's
+// sequence offsets were not a non-decreasing list inside [0, T].
+enum : unsigned { kErrWaitTimeout = 1u, kErrBadSeqlens = 2u };
+
+// Token range of the (sequence, head) handled by CTA `bid`. Dense batches
+// (cu == nullptr): one sequence of length L per row of the (B*H, L) token grid.
+// Packed variable-length batches: sequence n of head h is tokens cu[n] .. cu[n+1]-1
+// of row h of an (H, L) token grid (CTA bid = n * H + h). A malformed range is
+// recorded in the error word and handled as an empty sequence.
+struct SeqSpan {
+    int head_row;   // row of the token grid (and z coordinate of the TMA maps)
+    int t0;         // first token of the sequence in that row
+    int len;        // tokens in the sequence
+};
+__device__ __forceinline__ SeqSpan seq_span(const int *cu, int bid, int H, int L, unsigned *err) {
+    if (!cu) return SeqSpan{bid, 0, L};
+    const int n = bid / H, h = bid - n * H;
+    const int a = cu[n], b = cu[n + 1];
+    if (a < 0 || b < a || b > L) {
+        if (err && threadIdx.x == 0) atomicOr(err, kErrBadSeqlens);
+        return SeqSpan{h, 0, 0};
+    }
+    return SeqSpan{h, a, b - a};
+}
 
 template <typename T> __device__ __forceinline__ float ld_in(const T *p);
 template <> __device__ __forceinline__ float ld_in<float>(const float *p) { return *p; }
@@ -40,10 +62,12 @@ __device__ __forceinline__ void st_global4(float *p, float4 v) {
 
 // Host-side launchers implemented in the kernel translation units.
 namespace gdn {
+// cu (device, nullable): sequence offsets of a packed batch; B is then the number of
+// sequences and L the packed length T of each head row.
 gdn_status_t launch_simt_fwd(const void *q, const void *k, const void *v, const float *beta,
-                             const float *g, float *o, const float *s0, float *s_final, int B,
-                             int H, int L, int dk, int dv, int chunk, float scale,
-                             gdn_dtype_t in_dtype, cudaStream_t stream);
+                             const float *g, float *o, const float *s0, float *s_final,
+                             const int *cu, int B, int H, int L, int dk, int dv, int chunk,
+                             float scale, gdn_dtype_t in_dtype, cudaStream_t stream);
 gdn_status_t launch_decode(const void *q, const void *k, const void *v, const float *beta,
                            const float *g, float *state, float *o, int N, int H, int dk, int dv,
                            float scale, gdn_dtype_t in_dtype, cudaStream_t stream);

@@ -14,6 +14,7 @@
 //   O = diag(gamma) Q S + (Q K^T o Gamma) Ut
 //   S <- gamma_n S + sum_s exp(G_n - G_s) k_s Ut_s^T
 #include "common.cuh"
+#include "tc_kernels.cuh"
 
 namespace gdn {
 namespace {
@@ -44,21 +45,25 @@ __global__ void __launch_bounds__(kSimtThreads)
 simt_chunk_fwd_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT *__restrict__ v,
                       const float *__restrict__ beta, const float *__restrict__ g,
                       float *__restrict__ o, const float *__restrict__ s0,
-                      float *__restrict__ s_final, int L, int dv, int C, float scale) {
+                      float *__restrict__ s_final, const int *__restrict__ cu, int H, int Lrow,
+                      int dv, int C, float scale, unsigned *__restrict__ err) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     using Sm = SimtSmem<DK>;
     Sm &sm = *reinterpret_cast<Sm *>(smem_raw);
     constexpr int KP = Sm::KP, CP = Sm::CP;
     const int tid = threadIdx.x;
-    const long bh = blockIdx.x;
+    const long bh = blockIdx.x;                  // (sequence, head): state index
     const int c0 = blockIdx.y * kDvs;            // first value column of this CTA
+    const SeqSpan sp = seq_span(cu, blockIdx.x, H, Lrow, err);
+    const int L = sp.len;                        // tokens of this sequence
+    const long r0 = (long)sp.head_row * Lrow + sp.t0;   // its first row in the token grid
 
-    const IT *qh = q + bh * (long)L * DK;
-    const IT *kh = k + bh * (long)L * DK;
-    const IT *vh = v + bh * (long)L * dv;
-    const float *bh_beta = DELTA ? beta + bh * (long)L : nullptr;
-    const float *bh_g = g ? g + bh * (long)L : nullptr;
-    float *oh = o + bh * (long)L * dv;
+    const IT *qh = q + r0 * DK;
+    const IT *kh = k + r0 * DK;
+    const IT *vh = v + r0 * dv;
+    const float *bh_beta = DELTA ? beta + r0 : nullptr;
+    const float *bh_g = g ? g + r0 : nullptr;
+    float *oh = o + r0 * dv;
 
     for (int i = tid; i < DK * kDvs; i += kSimtThreads) {
         const int j = i / kDvs, c = i % kDvs;
@@ -185,31 +190,34 @@ simt_chunk_fwd_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const 
 
 template <int DK, typename IT, bool DELTA>
 gdn_status_t launch_simt_t(const void *q, const void *k, const void *v, const float *beta,
-                           const float *g, float *o, const float *s0, float *s_final, int BH,
-                           int L, int dv, int chunk, float scale, cudaStream_t stream) {
+                           const float *g, float *o, const float *s0, float *s_final, const int *cu,
+                           int BH, int H, int L, int dv, int chunk, float scale, unsigned *err,
+                           cudaStream_t stream) {
     auto kern = simt_chunk_fwd_kernel<DK, IT, DELTA>;
     const int smem = (int)sizeof(SimtSmem<DK>);
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return GDN_ERR_CUDA;
     dim3 grid(BH, dv / kDvs);
     kern<<<grid, kSimtThreads, smem, stream>>>((const IT *)q, (const IT *)k, (const IT *)v, beta, g,
-                                               o, s0, s_final, L, dv, chunk, scale);
+                                               o, s0, s_final, cu, H, L, dv, chunk, scale, err);
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
 }  // namespace
 
 gdn_status_t launch_simt_fwd(const void *q, const void *k, const void *v, const float *beta,
-                             const float *g, float *o, const float *s0, float *s_final, int B,
-                             int H, int L, int dk, int dv, int chunk, float scale,
-                             gdn_dtype_t in_dtype, cudaStream_t stream) {
+                             const float *g, float *o, const float *s0, float *s_final,
+                             const int *cu, int B, int H, int L, int dk, int dv, int chunk,
+                             float scale, gdn_dtype_t in_dtype, cudaStream_t stream) {
     const int BH = B * H;
     const bool delta = beta != nullptr;
+    unsigned *err = nullptr;
+    if (cu && !(err = device_error_word())) return GDN_ERR_CUDA;
 #define GDN_SIMT_CASE(DKV, IT)                                                                     \
-    return delta ? launch_simt_t<DKV, IT, true>(q, k, v, beta, g, o, s0, s_final, BH, L, dv, chunk, \
-                                                scale, stream)                                     \
-                 : launch_simt_t<DKV, IT, false>(q, k, v, beta, g, o, s0, s_final, BH, L, dv,     \
-                                                 chunk, scale, stream)
+    return delta ? launch_simt_t<DKV, IT, true>(q, k, v, beta, g, o, s0, s_final, cu, BH, H, L, dv, \
+                                                chunk, scale, err, stream)                         \
+                 : launch_simt_t<DKV, IT, false>(q, k, v, beta, g, o, s0, s_final, cu, BH, H, L,  \
+                                                 dv, chunk, scale, err, stream)
     if (in_dtype == GDN_F32) {
         if (dk == 64) { GDN_SIMT_CASE(64, float); }
         GDN_SIMT_CASE(128, float);

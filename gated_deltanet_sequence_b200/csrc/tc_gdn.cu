@@ -267,8 +267,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ beta,
               const float *__restrict__ g, float *__restrict__ o, const float *__restrict__ s0,
-              float *__restrict__ s_final, int L, float scale, long long wait_limit,
-              unsigned *__restrict__ err_word) {
+              float *__restrict__ s_final, const int *__restrict__ cu, int H, int Lrow, float scale,
+              long long wait_limit, unsigned *__restrict__ err_word) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned base derived by pointer arithmetic on the shared array, so the
     // compiler keeps every access below in the shared address space (LDS/STS)
@@ -281,9 +281,12 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const Ctl ctl{bars, abort_flag, err_word, wait_limit};
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int bh = blockIdx.x;
+    const int bh = blockIdx.x;                          // (sequence, head): state index
+    const SeqSpan sp = seq_span(cu, bh, H, Lrow, err_word);
+    const int L = sp.len;                               // tokens of this sequence
+    const int zc = sp.head_row, ty0 = sp.t0;            // TMA head and first-token coordinates
     const int nchunks = (L + kC - 1) / kC;
-    const size_t row0 = static_cast<size_t>(bh) * L;   // first token row of this head
+    const size_t row0 = static_cast<size_t>(zc) * Lrow + ty0;   // first token row in the grid
 
     if (tid == 0) {
         for (int b = 0; b < kNumBars; ++b) mbar_init(&bars[b], 1);
@@ -312,12 +315,12 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 uint8_t *st = smem + s * kStageBytes;
                 uint64_t *fb = &bars[B_FULL + s];
                 mbar_arrive_expect_tx(fb, kStageBytes);
-                tma_load_3d(st + ST_K0, &tm_k, fb, 0, c * kC, bh);
-                tma_load_3d(st + ST_Q0, &tm_q, fb, 0, c * kC, bh);
-                tma_load_3d(st + ST_K1, &tm_k, fb, 64, c * kC, bh);
-                tma_load_3d(st + ST_Q1, &tm_q, fb, 64, c * kC, bh);
-                tma_load_3d(st + ST_V0, &tm_v, fb, 0, c * kC, bh);
-                tma_load_3d(st + ST_V1, &tm_v, fb, 64, c * kC, bh);
+                tma_load_3d(st + ST_K0, &tm_k, fb, 0, ty0 + c * kC, zc);
+                tma_load_3d(st + ST_Q0, &tm_q, fb, 0, ty0 + c * kC, zc);
+                tma_load_3d(st + ST_K1, &tm_k, fb, 64, ty0 + c * kC, zc);
+                tma_load_3d(st + ST_Q1, &tm_q, fb, 64, ty0 + c * kC, zc);
+                tma_load_3d(st + ST_V0, &tm_v, fb, 0, ty0 + c * kC, zc);
+                tma_load_3d(st + ST_V1, &tm_v, fb, 64, ty0 + c * kC, zc);
                 last[s] = c;
             }
             // never leave a copy in flight past the end of the CTA
@@ -887,8 +890,8 @@ namespace {
 
 template <bool GATED>
 gdn_status_t launch_gdn_t(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const float *beta,
-                          const float *g, float *o, const float *s0, float *s_final, int BH, int L, float scale,
-                          cudaStream_t stream) {
+                          const float *g, float *o, const float *s0, float *s_final, const int *cu, int nctas,
+                          int H, int L, float scale, cudaStream_t stream) {
     auto kern = tc_gdn_kernel<GATED>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
@@ -898,8 +901,8 @@ gdn_status_t launch_gdn_t(const CUtensorMap &mq, const CUtensorMap &mk, const CU
     if (attr_err != cudaSuccess) return GDN_ERR_CUDA;
     unsigned *err = device_error_word();
     if (!err) return GDN_ERR_CUDA;
-    kern<<<BH, kThreads, kSmemAlloc, stream>>>(mq, mk, mv, beta, g, o, s0, s_final, L, scale, kWaitLimitCycles,
-                                               err);
+    kern<<<nctas, kThreads, kSmemAlloc, stream>>>(mq, mk, mv, beta, g, o, s0, s_final, cu, H, L, scale,
+                                                  kWaitLimitCycles, err);
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
@@ -910,14 +913,15 @@ bool tc_supported(gdn_dtype_t in_dtype, int dk, int dv, int chunk) {
 }
 
 gdn_status_t launch_tc_gdn(const void *q, const void *k, const void *v, const float *beta, const float *g,
-                           float *o, const float *s0, float *s_final, int B, int H, int L, float scale,
-                           cudaStream_t stream) {
-    const int BH = B * H;
+                           float *o, const float *s0, float *s_final, const int *cu, int B, int H, int L,
+                           float scale, cudaStream_t stream) {
+    const int nctas = B * H;                 // one CTA per (sequence, head)
+    const int rows = cu ? H : B * H;         // rows of the (rows, L) token grid
     CUtensorMap mq, mk, mv;
-    if (!make_qkv_map(&mq, q, L, BH) || !make_qkv_map(&mk, k, L, BH) || !make_qkv_map(&mv, v, L, BH))
+    if (!make_qkv_map(&mq, q, L, rows) || !make_qkv_map(&mk, k, L, rows) || !make_qkv_map(&mv, v, L, rows))
         return GDN_ERR_CUDA;
-    return g ? launch_gdn_t<true>(mq, mk, mv, beta, g, o, s0, s_final, BH, L, scale, stream)
-             : launch_gdn_t<false>(mq, mk, mv, beta, g, o, s0, s_final, BH, L, scale, stream);
+    return g ? launch_gdn_t<true>(mq, mk, mv, beta, g, o, s0, s_final, cu, nctas, H, L, scale, stream)
+             : launch_gdn_t<false>(mq, mk, mv, beta, g, o, s0, s_final, cu, nctas, H, L, scale, stream);
 }
 
 }  // namespace gdn

@@ -5,12 +5,14 @@
 namespace gdn {
 // True when the tcgen05 kernels handle this configuration.
 bool tc_supported(gdn_dtype_t in_dtype, int dk, int dv, int chunk);
+// cu (device, nullable): sequence offsets of a packed batch; B is then the number of
+// sequences and L the packed length T of each head row (tokens of head h at rows h*T ..).
 gdn_status_t launch_tc_gdn(const void *q, const void *k, const void *v, const float *beta,
-                           const float *g, float *o, const float *s0, float *s_final, int B, int H,
-                           int L, float scale, cudaStream_t stream);
+                           const float *g, float *o, const float *s0, float *s_final, const int *cu,
+                           int B, int H, int L, float scale, cudaStream_t stream);
 gdn_status_t launch_tc_la(const void *q, const void *k, const void *v, const float *g, float *o,
-                          const float *s0, float *s_final, int B, int H, int L, float scale,
-                          cudaStream_t stream);
+                          const float *s0, float *s_final, const int *cu, int B, int H, int L,
+                          float scale, cudaStream_t stream);
 // Reads and clears the device-side error word of the current device.
 bool read_and_clear_device_error(unsigned *err);
 // Device address of that word on the current device (looked up once per device),

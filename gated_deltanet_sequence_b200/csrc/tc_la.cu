@@ -147,8 +147,8 @@ template <bool GATED>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
              const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ g, float *__restrict__ o,
-             const float *__restrict__ s0, float *__restrict__ s_final, int L, float scale,
-             long long wait_limit, unsigned *__restrict__ err_word) {
+             const float *__restrict__ s0, float *__restrict__ s_final, const int *__restrict__ cu, int H,
+             int Lrow, float scale, long long wait_limit, unsigned *__restrict__ err_word) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned base derived by pointer arithmetic on the shared array, so the
     // compiler keeps every access below in the shared address space (LDS/STS)
@@ -162,9 +162,12 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     const Ctl ctl{bars, abort_flag, err_word, wait_limit};
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int bh = blockIdx.x;
+    const int bh = blockIdx.x;                          // (sequence, head): state index
+    const SeqSpan sp = seq_span(cu, bh, H, Lrow, err_word);
+    const int L = sp.len;                               // tokens of this sequence
+    const int zc = sp.head_row, ty0 = sp.t0;            // TMA head and first-token coordinates
     const int nchunks = (L + kC - 1) / kC;
-    const size_t row0 = static_cast<size_t>(bh) * L;
+    const size_t row0 = static_cast<size_t>(zc) * Lrow + ty0;   // first token row in the grid
 
     if (tid == 0) {
         for (int b = 0; b < kNumBars; ++b) mbar_init(&bars[b], 1);
@@ -203,12 +206,12 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 uint8_t *st = smem + s * kStageBytes;
                 uint64_t *fb = &bars[B_FULL + s];
                 mbar_arrive_expect_tx(fb, kStageBytes);
-                tma_load_3d(st + ST_Q0, &tm_q, fb, 0, c * kC, bh);
-                tma_load_3d(st + ST_K0, &tm_k, fb, 0, c * kC, bh);
-                tma_load_3d(st + ST_Q1, &tm_q, fb, 64, c * kC, bh);
-                tma_load_3d(st + ST_K1, &tm_k, fb, 64, c * kC, bh);
-                tma_load_3d(st + ST_V0, &tm_v, fb, 0, c * kC, bh);
-                tma_load_3d(st + ST_V1, &tm_v, fb, 64, c * kC, bh);
+                tma_load_3d(st + ST_Q0, &tm_q, fb, 0, ty0 + c * kC, zc);
+                tma_load_3d(st + ST_K0, &tm_k, fb, 0, ty0 + c * kC, zc);
+                tma_load_3d(st + ST_Q1, &tm_q, fb, 64, ty0 + c * kC, zc);
+                tma_load_3d(st + ST_K1, &tm_k, fb, 64, ty0 + c * kC, zc);
+                tma_load_3d(st + ST_V0, &tm_v, fb, 0, ty0 + c * kC, zc);
+                tma_load_3d(st + ST_V1, &tm_v, fb, 64, ty0 + c * kC, zc);
                 last[s] = c;
             }
             // never leave a copy in flight past the end of the CTA
@@ -382,7 +385,18 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             if (lead) mbar_arrive(&bars[B_SRDY]);
             done = c;
         }
-        if (s_final && nchunks > 0 && done == nchunks - 1 &&
+        if (s_final && nchunks == 0) {
+            // empty sequence: the final state is the initial one (TMEM holds it)
+            float *dst = s_final + static_cast<size_t>(bh) * kD * kD + v;
+#pragma unroll 1
+            for (int cc = 0; cc < 8; ++cc) {
+                float sv[16];
+                tmem_ld16(trow + TM_S + cc * 16, sv);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 16; ++e) dst[static_cast<size_t>(cc * 16 + e) * kD] = sv[e];
+            }
+        } else if (s_final && nchunks > 0 && done == nchunks - 1 &&
             ctl.group_wait(B_SDONE, (nchunks - 1) & 1, kBarState, abort_s, lead, 128)) {
             tc_fence_after();
             // column v of the final state (a warp writes 32 consecutive floats)
@@ -499,6 +513,7 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             const int s = c % kStages, p = c & 1;
             const float *vec = reinterpret_cast<const float *>(smem + OFF_VEC + p * kVecBytes);
             uint8_t *st = smem + s * kStageBytes;
+            const int nvalid = min(kC, L - c * kC);
             if (!ctl.group_wait(B_FULL + s, (c / kStages) & 1, kBarConv, abort_cv, lead, 128)) break;
             if (GATED && !ctl.group_wait(B_GATE + p, (c >> 1) & 1, kBarConv, abort_cv, lead, 128)) break;
             if (!ctl.group_wait(B_GREAD + s, (c / kStages) & 1, kBarConv, abort_cv, lead, 128)) break;
@@ -517,8 +532,10 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                         off[i] = ST_Q0 + box * 16384u + (idx & 511u) * 16u;
                         f[i] = scale * (GATED ? vec[V_GAM + row] : 1.f);
                     } else {
+                        // rows past the end of the sequence (the next sequence of a packed
+                        // batch, or TMA zero fill) must not reach the state
                         off[i] = ST_K0 + box * 16384u + (idx & 511u) * 16u;
-                        f[i] = GATED ? vec[V_D + row] : 1.f;
+                        f[i] = static_cast<int>(row) < nvalid ? (GATED ? vec[V_D + row] : 1.f) : 0.f;
                     }
                     x[i] = *reinterpret_cast<const uint4 *>(st + off[i]);
                 }
@@ -541,8 +558,8 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 
 template <bool GATED>
 gdn_status_t launch_la_t(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const float *g,
-                         float *o, const float *s0, float *s_final, int BH, int L, float scale,
-                         cudaStream_t stream) {
+                         float *o, const float *s0, float *s_final, const int *cu, int nctas, int H, int L,
+                         float scale, cudaStream_t stream) {
     auto kern = tc_la_kernel<GATED>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
@@ -552,21 +569,23 @@ gdn_status_t launch_la_t(const CUtensorMap &mq, const CUtensorMap &mk, const CUt
     if (attr_err != cudaSuccess) return GDN_ERR_CUDA;
     unsigned *err = device_error_word();
     if (!err) return GDN_ERR_CUDA;
-    kern<<<BH, kThreads, kSmemAlloc, stream>>>(mq, mk, mv, g, o, s0, s_final, L, scale, kWaitLimitCycles, err);
+    kern<<<nctas, kThreads, kSmemAlloc, stream>>>(mq, mk, mv, g, o, s0, s_final, cu, H, L, scale, kWaitLimitCycles,
+                                                  err);
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
 }  // namespace
 
 gdn_status_t launch_tc_la(const void *q, const void *k, const void *v, const float *g, float *o,
-                          const float *s0, float *s_final, int B, int H, int L, float scale,
+                          const float *s0, float *s_final, const int *cu, int B, int H, int L, float scale,
                           cudaStream_t stream) {
-    const int BH = B * H;
+    const int nctas = B * H;                 // one CTA per (sequence, head)
+    const int rows = cu ? H : B * H;         // rows of the (rows, L) token grid
     CUtensorMap mq, mk, mv;
-    if (!make_qkv_map(&mq, q, L, BH) || !make_qkv_map(&mk, k, L, BH) || !make_qkv_map(&mv, v, L, BH))
+    if (!make_qkv_map(&mq, q, L, rows) || !make_qkv_map(&mk, k, L, rows) || !make_qkv_map(&mv, v, L, rows))
         return GDN_ERR_CUDA;
-    return g ? launch_la_t<true>(mq, mk, mv, g, o, s0, s_final, BH, L, scale, stream)
-             : launch_la_t<false>(mq, mk, mv, g, o, s0, s_final, BH, L, scale, stream);
+    return g ? launch_la_t<true>(mq, mk, mv, g, o, s0, s_final, cu, nctas, H, L, scale, stream)
+             : launch_la_t<false>(mq, mk, mv, g, o, s0, s_final, cu, nctas, H, L, scale, stream);
 }
 
 }  // namespace gdn

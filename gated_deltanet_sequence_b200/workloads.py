@@ -96,6 +96,49 @@ def make_prefill_inputs(B: int, H: int, L: int, dk: int, dv: int, *, mode: str =
                 v=v.to(in_dtype).contiguous(), beta=beta, g=g, s0=st)
 
 
+# Packed variable-length Gated DeltaNet prefill: 24 sequences (log-uniform length mix
+# over two decades, each at least 64 tokens) summing to 32768 tokens per head, 16 heads,
+# dk = dv = 128, C = 64.
+VARLEN_WORKLOAD = dict(name="gdn_varlen_bf16_N24_H16_T32768_d128", N=24, H=16, T=32768, min_len=64,
+                       seed=SEED_BASE + 5)
+
+
+def draw_seqlens(N: int, total: int, *, seed: int = SEED_BASE, min_len: int = 1) -> list:
+    """N sequence lengths >= min_len summing to ``total``, with a long-tailed mix
+    (log-uniform weights over two decades), drawn from a seeded CPU generator."""
+    if N * min_len > total:
+        raise ValueError("total is too small for N sequences of min_len")
+    gen = torch.Generator("cpu").manual_seed(int(seed))
+    w = torch.exp(torch.rand(N, generator=gen, dtype=torch.float64) * math.log(100.0))
+    extra = total - N * min_len
+    lens = [min_len + int(x) for x in torch.floor(w / w.sum() * extra).tolist()]
+    lens[int(torch.argmax(w))] += total - sum(lens)
+    return lens
+
+
+def make_varlen_inputs(lens, H: int, dk: int, dv: int, *, mode: str = "gdn",
+                       in_dtype: torch.dtype = torch.bfloat16, s0: bool = False, seed: int = SEED_BASE,
+                       device="cpu", gated: Optional[bool] = None, g_low: float = -0.05,
+                       pad: int = 0) -> dict:
+    """Draw one packed variable-length batch with the distributions of
+    :func:`make_prefill_inputs`: head-major (H, T, d) tensors with T = sum(lens) + pad
+    (``pad`` trailing rows belong to no sequence), cu_seqlens (N + 1,) int32 and
+    s0 (N, H, dk, dv) when asked."""
+    T = int(sum(lens)) + int(pad)
+    d = make_prefill_inputs(1, H, T, dk, dv, mode=mode, in_dtype=in_dtype, s0=False, seed=seed,
+                            device=device, gated=gated, g_low=g_low)
+    out = {name: (None if x is None else x[0].contiguous()) for name, x in d.items() if name != "s0"}
+    cu = [0]
+    for n in lens:
+        cu.append(cu[-1] + int(n))
+    out["cu_seqlens"] = torch.tensor(cu, dtype=torch.int32, device=device)
+    out["s0"] = None
+    if s0:
+        gen = _gen(seed + 7, device)
+        out["s0"] = torch.randn(len(lens), H, dk, dv, dtype=torch.float32, device=device, generator=gen) * 0.1
+    return out
+
+
 def make_decode_inputs(N: int, H: int, dk: int, dv: int, steps: int, *,
                        in_dtype: torch.dtype = torch.bfloat16, seed: int = SEED_BASE + 4,
                        device="cpu", delta: bool = True, gated: bool = True) -> dict:

@@ -89,6 +89,38 @@ gdn_status_t gdn_chunk_fwd(const void *q, const void *k, const void *v, const fl
                            gdn_dtype_t in_dtype, void *cuda_stream);
 
 /*
+ * Packed variable-length batches. N sequences of different lengths share one
+ * head-major token grid: sequence n of head h is rows cu_seqlens[n] ..
+ * cu_seqlens[n+1]-1 of row h of (H, T, d) tensors. Each (sequence, head) is an
+ * independent recurrence with its own initial and final state. The pages serve
+ * prefill and decode batches ("【CS336】lecture4", section "朴素线性注意力": the
+ * prefill/decode split); packing sequences of different lengths is this library's
+ * layout for such a prefill batch, with exactly the per-sequence result of the
+ * dense entry points.
+ *
+ *  q, k        (H, T, dk) in_dtype; v (H, T, dv) in_dtype     device, read
+ *  beta, g     (H, T) fp32 (g nullable)                        device, read
+ *  o           (H, T, dv) fp32                                 device, written at the
+ *              rows of the N sequences (rows outside every sequence are not written)
+ *  s0, s_final (N, H, dk, dv) fp32, nullable as in the dense calls
+ *  cu_seqlens  (N + 1) int32, device, 4-byte aligned: 0 <= cu[0] <= cu[1] <= ... <=
+ *              cu[N] <= T. Sequences may be empty (then s_final = s0 or 0). The
+ *              offsets are read on the device; a list that breaks this rule makes
+ *              the affected (sequence, head) empty and is reported by the next
+ *              gdn_sync_status() as GDN_ERR_INVALID_ARG.
+ *  N, H >= 1; T >= 0; other arguments as for the dense calls.
+ */
+gdn_status_t lin_attn_chunk_fwd_varlen(const void *q, const void *k, const void *v, const float *g,
+                                       float *o, const float *s0, float *s_final,
+                                       const int *cu_seqlens, int N, int H, int T, int dk, int dv,
+                                       int chunk, float scale, gdn_dtype_t in_dtype,
+                                       void *cuda_stream);
+gdn_status_t gdn_chunk_fwd_varlen(const void *q, const void *k, const void *v, const float *beta,
+                                  const float *g, float *o, const float *s0, float *s_final,
+                                  const int *cu_seqlens, int N, int H, int T, int dk, int dv,
+                                  int chunk, float scale, gdn_dtype_t in_dtype, void *cuda_stream);
+
+/*
  * gdn_decode_step — one token for N independent sequences, state updated in place:
  *   u = beta (v - alpha S^T k);  o = alpha S^T q' + (q'.k) u;  S <- alpha S + k u^T
  * with q' = scale q (o equals S_new^T q'). The state is read once and written
@@ -111,9 +143,10 @@ const char *gdn_status_str(gdn_status_t status);
 
 /*
  * gdn_sync_status — synchronise `cuda_stream`, then report (and clear) whether any
- * kernel of this library on the current device gave up on a bounded wait since
- * the last call: GDN_ERR_TIMEOUT in that case, GDN_ERR_CUDA if the stream
- * reported an error, GDN_OK otherwise.
+ * kernel of this library on the current device met a device-side error since the
+ * last call: GDN_ERR_INVALID_ARG for a malformed cu_seqlens list, GDN_ERR_TIMEOUT
+ * for a bounded wait that gave up, GDN_ERR_CUDA if the stream reported an error,
+ * GDN_OK otherwise.
  */
 gdn_status_t gdn_sync_status(void *cuda_stream);
 

@@ -122,6 +122,35 @@ def recurrent_fwd(q, k, v, beta=None, g=None, s0=None, scale: float = 1.0,
     return o, sf
 
 
+def recurrent_fwd_varlen(q, k, v, cu_seqlens, beta=None, g=None, s0=None, scale: float = 1.0,
+                         nthreads: Optional[int] = None, lib=None):
+    """Packed variable-length batch: every sequence is its own recurrence.
+
+    q, k: (H, T, dk); v: (H, T, dv); beta, g: (H, T) or None; cu_seqlens: N + 1 offsets
+    (sequence n of every head is tokens cu[n] .. cu[n+1]-1); s0: (N, H, dk, dv) or None.
+    Each sequence runs through :func:`recurrent_fwd` from its own initial state. Returns
+    (o (H, T, dv) with zeros at rows outside every sequence, S_final (N, H, dk, dv)).
+    """
+    q, k, v, beta, g, s0 = map(_f64, (q, k, v, beta, g, s0))
+    cu = [int(x) for x in np.asarray(cu_seqlens).reshape(-1)]
+    H, T, dk = q.shape
+    dv = v.shape[-1]
+    N = len(cu) - 1
+    o = np.zeros((H, T, dv), np.float64)
+    sf = np.zeros((N, H, dk, dv), np.float64)
+    for n in range(N):
+        a, b = cu[n], cu[n + 1]
+        if not (0 <= a <= b <= T):
+            raise ValueError(f"cu_seqlens[{n}:{n + 2}] = {a}, {b} is not a range inside [0, {T}]")
+        sl = slice(a, b)
+        on, sfn = recurrent_fwd(q[:, sl], k[:, sl], v[:, sl],
+                                None if beta is None else beta[:, sl], None if g is None else g[:, sl],
+                                None if s0 is None else s0[n], scale, nthreads, lib)
+        o[:, sl] = on
+        sf[n] = sfn
+    return o, sf
+
+
 def decode_step(q, k, v, beta, g, state: np.ndarray, scale: float = 1.0,
                 nthreads: Optional[int] = None, lib=None):
     """One decode token for every head; ``state`` (fp64, (..., dk, dv)) is updated in place.

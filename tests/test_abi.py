@@ -26,8 +26,8 @@ def _declared_functions():
 
 def test_header_declares_the_boundary():
     names = _declared_functions()
-    for want in ("lin_attn_chunk_fwd", "gdn_chunk_fwd", "gdn_decode_step", "gdn_status_str",
-                 "gdn_sync_status", "gdn_version"):
+    for want in ("lin_attn_chunk_fwd", "gdn_chunk_fwd", "lin_attn_chunk_fwd_varlen", "gdn_chunk_fwd_varlen",
+                 "gdn_decode_step", "gdn_status_str", "gdn_sync_status", "gdn_version"):
         assert want in names
 
 
@@ -95,3 +95,41 @@ def test_binding_raises_on_bad_shapes(lib):
     q = torch.zeros(1, 1, 4, 64)
     with pytest.raises(ValueError):
         lib.gdn_chunk_fwd(q, q, torch.zeros(1, 1, 5, 64), torch.zeros(1, 1, 4))
+
+
+def _varlen(lib, fn, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, beta=FAKE, g=None, o=FAKE, s0=None, s_final=None, cu=FAKE,
+             N=2, H=1, T=8, dk=64, dv=64, chunk=64, scale=1.0, dt=1)
+    a.update(kw)
+    P = ctypes.c_void_p
+    if fn == "gdn":
+        return lib.lib.gdn_chunk_fwd_varlen(P(a["q"]), P(a["k"]), P(a["v"]), P(a["beta"]), P(a["g"]),
+                                            P(a["o"]), P(a["s0"]), P(a["s_final"]), P(a["cu"]), a["N"],
+                                            a["H"], a["T"], a["dk"], a["dv"], a["chunk"], a["scale"],
+                                            a["dt"], None)
+    return lib.lib.lin_attn_chunk_fwd_varlen(P(a["q"]), P(a["k"]), P(a["v"]), P(a["g"]), P(a["o"]),
+                                             P(a["s0"]), P(a["s_final"]), P(a["cu"]), a["N"], a["H"],
+                                             a["T"], a["dk"], a["dv"], a["chunk"], a["scale"], a["dt"], None)
+
+
+@pytest.mark.parametrize("fn", ["gdn", "la"])
+@pytest.mark.parametrize("kw,want", [
+    (dict(N=0), 1), (dict(cu=None), 1), (dict(cu=FAKE + 2), 1), (dict(H=0), 1), (dict(T=-1), 1),
+    (dict(q=None), 1), (dict(o=FAKE + 8), 1), (dict(dt=5), 1), (dict(dk=96), 2), (dict(chunk=65), 2),
+])
+def test_varlen_rejects_bad_arguments(lib, fn, kw, want):
+    assert _varlen(lib, fn, **kw) == want
+
+
+def test_varlen_gdn_requires_beta(lib):
+    assert _varlen(lib, "gdn", beta=None) == 1
+
+
+def test_varlen_binding_checks_shapes(lib):
+    import torch
+    q = torch.zeros(2, 8, 64)
+    cu = torch.tensor([0, 3, 8], dtype=torch.int32)
+    with pytest.raises(ValueError):
+        lib.gdn_chunk_fwd_varlen(q, q, torch.zeros(2, 9, 64), torch.zeros(2, 8), cu)
+    with pytest.raises(TypeError):
+        lib.lin_attn_chunk_fwd_varlen(q, q, q, cu.long())

@@ -249,3 +249,17 @@ def test_nan_free_with_strong_decay(lib):
     o_ref, s_ref = oracle.recurrent_fwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["g"], inp["s0"])
     check(o, o_ref, 2e-3, "o strong decay")
     check(sf, s_ref, 2e-3, "S strong decay")
+
+
+@pytest.mark.parametrize("mode", ["gdn", "delta"])
+def test_cluster_and_one_cta_forms_give_the_same_bits(lib, mode):
+    # few heads take the cluster form (one chain CTA + two prep CTAs per head); 64 heads
+    # take the one-CTA form. The same two heads, alone and inside the 64-head batch.
+    small = _inputs(1, 2, 333, 128, 128, mode, torch.bfloat16, True, seed=4242)
+    big = _inputs(1, 64, 333, 128, 128, mode, torch.bfloat16, True, seed=4243)
+    for name in ("q", "k", "v", "beta", "g", "s0"):
+        if small[name] is not None:
+            big[name][:, :2] = small[name]
+    o1, s1 = gpu_prefill(lib, small)
+    o2, s2 = gpu_prefill(lib, big)
+    assert torch.equal(o1, o2[:, :2]) and torch.equal(s1, s2[:, :2])

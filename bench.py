@@ -271,7 +271,7 @@ def measure_rows(gdn, peaks, peak_src, args):
     ms = timed(fn, max(3, args.steps // 4), 2)
     nb = prefill_bytes(w.B, w.H, w.L, w.dk, w.dv, 2, True, True, True, True)
     fl = flops_per_head_token("gdn", w.dk, w.dv, w.chunk) * w.B * w.H * w.L
-    rows["gdn_prefill_long"] = _row(w, ms, nb, fl, peaks, peak_src, "hbm", w.B * w.L)
+    rows["gdn_prefill_long"] = _row(w, ms, nb, fl, peaks, peak_src, "hbm", w.B * w.L, "gdn_prefill_cluster")
     del inp, o, sf
     torch.cuda.empty_cache()
     # packed variable-length Gated DeltaNet: 24 sequences (log-uniform length mix), 16 heads
@@ -392,7 +392,8 @@ def run_reference(args, rank, world):
 def run_profile(spec: str):
     """Run one kernel a few times on one case (for an ncu capture; prints nothing timed).
     spec: gdn[:B] (GDN bf16, B x 16 x 4096 x 128), la[:B] (plain LA, B x 16 x 4096 x 128),
-    decode[:N] (N x 32 heads, 3 steps), gdn_long (1 x 32 x 65536)."""
+    decode[:N] (N x 32 heads, 3 steps), gdn_long (1 x 32 x 65536), gdnh[:H[:L]] (1 x H x L,
+    the cluster form when 3 H fits the SM count)."""
     from gated_deltanet_sequence_b200 import _lib as gdn
     kind, _, arg = spec.partition(":")
     torch.cuda.set_device(0)
@@ -408,6 +409,16 @@ def run_profile(spec: str):
                 gdn.gdn_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["g"], o=o, s_final=sf)
             else:
                 gdn.lin_attn_chunk_fwd(inp["q"], inp["k"], inp["v"], None, o=o, s_final=sf)
+    elif kind == "gdnh":
+        # B=1, H heads of L tokens (few heads: the cluster form), S0 != 0
+        H, _, L = arg.partition(":")
+        H, L = int(H or 32), int(L or 8192)
+        inp = W.make_prefill_inputs(1, H, L, 128, 128, mode="gdn", in_dtype=torch.bfloat16, s0=True,
+                                    seed=W.SEED_BASE + 3, device="cuda")
+        o = torch.empty(1, H, L, 128, device="cuda")
+        sf = torch.empty(1, H, 128, 128, device="cuda")
+        for _ in range(2):
+            gdn.gdn_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["g"], o=o, s0=inp["s0"], s_final=sf)
     elif kind == "gdn_long":
         w = W.WORKLOADS[3]
         inp = W.make_workload_inputs(w, device="cuda")

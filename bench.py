@@ -162,13 +162,42 @@ def traffic_from_profiles(kernel_key: str):
 
 
 # ------------------------------------------------------------------------- our arm
+# ------------------------------------------------------------------------- ranks
+def rank_seed(rank: int) -> int:
+    """Seed of this rank's own batch of the headline workload: ranks process independent
+    batches (weak scaling), so no data-path collective is needed."""
+    return W.SEED_BASE + 2 + 1000 * rank
+
+
+def rank_collectives(world: int, device=None):
+    """(barrier, max_over_ranks) over the default process group; (None, identity) for one
+    rank. ``device`` holds the reduction tensor: the GPU for NCCL, None (CPU) for gloo."""
+    if world <= 1:
+        return None, (lambda x: x)
+    import torch.distributed as dist
+
+    def barrier():
+        dist.barrier()
+
+    def max_over_ranks(x):
+        t = torch.tensor([float(x)], device=device if device is not None else "cpu")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+    return barrier, max_over_ranks
+
+
+def aggregate_tokens_per_s(tokens_per_rank: int, world: int, ms_max: float) -> float:
+    """Whole-job throughput: every rank's tokens over the slowest rank's time."""
+    return world * tokens_per_rank / (ms_max * 1e-3)
+
+
 def run_ours(args, rank, world, barrier, max_over_ranks):
     from gated_deltanet_sequence_b200 import _lib as gdn
     peaks, peak_src = load_peaks()
     w = W.WORKLOADS[2]
     B, H, L, dk, dv, C = w.B, w.H, w.L, w.dk, w.dv, w.chunk
     inp = W.make_prefill_inputs(B, H, L, dk, dv, mode="gdn", in_dtype=torch.bfloat16,
-                                seed=W.SEED_BASE + 2 + 1000 * rank, device="cuda")
+                                seed=rank_seed(rank), device="cuda")
     q, k, v, beta, g = inp["q"], inp["k"], inp["v"], inp["beta"], inp["g"]
     o = torch.empty(B, H, L, dv, device="cuda")
     sf = torch.empty(B, H, dk, dv, device="cuda")
@@ -186,7 +215,7 @@ def run_ours(args, rank, world, barrier, max_over_ranks):
         ms = timed(step, args.steps, 0, barrier)
     ms_max = max_over_ranks(ms)
     tokens = B * L
-    value = world * tokens / (ms_max * 1e-3)
+    value = aggregate_tokens_per_s(tokens, world, ms_max)
     flop = flops_per_head_token("gdn", dk, dv, C) * B * H * L
     nbytes = prefill_bytes(B, H, L, dk, dv, 2, True, True, False, True)
     gbs = nbytes / (ms * 1e-3) / 1e9
@@ -220,7 +249,7 @@ def run_ours(args, rank, world, barrier, max_over_ranks):
         ms_e = max_over_ranks(timed(e2e_step, e_steps, 2, barrier))
         h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hb, hg))
         d2h = ho.numel() * 4 + hs.numel() * 4
-        e2e = {"value": round(world * tokens / (ms_e * 1e-3), 1), "unit": "tokens/s",
+        e2e = {"value": round(aggregate_tokens_per_s(tokens, world, ms_e), 1), "unit": "tokens/s",
                "ms_per_step": round(ms_e, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
         del hq, hk, hv, hb, hg, ho, hs, dq, dk_, dv_, db, dg
 
@@ -470,7 +499,6 @@ def main():
         return
 
     torch.cuda.set_device(local)
-    barrier, max_over_ranks = None, (lambda x: x)
     pg = False
     if world > 1:
         import datetime
@@ -478,14 +506,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
         pg = True
-
-        def barrier():
-            dist.barrier()
-
-        def max_over_ranks(x):
-            t = torch.tensor([float(x)], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            return float(t.item())
+    barrier, max_over_ranks = rank_collectives(world, torch.device("cuda", local))
     try:
         line = run_ours(args, rank, world, barrier, max_over_ranks)
         if rank == 0:

@@ -263,3 +263,18 @@ def test_cluster_and_one_cta_forms_give_the_same_bits(lib, mode):
     o1, s1 = gpu_prefill(lib, small)
     o2, s2 = gpu_prefill(lib, big)
     assert torch.equal(o1, o2[:, :2]) and torch.equal(s1, s2[:, :2])
+
+
+@pytest.mark.parametrize("mode", ["gdn", "delta", "gated", "plain"])
+@pytest.mark.parametrize("L", [1, 65, 130, 300])
+def test_one_cta_form_small_lengths(lib, mode, L):
+    # 64 heads take the one-CTA form (the cluster form takes batches whose clusters all fit
+    # on the device at once); ragged and one-token lengths, checked on sampled heads
+    inp = _inputs(1, 64, L, 128, 128, mode, torch.bfloat16, True, seed=5150 + L)
+    o, sf = gpu_prefill(lib, inp)
+    heads = [0, 17, 63]
+    sl = lambda x: None if x is None else x[:, heads]
+    ro, rs = oracle.recurrent_fwd(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]), sl(inp["beta"]), sl(inp["g"]),
+                                  sl(inp["s0"]))
+    check(o[:, heads].numpy(), ro, TOL[torch.bfloat16], f"o {mode} L={L}")
+    check(sf[:, heads].numpy(), rs, TOL[torch.bfloat16], f"S {mode} L={L}")

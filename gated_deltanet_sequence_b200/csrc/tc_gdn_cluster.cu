@@ -250,6 +250,19 @@ tc_gdn_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         mma_f16(tmem + TM_S, sdesc_sw128(stg + ST_K0 + kk * 2048, 16384, 1024),
                                 sdesc_sw128(sb + C_UB + kk * 32, 16, 1024), ID_ST, 1u);
                     mma_commit(&bars[B_SDONE]);
+                    last_bar = B_SDONE;
+                    last_par = c & 1;
+                    // W/U of the next chunk ahead of this chunk's output product, so it runs
+                    // while the next fp16 state is formed (Ut^T was read by the Ut epilogue,
+                    // W^T by the W epilogue)
+                    if (c + 1 < nchunks) {
+                        if (!ready(c + 1)) break;
+                        if (!ctl.wait(B_XFREE, c & 1)) break;
+                        wu(c + 1);
+                        last_bar = B_WU;
+                        last_par = (c + 1) & 1;
+                    }
+                    tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         mma_f16(tmem + TM_O + s * 64, sdesc_sw128(sb + C_UB + kk * 32, 16, 1024),
@@ -257,14 +270,6 @@ tc_gdn_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     mma_commit(&bars[B_CDONE + s]);
                     last_bar = B_CDONE + s;
                     last_par = (c >> 1) & 1;
-                    if (c + 1 < nchunks) {
-                        // W/U of the next chunk: its T factors, and W^T of this chunk read
-                        if (!ready(c + 1)) break;
-                        if (!ctl.wait(B_XFREE, c & 1)) break;
-                        wu(c + 1);
-                        last_bar = B_WU;
-                        last_par = (c + 1) & 1;
-                    }
                 }
                 // UMMAs complete in issue order: the last commit covers everything issued
                 if (last_bar >= 0) ctl.drain(last_bar, last_par);

@@ -194,7 +194,7 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             int last[2] = {-1, -1};   // last chunk loaded into each stage
             for (int c = 0; c < nchunks; ++c) {
                 const int s = c & 1;
-                if (c >= 2 && !ctl.wait(B_CDONE + s, ((c - 2) >> 1) & 1)) break;
+                if (c >= 2 && !ctl.wait_lazy(B_CDONE + s, ((c - 2) >> 1) & 1)) break;
                 uint8_t *st = smem + s * kStageBytes;
                 uint64_t *fb = &bars[B_FULL + s];
                 mbar_arrive_expect_tx(fb, kStageBytes);
@@ -219,8 +219,8 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             for (int c = 0; c < nchunks; ++c) {
                 const int s = c & 1;
                 const uint32_t stg = sb + s * kStageBytes;
-                if (!ctl.wait(B_FULL + s, (c >> 1) & 1)) break;
-                if (c >= 1 && !ctl.wait(B_GFREE, (c - 1) & 1)) break;
+                if (!ctl.wait_lazy(B_FULL + s, (c >> 1) & 1)) break;
+                if (c >= 1 && !ctl.wait_lazy(B_GFREE, (c - 1) & 1)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
@@ -330,8 +330,10 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             const float *vec = reinterpret_cast<const float *>(smem + OFF_VEC + s * kVecBytes);
             uint8_t *st = smem + s * kStageBytes;
             // S(c) complete, and this chunk's gate values
-            if (c >= 1 && !ctl.group_wait(B_CDONE + ((c - 1) & 1), ((c - 1) >> 1) & 1, kBarS, abort_s, lead)) break;
-            if (!ctl.group_wait(B_GATE + s, (c >> 1) & 1, kBarS, abort_s, lead)) break;
+            if (!ctl.group_wait_all({c >= 1 ? B_CDONE + ((c - 1) & 1) : -1, B_GATE + s},
+                                    {static_cast<uint32_t>((c - 1) >> 1) & 1u, static_cast<uint32_t>(c >> 1) & 1u},
+                                    kBarS, abort_s, lead))
+                break;
             tc_fence_after();
             // ---- S row j -> fp16 MN-major operand; S <- gamma_last S (ahead of the update)
             {
@@ -441,10 +443,11 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             uint8_t *st = smem + s * kStageBytes;
             // PG of parity s is free once chunk c-2 is complete; then this chunk's gate
             // values, its tiles and its Gram
-            if (c >= 2 && !ctl.group_wait(B_CDONE + s, ((c - 2) >> 1) & 1, kBarP, abort_p, p == 0, kNP)) break;
-            if (!ctl.group_wait(B_GATEP + s, (c >> 1) & 1, kBarP, abort_p, p == 0, kNP)) break;
-            if (!ctl.group_wait(B_FULL + s, (c >> 1) & 1, kBarP, abort_p, p == 0, kNP)) break;
-            if (!ctl.group_wait(B_GRAM, c & 1, kBarP, abort_p, p == 0, kNP)) break;
+            if (!ctl.group_wait_all({c >= 2 ? B_CDONE + s : -1, B_GATEP + s, B_FULL + s, B_GRAM},
+                                    {static_cast<uint32_t>((c - 2) >> 1) & 1u, static_cast<uint32_t>(c >> 1) & 1u,
+                                     static_cast<uint32_t>(c >> 1) & 1u, static_cast<uint32_t>(c) & 1u},
+                                    kBarP, abort_p, p == 0, kNP))
+                break;
             tc_fence_after();
             const bool fast = !GATED || reinterpret_cast<const int *>(vec)[V_FAST] != 0;
             // ---- Gram rows (lane quarter `sub`, columns 32 hh .. 32 hh + 31):
@@ -689,7 +692,7 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             // vec of parity s is free once chunk c-2 is complete
             if (c >= 2) {
                 int w = 1;
-                if (lane == 0) w = ctl.wait(B_CDONE + s, ((c - 2) >> 1) & 1) ? 1 : 0;
+                if (lane == 0) w = ctl.wait_lazy(B_CDONE + s, ((c - 2) >> 1) & 1) ? 1 : 0;
                 ok = __shfl_sync(0xffffffffu, w, 0) != 0;
                 if (!ok) break;
             }

@@ -43,6 +43,36 @@ struct Ctl {
         named_bar(bar_id, nthreads);
         return *reinterpret_cast<volatile int *>(group_abort) == 0;
     }
+    // Bounded wait that sleeps between polls, for roles off the critical path (their
+    // polling would otherwise take issue slots from the warps they share a scheduler with).
+    __device__ __forceinline__ bool wait_lazy(int b, uint32_t parity) const {
+        if (*reinterpret_cast<volatile int *>(abort_flag)) return false;
+        const uint32_t a = smem_u32(&bar[b]);
+        if (mbar_try_wait(a, parity)) return true;
+        const long long t0 = clock64();
+        do {
+            __nanosleep(100);
+            if (mbar_try_wait(a, parity)) return true;
+        } while (clock64() - t0 <= limit);
+        atomicOr(err, kErrWaitTimeout);
+        *reinterpret_cast<volatile int *>(abort_flag) = 1;
+        return false;
+    }
+    // Group-uniform wait on several phases with one barrier: the leader polls each in
+    // turn (entries with b < 0 are skipped), then the group meets once.
+    template <int N>
+    __device__ __forceinline__ bool group_wait_all(const int (&b)[N], const uint32_t (&parity)[N], int bar_id,
+                                                   int *group_abort, bool leader, int nthreads = 128) const {
+        if (leader) {
+            bool ok = true;
+#pragma unroll
+            for (int i = 0; i < N; ++i)
+                if (ok && b[i] >= 0) ok = wait(b[i], parity[i]);
+            if (!ok) *reinterpret_cast<volatile int *>(group_abort) = 1;
+        }
+        named_bar(bar_id, nthreads);
+        return *reinterpret_cast<volatile int *>(group_abort) == 0;
+    }
     // bounded wait that ignores the abort flag (final drain of in-flight operations)
     __device__ __forceinline__ void drain(int b, uint32_t parity) const { mbar_wait(&bar[b], parity, limit); }
     // Group-uniform wait for a group of warps: the leader polls, the group meets on

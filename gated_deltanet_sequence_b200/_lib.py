@@ -22,7 +22,13 @@ GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_TIMEOUT 
 GDN_F32, GDN_BF16 = 0, 1
 
 EXPORTS = ("lin_attn_chunk_fwd", "gdn_chunk_fwd", "lin_attn_chunk_fwd_varlen", "gdn_chunk_fwd_varlen",
-           "gdn_decode_step", "gdn_status_str", "gdn_sync_status", "gdn_version")
+           "lin_attn_chunk_fwd_ex", "gdn_chunk_fwd_ex", "gdn_decode_step", "gdn_status_str",
+           "gdn_sync_status", "gdn_version")
+
+
+class OutOpts(ctypes.Structure):
+    """gdn_out_opts_t: dtype of o and the D-skip weights (H, dv) (device pointer or None)."""
+    _fields_ = [("out_dtype", ctypes.c_int), ("d_skip", ctypes.c_void_p)]
 
 
 class GdnError(RuntimeError):
@@ -41,13 +47,16 @@ def _load() -> ctypes.CDLL:
     lib.gdn_chunk_fwd.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
     lib.lin_attn_chunk_fwd_varlen.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
     lib.gdn_chunk_fwd_varlen.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
+    lib.lin_attn_chunk_fwd_ex.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P, P]
+    lib.gdn_chunk_fwd_ex.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P, P]
     lib.gdn_decode_step.argtypes = [P, P, P, P, P, P, P, I, I, I, I, F, I, P]
     lib.gdn_status_str.argtypes = [I]
     lib.gdn_status_str.restype = ctypes.c_char_p
     lib.gdn_sync_status.argtypes = [P]
     lib.gdn_version.argtypes = []
     for f in (lib.lin_attn_chunk_fwd, lib.gdn_chunk_fwd, lib.lin_attn_chunk_fwd_varlen,
-              lib.gdn_chunk_fwd_varlen, lib.gdn_decode_step, lib.gdn_sync_status, lib.gdn_version):
+              lib.gdn_chunk_fwd_varlen, lib.lin_attn_chunk_fwd_ex, lib.gdn_chunk_fwd_ex,
+              lib.gdn_decode_step, lib.gdn_sync_status, lib.gdn_version):
         f.restype = ctypes.c_int
     return lib
 
@@ -99,9 +108,25 @@ def _raise(fn: str, st: int):
         raise GdnError(fn, st)
 
 
+def _out_opts(o, out_dtype, d_skip, H, dv, dev):
+    """Output dtype (from ``o`` when given, else ``out_dtype``, default fp32) and the
+    checked D-skip weights; returns (dtype, OutOpts or None when both are defaults)."""
+    dt = o.dtype if o is not None else (out_dtype or torch.float32)
+    if dt not in (torch.float32, torch.bfloat16):
+        raise TypeError(f"o / out_dtype must be float32 or bfloat16, got {dt}")
+    _check("d_skip", d_skip, (H, dv), torch.float32, dev, required=False)
+    if dt == torch.float32 and d_skip is None:
+        return dt, None
+    return dt, OutOpts(GDN_BF16 if dt == torch.bfloat16 else GDN_F32,
+                       None if d_skip is None else d_skip.data_ptr())
+
+
 def lin_attn_chunk_fwd(q, k, v, g=None, o=None, s0=None, s_final=None, chunk: int = 64,
-                       scale: float = 1.0, stream=None):
-    """Plain (g None) or gated causal linear attention. Returns (o, s_final)."""
+                       scale: float = 1.0, stream=None, out_dtype=None, d_skip=None):
+    """Plain (g None) or gated causal linear attention. Returns (o, s_final).
+
+    out_dtype (torch.float32 / torch.bfloat16) sets the dtype of a new ``o``; d_skip (H, dv)
+    fp32 adds the skip term o_t += d_skip[h] * v_t."""
     B, H, L, dk = q.shape
     dv = v.shape[-1]
     dev = q.device
@@ -110,20 +135,28 @@ def lin_attn_chunk_fwd(q, k, v, g=None, o=None, s0=None, s_final=None, chunk: in
     _check("v", v, (B, H, L, dv), q.dtype, dev)
     _check("g", g, (B, H, L), torch.float32, dev, required=False)
     _check("s0", s0, (B, H, dk, dv), torch.float32, dev, required=False)
+    odt, opts = _out_opts(o, out_dtype, d_skip, H, dv, dev)
     if o is None:
-        o = torch.empty(B, H, L, dv, dtype=torch.float32, device=dev)
-    _check("o", o, (B, H, L, dv), torch.float32, dev)
+        o = torch.empty(B, H, L, dv, dtype=odt, device=dev)
+    _check("o", o, (B, H, L, dv), odt, dev)
     _check("s_final", s_final, (B, H, dk, dv), torch.float32, dev, required=False)
-    st = lib.lin_attn_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(o), _ptr(s0),
-                                _ptr(s_final), B, H, L, dk, dv, int(chunk), float(scale),
-                                _dtype_code(q), _stream(stream))
-    _raise("lin_attn_chunk_fwd", st)
+    if opts is None:
+        st = lib.lin_attn_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(o), _ptr(s0),
+                                    _ptr(s_final), B, H, L, dk, dv, int(chunk), float(scale),
+                                    _dtype_code(q), _stream(stream))
+        _raise("lin_attn_chunk_fwd", st)
+    else:
+        st = lib.lin_attn_chunk_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(o), _ptr(s0),
+                                       _ptr(s_final), None, B, H, L, dk, dv, int(chunk), float(scale),
+                                       _dtype_code(q), ctypes.byref(opts), _stream(stream))
+        _raise("lin_attn_chunk_fwd_ex", st)
     return o, s_final
 
 
 def gdn_chunk_fwd(q, k, v, beta, g=None, o=None, s0=None, s_final=None, chunk: int = 64,
-                  scale: float = 1.0, stream=None):
-    """DeltaNet (g None) or Gated DeltaNet chunkwise prefill. Returns (o, s_final)."""
+                  scale: float = 1.0, stream=None, out_dtype=None, d_skip=None):
+    """DeltaNet (g None) or Gated DeltaNet chunkwise prefill. Returns (o, s_final).
+    out_dtype and d_skip as for :func:`lin_attn_chunk_fwd`."""
     B, H, L, dk = q.shape
     dv = v.shape[-1]
     dev = q.device
@@ -133,14 +166,21 @@ def gdn_chunk_fwd(q, k, v, beta, g=None, o=None, s0=None, s_final=None, chunk: i
     _check("beta", beta, (B, H, L), torch.float32, dev, required=L > 0)
     _check("g", g, (B, H, L), torch.float32, dev, required=False)
     _check("s0", s0, (B, H, dk, dv), torch.float32, dev, required=False)
+    odt, opts = _out_opts(o, out_dtype, d_skip, H, dv, dev)
     if o is None:
-        o = torch.empty(B, H, L, dv, dtype=torch.float32, device=dev)
-    _check("o", o, (B, H, L, dv), torch.float32, dev)
+        o = torch.empty(B, H, L, dv, dtype=odt, device=dev)
+    _check("o", o, (B, H, L, dv), odt, dev)
     _check("s_final", s_final, (B, H, dk, dv), torch.float32, dev, required=False)
-    st = lib.gdn_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(o), _ptr(s0),
-                           _ptr(s_final), B, H, L, dk, dv, int(chunk), float(scale),
-                           _dtype_code(q), _stream(stream))
-    _raise("gdn_chunk_fwd", st)
+    if opts is None:
+        st = lib.gdn_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(o), _ptr(s0),
+                               _ptr(s_final), B, H, L, dk, dv, int(chunk), float(scale),
+                               _dtype_code(q), _stream(stream))
+        _raise("gdn_chunk_fwd", st)
+    else:
+        st = lib.gdn_chunk_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(o), _ptr(s0),
+                                  _ptr(s_final), None, B, H, L, dk, dv, int(chunk), float(scale),
+                                  _dtype_code(q), ctypes.byref(opts), _stream(stream))
+        _raise("gdn_chunk_fwd_ex", st)
     return o, s_final
 
 
@@ -163,38 +203,54 @@ def _check_varlen(q, k, v, cu_seqlens, s0, s_final):
 
 
 def lin_attn_chunk_fwd_varlen(q, k, v, cu_seqlens, g=None, o=None, s0=None, s_final=None,
-                              chunk: int = 64, scale: float = 1.0, stream=None):
+                              chunk: int = 64, scale: float = 1.0, stream=None, out_dtype=None,
+                              d_skip=None):
     """Packed variable-length batch of plain / gated linear attention.
 
     q, k (H, T, dk); v (H, T, dv); g (H, T) or None; cu_seqlens (N + 1,) int32 on the device
     (sequence n is tokens cu[n] .. cu[n+1]-1 of every head). s0, s_final (N, H, dk, dv).
-    Returns (o, s_final); rows outside every sequence are left as they were in ``o``."""
+    Returns (o, s_final); rows outside every sequence are left as they were in ``o``.
+    out_dtype and d_skip as for :func:`lin_attn_chunk_fwd`."""
     N, H, T, dk, dv, dev = _check_varlen(q, k, v, cu_seqlens, s0, s_final)
     _check("g", g, (H, T), torch.float32, dev, required=False)
+    odt, opts = _out_opts(o, out_dtype, d_skip, H, dv, dev)
     if o is None:
-        o = torch.zeros(H, T, dv, dtype=torch.float32, device=dev)
-    _check("o", o, (H, T, dv), torch.float32, dev)
-    st = lib.lin_attn_chunk_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(o), _ptr(s0),
+        o = torch.zeros(H, T, dv, dtype=odt, device=dev)
+    _check("o", o, (H, T, dv), odt, dev)
+    if opts is None:
+        st = lib.lin_attn_chunk_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(o), _ptr(s0),
+                                           _ptr(s_final), _ptr(cu_seqlens), N, H, T, dk, dv, int(chunk),
+                                           float(scale), _dtype_code(q), _stream(stream))
+        _raise("lin_attn_chunk_fwd_varlen", st)
+    else:
+        st = lib.lin_attn_chunk_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(o), _ptr(s0),
                                        _ptr(s_final), _ptr(cu_seqlens), N, H, T, dk, dv, int(chunk),
-                                       float(scale), _dtype_code(q), _stream(stream))
-    _raise("lin_attn_chunk_fwd_varlen", st)
+                                       float(scale), _dtype_code(q), ctypes.byref(opts), _stream(stream))
+        _raise("lin_attn_chunk_fwd_ex", st)
     return o, s_final
 
 
 def gdn_chunk_fwd_varlen(q, k, v, beta, cu_seqlens, g=None, o=None, s0=None, s_final=None,
-                         chunk: int = 64, scale: float = 1.0, stream=None):
+                         chunk: int = 64, scale: float = 1.0, stream=None, out_dtype=None, d_skip=None):
     """Packed variable-length batch of DeltaNet / Gated DeltaNet (see lin_attn_chunk_fwd_varlen);
     beta (H, T) fp32."""
     N, H, T, dk, dv, dev = _check_varlen(q, k, v, cu_seqlens, s0, s_final)
     _check("beta", beta, (H, T), torch.float32, dev, required=T > 0)
     _check("g", g, (H, T), torch.float32, dev, required=False)
+    odt, opts = _out_opts(o, out_dtype, d_skip, H, dv, dev)
     if o is None:
-        o = torch.zeros(H, T, dv, dtype=torch.float32, device=dev)
-    _check("o", o, (H, T, dv), torch.float32, dev)
-    st = lib.gdn_chunk_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(o), _ptr(s0),
+        o = torch.zeros(H, T, dv, dtype=odt, device=dev)
+    _check("o", o, (H, T, dv), odt, dev)
+    if opts is None:
+        st = lib.gdn_chunk_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(o), _ptr(s0),
+                                      _ptr(s_final), _ptr(cu_seqlens), N, H, T, dk, dv, int(chunk),
+                                      float(scale), _dtype_code(q), _stream(stream))
+        _raise("gdn_chunk_fwd_varlen", st)
+    else:
+        st = lib.gdn_chunk_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(o), _ptr(s0),
                                   _ptr(s_final), _ptr(cu_seqlens), N, H, T, dk, dv, int(chunk),
-                                  float(scale), _dtype_code(q), _stream(stream))
-    _raise("gdn_chunk_fwd_varlen", st)
+                                  float(scale), _dtype_code(q), ctypes.byref(opts), _stream(stream))
+        _raise("gdn_chunk_fwd_ex", st)
     return o, s_final
 
 

@@ -11,6 +11,7 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 bool opt_aligned16(const void *p) { return p == nullptr || aligned16(p); }
 bool opt_aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 bool head_dim_ok(int d) { return d == 64 || d == 128; }
+constexpr gdn::OutOpts kDefaultOut{false, nullptr};   // fp32 o, no D-skip term
 
 gdn_status_t check_prefill(const void *q, const void *k, const void *v, const float *g, float *o,
                            const float *s0, float *s_final, int B, int H, int L, int dk, int dv,
@@ -55,9 +56,9 @@ gdn_status_t lin_attn_chunk_fwd(const void *q, const void *k, const void *v, con
     if (st != GDN_OK) return st;
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
     if (gdn::tc_supported(in_dtype, dk, dv, chunk) && L > 0)
-        return gdn::launch_tc_la(q, k, v, g, o, s0, s_final, nullptr, B, H, L, scale, stream);
+        return gdn::launch_tc_la(q, k, v, g, o, s0, s_final, nullptr, B, H, L, scale, kDefaultOut, stream);
     return gdn::launch_simt_fwd(q, k, v, nullptr, g, o, s0, s_final, nullptr, B, H, L, dk, dv, chunk,
-                                scale, in_dtype, stream);
+                                scale, in_dtype, kDefaultOut, stream);
 }
 
 gdn_status_t gdn_chunk_fwd(const void *q, const void *k, const void *v, const float *beta,
@@ -70,10 +71,10 @@ gdn_status_t gdn_chunk_fwd(const void *q, const void *k, const void *v, const fl
     if (!opt_aligned4(beta)) return GDN_ERR_INVALID_ARG;
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
     if (gdn::tc_supported(in_dtype, dk, dv, chunk) && L > 0)
-        return gdn::launch_tc_gdn(q, k, v, beta, g, o, s0, s_final, nullptr, B, H, L, scale, stream);
+        return gdn::launch_tc_gdn(q, k, v, beta, g, o, s0, s_final, nullptr, B, H, L, scale, kDefaultOut, stream);
     // with L == 0 beta may be NULL: the kernel then only writes s0 (or zeros) to s_final
     return gdn::launch_simt_fwd(q, k, v, beta, g, o, s0, s_final, nullptr, B, H, L, dk, dv, chunk,
-                                scale, in_dtype, stream);
+                                scale, in_dtype, kDefaultOut, stream);
 }
 
 gdn_status_t lin_attn_chunk_fwd_varlen(const void *q, const void *k, const void *v, const float *g,
@@ -87,9 +88,9 @@ gdn_status_t lin_attn_chunk_fwd_varlen(const void *q, const void *k, const void 
     if ((double)N * H > 2147483647.0) return GDN_ERR_INVALID_ARG;
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
     if (gdn::tc_supported(in_dtype, dk, dv, chunk) && T > 0)
-        return gdn::launch_tc_la(q, k, v, g, o, s0, s_final, cu_seqlens, N, H, T, scale, stream);
+        return gdn::launch_tc_la(q, k, v, g, o, s0, s_final, cu_seqlens, N, H, T, scale, kDefaultOut, stream);
     return gdn::launch_simt_fwd(q, k, v, nullptr, g, o, s0, s_final, cu_seqlens, N, H, T, dk, dv, chunk,
-                                scale, in_dtype, stream);
+                                scale, in_dtype, kDefaultOut, stream);
 }
 
 gdn_status_t gdn_chunk_fwd_varlen(const void *q, const void *k, const void *v, const float *beta,
@@ -104,9 +105,54 @@ gdn_status_t gdn_chunk_fwd_varlen(const void *q, const void *k, const void *v, c
     if (!opt_aligned4(beta)) return GDN_ERR_INVALID_ARG;
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
     if (gdn::tc_supported(in_dtype, dk, dv, chunk) && T > 0)
-        return gdn::launch_tc_gdn(q, k, v, beta, g, o, s0, s_final, cu_seqlens, N, H, T, scale, stream);
+        return gdn::launch_tc_gdn(q, k, v, beta, g, o, s0, s_final, cu_seqlens, N, H, T, scale, kDefaultOut, stream);
     return gdn::launch_simt_fwd(q, k, v, beta, g, o, s0, s_final, cu_seqlens, N, H, T, dk, dv, chunk,
-                                scale, in_dtype, stream);
+                                scale, in_dtype, kDefaultOut, stream);
+}
+
+// The general prefill call: dense (cu_seqlens == NULL) or packed batches, with the output
+// options. Validation as for the dense / packed calls, plus the options.
+static gdn_status_t prefill_ex(bool delta, const void *q, const void *k, const void *v, const float *beta,
+                               const float *g, void *o, const float *s0, float *s_final, const int *cu_seqlens,
+                               int B, int H, int L, int dk, int dv, int chunk, float scale, gdn_dtype_t in_dtype,
+                               const gdn_out_opts_t *opts, void *cuda_stream) {
+    gdn::OutOpts oo = kDefaultOut;
+    if (opts) {
+        if (opts->out_dtype != GDN_F32 && opts->out_dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+        if (!opt_aligned4(opts->d_skip)) return GDN_ERR_INVALID_ARG;
+        oo.bf16 = opts->out_dtype == GDN_BF16;
+        oo.dskip = opts->d_skip;
+    }
+    if (B < 1 || !opt_aligned4(cu_seqlens)) return GDN_ERR_INVALID_ARG;
+    const int grid_b = cu_seqlens ? 1 : B;   // batch extent of the token grid
+    gdn_status_t st = check_prefill(q, k, v, g, static_cast<float *>(o), s0, s_final, grid_b, H, L, dk, dv, chunk,
+                                    scale, in_dtype);
+    if (st != GDN_OK) return st;
+    if ((double)B * H > 2147483647.0) return GDN_ERR_INVALID_ARG;
+    if (delta && L > 0 && !beta) return GDN_ERR_INVALID_ARG;
+    if (!opt_aligned4(beta)) return GDN_ERR_INVALID_ARG;
+    cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+    if (gdn::tc_supported(in_dtype, dk, dv, chunk) && L > 0)
+        return delta ? gdn::launch_tc_gdn(q, k, v, beta, g, o, s0, s_final, cu_seqlens, B, H, L, scale, oo, stream)
+                     : gdn::launch_tc_la(q, k, v, g, o, s0, s_final, cu_seqlens, B, H, L, scale, oo, stream);
+    return gdn::launch_simt_fwd(q, k, v, delta ? beta : nullptr, g, o, s0, s_final, cu_seqlens, B, H, L, dk, dv,
+                                chunk, scale, in_dtype, oo, stream);
+}
+
+gdn_status_t lin_attn_chunk_fwd_ex(const void *q, const void *k, const void *v, const float *g, void *o,
+                                   const float *s0, float *s_final, const int *cu_seqlens, int B, int H, int L,
+                                   int dk, int dv, int chunk, float scale, gdn_dtype_t in_dtype,
+                                   const gdn_out_opts_t *opts, void *cuda_stream) {
+    return prefill_ex(false, q, k, v, nullptr, g, o, s0, s_final, cu_seqlens, B, H, L, dk, dv, chunk, scale,
+                      in_dtype, opts, cuda_stream);
+}
+
+gdn_status_t gdn_chunk_fwd_ex(const void *q, const void *k, const void *v, const float *beta, const float *g,
+                              void *o, const float *s0, float *s_final, const int *cu_seqlens, int B, int H, int L,
+                              int dk, int dv, int chunk, float scale, gdn_dtype_t in_dtype,
+                              const gdn_out_opts_t *opts, void *cuda_stream) {
+    return prefill_ex(true, q, k, v, beta, g, o, s0, s_final, cu_seqlens, B, H, L, dk, dv, chunk, scale, in_dtype,
+                      opts, cuda_stream);
 }
 
 gdn_status_t gdn_decode_step(const void *q, const void *k, const void *v, const float *beta,

@@ -58,6 +58,51 @@ __device__ __forceinline__ void st_global4(float *p, float4 v) {
                  "f"(v.w) : "memory");
 }
 
+// Output epilogue options of the prefill kernels: o in fp32 or bf16, and the Mamba
+// D-skip term o_t += D_h (elementwise) v_t, D of shape (H, dv) (page "【CS336】lecture4",
+// section "继续改进：Mamba": a term in v added at the output, like a residual branch).
+struct OutOpts {
+    bool bf16;            // o is bf16 (round to nearest even), else fp32
+    const float *dskip;   // (H, dv) fp32, nullable (no skip term)
+};
+// The same, as a kernel argument: o, and for the D-skip term the input v (bf16 for the
+// tensor-core kernels; same (rows, dv) layout as o) with D.
+struct OutArgs {
+    void *o;
+    const __nv_bfloat16 *v;   // nullptr: no D-skip term
+    const float *dskip;       // (H, dv)
+    int bf16;
+};
+
+// One value column of a 64-token output tile: ov[r] = o[row r][column] for r < n, at
+// element offset elem0 + r * stride of o. Adds dj * v at the same offsets when v is
+// given (the D-skip term, fp32 fused multiply-add), then stores fp32 or bf16.
+__device__ __forceinline__ void store_out_rows(float (&ov)[64], void *o, size_t elem0, int n, int stride,
+                                               bool bf16, float dj, const __nv_bfloat16 *v) {
+#pragma unroll
+    for (int r0 = 0; r0 < 64; r0 += 16) {
+        float x[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) x[r] = ov[r0 + r];
+        if (v) {
+#pragma unroll
+            for (int r = 0; r < 16; ++r)
+                if (r0 + r < n) x[r] = fmaf(dj, __bfloat162float(v[elem0 + static_cast<size_t>(r0 + r) * stride]), x[r]);
+        }
+        if (bf16) {
+            __nv_bfloat16 *ob = static_cast<__nv_bfloat16 *>(o) + elem0;
+#pragma unroll
+            for (int r = 0; r < 16; ++r)
+                if (r0 + r < n) ob[static_cast<size_t>(r0 + r) * stride] = __float2bfloat16_rn(x[r]);
+        } else {
+            float *of = static_cast<float *>(o) + elem0;
+#pragma unroll
+            for (int r = 0; r < 16; ++r)
+                if (r0 + r < n) of[static_cast<size_t>(r0 + r) * stride] = x[r];
+        }
+    }
+}
+
 }  // namespace gdn
 
 // Host-side launchers implemented in the kernel translation units.
@@ -65,9 +110,9 @@ namespace gdn {
 // cu (device, nullable): sequence offsets of a packed batch; B is then the number of
 // sequences and L the packed length T of each head row.
 gdn_status_t launch_simt_fwd(const void *q, const void *k, const void *v, const float *beta,
-                             const float *g, float *o, const float *s0, float *s_final,
+                             const float *g, void *o, const float *s0, float *s_final,
                              const int *cu, int B, int H, int L, int dk, int dv, int chunk,
-                             float scale, gdn_dtype_t in_dtype, cudaStream_t stream);
+                             float scale, gdn_dtype_t in_dtype, OutOpts oo, cudaStream_t stream);
 gdn_status_t launch_decode(const void *q, const void *k, const void *v, const float *beta,
                            const float *g, float *state, float *o, int N, int H, int dk, int dv,
                            float scale, gdn_dtype_t in_dtype, cudaStream_t stream);

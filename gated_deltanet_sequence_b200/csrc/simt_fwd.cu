@@ -44,7 +44,8 @@ template <int DK, typename IT, bool DELTA>
 __global__ void __launch_bounds__(kSimtThreads)
 simt_chunk_fwd_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT *__restrict__ v,
                       const float *__restrict__ beta, const float *__restrict__ g,
-                      float *__restrict__ o, const float *__restrict__ s0,
+                      void *__restrict__ o, int out_bf16, const float *__restrict__ dskip,
+                      const float *__restrict__ s0,
                       float *__restrict__ s_final, const int *__restrict__ cu, int H, int Lrow,
                       int dv, int C, float scale, unsigned *__restrict__ err) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -63,7 +64,8 @@ simt_chunk_fwd_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const 
     const IT *vh = v + r0 * dv;
     const float *bh_beta = DELTA ? beta + r0 : nullptr;
     const float *bh_g = g ? g + r0 : nullptr;
-    float *oh = o + r0 * dv;
+    const long o0 = r0 * dv;                     // first output element of the sequence
+    const float *dsk = dskip ? dskip + static_cast<long>(sp.head_row % H) * dv + c0 : nullptr;
 
     for (int i = tid; i < DK * kDvs; i += kSimtThreads) {
         const int j = i / kDvs, c = i % kDvs;
@@ -164,7 +166,11 @@ simt_chunk_fwd_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const 
             for (int j = 0; j < DK; ++j) qs = fmaf(sm.Q[r * KP + j], sm.S[j * kDvs + c], qs);
             float pu = 0.f;
             for (int s = 0; s <= r; ++s) pu = fmaf(sm.P[r * CP + s], Ut[s * kDvs + c], pu);
-            oh[(long)(t0 + r) * dv + c0 + c] = expf(sm.G[r]) * qs + pu;
+            float ov = expf(sm.G[r]) * qs + pu;
+            if (dsk) ov = fmaf(dsk[c], sm.V[i], ov);     // D-skip term D_h v_t
+            const long oi = o0 + (long)(t0 + r) * dv + c0 + c;
+            if (out_bf16) static_cast<__nv_bfloat16 *>(o)[oi] = __float2bfloat16_rn(ov);
+            else static_cast<float *>(o)[oi] = ov;
         }
         __syncthreads();
         // ---- S <- gamma_n S + sum_s exp(G_n - G_s) k_s Ut_s^T ----------------------
@@ -190,8 +196,8 @@ simt_chunk_fwd_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const 
 
 template <int DK, typename IT, bool DELTA>
 gdn_status_t launch_simt_t(const void *q, const void *k, const void *v, const float *beta,
-                           const float *g, float *o, const float *s0, float *s_final, const int *cu,
-                           int BH, int H, int L, int dv, int chunk, float scale, unsigned *err,
+                           const float *g, void *o, const float *s0, float *s_final, const int *cu,
+                           int BH, int H, int L, int dv, int chunk, float scale, OutOpts oo, unsigned *err,
                            cudaStream_t stream) {
     auto kern = simt_chunk_fwd_kernel<DK, IT, DELTA>;
     const int smem = (int)sizeof(SimtSmem<DK>);
@@ -199,25 +205,26 @@ gdn_status_t launch_simt_t(const void *q, const void *k, const void *v, const fl
         return GDN_ERR_CUDA;
     dim3 grid(BH, dv / kDvs);
     kern<<<grid, kSimtThreads, smem, stream>>>((const IT *)q, (const IT *)k, (const IT *)v, beta, g,
-                                               o, s0, s_final, cu, H, L, dv, chunk, scale, err);
+                                               o, oo.bf16 ? 1 : 0, oo.dskip, s0, s_final, cu, H, L, dv,
+                                               chunk, scale, err);
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
 }  // namespace
 
 gdn_status_t launch_simt_fwd(const void *q, const void *k, const void *v, const float *beta,
-                             const float *g, float *o, const float *s0, float *s_final,
+                             const float *g, void *o, const float *s0, float *s_final,
                              const int *cu, int B, int H, int L, int dk, int dv, int chunk,
-                             float scale, gdn_dtype_t in_dtype, cudaStream_t stream) {
+                             float scale, gdn_dtype_t in_dtype, OutOpts oo, cudaStream_t stream) {
     const int BH = B * H;
     const bool delta = beta != nullptr;
     unsigned *err = nullptr;
     if (cu && !(err = device_error_word())) return GDN_ERR_CUDA;
 #define GDN_SIMT_CASE(DKV, IT)                                                                     \
     return delta ? launch_simt_t<DKV, IT, true>(q, k, v, beta, g, o, s0, s_final, cu, BH, H, L, dv, \
-                                                chunk, scale, err, stream)                         \
+                                                chunk, scale, oo, err, stream)                     \
                  : launch_simt_t<DKV, IT, false>(q, k, v, beta, g, o, s0, s_final, cu, BH, H, L,  \
-                                                 dv, chunk, scale, err, stream)
+                                                 dv, chunk, scale, oo, err, stream)
     if (in_dtype == GDN_F32) {
         if (dk == 64) { GDN_SIMT_CASE(64, float); }
         GDN_SIMT_CASE(128, float);

@@ -145,11 +145,11 @@ enum : int {
     kNumBars = 20
 };
 
-template <bool GATED>
+template <bool GATED, bool OPTS>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ beta,
-              const float *__restrict__ g, float *__restrict__ o, const float *__restrict__ s0,
+              const float *__restrict__ g, const OutArgs out, const float *__restrict__ s0,
               float *__restrict__ s_final, const int *__restrict__ cu, int H, int Lrow, float scale,
               long long wait_limit, unsigned *__restrict__ err_word) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -307,6 +307,8 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         // ================================================================ state group
         const int j = tid - kGroupS * 32;                // = TMEM lane (key row j / value column v)
         const bool lead = (j == 0);
+        // D-skip weight of value column j (head zc mod H: dense and packed grids alike)
+        const float dj = (OPTS && out.v) ? out.dskip[(zc % H) * kD + j] : 0.f;
         const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
         {
             const float *src = s0 ? s0 + (static_cast<size_t>(bh) * kD + j) * kD : nullptr;
@@ -385,7 +387,7 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             // ---- output of the previous chunk (its O tile is complete)
             if (c >= 1) {
                 const int cp = c - 1;
-                store_out_col(trow + TM_O + (cp & 1) * 64, o + (row0 + static_cast<size_t>(cp) * kC) * kD + j, kC);
+                store_out_col<OPTS>(trow + TM_O + (cp & 1) * 64, out, (row0 + static_cast<size_t>(cp) * kC) * kD + j, kC, dj);
                 done = c;
             }
             // ---- Ut^T row v -> Ut operand (K-major, rows v)
@@ -408,8 +410,8 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             const int cp = nchunks - 1;
             if (ctl.group_wait(B_CDONE + (cp & 1), (cp >> 1) & 1, kBarS, abort_s, lead)) {
                 tc_fence_after();
-                store_out_col(trow + TM_O + (cp & 1) * 64, o + (row0 + static_cast<size_t>(cp) * kC) * kD + j,
-                              L - cp * kC);
+                store_out_col<OPTS>(trow + TM_O + (cp & 1) * 64, out, (row0 + static_cast<size_t>(cp) * kC) * kD + j,
+                              L - cp * kC, dj);
                 done = nchunks;
             }
         }
@@ -774,11 +776,11 @@ bool make_qkv_map(CUtensorMap *m, const void *ptr, int L, int BH) {
 
 namespace {
 
-template <bool GATED>
+template <bool GATED, bool OPTS>
 gdn_status_t launch_gdn_t(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const float *beta,
-                          const float *g, float *o, const float *s0, float *s_final, const int *cu, int nctas,
-                          int H, int L, float scale, cudaStream_t stream) {
-    auto kern = tc_gdn_kernel<GATED>;
+                          const float *g, const OutArgs &out, const float *s0, float *s_final, const int *cu,
+                          int nctas, int H, int L, float scale, cudaStream_t stream) {
+    auto kern = tc_gdn_kernel<GATED, OPTS>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [&] {
@@ -787,7 +789,7 @@ gdn_status_t launch_gdn_t(const CUtensorMap &mq, const CUtensorMap &mk, const CU
     if (attr_err != cudaSuccess) return GDN_ERR_CUDA;
     unsigned *err = device_error_word();
     if (!err) return GDN_ERR_CUDA;
-    kern<<<nctas, kThreads, kSmemAlloc, stream>>>(mq, mk, mv, beta, g, o, s0, s_final, cu, H, L, scale,
+    kern<<<nctas, kThreads, kSmemAlloc, stream>>>(mq, mk, mv, beta, g, out, s0, s_final, cu, H, L, scale,
                                                   kWaitLimitCycles, err);
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
@@ -799,18 +801,22 @@ bool tc_supported(gdn_dtype_t in_dtype, int dk, int dv, int chunk) {
 }
 
 gdn_status_t launch_tc_gdn(const void *q, const void *k, const void *v, const float *beta, const float *g,
-                           float *o, const float *s0, float *s_final, const int *cu, int B, int H, int L,
-                           float scale, cudaStream_t stream) {
+                           void *o, const float *s0, float *s_final, const int *cu, int B, int H, int L,
+                           float scale, OutOpts oo, cudaStream_t stream) {
     const int nctas = B * H;                 // one CTA per (sequence, head)
     // few (sequence, head) pairs: the cluster form spreads each chunk's prep over two more SMs
     if (tc_gdn_cluster_fits(nctas))
-        return launch_tc_gdn_cluster(q, k, v, beta, g, o, s0, s_final, cu, B, H, L, scale, stream);
+        return launch_tc_gdn_cluster(q, k, v, beta, g, o, s0, s_final, cu, B, H, L, scale, oo, stream);
+    const OutArgs out{o, oo.dskip ? static_cast<const __nv_bfloat16 *>(v) : nullptr, oo.dskip, oo.bf16 ? 1 : 0};
     const int rows = cu ? H : B * H;         // rows of the (rows, L) token grid
     CUtensorMap mq, mk, mv;
     if (!make_qkv_map(&mq, q, L, rows) || !make_qkv_map(&mk, k, L, rows) || !make_qkv_map(&mv, v, L, rows))
         return GDN_ERR_CUDA;
-    return g ? launch_gdn_t<true>(mq, mk, mv, beta, g, o, s0, s_final, cu, nctas, H, L, scale, stream)
-             : launch_gdn_t<false>(mq, mk, mv, beta, g, o, s0, s_final, cu, nctas, H, L, scale, stream);
+    const bool opts = oo.bf16 || oo.dskip != nullptr;   // the general output epilogue
+    if (g) return opts ? launch_gdn_t<true, true>(mq, mk, mv, beta, g, out, s0, s_final, cu, nctas, H, L, scale, stream)
+                       : launch_gdn_t<true, false>(mq, mk, mv, beta, g, out, s0, s_final, cu, nctas, H, L, scale, stream);
+    return opts ? launch_gdn_t<false, true>(mq, mk, mv, beta, g, out, s0, s_final, cu, nctas, H, L, scale, stream)
+                : launch_gdn_t<false, false>(mq, mk, mv, beta, g, out, s0, s_final, cu, nctas, H, L, scale, stream);
 }
 
 }  // namespace gdn

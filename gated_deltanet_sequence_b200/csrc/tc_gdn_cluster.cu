@@ -113,11 +113,11 @@ enum : int {
     kNumBars = 30
 };
 
-template <bool GATED>
+template <bool GATED, bool OPTS>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_gdn_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ beta,
-                 const float *__restrict__ g, float *__restrict__ o, const float *__restrict__ s0,
+                 const float *__restrict__ g, const OutArgs out, const float *__restrict__ s0,
                  float *__restrict__ s_final, const int *__restrict__ cu, int H, int Lrow, float scale,
                  long long wait_limit, unsigned *__restrict__ err_word) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -278,6 +278,8 @@ tc_gdn_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             // ================================================================ state group
             const int j = tid - kGroupS * 32;                // = TMEM lane (key row j / value column v)
             const bool lead = (j == 0);
+            // D-skip weight of value column j (head zc mod H: dense and packed grids alike)
+            const float dj = (OPTS && out.v) ? out.dskip[(zc % H) * kD + j] : 0.f;
             const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
             {
                 const float *src = s0 ? s0 + (static_cast<size_t>(bh) * kD + j) * kD : nullptr;
@@ -352,7 +354,7 @@ tc_gdn_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     if (c + 2 < nchunks && lead)
                         mbar_arrive_cluster(mapa_shared(smem_u32(&bars[B_SFREE + (((c - 1) >> 1) & 1)]), 1 + (c & 1)));
                     tc_fence_after();
-                    store_out_col(trow + TM_O + (cp & 1) * 64, o + (row0 + static_cast<size_t>(cp) * kC) * kD + j, kC);
+                    store_out_col<OPTS>(trow + TM_O + (cp & 1) * 64, out, (row0 + static_cast<size_t>(cp) * kC) * kD + j, kC, dj);
                     done = c;
                 }
                 // ---- Ut^T row v -> Ut operand (K-major, rows v)
@@ -374,8 +376,8 @@ tc_gdn_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 const int cp = nchunks - 1;
                 if (ctl.group_wait(B_CDONE + (cp & 1), (cp >> 1) & 1, kBarS, abort_s, lead)) {
                     tc_fence_after();
-                    store_out_col(trow + TM_O + (cp & 1) * 64, o + (row0 + static_cast<size_t>(cp) * kC) * kD + j,
-                                  L - cp * kC);
+                    store_out_col<OPTS>(trow + TM_O + (cp & 1) * 64, out, (row0 + static_cast<size_t>(cp) * kC) * kD + j,
+                                  L - cp * kC, dj);
                     done = nchunks;
                 }
             }
@@ -799,11 +801,11 @@ tc_gdn_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     cluster_sync();
 }
 
-template <bool GATED>
+template <bool GATED, bool OPTS>
 gdn_status_t launch_cl_t(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const float *beta,
-                         const float *g, float *o, const float *s0, float *s_final, const int *cu, int nctas,
-                         int H, int L, float scale, cudaStream_t stream) {
-    auto kern = tc_gdn_cl_kernel<GATED>;
+                         const float *g, const OutArgs &out, const float *s0, float *s_final, const int *cu,
+                         int nctas, int H, int L, float scale, cudaStream_t stream) {
+    auto kern = tc_gdn_cl_kernel<GATED, OPTS>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [&] {
@@ -825,7 +827,7 @@ gdn_status_t launch_cl_t(const CUtensorMap &mq, const CUtensorMap &mk, const CUt
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     const long long limit = kWaitLimitCycles;
-    return cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, beta, g, o, s0, s_final, cu, H, L, scale, limit, err) ==
+    return cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, beta, g, out, s0, s_final, cu, H, L, scale, limit, err) ==
                    cudaSuccess
                ? GDN_OK
                : GDN_ERR_CUDA;
@@ -845,15 +847,19 @@ bool tc_gdn_cluster_fits(int nctas) {
 }
 
 gdn_status_t launch_tc_gdn_cluster(const void *q, const void *k, const void *v, const float *beta, const float *g,
-                                   float *o, const float *s0, float *s_final, const int *cu, int B, int H, int L,
-                                   float scale, cudaStream_t stream) {
+                                   void *o, const float *s0, float *s_final, const int *cu, int B, int H, int L,
+                                   float scale, OutOpts oo, cudaStream_t stream) {
     const int nctas = B * H;                 // one cluster per (sequence, head)
+    const OutArgs out{o, oo.dskip ? static_cast<const __nv_bfloat16 *>(v) : nullptr, oo.dskip, oo.bf16 ? 1 : 0};
     const int rows = cu ? H : B * H;         // rows of the (rows, L) token grid
     CUtensorMap mq, mk, mv;
     if (!make_qkv_map(&mq, q, L, rows) || !make_qkv_map(&mk, k, L, rows) || !make_qkv_map(&mv, v, L, rows))
         return GDN_ERR_CUDA;
-    return g ? launch_cl_t<true>(mq, mk, mv, beta, g, o, s0, s_final, cu, nctas, H, L, scale, stream)
-             : launch_cl_t<false>(mq, mk, mv, beta, g, o, s0, s_final, cu, nctas, H, L, scale, stream);
+    const bool opts = oo.bf16 || oo.dskip != nullptr;   // the general output epilogue
+    if (g) return opts ? launch_cl_t<true, true>(mq, mk, mv, beta, g, out, s0, s_final, cu, nctas, H, L, scale, stream)
+                       : launch_cl_t<true, false>(mq, mk, mv, beta, g, out, s0, s_final, cu, nctas, H, L, scale, stream);
+    return opts ? launch_cl_t<false, true>(mq, mk, mv, beta, g, out, s0, s_final, cu, nctas, H, L, scale, stream)
+                : launch_cl_t<false, false>(mq, mk, mv, beta, g, out, s0, s_final, cu, nctas, H, L, scale, stream);
 }
 
 }  // namespace gdn

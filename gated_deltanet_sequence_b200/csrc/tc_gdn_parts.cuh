@@ -107,13 +107,20 @@ __device__ __forceinline__ void st_row16_h(uint32_t tile, uint32_t row, int ch, 
                  pack_h2(x[14], x[15]));
 }
 
-// 64 output rows of one value column from TMEM to HBM (rows >= n are padding)
-__device__ __forceinline__ void store_out_col(uint32_t taddr, float *ocol, int n) {
+// 64 output rows of one value column from TMEM to HBM (rows >= n are padding), with the
+// output options (fp32 / bf16, D-skip term dj * v) when OPTS, plain fp32 otherwise
+template <bool OPTS>
+__device__ __forceinline__ void store_out_col(uint32_t taddr, const OutArgs &out, size_t elem0, int n, float dj) {
     float ov[64];
     ld_cols<64>(taddr, ov);
+    if constexpr (OPTS) {
+        store_out_rows(ov, out.o, elem0, n, kD, out.bf16 != 0, dj, out.v);
+    } else {
+        float *ocol = static_cast<float *>(out.o) + elem0;
 #pragma unroll
-    for (int r = 0; r < 64; ++r)
-        if (r < n) ocol[static_cast<size_t>(r) * kD] = ov[r];
+        for (int r = 0; r < 64; ++r)
+            if (r < n) ocol[static_cast<size_t>(r) * kD] = ov[r];
+    }
 }
 
 // W^T row j (TMEM) -> fp16 MN-major W operand in a stage's V slot

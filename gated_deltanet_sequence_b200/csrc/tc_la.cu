@@ -143,10 +143,10 @@ __device__ __forceinline__ uint4 scale_chunk(uint4 x, float f) {
     return x;
 }
 
-template <bool GATED>
+template <bool GATED, bool OPTS>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-             const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ g, float *__restrict__ o,
+             const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ g, const OutArgs out,
              const float *__restrict__ s0, float *__restrict__ s_final, const int *__restrict__ cu, int H,
              int Lrow, float scale, long long wait_limit, unsigned *__restrict__ err_word) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -415,6 +415,8 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         const int v = tid - 256;                          // TMEM lane = value column
         const bool lead = (v == 0);
         const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+        // D-skip weight of value column v (head zc mod H: dense and packed grids alike)
+        const float dv_skip = (OPTS && out.v) ? out.dskip[(zc % H) * kD + v] : 0.f;
 #pragma unroll 1
         for (int c = 0; c < nchunks; ++c) {
             const int p = c & 1;
@@ -426,10 +428,15 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             named_bar(kBarOut, 128);
             if (lead) mbar_arrive(&bars[B_OFREE + p]);
             const int n = min(kC, L - c * kC);
-            float *ocol = o + (row0 + static_cast<size_t>(c) * kC) * kD + v;
+            if constexpr (OPTS) {
+                store_out_rows(ov, out.o, (row0 + static_cast<size_t>(c) * kC) * kD + v, n, kD, out.bf16 != 0,
+                               dv_skip, out.v);
+            } else {
+                float *ocol = static_cast<float *>(out.o) + (row0 + static_cast<size_t>(c) * kC) * kD + v;
 #pragma unroll
-            for (int r = 0; r < 64; ++r)
-                if (r < n) ocol[static_cast<size_t>(r) * kD] = ov[r];
+                for (int r = 0; r < 64; ++r)
+                    if (r < n) ocol[static_cast<size_t>(r) * kD] = ov[r];
+            }
         }
     } else if (warp >= 18) {
         // ================================================================ P writers
@@ -556,11 +563,11 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     }
 }
 
-template <bool GATED>
+template <bool GATED, bool OPTS>
 gdn_status_t launch_la_t(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const float *g,
-                         float *o, const float *s0, float *s_final, const int *cu, int nctas, int H, int L,
-                         float scale, cudaStream_t stream) {
-    auto kern = tc_la_kernel<GATED>;
+                         const OutArgs &out, const float *s0, float *s_final, const int *cu, int nctas, int H,
+                         int L, float scale, cudaStream_t stream) {
+    auto kern = tc_la_kernel<GATED, OPTS>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [&] {
@@ -569,23 +576,27 @@ gdn_status_t launch_la_t(const CUtensorMap &mq, const CUtensorMap &mk, const CUt
     if (attr_err != cudaSuccess) return GDN_ERR_CUDA;
     unsigned *err = device_error_word();
     if (!err) return GDN_ERR_CUDA;
-    kern<<<nctas, kThreads, kSmemAlloc, stream>>>(mq, mk, mv, g, o, s0, s_final, cu, H, L, scale, kWaitLimitCycles,
+    kern<<<nctas, kThreads, kSmemAlloc, stream>>>(mq, mk, mv, g, out, s0, s_final, cu, H, L, scale, kWaitLimitCycles,
                                                   err);
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
 }  // namespace
 
-gdn_status_t launch_tc_la(const void *q, const void *k, const void *v, const float *g, float *o,
+gdn_status_t launch_tc_la(const void *q, const void *k, const void *v, const float *g, void *o,
                           const float *s0, float *s_final, const int *cu, int B, int H, int L, float scale,
-                          cudaStream_t stream) {
+                          OutOpts oo, cudaStream_t stream) {
     const int nctas = B * H;                 // one CTA per (sequence, head)
+    const OutArgs out{o, oo.dskip ? static_cast<const __nv_bfloat16 *>(v) : nullptr, oo.dskip, oo.bf16 ? 1 : 0};
     const int rows = cu ? H : B * H;         // rows of the (rows, L) token grid
     CUtensorMap mq, mk, mv;
     if (!make_qkv_map(&mq, q, L, rows) || !make_qkv_map(&mk, k, L, rows) || !make_qkv_map(&mv, v, L, rows))
         return GDN_ERR_CUDA;
-    return g ? launch_la_t<true>(mq, mk, mv, g, o, s0, s_final, cu, nctas, H, L, scale, stream)
-             : launch_la_t<false>(mq, mk, mv, g, o, s0, s_final, cu, nctas, H, L, scale, stream);
+    const bool opts = oo.bf16 || oo.dskip != nullptr;   // the general output epilogue
+    if (g) return opts ? launch_la_t<true, true>(mq, mk, mv, g, out, s0, s_final, cu, nctas, H, L, scale, stream)
+                       : launch_la_t<true, false>(mq, mk, mv, g, out, s0, s_final, cu, nctas, H, L, scale, stream);
+    return opts ? launch_la_t<false, true>(mq, mk, mv, g, out, s0, s_final, cu, nctas, H, L, scale, stream)
+                : launch_la_t<false, false>(mq, mk, mv, g, out, s0, s_final, cu, nctas, H, L, scale, stream);
 }
 
 }  // namespace gdn

@@ -139,6 +139,12 @@ def make_varlen_inputs(lens, H: int, dk: int, dv: int, *, mode: str = "gdn",
     return out
 
 
+def make_dskip(H: int, dv: int, *, seed: int = SEED_BASE, device="cpu") -> torch.Tensor:
+    """Skip-term weights D (H, dv) fp32 ~ N(0, 1) for the output option o_t += D_h v_t (the
+    pages give no distribution for them)."""
+    return torch.randn(H, dv, dtype=torch.float32, device=device, generator=_gen(seed, device))
+
+
 def make_decode_inputs(N: int, H: int, dk: int, dv: int, steps: int, *,
                        in_dtype: torch.dtype = torch.bfloat16, seed: int = SEED_BASE + 4,
                        device="cpu", delta: bool = True, gated: bool = True) -> dict:

@@ -121,6 +121,44 @@ gdn_status_t gdn_chunk_fwd_varlen(const void *q, const void *k, const void *v, c
                                   int chunk, float scale, gdn_dtype_t in_dtype, void *cuda_stream);
 
 /*
+ * Output options of the *_ex prefill calls (zero-initialise, then set what is used;
+ * a NULL options pointer means the defaults).
+ *  out_dtype  dtype of o: GDN_F32 (default) or GDN_BF16 (each fp32 result rounded to
+ *             the nearest bf16, ties to even; an option of this library that halves the
+ *             output bytes).
+ *  d_skip     (H, dv) fp32 device pointer, 4-byte aligned, nullable. When set, the
+ *             output gains the skip term of Mamba: o_t += d_skip[h] (elementwise) v_t,
+ *             v_t being the input value row (page "【CS336】lecture4", section
+ *             "继续改进：Mamba": a term in v added at the output, like a residual
+ *             connection, so the input reaches the output without the state).
+ */
+typedef struct gdn_out_opts {
+    gdn_dtype_t out_dtype;
+    const float *d_skip;
+} gdn_out_opts_t;
+
+/*
+ * lin_attn_chunk_fwd_ex / gdn_chunk_fwd_ex — the prefill calls with output options and
+ * an optional packed layout:
+ *  cu_seqlens == NULL: dense batch, arguments exactly as lin_attn_chunk_fwd /
+ *                      gdn_chunk_fwd (B sequences, L tokens each, (B, H, L, d) tensors).
+ *  cu_seqlens != NULL: packed batch, arguments as the *_varlen calls with B = N (the
+ *                      number of sequences) and L = T (the packed length of each head).
+ *  o          written in opts->out_dtype (fp32 when opts is NULL), same shape as before.
+ *  opts       nullable, see gdn_out_opts_t; an unknown out_dtype or a misaligned d_skip
+ *             returns GDN_ERR_INVALID_ARG.
+ * Every other rule (sizes, alignment, aliasing, errors) is that of the dense / packed call.
+ */
+gdn_status_t lin_attn_chunk_fwd_ex(const void *q, const void *k, const void *v, const float *g, void *o,
+                                   const float *s0, float *s_final, const int *cu_seqlens, int B, int H, int L,
+                                   int dk, int dv, int chunk, float scale, gdn_dtype_t in_dtype,
+                                   const gdn_out_opts_t *opts, void *cuda_stream);
+gdn_status_t gdn_chunk_fwd_ex(const void *q, const void *k, const void *v, const float *beta, const float *g,
+                              void *o, const float *s0, float *s_final, const int *cu_seqlens, int B, int H, int L,
+                              int dk, int dv, int chunk, float scale, gdn_dtype_t in_dtype,
+                              const gdn_out_opts_t *opts, void *cuda_stream);
+
+/*
  * gdn_decode_step — one token for N independent sequences, state updated in place:
  *   u = beta (v - alpha S^T k);  o = alpha S^T q' + (q'.k) u;  S <- alpha S + k u^T
  * with q' = scale q (o equals S_new^T q'). The state is read once and written

@@ -6,7 +6,8 @@ library: the arithmetic lives in ``gdn_oracle.c`` (plain C, IEEE double, no
 fast-math), compiled here with gcc and called through ctypes.
 
 Functions (each cites the passages it follows in ``gdn_oracle.c``):
-  recurrent_fwd  token-by-token recurrence, the definition of the operator
+  recurrent_fwd  token-by-token recurrence, the definition of the operator (optionally
+                 with Mamba's skip term o_t += D_h v_t, added here in numpy)
   decode_step    one token for many independent heads, state in place
   chunked_fwd    fp64 chunkwise re-derivation (UT/WY form) for invariance tests
   ut_transform   the per-chunk T = (I + A)^-1 factor
@@ -101,11 +102,15 @@ def _ptr(a: Optional[np.ndarray]):
 
 
 def recurrent_fwd(q, k, v, beta=None, g=None, s0=None, scale: float = 1.0,
-                  nthreads: Optional[int] = None, lib=None):
+                  nthreads: Optional[int] = None, lib=None, d_skip=None):
     """Token-by-token fp64 recurrence.
 
-    q, k: (..., L, dk); v: (..., L, dv); beta, g: (..., L) or None; s0: (..., dk, dv)
-    or None. Returns (o (..., L, dv), S_final (..., dk, dv)) as float64 arrays.
+    q, k: (..., H, L, dk); v: (..., H, L, dv); beta, g: (..., H, L) or None; s0:
+    (..., H, dk, dv) or None. d_skip: (H, dv) or None, the skip term of Mamba (page
+    "【CS336】lecture4", section "继续改进：Mamba": a term in v is added to the output, like
+    a residual connection, so the input reaches the output without passing the state):
+    o_t += d_skip[h] * v_t elementwise. Returns (o (..., H, L, dv), S_final (..., H, dk,
+    dv)) as float64 arrays.
     """
     q, k, v, beta, g, s0 = map(_f64, (q, k, v, beta, g, s0))
     lead = q.shape[:-2]
@@ -119,17 +124,23 @@ def recurrent_fwd(q, k, v, beta=None, g=None, s0=None, scale: float = 1.0,
                                       nthreads or default_threads())
     if rc:
         raise ValueError("oracle_recurrent_fwd: bad sizes")
+    if d_skip is not None:
+        D = _f64(d_skip)
+        if not lead or D.shape != (lead[-1], dv):
+            raise ValueError(f"d_skip: expected (H, dv) = ({lead[-1] if lead else '?'}, {dv}), got {D.shape}")
+        o += D.reshape((1,) * (len(lead) - 1) + (lead[-1], 1, dv)) * v
     return o, sf
 
 
 def recurrent_fwd_varlen(q, k, v, cu_seqlens, beta=None, g=None, s0=None, scale: float = 1.0,
-                         nthreads: Optional[int] = None, lib=None):
+                         nthreads: Optional[int] = None, lib=None, d_skip=None):
     """Packed variable-length batch: every sequence is its own recurrence.
 
     q, k: (H, T, dk); v: (H, T, dv); beta, g: (H, T) or None; cu_seqlens: N + 1 offsets
     (sequence n of every head is tokens cu[n] .. cu[n+1]-1); s0: (N, H, dk, dv) or None.
     Each sequence runs through :func:`recurrent_fwd` from its own initial state. Returns
     (o (H, T, dv) with zeros at rows outside every sequence, S_final (N, H, dk, dv)).
+    d_skip (H, dv) as for :func:`recurrent_fwd`.
     """
     q, k, v, beta, g, s0 = map(_f64, (q, k, v, beta, g, s0))
     cu = [int(x) for x in np.asarray(cu_seqlens).reshape(-1)]
@@ -145,7 +156,7 @@ def recurrent_fwd_varlen(q, k, v, cu_seqlens, beta=None, g=None, s0=None, scale:
         sl = slice(a, b)
         on, sfn = recurrent_fwd(q[:, sl], k[:, sl], v[:, sl],
                                 None if beta is None else beta[:, sl], None if g is None else g[:, sl],
-                                None if s0 is None else s0[n], scale, nthreads, lib)
+                                None if s0 is None else s0[n], scale, nthreads, lib, d_skip)
         o[:, sl] = on
         sf[n] = sfn
     return o, sf

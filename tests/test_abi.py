@@ -27,7 +27,8 @@ def _declared_functions():
 def test_header_declares_the_boundary():
     names = _declared_functions()
     for want in ("lin_attn_chunk_fwd", "gdn_chunk_fwd", "lin_attn_chunk_fwd_varlen", "gdn_chunk_fwd_varlen",
-                 "gdn_decode_step", "gdn_status_str", "gdn_sync_status", "gdn_version"):
+                 "lin_attn_chunk_fwd_ex", "gdn_chunk_fwd_ex", "gdn_decode_step", "gdn_status_str",
+                 "gdn_sync_status", "gdn_version"):
         assert want in names
 
 
@@ -133,3 +134,44 @@ def test_varlen_binding_checks_shapes(lib):
         lib.gdn_chunk_fwd_varlen(q, q, torch.zeros(2, 9, 64), torch.zeros(2, 8), cu)
     with pytest.raises(TypeError):
         lib.lin_attn_chunk_fwd_varlen(q, q, q, cu.long())
+
+
+def _ex(lib, fn, out_dtype=0, d_skip=None, no_opts=False, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, beta=FAKE, g=None, o=FAKE, s0=None, s_final=None, cu=None,
+             B=1, H=1, L=8, dk=64, dv=64, chunk=64, scale=1.0, dt=1)
+    a.update(kw)
+    P = ctypes.c_void_p
+    opts = None if no_opts else ctypes.byref(lib.OutOpts(out_dtype, d_skip))
+    if fn == "gdn":
+        return lib.lib.gdn_chunk_fwd_ex(P(a["q"]), P(a["k"]), P(a["v"]), P(a["beta"]), P(a["g"]), P(a["o"]),
+                                        P(a["s0"]), P(a["s_final"]), P(a["cu"]), a["B"], a["H"], a["L"],
+                                        a["dk"], a["dv"], a["chunk"], a["scale"], a["dt"], opts, None)
+    return lib.lib.lin_attn_chunk_fwd_ex(P(a["q"]), P(a["k"]), P(a["v"]), P(a["g"]), P(a["o"]), P(a["s0"]),
+                                         P(a["s_final"]), P(a["cu"]), a["B"], a["H"], a["L"], a["dk"], a["dv"],
+                                         a["chunk"], a["scale"], a["dt"], opts, None)
+
+
+@pytest.mark.parametrize("fn", ["gdn", "la"])
+@pytest.mark.parametrize("kw,want", [
+    (dict(out_dtype=2), 1), (dict(out_dtype=-1), 1), (dict(d_skip=FAKE + 2), 1),
+    (dict(B=0), 1), (dict(o=FAKE + 8), 1), (dict(dt=7), 1), (dict(dk=96), 2), (dict(chunk=65), 2),
+    (dict(cu=FAKE + 2), 1), (dict(cu=FAKE, B=0), 1), (dict(no_opts=True, q=None), 1),
+])
+def test_ex_rejects_bad_arguments(lib, fn, kw, want):
+    assert _ex(lib, fn, **kw) == want
+
+
+def test_ex_gdn_requires_beta(lib):
+    assert _ex(lib, "gdn", beta=None) == 1
+    assert _ex(lib, "gdn", beta=None, cu=FAKE) == 1
+
+
+def test_binding_checks_output_options(lib):
+    import torch
+    q = torch.zeros(1, 2, 4, 64)
+    with pytest.raises(TypeError):      # o dtype must be fp32 or bf16
+        lib.lin_attn_chunk_fwd(q, q, q, out_dtype=torch.float16)
+    with pytest.raises(ValueError):     # d_skip is (H, dv)
+        lib.lin_attn_chunk_fwd(q, q, q, d_skip=torch.zeros(3, 64))
+    with pytest.raises(TypeError):      # d_skip is fp32
+        lib.gdn_chunk_fwd(q, q, q, torch.zeros(1, 2, 4), d_skip=torch.zeros(2, 64, dtype=torch.float64))

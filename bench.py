@@ -56,10 +56,11 @@ def flops_per_head_token(mode: str, dk: int, dv: int, C: int) -> float:
     return 2 * C * (dk + dv) + 4 * dk * dv
 
 
-def prefill_bytes(B, H, L, dk, dv, in_bytes, delta, gated, s0, s_final) -> float:
-    """Algorithmic HBM bytes of one prefill launch: each input read once, each output written once."""
+def prefill_bytes(B, H, L, dk, dv, in_bytes, delta, gated, s0, s_final, out_bytes=4) -> float:
+    """Algorithmic HBM bytes of one prefill launch: each input read once, each output written once
+    (o in fp32, out_bytes = 4, or bf16, out_bytes = 2)."""
     n = B * H * L
-    b = n * (2 * dk + dv) * in_bytes + n * dv * 4
+    b = n * (2 * dk + dv) * in_bytes + n * dv * out_bytes
     b += n * 4 * (int(delta) + int(gated))
     b += B * H * dk * dv * 4 * (int(s0) + int(s_final))
     return float(b)
@@ -289,7 +290,26 @@ def measure_rows(gdn, peaks, peak_src, args):
     nb = prefill_bytes(w.B, w.H, w.L, w.dk, w.dv, 2, False, False, False, False)
     fl = flops_per_head_token("la", w.dk, w.dv, w.chunk) * w.B * w.H * w.L
     rows["la_prefill"] = _row(w, ms, nb, fl, peaks, peak_src, "hbm", w.B * w.L, "lin_attn_tc")
-    del inp, o
+    # the same with the bf16 output option (half the output bytes)
+    ob = torch.empty(w.B, w.H, w.L, w.dv, device="cuda", dtype=torch.bfloat16)
+    fn = lambda: gdn.lin_attn_chunk_fwd(inp["q"], inp["k"], inp["v"], None, o=ob, chunk=w.chunk)
+    ms = timed(fn, max(5, args.steps), 3)
+    nb = prefill_bytes(w.B, w.H, w.L, w.dk, w.dv, 2, False, False, False, False, out_bytes=2)
+    rows["la_prefill_bf16_out"] = _row(w, ms, nb, fl, peaks, peak_src, "hbm", w.B * w.L)
+    del inp, o, ob
+    # Gated DeltaNet 8 x 16 x 4096 x 128 with both output options: bf16 o and the skip term
+    w = W.WORKLOADS[2]
+    inp = W.make_workload_inputs(w, device="cuda")
+    D = W.make_dskip(w.H, w.dv, seed=W.SEED_BASE + 6, device="cuda")
+    ob = torch.empty(w.B, w.H, w.L, w.dv, device="cuda", dtype=torch.bfloat16)
+    sf = torch.empty(w.B, w.H, w.dk, w.dv, device="cuda")
+    fn = lambda: gdn.gdn_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["g"], o=ob, s_final=sf,
+                                   chunk=w.chunk, d_skip=D)
+    ms = timed(fn, max(5, args.steps), 3)
+    nb = prefill_bytes(w.B, w.H, w.L, w.dk, w.dv, 2, True, True, False, True, out_bytes=2) + w.H * w.dv * 4
+    fl = flops_per_head_token("gdn", w.dk, w.dv, w.chunk) * w.B * w.H * w.L
+    rows["gdn_prefill_bf16_out_skip"] = _row(w, ms, nb, fl, peaks, peak_src, "hbm", w.B * w.L)
+    del inp, ob, sf
     # long-context Gated DeltaNet, 1 x 32 x 65536 x 128, S0 != 0
     w = W.WORKLOADS[3]
     inp = W.make_workload_inputs(w, device="cuda")

@@ -168,7 +168,7 @@ tc_gdn_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 int last[2] = {-1, -1};
                 for (int c = 0; c < nchunks; ++c) {
                     const int s = c & 1;
-                    if (c >= 2 && !ctl.wait(B_CDONE + s, ((c - 2) >> 1) & 1)) break;
+                    if (c >= 2 && !ctl.wait_lazy(B_CDONE + s, ((c - 2) >> 1) & 1)) break;
                     uint8_t *st = smem + s * kStageBytes;
                     uint64_t *fb = &bars[B_FULL + s];
                     mbar_arrive_expect_tx(fb, kStageBytes);
@@ -302,8 +302,10 @@ tc_gdn_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 const int s = c & 1;
                 const float *vec = reinterpret_cast<const float *>(smem + C_SLOT + (c % kSlots) * kSlotBytes + SL_VEC);
                 // S(c) complete (state-update UMMAs of chunk c-1), and this chunk's gate values
-                if (c >= 1 && !ctl.group_wait(B_SDONE, (c - 1) & 1, kBarS, abort_s, lead)) break;
-                if (!ctl.group_wait_cluster(B_SLOT + c % kSlots, (c / kSlots) & 1, kBarS, abort_s, lead)) break;
+                if (!ctl.group_wait_all({c >= 1 ? static_cast<int>(B_SDONE) : -1, B_SLOT + c % kSlots},
+                                        {static_cast<uint32_t>(c - 1) & 1u, static_cast<uint32_t>(c / kSlots) & 1u},
+                                        kBarS, abort_s, lead, 128, 2u))
+                    break;
                 tc_fence_after();
                 // ---- S row j -> fp16 MN-major operand; S <- gamma_last S (ahead of the update)
                 {
@@ -404,8 +406,10 @@ tc_gdn_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 const int s = c & 1;
                 uint8_t *st = smem + s * kStageBytes;
                 const float *vec = reinterpret_cast<const float *>(smem + C_SLOT + (c % kSlots) * kSlotBytes + SL_VEC);
-                if (!ctl.group_wait(B_FULL + s, (c >> 1) & 1, kBarC, abort_p, lead)) break;
-                if (!ctl.group_wait_cluster(B_SLOT + c % kSlots, (c / kSlots) & 1, kBarC, abort_p, lead)) break;
+                if (!ctl.group_wait_all({B_FULL + s, B_SLOT + c % kSlots},
+                                        {static_cast<uint32_t>(c >> 1) & 1u, static_cast<uint32_t>(c / kSlots) & 1u},
+                                        kBarC, abort_p, lead, 128, 2u))
+                    break;
                 // K and V: 2048 chunks of 16 B at [0,8K) [16K,24K) [32K,48K)
 #pragma unroll
                 for (int part = 0; part < 2; ++part) {
@@ -487,7 +491,7 @@ tc_gdn_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 int last[2] = {-1, -1};
                 for (int i = 0; i < nmine; ++i) {
                     const int s = i & 1, c = pc + 2 * i;
-                    if (i >= 2 && !ctl.wait(B_GREAD + s, ((i - 2) >> 1) & 1)) break;
+                    if (i >= 2 && !ctl.wait_lazy(B_GREAD + s, ((i - 2) >> 1) & 1)) break;
                     uint8_t *st = smem + s * kPStageBytes;
                     uint64_t *fb = &bars[B_PFULL + s];
                     mbar_arrive_expect_tx(fb, kPStageBytes);
@@ -507,8 +511,8 @@ tc_gdn_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 for (int i = 0; i < nmine; ++i) {
                     const int s = i & 1;
                     const uint32_t stg = sb + s * kPStageBytes;
-                    if (!ctl.wait(B_PFULL + s, (i >> 1) & 1)) break;
-                    if (i >= 1 && !ctl.wait(B_GFREE, (i - 1) & 1)) break;
+                    if (!ctl.wait_lazy(B_PFULL + s, (i >> 1) & 1)) break;
+                    if (i >= 1 && !ctl.wait_lazy(B_GFREE, (i - 1) & 1)) break;
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
@@ -542,7 +546,7 @@ tc_gdn_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 // gate values of parity s are free once the prep group finished local chunk i-2
                 if (i >= 2) {
                     int w = 1;
-                    if (lane == 0) w = ctl.wait(B_PDONE + s, ((i - 2) >> 1) & 1) ? 1 : 0;
+                    if (lane == 0) w = ctl.wait_lazy(B_PDONE + s, ((i - 2) >> 1) & 1) ? 1 : 0;
                     if (__shfl_sync(0xffffffffu, w, 0) == 0) break;
                 }
                 const float g0 = g_nx[0], g1 = g_nx[1], b0 = b_nx[0], b1 = b_nx[1];
@@ -600,10 +604,11 @@ tc_gdn_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 const uint32_t rslot = mapa_shared(sb + C_SLOT + (c % kSlots) * kSlotBytes, 0);   // in CTA 0
                 // gate values, the Gram, and the slot (free once the chain CTA finished the
                 // chunk it held, kSlots chunks earlier)
-                if (!ctl.group_wait(B_PGATE + s, (i >> 1) & 1, kBarP, abort_p, p == 0, kNP)) break;
-                if (!ctl.group_wait(B_GRAM, i & 1, kBarP, abort_p, p == 0, kNP)) break;
-                if (i >= i_reuse && !ctl.group_wait_cluster(B_SFREE + ((i - i_reuse) & 1), ((i - i_reuse) >> 1) & 1,
-                                                            kBarP, abort_p, p == 0, kNP))
+                if (!ctl.group_wait_all({B_PGATE + s, static_cast<int>(B_GRAM),
+                                         i >= i_reuse ? B_SFREE + ((i - i_reuse) & 1) : -1},
+                                        {static_cast<uint32_t>(i >> 1) & 1u, static_cast<uint32_t>(i) & 1u,
+                                         static_cast<uint32_t>((i - i_reuse) >> 1) & 1u},
+                                        kBarP, abort_p, p == 0, kNP, 4u))
                     break;
                 // gate values -> slot (96 chunks of 16 B)
                 if (p < 96) {

@@ -59,15 +59,17 @@ struct Ctl {
         return false;
     }
     // Group-uniform wait on several phases with one barrier: the leader polls each in
-    // turn (entries with b < 0 are skipped), then the group meets once.
+    // turn (entries with b < 0 are skipped; bit i of cluster_mask selects the cluster-scope
+    // acquire for entry i), then the group meets once.
     template <int N>
     __device__ __forceinline__ bool group_wait_all(const int (&b)[N], const uint32_t (&parity)[N], int bar_id,
-                                                   int *group_abort, bool leader, int nthreads = 128) const {
+                                                   int *group_abort, bool leader, int nthreads = 128,
+                                                   unsigned cluster_mask = 0u) const {
         if (leader) {
             bool ok = true;
 #pragma unroll
             for (int i = 0; i < N; ++i)
-                if (ok && b[i] >= 0) ok = wait(b[i], parity[i]);
+                if (ok && b[i] >= 0) ok = ((cluster_mask >> i) & 1u) ? wait_cluster(b[i], parity[i]) : wait(b[i], parity[i]);
             if (!ok) *reinterpret_cast<volatile int *>(group_abort) = 1;
         }
         named_bar(bar_id, nthreads);

@@ -26,9 +26,10 @@ EXPORTS = ("lin_attn_chunk_fwd", "gdn_chunk_fwd", "lin_attn_chunk_fwd_varlen", "
            "gdn_sync_status", "gdn_version")
 
 
-class OutOpts(ctypes.Structure):
-    """gdn_out_opts_t: dtype of o and the D-skip weights (H, dv) (device pointer or None)."""
-    _fields_ = [("out_dtype", ctypes.c_int), ("d_skip", ctypes.c_void_p)]
+class FwdOpts(ctypes.Structure):
+    """gdn_fwd_opts_t: dtype of o, the D-skip weights (H, dv) (device pointer or None) and
+    the vector-valued gate flag (g holds one log-decay per key coordinate)."""
+    _fields_ = [("out_dtype", ctypes.c_int), ("d_skip", ctypes.c_void_p), ("g_per_key", ctypes.c_int)]
 
 
 class GdnError(RuntimeError):
@@ -108,17 +109,28 @@ def _raise(fn: str, st: int):
         raise GdnError(fn, st)
 
 
-def _out_opts(o, out_dtype, d_skip, H, dv, dev):
-    """Output dtype (from ``o`` when given, else ``out_dtype``, default fp32) and the
-    checked D-skip weights; returns (dtype, OutOpts or None when both are defaults)."""
+def _check_gate(g, tok_shape, dk, dev):
+    """g is one log-decay per token (tok_shape) or per token and key coordinate
+    (tok_shape + (dk,), a vector-valued gate); returns whether it is the latter."""
+    if g is None:
+        return False
+    vec = g.dim() == len(tok_shape) + 1
+    _check("g", g, tuple(tok_shape) + ((dk,) if vec else ()), torch.float32, dev)
+    return vec
+
+
+def _out_opts(o, out_dtype, d_skip, H, dv, dev, g_per_key=False):
+    """Output dtype (from ``o`` when given, else ``out_dtype``, default fp32), the checked
+    D-skip weights and the vector-gate flag; returns (dtype, FwdOpts or None when all are
+    defaults)."""
     dt = o.dtype if o is not None else (out_dtype or torch.float32)
     if dt not in (torch.float32, torch.bfloat16):
         raise TypeError(f"o / out_dtype must be float32 or bfloat16, got {dt}")
     _check("d_skip", d_skip, (H, dv), torch.float32, dev, required=False)
-    if dt == torch.float32 and d_skip is None:
+    if dt == torch.float32 and d_skip is None and not g_per_key:
         return dt, None
-    return dt, OutOpts(GDN_BF16 if dt == torch.bfloat16 else GDN_F32,
-                       None if d_skip is None else d_skip.data_ptr())
+    return dt, FwdOpts(GDN_BF16 if dt == torch.bfloat16 else GDN_F32,
+                       None if d_skip is None else d_skip.data_ptr(), int(bool(g_per_key)))
 
 
 def lin_attn_chunk_fwd(q, k, v, g=None, o=None, s0=None, s_final=None, chunk: int = 64,
@@ -126,16 +138,18 @@ def lin_attn_chunk_fwd(q, k, v, g=None, o=None, s0=None, s_final=None, chunk: in
     """Plain (g None) or gated causal linear attention. Returns (o, s_final).
 
     out_dtype (torch.float32 / torch.bfloat16) sets the dtype of a new ``o``; d_skip (H, dv)
-    fp32 adds the skip term o_t += d_skip[h] * v_t."""
+    fp32 adds the skip term o_t += d_skip[h] * v_t. g of shape (B, H, L, dk) is a
+    vector-valued gate (row j of the state decays by exp(g_t[j])); it runs on the fp32
+    chunk kernel."""
     B, H, L, dk = q.shape
     dv = v.shape[-1]
     dev = q.device
     _check("q", q, (B, H, L, dk), device=dev)
     _check("k", k, (B, H, L, dk), q.dtype, dev)
     _check("v", v, (B, H, L, dv), q.dtype, dev)
-    _check("g", g, (B, H, L), torch.float32, dev, required=False)
+    vec = _check_gate(g, (B, H, L), dk, dev)
     _check("s0", s0, (B, H, dk, dv), torch.float32, dev, required=False)
-    odt, opts = _out_opts(o, out_dtype, d_skip, H, dv, dev)
+    odt, opts = _out_opts(o, out_dtype, d_skip, H, dv, dev, vec)
     if o is None:
         o = torch.empty(B, H, L, dv, dtype=odt, device=dev)
     _check("o", o, (B, H, L, dv), odt, dev)
@@ -164,9 +178,9 @@ def gdn_chunk_fwd(q, k, v, beta, g=None, o=None, s0=None, s_final=None, chunk: i
     _check("k", k, (B, H, L, dk), q.dtype, dev)
     _check("v", v, (B, H, L, dv), q.dtype, dev)
     _check("beta", beta, (B, H, L), torch.float32, dev, required=L > 0)
-    _check("g", g, (B, H, L), torch.float32, dev, required=False)
+    vec = _check_gate(g, (B, H, L), dk, dev)
     _check("s0", s0, (B, H, dk, dv), torch.float32, dev, required=False)
-    odt, opts = _out_opts(o, out_dtype, d_skip, H, dv, dev)
+    odt, opts = _out_opts(o, out_dtype, d_skip, H, dv, dev, vec)
     if o is None:
         o = torch.empty(B, H, L, dv, dtype=odt, device=dev)
     _check("o", o, (B, H, L, dv), odt, dev)
@@ -212,8 +226,8 @@ def lin_attn_chunk_fwd_varlen(q, k, v, cu_seqlens, g=None, o=None, s0=None, s_fi
     Returns (o, s_final); rows outside every sequence are left as they were in ``o``.
     out_dtype and d_skip as for :func:`lin_attn_chunk_fwd`."""
     N, H, T, dk, dv, dev = _check_varlen(q, k, v, cu_seqlens, s0, s_final)
-    _check("g", g, (H, T), torch.float32, dev, required=False)
-    odt, opts = _out_opts(o, out_dtype, d_skip, H, dv, dev)
+    vec = _check_gate(g, (H, T), dk, dev)
+    odt, opts = _out_opts(o, out_dtype, d_skip, H, dv, dev, vec)
     if o is None:
         o = torch.zeros(H, T, dv, dtype=odt, device=dev)
     _check("o", o, (H, T, dv), odt, dev)
@@ -236,8 +250,8 @@ def gdn_chunk_fwd_varlen(q, k, v, beta, cu_seqlens, g=None, o=None, s0=None, s_f
     beta (H, T) fp32."""
     N, H, T, dk, dv, dev = _check_varlen(q, k, v, cu_seqlens, s0, s_final)
     _check("beta", beta, (H, T), torch.float32, dev, required=T > 0)
-    _check("g", g, (H, T), torch.float32, dev, required=False)
-    odt, opts = _out_opts(o, out_dtype, d_skip, H, dv, dev)
+    vec = _check_gate(g, (H, T), dk, dev)
+    odt, opts = _out_opts(o, out_dtype, d_skip, H, dv, dev, vec)
     if o is None:
         o = torch.zeros(H, T, dv, dtype=odt, device=dev)
     _check("o", o, (H, T, dv), odt, dev)

@@ -11,7 +11,7 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 bool opt_aligned16(const void *p) { return p == nullptr || aligned16(p); }
 bool opt_aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 bool head_dim_ok(int d) { return d == 64 || d == 128; }
-constexpr gdn::OutOpts kDefaultOut{false, nullptr};   // fp32 o, no D-skip term
+constexpr gdn::FwdOpts kDefaultOut{false, nullptr};   // fp32 o, no D-skip term
 
 gdn_status_t check_prefill(const void *q, const void *k, const void *v, const float *g, float *o,
                            const float *s0, float *s_final, int B, int H, int L, int dk, int dv,
@@ -115,13 +115,15 @@ gdn_status_t gdn_chunk_fwd_varlen(const void *q, const void *k, const void *v, c
 static gdn_status_t prefill_ex(bool delta, const void *q, const void *k, const void *v, const float *beta,
                                const float *g, void *o, const float *s0, float *s_final, const int *cu_seqlens,
                                int B, int H, int L, int dk, int dv, int chunk, float scale, gdn_dtype_t in_dtype,
-                               const gdn_out_opts_t *opts, void *cuda_stream) {
-    gdn::OutOpts oo = kDefaultOut;
+                               const gdn_fwd_opts_t *opts, void *cuda_stream) {
+    gdn::FwdOpts oo = kDefaultOut;
     if (opts) {
         if (opts->out_dtype != GDN_F32 && opts->out_dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
         if (!opt_aligned4(opts->d_skip)) return GDN_ERR_INVALID_ARG;
+        if (opts->g_per_key != 0 && opts->g_per_key != 1) return GDN_ERR_INVALID_ARG;
         oo.bf16 = opts->out_dtype == GDN_BF16;
         oo.dskip = opts->d_skip;
+        oo.gate_per_key = opts->g_per_key == 1 && g != nullptr;
     }
     if (B < 1 || !opt_aligned4(cu_seqlens)) return GDN_ERR_INVALID_ARG;
     const int grid_b = cu_seqlens ? 1 : B;   // batch extent of the token grid
@@ -131,8 +133,10 @@ static gdn_status_t prefill_ex(bool delta, const void *q, const void *k, const v
     if ((double)B * H > 2147483647.0) return GDN_ERR_INVALID_ARG;
     if (delta && L > 0 && !beta) return GDN_ERR_INVALID_ARG;
     if (!opt_aligned4(beta)) return GDN_ERR_INVALID_ARG;
+    if ((double)B * H * (double)L * dk > 9.0e18) return GDN_ERR_INVALID_ARG;   // g of (rows, dk)
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
-    if (gdn::tc_supported(in_dtype, dk, dv, chunk) && L > 0)
+    // vector-valued gates run on the fp32 chunk kernel (any input dtype and size)
+    if (gdn::tc_supported(in_dtype, dk, dv, chunk) && L > 0 && !oo.gate_per_key)
         return delta ? gdn::launch_tc_gdn(q, k, v, beta, g, o, s0, s_final, cu_seqlens, B, H, L, scale, oo, stream)
                      : gdn::launch_tc_la(q, k, v, g, o, s0, s_final, cu_seqlens, B, H, L, scale, oo, stream);
     return gdn::launch_simt_fwd(q, k, v, delta ? beta : nullptr, g, o, s0, s_final, cu_seqlens, B, H, L, dk, dv,
@@ -142,7 +146,7 @@ static gdn_status_t prefill_ex(bool delta, const void *q, const void *k, const v
 gdn_status_t lin_attn_chunk_fwd_ex(const void *q, const void *k, const void *v, const float *g, void *o,
                                    const float *s0, float *s_final, const int *cu_seqlens, int B, int H, int L,
                                    int dk, int dv, int chunk, float scale, gdn_dtype_t in_dtype,
-                                   const gdn_out_opts_t *opts, void *cuda_stream) {
+                                   const gdn_fwd_opts_t *opts, void *cuda_stream) {
     return prefill_ex(false, q, k, v, nullptr, g, o, s0, s_final, cu_seqlens, B, H, L, dk, dv, chunk, scale,
                       in_dtype, opts, cuda_stream);
 }
@@ -150,7 +154,7 @@ gdn_status_t lin_attn_chunk_fwd_ex(const void *q, const void *k, const void *v, 
 gdn_status_t gdn_chunk_fwd_ex(const void *q, const void *k, const void *v, const float *beta, const float *g,
                               void *o, const float *s0, float *s_final, const int *cu_seqlens, int B, int H, int L,
                               int dk, int dv, int chunk, float scale, gdn_dtype_t in_dtype,
-                              const gdn_out_opts_t *opts, void *cuda_stream) {
+                              const gdn_fwd_opts_t *opts, void *cuda_stream) {
     return prefill_ex(true, q, k, v, beta, g, o, s0, s_final, cu_seqlens, B, H, L, dk, dv, chunk, scale, in_dtype,
                       opts, cuda_stream);
 }

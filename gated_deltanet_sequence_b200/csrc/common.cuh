@@ -58,12 +58,13 @@ __device__ __forceinline__ void st_global4(float *p, float4 v) {
                  "f"(v.w) : "memory");
 }
 
-// Output epilogue options of the prefill kernels: o in fp32 or bf16, and the Mamba
+// Options of the prefill kernels: o in fp32 or bf16, vector-valued gates, and the Mamba
 // D-skip term o_t += D_h (elementwise) v_t, D of shape (H, dv) (page "【CS336】lecture4",
 // section "继续改进：Mamba": a term in v added at the output, like a residual branch).
-struct OutOpts {
+struct FwdOpts {
     bool bf16;            // o is bf16 (round to nearest even), else fp32
     const float *dskip;   // (H, dv) fp32, nullable (no skip term)
+    bool gate_per_key;    // g holds one log-decay per key coordinate ((rows, dk)), fp32 kernel only
 };
 // The same, as a kernel argument: o, and for the D-skip term the input v (bf16 for the
 // tensor-core kernels; same (rows, dv) layout as o) with D.
@@ -112,7 +113,7 @@ namespace gdn {
 gdn_status_t launch_simt_fwd(const void *q, const void *k, const void *v, const float *beta,
                              const float *g, void *o, const float *s0, float *s_final,
                              const int *cu, int B, int H, int L, int dk, int dv, int chunk,
-                             float scale, gdn_dtype_t in_dtype, OutOpts oo, cudaStream_t stream);
+                             float scale, gdn_dtype_t in_dtype, FwdOpts oo, cudaStream_t stream);
 gdn_status_t launch_decode(const void *q, const void *k, const void *v, const float *beta,
                            const float *g, float *state, float *o, int N, int H, int dk, int dv,
                            float scale, gdn_dtype_t in_dtype, cudaStream_t stream);

@@ -13,6 +13,13 @@
 //   W = T diag(beta gamma) K;  Ut = T diag(beta) V - W S    (Ut = V without delta)
 //   O = diag(gamma) Q S + (Q K^T o Gamma) Ut
 //   S <- gamma_n S + sum_s exp(G_n - G_s) k_s Ut_s^T
+// Vector-valued gates (one log-decay per key coordinate; row j of S decays by
+// exp(g_t[j])) give the same steps with a decay per key coordinate: G_r[j] is the
+// cumulative sum per coordinate, the masks become A_rs = beta_r sum_j k_r[j] k_s[j]
+// exp(G_r[j] - G_s[j]) and P_rs = sum_j q_r[j] k_s[j] exp(G_r[j] - G_s[j]), W =
+// T diag(beta) (K o exp(G)), the inter-chunk output uses Q o exp(G), and the state
+// update uses k_s o exp(G_n - G_s) with row j of S scaled by exp(G_n[j]). Every decay
+// factor is one exp of a difference of cumulative sums, so no decay strength overflows.
 #include "common.cuh"
 #include "tc_kernels.cuh"
 
@@ -23,7 +30,7 @@ constexpr int kSimtThreads = 256;
 constexpr int kDvs = 32;      // value columns per CTA
 constexpr int kCmax = 64;     // largest supported chunk
 
-template <int DK>
+template <int DK, bool VEC>
 struct SimtSmem {
     static constexpr int KP = DK + 1;            // padded row pitch for K, Q, W
     static constexpr int CP = kCmax + 1;         // padded row pitch for A, T, P
@@ -38,9 +45,10 @@ struct SimtSmem {
     float P[kCmax * CP];
     float G[kCmax];
     float bt[kCmax];
+    float GV[VEC ? kCmax * KP : 1];              // per-key cumulative log-decay (vector gates)
 };
 
-template <int DK, typename IT, bool DELTA>
+template <int DK, typename IT, bool DELTA, bool VEC>
 __global__ void __launch_bounds__(kSimtThreads)
 simt_chunk_fwd_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT *__restrict__ v,
                       const float *__restrict__ beta, const float *__restrict__ g,
@@ -49,7 +57,7 @@ simt_chunk_fwd_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const 
                       float *__restrict__ s_final, const int *__restrict__ cu, int H, int Lrow,
                       int dv, int C, float scale, unsigned *__restrict__ err) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    using Sm = SimtSmem<DK>;
+    using Sm = SimtSmem<DK, VEC>;
     Sm &sm = *reinterpret_cast<Sm *>(smem_raw);
     constexpr int KP = Sm::KP, CP = Sm::CP;
     const int tid = threadIdx.x;
@@ -63,7 +71,8 @@ simt_chunk_fwd_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const 
     const IT *kh = k + r0 * DK;
     const IT *vh = v + r0 * dv;
     const float *bh_beta = DELTA ? beta + r0 : nullptr;
-    const float *bh_g = g ? g + r0 : nullptr;
+    const float *bh_g = (g && !VEC) ? g + r0 : nullptr;
+    const float *bh_gv = (g && VEC) ? g + r0 * DK : nullptr;   // (L, DK) log-decays per key
     const long o0 = r0 * dv;                     // first output element of the sequence
     const float *dsk = dskip ? dskip + static_cast<long>(sp.head_row % H) * dv + c0 : nullptr;
 
@@ -85,7 +94,16 @@ simt_chunk_fwd_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const 
             const int r = i / kDvs, c = i % kDvs;
             sm.V[i] = ld_in(vh + (long)(t0 + r) * dv + c0 + c);
         }
-        if (tid < 32) {
+        if (VEC && tid >= kSimtThreads - DK) {
+            // per key coordinate j: inclusive within-chunk cumulative sum of g[:, j]
+            const int j = tid - (kSimtThreads - DK);
+            float carry = 0.f;
+            for (int r = 0; r < n; ++r) {
+                carry += bh_gv ? bh_gv[(long)(t0 + r) * DK + j] : 0.f;
+                sm.GV[r * KP + j] = carry;
+            }
+        }
+        if (!VEC && tid < 32) {
             // inclusive within-chunk cumulative sum of g (warp scan, two passes of 32)
             float carry = 0.f;
             for (int base = 0; base < n; base += 32) {
@@ -107,7 +125,16 @@ simt_chunk_fwd_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const 
         for (int i = tid; i < n * n; i += kSimtThreads) {
             const int r = i / n, s = i % n;
             float p = 0.f, a = 0.f;
-            if (s <= r) {
+            if (s <= r && VEC) {
+#pragma unroll 4
+                for (int j = 0; j < DK; ++j) {
+                    const float dec = expf(sm.GV[r * KP + j] - sm.GV[s * KP + j]);
+                    const float ks = dec * sm.K[s * KP + j];
+                    p = fmaf(sm.Q[r * KP + j], ks, p);
+                    if (DELTA) a = fmaf(sm.K[r * KP + j], ks, a);
+                }
+                if (DELTA) a = (s < r) ? sm.bt[r] * a : 0.f;
+            } else if (s <= r) {
                 const float dec = expf(sm.G[r] - sm.G[s]);
 #pragma unroll 8
                 for (int j = 0; j < DK; ++j) {
@@ -133,12 +160,26 @@ simt_chunk_fwd_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const 
             }
             __syncthreads();
             // ---- W = T diag(beta gamma) K ;  U = T diag(beta) V ----------------------
-            for (int i = tid; i < n * DK; i += kSimtThreads) {
-                const int r = i / DK, j = i % DK;
-                float w = 0.f;
-                for (int s = 0; s <= r; ++s)
-                    w = fmaf(sm.T[r * CP + s] * sm.bt[s] * expf(sm.G[s]), sm.K[s * KP + j], w);
-                sm.W[r * KP + j] = w;
+            if (VEC) {
+                // thread per key column j: W[:, j] = T (beta o exp(G[:, j]) o K[:, j]), formed
+                // in place from the last row up (row r reads rows s <= r only)
+                for (int j = tid; j < DK; j += kSimtThreads) {
+                    for (int s = 0; s < n; ++s)
+                        sm.W[s * KP + j] = sm.bt[s] * expf(sm.GV[s * KP + j]) * sm.K[s * KP + j];
+                    for (int r = n - 1; r >= 0; --r) {
+                        float w = 0.f;
+                        for (int s = 0; s <= r; ++s) w = fmaf(sm.T[r * CP + s], sm.W[s * KP + j], w);
+                        sm.W[r * KP + j] = w;
+                    }
+                }
+            } else {
+                for (int i = tid; i < n * DK; i += kSimtThreads) {
+                    const int r = i / DK, j = i % DK;
+                    float w = 0.f;
+                    for (int s = 0; s <= r; ++s)
+                        w = fmaf(sm.T[r * CP + s] * sm.bt[s] * expf(sm.G[s]), sm.K[s * KP + j], w);
+                    sm.W[r * KP + j] = w;
+                }
             }
             for (int i = tid; i < n * kDvs; i += kSimtThreads) {
                 const int r = i / kDvs, c = i % kDvs;
@@ -158,6 +199,16 @@ simt_chunk_fwd_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const 
             __syncthreads();
         }
         const float *Ut = DELTA ? sm.U : sm.V;
+        if (VEC) {
+            // the raw tiles are no longer read: Q <- Q o exp(G), K <- K o exp(G_n - G)
+            for (int i = tid; i < n * DK; i += kSimtThreads) {
+                const int r = i / DK, j = i % DK;
+                const float gr = sm.GV[r * KP + j];
+                sm.Q[r * KP + j] *= expf(gr);
+                sm.K[r * KP + j] *= expf(sm.GV[(n - 1) * KP + j] - gr);
+            }
+            __syncthreads();
+        }
         // ---- O = diag(gamma) Q S + P Ut ---------------------------------------------
         for (int i = tid; i < n * kDvs; i += kSimtThreads) {
             const int r = i / kDvs, c = i % kDvs;
@@ -166,7 +217,7 @@ simt_chunk_fwd_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const 
             for (int j = 0; j < DK; ++j) qs = fmaf(sm.Q[r * KP + j], sm.S[j * kDvs + c], qs);
             float pu = 0.f;
             for (int s = 0; s <= r; ++s) pu = fmaf(sm.P[r * CP + s], Ut[s * kDvs + c], pu);
-            float ov = expf(sm.G[r]) * qs + pu;
+            float ov = (VEC ? qs : expf(sm.G[r]) * qs) + pu;
             if (dsk) ov = fmaf(dsk[c], sm.V[i], ov);     // D-skip term D_h v_t
             const long oi = o0 + (long)(t0 + r) * dv + c0 + c;
             if (out_bf16) static_cast<__nv_bfloat16 *>(o)[oi] = __float2bfloat16_rn(ov);
@@ -178,10 +229,17 @@ simt_chunk_fwd_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const 
             const float Gn = sm.G[n - 1];
             for (int i = tid; i < DK * kDvs; i += kSimtThreads) {
                 const int j = i / kDvs, c = i % kDvs;
-                float x = expf(Gn) * sm.S[i];
-                for (int s = 0; s < n; ++s)
-                    x = fmaf(expf(Gn - sm.G[s]) * sm.K[s * KP + j], Ut[s * kDvs + c], x);
-                sm.S[i] = x;
+                if (VEC) {
+                    // K already holds k_s o exp(G_n - G_s)
+                    float x = expf(sm.GV[(n - 1) * KP + j]) * sm.S[i];
+                    for (int s = 0; s < n; ++s) x = fmaf(sm.K[s * KP + j], Ut[s * kDvs + c], x);
+                    sm.S[i] = x;
+                } else {
+                    float x = expf(Gn) * sm.S[i];
+                    for (int s = 0; s < n; ++s)
+                        x = fmaf(expf(Gn - sm.G[s]) * sm.K[s * KP + j], Ut[s * kDvs + c], x);
+                    sm.S[i] = x;
+                }
             }
         }
     }
@@ -194,13 +252,13 @@ simt_chunk_fwd_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const 
     }
 }
 
-template <int DK, typename IT, bool DELTA>
+template <int DK, typename IT, bool DELTA, bool VEC>
 gdn_status_t launch_simt_t(const void *q, const void *k, const void *v, const float *beta,
                            const float *g, void *o, const float *s0, float *s_final, const int *cu,
-                           int BH, int H, int L, int dv, int chunk, float scale, OutOpts oo, unsigned *err,
+                           int BH, int H, int L, int dv, int chunk, float scale, FwdOpts oo, unsigned *err,
                            cudaStream_t stream) {
-    auto kern = simt_chunk_fwd_kernel<DK, IT, DELTA>;
-    const int smem = (int)sizeof(SimtSmem<DK>);
+    auto kern = simt_chunk_fwd_kernel<DK, IT, DELTA, VEC>;
+    const int smem = (int)sizeof(SimtSmem<DK, VEC>);
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return GDN_ERR_CUDA;
     dim3 grid(BH, dv / kDvs);
@@ -215,16 +273,21 @@ gdn_status_t launch_simt_t(const void *q, const void *k, const void *v, const fl
 gdn_status_t launch_simt_fwd(const void *q, const void *k, const void *v, const float *beta,
                              const float *g, void *o, const float *s0, float *s_final,
                              const int *cu, int B, int H, int L, int dk, int dv, int chunk,
-                             float scale, gdn_dtype_t in_dtype, OutOpts oo, cudaStream_t stream) {
+                             float scale, gdn_dtype_t in_dtype, FwdOpts oo, cudaStream_t stream) {
     const int BH = B * H;
     const bool delta = beta != nullptr;
     unsigned *err = nullptr;
     if (cu && !(err = device_error_word())) return GDN_ERR_CUDA;
-#define GDN_SIMT_CASE(DKV, IT)                                                                     \
-    return delta ? launch_simt_t<DKV, IT, true>(q, k, v, beta, g, o, s0, s_final, cu, BH, H, L, dv, \
-                                                chunk, scale, oo, err, stream)                     \
-                 : launch_simt_t<DKV, IT, false>(q, k, v, beta, g, o, s0, s_final, cu, BH, H, L,  \
-                                                 dv, chunk, scale, oo, err, stream)
+#define GDN_SIMT_CASE(DKV, IT)                                                                          \
+    return delta ? (vec ? launch_simt_t<DKV, IT, true, true>(q, k, v, beta, g, o, s0, s_final, cu, BH, H, L, dv, \
+                                                           chunk, scale, oo, err, stream)                   \
+                        : launch_simt_t<DKV, IT, true, false>(q, k, v, beta, g, o, s0, s_final, cu, BH, H, L,  \
+                                                            dv, chunk, scale, oo, err, stream))             \
+                 : (vec ? launch_simt_t<DKV, IT, false, true>(q, k, v, beta, g, o, s0, s_final, cu, BH, H, L,  \
+                                                            dv, chunk, scale, oo, err, stream)              \
+                        : launch_simt_t<DKV, IT, false, false>(q, k, v, beta, g, o, s0, s_final, cu, BH, H, L, \
+                                                             dv, chunk, scale, oo, err, stream))
+    const bool vec = oo.gate_per_key && g != nullptr;   // one log-decay per key coordinate
     if (in_dtype == GDN_F32) {
         if (dk == 64) { GDN_SIMT_CASE(64, float); }
         GDN_SIMT_CASE(128, float);

@@ -802,7 +802,7 @@ bool tc_supported(gdn_dtype_t in_dtype, int dk, int dv, int chunk) {
 
 gdn_status_t launch_tc_gdn(const void *q, const void *k, const void *v, const float *beta, const float *g,
                            void *o, const float *s0, float *s_final, const int *cu, int B, int H, int L,
-                           float scale, OutOpts oo, cudaStream_t stream) {
+                           float scale, FwdOpts oo, cudaStream_t stream) {
     const int nctas = B * H;                 // one CTA per (sequence, head)
     // few (sequence, head) pairs: the cluster form spreads each chunk's prep over two more SMs
     if (tc_gdn_cluster_fits(nctas))

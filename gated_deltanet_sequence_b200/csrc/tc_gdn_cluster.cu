@@ -853,7 +853,7 @@ bool tc_gdn_cluster_fits(int nctas) {
 
 gdn_status_t launch_tc_gdn_cluster(const void *q, const void *k, const void *v, const float *beta, const float *g,
                                    void *o, const float *s0, float *s_final, const int *cu, int B, int H, int L,
-                                   float scale, OutOpts oo, cudaStream_t stream) {
+                                   float scale, FwdOpts oo, cudaStream_t stream) {
     const int nctas = B * H;                 // one cluster per (sequence, head)
     const OutArgs out{o, oo.dskip ? static_cast<const __nv_bfloat16 *>(v) : nullptr, oo.dskip, oo.bf16 ? 1 : 0};
     const int rows = cu ? H : B * H;         // rows of the (rows, L) token grid

@@ -11,18 +11,18 @@ bool tc_supported(gdn_dtype_t in_dtype, int dk, int dv, int chunk);
 // from global memory by the output epilogue).
 gdn_status_t launch_tc_gdn(const void *q, const void *k, const void *v, const float *beta,
                            const float *g, void *o, const float *s0, float *s_final, const int *cu,
-                           int B, int H, int L, float scale, OutOpts oo, cudaStream_t stream);
+                           int B, int H, int L, float scale, FwdOpts oo, cudaStream_t stream);
 // Cluster form (one chain CTA + two prep CTAs per (sequence, head)); same arguments and
 // the same bits as launch_tc_gdn. tc_gdn_cluster_fits: every cluster fits on the device
 // at once (3 x B*H <= SM count), i.e. the one-CTA form would leave most SMs idle.
 gdn_status_t launch_tc_gdn_cluster(const void *q, const void *k, const void *v, const float *beta,
                                    const float *g, void *o, const float *s0, float *s_final,
-                                   const int *cu, int B, int H, int L, float scale, OutOpts oo,
+                                   const int *cu, int B, int H, int L, float scale, FwdOpts oo,
                                    cudaStream_t stream);
 bool tc_gdn_cluster_fits(int nctas);
 gdn_status_t launch_tc_la(const void *q, const void *k, const void *v, const float *g, void *o,
                           const float *s0, float *s_final, const int *cu, int B, int H, int L,
-                          float scale, OutOpts oo, cudaStream_t stream);
+                          float scale, FwdOpts oo, cudaStream_t stream);
 // Reads and clears the device-side error word of the current device.
 bool read_and_clear_device_error(unsigned *err);
 // Device address of that word on the current device (looked up once per device),

@@ -139,6 +139,14 @@ def make_varlen_inputs(lens, H: int, dk: int, dv: int, *, mode: str = "gdn",
     return out
 
 
+def make_gate_per_key(lead: tuple, L: int, dk: int, *, seed: int = SEED_BASE, g_low: float = -0.05,
+                      device="cpu") -> torch.Tensor:
+    """Vector-valued log-decays g (*lead, L, dk) fp32 ~ U(g_low, 0), one per token and key
+    coordinate (the scalar gate's distribution, drawn per coordinate)."""
+    gen = _gen(seed, device)
+    return g_low * torch.rand(*lead, L, dk, dtype=torch.float32, device=device, generator=gen)
+
+
 def make_dskip(H: int, dv: int, *, seed: int = SEED_BASE, device="cpu") -> torch.Tensor:
     """Skip-term weights D (H, dv) fp32 ~ N(0, 1) for the output option o_t += D_h v_t (the
     pages give no distribution for them)."""

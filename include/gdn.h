@@ -121,8 +121,8 @@ gdn_status_t gdn_chunk_fwd_varlen(const void *q, const void *k, const void *v, c
                                   int chunk, float scale, gdn_dtype_t in_dtype, void *cuda_stream);
 
 /*
- * Output options of the *_ex prefill calls (zero-initialise, then set what is used;
- * a NULL options pointer means the defaults).
+ * Options of the *_ex prefill calls (zero-initialise, then set what is used; a NULL
+ * options pointer means the defaults).
  *  out_dtype  dtype of o: GDN_F32 (default) or GDN_BF16 (each fp32 result rounded to
  *             the nearest bf16, ties to even; an option of this library that halves the
  *             output bytes).
@@ -131,11 +131,20 @@ gdn_status_t gdn_chunk_fwd_varlen(const void *q, const void *k, const void *v, c
  *             v_t being the input value row (page "【CS336】lecture4", section
  *             "继续改进：Mamba": a term in v added at the output, like a residual
  *             connection, so the input reaches the output without the state).
+ *  g_per_key  0 (default): g holds one log-decay per token, (B, H, L) or (H, T).
+ *             1: vector-valued gate, g holds one log-decay per token and key
+ *             coordinate, (B, H, L, dk) or (H, T, dk) fp32, and row j of the state
+ *             decays by exp(g_t[j]):  S_t = (I - beta_t k_t k_t^T) diag(exp(g_t)) S_{t-1}
+ *             + beta_t k_t v_t^T (without beta: S_t = diag(exp(g_t)) S_{t-1} + k_t v_t^T),
+ *             the per-coordinate form of the scalar gate (GLA-style gates, next to the
+ *             scalar gate of page "混合注意力学习(1)", section "Gated DeltaNet"). These
+ *             calls run on the fp32 chunk kernel. Any other value: GDN_ERR_INVALID_ARG.
  */
-typedef struct gdn_out_opts {
+typedef struct gdn_fwd_opts {
     gdn_dtype_t out_dtype;
     const float *d_skip;
-} gdn_out_opts_t;
+    int g_per_key;
+} gdn_fwd_opts_t;
 
 /*
  * lin_attn_chunk_fwd_ex / gdn_chunk_fwd_ex — the prefill calls with output options and
@@ -145,18 +154,18 @@ typedef struct gdn_out_opts {
  *  cu_seqlens != NULL: packed batch, arguments as the *_varlen calls with B = N (the
  *                      number of sequences) and L = T (the packed length of each head).
  *  o          written in opts->out_dtype (fp32 when opts is NULL), same shape as before.
- *  opts       nullable, see gdn_out_opts_t; an unknown out_dtype or a misaligned d_skip
+ *  opts       nullable, see gdn_fwd_opts_t; an unknown out_dtype or a misaligned d_skip
  *             returns GDN_ERR_INVALID_ARG.
  * Every other rule (sizes, alignment, aliasing, errors) is that of the dense / packed call.
  */
 gdn_status_t lin_attn_chunk_fwd_ex(const void *q, const void *k, const void *v, const float *g, void *o,
                                    const float *s0, float *s_final, const int *cu_seqlens, int B, int H, int L,
                                    int dk, int dv, int chunk, float scale, gdn_dtype_t in_dtype,
-                                   const gdn_out_opts_t *opts, void *cuda_stream);
+                                   const gdn_fwd_opts_t *opts, void *cuda_stream);
 gdn_status_t gdn_chunk_fwd_ex(const void *q, const void *k, const void *v, const float *beta, const float *g,
                               void *o, const float *s0, float *s_final, const int *cu_seqlens, int B, int H, int L,
                               int dk, int dv, int chunk, float scale, gdn_dtype_t in_dtype,
-                              const gdn_out_opts_t *opts, void *cuda_stream);
+                              const gdn_fwd_opts_t *opts, void *cuda_stream);
 
 /*
  * gdn_decode_step — one token for N independent sequences, state updated in place:

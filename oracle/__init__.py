@@ -60,11 +60,12 @@ def _bind(path: str):
     P = ctypes.c_void_p
     l, d, i = ctypes.c_long, ctypes.c_double, ctypes.c_int
     lib.oracle_recurrent_fwd.argtypes = [P, P, P, P, P, P, P, P, l, l, l, l, d, i]
+    lib.oracle_recurrent_fwd_vg.argtypes = [P, P, P, P, P, P, P, P, l, l, l, l, d, i]
     lib.oracle_decode_step.argtypes = [P, P, P, P, P, P, P, l, l, l, d, i]
     lib.oracle_chunked_fwd.argtypes = [P, P, P, P, P, P, P, P, l, l, l, l, l, d, i]
     lib.oracle_ut_transform.argtypes = [P, P, P, P, l, l]
-    for f in (lib.oracle_recurrent_fwd, lib.oracle_decode_step, lib.oracle_chunked_fwd,
-              lib.oracle_ut_transform):
+    for f in (lib.oracle_recurrent_fwd, lib.oracle_recurrent_fwd_vg, lib.oracle_decode_step,
+              lib.oracle_chunked_fwd, lib.oracle_ut_transform):
         f.restype = ctypes.c_int
     return lib
 
@@ -105,8 +106,10 @@ def recurrent_fwd(q, k, v, beta=None, g=None, s0=None, scale: float = 1.0,
                   nthreads: Optional[int] = None, lib=None, d_skip=None):
     """Token-by-token fp64 recurrence.
 
-    q, k: (..., H, L, dk); v: (..., H, L, dv); beta, g: (..., H, L) or None; s0:
-    (..., H, dk, dv) or None. d_skip: (H, dv) or None, the skip term of Mamba (page
+    q, k: (..., H, L, dk); v: (..., H, L, dv); beta: (..., H, L) or None; g: (..., H, L)
+    (one log-decay per token) or (..., H, L, dk) (vector-valued gate, one log-decay per key
+    coordinate: row j of the state decays by exp(g_t[j]), the GLA-style variant next to the
+    scalar gate) or None; s0: (..., H, dk, dv) or None. d_skip: (H, dv) or None, the skip term of Mamba (page
     "【CS336】lecture4", section "继续改进：Mamba": a term in v is added to the output, like
     a residual connection, so the input reaches the output without passing the state):
     o_t += d_skip[h] * v_t elementwise. Returns (o (..., H, L, dv), S_final (..., H, dk,
@@ -119,9 +122,13 @@ def recurrent_fwd(q, k, v, beta=None, g=None, s0=None, scale: float = 1.0,
     BH = int(np.prod(lead)) if lead else 1
     o = np.zeros(lead + (L, dv), np.float64)
     sf = np.zeros(lead + (dk, dv), np.float64)
-    rc = (lib or _load()).oracle_recurrent_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(s0),
-                                      _ptr(o), _ptr(sf), BH, L, dk, dv, float(scale),
-                                      nthreads or default_threads())
+    vector_gate = g is not None and g.ndim == q.ndim
+    if g is not None and g.shape != (q.shape if vector_gate else q.shape[:-1]):
+        raise ValueError(f"g: expected {q.shape[:-1]} or {q.shape}, got {g.shape}")
+    lib_ = lib or _load()
+    fn = lib_.oracle_recurrent_fwd_vg if vector_gate else lib_.oracle_recurrent_fwd
+    rc = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(s0), _ptr(o), _ptr(sf), BH, L, dk, dv,
+            float(scale), nthreads or default_threads())
     if rc:
         raise ValueError("oracle_recurrent_fwd: bad sizes")
     if d_skip is not None:

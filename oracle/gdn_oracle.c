@@ -30,6 +30,12 @@
  *        o_t = S_t^T (scale * q_t)
  *  - Without beta (plain / gated linear attention): S_t = alpha_t S_{t-1} + k_t v_t^T.
  *  - Without g: alpha_t = 1.  With g: alpha_t = exp(g_t) (g is log-alpha).
+ *  - Vector-valued gates (one log-decay per key coordinate, g_t in R^dk; the
+ *    GLA-style variant next to the scalar gate flag): alpha_t = exp(g_t)
+ *    elementwise decays row j of S by alpha_t[j]:
+ *        u_t = beta_t (v_t - (diag(alpha_t) S_{t-1})^T k_t)
+ *        S_t = diag(alpha_t) S_{t-1} + k_t u_t^T
+ *    i.e. S_t = (I - beta_t k_t k_t^T) diag(alpha_t) S_{t-1} + beta_t k_t v_t^T.
  *
  * Everything is IEEE double, no fast-math; heads run on plain pthreads.
  */
@@ -70,6 +76,32 @@ static void token_step(double *S, const double *q, const double *k, const double
     for (long j = 0; j < dk; ++j)
         for (long c = 0; c < dv; ++c) S[j * dv + c] = alpha * S[j * dv + c] + k[j] * sk[c];
     /* output from the state after this token's write */
+    read_out(S, q, scale, dk, dv, o);
+}
+
+/* ------------------------------------------------------------------------- */
+/* One token with a vector-valued gate gv (dk log-decays, one per key row).  */
+/* S: dk x dv, in place.  sk: dv scratch, a: dk scratch.                      */
+static void token_step_vg(double *S, const double *q, const double *k, const double *v,
+                          const double *beta, const double *gv, double scale,
+                          long dk, long dv, double *o, double *sk, double *a)
+{
+    for (long j = 0; j < dk; ++j) a[j] = gv ? exp(gv[j]) : 1.0;
+    /* decay first: row j of the state by alpha[j] */
+    for (long j = 0; j < dk; ++j)
+        for (long c = 0; c < dv; ++c) S[j * dv + c] *= a[j];
+    if (beta) {
+        /* read the decayed memory at key k (column by column), then u = beta (v - read) */
+        for (long col = 0; col < dv; ++col) {
+            double rd = 0.0;
+            for (long row = 0; row < dk; ++row) rd += k[row] * S[row * dv + col];
+            sk[col] = (*beta) * (v[col] - rd);
+        }
+    } else {
+        memcpy(sk, v, sizeof(double) * (size_t)dv);
+    }
+    for (long row = 0; row < dk; ++row)
+        for (long col = 0; col < dv; ++col) S[row * dv + col] += sk[col] * k[row];
     read_out(S, q, scale, dk, dv, o);
 }
 
@@ -151,6 +183,34 @@ int oracle_recurrent_fwd(const double *q, const double *k, const double *v,
     if (BH < 0 || L < 0 || dk < 1 || dv < 1) return 1;
     fwd_ctx c = {q, k, v, beta, g, s0, o, s_final, L, dk, dv, scale};
     run_heads(fwd_head, &c, BH, dk * dv + dv, nthreads);
+    return 0;
+}
+
+/* Prefill with vector-valued gates: g (BH, L, dk) or NULL; the rest as above. */
+static void fwd_head_vg(void *vctx, long h, double *scratch)
+{
+    fwd_ctx *c = (fwd_ctx *)vctx;
+    const long L = c->L, dk = c->dk, dv = c->dv;
+    double *S = scratch, *sk = scratch + dk * dv, *a = sk + dv;
+    if (c->s0) memcpy(S, c->s0 + h * dk * dv, sizeof(double) * (size_t)(dk * dv));
+    else memset(S, 0, sizeof(double) * (size_t)(dk * dv));
+    for (long t = 0; t < L; ++t) {
+        const long r = h * L + t;
+        token_step_vg(S, c->q + r * dk, c->k + r * dk, c->v + r * dv,
+                      c->beta ? c->beta + r : NULL, c->g ? c->g + r * dk : NULL, c->scale,
+                      dk, dv, c->o + r * dv, sk, a);
+    }
+    if (c->s_final) memcpy(c->s_final + h * dk * dv, S, sizeof(double) * (size_t)(dk * dv));
+}
+
+int oracle_recurrent_fwd_vg(const double *q, const double *k, const double *v,
+                            const double *beta, const double *g, const double *s0,
+                            double *o, double *s_final, long BH, long L, long dk, long dv,
+                            double scale, int nthreads)
+{
+    if (BH < 0 || L < 0 || dk < 1 || dv < 1) return 1;
+    fwd_ctx c = {q, k, v, beta, g, s0, o, s_final, L, dk, dv, scale};
+    run_heads(fwd_head_vg, &c, BH, dk * dv + dv + dk, nthreads);
     return 0;
 }
 

@@ -136,12 +136,12 @@ def test_varlen_binding_checks_shapes(lib):
         lib.lin_attn_chunk_fwd_varlen(q, q, q, cu.long())
 
 
-def _ex(lib, fn, out_dtype=0, d_skip=None, no_opts=False, **kw):
+def _ex(lib, fn, out_dtype=0, d_skip=None, g_per_key=0, no_opts=False, **kw):
     a = dict(q=FAKE, k=FAKE, v=FAKE, beta=FAKE, g=None, o=FAKE, s0=None, s_final=None, cu=None,
              B=1, H=1, L=8, dk=64, dv=64, chunk=64, scale=1.0, dt=1)
     a.update(kw)
     P = ctypes.c_void_p
-    opts = None if no_opts else ctypes.byref(lib.OutOpts(out_dtype, d_skip))
+    opts = None if no_opts else ctypes.byref(lib.FwdOpts(out_dtype, d_skip, g_per_key))
     if fn == "gdn":
         return lib.lib.gdn_chunk_fwd_ex(P(a["q"]), P(a["k"]), P(a["v"]), P(a["beta"]), P(a["g"]), P(a["o"]),
                                         P(a["s0"]), P(a["s_final"]), P(a["cu"]), a["B"], a["H"], a["L"],
@@ -153,7 +153,7 @@ def _ex(lib, fn, out_dtype=0, d_skip=None, no_opts=False, **kw):
 
 @pytest.mark.parametrize("fn", ["gdn", "la"])
 @pytest.mark.parametrize("kw,want", [
-    (dict(out_dtype=2), 1), (dict(out_dtype=-1), 1), (dict(d_skip=FAKE + 2), 1),
+    (dict(out_dtype=2), 1), (dict(out_dtype=-1), 1), (dict(d_skip=FAKE + 2), 1), (dict(g_per_key=2), 1),
     (dict(B=0), 1), (dict(o=FAKE + 8), 1), (dict(dt=7), 1), (dict(dk=96), 2), (dict(chunk=65), 2),
     (dict(cu=FAKE + 2), 1), (dict(cu=FAKE, B=0), 1), (dict(no_opts=True, q=None), 1),
 ])
@@ -175,3 +175,10 @@ def test_binding_checks_output_options(lib):
         lib.lin_attn_chunk_fwd(q, q, q, d_skip=torch.zeros(3, 64))
     with pytest.raises(TypeError):      # d_skip is fp32
         lib.gdn_chunk_fwd(q, q, q, torch.zeros(1, 2, 4), d_skip=torch.zeros(2, 64, dtype=torch.float64))
+
+
+def test_binding_checks_vector_gate_shape(lib):
+    import torch
+    q = torch.zeros(1, 2, 4, 64)
+    with pytest.raises(ValueError):     # (B, H, L) or (B, H, L, dk)
+        lib.lin_attn_chunk_fwd(q, q, q, torch.zeros(1, 2, 4, 32))

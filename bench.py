@@ -309,7 +309,18 @@ def measure_rows(gdn, peaks, peak_src, args):
     nb = prefill_bytes(w.B, w.H, w.L, w.dk, w.dv, 2, True, True, False, True, out_bytes=2) + w.H * w.dv * 4
     fl = flops_per_head_token("gdn", w.dk, w.dv, w.chunk) * w.B * w.H * w.L
     rows["gdn_prefill_bf16_out_skip"] = _row(w, ms, nb, fl, peaks, peak_src, "hbm", w.B * w.L)
-    del inp, ob, sf
+    del ob
+    # the same workload with vector-valued gates (one log-decay per token and key coordinate),
+    # which run on the fp32 CUDA-core chunk kernel
+    gv = W.make_gate_per_key((w.B, w.H), w.L, w.dk, seed=W.SEED_BASE + 7, device="cuda")
+    o = torch.empty(w.B, w.H, w.L, w.dv, device="cuda")
+    fn = lambda: gdn.gdn_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["beta"], gv, o=o, s_final=sf, chunk=w.chunk)
+    ms = timed(fn, max(3, args.steps // 6), 2)
+    nb = prefill_bytes(w.B, w.H, w.L, w.dk, w.dv, 2, True, False, False, True) + w.B * w.H * w.L * w.dk * 4
+    row = _row(w, ms, nb, fl, peaks, peak_src, "hbm", w.B * w.L)
+    row["path"] = "fp32 chunk kernel (CUDA cores; every decay factor an exp)"
+    rows["gdn_prefill_vector_gate"] = row
+    del inp, o, sf, gv
     # long-context Gated DeltaNet, 1 x 32 x 65536 x 128, S0 != 0
     w = W.WORKLOADS[3]
     inp = W.make_workload_inputs(w, device="cuda")

@@ -22,8 +22,8 @@ GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_TIMEOUT 
 GDN_F32, GDN_BF16 = 0, 1
 
 EXPORTS = ("lin_attn_chunk_fwd", "gdn_chunk_fwd", "lin_attn_chunk_fwd_varlen", "gdn_chunk_fwd_varlen",
-           "lin_attn_chunk_fwd_ex", "gdn_chunk_fwd_ex", "gdn_decode_step", "gdn_status_str",
-           "gdn_sync_status", "gdn_version")
+           "lin_attn_chunk_fwd_ex", "gdn_chunk_fwd_ex", "gdn_decode_step", "gdn_decode_step_ex",
+           "gdn_status_str", "gdn_sync_status", "gdn_version")
 
 
 class FwdOpts(ctypes.Structure):
@@ -51,13 +51,14 @@ def _load() -> ctypes.CDLL:
     lib.lin_attn_chunk_fwd_ex.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P, P]
     lib.gdn_chunk_fwd_ex.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P, P]
     lib.gdn_decode_step.argtypes = [P, P, P, P, P, P, P, I, I, I, I, F, I, P]
+    lib.gdn_decode_step_ex.argtypes = [P, P, P, P, P, P, P, I, I, I, I, F, I, P, P]
     lib.gdn_status_str.argtypes = [I]
     lib.gdn_status_str.restype = ctypes.c_char_p
     lib.gdn_sync_status.argtypes = [P]
     lib.gdn_version.argtypes = []
     for f in (lib.lin_attn_chunk_fwd, lib.gdn_chunk_fwd, lib.lin_attn_chunk_fwd_varlen,
               lib.gdn_chunk_fwd_varlen, lib.lin_attn_chunk_fwd_ex, lib.gdn_chunk_fwd_ex,
-              lib.gdn_decode_step, lib.gdn_sync_status, lib.gdn_version):
+              lib.gdn_decode_step, lib.gdn_decode_step_ex, lib.gdn_sync_status, lib.gdn_version):
         f.restype = ctypes.c_int
     return lib
 
@@ -268,8 +269,10 @@ def gdn_chunk_fwd_varlen(q, k, v, beta, cu_seqlens, g=None, o=None, s0=None, s_f
     return o, s_final
 
 
-def gdn_decode_step(q, k, v, beta, g, state, o=None, scale: float = 1.0, stream=None):
-    """One decode token for (N, H) heads; ``state`` (N, H, dk, dv) fp32 is updated in place."""
+def gdn_decode_step(q, k, v, beta, g, state, o=None, scale: float = 1.0, stream=None, out_dtype=None,
+                    d_skip=None):
+    """One decode token for (N, H) heads; ``state`` (N, H, dk, dv) fp32 is updated in place.
+    g (N, H) or (N, H, dk) (vector-valued gate); out_dtype and d_skip as for the prefill calls."""
     N, H, dk = q.shape
     dv = v.shape[-1]
     dev = q.device
@@ -277,14 +280,21 @@ def gdn_decode_step(q, k, v, beta, g, state, o=None, scale: float = 1.0, stream=
     _check("k", k, (N, H, dk), q.dtype, dev)
     _check("v", v, (N, H, dv), q.dtype, dev)
     _check("beta", beta, (N, H), torch.float32, dev, required=False)
-    _check("g", g, (N, H), torch.float32, dev, required=False)
+    vec = _check_gate(g, (N, H), dk, dev)
     _check("state", state, (N, H, dk, dv), torch.float32, dev)
+    odt, opts = _out_opts(o, out_dtype, d_skip, H, dv, dev, vec)
     if o is None:
-        o = torch.empty(N, H, dv, dtype=torch.float32, device=dev)
-    _check("o", o, (N, H, dv), torch.float32, dev)
-    st = lib.gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(state),
-                             _ptr(o), N, H, dk, dv, float(scale), _dtype_code(q), _stream(stream))
-    _raise("gdn_decode_step", st)
+        o = torch.empty(N, H, dv, dtype=odt, device=dev)
+    _check("o", o, (N, H, dv), odt, dev)
+    if opts is None:
+        st = lib.gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(state),
+                                 _ptr(o), N, H, dk, dv, float(scale), _dtype_code(q), _stream(stream))
+        _raise("gdn_decode_step", st)
+    else:
+        st = lib.gdn_decode_step_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(state),
+                                    _ptr(o), N, H, dk, dv, float(scale), _dtype_code(q), ctypes.byref(opts),
+                                    _stream(stream))
+        _raise("gdn_decode_step_ex", st)
     return o
 
 

@@ -159,19 +159,42 @@ gdn_status_t gdn_chunk_fwd_ex(const void *q, const void *k, const void *v, const
                       opts, cuda_stream);
 }
 
-gdn_status_t gdn_decode_step(const void *q, const void *k, const void *v, const float *beta,
-                             const float *g, float *state, float *o, int N, int H, int dk, int dv,
-                             float scale, gdn_dtype_t in_dtype, void *cuda_stream) {
+static gdn_status_t decode_impl(const void *q, const void *k, const void *v, const float *beta,
+                                const float *g, float *state, void *o, int N, int H, int dk, int dv,
+                                float scale, gdn_dtype_t in_dtype, const gdn_fwd_opts_t *opts,
+                                void *cuda_stream) {
     if (N < 1 || H < 1 || !isfinite(scale)) return GDN_ERR_INVALID_ARG;
     if (in_dtype != GDN_F32 && in_dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
     if (!q || !k || !v || !state || !o) return GDN_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(state) || !aligned16(o) ||
         !opt_aligned4(beta) || !opt_aligned4(g))
         return GDN_ERR_INVALID_ARG;
+    gdn::FwdOpts oo = kDefaultOut;
+    if (opts) {
+        if (opts->out_dtype != GDN_F32 && opts->out_dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+        if (opts->g_per_key != 0 && opts->g_per_key != 1) return GDN_ERR_INVALID_ARG;
+        if (!opt_aligned4(opts->d_skip)) return GDN_ERR_INVALID_ARG;
+        oo.bf16 = opts->out_dtype == GDN_BF16;
+        oo.dskip = opts->d_skip;
+        oo.gate_per_key = opts->g_per_key == 1 && g != nullptr;
+    }
     if (!head_dim_ok(dk) || !head_dim_ok(dv)) return GDN_ERR_UNSUPPORTED;
     if ((double)N * H > 2147483647.0) return GDN_ERR_INVALID_ARG;
-    return gdn::launch_decode(q, k, v, beta, g, state, o, N, H, dk, dv, scale, in_dtype,
+    return gdn::launch_decode(q, k, v, beta, g, state, o, N, H, dk, dv, scale, in_dtype, oo,
                               static_cast<cudaStream_t>(cuda_stream));
+}
+
+gdn_status_t gdn_decode_step(const void *q, const void *k, const void *v, const float *beta,
+                             const float *g, float *state, float *o, int N, int H, int dk, int dv,
+                             float scale, gdn_dtype_t in_dtype, void *cuda_stream) {
+    return decode_impl(q, k, v, beta, g, state, o, N, H, dk, dv, scale, in_dtype, nullptr, cuda_stream);
+}
+
+gdn_status_t gdn_decode_step_ex(const void *q, const void *k, const void *v, const float *beta,
+                                const float *g, float *state, void *o, int N, int H, int dk, int dv,
+                                float scale, gdn_dtype_t in_dtype, const gdn_fwd_opts_t *opts,
+                                void *cuda_stream) {
+    return decode_impl(q, k, v, beta, g, state, o, N, H, dk, dv, scale, in_dtype, opts, cuda_stream);
 }
 
 gdn_status_t gdn_sync_status(void *cuda_stream) {

@@ -64,7 +64,8 @@ __device__ __forceinline__ void st_global4(float *p, float4 v) {
 struct FwdOpts {
     bool bf16;            // o is bf16 (round to nearest even), else fp32
     const float *dskip;   // (H, dv) fp32, nullable (no skip term)
-    bool gate_per_key;    // g holds one log-decay per key coordinate ((rows, dk)), fp32 kernel only
+    bool gate_per_key;    // g holds one log-decay per key coordinate: (rows, dk) in prefill (fp32
+                          // chunk kernel), (N, H, dk) in decode
 };
 // The same, as a kernel argument: o, and for the D-skip term the input v (bf16 for the
 // tensor-core kernels; same (rows, dv) layout as o) with D.
@@ -115,6 +116,6 @@ gdn_status_t launch_simt_fwd(const void *q, const void *k, const void *v, const 
                              const int *cu, int B, int H, int L, int dk, int dv, int chunk,
                              float scale, gdn_dtype_t in_dtype, FwdOpts oo, cudaStream_t stream);
 gdn_status_t launch_decode(const void *q, const void *k, const void *v, const float *beta,
-                           const float *g, float *state, float *o, int N, int H, int dk, int dv,
-                           float scale, gdn_dtype_t in_dtype, cudaStream_t stream);
+                           const float *g, float *state, void *o, int N, int H, int dk, int dv,
+                           float scale, gdn_dtype_t in_dtype, FwdOpts oo, cudaStream_t stream);
 }  // namespace gdn

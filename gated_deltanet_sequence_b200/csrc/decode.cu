@@ -8,6 +8,10 @@
 //   o  = alpha sq + (q'.k) u    (= S_new^T q')
 //   S <- alpha S + k u^T        (written back from registers)
 // The state is read once and written once; everything else is O(d).
+// With a vector-valued gate (alpha_t[j] per key row j) the decayed state diag(alpha) S
+// replaces alpha S: sk = (diag(alpha) S)^T k, sq = (diag(alpha) S)^T q', o = sq + (q'.k) u,
+// S <- diag(alpha) S + k u^T. The options variant also takes the skip term o += D_h v
+// and a bf16 output.
 //
 // Layout: one CTA per (sequence, head); thread t owns 4 consecutive value
 // columns (float4) of RPT rows strided by the number of row groups, so every
@@ -19,11 +23,13 @@ namespace {
 
 constexpr int kDecThreads = 256;
 
-template <int DK, int DV, typename IT, bool DELTA>
+// OPT: the options variant (vector gate when vec, skip term when dskip, bf16 o when out_bf16)
+template <int DK, int DV, typename IT, bool DELTA, bool OPT>
 __global__ void __launch_bounds__(kDecThreads)
 decode_step_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT *__restrict__ v,
                    const float *__restrict__ beta, const float *__restrict__ g,
-                   float *__restrict__ state, float *__restrict__ o, float scale) {
+                   float *__restrict__ state, void *__restrict__ o, float scale, int H, int vec,
+                   int out_bf16, const float *__restrict__ dskip) {
     constexpr int CG = DV / 4;               // float4 column groups
     constexpr int RG = kDecThreads / CG;     // row groups
     constexpr int RPT = DK / RG;             // rows per thread
@@ -32,6 +38,8 @@ decode_step_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
     __shared__ float red_k[DELTA ? RG : 1][DV];
     __shared__ float red_q[RG][DV];
     __shared__ float s_qk;
+    __shared__ float s_a[OPT ? DK : 1];   // per-row decay (vector gate)
+    const bool vg = OPT && vec;
 
     const long head = blockIdx.x;
     const int tid = threadIdx.x;
@@ -48,7 +56,9 @@ decode_step_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
         s_q[i] = scale * ld_in(q + head * DK + i);
     }
     for (int i = tid; i < DV; i += kDecThreads) s_v[i] = ld_in(v + head * DV + i);
-    const float alpha = g ? expf(g[head]) : 1.f;
+    if (vg)
+        for (int i = tid; i < DK; i += kDecThreads) s_a[i] = g ? expf(g[head * DK + i]) : 1.f;
+    const float alpha = (g && !vg) ? expf(g[head]) : 1.f;
     const float bt = DELTA ? beta[head] : 0.f;
     __syncthreads();
 
@@ -57,7 +67,11 @@ decode_step_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
 #pragma unroll
     for (int i = 0; i < RPT; ++i) {
         const int j = rg + RG * i;
-        const float kj = s_k[j], qj = s_q[j];
+        float kj = s_k[j], qj = s_q[j];
+        if (vg) {           // read the decayed row alpha_j S[j, :]
+            kj *= s_a[j];
+            qj *= s_a[j];
+        }
         if (DELTA) {
             pk.x = fmaf(sreg[i].x, kj, pk.x); pk.y = fmaf(sreg[i].y, kj, pk.y);
             pk.z = fmaf(sreg[i].z, kj, pk.z); pk.w = fmaf(sreg[i].w, kj, pk.w);
@@ -90,7 +104,7 @@ decode_step_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
         const float vc = s_v[4 * cg + c];
-        u[c] = DELTA ? bt * (vc - alpha * sk[c]) : vc;
+        u[c] = DELTA ? bt * (vc - alpha * sk[c]) : vc;   // alpha = 1 with a vector gate
     }
     if (rg == 0) {
         const float qk = s_qk;
@@ -99,53 +113,80 @@ decode_step_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
         ov.y = fmaf(alpha, sq[1], qk * u[1]);
         ov.z = fmaf(alpha, sq[2], qk * u[2]);
         ov.w = fmaf(alpha, sq[3], qk * u[3]);
-        st_global4(o + head * DV + 4 * cg, ov);
+        if (!OPT) {
+            st_global4(static_cast<float *>(o) + head * DV + 4 * cg, ov);
+        } else {
+            if (dskip) {        // skip term D_h v (head = sequence * H + h)
+                const float *dh = dskip + (head % H) * DV + 4 * cg;
+                ov.x = fmaf(dh[0], s_v[4 * cg], ov.x);
+                ov.y = fmaf(dh[1], s_v[4 * cg + 1], ov.y);
+                ov.z = fmaf(dh[2], s_v[4 * cg + 2], ov.z);
+                ov.w = fmaf(dh[3], s_v[4 * cg + 3], ov.w);
+            }
+            if (out_bf16) {
+                __nv_bfloat16 *ob = static_cast<__nv_bfloat16 *>(o) + head * DV + 4 * cg;
+                ob[0] = __float2bfloat16_rn(ov.x);
+                ob[1] = __float2bfloat16_rn(ov.y);
+                ob[2] = __float2bfloat16_rn(ov.z);
+                ob[3] = __float2bfloat16_rn(ov.w);
+            } else {
+                st_global4(static_cast<float *>(o) + head * DV + 4 * cg, ov);
+            }
+        }
     }
 #pragma unroll
     for (int i = 0; i < RPT; ++i) {
         const int j = rg + RG * i;
         const float kj = s_k[j];
+        const float aj = vg ? s_a[j] : alpha;
         float4 s = sreg[i];
-        s.x = fmaf(alpha, s.x, kj * u[0]);
-        s.y = fmaf(alpha, s.y, kj * u[1]);
-        s.z = fmaf(alpha, s.z, kj * u[2]);
-        s.w = fmaf(alpha, s.w, kj * u[3]);
+        s.x = fmaf(aj, s.x, kj * u[0]);
+        s.y = fmaf(aj, s.y, kj * u[1]);
+        s.z = fmaf(aj, s.z, kj * u[2]);
+        s.w = fmaf(aj, s.w, kj * u[3]);
         st_global4(S + (long)j * DV + 4 * cg, s);
     }
 }
 
-template <int DK, int DV, typename IT>
+template <int DK, int DV, typename IT, bool OPT>
 gdn_status_t launch_dec_t(const void *q, const void *k, const void *v, const float *beta,
-                          const float *g, float *state, float *o, long NH, float scale,
+                          const float *g, float *state, void *o, long NH, int H, float scale, const FwdOpts &oo,
                           cudaStream_t stream) {
+    const int vec = oo.gate_per_key ? 1 : 0, ob = oo.bf16 ? 1 : 0;
     if (beta)
-        decode_step_kernel<DK, DV, IT, true><<<(unsigned)NH, kDecThreads, 0, stream>>>(
-            (const IT *)q, (const IT *)k, (const IT *)v, beta, g, state, o, scale);
+        decode_step_kernel<DK, DV, IT, true, OPT><<<(unsigned)NH, kDecThreads, 0, stream>>>(
+            (const IT *)q, (const IT *)k, (const IT *)v, beta, g, state, o, scale, H, vec, ob, oo.dskip);
     else
-        decode_step_kernel<DK, DV, IT, false><<<(unsigned)NH, kDecThreads, 0, stream>>>(
-            (const IT *)q, (const IT *)k, (const IT *)v, beta, g, state, o, scale);
+        decode_step_kernel<DK, DV, IT, false, OPT><<<(unsigned)NH, kDecThreads, 0, stream>>>(
+            (const IT *)q, (const IT *)k, (const IT *)v, beta, g, state, o, scale, H, vec, ob, oo.dskip);
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
-template <typename IT>
+template <typename IT, bool OPT>
 gdn_status_t launch_dec_dt(const void *q, const void *k, const void *v, const float *beta,
-                           const float *g, float *state, float *o, long NH, int dk, int dv,
-                           float scale, cudaStream_t stream) {
-    if (dk == 128 && dv == 128) return launch_dec_t<128, 128, IT>(q, k, v, beta, g, state, o, NH, scale, stream);
-    if (dk == 128 && dv == 64) return launch_dec_t<128, 64, IT>(q, k, v, beta, g, state, o, NH, scale, stream);
-    if (dk == 64 && dv == 128) return launch_dec_t<64, 128, IT>(q, k, v, beta, g, state, o, NH, scale, stream);
-    return launch_dec_t<64, 64, IT>(q, k, v, beta, g, state, o, NH, scale, stream);
+                           const float *g, float *state, void *o, long NH, int H, int dk, int dv,
+                           float scale, const FwdOpts &oo, cudaStream_t stream) {
+    if (dk == 128 && dv == 128)
+        return launch_dec_t<128, 128, IT, OPT>(q, k, v, beta, g, state, o, NH, H, scale, oo, stream);
+    if (dk == 128 && dv == 64)
+        return launch_dec_t<128, 64, IT, OPT>(q, k, v, beta, g, state, o, NH, H, scale, oo, stream);
+    if (dk == 64 && dv == 128)
+        return launch_dec_t<64, 128, IT, OPT>(q, k, v, beta, g, state, o, NH, H, scale, oo, stream);
+    return launch_dec_t<64, 64, IT, OPT>(q, k, v, beta, g, state, o, NH, H, scale, oo, stream);
 }
 
 }  // namespace
 
 gdn_status_t launch_decode(const void *q, const void *k, const void *v, const float *beta,
-                           const float *g, float *state, float *o, int N, int H, int dk, int dv,
-                           float scale, gdn_dtype_t in_dtype, cudaStream_t stream) {
+                           const float *g, float *state, void *o, int N, int H, int dk, int dv,
+                           float scale, gdn_dtype_t in_dtype, FwdOpts oo, cudaStream_t stream) {
     const long NH = (long)N * H;
+    const bool opt = oo.bf16 || oo.dskip || oo.gate_per_key;
     if (in_dtype == GDN_F32)
-        return launch_dec_dt<float>(q, k, v, beta, g, state, o, NH, dk, dv, scale, stream);
-    return launch_dec_dt<__nv_bfloat16>(q, k, v, beta, g, state, o, NH, dk, dv, scale, stream);
+        return opt ? launch_dec_dt<float, true>(q, k, v, beta, g, state, o, NH, H, dk, dv, scale, oo, stream)
+                   : launch_dec_dt<float, false>(q, k, v, beta, g, state, o, NH, H, dk, dv, scale, oo, stream);
+    return opt ? launch_dec_dt<__nv_bfloat16, true>(q, k, v, beta, g, state, o, NH, H, dk, dv, scale, oo, stream)
+               : launch_dec_dt<__nv_bfloat16, false>(q, k, v, beta, g, state, o, NH, H, dk, dv, scale, oo, stream);
 }
 
 }  // namespace gdn

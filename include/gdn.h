@@ -185,6 +185,18 @@ gdn_status_t gdn_decode_step(const void *q, const void *k, const void *v, const 
                              const float *g, float *state, float *o, int N, int H, int dk,
                              int dv, float scale, gdn_dtype_t in_dtype, void *cuda_stream);
 
+/*
+ * gdn_decode_step_ex — gdn_decode_step with the options of gdn_fwd_opts_t (opts NULL: the
+ * plain call). g_per_key = 1: g is (N, H, dk), row j of each state decays by
+ * exp(g[n, h, j]) (o = (diag(alpha) S)^T q' + (q'.k) u, S <- diag(alpha) S + k u^T);
+ * out_dtype GDN_BF16: o is bf16 (N, H, dv); d_skip (H, dv): o += d_skip[h] * v.
+ * Validation as for gdn_decode_step, plus the options' own rules.
+ */
+gdn_status_t gdn_decode_step_ex(const void *q, const void *k, const void *v, const float *beta,
+                                const float *g, float *state, void *o, int N, int H, int dk, int dv,
+                                float scale, gdn_dtype_t in_dtype, const gdn_fwd_opts_t *opts,
+                                void *cuda_stream);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 const char *gdn_status_str(gdn_status_t status);
 

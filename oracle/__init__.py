@@ -62,9 +62,10 @@ def _bind(path: str):
     lib.oracle_recurrent_fwd.argtypes = [P, P, P, P, P, P, P, P, l, l, l, l, d, i]
     lib.oracle_recurrent_fwd_vg.argtypes = [P, P, P, P, P, P, P, P, l, l, l, l, d, i]
     lib.oracle_decode_step.argtypes = [P, P, P, P, P, P, P, l, l, l, d, i]
+    lib.oracle_decode_step_vg.argtypes = [P, P, P, P, P, P, P, l, l, l, d, i]
     lib.oracle_chunked_fwd.argtypes = [P, P, P, P, P, P, P, P, l, l, l, l, l, d, i]
     lib.oracle_ut_transform.argtypes = [P, P, P, P, l, l]
-    for f in (lib.oracle_recurrent_fwd, lib.oracle_recurrent_fwd_vg, lib.oracle_decode_step,
+    for f in (lib.oracle_recurrent_fwd, lib.oracle_recurrent_fwd_vg, lib.oracle_decode_step, lib.oracle_decode_step_vg,
               lib.oracle_chunked_fwd, lib.oracle_ut_transform):
         f.restype = ctypes.c_int
     return lib
@@ -170,10 +171,12 @@ def recurrent_fwd_varlen(q, k, v, cu_seqlens, beta=None, g=None, s0=None, scale:
 
 
 def decode_step(q, k, v, beta, g, state: np.ndarray, scale: float = 1.0,
-                nthreads: Optional[int] = None, lib=None):
+                nthreads: Optional[int] = None, lib=None, d_skip=None):
     """One decode token for every head; ``state`` (fp64, (..., dk, dv)) is updated in place.
 
-    q, k: (..., dk); v: (..., dv); beta, g: (...) or None. Returns o (..., dv).
+    q, k: (..., H, dk); v: (..., H, dv); beta: (..., H) or None; g: (..., H) or (..., H, dk)
+    (vector-valued gate, as in :func:`recurrent_fwd`) or None; d_skip (H, dv) or None (the
+    skip term of :func:`recurrent_fwd`). Returns o (..., H, dv).
     """
     q, k, v, beta, g = map(_f64, (q, k, v, beta, g))
     assert state.dtype == np.float64 and state.flags.c_contiguous
@@ -181,10 +184,18 @@ def decode_step(q, k, v, beta, g, state: np.ndarray, scale: float = 1.0,
     dk, dv = state.shape[-2:]
     NH = int(np.prod(lead)) if lead else 1
     o = np.zeros(lead + (dv,), np.float64)
-    rc = (lib or _load()).oracle_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(state),
-                                    _ptr(o), NH, dk, dv, float(scale), nthreads or default_threads())
+    vector_gate = g is not None and g.ndim == q.ndim
+    lib_ = lib or _load()
+    fn = lib_.oracle_decode_step_vg if vector_gate else lib_.oracle_decode_step
+    rc = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(state), _ptr(o), NH, dk, dv, float(scale),
+            nthreads or default_threads())
     if rc:
         raise ValueError("oracle_decode_step: bad sizes")
+    if d_skip is not None:
+        D = _f64(d_skip)
+        if not lead or D.shape != (lead[-1], dv):
+            raise ValueError(f"d_skip: expected (H, dv), got {D.shape}")
+        o += D * v
     return o
 
 

@@ -241,6 +241,25 @@ int oracle_decode_step(const double *q, const double *k, const double *v,
     return 0;
 }
 
+/* Decode with vector-valued gates: g (NH, dk) or NULL. */
+static void dec_head_vg(void *vctx, long h, double *scratch)
+{
+    dec_ctx *c = (dec_ctx *)vctx;
+    token_step_vg(c->state + h * c->dk * c->dv, c->q + h * c->dk, c->k + h * c->dk,
+                  c->v + h * c->dv, c->beta ? c->beta + h : NULL, c->g ? c->g + h * c->dk : NULL,
+                  c->scale, c->dk, c->dv, c->o + h * c->dv, scratch, scratch + c->dv);
+}
+
+int oracle_decode_step_vg(const double *q, const double *k, const double *v,
+                          const double *beta, const double *g, double *state, double *o,
+                          long NH, long dk, long dv, double scale, int nthreads)
+{
+    if (NH < 0 || dk < 1 || dv < 1) return 1;
+    dec_ctx c = {q, k, v, beta, g, state, o, dk, dv, scale};
+    run_heads(dec_head_vg, &c, NH, dv + dk, nthreads);
+    return 0;
+}
+
 /* ------------------------------------------------------------------------- */
 /* Chunkwise re-derivation (test-only cross-check of the chunk algebra).
  *

@@ -27,8 +27,8 @@ def _declared_functions():
 def test_header_declares_the_boundary():
     names = _declared_functions()
     for want in ("lin_attn_chunk_fwd", "gdn_chunk_fwd", "lin_attn_chunk_fwd_varlen", "gdn_chunk_fwd_varlen",
-                 "lin_attn_chunk_fwd_ex", "gdn_chunk_fwd_ex", "gdn_decode_step", "gdn_status_str",
-                 "gdn_sync_status", "gdn_version"):
+                 "lin_attn_chunk_fwd_ex", "gdn_chunk_fwd_ex", "gdn_decode_step", "gdn_decode_step_ex",
+                 "gdn_status_str", "gdn_sync_status", "gdn_version"):
         assert want in names
 
 
@@ -182,3 +182,18 @@ def test_binding_checks_vector_gate_shape(lib):
     q = torch.zeros(1, 2, 4, 64)
     with pytest.raises(ValueError):     # (B, H, L) or (B, H, L, dk)
         lib.lin_attn_chunk_fwd(q, q, q, torch.zeros(1, 2, 4, 32))
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(g_per_key=3), 1), (dict(out_dtype=9), 1), (dict(d_skip=FAKE + 2), 1), (dict(N=0), 1), (dict(dk=32), 2),
+])
+def test_decode_ex_rejects_bad_arguments(lib, kw, want):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, beta=None, g=None, state=FAKE, o=FAKE, N=1, H=1, dk=64, dv=64, scale=1.0, dt=1,
+             out_dtype=0, d_skip=None, g_per_key=0)
+    a.update(kw)
+    P = ctypes.c_void_p
+    opts = lib.FwdOpts(a["out_dtype"], a["d_skip"], a["g_per_key"])
+    st = lib.lib.gdn_decode_step_ex(P(a["q"]), P(a["k"]), P(a["v"]), P(a["beta"]), P(a["g"]), P(a["state"]),
+                                    P(a["o"]), a["N"], a["H"], a["dk"], a["dv"], a["scale"], a["dt"],
+                                    ctypes.byref(opts), None)
+    assert st == want

@@ -112,3 +112,49 @@ def test_vector_gate_packed_batch(lib, delta):
     assert torch.all(o[:, used:] == 7.0)
     assert oracle.max_norm_err(o[:, :used].numpy(), o_ref[:, :used]) <= 1e-5
     assert oracle.max_norm_err(sf.cpu().numpy(), s_ref) <= 1e-5
+
+
+# ---------------------------------------------------------------- decode step options
+@pytest.mark.parametrize("delta", [True, False])
+@pytest.mark.parametrize("dk,dv,dtype", [(128, 128, torch.bfloat16), (64, 128, torch.float32)])
+def test_decode_vector_gate(lib, delta, dk, dv, dtype):
+    inp = W.make_decode_inputs(3, 5, dk, dv, 6, in_dtype=dtype, seed=98, device="cuda", delta=delta)
+    gv = W.make_gate_per_key((6, 3, 5), 1, dk, seed=99, g_low=-0.3)[..., 0, :].contiguous().cuda()
+    state = inp["state"].clone()
+    ref_state = inp["state"].cpu().double().numpy().copy()
+    for t in range(6):
+        b = inp["beta"][t] if delta else None
+        o = lib.gdn_decode_step(inp["q"][t], inp["k"][t], inp["v"][t], b, gv[t], state, scale=0.9)
+        assert lib.gdn_sync_status() == 0
+        o_ref = oracle.decode_step(inp["q"][t].cpu(), inp["k"][t].cpu(), inp["v"][t].cpu(),
+                                   None if b is None else b.cpu(), gv[t].cpu(), ref_state, scale=0.9)
+        assert _err(o.cpu(), o_ref) <= TOL[dtype], f"o t={t}: {_err(o.cpu(), o_ref):.3e}"
+    assert _err(state.cpu(), ref_state) <= TOL[dtype]
+
+
+def test_decode_skip_term_and_bf16_output(lib):
+    inp = W.make_decode_inputs(4, 3, 128, 128, 3, in_dtype=torch.bfloat16, seed=100, device="cuda")
+    D = W.make_dskip(3, 128, seed=101).cuda()
+    s32, sb = inp["state"].clone(), inp["state"].clone()
+    ref_state = inp["state"].cpu().double().numpy().copy()
+    for t in range(3):
+        args = (inp["q"][t], inp["k"][t], inp["v"][t], inp["beta"][t], inp["g"][t])
+        o32 = lib.gdn_decode_step(*args, s32, d_skip=D)
+        ob = lib.gdn_decode_step(*args, sb, d_skip=D, out_dtype=torch.bfloat16)
+        assert lib.gdn_sync_status() == 0
+        o_ref = oracle.decode_step(*(a.cpu() for a in args), ref_state, d_skip=D.cpu())
+        assert _err(o32.cpu(), o_ref) <= 2e-3
+        assert ob.dtype == torch.bfloat16 and torch.equal(ob, o32.to(torch.bfloat16))
+        assert torch.equal(sb, s32)
+    assert _err(s32.cpu(), ref_state) <= 2e-3
+
+
+def test_decode_equal_coordinates_match_scalar_gate(lib):
+    inp = W.make_decode_inputs(2, 4, 64, 64, 3, in_dtype=torch.float32, seed=102, device="cuda")
+    sa, sv = inp["state"].clone(), inp["state"].clone()
+    for t in range(3):
+        args = (inp["q"][t], inp["k"][t], inp["v"][t], inp["beta"][t])
+        oa = lib.gdn_decode_step(*args, inp["g"][t], sa)
+        ov = lib.gdn_decode_step(*args, inp["g"][t][..., None].expand(2, 4, 64).contiguous(), sv)
+        assert _err(ov.cpu(), oa.cpu().double().numpy()) <= 1e-6
+    assert _err(sv.cpu(), sa.cpu().double().numpy()) <= 1e-6

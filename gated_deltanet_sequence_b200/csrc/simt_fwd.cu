@@ -20,6 +20,9 @@
 // T diag(beta) (K o exp(G)), the inter-chunk output uses Q o exp(G), and the state
 // update uses k_s o exp(G_n - G_s) with row j of S scaled by exp(G_n[j]). Every decay
 // factor is one exp of a difference of cumulative sums, so no decay strength overflows.
+// Chunks whose cumulative log-decays all lie in [-60, 60] take the factored form
+// exp(G_r - G_s) = exp(G_r) exp(-G_s) (both factors far inside fp32 range): Q, K and
+// beta-free W are pre-scaled per element and the masks become plain dot products.
 #include "common.cuh"
 #include "tc_kernels.cuh"
 
@@ -94,13 +97,22 @@ simt_chunk_fwd_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const 
             const int r = i / kDvs, c = i % kDvs;
             sm.V[i] = ld_in(vh + (long)(t0 + r) * dv + c0 + c);
         }
-        if (VEC && tid >= kSimtThreads - DK) {
-            // per key coordinate j: inclusive within-chunk cumulative sum of g[:, j]
-            const int j = tid - (kSimtThreads - DK);
-            float carry = 0.f;
-            for (int r = 0; r < n; ++r) {
-                carry += bh_gv ? bh_gv[(long)(t0 + r) * DK + j] : 0.f;
-                sm.GV[r * KP + j] = carry;
+        int wide = 0;   // a cumulative log-decay of this chunk is outside [-60, 60]
+        if (VEC) {
+            // the chunk's log-decays (n x DK, coalesced), then per key coordinate j the
+            // inclusive within-chunk cumulative sum of g[:, j], in place
+            for (int i = tid; i < n * DK; i += kSimtThreads) {
+                const int r = i / DK, j = i % DK;
+                sm.GV[r * KP + j] = bh_gv ? bh_gv[(long)(t0 + r) * DK + j] : 0.f;
+            }
+            __syncthreads();
+            if (tid < DK) {
+                float carry = 0.f;
+                for (int r = 0; r < n; ++r) {
+                    carry += sm.GV[r * KP + tid];
+                    sm.GV[r * KP + tid] = carry;
+                    wide |= !(fabsf(carry) <= 60.f);
+                }
             }
         }
         if (!VEC && tid < 32) {
@@ -120,12 +132,32 @@ simt_chunk_fwd_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const 
             const int r = tid - 64;
             if (r < n) sm.bt[r] = bh_beta[t0 + r];
         }
-        __syncthreads();
+        const bool direct = VEC && __syncthreads_or(wide);   // VEC: direct exp per decay factor
+        if (!VEC) __syncthreads();
+        if (VEC && !direct) {
+            // factored decays: Q <- Q o exp(G), K <- K o exp(-G), W <- K o exp(G) (delta term)
+            for (int i = tid; i < n * DK; i += kSimtThreads) {
+                const int r = i / DK, j = i % DK;
+                const float gr = sm.GV[r * KP + j], kv = sm.K[r * KP + j];
+                const float e = expf(gr);
+                sm.Q[r * KP + j] *= e;
+                sm.K[r * KP + j] = kv * expf(-gr);
+                if (DELTA) sm.W[r * KP + j] = kv * e;
+            }
+            __syncthreads();
+        }
         // ---- Gram products with the decay mask ---------------------------------
         for (int i = tid; i < n * n; i += kSimtThreads) {
             const int r = i / n, s = i % n;
             float p = 0.f, a = 0.f;
-            if (s <= r && VEC) {
+            if (s <= r && VEC && !direct) {
+#pragma unroll 8
+                for (int j = 0; j < DK; ++j) {
+                    p = fmaf(sm.Q[r * KP + j], sm.K[s * KP + j], p);
+                    if (DELTA) a = fmaf(sm.W[r * KP + j], sm.K[s * KP + j], a);
+                }
+                if (DELTA) a = (s < r) ? sm.bt[r] * a : 0.f;
+            } else if (s <= r && VEC) {
 #pragma unroll 4
                 for (int j = 0; j < DK; ++j) {
                     const float dec = expf(sm.GV[r * KP + j] - sm.GV[s * KP + j]);
@@ -164,8 +196,9 @@ simt_chunk_fwd_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const 
                 // thread per key column j: W[:, j] = T (beta o exp(G[:, j]) o K[:, j]), formed
                 // in place from the last row up (row r reads rows s <= r only)
                 for (int j = tid; j < DK; j += kSimtThreads) {
-                    for (int s = 0; s < n; ++s)
-                        sm.W[s * KP + j] = sm.bt[s] * expf(sm.GV[s * KP + j]) * sm.K[s * KP + j];
+                    for (int s = 0; s < n; ++s)   // factored chunks: W already holds K o exp(G)
+                        sm.W[s * KP + j] = sm.bt[s] * (direct ? expf(sm.GV[s * KP + j]) * sm.K[s * KP + j]
+                                                              : sm.W[s * KP + j]);
                     for (int r = n - 1; r >= 0; --r) {
                         float w = 0.f;
                         for (int s = 0; s <= r; ++s) w = fmaf(sm.T[r * CP + s], sm.W[s * KP + j], w);
@@ -201,11 +234,16 @@ simt_chunk_fwd_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const 
         const float *Ut = DELTA ? sm.U : sm.V;
         if (VEC) {
             // the raw tiles are no longer read: Q <- Q o exp(G), K <- K o exp(G_n - G)
+            // (factored chunks: Q is already scaled and K holds K o exp(-G))
             for (int i = tid; i < n * DK; i += kSimtThreads) {
                 const int r = i / DK, j = i % DK;
-                const float gr = sm.GV[r * KP + j];
-                sm.Q[r * KP + j] *= expf(gr);
-                sm.K[r * KP + j] *= expf(sm.GV[(n - 1) * KP + j] - gr);
+                const float gr = sm.GV[r * KP + j], gn = sm.GV[(n - 1) * KP + j];
+                if (direct) {
+                    sm.Q[r * KP + j] *= expf(gr);
+                    sm.K[r * KP + j] *= expf(gn - gr);
+                } else {
+                    sm.K[r * KP + j] *= expf(gn);
+                }
             }
             __syncthreads();
         }

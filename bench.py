@@ -47,6 +47,9 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+FP32_CLOCK_GHZ = 1.965   # B200 max SM clock (clocks.max.sm 1965 MHz)
+
+
 def flops_per_head_token(mode: str, dk: int, dv: int, C: int) -> float:
     """Algorithmic FLOPs per head-token of the chunk form (dense tiles, T solve excluded):
     GDN  2C(3dk + 2dv) + 6 dk dv  (Gram [K;Q]K^T, W, U, [W;Q]S, P Ut, K~^T Ut)
@@ -328,7 +331,15 @@ def measure_rows(gdn, peaks, peak_src, args):
     ms = timed(fn, max(3, args.steps // 6), 2)
     nb = prefill_bytes(w.B, w.H, w.L, w.dk, w.dv, 2, True, False, False, True) + w.B * w.H * w.L * w.dk * 4
     row = _row(w, ms, nb, fl, peaks, peak_src, "hbm", w.B * w.L)
-    row["path"] = "fp32 chunk kernel (CUDA cores; every decay factor an exp)"
+    row["path"] = "fp32 chunk kernel (CUDA cores)"
+    # fp32 CUDA-core arithmetic bounds this path: peak = SMs x 128 fp32 lanes x 2 FLOP x max SM clock
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    peak_f32 = sms * 128 * 2 * FP32_CLOCK_GHZ / 1e3
+    tf32 = fl / (ms * 1e-3) / 1e12
+    row["roofline"] = {"bound": "alu", "achieved": round(tf32, 2), "peak": round(peak_f32, 1), "unit": "TFLOP/s",
+                       "frac": round(tf32 / peak_f32, 4), "traffic": None,
+                       "peak_source": f"derived: {sms} SMs x 128 fp32 lanes x 2 FLOP x {FP32_CLOCK_GHZ} GHz",
+                       "algorithmic_flop_per_launch": fl}
     rows["gdn_prefill_vector_gate"] = row
     del inp, o, sf, gv
     # long-context Gated DeltaNet, 1 x 32 x 65536 x 128, S0 != 0
@@ -463,7 +474,8 @@ def run_profile(spec: str):
     """Run one kernel a few times on one case (for an ncu capture; prints nothing timed).
     spec: gdn[:B] (GDN bf16, B x 16 x 4096 x 128), la[:B] (plain LA, B x 16 x 4096 x 128),
     decode[:N] (N x 32 heads, 3 steps), gdn_long (1 x 32 x 65536), gdnh[:H[:L]] (1 x H x L,
-    the cluster form when 3 H fits the SM count)."""
+    the cluster form when 3 H fits the SM count), gdnvec[:B[:L]] (vector-valued gates, B x 16 x L,
+    the fp32 chunk kernel)."""
     from gated_deltanet_sequence_b200 import _lib as gdn
     kind, _, arg = spec.partition(":")
     torch.cuda.set_device(0)
@@ -489,6 +501,17 @@ def run_profile(spec: str):
         sf = torch.empty(1, H, 128, 128, device="cuda")
         for _ in range(2):
             gdn.gdn_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["g"], o=o, s0=inp["s0"], s_final=sf)
+    elif kind == "gdnvec":
+        # vector-valued gates (fp32 chunk kernel): B x 16 heads x L tokens, d = 128, bf16 inputs
+        B, _, L = arg.partition(":")
+        B, L = int(B or 1), int(L or 1024)
+        inp = W.make_prefill_inputs(B, 16, L, 128, 128, mode="gdn", in_dtype=torch.bfloat16,
+                                    seed=W.SEED_BASE + 7, device="cuda")
+        gv = W.make_gate_per_key((B, 16), L, 128, seed=W.SEED_BASE + 7, device="cuda")
+        o = torch.empty(B, 16, L, 128, device="cuda")
+        sf = torch.empty(B, 16, 128, 128, device="cuda")
+        for _ in range(2):
+            gdn.gdn_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["beta"], gv, o=o, s_final=sf)
     elif kind == "gdn_long":
         w = W.WORKLOADS[3]
         inp = W.make_workload_inputs(w, device="cuda")

@@ -29,7 +29,7 @@
 namespace gdn {
 namespace {
 
-constexpr int kSimtThreads = 256;
+constexpr int kSimtThreads = 1024;   // one CTA per SM (the tiles take 215 KB of shared memory): all warps in one block
 constexpr int kDvs = 32;      // value columns per CTA
 constexpr int kCmax = 64;     // largest supported chunk
 

@@ -143,3 +143,67 @@ def test_planted_mistake_is_caught(name, src_text, tmp_path):
     assert src_text.count(old) == 1, f"mutation site for {name} not unique"
     failed = _pins(_compile(src_text.replace(old, new), tmp_path, name))
     assert failed, f"planted mistake {name} passed every pin"
+
+
+# ------------------------------------------------------------- vector-valued gates
+VG_MUTANTS = {
+    "vg_log_alpha_sign": ("a[j] = gv ? exp(gv[j]) : 1.0", "a[j] = gv ? exp(-gv[j]) : 1.0"),
+    "vg_decay_on_value_columns": ("for (long c = 0; c < dv; ++c) S[j * dv + c] *= a[j];",
+                                  "for (long c = 0; c < dv; ++c) S[j * dv + c] *= a[c % dk];"),
+    "vg_read_before_decay": (
+        "    /* decay first: row j of the state by alpha[j] */\n"
+        "    for (long j = 0; j < dk; ++j)\n"
+        "        for (long c = 0; c < dv; ++c) S[j * dv + c] *= a[j];\n"
+        "    if (beta) {",
+        "    if (beta) {"),
+    "vg_blend_sign": ("sk[col] = (*beta) * (v[col] - rd);", "sk[col] = (*beta) * (v[col] + rd);"),
+}
+
+
+def _vg_pins(lib):
+    """The vector-gate pins of tests/test_oracle_vector_gate.py against ``lib``; names that fail."""
+    failed = []
+    rng = np.random.default_rng(3)
+    # equal coordinates reduce to the scalar gate (GDN, dk != dv)
+    L, dk, dv = 13, 6, 4
+    q, k, v = rng.standard_normal((L, dk)), rng.standard_normal((L, dk)), rng.standard_normal((L, dv))
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    beta = rng.uniform(0.2, 0.9, L)
+    g = rng.uniform(-0.4, 0.0, L)
+    o1, S1 = oracle.recurrent_fwd(q, k, v, beta, g, lib=lib)
+    o2, S2 = oracle.recurrent_fwd(q, k, v, beta, np.repeat(g[:, None], dk, 1), lib=lib)
+    if not (np.allclose(o1, o2, atol=1e-12) and np.allclose(S1, S2, atol=1e-12)):
+        failed.append("vg_equal_coordinates")
+    # brute-force transition products with per-coordinate decays
+    gv = rng.uniform(-0.6, 0.0, (L, dk))
+    S0 = rng.standard_normal((dk, dv))
+    o, S = oracle.recurrent_fwd(q, k, v, beta, gv, S0, lib=lib)
+    St = S0.copy()
+    ok = True
+    for t in range(L):
+        M = (np.eye(dk) - beta[t] * np.outer(k[t], k[t])) @ np.diag(np.exp(gv[t]))
+        St = M @ St + beta[t] * np.outer(k[t], v[t])
+        ok = ok and np.allclose(o[t], St.T @ q[t], atol=1e-10)
+    if not (ok and np.allclose(S, St, atol=1e-10)):
+        failed.append("vg_transition_products")
+    # a zeroed coordinate erases its key row only
+    kk = np.zeros((2, 3)); kk[0] = [1.0, 2.0, 0.5]
+    vv = np.zeros((2, 4)); vv[0] = [1.0, -1.0, 3.0, 2.0]
+    gz = np.zeros((2, 3)); gz[1, 0] = -np.inf
+    _, Sz = oracle.recurrent_fwd(np.zeros((2, 3)), kk, vv, None, gz, lib=lib)
+    want = np.outer(kk[0], vv[0]); want[0] = 0.0
+    if not np.array_equal(Sz, want):
+        failed.append("vg_key_rows")
+    return failed
+
+
+def test_unmodified_copy_passes_vector_gate_pins(src_text, tmp_path):
+    assert _vg_pins(_compile(src_text, tmp_path, "clean_vg")) == []
+
+
+@pytest.mark.parametrize("name", list(VG_MUTANTS))
+def test_planted_vector_gate_mistake_is_caught(name, src_text, tmp_path):
+    old, new = VG_MUTANTS[name]
+    assert src_text.count(old) == 1, f"mutation site for {name} not unique"
+    failed = _vg_pins(_compile(src_text.replace(old, new), tmp_path, name))
+    assert failed, f"planted mistake {name} passed every vector-gate pin"

@@ -8,14 +8,17 @@ fast-math), compiled here with gcc and called through ctypes.
 Functions (each cites the passages it follows in ``gdn_oracle.c``):
   recurrent_fwd  token-by-token recurrence, the definition of the operator (optionally
                  with Mamba's skip term o_t += D_h v_t, added here in numpy)
-  decode_step    one token for many independent heads, state in place
+  decode_step    one token for many independent heads, state in place (scalar or
+                 vector-valued gates, optional skip term)
   chunked_fwd    fp64 chunkwise re-derivation (UT/WY form) for invariance tests
   ut_transform   the per-chunk T = (I + A)^-1 factor
 
 Pins (tests/test_oracle_pins.py) tie these to what the pages fix: the masked
 parallel form, the positions 1-4 cumulative-sum example, the delta rule as one
 gradient step, exact key->value recall, the Householder reflection, brute-force
-transition products, the WY product form and chunk-size invariance.
+transition products, the WY product form and chunk-size invariance; the skip term and
+the vector-valued gates have their own (tests/test_oracle_dskip.py,
+tests/test_oracle_vector_gate.py).
 """
 from __future__ import annotations
 

@@ -157,6 +157,7 @@ VG_MUTANTS = {
         "    if (beta) {",
         "    if (beta) {"),
     "vg_blend_sign": ("sk[col] = (*beta) * (v[col] - rd);", "sk[col] = (*beta) * (v[col] + rd);"),
+    "vg_decode_head_index": ("c->g ? c->g + h * c->dk : NULL", "c->g ? c->g + h : NULL"),
 }
 
 
@@ -194,7 +195,31 @@ def _vg_pins(lib):
     want = np.outer(kk[0], vv[0]); want[0] = 0.0
     if not np.array_equal(Sz, want):
         failed.append("vg_key_rows")
+    # decode steps with vector-valued gates equal the recurrence over the same tokens
+    if not _decode_matches_prefill(lib, rng, vector_gate=True):
+        failed.append("vg_decode_steps")
     return failed
+
+
+def _decode_matches_prefill(lib, rng, vector_gate, d_skip=False, mod=oracle):
+    """L decode steps of ``mod.decode_step`` (oracle library ``lib``) from S0 against the
+    token recurrence of the unmodified oracle over the same tokens (several heads)."""
+    N, H, L, dk, dv = 2, 3, 7, 5, 4
+    q = rng.standard_normal((N, H, L, dk))
+    k = rng.standard_normal((N, H, L, dk))
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((N, H, L, dv))
+    beta = rng.uniform(0.1, 0.9, (N, H, L))
+    g = rng.uniform(-0.6, 0.0, (N, H, L, dk) if vector_gate else (N, H, L))
+    s0 = rng.standard_normal((N, H, dk, dv))
+    D = rng.standard_normal((H, dv)) if d_skip else None
+    o, S = oracle.recurrent_fwd(q, k, v, beta, g, s0, d_skip=D)
+    st = np.ascontiguousarray(s0.copy())
+    for t in range(L):
+        ot = mod.decode_step(q[:, :, t], k[:, :, t], v[:, :, t], beta[:, :, t], g[:, :, t], st, lib=lib, d_skip=D)
+        if not np.allclose(ot, o[:, :, t], rtol=0, atol=1e-10):
+            return False
+    return bool(np.allclose(st, S, rtol=0, atol=1e-10))
 
 
 def test_unmodified_copy_passes_vector_gate_pins(src_text, tmp_path):
@@ -207,3 +232,22 @@ def test_planted_vector_gate_mistake_is_caught(name, src_text, tmp_path):
     assert src_text.count(old) == 1, f"mutation site for {name} not unique"
     failed = _vg_pins(_compile(src_text.replace(old, new), tmp_path, name))
     assert failed, f"planted mistake {name} passed every vector-gate pin"
+
+
+# ------------------------------------------------------------- decode skip term (numpy side)
+def test_planted_decode_skip_mistake_is_caught(tmp_path):
+    # the decode skip term is numpy code in oracle/__init__.py: drop it in a copy of that
+    # module and check that the decode-vs-recurrence pin rejects the copy (and accepts the
+    # unmodified module)
+    import importlib.util
+    src = open(oracle.__file__).read()
+    old = "        o += D * v\n    return o"
+    assert src.count(old) == 1, "mutation site of the decode skip term not unique"
+    mod_path = tmp_path / "oracle_mut.py"
+    mod_path.write_text(src.replace(old, "    return o"))
+    spec = importlib.util.spec_from_file_location("oracle_mut", mod_path)
+    mut = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mut)
+    lib = oracle._load()
+    assert _decode_matches_prefill(lib, np.random.default_rng(5), vector_gate=False, d_skip=True)
+    assert not _decode_matches_prefill(lib, np.random.default_rng(5), vector_gate=False, d_skip=True, mod=mut)

@@ -103,3 +103,25 @@ def test_gate_shape_is_checked():
     q = _rand((2, 5, 3), rng)
     with pytest.raises(ValueError):
         oracle.recurrent_fwd(q, q, q, None, np.zeros((2, 5, 4)))
+
+
+@pytest.mark.parametrize("delta", [True, False])
+def test_decode_steps_with_vector_gate_and_skip_match_prefill(delta):
+    # the decode entry of the oracle (its own head indexing of g, (N, H, dk), and its own
+    # numpy skip term) against the pinned token recurrence over the same tokens: L decode
+    # steps from S0 give the prefill's o_t at every step and its final state
+    rng = np.random.default_rng(31)
+    N, H, L, dk, dv = 2, 3, 12, 6, 5
+    q, k = _rand((N, H, L, dk), rng), _rand((N, H, L, dk), rng, unit=True)
+    v = _rand((N, H, L, dv), rng)
+    beta = rng.uniform(0.1, 0.9, (N, H, L)) if delta else None
+    gv = rng.uniform(-0.6, 0.0, (N, H, L, dk))
+    s0 = 0.3 * _rand((N, H, dk, dv), rng)
+    D = rng.standard_normal((H, dv))
+    o, S = oracle.recurrent_fwd(q, k, v, beta, gv, s0, d_skip=D)
+    st = np.ascontiguousarray(s0.copy())
+    for t in range(L):
+        ot = oracle.decode_step(q[:, :, t], k[:, :, t], v[:, :, t], None if beta is None else beta[:, :, t],
+                                gv[:, :, t], st, d_skip=D)
+        np.testing.assert_allclose(ot, o[:, :, t], rtol=0, atol=1e-13 * np.abs(o).max())
+    np.testing.assert_allclose(st, S, rtol=0, atol=1e-13 * np.abs(S).max())

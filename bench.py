@@ -82,7 +82,7 @@ class ClockSampler:
     SW_THERMAL = 0x20
     SW_POWER = 0x4
 
-    def __init__(self, index: int, period_s: float = 0.005):
+    def __init__(self, index: int, period_s: float = 0.001):
         self.samples, self.reasons, self.max_mhz = [], 0, None
         self._stop = threading.Event()
         self._period = period_s
@@ -195,6 +195,14 @@ def aggregate_tokens_per_s(tokens_per_rank: int, world: int, ms_max: float) -> f
     return world * tokens_per_rank / (ms_max * 1e-3)
 
 
+def headline_config(world: int) -> dict:
+    """The ``config`` of the JSON line: the headline workload, identical in both arms."""
+    w = W.WORKLOADS[2]
+    return {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "dk": w.dk, "dv": w.dv, "chunk": w.chunk,
+            "global_batch": w.B * world, "seq_len": w.L, "parallelism": f"independent batches x{world}",
+            "l2": "inputs (403 MB) and outputs (277 MB) exceed the 126 MB L2"}
+
+
 def run_ours(args, rank, world, barrier, max_over_ranks):
     from gated_deltanet_sequence_b200 import _lib as gdn
     peaks, peak_src = load_peaks()
@@ -218,6 +226,13 @@ def run_ours(args, rank, world, barrier, max_over_ranks):
     with ClockSampler(dev_index) as clk:
         ms = timed(step, args.steps, 0, barrier)
     ms_max = max_over_ranks(ms)
+    # the same launch over a longer timed region (steadier clocks), reported beside the value
+    long_steps = 0 if args.quick else 200
+    stability = None
+    if long_steps:
+        with ClockSampler(dev_index) as clk_long:
+            ms_long = max_over_ranks(timed(step, long_steps, 0, barrier))
+        stability = {"launches": long_steps, "ms_per_launch": round(ms_long, 5), "clocks": clk_long.summary()}
     tokens = B * L
     value = aggregate_tokens_per_s(tokens, world, ms_max)
     flop = flops_per_head_token("gdn", dk, dv, C) * B * H * L
@@ -282,10 +297,8 @@ def run_ours(args, rank, world, barrier, max_over_ranks):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; q,k unit-norm, v~N(0,1), beta=sigmoid(N(0,1)), log-alpha~U(-0.05,0))",
-        "config": {"workload": w.name, "B": B, "H": H, "L": L, "dk": dk, "dv": dv, "chunk": C,
-                   "global_batch": B * world, "seq_len": L, "parallelism": f"independent batches x{world}",
-                   "l2": "inputs (403 MB) and outputs (277 MB) exceed the 126 MB L2"},
-        "roofline": roofline, "tensor": tensor, "clocks": clk.summary(),
+        "config": headline_config(world),
+        "roofline": roofline, "tensor": tensor, "clocks": clk.summary(), "long_region": stability,
         "e2e": e2e, "gpu_launches": args.steps, "head_tokens_per_s": round(value * H, 1),
         "rows": rows, "cpu_baseline": cpu,
     }
@@ -463,8 +476,7 @@ def run_reference(args, rank, world):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded; same generator and seed as the GPU arm)",
-            "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "dk": w.dk, "dv": w.dv,
-                       "chunk": w.chunk},
+            "config": headline_config(world),
             "cpu_baseline": cb,
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 

@@ -23,7 +23,7 @@ GDN_F32, GDN_BF16 = 0, 1
 
 EXPORTS = ("lin_attn_chunk_fwd", "gdn_chunk_fwd", "lin_attn_chunk_fwd_varlen", "gdn_chunk_fwd_varlen",
            "lin_attn_chunk_fwd_ex", "gdn_chunk_fwd_ex", "gdn_decode_step", "gdn_decode_step_ex",
-           "gdn_status_str", "gdn_sync_status", "gdn_version")
+           "gdn_status_str", "gdn_sync_status", "gdn_set_wait_limit_for_testing", "gdn_version")
 
 
 class FwdOpts(ctypes.Structure):
@@ -56,6 +56,8 @@ def _load() -> ctypes.CDLL:
     lib.gdn_status_str.restype = ctypes.c_char_p
     lib.gdn_sync_status.argtypes = [P]
     lib.gdn_version.argtypes = []
+    lib.gdn_set_wait_limit_for_testing.argtypes = [ctypes.c_longlong]
+    lib.gdn_set_wait_limit_for_testing.restype = None
     for f in (lib.lin_attn_chunk_fwd, lib.gdn_chunk_fwd, lib.lin_attn_chunk_fwd_varlen,
               lib.gdn_chunk_fwd_varlen, lib.lin_attn_chunk_fwd_ex, lib.gdn_chunk_fwd_ex,
               lib.gdn_decode_step, lib.gdn_decode_step_ex, lib.gdn_sync_status, lib.gdn_version):
@@ -299,8 +301,15 @@ def gdn_decode_step(q, k, v, beta, g, state, o=None, scale: float = 1.0, stream=
 
 
 def gdn_sync_status(stream=None) -> int:
-    """Synchronise the stream; return the library's status word (GDN_OK / GDN_ERR_TIMEOUT / ...)."""
+    """Synchronise the stream; report and clear one pending device-side condition
+    (GDN_ERR_INVALID_ARG first, then GDN_ERR_TIMEOUT; GDN_OK when none is pending)."""
     return lib.gdn_sync_status(_stream(stream))
+
+
+def gdn_set_wait_limit_for_testing(cycles: int) -> None:
+    """Tests of the failure path only: bounded-wait limit (clock cycles) of the tensor-core
+    kernels launched afterwards; cycles <= 0 restores the default (about 2 s)."""
+    lib.gdn_set_wait_limit_for_testing(int(cycles))
 
 
 def gdn_version() -> int:

@@ -197,13 +197,4 @@ gdn_status_t gdn_decode_step_ex(const void *q, const void *k, const void *v, con
     return decode_impl(q, k, v, beta, g, state, o, N, H, dk, dv, scale, in_dtype, opts, cuda_stream);
 }
 
-gdn_status_t gdn_sync_status(void *cuda_stream) {
-    cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
-    if (cudaStreamSynchronize(stream) != cudaSuccess) return GDN_ERR_CUDA;
-    unsigned err = 0u;
-    if (!gdn::read_and_clear_device_error(&err)) return GDN_ERR_CUDA;
-    if (err & gdn::kErrBadSeqlens) return GDN_ERR_INVALID_ARG;
-    return err ? GDN_ERR_TIMEOUT : GDN_OK;
-}
-
 }  // extern "C"

@@ -40,36 +40,9 @@
 // computed operand (T, P, W, S, Ut) is rounded to fp16, which keeps the rounding of
 // the chunk intermediates ~8x below what bf16 operands give. Shared-memory
 // operands use the 128-byte swizzled canonical layouts.
-#include <mutex>
-
 #include "tc_gdn_parts.cuh"
 
 namespace gdn {
-
-// Device-side error word (static storage in the library image, one per device).
-__device__ unsigned g_device_error = 0u;
-
-unsigned *device_error_word() {
-    static std::mutex mu;
-    static unsigned *addr[64] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
-        addr[dev] = static_cast<unsigned *>(p);
-    }
-    return addr[dev];
-}
-
-bool read_and_clear_device_error(unsigned *err) {
-    const unsigned zero = 0u;
-    if (cudaMemcpyFromSymbol(err, g_device_error, sizeof(unsigned)) != cudaSuccess) return false;
-    if (*err != 0u && cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess)
-        return false;
-    return true;
-}
 
 namespace {
 using namespace ptx;
@@ -160,7 +133,6 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kNumBars);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
-    int *abort_s = abort_flag + 1, *abort_p = abort_flag + 2;   // state / prep group verdicts
     const Ctl ctl{bars, abort_flag, err_word, wait_limit};
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -173,7 +145,7 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
     if (tid == 0) {
         for (int b = 0; b < kNumBars; ++b) mbar_init(&bars[b], 1);
-        abort_flag[0] = abort_flag[1] = abort_flag[2] = 0;
+        abort_flag[0] = 0;
         fence_mbar_init();
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
@@ -334,7 +306,7 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             // S(c) complete, and this chunk's gate values
             if (!ctl.group_wait_all({c >= 1 ? B_CDONE + ((c - 1) & 1) : -1, B_GATE + s},
                                     {static_cast<uint32_t>((c - 1) >> 1) & 1u, static_cast<uint32_t>(c >> 1) & 1u},
-                                    kBarS, abort_s, lead))
+                                    kBarS, lead))
                 break;
             tc_fence_after();
             // ---- S row j -> fp16 MN-major operand; S <- gamma_last S (ahead of the update)
@@ -360,7 +332,7 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             if (lead) mbar_arrive(&bars[B_SRDY]);
             // ---- W operand of this chunk (its V slot is consumed) and K <- diag(d) K
             //      (K's last reader before the state update was W/U)
-            if (!ctl.group_wait(B_WU, c & 1, kBarS, abort_s, lead)) break;
+            if (!ctl.group_wait(B_WU, c & 1, kBarS, lead)) break;
             tc_fence_after();
             store_w_row(trow + TM_W, sb + s * kStageBytes + ST_W, j);
             if (GATED) {
@@ -391,7 +363,7 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 done = c;
             }
             // ---- Ut^T row v -> Ut operand (K-major, rows v)
-            if (!ctl.group_wait(B_ADONE, c & 1, kBarS, abort_s, lead)) break;
+            if (!ctl.group_wait(B_ADONE, c & 1, kBarS, lead)) break;
             tc_fence_after();
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
@@ -408,7 +380,7 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         // ---- last output tile and the final state
         if (nchunks > 0 && done == nchunks - 1) {
             const int cp = nchunks - 1;
-            if (ctl.group_wait(B_CDONE + (cp & 1), (cp >> 1) & 1, kBarS, abort_s, lead)) {
+            if (ctl.group_wait(B_CDONE + (cp & 1), (cp >> 1) & 1, kBarS, lead)) {
                 tc_fence_after();
                 store_out_col<OPTS>(trow + TM_O + (cp & 1) * 64, out, (row0 + static_cast<size_t>(cp) * kC) * kD + j,
                               L - cp * kC, dj);
@@ -448,7 +420,7 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             if (!ctl.group_wait_all({c >= 2 ? B_CDONE + s : -1, B_GATEP + s, B_FULL + s, B_GRAM},
                                     {static_cast<uint32_t>((c - 2) >> 1) & 1u, static_cast<uint32_t>(c >> 1) & 1u,
                                      static_cast<uint32_t>(c >> 1) & 1u, static_cast<uint32_t>(c) & 1u},
-                                    kBarP, abort_p, p == 0, kNP))
+                                    kBarP, p == 0, kNP))
                 break;
             tc_fence_after();
             const bool fast = !GATED || reinterpret_cast<const int *>(vec)[V_FAST] != 0;
@@ -509,6 +481,7 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 }
             }
             named_bar(kBarP, kNP);                           // A^T complete
+            bool solve_ok = true;                            // the solve warps' wait for W/U (c-1)
             if (w8 < 4) {
                 // ---- UT solve on warps 8-11. Blocks of T are kept in fp32 (Tf) for the
                 //      products that follow and copied, once final, into the fp16 factors
@@ -565,10 +538,9 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     }
                 }
                 // T1/T2 of chunk c-1 must have been read by its W/U before they are overwritten
-                bool ok = true;
-                if (c >= 1) ok = ctl.group_wait(B_WU, (c - 1) & 1, 3, abort_p, p == 0, 128);
+                if (c >= 1) solve_ok = ctl.group_wait(B_WU, (c - 1) & 1, 3, p == 0, 128);
                 else asm volatile("bar.sync 3, 128;" ::: "memory");
-                if (ok) {
+                if (solve_ok) {
                     emit(bi, bi);
                     float *Rw = reinterpret_cast<float *>(smem + OFF_R);
                     // level 1 (warps 0, 1): T_10 = -D_1 (A_10 D_0), T_32 = -D_3 (A_32 D_2)
@@ -666,8 +638,7 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 }
             }
             fence_proxy_async();
-            named_bar(kBarP, kNP);
-            if (*reinterpret_cast<volatile int *>(abort_p)) break;   // the solve warps gave up waiting
+            if (named_bar_any(kBarP, kNP, !solve_ok)) break;   // the solve warps gave up waiting
             if (p == 0) {
                 mbar_arrive(&bars[B_TRDY + s]);
                 mbar_arrive(&bars[B_PREP + s]);
@@ -781,16 +752,11 @@ gdn_status_t launch_gdn_t(const CUtensorMap &mq, const CUtensorMap &mk, const CU
                           const float *g, const OutArgs &out, const float *s0, float *s_final, const int *cu,
                           int nctas, int H, int L, float scale, cudaStream_t stream) {
     auto kern = tc_gdn_kernel<GATED, OPTS>;
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [&] {
-        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
-    });
-    if (attr_err != cudaSuccess) return GDN_ERR_CUDA;
+    if (!ensure_smem_limit(reinterpret_cast<const void *>(kern), kSmemAlloc)) return GDN_ERR_CUDA;
     unsigned *err = device_error_word();
     if (!err) return GDN_ERR_CUDA;
     kern<<<nctas, kThreads, kSmemAlloc, stream>>>(mq, mk, mv, beta, g, out, s0, s_final, cu, H, L, scale,
-                                                  kWaitLimitCycles, err);
+                                                  wait_limit_cycles(), err);
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 

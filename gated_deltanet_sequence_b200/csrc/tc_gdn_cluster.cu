@@ -128,7 +128,6 @@ tc_gdn_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kNumBars);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
-    int *abort_s = abort_flag + 1, *abort_p = abort_flag + 2;   // group verdicts
     const Ctl ctl{bars, abort_flag, err_word, wait_limit};
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -143,7 +142,7 @@ tc_gdn_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
     if (tid == 0) {
         for (int b = 0; b < kNumBars; ++b) mbar_init(&bars[b], 1);
-        abort_flag[0] = abort_flag[1] = abort_flag[2] = 0;
+        abort_flag[0] = 0;
         fence_mbar_init();
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
@@ -304,7 +303,7 @@ tc_gdn_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 // S(c) complete (state-update UMMAs of chunk c-1), and this chunk's gate values
                 if (!ctl.group_wait_all({c >= 1 ? static_cast<int>(B_SDONE) : -1, B_SLOT + c % kSlots},
                                         {static_cast<uint32_t>(c - 1) & 1u, static_cast<uint32_t>(c / kSlots) & 1u},
-                                        kBarS, abort_s, lead, 128, 2u))
+                                        kBarS, lead, 128, 2u))
                     break;
                 tc_fence_after();
                 // ---- S row j -> fp16 MN-major operand; S <- gamma_last S (ahead of the update)
@@ -332,7 +331,7 @@ tc_gdn_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 named_bar(kBarS, 128);
                 if (lead) mbar_arrive(&bars[B_SRDY]);
                 // ---- W operand of this chunk (its V slot is consumed); the converter scales K
-                if (!ctl.group_wait(B_WU, c & 1, kBarS, abort_s, lead)) break;
+                if (!ctl.group_wait(B_WU, c & 1, kBarS, lead)) break;
                 tc_fence_after();
                 {
                     float w[64];
@@ -352,7 +351,7 @@ tc_gdn_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 //      ((c - 1) >> 1)-th slot reuse)
                 if (c >= 1) {
                     const int cp = c - 1;
-                    if (!ctl.group_wait(B_CDONE + (cp & 1), (cp >> 1) & 1, kBarS, abort_s, lead)) break;
+                    if (!ctl.group_wait(B_CDONE + (cp & 1), (cp >> 1) & 1, kBarS, lead)) break;
                     if (c + 2 < nchunks && lead)
                         mbar_arrive_cluster(mapa_shared(smem_u32(&bars[B_SFREE + (((c - 1) >> 1) & 1)]), 1 + (c & 1)));
                     tc_fence_after();
@@ -360,7 +359,7 @@ tc_gdn_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     done = c;
                 }
                 // ---- Ut^T row v -> Ut operand (K-major, rows v)
-                if (!ctl.group_wait(B_ADONE, c & 1, kBarS, abort_s, lead)) break;
+                if (!ctl.group_wait(B_ADONE, c & 1, kBarS, lead)) break;
                 tc_fence_after();
                 {
                     float u[64];
@@ -376,7 +375,7 @@ tc_gdn_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             // ---- last output tile and the final state
             if (nchunks > 0 && done == nchunks - 1) {
                 const int cp = nchunks - 1;
-                if (ctl.group_wait(B_CDONE + (cp & 1), (cp >> 1) & 1, kBarS, abort_s, lead)) {
+                if (ctl.group_wait(B_CDONE + (cp & 1), (cp >> 1) & 1, kBarS, lead)) {
                     tc_fence_after();
                     store_out_col<OPTS>(trow + TM_O + (cp & 1) * 64, out, (row0 + static_cast<size_t>(cp) * kC) * kD + j,
                                   L - cp * kC, dj);
@@ -408,7 +407,7 @@ tc_gdn_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 const float *vec = reinterpret_cast<const float *>(smem + C_SLOT + (c % kSlots) * kSlotBytes + SL_VEC);
                 if (!ctl.group_wait_all({B_FULL + s, B_SLOT + c % kSlots},
                                         {static_cast<uint32_t>(c >> 1) & 1u, static_cast<uint32_t>(c / kSlots) & 1u},
-                                        kBarC, abort_p, lead, 128, 2u))
+                                        kBarC, lead, 128, 2u))
                     break;
                 // K and V: 2048 chunks of 16 B at [0,8K) [16K,24K) [32K,48K)
 #pragma unroll
@@ -456,7 +455,7 @@ tc_gdn_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 if (lead) mbar_arrive(&bars[B_CONV + s]);
                 // K <- diag(d) K for the state update, once W/U (its last reader) is done
                 if (GATED) {
-                    if (!ctl.group_wait(B_WU, c & 1, kBarC, abort_p, lead)) break;
+                    if (!ctl.group_wait(B_WU, c & 1, kBarC, lead)) break;
                     uint4 x[8];
                     __half2 f[8];
 #pragma unroll
@@ -608,7 +607,7 @@ tc_gdn_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                                          i >= i_reuse ? B_SFREE + ((i - i_reuse) & 1) : -1},
                                         {static_cast<uint32_t>(i >> 1) & 1u, static_cast<uint32_t>(i) & 1u,
                                          static_cast<uint32_t>((i - i_reuse) >> 1) & 1u},
-                                        kBarP, abort_p, p == 0, kNP, 4u))
+                                        kBarP, p == 0, kNP, 4u))
                     break;
                 // gate values -> slot (96 chunks of 16 B)
                 if (p < 96) {
@@ -786,7 +785,6 @@ tc_gdn_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 // hand the slot to the chain CTA
                 fence_proxy_async_cluster();
                 named_bar(kBarP, kNP);
-                if (*reinterpret_cast<volatile int *>(abort_p)) break;
                 if (p == 0) {
                     mbar_arrive_cluster(mapa_shared(smem_u32(&bars[B_SLOT + c % kSlots]), 0));
                     mbar_arrive(&bars[B_PDONE + s]);
@@ -811,12 +809,7 @@ gdn_status_t launch_cl_t(const CUtensorMap &mq, const CUtensorMap &mk, const CUt
                          const float *g, const OutArgs &out, const float *s0, float *s_final, const int *cu,
                          int nctas, int H, int L, float scale, cudaStream_t stream) {
     auto kern = tc_gdn_cl_kernel<GATED, OPTS>;
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [&] {
-        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
-    });
-    if (attr_err != cudaSuccess) return GDN_ERR_CUDA;
+    if (!ensure_smem_limit(reinterpret_cast<const void *>(kern), kSmemAlloc)) return GDN_ERR_CUDA;
     unsigned *err = device_error_word();
     if (!err) return GDN_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
@@ -831,7 +824,7 @@ gdn_status_t launch_cl_t(const CUtensorMap &mq, const CUtensorMap &mk, const CUt
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const long long limit = kWaitLimitCycles;
+    const long long limit = wait_limit_cycles();
     return cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, beta, g, out, s0, s_final, cu, H, L, scale, limit, err) ==
                    cudaSuccess
                ? GDN_OK

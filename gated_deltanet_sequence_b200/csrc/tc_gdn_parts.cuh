@@ -1,92 +1,17 @@
 // Device helpers shared by the Gated DeltaNet tensor-core kernels (one-CTA and
-// cluster forms): bounded mbarrier waits with a group-uniform abort protocol, TMEM
-// row loads, fp16 operand stores in the 128-byte swizzled layout, the output and W
-// epilogues, and the warp-level tf32 block products of the UT solve.
+// cluster forms): TMEM row loads, fp16 operand stores in the 128-byte swizzled
+// layout, the output and W epilogues, and the warp-level tf32 block products of the UT
+// solve. The bounded waits and the abort protocol are in tc_ctl.cuh.
 #pragma once
-#include "tc_kernels.cuh"
-#include "tc_ptx.cuh"
+#include "tc_ctl.cuh"
 
 namespace gdn {
 namespace tcgdn {
 using namespace ptx;
+using gdn::Ctl;
 
 constexpr int kC = 64;           // chunk rows
 constexpr int kD = 128;          // dk = dv
-
-struct Ctl {
-    uint64_t *bar;
-    int *abort_flag;     // CTA-wide: set by the first wait that gives up
-    unsigned *err;
-    long long limit;
-    // Bounded wait. After any timeout in the CTA every later wait fails at once; a
-    // role whose wait fails stops issuing (no further arrivals, copies or UMMAs)
-    // and leaves its loop, so the CTA winds down within a few wait limits.
-    __device__ __forceinline__ bool wait(int b, uint32_t parity) const {
-        if (*reinterpret_cast<volatile int *>(abort_flag)) return false;
-        if (mbar_wait(&bar[b], parity, limit)) return true;
-        atomicOr(err, kErrWaitTimeout);
-        *reinterpret_cast<volatile int *>(abort_flag) = 1;
-        return false;
-    }
-    // Bounded wait with a cluster-scope acquire, for phases completed by arrivals of
-    // another CTA of the cluster (its shared-memory writes become visible here).
-    __device__ __forceinline__ bool wait_cluster(int b, uint32_t parity) const {
-        if (*reinterpret_cast<volatile int *>(abort_flag)) return false;
-        if (mbar_wait_cluster(&bar[b], parity, limit)) return true;
-        atomicOr(err, kErrWaitTimeout);
-        *reinterpret_cast<volatile int *>(abort_flag) = 1;
-        return false;
-    }
-    __device__ __forceinline__ bool group_wait_cluster(int b, uint32_t parity, int bar_id, int *group_abort,
-                                                       bool leader, int nthreads = 128) const {
-        if (leader && !wait_cluster(b, parity)) *reinterpret_cast<volatile int *>(group_abort) = 1;
-        named_bar(bar_id, nthreads);
-        return *reinterpret_cast<volatile int *>(group_abort) == 0;
-    }
-    // Bounded wait that sleeps between polls, for roles off the critical path (their
-    // polling would otherwise take issue slots from the warps they share a scheduler with).
-    __device__ __forceinline__ bool wait_lazy(int b, uint32_t parity) const {
-        if (*reinterpret_cast<volatile int *>(abort_flag)) return false;
-        const uint32_t a = smem_u32(&bar[b]);
-        if (mbar_try_wait(a, parity)) return true;
-        const long long t0 = clock64();
-        do {
-            __nanosleep(100);
-            if (mbar_try_wait(a, parity)) return true;
-        } while (clock64() - t0 <= limit);
-        atomicOr(err, kErrWaitTimeout);
-        *reinterpret_cast<volatile int *>(abort_flag) = 1;
-        return false;
-    }
-    // Group-uniform wait on several phases with one barrier: the leader polls each in
-    // turn (entries with b < 0 are skipped; bit i of cluster_mask selects the cluster-scope
-    // acquire for entry i), then the group meets once.
-    template <int N>
-    __device__ __forceinline__ bool group_wait_all(const int (&b)[N], const uint32_t (&parity)[N], int bar_id,
-                                                   int *group_abort, bool leader, int nthreads = 128,
-                                                   unsigned cluster_mask = 0u) const {
-        if (leader) {
-            bool ok = true;
-#pragma unroll
-            for (int i = 0; i < N; ++i)
-                if (ok && b[i] >= 0) ok = ((cluster_mask >> i) & 1u) ? wait_cluster(b[i], parity[i]) : wait(b[i], parity[i]);
-            if (!ok) *reinterpret_cast<volatile int *>(group_abort) = 1;
-        }
-        named_bar(bar_id, nthreads);
-        return *reinterpret_cast<volatile int *>(group_abort) == 0;
-    }
-    // bounded wait that ignores the abort flag (final drain of in-flight operations)
-    __device__ __forceinline__ void drain(int b, uint32_t parity) const { mbar_wait(&bar[b], parity, limit); }
-    // Group-uniform wait for a group of warps: the leader polls, the group meets on
-    // its named barrier and every thread reads the same verdict (a sticky flag), so
-    // the whole group leaves its loop together.
-    __device__ __forceinline__ bool group_wait(int b, uint32_t parity, int bar_id, int *group_abort,
-                                               bool leader, int nthreads = 128) const {
-        if (leader && !wait(b, parity)) *reinterpret_cast<volatile int *>(group_abort) = 1;
-        named_bar(bar_id, nthreads);
-        return *reinterpret_cast<volatile int *>(group_abort) == 0;
-    }
-};
 
 template <int N>
 __device__ __forceinline__ void ld_cols(uint32_t taddr, float (&v)[N]) {

@@ -23,13 +23,24 @@ bool tc_gdn_cluster_fits(int nctas);
 gdn_status_t launch_tc_la(const void *q, const void *k, const void *v, const float *g, void *o,
                           const float *s0, float *s_final, const int *cu, int B, int H, int L,
                           float scale, FwdOpts oo, cudaStream_t stream);
-// Reads and clears the device-side error word of the current device.
-bool read_and_clear_device_error(unsigned *err);
+// Takes one condition out of the device-side error word of the current device, on
+// `stream` (a one-thread kernel clears only the bit it reports, atomically, so a bit
+// that another kernel sets meanwhile is kept for the next call): *err receives
+// kErrBadSeqlens if that bit was set, else kErrWaitTimeout if that one was, else 0.
+bool take_device_error(cudaStream_t stream, unsigned *err);
 // Device address of that word on the current device (looked up once per device),
 // handed to kernels that may record a bounded-wait timeout; nullptr on failure.
 unsigned *device_error_word();
-// Bounded-wait limit handed to the tensor-core kernels (clock cycles, ~2 s at 2 GHz).
+// Bounded-wait limit of the tensor-core kernels (clock cycles, ~2 s at 2 GHz), and the
+// limit of their final drains of copies and UMMAs already issued (always this value).
 constexpr long long kWaitLimitCycles = 4000000000LL;
+constexpr long long kDrainLimitCycles = 4000000000LL;
+// The wait limit handed to the next launches: kWaitLimitCycles unless a test lowered it
+// through gdn_set_wait_limit_for_testing.
+long long wait_limit_cycles();
+// Raises the dynamic shared-memory limit of kernel `fn` to `bytes` on the current device
+// (once per device and kernel). False on a CUDA error.
+bool ensure_smem_limit(const void *fn, unsigned bytes);
 }  // namespace gdn
 
 #include <cuda.h>

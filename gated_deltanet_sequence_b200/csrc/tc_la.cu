@@ -36,10 +36,7 @@
 // UMMA operands are fp16: the bf16 tiles are converted in place once the Gram has
 // read them (exact in fp16 range), the computed operands (S, P, Q', diag(d) K) are
 // rounded to fp16. Shared-memory operands use the 128-byte swizzled layouts.
-#include <mutex>
-
-#include "tc_kernels.cuh"
-#include "tc_ptx.cuh"
+#include "tc_ctl.cuh"
 
 namespace gdn {
 
@@ -99,31 +96,6 @@ enum : int {
 };
 constexpr int kBarState = 1, kBarOut = 2, kBarP = 3, kBarConv = 4, kBarV = 5;   // named barriers
 
-struct Ctl {
-    uint64_t *bar;
-    int *abort_flag;     // CTA-wide: set by the first wait that gives up
-    unsigned *err;
-    long long limit;
-    // Bounded wait; after any timeout in the CTA every later wait fails at once and
-    // each role leaves its loop without issuing further work.
-    __device__ __forceinline__ bool wait(int b, uint32_t parity) const {
-        if (*reinterpret_cast<volatile int *>(abort_flag)) return false;
-        if (mbar_wait(&bar[b], parity, limit)) return true;
-        atomicOr(err, kErrWaitTimeout);
-        *reinterpret_cast<volatile int *>(abort_flag) = 1;
-        return false;
-    }
-    __device__ __forceinline__ void drain(int b, uint32_t parity) const { mbar_wait(&bar[b], parity, limit); }
-    // Group-uniform wait: the leader polls, the group meets on its named barrier and
-    // every thread reads the same sticky verdict.
-    __device__ __forceinline__ bool group_wait(int b, uint32_t parity, int bar_id, int *group_abort, bool leader,
-                                               int nthreads) const {
-        if (leader && !wait(b, parity)) *reinterpret_cast<volatile int *>(group_abort) = 1;
-        named_bar(bar_id, nthreads);
-        return *reinterpret_cast<volatile int *>(group_abort) == 0;
-    }
-};
-
 template <int N>
 __device__ __forceinline__ void ld_cols(uint32_t taddr, float (&v)[N]) {
     static_assert(N % 16 == 0, "16-column pieces");
@@ -156,9 +128,7 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     const uint32_t sb = smem_u32(smem);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kNumBars);
-    int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);   // [0] CTA, [1..4] group verdicts
-    int *abort_s = abort_flag + 1, *abort_o = abort_flag + 2, *abort_cv = abort_flag + 3;
-    int *abort_v = abort_flag + 4, *abort_p = abort_flag + 5;
+    int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);   // CTA-wide abort flag
     const Ctl ctl{bars, abort_flag, err_word, wait_limit};
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -171,7 +141,7 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 
     if (tid == 0) {
         for (int b = 0; b < kNumBars; ++b) mbar_init(&bars[b], 1);
-        for (int i = 0; i < 6; ++i) abort_flag[i] = 0;
+        abort_flag[0] = 0;
         fence_mbar_init();
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
@@ -359,8 +329,8 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         for (int c = 0; c < nchunks; ++c) {
             const int p = c & 1;
             const float *vec = reinterpret_cast<const float *>(smem + OFF_VEC + p * kVecBytes);
-            if (c >= 1 && !ctl.group_wait(B_SDONE, (c - 1) & 1, kBarState, abort_s, lead, 128)) break;
-            if (GATED && !ctl.group_wait(B_GATE + p, (c >> 1) & 1, kBarState, abort_s, lead, 128)) break;
+            if (c >= 1 && !ctl.group_wait(B_SDONE, (c - 1) & 1, kBarState, lead, 128)) break;
+            if (GATED && !ctl.group_wait(B_GATE + p, (c >> 1) & 1, kBarState, lead, 128)) break;
             tc_fence_after();
             // S^T row v -> fp16 pairs (A operand of S^T Q'^T); S <- gamma_last S
             const float gl = GATED ? vec[V_GAM + 63] : 1.f;
@@ -397,7 +367,7 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 for (int e = 0; e < 16; ++e) dst[static_cast<size_t>(cc * 16 + e) * kD] = sv[e];
             }
         } else if (s_final && nchunks > 0 && done == nchunks - 1 &&
-            ctl.group_wait(B_SDONE, (nchunks - 1) & 1, kBarState, abort_s, lead, 128)) {
+            ctl.group_wait(B_SDONE, (nchunks - 1) & 1, kBarState, lead, 128)) {
             tc_fence_after();
             // column v of the final state (a warp writes 32 consecutive floats)
             float *dst = s_final + static_cast<size_t>(bh) * kD * kD + v;
@@ -420,7 +390,7 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 #pragma unroll 1
         for (int c = 0; c < nchunks; ++c) {
             const int p = c & 1;
-            if (!ctl.group_wait(B_ODONE + p, (c >> 1) & 1, kBarOut, abort_o, lead, 128)) break;
+            if (!ctl.group_wait(B_ODONE + p, (c >> 1) & 1, kBarOut, lead, 128)) break;
             tc_fence_after();
             float ov[64];
             ld_cols<64>(trow + TM_O + p * 64, ov);
@@ -449,9 +419,9 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             const int p = c & 1;
             const float *vec = reinterpret_cast<const float *>(smem + OFF_VEC + p * kVecBytes);
             // PG of parity p is free once chunk c-2 is complete
-            if (c >= 2 && !ctl.group_wait(B_ODONE + p, ((c - 2) >> 1) & 1, kBarP, abort_p, pl, 64)) break;
-            if (GATED && !ctl.group_wait(B_GATE + p, (c >> 1) & 1, kBarP, abort_p, pl, 64)) break;
-            if (!ctl.group_wait(B_GRAM + p, (c >> 1) & 1, kBarP, abort_p, pl, 64)) break;
+            if (c >= 2 && !ctl.group_wait(B_ODONE + p, ((c - 2) >> 1) & 1, kBarP, pl, 64)) break;
+            if (GATED && !ctl.group_wait(B_GATE + p, (c >> 1) & 1, kBarP, pl, 64)) break;
+            if (!ctl.group_wait(B_GRAM + p, (c >> 1) & 1, kBarP, pl, 64)) break;
             tc_fence_after();
             const bool fast = !GATED || reinterpret_cast<const int *>(vec)[V_FAST] != 0;
             const float fr = scale * (GATED ? vec[V_GAM + r] : 1.f);
@@ -494,7 +464,7 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 #pragma unroll 1
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % kStages;
-            if (!ctl.group_wait(B_FULL + s, (c / kStages) & 1, kBarV, abort_v, lead, 64)) break;
+            if (!ctl.group_wait(B_FULL + s, (c / kStages) & 1, kBarV, lead, 64)) break;
             uint8_t *vt = smem + s * kStageBytes + ST_V0;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -521,9 +491,9 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             const float *vec = reinterpret_cast<const float *>(smem + OFF_VEC + p * kVecBytes);
             uint8_t *st = smem + s * kStageBytes;
             const int nvalid = min(kC, L - c * kC);
-            if (!ctl.group_wait(B_FULL + s, (c / kStages) & 1, kBarConv, abort_cv, lead, 128)) break;
-            if (GATED && !ctl.group_wait(B_GATE + p, (c >> 1) & 1, kBarConv, abort_cv, lead, 128)) break;
-            if (!ctl.group_wait(B_GREAD + s, (c / kStages) & 1, kBarConv, abort_cv, lead, 128)) break;
+            if (!ctl.group_wait(B_FULL + s, (c / kStages) & 1, kBarConv, lead, 128)) break;
+            if (GATED && !ctl.group_wait(B_GATE + p, (c >> 1) & 1, kBarConv, lead, 128)) break;
+            if (!ctl.group_wait(B_GREAD + s, (c / kStages) & 1, kBarConv, lead, 128)) break;
             // 2 x 1024 chunks of 16 B; chunk i of a tensor sits in box i / 512 (key half),
             // row (i % 512) / 8 of that box (V is converted by the state group)
 #pragma unroll
@@ -568,16 +538,11 @@ gdn_status_t launch_la_t(const CUtensorMap &mq, const CUtensorMap &mk, const CUt
                          const OutArgs &out, const float *s0, float *s_final, const int *cu, int nctas, int H,
                          int L, float scale, cudaStream_t stream) {
     auto kern = tc_la_kernel<GATED, OPTS>;
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [&] {
-        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
-    });
-    if (attr_err != cudaSuccess) return GDN_ERR_CUDA;
+    if (!ensure_smem_limit(reinterpret_cast<const void *>(kern), kSmemAlloc)) return GDN_ERR_CUDA;
     unsigned *err = device_error_word();
     if (!err) return GDN_ERR_CUDA;
-    kern<<<nctas, kThreads, kSmemAlloc, stream>>>(mq, mk, mv, g, out, s0, s_final, cu, H, L, scale, kWaitLimitCycles,
-                                                  err);
+    kern<<<nctas, kThreads, kSmemAlloc, stream>>>(mq, mk, mv, g, out, s0, s_final, cu, H, L, scale,
+                                                  wait_limit_cycles(), err);
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 

@@ -18,7 +18,9 @@
  *
  * Conventions for every entry point
  *  - Ownership: the caller allocates and owns every buffer (device memory unless
- *    stated). The library allocates no memory and keeps no per-call state.
+ *    stated). The library allocates no memory and keeps no per-call state; its only
+ *    state is per device: the condition word that gdn_sync_status reads, cached
+ *    kernel attributes, and the wait limit of gdn_set_wait_limit_for_testing.
  *  - Layout: dense, contiguous, row-major, as annotated. Device pointers must be
  *    16-byte aligned, except beta and g, which need 4-byte alignment.
  *  - Asynchrony: work is enqueued on `cuda_stream` (a cudaStream_t; NULL = the
@@ -62,7 +64,9 @@ typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype_t;
  *  s0       (B, H, dk, dv) fp32 initial state, nullable (zero state)
  *  s_final  (B, H, dk, dv) fp32 final state,   nullable (not written)
  *  B, H >= 1; L >= 0 (L == 0: only s_final is written, = s0 or 0)
- *  dk, dv in {64, 128}; chunk: 1..64 (bf16 with dk = dv = 128 requires 64).
+ *  dk, dv in {64, 128}; chunk: 1..64. bf16 inputs with dk = dv = 128 and chunk 64 run on
+ *  the tensor-core kernels; every other combination runs on the fp32 chunk kernel (the
+ *  same result within its tolerance, at CUDA-core speed).
  *  scale multiplies q.  in_dtype: GDN_BF16 or GDN_F32 (q, k, v share it).
  */
 gdn_status_t lin_attn_chunk_fwd(const void *q, const void *k, const void *v, const float *g,
@@ -201,13 +205,29 @@ gdn_status_t gdn_decode_step_ex(const void *q, const void *k, const void *v, con
 const char *gdn_status_str(gdn_status_t status);
 
 /*
- * gdn_sync_status — synchronise `cuda_stream`, then report (and clear) whether any
- * kernel of this library on the current device met a device-side error since the
- * last call: GDN_ERR_INVALID_ARG for a malformed cu_seqlens list, GDN_ERR_TIMEOUT
- * for a bounded wait that gave up, GDN_ERR_CUDA if the stream reported an error,
- * GDN_OK otherwise.
+ * gdn_sync_status — synchronise `cuda_stream`, then report and clear one device-side
+ * condition met by a kernel of this library on the current device since it was last
+ * reported: GDN_ERR_INVALID_ARG for a malformed cu_seqlens list (reported first),
+ * GDN_ERR_TIMEOUT for a bounded wait that gave up, GDN_OK when neither is pending,
+ * GDN_ERR_CUDA if the stream or the read failed. When both conditions are pending the
+ * next call reports the other one. The conditions live in one word per device, shared by
+ * every caller and stream of this process: a condition raised by another caller's kernel
+ * is reported to whichever caller asks first. The word is taken with a one-thread kernel
+ * on `cuda_stream` (atomic, so a condition raised meanwhile on another stream is kept).
  */
 gdn_status_t gdn_sync_status(void *cuda_stream);
+
+/*
+ * gdn_set_wait_limit_for_testing — for tests of the failure path only: the number of
+ * clock cycles each bounded wait of the tensor-core prefill kernels may take before it
+ * gives up (default about 2 s; cycles <= 0 restores the default). It applies to kernels
+ * launched after the call, from any thread. With a limit of a few hundred cycles the waits
+ * give up while the work they wait for is still legitimately in flight: the kernel then
+ * stops issuing, waits for the copies and tensor-core products it has already issued
+ * (always with the default limit), frees its tensor memory and returns, and the next
+ * gdn_sync_status reports GDN_ERR_TIMEOUT; the outputs of that launch are undefined.
+ */
+void gdn_set_wait_limit_for_testing(long long cycles);
 
 /* Library version as major*10000 + minor*100 + patch. */
 int gdn_version(void);

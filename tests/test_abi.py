@@ -28,7 +28,7 @@ def test_header_declares_the_boundary():
     names = _declared_functions()
     for want in ("lin_attn_chunk_fwd", "gdn_chunk_fwd", "lin_attn_chunk_fwd_varlen", "gdn_chunk_fwd_varlen",
                  "lin_attn_chunk_fwd_ex", "gdn_chunk_fwd_ex", "gdn_decode_step", "gdn_decode_step_ex",
-                 "gdn_status_str", "gdn_sync_status", "gdn_version"):
+                 "gdn_status_str", "gdn_sync_status", "gdn_set_wait_limit_for_testing", "gdn_version"):
         assert want in names
 
 

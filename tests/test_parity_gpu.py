@@ -152,6 +152,33 @@ def test_decode_workload4_sampled_many_steps(lib):
     check(state[ns].cpu(), ref_state, 2e-3, "decode state")
 
 
+def test_decode_workload4_all_steps(lib):
+    # the benchmark's decode loop as timed: 256 sequences x 32 heads, 1000 consecutive steps,
+    # state in place; every step's o of 8 sampled sequences (all 32 heads) and their final
+    # state against the oracle's decode steps, so drift of the fp32 state over the whole
+    # workload shows
+    w = W.WORKLOADS[4]
+    steps = w.L
+    inp = W.make_workload_inputs(w, device="cuda", steps=steps)
+    state = inp["state"]
+    ns = torch.tensor([0, 37, 101, 128, 170, 200, 231, 255])
+    nsd = ns.cuda()
+    o = torch.empty(w.B, w.H, w.dv, device="cuda")
+    o_s = torch.empty(steps, len(ns), w.H, w.dv, device="cuda")
+    ref_state = np.ascontiguousarray(state[nsd].cpu().double().numpy())
+    sample = {n: inp[n][:, nsd].cpu() for n in ("q", "k", "v", "beta", "g")}
+    for t in range(steps):
+        lib.gdn_decode_step(inp["q"][t], inp["k"][t], inp["v"][t], inp["beta"][t], inp["g"][t], state, o=o)
+        o_s[t] = o[nsd]
+    assert lib.gdn_sync_status() == 0
+    o_s = o_s.cpu()
+    worst = 0.0
+    for t in range(steps):
+        o_ref = oracle.decode_step(*(sample[n][t] for n in ("q", "k", "v", "beta", "g")), ref_state)
+        worst = max(worst, check(o_s[t], o_ref, 2e-3, f"decode o step {t}"))
+    check(state[nsd].cpu(), ref_state, 2e-3, "decode state after 1000 steps")
+
+
 @pytest.mark.parametrize("delta,gated", [(False, False), (True, False), (False, True), (True, True)])
 @pytest.mark.parametrize("dk,dv,dtype", [(128, 128, torch.bfloat16), (64, 128, torch.float32),
                                          (128, 64, torch.bfloat16), (64, 64, torch.float32)])

@@ -355,6 +355,17 @@ def measure_rows(gdn, peaks, peak_src, args):
                        "algorithmic_flop_per_launch": fl}
     rows["gdn_prefill_vector_gate"] = row
     del inp, o, sf, gv
+    # backward pass (gradients of the prefill) on the headline shape: fp32 CUDA-core kernel whose
+    # per-token state traffic goes through the caller's workspace (checkpoints + chunk slab)
+    inp = W.make_workload_inputs(w, device="cuda")
+    do = torch.randn(w.B, w.H, w.L, w.dv, device="cuda")
+    ws = torch.empty(gdn.gdn_chunk_bwd_workspace_bytes(w.B, w.H, w.L, w.dk, w.dv, w.chunk), dtype=torch.uint8,
+                     device="cuda")
+    fn = lambda: gdn.gdn_chunk_bwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["g"], do, chunk=w.chunk, workspace=ws)
+    ms = timed(fn, max(3, args.steps // 10), 1)
+    rows["gdn_bwd"] = bwd_row(w, ms, peaks, peak_src)
+    del inp, do, ws
+    torch.cuda.empty_cache()
     # long-context Gated DeltaNet, 1 x 32 x 65536 x 128, S0 != 0
     w = W.WORKLOADS[3]
     inp = W.make_workload_inputs(w, device="cuda")
@@ -414,6 +425,39 @@ def measure_rows(gdn, peaks, peak_src, args):
     del inp, state, od
     torch.cuda.empty_cache()
     return rows
+
+
+def bwd_flops_per_head_token(dk: int, dv: int) -> float:
+    """FLOPs per head-token of the backward kernel: two forward token steps (the checkpoint
+    pass and the recompute: S^T k and the rank-1 update, 4 dk dv each) and the reverse step
+    (q' do^T, Lambda^T k, S_{t-1} du, <Lambda, S_{t-1}>, S_t do, Lambda u: 2 dk dv each; the
+    adjoint update 3 dk dv; its own forward step 4 dk dv)."""
+    return (4 + 4 + 6 * 2 + 3 + 4) * dk * dv
+
+
+def bwd_bytes(B, H, L, dk, dv, chunk, in_bytes=2) -> float:
+    """Bytes one backward launch moves: inputs q, k, v (in_bytes), beta, g, do (fp32); outputs
+    dq, dk, dv, dbeta, dg (fp32); and the workspace: every chunk checkpoint written once and read
+    once, every in-chunk state written once to the slab and read once."""
+    n = B * H * L
+    io = n * ((2 * dk + dv) * in_bytes + 8 + dv * 4) + n * ((2 * dk + dv) * 4 + 8)
+    nck = -(-L // chunk)
+    state = dk * dv * 4
+    wsb = B * H * (2 * nck * state + 2 * L * state)
+    return float(io + wsb)
+
+
+def bwd_row(w, ms, peaks, peak_src):
+    fl = bwd_flops_per_head_token(w.dk, w.dv) * w.B * w.H * w.L
+    nb = bwd_bytes(w.B, w.H, w.L, w.dk, w.dv, w.chunk)
+    row = _row(w, ms, nb, fl, peaks, peak_src, "hbm", w.B * w.L)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    peak_f32 = sms * 128 * 2 * FP32_CLOCK_GHZ / 1e3
+    tf = fl / (ms * 1e-3) / 1e12
+    row["path"] = "fp32 reverse-mode kernel (CUDA cores), state traffic through the workspace"
+    row["alu"] = {"achieved": round(tf, 2), "peak": round(peak_f32, 1), "unit": "TFLOP/s",
+                  "frac": round(tf / peak_f32, 4), "algorithmic_flop_per_launch": fl}
+    return row
 
 
 def _row(w, ms, nbytes, flop, peaks, peak_src, bound, tokens, traffic_key=None):

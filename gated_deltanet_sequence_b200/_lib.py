@@ -23,13 +23,19 @@ GDN_F32, GDN_BF16 = 0, 1
 
 EXPORTS = ("lin_attn_chunk_fwd", "gdn_chunk_fwd", "lin_attn_chunk_fwd_varlen", "gdn_chunk_fwd_varlen",
            "lin_attn_chunk_fwd_ex", "gdn_chunk_fwd_ex", "gdn_decode_step", "gdn_decode_step_ex",
-           "gdn_status_str", "gdn_sync_status", "gdn_set_wait_limit_for_testing", "gdn_version")
+           "gdn_status_str", "gdn_sync_status", "gdn_set_wait_limit_for_testing", "gdn_version",
+           "gdn_chunk_bwd", "gdn_chunk_bwd_workspace_bytes")
+
+
+GDN_XNORM = {None: 0, "rms": 1, "layer": 2}
 
 
 class FwdOpts(ctypes.Structure):
-    """gdn_fwd_opts_t: dtype of o, the D-skip weights (H, dv) (device pointer or None) and
-    the vector-valued gate flag (g holds one log-decay per key coordinate)."""
-    _fields_ = [("out_dtype", ctypes.c_int), ("d_skip", ctypes.c_void_p), ("g_per_key", ctypes.c_int)]
+    """gdn_fwd_opts_t: dtype of o, the D-skip weights (H, dv) (device pointer or None), the
+    vector-valued gate flag (g holds one log-decay per key coordinate) and the output
+    normalisation (kind, weights (H, dv) or None, eps)."""
+    _fields_ = [("out_dtype", ctypes.c_int), ("d_skip", ctypes.c_void_p), ("g_per_key", ctypes.c_int),
+                ("xnorm", ctypes.c_int), ("xnorm_weight", ctypes.c_void_p), ("xnorm_eps", ctypes.c_float)]
 
 
 class GdnError(RuntimeError):
@@ -57,6 +63,11 @@ def _load() -> ctypes.CDLL:
     lib.gdn_sync_status.argtypes = [P]
     lib.gdn_version.argtypes = []
     lib.gdn_set_wait_limit_for_testing.argtypes = [ctypes.c_longlong]
+    Z = ctypes.c_size_t
+    lib.gdn_chunk_bwd_workspace_bytes.argtypes = [I, I, I, I, I, I]
+    lib.gdn_chunk_bwd_workspace_bytes.restype = Z
+    lib.gdn_chunk_bwd.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, Z, I, I, I, I, I, I, F, I, P]
+    lib.gdn_chunk_bwd.restype = ctypes.c_int
     lib.gdn_set_wait_limit_for_testing.restype = None
     for f in (lib.lin_attn_chunk_fwd, lib.gdn_chunk_fwd, lib.lin_attn_chunk_fwd_varlen,
               lib.gdn_chunk_fwd_varlen, lib.lin_attn_chunk_fwd_ex, lib.gdn_chunk_fwd_ex,
@@ -122,28 +133,37 @@ def _check_gate(g, tok_shape, dk, dev):
     return vec
 
 
-def _out_opts(o, out_dtype, d_skip, H, dv, dev, g_per_key=False):
+def _out_opts(o, out_dtype, d_skip, H, dv, dev, g_per_key=False, xnorm=None, xnorm_weight=None, xnorm_eps=1e-6):
     """Output dtype (from ``o`` when given, else ``out_dtype``, default fp32), the checked
-    D-skip weights and the vector-gate flag; returns (dtype, FwdOpts or None when all are
-    defaults)."""
+    D-skip weights, the vector-gate flag and the output normalisation (xnorm None, "rms" or
+    "layer"; xnorm_weight (H, dv) fp32 or None; xnorm_eps); returns (dtype, FwdOpts or None
+    when all are defaults)."""
     dt = o.dtype if o is not None else (out_dtype or torch.float32)
     if dt not in (torch.float32, torch.bfloat16):
         raise TypeError(f"o / out_dtype must be float32 or bfloat16, got {dt}")
     _check("d_skip", d_skip, (H, dv), torch.float32, dev, required=False)
-    if dt == torch.float32 and d_skip is None and not g_per_key:
+    if xnorm not in GDN_XNORM:
+        raise ValueError(f"xnorm must be None, 'rms' or 'layer', got {xnorm!r}")
+    _check("xnorm_weight", xnorm_weight, (H, dv), torch.float32, dev, required=False)
+    if xnorm is None and xnorm_weight is not None:
+        raise ValueError("xnorm_weight given without xnorm")
+    if dt == torch.float32 and d_skip is None and not g_per_key and xnorm is None:
         return dt, None
     return dt, FwdOpts(GDN_BF16 if dt == torch.bfloat16 else GDN_F32,
-                       None if d_skip is None else d_skip.data_ptr(), int(bool(g_per_key)))
+                       None if d_skip is None else d_skip.data_ptr(), int(bool(g_per_key)), GDN_XNORM[xnorm],
+                       None if xnorm_weight is None else xnorm_weight.data_ptr(), float(xnorm_eps))
 
 
 def lin_attn_chunk_fwd(q, k, v, g=None, o=None, s0=None, s_final=None, chunk: int = 64,
-                       scale: float = 1.0, stream=None, out_dtype=None, d_skip=None):
+                       scale: float = 1.0, stream=None, out_dtype=None, d_skip=None, xnorm=None,
+                       xnorm_weight=None, xnorm_eps: float = 1e-6):
     """Plain (g None) or gated causal linear attention. Returns (o, s_final).
 
     out_dtype (torch.float32 / torch.bfloat16) sets the dtype of a new ``o``; d_skip (H, dv)
     fp32 adds the skip term o_t += d_skip[h] * v_t. g of shape (B, H, L, dk) is a
     vector-valued gate (row j of the state decays by exp(g_t[j])); it runs on the fp32
-    chunk kernel."""
+    chunk kernel. xnorm ("rms" / "layer"), xnorm_weight (H, dv) and xnorm_eps normalise each
+    output row over dv after the skip term (the output normalisation of the options)."""
     B, H, L, dk = q.shape
     dv = v.shape[-1]
     dev = q.device
@@ -152,7 +172,7 @@ def lin_attn_chunk_fwd(q, k, v, g=None, o=None, s0=None, s_final=None, chunk: in
     _check("v", v, (B, H, L, dv), q.dtype, dev)
     vec = _check_gate(g, (B, H, L), dk, dev)
     _check("s0", s0, (B, H, dk, dv), torch.float32, dev, required=False)
-    odt, opts = _out_opts(o, out_dtype, d_skip, H, dv, dev, vec)
+    odt, opts = _out_opts(o, out_dtype, d_skip, H, dv, dev, vec, xnorm, xnorm_weight, xnorm_eps)
     if o is None:
         o = torch.empty(B, H, L, dv, dtype=odt, device=dev)
     _check("o", o, (B, H, L, dv), odt, dev)
@@ -171,9 +191,10 @@ def lin_attn_chunk_fwd(q, k, v, g=None, o=None, s0=None, s_final=None, chunk: in
 
 
 def gdn_chunk_fwd(q, k, v, beta, g=None, o=None, s0=None, s_final=None, chunk: int = 64,
-                  scale: float = 1.0, stream=None, out_dtype=None, d_skip=None):
+                  scale: float = 1.0, stream=None, out_dtype=None, d_skip=None, xnorm=None,
+                  xnorm_weight=None, xnorm_eps: float = 1e-6):
     """DeltaNet (g None) or Gated DeltaNet chunkwise prefill. Returns (o, s_final).
-    out_dtype and d_skip as for :func:`lin_attn_chunk_fwd`."""
+    out_dtype, d_skip and the xnorm options as for :func:`lin_attn_chunk_fwd`."""
     B, H, L, dk = q.shape
     dv = v.shape[-1]
     dev = q.device
@@ -183,7 +204,7 @@ def gdn_chunk_fwd(q, k, v, beta, g=None, o=None, s0=None, s_final=None, chunk: i
     _check("beta", beta, (B, H, L), torch.float32, dev, required=L > 0)
     vec = _check_gate(g, (B, H, L), dk, dev)
     _check("s0", s0, (B, H, dk, dv), torch.float32, dev, required=False)
-    odt, opts = _out_opts(o, out_dtype, d_skip, H, dv, dev, vec)
+    odt, opts = _out_opts(o, out_dtype, d_skip, H, dv, dev, vec, xnorm, xnorm_weight, xnorm_eps)
     if o is None:
         o = torch.empty(B, H, L, dv, dtype=odt, device=dev)
     _check("o", o, (B, H, L, dv), odt, dev)
@@ -221,16 +242,16 @@ def _check_varlen(q, k, v, cu_seqlens, s0, s_final):
 
 def lin_attn_chunk_fwd_varlen(q, k, v, cu_seqlens, g=None, o=None, s0=None, s_final=None,
                               chunk: int = 64, scale: float = 1.0, stream=None, out_dtype=None,
-                              d_skip=None):
+                              d_skip=None, xnorm=None, xnorm_weight=None, xnorm_eps: float = 1e-6):
     """Packed variable-length batch of plain / gated linear attention.
 
     q, k (H, T, dk); v (H, T, dv); g (H, T) or None; cu_seqlens (N + 1,) int32 on the device
     (sequence n is tokens cu[n] .. cu[n+1]-1 of every head). s0, s_final (N, H, dk, dv).
     Returns (o, s_final); rows outside every sequence are left as they were in ``o``.
-    out_dtype and d_skip as for :func:`lin_attn_chunk_fwd`."""
+    out_dtype, d_skip and the xnorm options as for :func:`lin_attn_chunk_fwd`."""
     N, H, T, dk, dv, dev = _check_varlen(q, k, v, cu_seqlens, s0, s_final)
     vec = _check_gate(g, (H, T), dk, dev)
-    odt, opts = _out_opts(o, out_dtype, d_skip, H, dv, dev, vec)
+    odt, opts = _out_opts(o, out_dtype, d_skip, H, dv, dev, vec, xnorm, xnorm_weight, xnorm_eps)
     if o is None:
         o = torch.zeros(H, T, dv, dtype=odt, device=dev)
     _check("o", o, (H, T, dv), odt, dev)
@@ -248,13 +269,14 @@ def lin_attn_chunk_fwd_varlen(q, k, v, cu_seqlens, g=None, o=None, s0=None, s_fi
 
 
 def gdn_chunk_fwd_varlen(q, k, v, beta, cu_seqlens, g=None, o=None, s0=None, s_final=None,
-                         chunk: int = 64, scale: float = 1.0, stream=None, out_dtype=None, d_skip=None):
+                         chunk: int = 64, scale: float = 1.0, stream=None, out_dtype=None, d_skip=None,
+                         xnorm=None, xnorm_weight=None, xnorm_eps: float = 1e-6):
     """Packed variable-length batch of DeltaNet / Gated DeltaNet (see lin_attn_chunk_fwd_varlen);
     beta (H, T) fp32."""
     N, H, T, dk, dv, dev = _check_varlen(q, k, v, cu_seqlens, s0, s_final)
     _check("beta", beta, (H, T), torch.float32, dev, required=T > 0)
     vec = _check_gate(g, (H, T), dk, dev)
-    odt, opts = _out_opts(o, out_dtype, d_skip, H, dv, dev, vec)
+    odt, opts = _out_opts(o, out_dtype, d_skip, H, dv, dev, vec, xnorm, xnorm_weight, xnorm_eps)
     if o is None:
         o = torch.zeros(H, T, dv, dtype=odt, device=dev)
     _check("o", o, (H, T, dv), odt, dev)
@@ -272,9 +294,10 @@ def gdn_chunk_fwd_varlen(q, k, v, beta, cu_seqlens, g=None, o=None, s0=None, s_f
 
 
 def gdn_decode_step(q, k, v, beta, g, state, o=None, scale: float = 1.0, stream=None, out_dtype=None,
-                    d_skip=None):
+                    d_skip=None, xnorm=None, xnorm_weight=None, xnorm_eps: float = 1e-6):
     """One decode token for (N, H) heads; ``state`` (N, H, dk, dv) fp32 is updated in place.
-    g (N, H) or (N, H, dk) (vector-valued gate); out_dtype and d_skip as for the prefill calls."""
+    g (N, H) or (N, H, dk) (vector-valued gate); out_dtype, d_skip and the xnorm options as
+    for the prefill calls."""
     N, H, dk = q.shape
     dv = v.shape[-1]
     dev = q.device
@@ -284,7 +307,7 @@ def gdn_decode_step(q, k, v, beta, g, state, o=None, scale: float = 1.0, stream=
     _check("beta", beta, (N, H), torch.float32, dev, required=False)
     vec = _check_gate(g, (N, H), dk, dev)
     _check("state", state, (N, H, dk, dv), torch.float32, dev)
-    odt, opts = _out_opts(o, out_dtype, d_skip, H, dv, dev, vec)
+    odt, opts = _out_opts(o, out_dtype, d_skip, H, dv, dev, vec, xnorm, xnorm_weight, xnorm_eps)
     if o is None:
         o = torch.empty(N, H, dv, dtype=odt, device=dev)
     _check("o", o, (N, H, dv), odt, dev)
@@ -314,3 +337,40 @@ def gdn_set_wait_limit_for_testing(cycles: int) -> None:
 
 def gdn_version() -> int:
     return lib.gdn_version()
+
+
+def gdn_chunk_bwd(q, k, v, beta, g, d_o, s0=None, ds_final=None, chunk: int = 64, scale: float = 1.0,
+                  workspace=None, stream=None):
+    """Gradients of the prefill (beta None: linear attention) for the loss sum(o * d_o) +
+    sum(S_final * ds_final). Returns a dict of fp32 tensors dq, dk, dv, dbeta (None without
+    beta), dg (None without g), ds0. ``workspace``: a device tensor of at least
+    gdn_chunk_bwd_workspace_bytes(...) bytes (allocated here with torch when None)."""
+    B, H, L, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    _check("q", q, (B, H, L, dk), device=dev)
+    _check("k", k, (B, H, L, dk), q.dtype, dev)
+    _check("v", v, (B, H, L, dv), q.dtype, dev)
+    _check("beta", beta, (B, H, L), torch.float32, dev, required=False)
+    _check("g", g, (B, H, L), torch.float32, dev, required=False)
+    _check("d_o", d_o, (B, H, L, dv), torch.float32, dev)
+    _check("s0", s0, (B, H, dk, dv), torch.float32, dev, required=False)
+    _check("ds_final", ds_final, (B, H, dk, dv), torch.float32, dev, required=False)
+    need = gdn_chunk_bwd_workspace_bytes(B, H, L, dk, dv, chunk)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    out = {"dq": torch.empty(B, H, L, dk, **f32), "dk": torch.empty(B, H, L, dk, **f32),
+           "dv": torch.empty(B, H, L, dv, **f32), "dbeta": None if beta is None else torch.empty(B, H, L, **f32),
+           "dg": None if g is None else torch.empty(B, H, L, **f32), "ds0": torch.empty(B, H, dk, dv, **f32)}
+    st = lib.gdn_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(s0), _ptr(d_o), _ptr(ds_final),
+                           _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dbeta"]), _ptr(out["dg"]),
+                           _ptr(out["ds0"]), _ptr(workspace), workspace.numel() * workspace.element_size(), B, H, L,
+                           dk, dv, int(chunk), float(scale), _dtype_code(q), _stream(stream))
+    _raise("gdn_chunk_bwd", st)
+    return out
+
+
+def gdn_chunk_bwd_workspace_bytes(B: int, H: int, L: int, dk: int, dv: int, chunk: int = 64) -> int:
+    """Bytes of device workspace gdn_chunk_bwd needs (0 for unsupported sizes)."""
+    return int(lib.gdn_chunk_bwd_workspace_bytes(B, H, L, dk, dv, chunk))

@@ -11,7 +11,20 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 bool opt_aligned16(const void *p) { return p == nullptr || aligned16(p); }
 bool opt_aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 bool head_dim_ok(int d) { return d == 64 || d == 128; }
-constexpr gdn::FwdOpts kDefaultOut{false, nullptr};   // fp32 o, no D-skip term
+constexpr gdn::FwdOpts kDefaultOut{false, nullptr, false, gdn::kXNormNone, nullptr, 0.f};   // fp32 o, no options
+
+// The output-normalisation fields of the options: a known kind, a positive finite eps
+// when one is set, a 4-byte aligned weight.
+bool set_xnorm(const gdn_fwd_opts_t &opts, gdn::FwdOpts *oo) {
+    if (opts.xnorm != GDN_XNORM_NONE && opts.xnorm != GDN_XNORM_RMS && opts.xnorm != GDN_XNORM_LAYER) return false;
+    if (opts.xnorm != GDN_XNORM_NONE && !(isfinite(opts.xnorm_eps) && opts.xnorm_eps > 0.f)) return false;
+    if (!opt_aligned4(opts.xnorm_weight)) return false;
+    oo->xnorm = opts.xnorm == GDN_XNORM_RMS ? gdn::kXNormRms : opts.xnorm == GDN_XNORM_LAYER ? gdn::kXNormLayer
+                                                                                          : gdn::kXNormNone;
+    oo->xw = opts.xnorm_weight;
+    oo->xeps = opts.xnorm_eps;
+    return true;
+}
 
 gdn_status_t check_prefill(const void *q, const void *k, const void *v, const float *g, float *o,
                            const float *s0, float *s_final, int B, int H, int L, int dk, int dv,
@@ -46,7 +59,7 @@ const char *gdn_status_str(gdn_status_t s) {
     return "GDN_ERR_UNKNOWN";
 }
 
-int gdn_version(void) { return 100; }
+int gdn_version(void) { return 101; }
 
 gdn_status_t lin_attn_chunk_fwd(const void *q, const void *k, const void *v, const float *g,
                                 float *o, const float *s0, float *s_final, int B, int H, int L,
@@ -121,6 +134,7 @@ static gdn_status_t prefill_ex(bool delta, const void *q, const void *k, const v
         if (opts->out_dtype != GDN_F32 && opts->out_dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
         if (!opt_aligned4(opts->d_skip)) return GDN_ERR_INVALID_ARG;
         if (opts->g_per_key != 0 && opts->g_per_key != 1) return GDN_ERR_INVALID_ARG;
+        if (!set_xnorm(*opts, &oo)) return GDN_ERR_INVALID_ARG;
         oo.bf16 = opts->out_dtype == GDN_BF16;
         oo.dskip = opts->d_skip;
         oo.gate_per_key = opts->g_per_key == 1 && g != nullptr;
@@ -174,6 +188,7 @@ static gdn_status_t decode_impl(const void *q, const void *k, const void *v, con
         if (opts->out_dtype != GDN_F32 && opts->out_dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
         if (opts->g_per_key != 0 && opts->g_per_key != 1) return GDN_ERR_INVALID_ARG;
         if (!opt_aligned4(opts->d_skip)) return GDN_ERR_INVALID_ARG;
+        if (!set_xnorm(*opts, &oo)) return GDN_ERR_INVALID_ARG;
         oo.bf16 = opts->out_dtype == GDN_BF16;
         oo.dskip = opts->d_skip;
         oo.gate_per_key = opts->g_per_key == 1 && g != nullptr;
@@ -195,6 +210,33 @@ gdn_status_t gdn_decode_step_ex(const void *q, const void *k, const void *v, con
                                 float scale, gdn_dtype_t in_dtype, const gdn_fwd_opts_t *opts,
                                 void *cuda_stream) {
     return decode_impl(q, k, v, beta, g, state, o, N, H, dk, dv, scale, in_dtype, opts, cuda_stream);
+}
+
+size_t gdn_chunk_bwd_workspace_bytes(int B, int H, int L, int dk, int dv, int chunk) {
+    if (B < 1 || H < 1 || L < 0 || chunk < 1 || chunk > 128 || !head_dim_ok(dk) || !head_dim_ok(dv)) return 0;
+    return gdn::bwd_workspace_floats(static_cast<long>(B) * H, L, dk, dv, chunk) * sizeof(float);
+}
+
+gdn_status_t gdn_chunk_bwd(const void *q, const void *k, const void *v, const float *beta, const float *g,
+                           const float *s0, const float *d_o, const float *ds_final, float *dq, float *dk, float *dv,
+                           float *dbeta, float *dg, float *ds0, void *workspace, size_t workspace_bytes, int B, int H,
+                           int L, int dk_, int dv_, int chunk, float scale, gdn_dtype_t in_dtype, void *cuda_stream) {
+    if (B < 1 || H < 1 || L < 0 || !isfinite(scale) || chunk < 1) return GDN_ERR_INVALID_ARG;
+    if (in_dtype != GDN_F32 && in_dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (!head_dim_ok(dk_) || !head_dim_ok(dv_) || chunk > 128) return GDN_ERR_UNSUPPORTED;
+    if ((double)B * H > 2147483647.0 || (double)B * H * (double)L * 128.0 > 9.0e18) return GDN_ERR_INVALID_ARG;
+    if (L > 0 && (!q || !k || !v || !d_o || !dq || !dk || !dv)) return GDN_ERR_INVALID_ARG;
+    if (L > 0 && ((beta && !dbeta) || (g && !dg))) return GDN_ERR_INVALID_ARG;
+    if (!opt_aligned16(q) || !opt_aligned16(k) || !opt_aligned16(v) || !opt_aligned16(d_o) || !opt_aligned16(dq) ||
+        !opt_aligned16(dk) || !opt_aligned16(dv) || !opt_aligned16(s0) || !opt_aligned16(ds_final) ||
+        !opt_aligned16(ds0) || !opt_aligned16(workspace) || !opt_aligned4(beta) || !opt_aligned4(g) ||
+        !opt_aligned4(dbeta) || !opt_aligned4(dg))
+        return GDN_ERR_INVALID_ARG;
+    const size_t need = gdn_chunk_bwd_workspace_bytes(B, H, L, dk_, dv_, chunk);
+    if (!workspace || workspace_bytes < need) return GDN_ERR_INVALID_ARG;
+    return gdn::launch_bwd(q, k, v, beta, g, s0, d_o, ds_final, dq, dk, dv, beta ? dbeta : nullptr,
+                           g ? dg : nullptr, ds0, static_cast<float *>(workspace), B, H, L, dk_, dv_, chunk, scale,
+                           in_dtype, static_cast<cudaStream_t>(cuda_stream));
 }
 
 }  // extern "C"

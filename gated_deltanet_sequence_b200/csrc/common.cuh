@@ -61,11 +61,19 @@ __device__ __forceinline__ void st_global4(float *p, float4 v) {
 // Options of the prefill kernels: o in fp32 or bf16, vector-valued gates, and the Mamba
 // D-skip term o_t += D_h (elementwise) v_t, D of shape (H, dv) (page "【CS336】lecture4",
 // section "继续改进：Mamba": a term in v added at the output, like a residual branch).
+// Output normalisation (page "LinearAttention 概述", section "The Devil in Linear
+// Transformer": the normaliser's denominator is dropped and the output is normalised
+// instead, O = XNorm(Q (K^T V))): each output row of each head over its dv values, after
+// the skip term and before the output rounding, times a weight (H, dv) (nullable: ones).
+enum : int { kXNormNone = 0, kXNormRms = 1, kXNormLayer = 2 };
 struct FwdOpts {
     bool bf16;            // o is bf16 (round to nearest even), else fp32
     const float *dskip;   // (H, dv) fp32, nullable (no skip term)
     bool gate_per_key;    // g holds one log-decay per key coordinate: (rows, dk) in prefill (fp32
                           // chunk kernel), (N, H, dk) in decode
+    int xnorm;            // kXNorm*
+    const float *xw;      // (H, dv) fp32 weight of the output normalisation, nullable
+    float xeps;           // added under the root to the row's mean square (variance)
 };
 // The same, as a kernel argument: o, and for the D-skip term the input v (bf16 for the
 // tensor-core kernels; same (rows, dv) layout as o) with D.
@@ -74,35 +82,128 @@ struct OutArgs {
     const __nv_bfloat16 *v;   // nullptr: no D-skip term
     const float *dskip;       // (H, dv)
     int bf16;
+    int xnorm;                // kXNorm*
+    const float *xw;          // (H, dv), nullable
+    float xeps;
 };
 
-// One value column of a 64-token output tile: ov[r] = o[row r][column] for r < n, at
-// element offset elem0 + r * stride of o. Adds dj * v at the same offsets when v is
-// given (the D-skip term, fp32 fused multiply-add), then stores fp32 or bf16.
-__device__ __forceinline__ void store_out_rows(float (&ov)[64], void *o, size_t elem0, int n, int stride,
-                                               bool bf16, float dj, const __nv_bfloat16 *v) {
+// The kernel argument of the tensor-core kernels (bf16 v for the skip term).
+inline OutArgs make_out_args(void *o, const void *v, const FwdOpts &oo) {
+    return OutArgs{o, oo.dskip ? static_cast<const __nv_bfloat16 *>(v) : nullptr, oo.dskip, oo.bf16 ? 1 : 0,
+                   oo.xnorm, oo.xw, oo.xeps};
+}
+
+// ---------------------------------------------------------------- row statistics
+// A 64-row tile held by a warp with one column per lane (a[r] = this lane's value of row
+// r): on exit a[0] and a[1] hold the warp's sums over its 32 columns of rows 2 lane and
+// 2 lane + 1 (a transposing butterfly: each level keeps half of the rows and adds the
+// partner lane's values of them, 62 shuffles in all).
+template <int N>
+__device__ __forceinline__ void fold_rows(float *a, bool up, int k) {
 #pragma unroll
-    for (int r0 = 0; r0 < 64; r0 += 16) {
-        float x[16];
+    for (int i = 0; i < N; ++i) {
+        const float send = up ? a[i] : a[i + N];
+        const float keep = up ? a[i + N] : a[i];
+        a[i] = keep + __shfl_xor_sync(0xffffffffu, send, k);
+    }
+}
+__device__ __forceinline__ void warp_row_sums(float (&a)[64]) {
+    const int lane = threadIdx.x & 31;
+    fold_rows<32>(a, lane & 16, 16);
+    fold_rows<16>(a, lane & 8, 8);
+    fold_rows<8>(a, lane & 4, 4);
+    fold_rows<4>(a, lane & 2, 2);
+    fold_rows<2>(a, lane & 1, 1);
+}
+__device__ __forceinline__ void group_bar(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+// Row sums over the 128 columns (4 warps) of a 64-row tile held by a 128-thread group
+// (thread gt = column): red (4 x 64 floats of shared memory) takes the warp sums, and
+// out[r] = post_mul * sum of row r for r < 64. The group meets twice on bar_id.
+__device__ __forceinline__ void group_row_sums(float (&a)[64], int gt, int bar_id, float *red, float *out,
+                                               float post_mul) {
+    warp_row_sums(a);
+    const int w = gt >> 5, l = gt & 31;
+    red[w * 64 + 2 * l] = a[0];
+    red[w * 64 + 2 * l + 1] = a[1];
+    group_bar(bar_id, 128);
+    if (gt < 64) out[gt] = (red[gt] + red[64 + gt] + red[128 + gt] + red[192 + gt]) * post_mul;
+    group_bar(bar_id, 128);
+}
+// Output normalisation of a 64-row tile held by a 128-thread group, dv = 128 columns
+// (thread gt = column, x[r] its value of row r): x[r] <- (x[r] - mean_r) w / sqrt(var_r +
+// eps), with mean_r = 0 and var_r the mean square for the RMS form (two passes for the
+// layer form: the mean first, then the mean square of the centred row). red: 4 x 64
+// floats, stat: 2 x 64 floats of shared memory.
+__device__ __forceinline__ void group_xnorm_128(float (&x)[64], int kind, float eps, float w, int gt, int bar_id,
+                                                float *red, float *stat) {
+    float t[64];
+    if (kind == kXNormLayer) {
 #pragma unroll
-        for (int r = 0; r < 16; ++r) x[r] = ov[r0 + r];
-        if (v) {
+        for (int r = 0; r < 64; ++r) t[r] = x[r];
+        group_row_sums(t, gt, bar_id, red, stat, 1.f / 128.f);
 #pragma unroll
-            for (int r = 0; r < 16; ++r)
-                if (r0 + r < n) x[r] = fmaf(dj, __bfloat162float(v[elem0 + static_cast<size_t>(r0 + r) * stride]), x[r]);
-        }
-        if (bf16) {
-            __nv_bfloat16 *ob = static_cast<__nv_bfloat16 *>(o) + elem0;
-#pragma unroll
-            for (int r = 0; r < 16; ++r)
-                if (r0 + r < n) ob[static_cast<size_t>(r0 + r) * stride] = __float2bfloat16_rn(x[r]);
-        } else {
-            float *of = static_cast<float *>(o) + elem0;
-#pragma unroll
-            for (int r = 0; r < 16; ++r)
-                if (r0 + r < n) of[static_cast<size_t>(r0 + r) * stride] = x[r];
+        for (int r = 0; r < 64; r += 4) {
+            const float4 m = *reinterpret_cast<const float4 *>(stat + r);
+            x[r] -= m.x; x[r + 1] -= m.y; x[r + 2] -= m.z; x[r + 3] -= m.w;
         }
     }
+#pragma unroll
+    for (int r = 0; r < 64; ++r) t[r] = x[r] * x[r];
+    group_row_sums(t, gt, bar_id, red, stat + 64, 1.f / 128.f);
+#pragma unroll
+    for (int r = 0; r < 64; r += 4) {
+        const float4 m = *reinterpret_cast<const float4 *>(stat + 64 + r);
+        x[r] *= w * rsqrtf(m.x + eps);
+        x[r + 1] *= w * rsqrtf(m.y + eps);
+        x[r + 2] *= w * rsqrtf(m.z + eps);
+        x[r + 3] *= w * rsqrtf(m.w + eps);
+    }
+}
+
+// One value column of a 64-token output tile: stores ov[r] (r < n) at element offset
+// elem0 + r * stride of o, in fp32 or rounded to bf16 (nearest, ties to even).
+__device__ __forceinline__ void store_out_rows_final(const float (&ov)[64], void *o, size_t elem0, int n, int stride,
+                                                     bool bf16) {
+    if (bf16) {
+        __nv_bfloat16 *ob = static_cast<__nv_bfloat16 *>(o) + elem0;
+#pragma unroll
+        for (int r = 0; r < 64; ++r)
+            if (r < n) ob[static_cast<size_t>(r) * stride] = __float2bfloat16_rn(ov[r]);
+    } else {
+        float *of = static_cast<float *>(o) + elem0;
+#pragma unroll
+        for (int r = 0; r < 64; ++r)
+            if (r < n) of[static_cast<size_t>(r) * stride] = ov[r];
+    }
+}
+// The same after the D-skip term: adds dj * v at the same offsets when v is given (fp32
+// fused multiply-add).
+__device__ __forceinline__ void store_out_rows(float (&ov)[64], void *o, size_t elem0, int n, int stride,
+                                               bool bf16, float dj, const __nv_bfloat16 *v) {
+    if (v) {
+#pragma unroll
+        for (int r = 0; r < 64; ++r)
+            if (r < n) ov[r] = fmaf(dj, __bfloat162float(v[elem0 + static_cast<size_t>(r) * stride]), ov[r]);
+    }
+    store_out_rows_final(ov, o, elem0, n, stride, bf16);
+}
+// The same for a 128-thread group holding the tile's 128 value columns (thread gt =
+// column), with the output normalisation when out.xnorm is set. The whole group calls it
+// (it meets on bar_id); red and stat are shared scratch of 256 and 128 floats. head
+// indexes the (H, dv) weights of the skip term and of the normalisation.
+__device__ __forceinline__ void store_out_rows_group(float (&ov)[64], const OutArgs &out, size_t elem0, int n,
+                                                     int head, int gt, int bar_id, float *red, float *stat) {
+    if (out.v) {
+        const float dj = out.dskip[head * 128 + gt];
+#pragma unroll
+        for (int r = 0; r < 64; ++r)
+            if (r < n) ov[r] = fmaf(dj, __bfloat162float(out.v[elem0 + static_cast<size_t>(r) * 128]), ov[r]);
+    }
+    if (out.xnorm != kXNormNone)
+        group_xnorm_128(ov, out.xnorm, out.xeps, out.xw ? out.xw[head * 128 + gt] : 1.f, gt, bar_id, red, stat);
+    store_out_rows_final(ov, out.o, elem0, n, 128, out.bf16 != 0);
 }
 
 }  // namespace gdn
@@ -118,4 +219,10 @@ gdn_status_t launch_simt_fwd(const void *q, const void *k, const void *v, const 
 gdn_status_t launch_decode(const void *q, const void *k, const void *v, const float *beta,
                            const float *g, float *state, void *o, int N, int H, int dk, int dv,
                            float scale, gdn_dtype_t in_dtype, FwdOpts oo, cudaStream_t stream);
+// Backward pass: floats of workspace it needs, and the launch (ws: that many floats).
+size_t bwd_workspace_floats(long BH, int L, int dk, int dv, int chunk);
+gdn_status_t launch_bwd(const void *q, const void *k, const void *v, const float *beta, const float *g,
+                        const float *s0, const float *dout, const float *dsf, float *dq, float *dk, float *dv,
+                        float *dbeta, float *dg, float *ds0, float *ws, int B, int H, int L, int dk_, int dv_,
+                        int chunk, float scale, gdn_dtype_t in_dtype, cudaStream_t stream);
 }  // namespace gdn

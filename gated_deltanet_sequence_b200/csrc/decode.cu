@@ -11,7 +11,7 @@
 // With a vector-valued gate (alpha_t[j] per key row j) the decayed state diag(alpha) S
 // replaces alpha S: sk = (diag(alpha) S)^T k, sq = (diag(alpha) S)^T q', o = sq + (q'.k) u,
 // S <- diag(alpha) S + k u^T. The options variant also takes the skip term o += D_h v
-// and a bf16 output.
+// a bf16 output and the output normalisation of the prefill calls.
 //
 // Layout: one CTA per (sequence, head); thread t owns 4 consecutive value
 // columns (float4) of RPT rows strided by the number of row groups, so every
@@ -29,7 +29,8 @@ __global__ void __launch_bounds__(kDecThreads)
 decode_step_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT *__restrict__ v,
                    const float *__restrict__ beta, const float *__restrict__ g,
                    float *__restrict__ state, void *__restrict__ o, float scale, int H, int vec,
-                   int out_bf16, const float *__restrict__ dskip) {
+                   int out_bf16, const float *__restrict__ dskip, int xnorm, const float *__restrict__ xw,
+                   float xeps) {
     constexpr int CG = DV / 4;               // float4 column groups
     constexpr int RG = kDecThreads / CG;     // row groups
     constexpr int RPT = DK / RG;             // rows per thread
@@ -123,6 +124,27 @@ decode_step_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
                 ov.z = fmaf(dh[2], s_v[4 * cg + 2], ov.z);
                 ov.w = fmaf(dh[3], s_v[4 * cg + 3], ov.w);
             }
+            if (xnorm != kXNormNone) {
+                // output normalisation over the DV outputs, held 4 per lane by lanes 0..CG-1
+                constexpr unsigned mask = CG >= 32 ? 0xffffffffu : ((1u << CG) - 1u);
+                float mean = 0.f;
+                if (xnorm == kXNormLayer) {
+                    float s1 = (ov.x + ov.y) + (ov.z + ov.w);
+#pragma unroll
+                    for (int off = CG / 2; off > 0; off >>= 1) s1 += __shfl_xor_sync(mask, s1, off);
+                    mean = s1 * (1.f / DV);
+                }
+                ov.x -= mean; ov.y -= mean; ov.z -= mean; ov.w -= mean;
+                float s2 = (ov.x * ov.x + ov.y * ov.y) + (ov.z * ov.z + ov.w * ov.w);
+#pragma unroll
+                for (int off = CG / 2; off > 0; off >>= 1) s2 += __shfl_xor_sync(mask, s2, off);
+                const float rs = rsqrtf(s2 * (1.f / DV) + xeps);
+                const float *wh = xw ? xw + (head % H) * DV + 4 * cg : nullptr;
+                ov.x *= rs * (wh ? wh[0] : 1.f);
+                ov.y *= rs * (wh ? wh[1] : 1.f);
+                ov.z *= rs * (wh ? wh[2] : 1.f);
+                ov.w *= rs * (wh ? wh[3] : 1.f);
+            }
             if (out_bf16) {
                 __nv_bfloat16 *ob = static_cast<__nv_bfloat16 *>(o) + head * DV + 4 * cg;
                 ob[0] = __float2bfloat16_rn(ov.x);
@@ -155,10 +177,12 @@ gdn_status_t launch_dec_t(const void *q, const void *k, const void *v, const flo
     const int vec = oo.gate_per_key ? 1 : 0, ob = oo.bf16 ? 1 : 0;
     if (beta)
         decode_step_kernel<DK, DV, IT, true, OPT><<<(unsigned)NH, kDecThreads, 0, stream>>>(
-            (const IT *)q, (const IT *)k, (const IT *)v, beta, g, state, o, scale, H, vec, ob, oo.dskip);
+            (const IT *)q, (const IT *)k, (const IT *)v, beta, g, state, o, scale, H, vec, ob, oo.dskip, oo.xnorm,
+            oo.xw, oo.xeps);
     else
         decode_step_kernel<DK, DV, IT, false, OPT><<<(unsigned)NH, kDecThreads, 0, stream>>>(
-            (const IT *)q, (const IT *)k, (const IT *)v, beta, g, state, o, scale, H, vec, ob, oo.dskip);
+            (const IT *)q, (const IT *)k, (const IT *)v, beta, g, state, o, scale, H, vec, ob, oo.dskip, oo.xnorm,
+            oo.xw, oo.xeps);
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
@@ -181,7 +205,7 @@ gdn_status_t launch_decode(const void *q, const void *k, const void *v, const fl
                            const float *g, float *state, void *o, int N, int H, int dk, int dv,
                            float scale, gdn_dtype_t in_dtype, FwdOpts oo, cudaStream_t stream) {
     const long NH = (long)N * H;
-    const bool opt = oo.bf16 || oo.dskip || oo.gate_per_key;
+    const bool opt = oo.bf16 || oo.dskip || oo.gate_per_key || oo.xnorm != kXNormNone;
     if (in_dtype == GDN_F32)
         return opt ? launch_dec_dt<float, true>(q, k, v, beta, g, state, o, NH, H, dk, dv, scale, oo, stream)
                    : launch_dec_dt<float, false>(q, k, v, beta, g, state, o, NH, H, dk, dv, scale, oo, stream);

@@ -33,7 +33,7 @@ constexpr int kSimtThreads = 1024;   // one CTA per SM (the tiles take 215 KB of
 constexpr int kDvs = 32;      // value columns per CTA
 constexpr int kCmax = 64;     // largest supported chunk
 
-template <int DK, bool VEC>
+template <int DK, bool VEC, bool XN>
 struct SimtSmem {
     static constexpr int KP = DK + 1;            // padded row pitch for K, Q, W
     static constexpr int CP = kCmax + 1;         // padded row pitch for A, T, P
@@ -49,18 +49,42 @@ struct SimtSmem {
     float G[kCmax];
     float bt[kCmax];
     float GV[VEC ? kCmax * KP : 1];              // per-key cumulative log-decay (vector gates)
+    float Ob[XN ? kCmax * kDvs : 1];             // output tile before the normalisation
+    float part[XN ? 2 * kCmax : 1];              // this CTA's row sums, by reduction-round parity
 };
 
-template <int DK, typename IT, bool DELTA, bool VEC>
+// Sum over the cluster's CTAs (the dv / 32 value slices of one head) of x, one value per
+// output row r < n: each CTA leaves its row sums in its part[] buffer of this round's parity,
+// the cluster meets once, and every CTA adds all buffers through distributed shared
+// memory. Double buffering by round parity keeps a buffer untouched until every CTA has
+// passed the next round's barrier, i.e. has finished reading it.
+__device__ __forceinline__ float cluster_row_sum(float *part, int round, int r, float x, bool writer, int nslices) {
+    float *buf = part + (round & 1) * kCmax;
+    if (writer) buf[r] = x;
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+    float total = 0.f;
+    const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(buf + r));
+    for (int rank = 0; rank < nslices; ++rank) {
+        uint32_t ra;
+        float y;
+        asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
+        asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(y) : "r"(ra) : "memory");
+        total += y;
+    }
+    return total;
+}
+
+template <int DK, typename IT, bool DELTA, bool VEC, bool XN>
 __global__ void __launch_bounds__(kSimtThreads)
 simt_chunk_fwd_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT *__restrict__ v,
                       const float *__restrict__ beta, const float *__restrict__ g,
                       void *__restrict__ o, int out_bf16, const float *__restrict__ dskip,
+                      int xnorm, const float *__restrict__ xw, float xeps,
                       const float *__restrict__ s0,
                       float *__restrict__ s_final, const int *__restrict__ cu, int H, int Lrow,
                       int dv, int C, float scale, unsigned *__restrict__ err) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    using Sm = SimtSmem<DK, VEC>;
+    using Sm = SimtSmem<DK, VEC, XN>;
     Sm &sm = *reinterpret_cast<Sm *>(smem_raw);
     constexpr int KP = Sm::KP, CP = Sm::CP;
     const int tid = threadIdx.x;
@@ -84,6 +108,7 @@ simt_chunk_fwd_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const 
         sm.S[i] = s0 ? s0[(bh * DK + j) * dv + c0 + c] : 0.f;
     }
 
+    int round = 0;   // reduction rounds across the cluster (output normalisation)
     for (int t0 = 0; t0 < L; t0 += C) {
         const int n = min(C, L - t0);
         __syncthreads();
@@ -257,11 +282,47 @@ simt_chunk_fwd_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const 
             for (int s = 0; s <= r; ++s) pu = fmaf(sm.P[r * CP + s], Ut[s * kDvs + c], pu);
             float ov = (VEC ? qs : expf(sm.G[r]) * qs) + pu;
             if (dsk) ov = fmaf(dsk[c], sm.V[i], ov);     // D-skip term D_h v_t
+            if (XN) {
+                sm.Ob[i] = ov;
+                continue;
+            }
             const long oi = o0 + (long)(t0 + r) * dv + c0 + c;
             if (out_bf16) static_cast<__nv_bfloat16 *>(o)[oi] = __float2bfloat16_rn(ov);
             else static_cast<float *>(o)[oi] = ov;
         }
         __syncthreads();
+        if (XN) {
+            // ---- output normalisation of each row over all dv columns (the cluster's
+            //      slices): warp w takes rows w, w + 32 (lane = column of this slice)
+            const int lane = tid & 31, warp = tid >> 5, nsl = dv / kDvs;
+            const float wc = xw ? xw[static_cast<long>(sp.head_row % H) * dv + c0 + lane] : 1.f;
+#pragma unroll
+            for (int rr = 0; rr < kCmax; rr += 32) {
+                const int r = rr + warp;
+                // every thread takes part in both rounds (the cluster barrier is CTA-wide);
+                // rows past n contribute zeros and store nothing
+                float x = r < n ? sm.Ob[r * kDvs + lane] : 0.f;
+                float mean = 0.f;
+                if (xnorm == kXNormLayer) {
+                    float s1 = x;
+#pragma unroll
+                    for (int off = 16; off > 0; off >>= 1) s1 += __shfl_xor_sync(0xffffffffu, s1, off);
+                    mean = cluster_row_sum(sm.part, round++, r, s1, lane == 0, nsl) / dv;
+                }
+                x -= mean;
+                float s2 = x * x;
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, off);
+                const float ms = cluster_row_sum(sm.part, round++, r, s2, lane == 0, nsl) / dv;
+                const float y = x * rsqrtf(ms + xeps) * wc;
+                if (r < n) {
+                    const long oi = o0 + (long)(t0 + r) * dv + c0 + lane;
+                    if (out_bf16) static_cast<__nv_bfloat16 *>(o)[oi] = __float2bfloat16_rn(y);
+                    else static_cast<float *>(o)[oi] = y;
+                }
+            }
+            __syncthreads();
+        }
         // ---- S <- gamma_n S + sum_s exp(G_n - G_s) k_s Ut_s^T ----------------------
         {
             const float Gn = sm.G[n - 1];
@@ -290,20 +351,47 @@ simt_chunk_fwd_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const 
     }
 }
 
+template <int DK, typename IT, bool DELTA, bool VEC, bool XN>
+gdn_status_t launch_simt_x(const void *q, const void *k, const void *v, const float *beta,
+                           const float *g, void *o, const float *s0, float *s_final, const int *cu,
+                           int BH, int H, int L, int dv, int chunk, float scale, const FwdOpts &oo, unsigned *err,
+                           cudaStream_t stream) {
+    auto kern = simt_chunk_fwd_kernel<DK, IT, DELTA, VEC, XN>;
+    const unsigned smem = static_cast<unsigned>(sizeof(SimtSmem<DK, VEC, XN>));
+    if (!ensure_smem_limit(reinterpret_cast<const void *>(kern), smem)) return GDN_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(BH, dv / kDvs);
+    cfg.blockDim = dim3(kSimtThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    if (XN) {
+        // the value slices of one head form a cluster: the output normalisation adds their
+        // row sums through distributed shared memory
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 1;
+        attr[0].val.clusterDim.y = static_cast<unsigned>(dv / kDvs);
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    return cudaLaunchKernelEx(&cfg, kern, (const IT *)q, (const IT *)k, (const IT *)v, beta, g, o, oo.bf16 ? 1 : 0,
+                              oo.dskip, oo.xnorm, oo.xw, oo.xeps, s0, s_final, cu, H, L, dv, chunk, scale, err) ==
+                   cudaSuccess
+               ? GDN_OK
+               : GDN_ERR_CUDA;
+}
+
 template <int DK, typename IT, bool DELTA, bool VEC>
 gdn_status_t launch_simt_t(const void *q, const void *k, const void *v, const float *beta,
                            const float *g, void *o, const float *s0, float *s_final, const int *cu,
                            int BH, int H, int L, int dv, int chunk, float scale, FwdOpts oo, unsigned *err,
                            cudaStream_t stream) {
-    auto kern = simt_chunk_fwd_kernel<DK, IT, DELTA, VEC>;
-    const int smem = (int)sizeof(SimtSmem<DK, VEC>);
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-        return GDN_ERR_CUDA;
-    dim3 grid(BH, dv / kDvs);
-    kern<<<grid, kSimtThreads, smem, stream>>>((const IT *)q, (const IT *)k, (const IT *)v, beta, g,
-                                               o, oo.bf16 ? 1 : 0, oo.dskip, s0, s_final, cu, H, L, dv,
-                                               chunk, scale, err);
-    return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+    if (oo.xnorm != kXNormNone)
+        return launch_simt_x<DK, IT, DELTA, VEC, true>(q, k, v, beta, g, o, s0, s_final, cu, BH, H, L, dv, chunk,
+                                                       scale, oo, err, stream);
+    return launch_simt_x<DK, IT, DELTA, VEC, false>(q, k, v, beta, g, o, s0, s_final, cu, BH, H, L, dv, chunk, scale,
+                                                    oo, err, stream);
 }
 
 }  // namespace

@@ -63,7 +63,8 @@ constexpr int kTP = 68;
 constexpr uint32_t P_R = P_TF + 64 * kTP * 4; // 4 x 16 x 16 fp32 per-warp block scratch
 constexpr uint32_t P_VEC = P_R + 4096;        // 2 x gate values
 // ---- both: barriers at the same offset (remote arrivals address them by offset) -----
-constexpr uint32_t OFF_BAR = C_SLOT + kSlots * kSlotBytes;
+constexpr uint32_t C_XN = C_SLOT + kSlots * kSlotBytes;   // chain CTA: output-normalisation scratch
+constexpr uint32_t OFF_BAR = C_XN + 1536;
 constexpr uint32_t kSmemBytes = OFF_BAR + 512;
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;  // slack to align the base to 1024 B
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
@@ -277,8 +278,8 @@ tc_gdn_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             // ================================================================ state group
             const int j = tid - kGroupS * 32;                // = TMEM lane (key row j / value column v)
             const bool lead = (j == 0);
-            // D-skip weight of value column j (head zc mod H: dense and packed grids alike)
-            const float dj = (OPTS && out.v) ? out.dskip[(zc % H) * kD + j] : 0.f;
+            const int head = zc % H;                     // head of this row (dense and packed grids)
+            float *xn = reinterpret_cast<float *>(smem + C_XN);
             const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
             {
                 const float *src = s0 ? s0 + (static_cast<size_t>(bh) * kD + j) * kD : nullptr;
@@ -355,7 +356,7 @@ tc_gdn_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     if (c + 2 < nchunks && lead)
                         mbar_arrive_cluster(mapa_shared(smem_u32(&bars[B_SFREE + (((c - 1) >> 1) & 1)]), 1 + (c & 1)));
                     tc_fence_after();
-                    store_out_col<OPTS>(trow + TM_O + (cp & 1) * 64, out, (row0 + static_cast<size_t>(cp) * kC) * kD + j, kC, dj);
+                    store_out_col<OPTS>(trow + TM_O + (cp & 1) * 64, out, (row0 + static_cast<size_t>(cp) * kC) * kD + j, kC, head, j, kBarS, xn);
                     done = c;
                 }
                 // ---- Ut^T row v -> Ut operand (K-major, rows v)
@@ -378,7 +379,7 @@ tc_gdn_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 if (ctl.group_wait(B_CDONE + (cp & 1), (cp >> 1) & 1, kBarS, lead)) {
                     tc_fence_after();
                     store_out_col<OPTS>(trow + TM_O + (cp & 1) * 64, out, (row0 + static_cast<size_t>(cp) * kC) * kD + j,
-                                  L - cp * kC, dj);
+                                  L - cp * kC, head, j, kBarS, xn);
                     done = nchunks;
                 }
             }
@@ -848,12 +849,12 @@ gdn_status_t launch_tc_gdn_cluster(const void *q, const void *k, const void *v, 
                                    void *o, const float *s0, float *s_final, const int *cu, int B, int H, int L,
                                    float scale, FwdOpts oo, cudaStream_t stream) {
     const int nctas = B * H;                 // one cluster per (sequence, head)
-    const OutArgs out{o, oo.dskip ? static_cast<const __nv_bfloat16 *>(v) : nullptr, oo.dskip, oo.bf16 ? 1 : 0};
+    const OutArgs out = make_out_args(o, v, oo);
     const int rows = cu ? H : B * H;         // rows of the (rows, L) token grid
     CUtensorMap mq, mk, mv;
     if (!make_qkv_map(&mq, q, L, rows) || !make_qkv_map(&mk, k, L, rows) || !make_qkv_map(&mv, v, L, rows))
         return GDN_ERR_CUDA;
-    const bool opts = oo.bf16 || oo.dskip != nullptr;   // the general output epilogue
+    const bool opts = oo.bf16 || oo.dskip != nullptr || oo.xnorm != kXNormNone;   // the general output epilogue
     if (g) return opts ? launch_cl_t<true, true>(mq, mk, mv, beta, g, out, s0, s_final, cu, nctas, H, L, scale, stream)
                        : launch_cl_t<true, false>(mq, mk, mv, beta, g, out, s0, s_final, cu, nctas, H, L, scale, stream);
     return opts ? launch_cl_t<false, true>(mq, mk, mv, beta, g, out, s0, s_final, cu, nctas, H, L, scale, stream)

@@ -35,13 +35,16 @@ __device__ __forceinline__ void st_row16_h(uint32_t tile, uint32_t row, int ch, 
 }
 
 // 64 output rows of one value column from TMEM to HBM (rows >= n are padding), with the
-// output options (fp32 / bf16, D-skip term dj * v) when OPTS, plain fp32 otherwise
+// output options (fp32 / bf16, D-skip term, output normalisation) when OPTS, plain fp32
+// otherwise. With OPTS the whole 128-thread group (thread gt = value column) calls it
+// and meets on bar_id; xn: 384 floats of shared scratch; head indexes the (H, dv) weights.
 template <bool OPTS>
-__device__ __forceinline__ void store_out_col(uint32_t taddr, const OutArgs &out, size_t elem0, int n, float dj) {
+__device__ __forceinline__ void store_out_col(uint32_t taddr, const OutArgs &out, size_t elem0, int n, int head,
+                                              int gt, int bar_id, float *xn) {
     float ov[64];
     ld_cols<64>(taddr, ov);
     if constexpr (OPTS) {
-        store_out_rows(ov, out.o, elem0, n, kD, out.bf16 != 0, dj, out.v);
+        store_out_rows_group(ov, out, elem0, n, head, gt, bar_id, xn, xn + 256);
     } else {
         float *ocol = static_cast<float *>(out.o) + elem0;
 #pragma unroll

@@ -58,7 +58,8 @@ constexpr uint32_t OFF_PG = kStages * kStageBytes;   // 2 x P, K-major 64 x 64 f
 constexpr uint32_t OFF_VEC = OFF_PG + 16384;         // 2 x {G, gamma, d, exp(-G), flag}
 constexpr uint32_t kVecBytes = 1536;
 constexpr int V_G = 0, V_GAM = 64, V_D = 128, V_IG = 192, V_FAST = 256;
-constexpr uint32_t OFF_BAR = OFF_VEC + 2 * kVecBytes;
+constexpr uint32_t OFF_XN = OFF_VEC + 2 * kVecBytes;   // output-normalisation scratch (384 fp32)
+constexpr uint32_t OFF_BAR = OFF_XN + 1536;
 constexpr uint32_t kSmemBytes = OFF_BAR + 512;
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;   // slack to align the base to 1024 B
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
@@ -385,8 +386,8 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         const int v = tid - 256;                          // TMEM lane = value column
         const bool lead = (v == 0);
         const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-        // D-skip weight of value column v (head zc mod H: dense and packed grids alike)
-        const float dv_skip = (OPTS && out.v) ? out.dskip[(zc % H) * kD + v] : 0.f;
+        const int head = zc % H;                          // head of this row (dense and packed grids)
+        float *xn = reinterpret_cast<float *>(smem + OFF_XN);
 #pragma unroll 1
         for (int c = 0; c < nchunks; ++c) {
             const int p = c & 1;
@@ -399,8 +400,8 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             if (lead) mbar_arrive(&bars[B_OFREE + p]);
             const int n = min(kC, L - c * kC);
             if constexpr (OPTS) {
-                store_out_rows(ov, out.o, (row0 + static_cast<size_t>(c) * kC) * kD + v, n, kD, out.bf16 != 0,
-                               dv_skip, out.v);
+                store_out_rows_group(ov, out, (row0 + static_cast<size_t>(c) * kC) * kD + v, n, head, v, kBarOut, xn,
+                                     xn + 256);
             } else {
                 float *ocol = static_cast<float *>(out.o) + (row0 + static_cast<size_t>(c) * kC) * kD + v;
 #pragma unroll
@@ -552,12 +553,12 @@ gdn_status_t launch_tc_la(const void *q, const void *k, const void *v, const flo
                           const float *s0, float *s_final, const int *cu, int B, int H, int L, float scale,
                           FwdOpts oo, cudaStream_t stream) {
     const int nctas = B * H;                 // one CTA per (sequence, head)
-    const OutArgs out{o, oo.dskip ? static_cast<const __nv_bfloat16 *>(v) : nullptr, oo.dskip, oo.bf16 ? 1 : 0};
+    const OutArgs out = make_out_args(o, v, oo);
     const int rows = cu ? H : B * H;         // rows of the (rows, L) token grid
     CUtensorMap mq, mk, mv;
     if (!make_qkv_map(&mq, q, L, rows) || !make_qkv_map(&mk, k, L, rows) || !make_qkv_map(&mv, v, L, rows))
         return GDN_ERR_CUDA;
-    const bool opts = oo.bf16 || oo.dskip != nullptr;   // the general output epilogue
+    const bool opts = oo.bf16 || oo.dskip != nullptr || oo.xnorm != kXNormNone;   // the general output epilogue
     if (g) return opts ? launch_la_t<true, true>(mq, mk, mv, g, out, s0, s_final, cu, nctas, H, L, scale, stream)
                        : launch_la_t<true, false>(mq, mk, mv, g, out, s0, s_final, cu, nctas, H, L, scale, stream);
     return opts ? launch_la_t<false, true>(mq, mk, mv, g, out, s0, s_final, cu, nctas, H, L, scale, stream)

@@ -35,6 +35,8 @@
 #ifndef GDN_H_
 #define GDN_H_
 
+#include <stddef.h>
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -143,11 +145,26 @@ gdn_status_t gdn_chunk_fwd_varlen(const void *q, const void *k, const void *v, c
  *             the per-coordinate form of the scalar gate (GLA-style gates, next to the
  *             scalar gate of page "混合注意力学习(1)", section "Gated DeltaNet"). These
  *             calls run on the fp32 chunk kernel. Any other value: GDN_ERR_INVALID_ARG.
+ *  xnorm      output normalisation (page "LinearAttention 概述", section "The Devil in Linear
+ *             Transformer": the normaliser's denominator is dropped and the output is
+ *             normalised instead, O = XNorm(Q (K^T V))). GDN_XNORM_NONE (0, default),
+ *             GDN_XNORM_RMS: o_t <- w_h (elementwise) o_t / sqrt(mean(o_t^2) + eps), or
+ *             GDN_XNORM_LAYER: o_t <- w_h (elementwise) (o_t - mean(o_t)) / sqrt(var(o_t)
+ *             + eps), over the dv values of each output row of each head (var: mean square
+ *             of the centred row), after the skip term and before the output rounding.
+ *  xnorm_weight  (H, dv) fp32 device pointer, 4-byte aligned, nullable (w = 1).
+ *  xnorm_eps  > 0 and finite when xnorm is set (e.g. 1e-6).
+ *  An unknown xnorm value, or a non-positive eps with xnorm set, returns GDN_ERR_INVALID_ARG.
  */
+typedef enum { GDN_XNORM_NONE = 0, GDN_XNORM_RMS = 1, GDN_XNORM_LAYER = 2 } gdn_xnorm_t;
+
 typedef struct gdn_fwd_opts {
     gdn_dtype_t out_dtype;
     const float *d_skip;
     int g_per_key;
+    int xnorm;                  /* gdn_xnorm_t */
+    const float *xnorm_weight;
+    float xnorm_eps;
 } gdn_fwd_opts_t;
 
 /*
@@ -193,13 +210,43 @@ gdn_status_t gdn_decode_step(const void *q, const void *k, const void *v, const 
  * gdn_decode_step_ex — gdn_decode_step with the options of gdn_fwd_opts_t (opts NULL: the
  * plain call). g_per_key = 1: g is (N, H, dk), row j of each state decays by
  * exp(g[n, h, j]) (o = (diag(alpha) S)^T q' + (q'.k) u, S <- diag(alpha) S + k u^T);
- * out_dtype GDN_BF16: o is bf16 (N, H, dv); d_skip (H, dv): o += d_skip[h] * v.
+ * out_dtype GDN_BF16: o is bf16 (N, H, dv); d_skip (H, dv): o += d_skip[h] * v; xnorm:
+ * the output normalisation of each o row, as in the prefill calls.
  * Validation as for gdn_decode_step, plus the options' own rules.
  */
 gdn_status_t gdn_decode_step_ex(const void *q, const void *k, const void *v, const float *beta,
                                 const float *g, float *state, void *o, int N, int H, int dk, int dv,
                                 float scale, gdn_dtype_t in_dtype, const gdn_fwd_opts_t *opts,
                                 void *cuda_stream);
+
+/*
+ * gdn_chunk_bwd — gradients of the prefill for training on full sequences (page
+ * "混合注意力学习(1)", section "Transformers 就是 RNNs": on the full sequence every gradient
+ * follows from the chain rule through the recurrence). For the loss
+ * sum(o * d_o) + sum(S_final * ds_final) of the operator of lin_attn_chunk_fwd (beta ==
+ * NULL) or gdn_chunk_fwd (beta != NULL), with the same q, k, v, beta, g, s0 and scale:
+ *
+ *  d_o       (B, H, L, dv) fp32, the gradient of o                    device, read
+ *  ds_final  (B, H, dk, dv) fp32, nullable (zero)                     device, read
+ *  dq, dk    (B, H, L, dk) fp32; dv (B, H, L, dv) fp32                device, written
+ *  dbeta     (B, H, L) fp32, required when beta != NULL               device, written
+ *  dg        (B, H, L) fp32 (gradient of the log-decay g), required when g != NULL
+ *  ds0       (B, H, dk, dv) fp32, nullable (not written)              device, written
+ *  workspace device memory of at least gdn_chunk_bwd_workspace_bytes(B, H, L, dk, dv, chunk)
+ *            bytes, 16-byte aligned, owned by the caller; its contents on entry do not
+ *            matter and on return are unspecified. It holds the state at the start of every
+ *            chunk of `chunk` tokens and the recomputed states inside one chunk, per head.
+ *  chunk     1..128: tokens between stored states (a memory / recompute trade-off; the
+ *            result does not depend on it beyond rounding).
+ *  The kernel runs on CUDA cores in fp32 (a reverse-mode pass over the token recurrence).
+ *  Sizes, dtypes and alignment as for the prefill calls; L >= 0 (L == 0: ds0 = ds_final).
+ */
+size_t gdn_chunk_bwd_workspace_bytes(int B, int H, int L, int dk, int dv, int chunk);
+gdn_status_t gdn_chunk_bwd(const void *q, const void *k, const void *v, const float *beta, const float *g,
+                           const float *s0, const float *d_o, const float *ds_final, float *dq, float *dk,
+                           float *dv, float *dbeta, float *dg, float *ds0, void *workspace,
+                           size_t workspace_bytes, int B, int H, int L, int dk_size, int dv_size, int chunk,
+                           float scale, gdn_dtype_t in_dtype, void *cuda_stream);
 
 /* Human-readable name of a status code (static storage, never NULL). */
 const char *gdn_status_str(gdn_status_t status);

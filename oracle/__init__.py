@@ -10,8 +10,12 @@ Functions (each cites the passages it follows in ``gdn_oracle.c``):
                  with Mamba's skip term o_t += D_h v_t, added here in numpy)
   decode_step    one token for many independent heads, state in place (scalar or
                  vector-valued gates, optional skip term)
+  xnorm          the output normalisation of the "Devil in Linear Transformer" form (RMS
+                 or layer normalisation of each output row over dv, with weights (H, dv))
   chunked_fwd    fp64 chunkwise re-derivation (UT/WY form) for invariance tests
   ut_transform   the per-chunk T = (I + A)^-1 factor
+  recurrent_bwd  gradients of the operator (dq, dk, dv, dbeta, dg, ds0) by fp64 autograd of
+                 the token recurrence written out in PyTorch CPU ops
 
 Pins (tests/test_oracle_pins.py) tie these to what the pages fix: the masked
 parallel form, the positions 1-4 cumulative-sum example, the delta rule as one
@@ -104,6 +108,31 @@ def _f64(x) -> Optional[np.ndarray]:
 
 def _ptr(a: Optional[np.ndarray]):
     return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def xnorm(o, kind: str, weight=None, eps: float = 1e-6):
+    """Output normalisation of page "LinearAttention 概述", section "The Devil in Linear
+    Transformer": the normaliser's denominator is dropped and the output is normalised
+    instead, O = XNorm(Q (K^T V)). The page does not fix XNorm's form; the reading taken:
+    each output row o_t of each head is normalised over its dv values,
+      kind "rms":   o_t / sqrt(mean_c o_t[c]^2 + eps)
+      kind "layer": (o_t - mean_c o_t[c]) / sqrt(mean_c (o_t[c] - mean)^2 + eps)
+    then multiplied elementwise by weight[h] (shape (H, dv); None = ones).
+    o: (..., H, L, dv); returns a new float64 array."""
+    o = _f64(o)
+    if kind == "layer":
+        x = o - o.mean(axis=-1, keepdims=True)
+    elif kind == "rms":
+        x = o
+    else:
+        raise ValueError(f"xnorm kind {kind!r}")
+    out = x / np.sqrt((x * x).mean(axis=-1, keepdims=True) + eps)
+    if weight is not None:
+        w = _f64(weight)
+        if o.ndim < 3 or w.shape != (o.shape[-3], o.shape[-1]):
+            raise ValueError(f"xnorm weight: expected (H, dv), got {w.shape}")
+        out = out * w[:, None, :]
+    return out
 
 
 def recurrent_fwd(q, k, v, beta=None, g=None, s0=None, scale: float = 1.0,
@@ -229,6 +258,46 @@ def ut_transform(K, beta, g=None, lib=None):
     if rc:
         raise ValueError("oracle_ut_transform: bad sizes")
     return T
+
+
+def recurrent_bwd(q, k, v, beta=None, g=None, s0=None, do=None, ds_final=None, scale: float = 1.0):
+    """Gradients of the operator (page "混合注意力学习(1)", section "Transformers 就是 RNNs":
+    on the full training sequence every gradient follows from the chain rule through the
+    recurrence; the page's formulas are stripped, so the reading is the exact gradient of
+    the definition). The token recurrence of :func:`recurrent_fwd` (read, blend, write,
+    then read out) written out in fp64 PyTorch CPU ops and differentiated by autograd, for
+    the loss sum(o * do) + sum(S_final * ds_final).
+
+    q, k: (..., L, dk); v, do: (..., L, dv); beta, g: (..., L) or None; s0, ds_final:
+    (..., dk, dv) or None. Returns (o, S_final, grads) with grads a dict of float64 arrays:
+    dq, dk, dv, dbeta (or None), dg (or None), ds0 (zeros when s0 is None)."""
+    import torch
+    t = lambda x: None if x is None else torch.tensor(_f64(x), dtype=torch.float64, requires_grad=True)
+    q_, k_, v_, b_, g_ = map(t, (q, k, v, beta, g))
+    lead = q_.shape[:-2]
+    L, dk = q_.shape[-2:]
+    dv = v_.shape[-1]
+    s0_ = t(s0) if s0 is not None else torch.zeros(lead + (dk, dv), dtype=torch.float64, requires_grad=True)
+    S = s0_
+    outs = []
+    for i in range(L):
+        kt, vt = k_[..., i, :], v_[..., i, :]
+        alpha = torch.exp(g_[..., i]) if g_ is not None else torch.ones(lead, dtype=torch.float64)
+        if b_ is not None:
+            read = torch.einsum("...jc,...j->...c", S, kt)                  # S^T k
+            u = b_[..., i, None] * (vt - alpha[..., None] * read)
+        else:
+            u = vt
+        S = alpha[..., None, None] * S + kt[..., :, None] * u[..., None, :]
+        outs.append(torch.einsum("...jc,...j->...c", S, scale * q_[..., i, :]))
+    o = torch.stack(outs, -2) if L else torch.zeros(lead + (0, dv), dtype=torch.float64)
+    loss = (o * torch.tensor(_f64(do))).sum() if do is not None else o.sum() * 0
+    if ds_final is not None:
+        loss = loss + (S * torch.tensor(_f64(ds_final))).sum()
+    loss.backward()
+    grad = lambda x: None if x is None else (x.grad.numpy().copy() if x.grad is not None else np.zeros(x.shape))
+    grads = {"dq": grad(q_), "dk": grad(k_), "dv": grad(v_), "dbeta": grad(b_), "dg": grad(g_), "ds0": grad(s0_)}
+    return o.detach().numpy(), S.detach().numpy(), grads
 
 
 def max_norm_err(x, ref) -> float:

@@ -56,6 +56,17 @@ bool take_device_error(cudaStream_t stream, unsigned *err) {
     return cudaStreamSynchronize(stream) == cudaSuccess;
 }
 
+int sm_count() {
+    static std::mutex mu;
+    static int sms[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    std::lock_guard<std::mutex> lock(mu);
+    if (sms[dev] == 0 && cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 0;
+    return sms[dev];
+}
+
 long long wait_limit_cycles() { return g_wait_limit.load(std::memory_order_relaxed); }
 
 bool ensure_smem_limit(const void *fn, unsigned bytes) {

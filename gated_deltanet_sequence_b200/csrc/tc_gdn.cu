@@ -25,11 +25,11 @@
 //   warp 1      Gram and W/U issuer: issues whichever of Gram(c+1) / W/U(c) is ready
 //   warp 2      chain issuer: S Q', U - W S, state update, P Ut
 //   warp 3      gate warp: G, gamma, d, exp(-G), beta per chunk (3-buffer ring)
-//   warps 4-7   state group: S^T -> fp16 (and the decay), O^T -> o, Ut^T -> fp16 copies
+//   warps 4-7   state group: S^T -> fp16 (and the decay), O^T -> o, the W operand
+//               (W^T -> fp16), Ut^T -> fp16 copies
 //   warps 8-11  solve group: UT solve of A (16 x 16 diagonal blocks by substitution,
 //               off-diagonal blocks by warp-level tf32 MMA) and the fp16 T factors
-//   warps 12-15 prep group: A / P masks from the Gram, K, V -> fp16, Q -> -Q', and the
-//               W epilogue (W^T -> fp16 operand) one chunk behind
+//   warps 12-15 prep group: A / P masks from the Gram, K, V -> fp16, Q -> -Q'
 // The prep and solve of later chunks run while the chain works on chunk c; every
 // hand-off is an mbarrier with one arrival. Buffers shared by consecutive chunks are
 // multi-buffered (stages and gate values x3, A^T and P x2) with per-buffer barriers, so
@@ -122,7 +122,7 @@ enum : int {
     B_GRAM = 21,     // Gram done -> prep group
     B_GFREE = 22,    // prep group has read the Gram -> Gram/WU issuer
     B_TRDY = 23,     // T factors written -> Gram/WU issuer
-    B_WU = 24,       // W/U done -> prep group (W epilogue), solve group (T buffer free)
+    B_WU = 24,       // W/U done -> state group (W epilogue), solve group (T buffer free)
     B_WRDY = 25,     // W operand written, W^T read -> chain issuer, Gram/WU issuer
     B_SRDY = 26,     // -S^T fp16 written, S^T decayed -> chain issuer
     B_OFREE = 27,    // state group has read O^T -> chain issuer
@@ -435,16 +435,27 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             tc_fence_before();
             named_bar(kBarS, 128);
             if (lead) mbar_arrive(&bars[B_SRDY]);
-            // ---- output of chunk c-1 (complete since its P Ut): read it, release O^T, store
+            // ---- output of chunk c-1 (complete since its P Ut): read it, release O^T; then the
+            //      W epilogue of chunk c (W^T row j = TMEM lane v -> fp16 MN-major W in the V slot
+            //      of its stage, which U has consumed), then store the output tile
+            float ov[64];
             if (c >= 1) {
-                const int cp = c - 1;
-                if (!ctl.group_wait(B_ODONE, cp & 1, kBarS, lead)) break;
+                if (!ctl.group_wait(B_ODONE, (c - 1) & 1, kBarS, lead)) break;
                 tc_fence_after();
-                float ov[64];
                 ld_cols<64>(trow + TM_O, ov);
                 tc_fence_before();
                 named_bar(kBarS, 128);
                 if (lead) mbar_arrive(&bars[B_OFREE]);
+            }
+            if (!ctl.group_wait(B_WU, c & 1, kBarS, lead)) break;
+            tc_fence_after();
+            store_w_row(trow + TM_W, sb + (c % kStages) * kStageBytes + ST_W, v);
+            fence_proxy_async();
+            tc_fence_before();
+            named_bar(kBarS, 128);
+            if (lead) mbar_arrive(&bars[B_WRDY]);
+            if (c >= 1) {
+                const int cp = c - 1;
                 const size_t elem0 = (row0 + static_cast<size_t>(cp) * kC) * kD + v;
                 if constexpr (OPTS) {
                     store_out_rows_group(ov, out, elem0, kC, head, v, kBarS, xn, xn + 256);
@@ -570,15 +581,22 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 float acc[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) acc[i] = (i == cl) ? 1.f : 0.f;
+                // column s2 of A_ii: A[16 bi + i][16 bi + s2] (zero for i <= s2), 16 halves; the
+                // next step's column is loaded while this step's multiply-adds run
+                const uint4 *acol = reinterpret_cast<const uint4 *>(At + 16 * bi * 64 + 16 * bi);
+                uint4 cur0 = acol[0], cur1 = acol[1];
 #pragma unroll
                 for (int s2 = 0; s2 < 15; ++s2) {
+                    uint4 nx0 = cur0, nx1 = cur1;
+                    if (s2 < 14) {
+                        if (s2 + 1 < 7) nx0 = acol[(s2 + 1) * 8];
+                        nx1 = acol[(s2 + 1) * 8 + 1];
+                    }
                     const float xs = acc[s2];
-                    // column s2 of A_ii: A[16 bi + i][16 bi + s2] (zero for i <= s2)
-                    const uint4 *arow = reinterpret_cast<const uint4 *>(At + (16 * bi + s2) * 64 + 16 * bi);
 #pragma unroll
                     for (int k8 = 0; k8 < 2; ++k8) {
                         if (8 * k8 + 7 <= s2) continue;          // rows of this group are not below s2
-                        const uint4 a8 = arow[k8];
+                        const uint4 a8 = k8 == 0 ? cur0 : cur1;
                         const __half2 *h2 = reinterpret_cast<const __half2 *>(&a8);
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
@@ -587,6 +605,8 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                             acc[8 * k8 + 2 * e + 1] = fmaf(-a2.y, xs, acc[8 * k8 + 2 * e + 1]);
                         }
                     }
+                    cur0 = nx0;
+                    cur1 = nx1;
                 }
                 if (lane < 16) {
 #pragma unroll
@@ -653,14 +673,13 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
     } else if (warp >= kGroupM) {
         // ================================================================ prep group
-        // per chunk c: the A / P masks from the Gram, K, V -> fp16 and Q -> -Q' in place;
-        // then the W epilogue of chunk c-1 (W^T -> fp16 MN-major operand in its V slot)
+        // per chunk c: the A / P masks from the Gram, K, V -> fp16 and Q -> -Q' in place
         const int m = tid - kGroupM * 32;                // 0..127 = TMEM lane of the Gram row
         const bool lead = (m == 0);
         const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
 #pragma unroll 1
-        for (int c = 0; c <= nchunks; ++c) {
-            if (c < nchunks) {
+        for (int c = 0; c < nchunks; ++c) {
+            {
                 const int s = c % kStages, p = c & 1;
                 const float *vec = vec_of(c);
                 uint8_t *st = smem + s * kStageBytes;
@@ -680,33 +699,43 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     named_bar(kBarM, 128);                       // every Gram row has been read
                     if (lead) mbar_arrive(&bars[B_GFREE]);
                     const int r = m & 63;
+                    // x[e] <- the masked, decayed Gram value of column e, with every factor read
+                    // from shared memory before the first store (so no store orders a reload)
+                    {
+                        const float br = vec[V_B + r], gr = vec[V_GAM + r], Gr = vec[V_G + r];
+                        const float lead_r = m < 64 ? br * gr : scale * gr;
+                        const int lim = m < 64 ? r : r + 1;     // A: s < r; P: s <= r
+                        if (fast) {
+#pragma unroll
+                            for (int e4 = 0; e4 < 64; e4 += 4) {
+                                const float4 ig = *reinterpret_cast<const float4 *>(vec + V_IG + e4);
+                                x[e4] = e4 < lim ? lead_r * ig.x * x[e4] : 0.f;
+                                x[e4 + 1] = e4 + 1 < lim ? lead_r * ig.y * x[e4 + 1] : 0.f;
+                                x[e4 + 2] = e4 + 2 < lim ? lead_r * ig.z * x[e4 + 2] : 0.f;
+                                x[e4 + 3] = e4 + 3 < lim ? lead_r * ig.w * x[e4 + 3] : 0.f;
+                            }
+                        } else {
+                            const float f = m < 64 ? br : scale;
+#pragma unroll
+                            for (int e4 = 0; e4 < 64; e4 += 4) {
+                                const float4 gs = *reinterpret_cast<const float4 *>(vec + V_G + e4);
+                                x[e4] = e4 < lim ? f * __expf(Gr - gs.x) * x[e4] : 0.f;
+                                x[e4 + 1] = e4 + 1 < lim ? f * __expf(Gr - gs.y) * x[e4 + 1] : 0.f;
+                                x[e4 + 2] = e4 + 2 < lim ? f * __expf(Gr - gs.z) * x[e4 + 2] : 0.f;
+                                x[e4 + 3] = e4 + 3 < lim ? f * __expf(Gr - gs.w) * x[e4 + 3] : 0.f;
+                            }
+                        }
+                    }
                     if (m < 64) {
                         __half *At = reinterpret_cast<__half *>(smem + OFF_AT + p * kAtBytes);   // At[s*64+r]
-                        if (fast) {
-                            const float lead_r = vec[V_B + r] * vec[V_GAM + r];
 #pragma unroll
-                            for (int e = 0; e < 64; ++e)
-                                At[e * 64 + r] = __float2half_rn(e < r ? lead_r * vec[V_IG + e] * x[e] : 0.f);
-                        } else {
-                            const float br = vec[V_B + r], Gr = vec[V_G + r];
-#pragma unroll
-                            for (int e = 0; e < 64; ++e)
-                                At[e * 64 + r] = __float2half_rn(e < r ? br * __expf(Gr - vec[V_G + e]) * x[e] : 0.f);
-                        }
+                        for (int e = 0; e < 64; ++e) At[e * 64 + r] = __float2half_rn(x[e]);
                     } else {
-                        const float lead_r = scale * vec[V_GAM + r], Gr = vec[V_G + r];
 #pragma unroll
-                        for (int ch = 0; ch < 8; ++ch) {
-                            float pv[8];
-#pragma unroll
-                            for (int e8 = 0; e8 < 8; ++e8) {
-                                const int e = 8 * ch + e8;
-                                const float f = fast ? lead_r * vec[V_IG + e] : scale * __expf(Gr - vec[V_G + e]);
-                                pv[e8] = e <= r ? f * x[e] : 0.f;
-                            }
-                            st_shared_v4(sb + OFF_PG + p * 8192 + sw128(r, ch), pack_h2(pv[0], pv[1]), pack_h2(pv[2], pv[3]),
-                                         pack_h2(pv[4], pv[5]), pack_h2(pv[6], pv[7]));
-                        }
+                        for (int ch = 0; ch < 8; ++ch)
+                            st_shared_v4(sb + OFF_PG + p * 8192 + sw128(r, ch), pack_h2(x[8 * ch], x[8 * ch + 1]),
+                                         pack_h2(x[8 * ch + 2], x[8 * ch + 3]), pack_h2(x[8 * ch + 4], x[8 * ch + 5]),
+                                         pack_h2(x[8 * ch + 6], x[8 * ch + 7]));
                     }
                 }
                 fence_proxy_async();
@@ -743,9 +772,12 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         offs[i] = ST_Q0 + (idx >> 9) * 16384u + (idx & 511u) * 16u;
                         xv[i] = *reinterpret_cast<const uint4 *>(st + offs[i]);
                     }
+                    float fq[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) fq[i] = -scale * vec[V_GAM + ((offs[i] & 8191u) >> 7)];
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
-                        const float f = -scale * vec[V_GAM + ((offs[i] & 8191u) >> 7)];
+                        const float f = fq[i];
                         xv[i].x = pack_h2(f * bf_lo(xv[i].x), f * bf_hi(xv[i].x));
                         xv[i].y = pack_h2(f * bf_lo(xv[i].y), f * bf_hi(xv[i].y));
                         xv[i].z = pack_h2(f * bf_lo(xv[i].z), f * bf_hi(xv[i].z));
@@ -756,18 +788,6 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 fence_proxy_async();
                 named_bar(kBarM, 128);
                 if (lead) mbar_arrive(&bars[B_CONV + s]);
-            }
-            if (c >= 1) {
-                // ---- W epilogue of chunk c-1: W^T row j (TMEM lane m) -> fp16 MN-major W in the
-                //      V slot of its stage (U has been formed from V by the same W/U)
-                const int cw = c - 1;
-                if (!ctl.group_wait(B_WU, cw & 1, kBarM, lead)) break;
-                tc_fence_after();
-                store_w_row(trow + TM_W, sb + (cw % kStages) * kStageBytes + ST_W, m);
-                fence_proxy_async();
-                tc_fence_before();
-                named_bar(kBarM, 128);
-                if (lead) mbar_arrive(&bars[B_WRDY]);
             }
         }
     }

@@ -25,8 +25,6 @@
 // Warp roles. Chain CTA (rank 0): warp 0 TMA (Q, K, V, 2 stages), warp 2 UMMA issuer,
 // warps 4-7 state group, warps 8-11 tile converter (K, V -> fp16, Q -> Q'). Prep CTAs:
 // warp 0 TMA (K, Q), warp 1 Gram issuer, warp 3 gate warp, warps 8-15 prep group.
-#include <mutex>
-
 #include "tc_gdn_parts.cuh"
 
 namespace gdn {
@@ -834,16 +832,7 @@ gdn_status_t launch_cl_t(const CUtensorMap &mq, const CUtensorMap &mk, const CUt
 
 }  // namespace
 
-bool tc_gdn_cluster_fits(int nctas) {
-    static std::mutex mu;
-    static int sms[64] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
-    std::lock_guard<std::mutex> lock(mu);
-    if (sms[dev] == 0 && cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return false;
-    return static_cast<long long>(nctas) * kCluster <= sms[dev];
-}
+bool tc_gdn_cluster_fits(int nctas) { return static_cast<long long>(nctas) * kCluster <= sm_count(); }
 
 gdn_status_t launch_tc_gdn_cluster(const void *q, const void *k, const void *v, const float *beta, const float *g,
                                    void *o, const float *s0, float *s_final, const int *cu, int B, int H, int L,

@@ -305,3 +305,19 @@ def test_one_cta_form_small_lengths(lib, mode, L):
                                   sl(inp["s0"]))
     check(o[:, heads].numpy(), ro, TOL[torch.bfloat16], f"o {mode} L={L}")
     check(sf[:, heads].numpy(), rs, TOL[torch.bfloat16], f"S {mode} L={L}")
+
+
+@pytest.mark.parametrize("mode", ["plain", "gated"])
+def test_linear_attention_both_forms(lib, mode):
+    # up to half the SM count of (sequence, head) pairs take the pair form (two CTAs per
+    # head, the state split by key rows); 80 heads take the one-CTA form. Both against the
+    # oracle on sampled heads, ragged length.
+    for H in (4, 80):
+        inp = _inputs(1, H, 200, 128, 128, mode, torch.bfloat16, True, seed=6100 + H)
+        o, sf = gpu_prefill(lib, inp)
+        heads = [0, H // 2, H - 1]
+        sl = lambda x: None if x is None else x[:, heads]
+        ro, rs = oracle.recurrent_fwd(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]), sl(inp["beta"]), sl(inp["g"]),
+                                      sl(inp["s0"]))
+        check(o[:, heads].numpy(), ro, TOL[torch.bfloat16], f"o {mode} H={H}")
+        check(sf[:, heads].numpy(), rs, TOL[torch.bfloat16], f"S {mode} H={H}")

@@ -24,7 +24,7 @@ GDN_F32, GDN_BF16 = 0, 1
 EXPORTS = ("lin_attn_chunk_fwd", "gdn_chunk_fwd", "lin_attn_chunk_fwd_varlen", "gdn_chunk_fwd_varlen",
            "lin_attn_chunk_fwd_ex", "gdn_chunk_fwd_ex", "gdn_decode_step", "gdn_decode_step_ex",
            "gdn_status_str", "gdn_sync_status", "gdn_set_wait_limit_for_testing", "gdn_version",
-           "gdn_chunk_bwd", "gdn_chunk_bwd_workspace_bytes")
+           "gdn_chunk_bwd", "gdn_chunk_bwd_workspace_bytes", "gdn_chunk_bwd_noalloc")
 
 
 GDN_XNORM = {None: 0, "rms": 1, "layer": 2}
@@ -68,6 +68,8 @@ def _load() -> ctypes.CDLL:
     lib.gdn_chunk_bwd_workspace_bytes.restype = Z
     lib.gdn_chunk_bwd.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, Z, I, I, I, I, I, I, F, I, P]
     lib.gdn_chunk_bwd.restype = ctypes.c_int
+    lib.gdn_chunk_bwd_noalloc.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
+    lib.gdn_chunk_bwd_noalloc.restype = ctypes.c_int
     lib.gdn_set_wait_limit_for_testing.restype = None
     for f in (lib.lin_attn_chunk_fwd, lib.gdn_chunk_fwd, lib.lin_attn_chunk_fwd_varlen,
               lib.gdn_chunk_fwd_varlen, lib.lin_attn_chunk_fwd_ex, lib.gdn_chunk_fwd_ex,

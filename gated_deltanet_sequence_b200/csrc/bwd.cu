@@ -23,6 +23,8 @@
 // columns (float4) of RPT key rows strided by the number of row groups (the decode
 // step's tiling), for S and for Lambda alike; row reductions are warp shuffles over the
 // column groups of a row group, column reductions go through shared memory.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace gdn {
@@ -308,4 +310,46 @@ gdn_status_t launch_bwd(const void *q, const void *k, const void *v, const float
                                         dv_, chunk, scale, stream);
 }
 
+// ---------------------------------------------------------------- no-allocation variant
+// Workspace of gdn_chunk_bwd_noalloc: one fixed array in the library's static device memory.
+// Every device that loads the library holds it until the process exits; every call of the
+// entry point on a device shares it.
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;   // 16 MiB
+static __device__ __align__(256) float g_bwd_scratch[kNoAllocScratchBytes / sizeof(float)];
+
+// Device address of g_bwd_scratch on the current device, looked up once per device (with
+// that device current); nullptr if the lookup fails. In host code the array's name is only a
+// host-side stand-in, so kernels must be given this address, never the name.
+float *bwd_scratch_address() {
+    static std::mutex mu;
+    static float *addr[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_bwd_scratch) != cudaSuccess || p == nullptr) return nullptr;
+        addr[dev] = static_cast<float *>(p);
+    }
+    return addr[dev];
+}
+}  // namespace
+
 }  // namespace gdn
+
+extern "C" gdn_status_t gdn_chunk_bwd_noalloc(const void *q, const void *k, const void *v, const float *beta,
+                                              const float *g, const float *s0, const float *d_o,
+                                              const float *ds_final, float *dq, float *dk, float *dv,
+                                              float *dbeta, float *dg, float *ds0, int B, int H, int L,
+                                              int dk_size, int dv_size, int chunk, float scale,
+                                              gdn_dtype_t in_dtype, void *cuda_stream) {
+    const size_t need = gdn_chunk_bwd_workspace_bytes(B, H, L, dk_size, dv_size, chunk);
+    if (need == 0) return gdn_chunk_bwd(q, k, v, beta, g, s0, d_o, ds_final, dq, dk, dv, dbeta, dg, ds0, nullptr, 0,
+                                        B, H, L, dk_size, dv_size, chunk, scale, in_dtype, cuda_stream);
+    if (need > gdn::kNoAllocScratchBytes) return GDN_ERR_UNSUPPORTED;
+    float *ws = gdn::bwd_scratch_address();
+    if (!ws) return GDN_ERR_CUDA;
+    return gdn_chunk_bwd(q, k, v, beta, g, s0, d_o, ds_final, dq, dk, dv, dbeta, dg, ds0, ws, gdn::kNoAllocScratchBytes,
+                         B, H, L, dk_size, dv_size, chunk, scale, in_dtype, cuda_stream);
+}

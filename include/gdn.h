@@ -248,6 +248,33 @@ gdn_status_t gdn_chunk_bwd(const void *q, const void *k, const void *v, const fl
                            size_t workspace_bytes, int B, int H, int L, int dk_size, int dv_size, int chunk,
                            float scale, gdn_dtype_t in_dtype, void *cuda_stream);
 
+/*
+ * gdn_chunk_bwd_noalloc — gdn_chunk_bwd for callers that cannot allocate device memory:
+ * same arguments and results, without the workspace. (This entry point has no counterpart
+ * in the pages; it is a deployment convenience of this library.) Some callers have no
+ * allocator to hand when they run the backward — a plugin interface that passes only
+ * input and output buffers, or a runtime whose allocator has reserved all device memory
+ * up front so that a cudaMalloc would fail or fragment it — and cannot size and pass the
+ * workspace that gdn_chunk_bwd needs.
+ *
+ *  Workspace: a fixed 16 MiB array in the library's static device memory (every device
+ *  that loads the library holds it until the process exits). A call whose
+ *  gdn_chunk_bwd_workspace_bytes(B, H, L, dk, dv, chunk) exceeds 16 MiB returns
+ *  GDN_ERR_UNSUPPORTED and enqueues nothing (e.g. 2 heads of 4096 tokens at d = 128,
+ *  chunk 64, need 16 MiB; use gdn_chunk_bwd for larger calls).
+ *  The entry point calls no cudaMalloc, cudaFree or other allocating routine. Its first
+ *  call on a device looks up the array's device address (cudaGetSymbolAddress, with that
+ *  device current); make that first call before any stream capture.
+ *  Every call on a device shares the array and leaves its last contents there (the backward
+ *  writes every word it reads, so nothing needs clearing). Calls that overlap on the GPU
+ *  race on the array: serialise them (one stream, or events between streams).
+ */
+gdn_status_t gdn_chunk_bwd_noalloc(const void *q, const void *k, const void *v, const float *beta,
+                                   const float *g, const float *s0, const float *d_o, const float *ds_final,
+                                   float *dq, float *dk, float *dv, float *dbeta, float *dg, float *ds0,
+                                   int B, int H, int L, int dk_size, int dv_size, int chunk, float scale,
+                                   gdn_dtype_t in_dtype, void *cuda_stream);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 const char *gdn_status_str(gdn_status_t status);
 

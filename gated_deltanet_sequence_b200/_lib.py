@@ -24,7 +24,8 @@ GDN_F32, GDN_BF16 = 0, 1
 EXPORTS = ("lin_attn_chunk_fwd", "gdn_chunk_fwd", "lin_attn_chunk_fwd_varlen", "gdn_chunk_fwd_varlen",
            "lin_attn_chunk_fwd_ex", "gdn_chunk_fwd_ex", "gdn_decode_step", "gdn_decode_step_ex",
            "gdn_status_str", "gdn_sync_status", "gdn_set_wait_limit_for_testing", "gdn_version",
-           "gdn_chunk_bwd", "gdn_chunk_bwd_workspace_bytes", "gdn_chunk_bwd_noalloc")
+           "gdn_chunk_bwd", "gdn_chunk_bwd_workspace_bytes", "gdn_chunk_bwd_noalloc", "gdn_state_compose",
+           "gdn_state_identity")
 
 
 GDN_XNORM = {None: 0, "rms": 1, "layer": 2}
@@ -71,6 +72,10 @@ def _load() -> ctypes.CDLL:
     lib.gdn_chunk_bwd_noalloc.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
     lib.gdn_chunk_bwd_noalloc.restype = ctypes.c_int
     lib.gdn_set_wait_limit_for_testing.restype = None
+    lib.gdn_state_compose.argtypes = [P, P, P, P, F, I, I, P]
+    lib.gdn_state_compose.restype = ctypes.c_int
+    lib.gdn_state_identity.argtypes = [P, F, I, I, P]
+    lib.gdn_state_identity.restype = ctypes.c_int
     for f in (lib.lin_attn_chunk_fwd, lib.gdn_chunk_fwd, lib.lin_attn_chunk_fwd_varlen,
               lib.gdn_chunk_fwd_varlen, lib.lin_attn_chunk_fwd_ex, lib.gdn_chunk_fwd_ex,
               lib.gdn_decode_step, lib.gdn_decode_step_ex, lib.gdn_sync_status, lib.gdn_version):
@@ -376,3 +381,38 @@ def gdn_chunk_bwd(q, k, v, beta, g, d_o, s0=None, ds_final=None, chunk: int = 64
 def gdn_chunk_bwd_workspace_bytes(B: int, H: int, L: int, dk: int, dv: int, chunk: int = 64) -> int:
     """Bytes of device workspace gdn_chunk_bwd needs (0 for unsupported sizes)."""
     return int(lib.gdn_chunk_bwd_workspace_bytes(B, H, L, dk, dv, chunk))
+
+
+def _states(name, t, required=True):
+    """A batch of square fp32 states (..., d, d) on a CUDA device; returns (count, d)."""
+    if t is None:
+        if required:
+            raise ValueError(f"{name} is required")
+        return None
+    if t.dim() < 2 or t.shape[-1] != t.shape[-2]:
+        raise ValueError(f"{name}: expected (..., d, d), got {tuple(t.shape)}")
+    _check(name, t, tuple(t.shape), torch.float32)
+    d = t.shape[-1]
+    return t.numel() // (d * d) if d else 0, d
+
+
+def gdn_state_compose(mn, n, s_in, out, lam: float = 1.0, stream=None):
+    """out = ((lam M + N) - N) / lam s_in + N for a batch of d x d states (the composition step
+    of the sequence-split prefill: mn the end states of runs from lam * I, n those from 0;
+    s_in None: out = N). mn, n, s_in, out: same shape (..., d, d) fp32 on one device; out must
+    not overlap the others. Returns out."""
+    count, d = _states("out", out)
+    _check("mn", mn, tuple(out.shape), torch.float32, out.device)
+    _check("n", n, tuple(out.shape), torch.float32, out.device)
+    _check("s_in", s_in, tuple(out.shape), torch.float32, out.device, required=False)
+    st = lib.gdn_state_compose(_ptr(mn), _ptr(n), _ptr(s_in), _ptr(out), float(lam), count, d, _stream(stream))
+    _raise("gdn_state_compose", st)
+    return out
+
+
+def gdn_state_identity(s, value: float = 1.0, stream=None):
+    """Write value * I into every d x d state of ``s`` ((..., d, d) fp32). Returns s."""
+    count, d = _states("s", s)
+    st = lib.gdn_state_identity(_ptr(s), float(value), count, d, _stream(stream))
+    _raise("gdn_state_identity", st)
+    return s

@@ -239,4 +239,30 @@ gdn_status_t gdn_chunk_bwd(const void *q, const void *k, const void *v, const fl
                            in_dtype, static_cast<cudaStream_t>(cuda_stream));
 }
 
+gdn_status_t gdn_state_compose(const float *mn, const float *n, const float *s_in, float *s_out, float lambda,
+                               int count, int d, void *cuda_stream) {
+    if (count < 0 || !isfinite(lambda) || lambda == 0.f || !isfinite(1.f / lambda)) return GDN_ERR_INVALID_ARG;
+    if (!head_dim_ok(d)) return GDN_ERR_UNSUPPORTED;
+    if (count == 0) return GDN_OK;
+    if (!mn || !n || !s_out || !aligned16(mn) || !aligned16(n) || !aligned16(s_out) || !opt_aligned16(s_in))
+        return GDN_ERR_INVALID_ARG;
+    if ((double)count * d * d > 9.0e18 || count > 2147483647 / 4) return GDN_ERR_INVALID_ARG;
+    // s_out is written while mn, n and s_in are still being read by other CTAs
+    const size_t bytes = static_cast<size_t>(count) * d * d * sizeof(float);
+    auto overlaps = [&](const float *a) {
+        const char *x = reinterpret_cast<const char *>(a), *y = reinterpret_cast<const char *>(s_out);
+        return a && x < y + bytes && y < x + bytes;
+    };
+    if (overlaps(mn) || overlaps(n) || overlaps(s_in)) return GDN_ERR_INVALID_ARG;
+    return gdn::launch_state_compose(mn, n, s_in, s_out, lambda, count, d, static_cast<cudaStream_t>(cuda_stream));
+}
+
+gdn_status_t gdn_state_identity(float *s, float value, int count, int d, void *cuda_stream) {
+    if (count < 0 || !isfinite(value)) return GDN_ERR_INVALID_ARG;
+    if (!head_dim_ok(d)) return GDN_ERR_UNSUPPORTED;
+    if (count == 0) return GDN_OK;
+    if (!s || !aligned16(s)) return GDN_ERR_INVALID_ARG;
+    return gdn::launch_state_identity(s, value, count, d, static_cast<cudaStream_t>(cuda_stream));
+}
+
 }  // extern "C"

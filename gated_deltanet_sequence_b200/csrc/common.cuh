@@ -225,4 +225,9 @@ gdn_status_t launch_bwd(const void *q, const void *k, const void *v, const float
                         const float *s0, const float *dout, const float *dsf, float *dq, float *dk, float *dv,
                         float *dbeta, float *dg, float *ds0, float *ws, int B, int H, int L, int dk_, int dv_,
                         int chunk, float scale, gdn_dtype_t in_dtype, cudaStream_t stream);
+// Sequence-split prefill: s_out = ((lambda M + N) - N) / lambda s_in + N for `count` d x d
+// states, and scaled identity states (value on the diagonal).
+gdn_status_t launch_state_compose(const float *mn, const float *n, const float *s_in, float *s_out, float lambda,
+                                  int count, int d, cudaStream_t stream);
+gdn_status_t launch_state_identity(float *s, float value, int count, int d, cudaStream_t stream);
 }  // namespace gdn

@@ -20,12 +20,6 @@ gdn_status_t launch_tc_gdn_cluster(const void *q, const void *k, const void *v, 
                                    const int *cu, int B, int H, int L, float scale, FwdOpts oo,
                                    cudaStream_t stream);
 bool tc_gdn_cluster_fits(int nctas);
-// Pair form of linear attention (two CTAs per (sequence, head), the state split by key rows);
-// same arguments and result (within rounding) as launch_tc_la. launch_tc_la takes it when
-// every pair fits on the device at once (2 x B*H <= SM count).
-gdn_status_t launch_tc_la_pair(const void *q, const void *k, const void *v, const float *g, void *o,
-                               const float *s0, float *s_final, const int *cu, int B, int H, int L, float scale,
-                               FwdOpts oo, cudaStream_t stream);
 // Number of SMs of the current device (cached per device); 0 on error.
 int sm_count();
 gdn_status_t launch_tc_la(const void *q, const void *k, const void *v, const float *g, void *o,

@@ -553,9 +553,6 @@ gdn_status_t launch_tc_la(const void *q, const void *k, const void *v, const flo
                           const float *s0, float *s_final, const int *cu, int B, int H, int L, float scale,
                           FwdOpts oo, cudaStream_t stream) {
     const int nctas = B * H;                 // one CTA per (sequence, head)
-    // few (sequence, head) pairs: two CTAs per pair, the state split by key rows
-    if (2LL * nctas <= sm_count())
-        return launch_tc_la_pair(q, k, v, g, o, s0, s_final, cu, B, H, L, scale, oo, stream);
     const OutArgs out = make_out_args(o, v, oo);
     const int rows = cu ? H : B * H;         // rows of the (rows, L) token grid
     CUtensorMap mq, mk, mv;

@@ -275,6 +275,37 @@ gdn_status_t gdn_chunk_bwd_noalloc(const void *q, const void *k, const void *v, 
                                    int B, int H, int L, int dk_size, int dv_size, int chunk, float scale,
                                    gdn_dtype_t in_dtype, void *cuda_stream);
 
+/*
+ * Sequence-split (context-parallel) prefill: the segments of a long sequence run at once
+ * (on several devices, or as the sequences of one packed launch). Over a segment the
+ * token recurrence is affine in the state that enters it (page "混合注意力学习(1)",
+ * section "Gated DeltaNet": each token maps the key-row state by
+ * S -> alpha (I - beta k k^T) S + beta k v^T; plain and gated linear attention drop the
+ * erase term): S_out = M S_in + N, with M the ordered product of the segment's token maps
+ * and N the segment's end state from a zero start. With dk = dv = d, a prefill of the
+ * segment from s0 = lambda I ends in lambda M + N and one from s0 = 0 ends in N; composing
+ * these pairs in segment order gives the state entering each segment, from which a last
+ * prefill of the segment gives its outputs. A large lambda (a power of two, e.g. 256) keeps
+ * the rounding of N, which the composition subtracts, small next to M; it must keep
+ * lambda M + N inside the prefill's fp16 operand range (|entries| well below 65504).
+ *
+ * gdn_state_compose — s_out = ((lambda M + N) - N) / lambda s_in + N for `count` states, fp32:
+ *  mn        (count, d, d) fp32, the end states from s0 = lambda I      device, read
+ *  n         (count, d, d) fp32, the end states from s0 = 0 (N)         device, read
+ *  s_in      (count, d, d) fp32, nullable (zero: s_out = N)             device, read
+ *  s_out     (count, d, d) fp32, must not overlap mn, n or s_in         device, written
+ *  lambda    the diagonal of the s0 of the mn runs; finite, nonzero, 1/lambda finite
+ *  d in {64, 128}; count >= 0 (0: nothing is enqueued); pointers 16-byte aligned.
+ *  Returns GDN_ERR_INVALID_ARG for a NULL/misaligned pointer, an overlap or a bad lambda,
+ *  GDN_ERR_UNSUPPORTED for another d.
+ *
+ * gdn_state_identity — writes value * I into `count` d x d fp32 states at `s` (the initial
+ *  states of the s0 = lambda I runs); value finite; d in {64, 128}; s 16-byte aligned.
+ */
+gdn_status_t gdn_state_compose(const float *mn, const float *n, const float *s_in, float *s_out, float lambda,
+                               int count, int d, void *cuda_stream);
+gdn_status_t gdn_state_identity(float *s, float value, int count, int d, void *cuda_stream);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 const char *gdn_status_str(gdn_status_t status);
 

@@ -28,7 +28,8 @@ def test_header_declares_the_boundary():
     names = _declared_functions()
     for want in ("lin_attn_chunk_fwd", "gdn_chunk_fwd", "lin_attn_chunk_fwd_varlen", "gdn_chunk_fwd_varlen",
                  "lin_attn_chunk_fwd_ex", "gdn_chunk_fwd_ex", "gdn_decode_step", "gdn_decode_step_ex",
-                 "gdn_status_str", "gdn_sync_status", "gdn_set_wait_limit_for_testing", "gdn_version"):
+                 "gdn_status_str", "gdn_sync_status", "gdn_set_wait_limit_for_testing", "gdn_version",
+                 "gdn_chunk_bwd", "gdn_chunk_bwd_workspace_bytes", "gdn_state_compose", "gdn_state_identity"):
         assert want in names
 
 
@@ -197,3 +198,25 @@ def test_decode_ex_rejects_bad_arguments(lib, kw, want):
                                     P(a["o"]), a["N"], a["H"], a["dk"], a["dv"], a["scale"], a["dt"],
                                     ctypes.byref(opts), None)
     assert st == want
+
+
+def test_state_compose_and_identity_validate_on_the_host(lib):
+    P = ctypes.c_void_p
+    one = 128 * 128 * 4                                  # bytes of one d = 128 state
+    mn, n, out = P(FAKE), P(FAKE + 2 * one), P(FAKE + 4 * one)
+    compose, identity = lib.lib.gdn_state_compose, lib.lib.gdn_state_identity
+    assert compose(mn, n, None, out, 1.0, 1, 96, None) == 2            # d outside {64, 128}
+    assert compose(mn, n, None, out, 1.0, -1, 128, None) == 1
+    assert compose(mn, n, None, out, 0.0, 1, 128, None) == 1            # lambda 0
+    assert compose(mn, n, None, out, float("inf"), 1, 128, None) == 1
+    assert compose(mn, n, None, out, 1e-45, 1, 128, None) == 1          # 1 / lambda overflows
+    assert compose(None, n, None, out, 1.0, 1, 128, None) == 1
+    assert compose(P(FAKE + 4), n, None, out, 1.0, 1, 128, None) == 1   # misaligned
+    assert compose(mn, n, P(FAKE + 4 * one + 64), out, 1.0, 1, 128, None) == 1   # s_in overlaps s_out
+    assert compose(mn, n, None, P(FAKE + one // 2), 1.0, 1, 128, None) == 1      # s_out overlaps mn
+    assert compose(mn, n, None, out, 1.0, 0, 128, None) == 0           # nothing to do
+    assert identity(P(FAKE), 1.0, 1, 32, None) == 2
+    assert identity(P(FAKE + 8), 1.0, 1, 64, None) == 1
+    assert identity(None, 1.0, 1, 64, None) == 1
+    assert identity(P(FAKE), float("nan"), 1, 64, None) == 1
+    assert identity(P(FAKE), 1.0, 0, 64, None) == 0

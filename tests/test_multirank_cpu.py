@@ -30,7 +30,10 @@ def _worker(rank, world, port, case, q):
     sys.path.insert(0, ROOT)
     import torch
     import torch.distributed as dist
-    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=10))
+    # a short timeout where a rank is meant to die; elsewhere room for a loaded machine (rank 0
+    # times the oracle while rank 1 waits in the barrier)
+    pg_timeout = 10 if case == "dead_rank" else 120
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=pg_timeout))
     ok_exit = True
     try:
         import bench

@@ -308,10 +308,9 @@ def test_one_cta_form_small_lengths(lib, mode, L):
 
 
 @pytest.mark.parametrize("mode", ["plain", "gated"])
-def test_linear_attention_both_forms(lib, mode):
-    # up to half the SM count of (sequence, head) pairs take the pair form (two CTAs per
-    # head, the state split by key rows); 80 heads take the one-CTA form. Both against the
-    # oracle on sampled heads, ragged length.
+def test_linear_attention_few_and_many_heads(lib, mode):
+    # a grid far below the SM count (4 heads) and one above half of it (80 heads), against
+    # the oracle on sampled heads, ragged length.
     for H in (4, 80):
         inp = _inputs(1, H, 200, 128, 128, mode, torch.bfloat16, True, seed=6100 + H)
         o, sf = gpu_prefill(lib, inp)

@@ -55,7 +55,7 @@ __device__ __forceinline__ void store_out_col(uint32_t taddr, const OutArgs &out
 
 // W^T row j (TMEM) -> fp16 MN-major W operand in a stage's V slot
 __device__ __forceinline__ void store_w_row(uint32_t trow_x, uint32_t wtile, int j) {
-#pragma unroll
+#pragma unroll 1
     for (int cc = 0; cc < 4; ++cc) {
         float w[16];
         tmem_ld16(trow_x + cc * 16, w);
@@ -82,7 +82,7 @@ __device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&
 template <int KS, typename XF, typename ZF>
 __device__ __forceinline__ void block_mm(float (&acc)[2][4], XF xget, ZF zget, int lane) {
     const int g = lane >> 2, t = lane & 3;
-#pragma unroll
+#pragma unroll 1
     for (int ks = 0; ks < KS; ++ks) {
         const uint32_t a[4] = {to_tf32(xget(g, 8 * ks + t)), to_tf32(xget(g + 8, 8 * ks + t)),
                                to_tf32(xget(g, 8 * ks + t + 4)), to_tf32(xget(g + 8, 8 * ks + t + 4))};

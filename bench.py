@@ -146,9 +146,20 @@ def timed(fn, steps: int, warmup: int, barrier=None):
     return e0.elapsed_time(e1) / steps
 
 
+def kernel_source_hash(cu_name: str) -> str:
+    """sha256[:16] of a kernel's .cu file followed by every shared header of csrc/ (sorted), so
+    a change to the kernel or to any device code it may include changes the hash."""
+    csrc = os.path.join(ROOT, "gated_deltanet_sequence_b200", "csrc")
+    h = hashlib.sha256()
+    for name in [cu_name] + sorted(f for f in os.listdir(csrc) if f.endswith(".cuh")):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
 def traffic_from_profiles(kernel_key: str):
     """DRAM bytes per launch recorded by an ncu capture (profiles/ncu_traffic.txt) when the
-    kernel source is unchanged since the capture (sha256 of its .cu file); else None."""
+    kernel source is unchanged since the capture (kernel_source_hash); else None."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
     if not os.path.exists(path):
         return None
@@ -159,9 +170,7 @@ def traffic_from_profiles(kernel_key: str):
                 src = os.path.join(ROOT, "gated_deltanet_sequence_b200", "csrc", tok[1])
                 if not os.path.exists(src):
                     return None
-                with open(src, "rb") as s:
-                    h = hashlib.sha256(s.read()).hexdigest()[:16]
-                return float(tok[3]) if h == tok[2] else None
+                return float(tok[3]) if kernel_source_hash(tok[1]) == tok[2] else None
     return None
 
 

@@ -386,18 +386,19 @@ def measure_rows(gdn, peaks, peak_src, args):
     nb = prefill_bytes(w.B, w.H, w.L, w.dk, w.dv, 2, True, True, True, True)
     fl = flops_per_head_token("gdn", w.dk, w.dv, w.chunk) * w.B * w.H * w.L
     rows["gdn_prefill_long"] = _row(w, ms, nb, fl, peaks, peak_src, "hbm", w.B * w.L, "gdn_prefill_cluster")
-    # the same workload as a sequence split into 4 segments on this one device: segments 0-2
-    # (from s0 / from 0) with segments 1-2 from I alongside, the compositions, then segments
-    # 1-3 again from their incoming states; bytes and FLOP counted as for one pass (the
-    # algorithmic work of the operator), so the fraction shows what the split costs
+    # the same workload as a sequence split into 3 segments on this one device: segments 0-1
+    # (from s0 / from 0) with segment 1 from lambda I alongside (96 one-CTA sequences, one
+    # wave on 148 SMs), the composition, then segments 1-2 again from their incoming states;
+    # bytes and FLOP counted as for one pass (the algorithmic work of the operator), so the
+    # fraction shows what the split costs on one device
     from gated_deltanet_sequence_b200.context_parallel import segmented_prefill, segment_bounds
-    bounds = segment_bounds(w.L, 4, w.chunk)
+    bounds = segment_bounds(w.L, 3, w.chunk)
     fn = lambda: segmented_prefill(inp["q"], inp["k"], inp["v"], inp["beta"], inp["g"], inp["s0"], o=o,
                                    s_final=sf, chunk=w.chunk, bounds=bounds)
     ms = timed(fn, max(3, args.steps // 4), 2)
     row = _row(w, ms, nb, fl, peaks, peak_src, "hbm", w.B * w.L)
-    row["path"] = "sequence split, 4 segments on one device (3 packed launches + 2 compositions)"
-    rows["gdn_prefill_long_split4"] = row
+    row["path"] = "sequence split, 3 segments on one device (3 packed launches + 1 composition)"
+    rows["gdn_prefill_long_split3"] = row
     del inp, o, sf
     torch.cuda.empty_cache()
     # packed variable-length Gated DeltaNet: 24 sequences (log-uniform length mix), 16 heads

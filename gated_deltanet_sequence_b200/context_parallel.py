@@ -146,10 +146,11 @@ def segmented_prefill(q, k, v, beta=None, g=None, s0=None, *, segments: int = 4,
     if s_final is None:
         s_final = torch.empty(1, H, d, d, dtype=torch.float32, device=dev)
     packed = [t[0] if t is not None else None for t in (q, k, v, beta, g)]
+    bounds_dev = torch.tensor(b, dtype=torch.int32, device=dev)    # one copy; launches take slices
 
     def run(first, last, s_init, out, ends, stream=None):
         # segments first .. last - 1 as one packed launch
-        cu = torch.tensor(b[first:last + 1], dtype=torch.int32, device=dev)
+        cu = bounds_dev[first:last + 1]
         qq, kk, vv, bb, gg = packed
         if bb is None:
             _lib.lin_attn_chunk_fwd_varlen(qq, kk, vv, cu, gg, o=out, s0=s_init, s_final=ends, chunk=chunk,
@@ -161,35 +162,35 @@ def segmented_prefill(q, k, v, beta=None, g=None, s0=None, *, segments: int = 4,
     if P == 1:
         run(0, 1, s0, o[0], s_final)
         return o, s_final
-    # pass 1: segments 0 .. P-2 (segment 0 from s0, the rest from 0) ...
+    # every buffer is allocated on the main stream before the side stream forks, and the main
+    # stream waits for the side stream before any later use, so no buffer is reused early
     s_init = torch.zeros(P - 1, H, d, d, dtype=torch.float32, device=dev)
     if s0 is not None:
         s_init[0].copy_(s0[0])
     ends = torch.empty(P - 1, H, d, d, dtype=torch.float32, device=dev)   # N_p (p >= 1); S_in(1) at 0
+    s_in = torch.empty(P - 1, H, d, d, dtype=torch.float32, device=dev)
+    seg_ends = torch.empty(P - 1, H, d, d, dtype=torch.float32, device=dev)
     main = torch.cuda.current_stream(dev)
     mn = None
     if P > 2:
-        # ... and, concurrently, segments 1 .. P-2 from lambda I (lambda M + N), outputs to a
-        # scratch buffer
+        mn = torch.empty(P - 2, H, d, d, dtype=torch.float32, device=dev)
+        eye = torch.empty(P - 2, H, d, d, dtype=torch.float32, device=dev)
+        scratch = torch.empty(H, L, d, dtype=torch.float32, device=dev)
+        # pass 1b, concurrently with 1a: segments 1 .. P-2 from lambda I (lambda M + N), outputs
+        # to the scratch buffer
         side = torch.cuda.Stream(device=dev)
         side.wait_stream(main)
-        with torch.cuda.stream(side):
-            eye = CudaOps.identity((P - 2) * H, d, dev, START_SCALE, stream=side).view(P - 2, H, d, d)
-            mn = torch.empty(P - 2, H, d, d, dtype=torch.float32, device=dev)
-            scratch = torch.empty(H, L, d, dtype=torch.float32, device=dev)
-            run(1, P - 1, eye, scratch, mn, stream=side)
+        _lib.gdn_state_identity(eye, START_SCALE, stream=side)
+        run(1, P - 1, eye, scratch, mn, stream=side)
+    # pass 1a: segments 0 .. P-2 (segment 0 from s0, the rest from 0)
     run(0, P - 1, s_init, o[0], ends)
     if P > 2:
         main.wait_stream(side)
-        for t in (eye, mn, scratch):
-            t.record_stream(main)
     # compositions: the state entering segments 1 .. P-1
-    s_in = torch.empty(P - 1, H, d, d, dtype=torch.float32, device=dev)
     s_in[0].copy_(ends[0])
     for p in range(1, P - 1):
         CudaOps.compose(mn[p - 1], ends[p], s_in[p - 1], s_in[p], START_SCALE)
     # pass 2: segments 1 .. P-1 from their incoming states
-    seg_ends = torch.empty(P - 1, H, d, d, dtype=torch.float32, device=dev)
     run(1, P, s_in, o[0], seg_ends)
     s_final[0].copy_(seg_ends[P - 2])
     return o, s_final

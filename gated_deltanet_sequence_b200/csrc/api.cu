@@ -55,11 +55,12 @@ const char *gdn_status_str(gdn_status_t s) {
         case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED";
         case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
         case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT";
+        case GDN_ERR_NONFINITE: return "GDN_ERR_NONFINITE";
     }
     return "GDN_ERR_UNKNOWN";
 }
 
-int gdn_version(void) { return 101; }
+int gdn_version(void) { return 102; }
 
 gdn_status_t lin_attn_chunk_fwd(const void *q, const void *k, const void *v, const float *g,
                                 float *o, const float *s0, float *s_final, int B, int H, int L,

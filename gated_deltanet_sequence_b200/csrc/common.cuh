@@ -11,7 +11,42 @@ namespace gdn {
 // Codes a kernel ORs into the device-side error word (the word lives in the
 // tensor-core translation unit): a bounded wait gave up, or a packed batch's
 // sequence offsets were not a non-decreasing list inside [0, T].
-enum : unsigned { kErrWaitTimeout = 1u, kErrBadSeqlens = 2u };
+enum : unsigned { kErrWaitTimeout = 1u, kErrBadSeqlens = 2u, kErrNonFinite = 4u };
+
+// Non-finite detector for stored results: nf <- nf + 0 * x keeps nf at 0 for finite x and
+// turns it into NaN for an infinite or NaN x (0 * inf = NaN), one FMA per value (IEEE
+// arithmetic: the build does not relax it).
+__device__ __forceinline__ void probe_finite(float &nf, float x) { nf = fmaf(x, 0.f, nf); }
+// The probe over the first n values of a 64-value tile: a pairwise sum (an inf or NaN value
+// makes the sum inf or NaN; so would finite values summing beyond fp32 range, itself an
+// overflow), then one probe step. 63 adds of depth 6, so no long dependency chain.
+__device__ __forceinline__ void probe_tile(float &nf, const float (&x)[64], int n) {
+    float t[32];
+    if (n >= 64) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) t[i] = x[2 * i] + x[2 * i + 1];
+    } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) t[i] = (2 * i < n ? x[2 * i] : 0.f) + (2 * i + 1 < n ? x[2 * i + 1] : 0.f);
+    }
+#pragma unroll
+    for (int w = 16; w >= 1; w >>= 1)
+#pragma unroll
+        for (int i = 0; i < w; ++i) t[i] += t[i + w];
+    probe_finite(nf, t[0]);
+}
+// The kernels probe the last output tile of each sequence and the whole final state. A
+// non-finite value that reaches the state (any fp16 overflow of the state chain) stays in it
+// and so reaches the last tile and the final state; a non-finite value confined to rows of an
+// earlier tile is not seen. Probing every tile cost 1.5-2.5 % of the prefill time.
+__device__ __forceinline__ bool probe_chunk(int c, int nchunks) { return c == nchunks - 1; }
+// Records kErrNonFinite once per warp when some lane's probe saw a non-finite value. Every
+// lane of the warp calls it; a CTA that gave up on a wait passes 0 (its stores stopped early
+// and the timeout is what gdn_sync_status reports).
+__device__ __forceinline__ void report_nonfinite(float nf, unsigned *err) {
+    const bool bad = __any_sync(0xffffffffu, nf != nf);
+    if (bad && (threadIdx.x & 31) == 0 && err) atomicOr(err, kErrNonFinite);
+}
 
 // Token range of the (sequence, head) handled by CTA `bid`. Dense batches
 // (cu == nullptr): one sequence of length L per row of the (B*H, L) token grid.
@@ -163,9 +198,11 @@ __device__ __forceinline__ void group_xnorm_128(float (&x)[64], int kind, float 
 }
 
 // One value column of a 64-token output tile: stores ov[r] (r < n) at element offset
-// elem0 + r * stride of o, in fp32 or rounded to bf16 (nearest, ties to even).
+// elem0 + r * stride of o, in fp32 or rounded to bf16 (nearest, ties to even); with `probe`
+// the stored values go through the non-finite probe nf (probe_tile).
 __device__ __forceinline__ void store_out_rows_final(const float (&ov)[64], void *o, size_t elem0, int n, int stride,
-                                                     bool bf16) {
+                                                     bool bf16, bool probe, float &nf) {
+    if (probe) probe_tile(nf, ov, n);
     if (bf16) {
         __nv_bfloat16 *ob = static_cast<__nv_bfloat16 *>(o) + elem0;
 #pragma unroll
@@ -178,23 +215,13 @@ __device__ __forceinline__ void store_out_rows_final(const float (&ov)[64], void
             if (r < n) of[static_cast<size_t>(r) * stride] = ov[r];
     }
 }
-// The same after the D-skip term: adds dj * v at the same offsets when v is given (fp32
-// fused multiply-add).
-__device__ __forceinline__ void store_out_rows(float (&ov)[64], void *o, size_t elem0, int n, int stride,
-                                               bool bf16, float dj, const __nv_bfloat16 *v) {
-    if (v) {
-#pragma unroll
-        for (int r = 0; r < 64; ++r)
-            if (r < n) ov[r] = fmaf(dj, __bfloat162float(v[elem0 + static_cast<size_t>(r) * stride]), ov[r]);
-    }
-    store_out_rows_final(ov, o, elem0, n, stride, bf16);
-}
 // The same for a 128-thread group holding the tile's 128 value columns (thread gt =
 // column), with the output normalisation when out.xnorm is set. The whole group calls it
 // (it meets on bar_id); red and stat are shared scratch of 256 and 128 floats. head
 // indexes the (H, dv) weights of the skip term and of the normalisation.
 __device__ __forceinline__ void store_out_rows_group(float (&ov)[64], const OutArgs &out, size_t elem0, int n,
-                                                     int head, int gt, int bar_id, float *red, float *stat) {
+                                                     int head, int gt, int bar_id, float *red, float *stat, bool probe,
+                                                     float &nf) {
     if (out.v) {
         const float dj = out.dskip[head * 128 + gt];
 #pragma unroll
@@ -203,7 +230,7 @@ __device__ __forceinline__ void store_out_rows_group(float (&ov)[64], const OutA
     }
     if (out.xnorm != kXNormNone)
         group_xnorm_128(ov, out.xnorm, out.xeps, out.xw ? out.xw[head * 128 + gt] : 1.f, gt, bar_id, red, stat);
-    store_out_rows_final(ov, out.o, elem0, n, 128, out.bf16 != 0);
+    store_out_rows_final(ov, out.o, elem0, n, 128, out.bf16 != 0, probe, nf);
 }
 
 }  // namespace gdn

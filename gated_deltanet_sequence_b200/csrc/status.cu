@@ -21,11 +21,13 @@ namespace {
 std::atomic<long long> g_wait_limit{kWaitLimitCycles};
 
 // Reports one condition and clears only that bit, atomically: a malformed sequence-offset
-// list first, then a bounded wait that gave up. Bits set meanwhile by kernels on other
-// streams stay in the word.
+// list first, then a bounded wait that gave up, then a non-finite stored result. Bits set
+// meanwhile by kernels on other streams stay in the word.
 __global__ void take_error_kernel(unsigned *word, unsigned *taken) {
     const unsigned now = atomicOr(word, 0u);
-    const unsigned bit = (now & kErrBadSeqlens) ? kErrBadSeqlens : (now & kErrWaitTimeout);
+    const unsigned bit = (now & kErrBadSeqlens)    ? kErrBadSeqlens
+                         : (now & kErrWaitTimeout) ? kErrWaitTimeout
+                                                   : (now & kErrNonFinite);
     if (bit) atomicAnd(word, ~bit);
     *taken = bit;
 }
@@ -97,7 +99,8 @@ gdn_status_t gdn_sync_status(void *cuda_stream) {
     unsigned err = 0u;
     if (!gdn::take_device_error(stream, &err)) return GDN_ERR_CUDA;
     if (err & gdn::kErrBadSeqlens) return GDN_ERR_INVALID_ARG;
-    return err ? GDN_ERR_TIMEOUT : GDN_OK;
+    if (err & gdn::kErrWaitTimeout) return GDN_ERR_TIMEOUT;
+    return err ? GDN_ERR_NONFINITE : GDN_OK;
 }
 
 }  // extern "C"

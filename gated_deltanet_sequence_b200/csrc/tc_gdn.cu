@@ -299,6 +299,7 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             tmem_wait_st();
         }
         int done = 0;   // chunks whose output tile has been stored
+        float nf = 0.f;  // non-finite probe over sampled output tiles and the final state
 #pragma unroll 1
         for (int c = 0; c < nchunks; ++c) {
             const int s = c & 1;
@@ -360,7 +361,8 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             // ---- output of the previous chunk (its O tile is complete)
             if (c >= 1) {
                 const int cp = c - 1;
-                store_out_col<OPTS>(trow + TM_O + (cp & 1) * 64, out, (row0 + static_cast<size_t>(cp) * kC) * kD + j, kC, head, j, kBarS, xn);
+                store_out_col<OPTS>(trow + TM_O + (cp & 1) * 64, out, (row0 + static_cast<size_t>(cp) * kC) * kD + j, kC, head, j, kBarS, xn,
+                                    false, nf);   // the last tile is stored (and probed) after the loop
                 done = c;
             }
             // ---- Ut^T row v -> Ut operand (K-major, rows v)
@@ -384,7 +386,7 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             if (ctl.group_wait(B_CDONE + (cp & 1), (cp >> 1) & 1, kBarS, lead)) {
                 tc_fence_after();
                 store_out_col<OPTS>(trow + TM_O + (cp & 1) * 64, out, (row0 + static_cast<size_t>(cp) * kC) * kD + j,
-                              L - cp * kC, head, j, kBarS, xn);
+                              L - cp * kC, head, j, kBarS, xn, true, nf);
                 done = nchunks;
             }
         }
@@ -396,10 +398,13 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 tmem_ld16(trow + TM_S + cc * 16, sv);
                 tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 16; e += 4)
+                for (int e = 0; e < 16; e += 4) {
+                    probe_finite(nf, sv[e] + sv[e + 1] + sv[e + 2] + sv[e + 3]);
                     *reinterpret_cast<float4 *>(dst + cc * 16 + e) = make_float4(sv[e], sv[e + 1], sv[e + 2], sv[e + 3]);
+                }
             }
         }
+        report_nonfinite(ctl.aborted() ? 0.f : nf, err_word);
     } else if (warp >= kGroupP) {
         // ================================================================ prep group
         const int p = tid - kGroupP * 32;                // 0..255

@@ -295,6 +295,7 @@ tc_gdn_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 tmem_wait_st();
             }
             int done = 0;   // chunks whose output tile has been stored
+            float nf = 0.f;  // non-finite probe over sampled output tiles and the final state
 #pragma unroll 1
             for (int c = 0; c < nchunks; ++c) {
                 const int s = c & 1;
@@ -354,7 +355,8 @@ tc_gdn_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     if (c + 2 < nchunks && lead)
                         mbar_arrive_cluster(mapa_shared(smem_u32(&bars[B_SFREE + (((c - 1) >> 1) & 1)]), 1 + (c & 1)));
                     tc_fence_after();
-                    store_out_col<OPTS>(trow + TM_O + (cp & 1) * 64, out, (row0 + static_cast<size_t>(cp) * kC) * kD + j, kC, head, j, kBarS, xn);
+                    store_out_col<OPTS>(trow + TM_O + (cp & 1) * 64, out, (row0 + static_cast<size_t>(cp) * kC) * kD + j, kC, head, j, kBarS, xn,
+                                    false, nf);   // the last tile is stored (and probed) after the loop
                     done = c;
                 }
                 // ---- Ut^T row v -> Ut operand (K-major, rows v)
@@ -377,7 +379,7 @@ tc_gdn_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 if (ctl.group_wait(B_CDONE + (cp & 1), (cp >> 1) & 1, kBarS, lead)) {
                     tc_fence_after();
                     store_out_col<OPTS>(trow + TM_O + (cp & 1) * 64, out, (row0 + static_cast<size_t>(cp) * kC) * kD + j,
-                                  L - cp * kC, head, j, kBarS, xn);
+                                  L - cp * kC, head, j, kBarS, xn, true, nf);
                     done = nchunks;
                 }
             }
@@ -389,10 +391,13 @@ tc_gdn_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     tmem_ld16(trow + TM_S + cc * 16, sv);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 16; e += 4)
+                    for (int e = 0; e < 16; e += 4) {
+                        probe_finite(nf, sv[e] + sv[e + 1] + sv[e + 2] + sv[e + 3]);
                         *reinterpret_cast<float4 *>(dst + cc * 16 + e) = make_float4(sv[e], sv[e + 1], sv[e + 2], sv[e + 3]);
+                    }
                 }
             }
+            report_nonfinite(ctl.aborted() ? 0.f : nf, err_word);
         } else if (warp >= kGroupP && warp < kGroupP + 4) {
             // ------------------------------------------------------------ tile converter
             // K, V bf16 -> fp16 and Q -> Q' = fp16(scale gamma q), in place, once the tiles

@@ -38,18 +38,20 @@ __device__ __forceinline__ void st_row16_h(uint32_t tile, uint32_t row, int ch, 
 // output options (fp32 / bf16, D-skip term, output normalisation) when OPTS, plain fp32
 // otherwise. With OPTS the whole 128-thread group (thread gt = value column) calls it
 // and meets on bar_id; xn: 384 floats of shared scratch; head indexes the (H, dv) weights.
+// With `probe` the stored values go through the non-finite probe nf.
 template <bool OPTS>
 __device__ __forceinline__ void store_out_col(uint32_t taddr, const OutArgs &out, size_t elem0, int n, int head,
-                                              int gt, int bar_id, float *xn) {
+                                              int gt, int bar_id, float *xn, bool probe, float &nf) {
     float ov[64];
     ld_cols<64>(taddr, ov);
     if constexpr (OPTS) {
-        store_out_rows_group(ov, out, elem0, n, head, gt, bar_id, xn, xn + 256);
+        store_out_rows_group(ov, out, elem0, n, head, gt, bar_id, xn, xn + 256, probe, nf);
     } else {
         float *ocol = static_cast<float *>(out.o) + elem0;
 #pragma unroll
         for (int r = 0; r < 64; ++r)
             if (r < n) ocol[static_cast<size_t>(r) * kD] = ov[r];
+        if (probe) probe_tile(nf, ov, n);
     }
 }
 

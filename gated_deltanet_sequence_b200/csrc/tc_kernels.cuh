@@ -28,7 +28,8 @@ gdn_status_t launch_tc_la(const void *q, const void *k, const void *v, const flo
 // Takes one condition out of the device-side error word of the current device, on
 // `stream` (a one-thread kernel clears only the bit it reports, atomically, so a bit
 // that another kernel sets meanwhile is kept for the next call): *err receives
-// kErrBadSeqlens if that bit was set, else kErrWaitTimeout if that one was, else 0.
+// kErrBadSeqlens if that bit was set, else kErrWaitTimeout if that one was, else
+// kErrNonFinite if that one was, else 0.
 bool take_device_error(cudaStream_t stream, unsigned *err);
 // Device address of that word on the current device (looked up once per device),
 // handed to kernels that may record a bounded-wait timeout; nullptr on failure.

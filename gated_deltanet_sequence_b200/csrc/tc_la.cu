@@ -313,6 +313,7 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         const int v = tid - 128;                          // TMEM lane = value column
         const bool lead = (v == 0);
         const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+        float nf = 0.f;   // non-finite probe over the final state
         {
             // S^T row v = column v of the initial state (a warp reads 32 consecutive floats)
             const float *src = s0 ? s0 + static_cast<size_t>(bh) * kD * kD + v : nullptr;
@@ -378,9 +379,13 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 tmem_ld16(trow + TM_S + cc * 16, sv);
                 tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 16; ++e) dst[static_cast<size_t>(cc * 16 + e) * kD] = sv[e];
+                for (int e = 0; e < 16; ++e) {
+                    probe_finite(nf, sv[e]);
+                    dst[static_cast<size_t>(cc * 16 + e) * kD] = sv[e];
+                }
             }
         }
+        report_nonfinite(ctl.aborted() ? 0.f : nf, err_word);
     } else if (warp < 12) {
         // ================================================================ output group
         const int v = tid - 256;                          // TMEM lane = value column
@@ -388,6 +393,7 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
         const int head = zc % H;                          // head of this row (dense and packed grids)
         float *xn = reinterpret_cast<float *>(smem + OFF_XN);
+        float nf = 0.f;   // non-finite probe over sampled output tiles
 #pragma unroll 1
         for (int c = 0; c < nchunks; ++c) {
             const int p = c & 1;
@@ -401,14 +407,16 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             const int n = min(kC, L - c * kC);
             if constexpr (OPTS) {
                 store_out_rows_group(ov, out, (row0 + static_cast<size_t>(c) * kC) * kD + v, n, head, v, kBarOut, xn,
-                                     xn + 256);
+                                     xn + 256, probe_chunk(c, nchunks), nf);
             } else {
                 float *ocol = static_cast<float *>(out.o) + (row0 + static_cast<size_t>(c) * kC) * kD + v;
 #pragma unroll
                 for (int r = 0; r < 64; ++r)
                     if (r < n) ocol[static_cast<size_t>(r) * kD] = ov[r];
+                if (probe_chunk(c, nchunks)) probe_tile(nf, ov, n);
             }
         }
+        report_nonfinite(ctl.aborted() ? 0.f : nf, err_word);
     } else if (warp >= 18) {
         // ================================================================ P writers
         // P = scale (Q K^T o Gamma), s <= r, row r (Gram lane 64 + r) -> PG (fp16)

@@ -46,7 +46,9 @@ typedef enum {
     GDN_ERR_INVALID_ARG = 1,   /* NULL required pointer, bad size, misaligned pointer */
     GDN_ERR_UNSUPPORTED = 2,   /* valid but not implemented (head dim, chunk, dtype)  */
     GDN_ERR_CUDA = 3,          /* a CUDA runtime/driver call or launch failed          */
-    GDN_ERR_TIMEOUT = 4        /* a kernel gave up on a bounded wait (see sync_status) */
+    GDN_ERR_TIMEOUT = 4,       /* a kernel gave up on a bounded wait (see sync_status) */
+    GDN_ERR_NONFINITE = 5      /* a tensor-core prefill stored inf / NaN in o or S_final
+                                  (checked on a sample, see sync_status)               */
 } gdn_status_t;
 
 typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype_t;
@@ -312,10 +314,15 @@ const char *gdn_status_str(gdn_status_t status);
 /*
  * gdn_sync_status — synchronise `cuda_stream`, then report and clear one device-side
  * condition met by a kernel of this library on the current device since it was last
- * reported: GDN_ERR_INVALID_ARG for a malformed cu_seqlens list (reported first),
- * GDN_ERR_TIMEOUT for a bounded wait that gave up, GDN_OK when neither is pending,
- * GDN_ERR_CUDA if the stream or the read failed. When both conditions are pending the
- * next call reports the other one. The conditions live in one word per device, shared by
+ * reported, in this order: GDN_ERR_INVALID_ARG for a malformed cu_seqlens list,
+ * GDN_ERR_TIMEOUT for a bounded wait that gave up, GDN_ERR_NONFINITE when a tensor-core
+ * prefill kernel found inf or NaN among the results it stored (non-finite inputs, or an
+ * intermediate beyond the fp16 operand range, |x| > 65504, of those kernels). The kernels
+ * check the last 64-token output tile of each sequence and its final state: a non-finite
+ * value in the state reaches both, while one confined to rows of an earlier tile (inputs
+ * whose q or q.k exceed the fp16 range) can go unreported;
+ * GDN_OK when none is pending, GDN_ERR_CUDA if the stream or the read failed. When several
+ * conditions are pending the next calls report the others. The conditions live in one word per device, shared by
  * every caller and stream of this process: a condition raised by another caller's kernel
  * is reported to whichever caller asks first. The word is taken with a one-thread kernel
  * on `cuda_stream` (atomic, so a condition raised meanwhile on another stream is kept).

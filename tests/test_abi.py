@@ -42,6 +42,7 @@ def test_library_exports_every_declared_symbol(lib):
 def test_status_strings_and_version(lib):
     assert lib.status_str(0) == "GDN_OK"
     assert lib.status_str(4) == "GDN_ERR_TIMEOUT"
+    assert lib.status_str(5) == "GDN_ERR_NONFINITE"
     assert lib.status_str(99) == "GDN_ERR_UNKNOWN"
     assert lib.gdn_version() >= 100
 

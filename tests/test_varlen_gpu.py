@@ -113,7 +113,8 @@ def test_varlen_equals_dense_per_sequence(lib, mode):
 @pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.float32, 64)])
 def test_malformed_offsets_are_reported(lib, cu, dtype, d):
     H, T = 2, 24
-    q = torch.randn(H, T, d, device="cuda").to(dtype)
+    # unit-norm keys keep the valid sequences' states bounded (no other condition pending)
+    q = torch.nn.functional.normalize(torch.randn(H, T, d, device="cuda"), dim=-1).to(dtype)
     cu_t = torch.tensor(cu, dtype=torch.int32, device="cuda")
     beta = torch.full((H, T), 0.5, device="cuda")
     lib.gdn_chunk_fwd_varlen(q, q, q, beta, cu_t)

@@ -10,11 +10,16 @@
 //   Gram   [K;Q] K^T                     one M=128 UMMA (rows: K K^T, then Q K^T)
 //   UT     A = tril(diag(beta) KK^T o Gamma, -1), T = (I + A)^-1   (forward subst.)
 //   W, U   W^T = K^T (T diag(beta gamma))^T, U^T = V^T (T diag(beta))^T
-//   Ut     Ut^T = U^T - S^T W^T   (accumulated onto U^T with a negated operand)
-//   out    O^T = S^T Q'^T + Ut^T (scale Q K^T o Gamma)^T,  Q' = diag(scale gamma) Q
+//   Ut/out [O^T | Ut^T] += S^T [Q'^T | -W^T]   (one N=128 product: O^T starts at zero, Ut^T
+//          at U^T), Q' = diag(scale gamma) Q
+//   out    O^T += Ut^T (scale Q K^T o Gamma)^T
 //   state  S <- gamma_last S + (diag(d) K)^T Ut   (K scaled in place once W/U has read it)
 // Every product has dk or dv (= 128) as the UMMA M dimension, so each tcgen05.mma
-// is a full 128-lane instruction and TMEM lane = row of the result.
+// is a full 128-lane instruction and TMEM lane = row of the result. An M=128, K=16
+// tcgen05.mma issued back to back takes about 49 cycles at N=64 and 65 at N=128 on this
+// part (measured), so the state's two products above, which share their A operand, run as
+// one N=128 product: the serial chain issues 8 instructions for them instead of 16 (Q'^T
+// and -W are stored MN-major, one operand stride apart in each key half).
 //
 // Warp roles (512 threads):
 //   warp 0      TMA producer (2-stage ring of Q, K, V tiles)
@@ -52,17 +57,19 @@ constexpr int kGroupS = 4;       // first warp of the state group (4 warps)
 constexpr int kGroupP = 8;       // first warp of the prep group (8 warps)
 constexpr int kNP = 256;         // prep group threads
 constexpr int kBarS = 1, kBarP = 2;   // named barriers of the state (128) and prep (256) groups
+constexpr int kBarQ = 4;              // the prep group's four converter warps (id 3: its solve warps)
 constexpr float kFastDecayLimit = -60.f;   // G_last >= this: Gamma = gamma_r * exp(-G_s)
 
 // ---- shared memory map (byte offsets from a 1024-aligned base) ------------------
-constexpr uint32_t kStageBytes = 49152;   // one chunk of K, Q, V
+constexpr uint32_t kStageBytes = 49152;   // one chunk of K, Q, V; per key half h: [K_h Q_h V_h]
 constexpr uint32_t ST_K0 = 0;             // K, key columns 0-63   (64 rows x 128 B)
-constexpr uint32_t ST_Q0 = 8192;          // Q, key columns 0-63   (directly after K: [K;Q])
-constexpr uint32_t ST_K1 = 16384;         // K, key columns 64-127
-constexpr uint32_t ST_Q1 = 24576;         // Q, key columns 64-127
-constexpr uint32_t ST_V0 = 32768;         // V, value columns 0-63; holds W (MN-major, 128 key
-constexpr uint32_t ST_V1 = 40960;         //   rows x 64 r) once U has been formed
-constexpr uint32_t ST_W = ST_V0;
+constexpr uint32_t ST_Q0 = 8192;          // Q, key columns 0-63   (directly after K: [K;Q]); then Q'^T
+constexpr uint32_t ST_V0 = 16384;         // V, value columns 0-63; then -W, key rows 0-63
+constexpr uint32_t ST_K1 = 24576;         // K, key columns 64-127
+constexpr uint32_t ST_Q1 = 32768;         // Q, key columns 64-127; then Q'^T
+constexpr uint32_t ST_V1 = 40960;         // V, value columns 64-127; then -W, key rows 64-127
+constexpr uint32_t kHalf = ST_K1 - ST_K0;  // stride between the key (or value) halves of a tensor
+static_assert(ST_V0 - ST_Q0 == ST_V1 - ST_Q1, "Q'^T and W of a key half must be one operand stride apart");
 constexpr uint32_t OFF_AT = 2 * kStageBytes;        // A^T fp32 64 x 64 (UT-solve input)
 constexpr uint32_t OFF_TF = OFF_AT + 16384;         // T fp32 64 x 68 (pitch 68)
 constexpr int kTP = 68;
@@ -87,13 +94,13 @@ static_assert(OFF_T1 % 1024 == 0 && OFF_PG % 1024 == 0 && OFF_S % 1024 == 0 && O
 constexpr uint32_t TM_S = 0;      // state S: lane = key row j, 128 value columns
 constexpr uint32_t TM_G = 128;    // [K;Q] K^T: lanes 0-63 K K^T, 64-127 Q K^T; 64 columns s
 constexpr uint32_t TM_W = 192;    // W^T: lane = key j, 64 columns r
-constexpr uint32_t TM_U = 256;    // U^T then Ut^T: lane = value v, 64 columns r
-constexpr uint32_t TM_O = 320;    // 2 x O^T: lane = value v, 64 columns r
+constexpr uint32_t TM_OU = 256;   // 2 x [O^T | U^T then Ut^T]: lane = value v, 64 + 64 columns r
 
 constexpr uint32_t ID_GRAM = idesc_f16(128, 64, false, false, false, /*bf16=*/true);
 constexpr uint32_t ID_WU = idesc_f16(128, 64, true, false);
-constexpr uint32_t ID_SW = idesc_f16(128, 64, true, true, /*neg_a=*/true);
-constexpr uint32_t ID_SQ = idesc_f16(128, 64, true, false);
+// [O^T | Ut^T] += S^T [Q'^T | -W^T]: one N=128 product for both uses of the state (B = Q'^T and
+// -W, MN-major, one operand stride apart)
+constexpr uint32_t ID_SQW = idesc_f16(128, 128, true, true);
 constexpr uint32_t ID_ST = idesc_f16(128, 128, true, false);
 constexpr uint32_t ID_O = idesc_f16(128, 64, false, false);
 
@@ -197,7 +204,7 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
+                    const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32u;
                     mma_f16(tmem + TM_G, sdesc_sw128(stg + ST_K0 + off, 16, 1024),
                             sdesc_sw128(stg + ST_K0 + off, 16, 1024), ID_GRAM, kk > 0);
                 }
@@ -215,11 +222,11 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_f16(tmem + TM_W, sdesc_sw128(stg + ST_K0 + kk * 2048, 16384, 1024),
+                    mma_f16(tmem + TM_W, sdesc_sw128(stg + ST_K0 + kk * 2048, kHalf, 1024),
                             sdesc_sw128(sb + OFF_T1 + kk * 32, 16, 1024), ID_WU, kk > 0);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_f16(tmem + TM_U, sdesc_sw128(stg + ST_V0 + kk * 2048, 8192, 1024),
+                    mma_f16(tmem + TM_OU + (c & 1) * 128 + 64, sdesc_sw128(stg + ST_V0 + kk * 2048, kHalf, 1024),
                             sdesc_sw128(sb + OFF_T2 + kk * 32, 16, 1024), ID_WU, kk > 0);
                 mma_commit(&bars[B_WU]);
             };
@@ -236,17 +243,13 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 if (!ctl.wait(B_WRDY, c & 1)) break;
                 if (!ctl.wait(B_SRDY, c & 1)) break;
                 tc_fence_after();
-                // Ut^T = U^T - S^T W^T ;  O^T = S^T Q'^T
+                // [O^T | Ut^T] += S^T [Q'^T | -W^T]  (O^T starts zeroed, Ut^T holds U^T): the
+                // output's state part and U - W S in one N=128 product
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_f16(tmem + TM_U, sdesc_sw128(sb + OFF_S + kk * 2048, 16384, 1024),
-                            sdesc_sw128(stg + ST_W + kk * 2048, 8192, 1024), ID_SW, 1u);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
-                    mma_f16(tmem + TM_O + s * 64, sdesc_sw128(sb + OFF_S + kk * 2048, 16384, 1024),
-                            sdesc_sw128(stg + ST_Q0 + off, 16, 1024), ID_SQ, kk > 0);
-                }
+                    mma_f16(tmem + TM_OU + s * 128, sdesc_sw128(sb + OFF_S + kk * 2048, 16384, 1024),
+                            sdesc_sw128(stg + (kk >> 2) * kHalf + ST_Q0 + (kk & 3) * 2048, ST_V0 - ST_Q0, 1024),
+                            ID_SQW, 1u);
                 mma_commit(&bars[B_ADONE]);
                 last_bar = B_ADONE;
                 last_par = c & 1;
@@ -255,11 +258,11 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 // S += (diag(d) K)^T Ut ;  O^T += Ut^T PG^T
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_f16(tmem + TM_S, sdesc_sw128(stg + ST_K0 + kk * 2048, 16384, 1024),
+                    mma_f16(tmem + TM_S, sdesc_sw128(stg + ST_K0 + kk * 2048, kHalf, 1024),
                             sdesc_sw128(sb + OFF_UB + kk * 32, 16, 1024), ID_ST, 1u);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_f16(tmem + TM_O + s * 64, sdesc_sw128(sb + OFF_UB + kk * 32, 16, 1024),
+                    mma_f16(tmem + TM_OU + s * 128, sdesc_sw128(sb + OFF_UB + kk * 32, 16, 1024),
                             sdesc_sw128(sb + OFF_PG + s * 8192 + kk * 32, 16, 1024), ID_O, 1u);
                 mma_commit(&bars[B_CDONE + s]);
                 last_bar = B_CDONE + s;
@@ -296,6 +299,12 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 }
                 tmem_st16(trow + TM_S + cc * 16, r);
             }
+            // the O^T tiles start at zero (the merged state product accumulates onto them)
+            float z[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) z[e] = 0.f;
+#pragma unroll 1
+            for (int cc = 0; cc < 8; ++cc) tmem_st16(trow + TM_OU + (cc >> 2) * 128 + (cc & 3) * 16, z);
             tmem_wait_st();
         }
         int done = 0;   // chunks whose output tile has been stored
@@ -336,13 +345,25 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             //      (K's last reader before the state update was W/U)
             if (!ctl.group_wait(B_WU, c & 1, kBarS, lead)) break;
             tc_fence_after();
-            store_w_row(trow + TM_W, sb + s * kStageBytes + ST_W, j);
+            {
+                // W^T row j -> -W, MN-major: row j % 64 of the V slot of key half j / 64
+                const uint32_t wtile = sb + s * kStageBytes + (j >> 6) * kHalf + ST_V0;
+#pragma unroll 1
+                for (int cc = 0; cc < 4; ++cc) {
+                    float w[16];
+                    tmem_ld16(trow + TM_W + cc * 16, w);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) w[e] = -w[e];
+                    st_row16_h(wtile, j & 63, 2 * cc, w);
+                }
+            }
             if (GATED) {
                 // K tiles: 2 x 8 KB at ST_K0 / ST_K1, 64 rows of 128 B each; 1024 chunks of 16 B
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const uint32_t idx = static_cast<uint32_t>(i * 128 + j);
-                    const uint32_t off = (idx >> 9) * 16384u + ST_K0 + (idx & 511u) * 16u;
+                    const uint32_t off = (idx >> 9) * kHalf + ST_K0 + (idx & 511u) * 16u;
                     const __half2 f = __float2half2_rn(vec[V_D + ((idx & 511u) >> 3)]);
                     uint4 x = *reinterpret_cast<const uint4 *>(st + off);
                     __half2 *hh = reinterpret_cast<__half2 *>(&x);
@@ -361,8 +382,16 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             // ---- output of the previous chunk (its O tile is complete)
             if (c >= 1) {
                 const int cp = c - 1;
-                store_out_col<OPTS>(trow + TM_O + (cp & 1) * 64, out, (row0 + static_cast<size_t>(cp) * kC) * kD + j, kC, head, j, kBarS, xn,
+                store_out_col<OPTS>(trow + TM_OU + (cp & 1) * 128, out, (row0 + static_cast<size_t>(cp) * kC) * kD + j, kC, head, j, kBarS, xn,
                                     false, nf);   // the last tile is stored (and probed) after the loop
+                // chunk c + 1 accumulates onto this tile: zero it (ordered before that chunk's
+                // product by this group's state-ready hand-off)
+                float z[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) z[e] = 0.f;
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) tmem_st16(trow + TM_OU + (cp & 1) * 128 + cc * 16, z);
+                tmem_wait_st();
                 done = c;
             }
             // ---- Ut^T row v -> Ut operand (K-major, rows v)
@@ -371,7 +400,7 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
                 float u[16];
-                tmem_ld16(trow + TM_U + cc * 16, u);
+                tmem_ld16(trow + TM_OU + s * 128 + 64 + cc * 16, u);
                 tmem_wait_ld();
                 st_row16_h(sb + OFF_UB, j, 2 * cc, u);
             }
@@ -385,7 +414,7 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             const int cp = nchunks - 1;
             if (ctl.group_wait(B_CDONE + (cp & 1), (cp >> 1) & 1, kBarS, lead)) {
                 tc_fence_after();
-                store_out_col<OPTS>(trow + TM_O + (cp & 1) * 64, out, (row0 + static_cast<size_t>(cp) * kC) * kD + j,
+                store_out_col<OPTS>(trow + TM_OU + (cp & 1) * 128, out, (row0 + static_cast<size_t>(cp) * kC) * kD + j,
                               L - cp * kC, head, j, kBarS, xn, true, nf);
                 done = nchunks;
             }
@@ -598,10 +627,10 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     }
                 }
             } else {
-                // ---- meanwhile (the Gram has read the tiles): K, V bf16 -> fp16 and
-                //      Q -> Q' = fp16(scale gamma q), in place (128 threads)
+                // ---- meanwhile (the Gram has read the tiles): K, V bf16 -> fp16 in place and
+                //      Q -> Q'^T = fp16(scale gamma q)^T into the Q slots (128 threads)
                 const int t4 = p - 128;                      // 0..127
-                // K and V: 2048 chunks of 16 B at [0,8K) [16K,24K) [32K,48K)
+                // K and V: 2048 chunks of 16 B in the K0, K1, V0, V1 slots
 #pragma unroll
                 for (int part = 0; part < 2; ++part) {
                     uint4 x[8];
@@ -610,7 +639,7 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     for (int i = 0; i < 8; ++i) {
                         const uint32_t idx = static_cast<uint32_t>((part * 8 + i) * 128 + t4);   // 0..2047
                         const uint32_t reg = idx >> 9;                                            // 0..3
-                        offs[i] = (reg < 2 ? reg * 16384u : 32768u + (reg - 2) * 8192u) + (idx & 511u) * 16u;
+                        offs[i] = (reg & 1u) * kHalf + (reg < 2 ? ST_K0 : ST_V0) + (idx & 511u) * 16u;
                         x[i] = *reinterpret_cast<const uint4 *>(st + offs[i]);
                     }
 #pragma unroll
@@ -622,24 +651,33 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         *reinterpret_cast<uint4 *>(st + offs[i]) = x[i];
                     }
                 }
-                // Q: 1024 chunks at [8K,16K) [24K,32K), row r = (offset within the box) / 128
+                // Q -> Q'^T = fp16(scale gamma_r q_r)^T, transposed in place into the Q slots
+                // (MN-major: row k % 64 of the slot of key half k / 64 holds the 64 values r).
+                // Thread t4 takes row r = t4 % 64 and the logical 16-byte chunks kc = t4 / 64 + 2i
+                // (i < 4) of both key halves; all eight are read before any is overwritten, and a
+                // warp's threads then write consecutive r of one row (no bank conflicts)
                 {
+                    const int r = t4 & 63, kc0 = t4 >> 6;
+                    const float f = scale * vec[V_GAM + r];
                     uint4 x[8];
-                    uint32_t offs[8];
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
-                        const uint32_t idx = static_cast<uint32_t>(i * 128 + t4);                 // 0..1023
-                        offs[i] = ST_Q0 + (idx >> 9) * 16384u + (idx & 511u) * 16u;
-                        x[i] = *reinterpret_cast<const uint4 *>(st + offs[i]);
+                        const int h = i >> 2, kc = kc0 + 2 * (i & 3);
+                        x[i] = *reinterpret_cast<const uint4 *>(st + h * kHalf + ST_Q0 + r * 128 + ((kc ^ (r & 7)) << 4));
                     }
+                    named_bar(kBarQ, 128);
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
-                        const float f = scale * vec[V_GAM + ((offs[i] & 8191u) >> 7)];
-                        x[i].x = pack_h2(f * bf_lo(x[i].x), f * bf_hi(x[i].x));
-                        x[i].y = pack_h2(f * bf_lo(x[i].y), f * bf_hi(x[i].y));
-                        x[i].z = pack_h2(f * bf_lo(x[i].z), f * bf_hi(x[i].z));
-                        x[i].w = pack_h2(f * bf_lo(x[i].w), f * bf_hi(x[i].w));
-                        *reinterpret_cast<uint4 *>(st + offs[i]) = x[i];
+                        const int h = i >> 2, kc = kc0 + 2 * (i & 3);
+                        const uint32_t w[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const float q = (e & 1) ? bf_hi(w[e >> 1]) : bf_lo(w[e >> 1]);
+                            const int kr = 8 * kc + e;                   // key row within the half
+                            __half *dst = reinterpret_cast<__half *>(st + h * kHalf + ST_Q0 + kr * 128 +
+                                                                     ((((r >> 3) ^ kr) & 7) << 4)) + (r & 7);
+                            *dst = __float2half_rn(f * q);
+                        }
                     }
                 }
             }

@@ -25,7 +25,7 @@ EXPORTS = ("lin_attn_chunk_fwd", "gdn_chunk_fwd", "lin_attn_chunk_fwd_varlen", "
            "lin_attn_chunk_fwd_ex", "gdn_chunk_fwd_ex", "gdn_decode_step", "gdn_decode_step_ex",
            "gdn_status_str", "gdn_sync_status", "gdn_set_wait_limit_for_testing", "gdn_version",
            "gdn_chunk_bwd", "gdn_chunk_bwd_workspace_bytes", "gdn_chunk_bwd_noalloc", "gdn_state_compose",
-           "gdn_state_identity")
+           "gdn_state_identity", "gdn_chunk_fwd_host", "gdn_chunk_fwd_host_staging_bytes")
 
 
 GDN_XNORM = {None: 0, "rms": 1, "layer": 2}
@@ -75,6 +75,10 @@ def _load() -> ctypes.CDLL:
     lib.gdn_state_compose.argtypes = [P, P, P, P, F, I, I, P]
     lib.gdn_state_compose.restype = ctypes.c_int
     lib.gdn_state_identity.argtypes = [P, F, I, I, P]
+    lib.gdn_chunk_fwd_host_staging_bytes.argtypes = [I, I, I, I, I, I, I, I, I, I]
+    lib.gdn_chunk_fwd_host_staging_bytes.restype = Z
+    lib.gdn_chunk_fwd_host.argtypes = [P, P, P, P, P, P, P, P, P, Z, I, I, I, I, I, I, F, I, I, P]
+    lib.gdn_chunk_fwd_host.restype = ctypes.c_int
     lib.gdn_state_identity.restype = ctypes.c_int
     for f in (lib.lin_attn_chunk_fwd, lib.gdn_chunk_fwd, lib.lin_attn_chunk_fwd_varlen,
               lib.gdn_chunk_fwd_varlen, lib.lin_attn_chunk_fwd_ex, lib.gdn_chunk_fwd_ex,

@@ -308,6 +308,34 @@ gdn_status_t gdn_state_compose(const float *mn, const float *n, const float *s_i
                                int count, int d, void *cuda_stream);
 gdn_status_t gdn_state_identity(float *s, float value, int count, int d, void *cuda_stream);
 
+/*
+ * gdn_chunk_fwd_host — gdn_chunk_fwd from pinned host buffers, the copies overlapped with the
+ * computation (a serving step whose inputs are in host memory). The batch crosses PCIe in
+ * groups of `group` sequences: while group i is computed, group i + 1 is uploaded and group
+ * i - 1 downloaded, on three streams of the library's own (created and released by the call)
+ * with two staging slots in `staging`; every tensor of a group is one cudaMemcpyAsync. Each
+ * group is one dense prefill, and the (sequence, head) recurrences are independent, so the
+ * result equals one gdn_chunk_fwd on the whole batch, bit for bit.
+ *
+ *  q, k, v, beta, g, s0    as gdn_chunk_fwd, in page-locked (pinned) host memory
+ *  o, s_final              as gdn_chunk_fwd, in pinned host memory (s_final nullable)
+ *  staging                 device memory of at least gdn_chunk_fwd_host_staging_bytes(...)
+ *                          bytes, 256-byte aligned, owned by the caller (contents on entry
+ *                          irrelevant, unspecified on return)
+ *  group                   sequences per transfer (>= 1)
+ *  cuda_stream             the caller's stream: the call's work starts after the work already
+ *                          enqueued on it, and work enqueued on it afterwards starts after the
+ *                          call's last download. The call returns without waiting.
+ *  Returns GDN_ERR_INVALID_ARG for a pageable or NULL required host pointer, a staging buffer
+ *  too small or misaligned, or a bad size (L >= 1); other rules as gdn_chunk_fwd.
+ */
+size_t gdn_chunk_fwd_host_staging_bytes(int B, int H, int L, int dk, int dv, int group, gdn_dtype_t in_dtype,
+                                        int has_g, int has_s0, int has_s_final);
+gdn_status_t gdn_chunk_fwd_host(const void *q, const void *k, const void *v, const float *beta, const float *g,
+                                float *o, const float *s0, float *s_final, void *staging, size_t staging_bytes,
+                                int B, int H, int L, int dk, int dv, int chunk, float scale, gdn_dtype_t in_dtype,
+                                int group, void *cuda_stream);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 const char *gdn_status_str(gdn_status_t status);
 

@@ -29,7 +29,8 @@ def test_header_declares_the_boundary():
     for want in ("lin_attn_chunk_fwd", "gdn_chunk_fwd", "lin_attn_chunk_fwd_varlen", "gdn_chunk_fwd_varlen",
                  "lin_attn_chunk_fwd_ex", "gdn_chunk_fwd_ex", "gdn_decode_step", "gdn_decode_step_ex",
                  "gdn_status_str", "gdn_sync_status", "gdn_set_wait_limit_for_testing", "gdn_version",
-                 "gdn_chunk_bwd", "gdn_chunk_bwd_workspace_bytes", "gdn_state_compose", "gdn_state_identity"):
+                 "gdn_chunk_bwd", "gdn_chunk_bwd_workspace_bytes", "gdn_state_compose", "gdn_state_identity",
+                 "gdn_chunk_fwd_host", "gdn_chunk_fwd_host_staging_bytes"):
         assert want in names
 
 
@@ -221,3 +222,20 @@ def test_state_compose_and_identity_validate_on_the_host(lib):
     assert identity(None, 1.0, 1, 64, None) == 1
     assert identity(P(FAKE), float("nan"), 1, 64, None) == 1
     assert identity(P(FAKE), 1.0, 0, 64, None) == 0
+
+
+def test_host_pipeline_entry_validates_on_the_host(lib):
+    P = ctypes.c_void_p
+    f = lib.lib.gdn_chunk_fwd_host
+    size = lib.lib.gdn_chunk_fwd_host_staging_bytes
+    need = size(2, 3, 100, 128, 128, 1, 1, 1, 0, 1)
+    assert need > 0 and need % 256 == 0
+    assert size(2, 3, 100, 128, 128, 0, 1, 1, 0, 1) == 0                  # group < 1
+    args = [P(FAKE)] * 4 + [None, P(FAKE), None, None, P(FAKE), need, 2, 3, 100, 128, 128, 64, 1.0, 1, 1, None]
+    a = list(args); a[0] = None
+    assert f(*a) == 1                                                       # q missing
+    a = list(args); a[13] = 96
+    assert f(*a) == 2                                                       # dk outside {64, 128}
+    a = list(args); a[12] = 0
+    assert f(*a) == 1                                                       # L < 1
+    assert f(*args) == 1                  # these host pointers are not page-locked memory

@@ -1,5 +1,6 @@
 // C-ABI entry points of libgdn.so: argument validation and kernel dispatch.
-// Every launch goes on the caller's stream; nothing here allocates memory.
+// Every launch goes on the caller's stream. Only the vector-gate tensor-core form (tc_vg.cu) takes
+// memory: a stream-ordered workspace from a pool the library owns.
 #include <math.h>
 
 #include "common.cuh"
@@ -45,6 +46,15 @@ gdn_status_t check_prefill(const void *q, const void *k, const void *v, const fl
 }
 
 }  // namespace
+
+namespace gdn {
+// Vector-valued gates on the tensor cores (dense batches; tc_vg.cu): a per-chunk prep kernel
+// and a per-head chain kernel with a stream-ordered workspace. *fallback is set when the call
+// cannot run there (no workspace, or too many chunks); nothing has been launched then.
+gdn_status_t launch_tc_vg(bool delta, const void *q, const void *k, const void *v, const float *beta, const float *g,
+                          void *o, const float *s0, float *s_final, int B, int H, int L, float scale, FwdOpts oo,
+                          cudaStream_t stream, bool *fallback);
+}  // namespace gdn
 
 extern "C" {
 
@@ -150,7 +160,14 @@ static gdn_status_t prefill_ex(bool delta, const void *q, const void *k, const v
     if (!opt_aligned4(beta)) return GDN_ERR_INVALID_ARG;
     if ((double)B * H * (double)L * dk > 9.0e18) return GDN_ERR_INVALID_ARG;   // g of (rows, dk)
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
-    // vector-valued gates run on the fp32 chunk kernel (any input dtype and size)
+    // vector-valued gates: the two tensor-core kernels for dense bf16 batches at dk = dv = 128,
+    // C = 64; the fp32 chunk kernel for every other input dtype, size and layout
+    if (gdn::tc_supported(in_dtype, dk, dv, chunk) && L > 0 && oo.gate_per_key && !cu_seqlens) {
+        bool fallback = false;
+        const gdn_status_t vs = gdn::launch_tc_vg(delta, q, k, v, beta, g, o, s0, s_final, B, H, L, scale, oo,
+                                                  stream, &fallback);
+        if (!fallback) return vs;
+    }
     if (gdn::tc_supported(in_dtype, dk, dv, chunk) && L > 0 && !oo.gate_per_key)
         return delta ? gdn::launch_tc_gdn(q, k, v, beta, g, o, s0, s_final, cu_seqlens, B, H, L, scale, oo, stream)
                      : gdn::launch_tc_la(q, k, v, g, o, s0, s_final, cu_seqlens, B, H, L, scale, oo, stream);

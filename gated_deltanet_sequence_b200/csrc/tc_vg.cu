@@ -1,0 +1,890 @@
+// Tensor-core chunkwise prefill with vector-valued gates (one log-decay per token and key
+// coordinate) for sm_100a: Gated DeltaNet and gated linear attention, bf16 inputs,
+// dk = dv = 128, chunk C = 64, fp32 accumulation, output and state.
+//
+// The recurrence (page "混合注意力学习(1)", section "Gated DeltaNet", with the decay read per
+// key coordinate, a GLA-style gate): row j of the state decays by exp(g_t[j]) before the
+// token's read and write,
+//   S_t = (I - beta_t k_t k_t^T) diag(exp(g_t)) S_{t-1} + beta_t k_t v_t^T,   o_t = scale S_t^T q_t
+// (linear attention: S_t = diag(exp(g_t)) S_{t-1} + k_t v_t^T). Per chunk of C rows, with
+// G_r[j] the within-chunk cumulative log-decay of coordinate j up to row r and GL = G of the
+// chunk's last row (sections "DeltaNet 分块并行机制" and "HouseHolder变换和WY表示" of the same
+// page, with the scalar decay factors replaced by per-coordinate ones):
+//   A_rs = beta_r sum_j k_r[j] k_s[j] exp(G_r[j] - G_s[j])    (s < r)
+//   P_rs = scale sum_j q_r[j] k_s[j] exp(G_r[j] - G_s[j])      (s <= r)
+//   T = (I + A)^-1,  W = T diag(beta) (K o exp(G)),  U = T diag(beta) V
+//   Ut = U - W S,   O = (scale Q o exp(G)) S + P Ut,   S <- diag(exp(GL)) S + (K o exp(GL - G))^T Ut
+// (linear attention: T = I, W = 0, U = V). Only the last line and the two products with S
+// before it depend on the previous chunk, so a call runs as two kernels:
+//
+//   vg_prep_kernel   one CTA per chunk of every head (two CTAs per SM): the per-coordinate
+//                    gate sums, the decay-weighted Gram on the tensor cores, the UT solve and
+//                    the W / U products. It writes one record per chunk to a workspace:
+//                    Q'^T = (scale Q o exp(G))^T, -W^T, Kd^T = (K o exp(GL - G))^T, U^T and P
+//                    (fp16, 128-byte rows), plus exp(GL) (fp32).
+//   vg_chain_kernel  one CTA per (sequence, head): the fp32 state lives in tensor memory; per
+//                    chunk the record arrives by TMA and the chain takes three products,
+//                    [O^T | Ut^T] += S^T [Q'^T | -W^T] (Ut^T preloaded with U^T),
+//                    S <- exp(GL) o S + Kd^T Ut and O^T += Ut^T P^T.
+//
+// The decay-weighted Gram: exp(G_r - G_s) = exp(G_r - c) exp(c - G_s) with c[j] the midpoint
+// of coordinate j's range of G over the chunk, so the UMMA takes [K o e; Q o e] (K o 1/e)^T
+// with fp16 factors within [e^-6, e^6] whenever that range is at most 12 ("fast"
+// coordinates). The other coordinates are zero in those tiles and their exact terms,
+// one exp per element, are added on the CUDA cores; when more than 32 coordinates of a chunk
+// are such, the whole Gram of that chunk is formed that way. Every other factor (exp(G),
+// exp(GL - G), exp(GL)) is at most 1 for non-positive log-decays and is formed directly.
+#include <mutex>
+
+#include "tc_gdn_parts.cuh"
+
+namespace gdn {
+
+namespace {
+using namespace ptx;
+using namespace tcgdn;
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+        : "memory");
+}
+__device__ __forceinline__ void st_shared_b32(uint32_t addr, uint32_t a) {
+    asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(a) : "memory");
+}
+__device__ __forceinline__ float h_lo(uint32_t w) { return __low2float(*reinterpret_cast<const __half2 *>(&w)); }
+__device__ __forceinline__ float h_hi(uint32_t w) { return __high2float(*reinterpret_cast<const __half2 *>(&w)); }
+
+// ---- the per-chunk record (fp16, rows of 64 values = 128 bytes)
+constexpr int kRQ = 0;        // Q'^T: row j holds scale q_r[j] exp(G_r[j]), r = 0..63
+constexpr int kRW = 128;      // -W^T: row j holds -W[r][j]
+constexpr int kRKD = 256;     // Kd^T: row j holds k_r[j] exp(GL[j] - G_r[j])
+constexpr int kRU = 384;      // U^T: row v holds U[r][v]
+constexpr int kRP = 512;      // P: row r holds P[r][s], s = 0..63
+constexpr int kRecRows = 576;
+constexpr uint32_t kRecBytes = kRecRows * 128u;   // 73728 (a multiple of 1024)
+constexpr int kBoxRows = 192;                     // TMA box: 192 rows x 64 values, three per record
+constexpr float kSpanFast = 12.f;                 // coordinate's range of G within a chunk, factored Gram
+constexpr int kSlowCap = 32;                      // at most this many exact coordinates next to the UMMA Gram
+
+// ================================================================== prep kernel
+constexpr int kVPThreads = 256;
+// shared memory (byte offsets from a 1024-aligned base)
+constexpr uint32_t VP_KA = 0;          // per key half h at h * 16384: [K o e rows 0-63 | Q o e rows 0-63]
+constexpr uint32_t VP_KB = 32768;      // K o (1/e), per key half at h * 8192
+constexpr uint32_t VP_AT = 49152;      // A^T fp32 64 x 64; before it the gate sums, then exact-coordinate data
+constexpr uint32_t VP_TF = 0;          // T fp32 64 x 68 (once the Gram operands are dead)
+constexpr int kTP = 68;
+constexpr uint32_t VP_RS = 17408;      // 4 x 16 x 16 fp32 block scratch of the solve
+constexpr uint32_t VP_KG = 65536;      // K o exp(G), per key half at h * 8192 (rows r; MN-major A of W^T)
+constexpr uint32_t VP_V = 81920;       // V, per value half at h * 8192 (TMA, bf16 -> fp16 in place)
+constexpr uint32_t VP_T2 = 98304;      // T diag(beta) fp16, K-major 64 x 64
+constexpr uint32_t VP_VEC = 106496;    // beta[64] | slot u8[128] | count | bars | tmem | abort
+constexpr uint32_t kVPSmem = VP_VEC + 1024;
+constexpr uint32_t kVPAlloc = kVPSmem + 1024;
+static_assert(kVPAlloc * 2 + 2048 <= 233472, "two prep CTAs per SM");
+constexpr uint32_t V_BETA = 0, V_SLOT = 256, V_NSLOW = 384, V_BARS = 448, V_TMEM = 480, V_ABORT = 484;
+// tensor memory (256 columns)
+constexpr uint32_t TMV_G = 0, TMV_W = 64, TMV_U = 128;
+constexpr uint32_t ID_G16 = idesc_f16(128, 64, false, false);   // Gram: both K-major, fp16
+constexpr uint32_t ID_WU = idesc_f16(128, 64, true, false);     // W^T, U^T: A MN-major
+enum : int { VB_V = 0, VB_G = 1, VB_WU = 2, kVPBars = 3 };
+
+template <bool DELTA>
+__global__ void __launch_bounds__(kVPThreads, 2)
+vg_prep_kernel(const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__restrict__ q,
+               const __nv_bfloat16 *__restrict__ k, const float *__restrict__ beta, const float *__restrict__ g,
+               uint8_t *__restrict__ recs, float *__restrict__ egl, int L, int nch, float scale,
+               long long wait_limit, unsigned *__restrict__ err_word) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const uint32_t sb = smem_u32(smem);
+    uint8_t *vec = smem + VP_VEC;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(vec + V_BARS);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(vec + V_TMEM);
+    int *abort_flag = reinterpret_cast<int *>(vec + V_ABORT);
+    const Ctl ctl{bars, abort_flag, err_word, wait_limit};
+    float *betav = reinterpret_cast<float *>(vec + V_BETA);
+    uint8_t *slot = vec + V_SLOT;
+    int *nslow_p = reinterpret_cast<int *>(vec + V_NSLOW);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const long long rec_id = blockIdx.x;
+    const int bh = static_cast<int>(rec_id / nch), c = static_cast<int>(rec_id - static_cast<long long>(bh) * nch);
+    const int nvalid = min(kC, L - c * kC);
+    const size_t row0 = static_cast<size_t>(bh) * L + static_cast<size_t>(c) * kC;
+    uint8_t *rec = recs + static_cast<size_t>(rec_id) * kRecBytes;
+
+    if (tid == 0) {
+        for (int b = 0; b < kVPBars; ++b) mbar_init(&bars[b], 1);
+        *abort_flag = 0;
+        *nslow_p = 0;
+        fence_mbar_init();
+        // V of this chunk (two value halves; rows past L read as zeros)
+        mbar_arrive_expect_tx(&bars[VB_V], 16384);
+        tma_load_3d(smem + VP_V, &tm_v, &bars[VB_V], 0, c * kC, bh);
+        tma_load_3d(smem + VP_V + 8192, &tm_v, &bars[VB_V], 64, c * kC, bh);
+    }
+    if (tid < kC) betav[tid] = (DELTA && tid < nvalid) ? beta[row0 + tid] : 0.f;
+    for (int i = tid; i < 8192 / 16; i += kVPThreads)      // T2: upper blocks stay zero
+        *reinterpret_cast<uint4 *>(smem + VP_T2 + i * 16) = make_uint4(0u, 0u, 0u, 0u);
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 256);
+        tmem_relinquish();
+    }
+
+    // ---- gate sums and the operand tiles: thread (p, h) takes coordinates 2p, 2p+1 and
+    //      rows 16h .. 16h+15
+    const int p = tid & 63, h = tid >> 6;
+    const int j0 = 2 * p, kh = j0 >> 6, jc = j0 & 63, r0 = 16 * h;
+    float G0[16], G1[16];
+    uint32_t kw[16], qw[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int r = r0 + i;
+        if (r < nvalid) {
+            const size_t e = (row0 + r) * kD + j0;
+            const float2 gg = *reinterpret_cast<const float2 *>(g + e);
+            G0[i] = gg.x;
+            G1[i] = gg.y;
+            kw[i] = *reinterpret_cast<const uint32_t *>(k + e);
+            qw[i] = *reinterpret_cast<const uint32_t *>(q + e);
+        } else {
+            G0[i] = G1[i] = 0.f;
+            kw[i] = qw[i] = 0u;
+        }
+    }
+#pragma unroll
+    for (int i = 1; i < 16; ++i) {
+        G0[i] += G0[i - 1];
+        G1[i] += G1[i - 1];
+    }
+    float *tot = reinterpret_cast<float *>(smem + VP_AT);   // [4][128] quarter sums, then min, max
+    tot[h * 128 + j0] = G0[15];
+    tot[h * 128 + j0 + 1] = G1[15];
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    float o0 = 0.f, o1 = 0.f, gl0 = 0.f, gl1 = 0.f;
+#pragma unroll
+    for (int hh = 0; hh < 4; ++hh) {
+        const float a = tot[hh * 128 + j0], b = tot[hh * 128 + j0 + 1];
+        if (hh < h) {
+            o0 += a;
+            o1 += b;
+        }
+        gl0 += a;
+        gl1 += b;
+    }
+    float mn0 = 3.0e38f, mx0 = -3.0e38f, mn1 = 3.0e38f, mx1 = -3.0e38f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        G0[i] += o0;
+        G1[i] += o1;
+        mn0 = fminf(mn0, G0[i]);
+        mx0 = fmaxf(mx0, G0[i]);
+        mn1 = fminf(mn1, G1[i]);
+        mx1 = fmaxf(mx1, G1[i]);
+    }
+    tot[512 + h * 128 + j0] = mn0;
+    tot[512 + h * 128 + j0 + 1] = mn1;
+    tot[1024 + h * 128 + j0] = mx0;
+    tot[1024 + h * 128 + j0 + 1] = mx1;
+    __syncthreads();
+    float lo0 = tot[512 + j0], lo1 = tot[512 + j0 + 1], hi0 = tot[1024 + j0], hi1 = tot[1024 + j0 + 1];
+#pragma unroll
+    for (int hh = 1; hh < 4; ++hh) {
+        lo0 = fminf(lo0, tot[512 + hh * 128 + j0]);
+        lo1 = fminf(lo1, tot[512 + hh * 128 + j0 + 1]);
+        hi0 = fmaxf(hi0, tot[1024 + hh * 128 + j0]);
+        hi1 = fmaxf(hi1, tot[1024 + hh * 128 + j0 + 1]);
+    }
+    const bool f0 = hi0 - lo0 <= kSpanFast, f1 = hi1 - lo1 <= kSpanFast;   // false for NaN ranges
+    if (h == 0) {
+        if (!f0) {
+            const int f = atomicAdd(nslow_p, 1);
+            slot[j0] = static_cast<uint8_t>(f);
+        }
+        if (!f1) {
+            const int f = atomicAdd(nslow_p, 1);
+            slot[j0 + 1] = static_cast<uint8_t>(f);
+        }
+        egl[static_cast<size_t>(rec_id) * kD + j0] = __expf(gl0);
+        egl[static_cast<size_t>(rec_id) * kD + j0 + 1] = __expf(gl1);
+    }
+    __syncthreads();   // gate sums read; the slow list is complete
+    const int nslow = *nslow_p;
+    const bool allslow = nslow > kSlowCap;
+    const bool fa0 = f0 && !allslow, fa1 = f1 && !allslow;
+    const float c0 = 0.5f * (lo0 + hi0), c1 = 0.5f * (lo1 + hi1);
+    const float ec0 = fa0 ? __expf(c0) : 0.f, ec1 = fa1 ? __expf(c1) : 0.f;
+    const float edc0 = fa0 ? __expf(gl0 - c0) : 0.f, edc1 = fa1 ? __expf(gl1 - c1) : 0.f;
+    uint32_t qT0[8], qT1[8], dT0[8], dT1[8];   // fp16 pairs along r for the transposed record rows
+    float pq0 = 0.f, pq1 = 0.f, pd0 = 0.f, pd1 = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int r = r0 + i;
+        const float k0 = bf_lo(kw[i]), k1 = bf_hi(kw[i]), q0 = bf_lo(qw[i]), q1 = bf_hi(qw[i]);
+        float ka0 = 0.f, qa0 = 0.f, kb0 = 0.f, eg0, ed0, ka1 = 0.f, qa1 = 0.f, kb1 = 0.f, eg1, ed1;
+        if (fa0) {
+            const float e1 = __expf(G0[i] - c0), e2 = __expf(c0 - G0[i]);
+            ka0 = k0 * e1;
+            qa0 = q0 * e1;
+            kb0 = k0 * e2;
+            eg0 = e1 * ec0;
+            ed0 = e2 * edc0;
+        } else {
+            eg0 = __expf(G0[i]);
+            ed0 = __expf(gl0 - G0[i]);
+        }
+        if (fa1) {
+            const float e1 = __expf(G1[i] - c1), e2 = __expf(c1 - G1[i]);
+            ka1 = k1 * e1;
+            qa1 = q1 * e1;
+            kb1 = k1 * e2;
+            eg1 = e1 * ec1;
+            ed1 = e2 * edc1;
+        } else {
+            eg1 = __expf(G1[i]);
+            ed1 = __expf(gl1 - G1[i]);
+        }
+        const uint32_t sw = sw128(r, jc >> 3) + (jc & 7) * 2;
+        if (!allslow) {
+            st_shared_b32(sb + VP_KA + kh * 16384 + sw, pack_h2(ka0, ka1));
+            st_shared_b32(sb + VP_KA + kh * 16384 + 8192 + sw, pack_h2(qa0, qa1));
+            st_shared_b32(sb + VP_KB + kh * 8192 + sw, pack_h2(kb0, kb1));
+        }
+        st_shared_b32(sb + VP_KG + kh * 8192 + sw, pack_h2(k0 * eg0, k1 * eg1));
+        const float qp0 = scale * q0 * eg0, qp1 = scale * q1 * eg1, kd0 = k0 * ed0, kd1 = k1 * ed1;
+        if (i & 1) {
+            qT0[i >> 1] = pack_h2(pq0, qp0);
+            qT1[i >> 1] = pack_h2(pq1, qp1);
+            dT0[i >> 1] = pack_h2(pd0, kd0);
+            dT1[i >> 1] = pack_h2(pd1, kd1);
+        } else {
+            pq0 = qp0;
+            pq1 = qp1;
+            pd0 = kd0;
+            pd1 = kd1;
+        }
+        if ((i & 7) == 7) {
+            // rows j0, j0+1 of Q'^T and Kd^T: the 8 values r = r0 + i - 7 .. r0 + i
+            const int b = (i >> 3) * 4, off = 32 * h + 16 * (i >> 3);
+            uint8_t *rq = rec + static_cast<size_t>(kRQ + j0) * 128 + off;
+            uint8_t *rd = rec + static_cast<size_t>(kRKD + j0) * 128 + off;
+            *reinterpret_cast<uint4 *>(rq) = make_uint4(qT0[b], qT0[b + 1], qT0[b + 2], qT0[b + 3]);
+            *reinterpret_cast<uint4 *>(rq + 128) = make_uint4(qT1[b], qT1[b + 1], qT1[b + 2], qT1[b + 3]);
+            *reinterpret_cast<uint4 *>(rd) = make_uint4(dT0[b], dT0[b + 1], dT0[b + 2], dT0[b + 3]);
+            *reinterpret_cast<uint4 *>(rd + 128) = make_uint4(dT1[b], dT1[b + 1], dT1[b + 2], dT1[b + 3]);
+        }
+    }
+    // exact coordinates: G (fp32), k and q (bf16) by coordinate slot, rows contiguous
+    const int NF = allslow ? kD : kSlowCap;
+    const uint32_t sbase = allslow ? 0u : VP_AT;
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+        const bool ex = allslow || !(e ? f1 : f0);
+        if (!ex) continue;
+        const int j = j0 + e;
+        const int f = allslow ? j : slot[j];
+        const float *Gv = e ? G1 : G0;
+        float *sg = reinterpret_cast<float *>(smem + sbase) + f * 64 + r0;
+#pragma unroll
+        for (int i = 0; i < 16; i += 4)
+            *reinterpret_cast<float4 *>(sg + i) = make_float4(Gv[i], Gv[i + 1], Gv[i + 2], Gv[i + 3]);
+        uint32_t kk[8], qq[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t a = kw[2 * i], b = kw[2 * i + 1], x = qw[2 * i], y = qw[2 * i + 1];
+            kk[i] = e ? ((a >> 16) | (b & 0xFFFF0000u)) : ((a & 0xFFFFu) | (b << 16));
+            qq[i] = e ? ((x >> 16) | (y & 0xFFFF0000u)) : ((x & 0xFFFFu) | (y << 16));
+        }
+        uint8_t *sk = smem + sbase + NF * 256 + f * 128 + r0 * 2;
+        uint8_t *sq = smem + sbase + NF * 384 + f * 128 + r0 * 2;
+        *reinterpret_cast<uint4 *>(sk) = make_uint4(kk[0], kk[1], kk[2], kk[3]);
+        *reinterpret_cast<uint4 *>(sk + 16) = make_uint4(kk[4], kk[5], kk[6], kk[7]);
+        *reinterpret_cast<uint4 *>(sq) = make_uint4(qq[0], qq[1], qq[2], qq[3]);
+        *reinterpret_cast<uint4 *>(sq + 16) = make_uint4(qq[4], qq[5], qq[6], qq[7]);
+    }
+    fence_proxy_async();
+    __syncthreads();
+
+    // ---- decay-weighted Gram [K o e; Q o e] (K o 1/e)^T: rows 0-63 -> A, 64-127 -> P
+    bool ok = true;
+    if (!allslow) {
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+                mma_f16(tmem + TMV_G, sdesc_sw128(sb + VP_KA + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                        sdesc_sw128(sb + VP_KB + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), ID_G16, kk > 0);
+            mma_commit(&bars[VB_G]);
+        }
+        ok = ctl.wait(VB_G, 0);
+        tc_fence_after();
+    }
+    const int sub = warp & 3, hh = warp >> 2, R = sub * 32 + lane;
+    const int r = R & 63;
+    const bool isP = R >= 64;
+    const uint32_t trow = tmem + (static_cast<uint32_t>(sub * 32) << 16);
+    float v[32];
+    if (!allslow && !__syncthreads_or(!ok)) {
+        ld_cols<32>(trow + TMV_G + 32 * hh, v);
+    } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = 0.f;
+    }
+    if (nslow > 0 && r >= 32 * hh && (DELTA || isP)) {
+        // exact terms of the coordinates left out of the factored Gram
+        const float *SG = reinterpret_cast<const float *>(smem + sbase);
+        const __nv_bfloat16 *SK = reinterpret_cast<const __nv_bfloat16 *>(smem + sbase + NF * 256);
+        const __nv_bfloat16 *SX = reinterpret_cast<const __nv_bfloat16 *>(smem + sbase + NF * (isP ? 384 : 256));
+        const int nf = allslow ? kD : nslow;
+#pragma unroll 1
+        for (int f = 0; f < nf; ++f) {
+            const float Gr = SG[f * 64 + r], xr = __bfloat162float(SX[f * 64 + r]);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const int s = 32 * hh + e;
+                if (s < r || (isP && s == r))
+                    v[e] = fmaf(xr * __bfloat162float(SK[f * 64 + s]), __expf(Gr - SG[f * 64 + s]), v[e]);
+            }
+        }
+    }
+    tc_fence_before();
+    ok = !__syncthreads_or(!ok);   // Gram and exact-coordinate data read: A^T may overwrite them
+    if (!isP) {
+        if (DELTA) {
+            float *At = reinterpret_cast<float *>(smem + VP_AT);   // At[s * 64 + r] = A[r][s]
+            const float br = betav[r];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) At[(32 * hh + e) * 64 + r] = (32 * hh + e < r) ? br * v[e] : 0.f;
+        }
+    } else {
+        uint8_t *prow = rec + static_cast<size_t>(kRP + r) * 128 + 64 * hh;
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+            float pv[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) pv[e] = (32 * hh + 8 * ch + e <= r) ? scale * v[8 * ch + e] : 0.f;
+            *reinterpret_cast<uint4 *>(prow + 16 * ch) =
+                make_uint4(pack_h2(pv[0], pv[1]), pack_h2(pv[2], pv[3]), pack_h2(pv[4], pv[5]), pack_h2(pv[6], pv[7]));
+        }
+    }
+    __syncthreads();   // A^T complete
+
+    // ---- UT solve (warps 0-3) while warps 4-7 convert V to fp16
+    if (warp < 4) {
+        const float *At = reinterpret_cast<const float *>(smem + VP_AT);
+        float *Tf = reinterpret_cast<float *>(smem + VP_TF);    // Tf[r * kTP + c] = T[r][c]
+        if (!DELTA) {
+            // linear attention: T = I, so T diag(beta) is the identity (U = V)
+            if (tid < 64)
+                *reinterpret_cast<__half *>(smem + VP_T2 + sw128(tid, tid >> 3) + (tid & 7) * 2) = __float2half_rn(1.f);
+        } else {
+            // one 16 x 16 block (bi, bj) of Tf -> T2 = T diag(beta) (K-major rows r)
+            auto emit = [&](int bi2, int bj2) {
+                __syncwarp();
+                const int rr = 16 * bi2 + (lane >> 1), cc0 = 16 * bj2 + 8 * (lane & 1);
+                const float4 b0 = *reinterpret_cast<const float4 *>(betav + cc0);
+                const float4 b1 = *reinterpret_cast<const float4 *>(betav + cc0 + 4);
+                const float4 t0 = *reinterpret_cast<const float4 *>(Tf + rr * kTP + cc0);
+                const float4 t1 = *reinterpret_cast<const float4 *>(Tf + rr * kTP + cc0 + 4);
+                st_shared_v4(sb + VP_T2 + sw128(rr, cc0 >> 3), pack_h2(t0.x * b0.x, t0.y * b0.y),
+                             pack_h2(t0.z * b0.z, t0.w * b0.w), pack_h2(t1.x * b1.x, t1.y * b1.y),
+                             pack_h2(t1.z * b1.z, t1.w * b1.w));
+            };
+            const int bi = warp, cl = lane & 15;
+            {
+                // diagonal block D_i = (I + A_ii)^-1 by right-looking substitution (lane = column)
+                float acc[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) acc[i] = (i == cl) ? 1.f : 0.f;
+#pragma unroll
+                for (int s2 = 0; s2 < 15; ++s2) {
+                    const float xs = acc[s2];
+                    const float *arow = At + (16 * bi + s2) * 64 + 16 * bi;
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        if (4 * k4 + 3 <= s2) continue;
+                        const float4 a4 = *reinterpret_cast<const float4 *>(arow + 4 * k4);
+                        acc[4 * k4 + 0] = fmaf(-a4.x, xs, acc[4 * k4 + 0]);
+                        acc[4 * k4 + 1] = fmaf(-a4.y, xs, acc[4 * k4 + 1]);
+                        acc[4 * k4 + 2] = fmaf(-a4.z, xs, acc[4 * k4 + 2]);
+                        acc[4 * k4 + 3] = fmaf(-a4.w, xs, acc[4 * k4 + 3]);
+                    }
+                }
+                if (lane < 16) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) Tf[(16 * bi + i) * kTP + 16 * bi + cl] = acc[i];
+                }
+            }
+            asm volatile("bar.sync 3, 128;" ::: "memory");
+            emit(bi, bi);
+            float *Rw = reinterpret_cast<float *>(smem + VP_RS);
+            // T_10 = -D_1 (A_10 D_0), T_32 = -D_3 (A_32 D_2)
+            if (bi < 2) {
+                const int i = 2 * bi + 1, j = 2 * bi;
+                float *Rb = Rw + bi * 256;
+                float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                block_mm<2>(acc2, [&](int rr, int kx) { return At[(16 * j + kx) * 64 + 16 * i + rr]; },
+                            [&](int kx, int n) { return Tf[(16 * j + kx) * kTP + 16 * j + n]; }, lane);
+                block_store(acc2, [&](int rr, int n, float x) { Rb[rr * 16 + n] = x; }, lane, 1.f);
+                __syncwarp();
+                float acc3[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                block_mm<2>(acc3, [&](int rr, int kx) { return Tf[(16 * i + rr) * kTP + 16 * i + kx]; },
+                            [&](int kx, int n) { return Rb[kx * 16 + n]; }, lane);
+                block_store(acc3, [&](int rr, int n, float x) { Tf[(16 * i + rr) * kTP + 16 * j + n] = x; }, lane,
+                            -1.f);
+                emit(i, j);
+            }
+            asm volatile("bar.sync 3, 128;" ::: "memory");
+            // X_ij = A_{i,0..1} T_{0..1,j} for (i, j) = (2 + w / 2, w % 2)
+            const int ii = 2 + (bi >> 1), jj = bi & 1;
+            {
+                float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                if (jj == 0)
+                    block_mm<4>(acc2, [&](int rr, int kx) { return At[kx * 64 + 16 * ii + rr]; },
+                                [&](int kx, int n) { return Tf[kx * kTP + n]; }, lane);
+                else
+                    block_mm<2>(acc2, [&](int rr, int kx) { return At[(16 + kx) * 64 + 16 * ii + rr]; },
+                                [&](int kx, int n) { return Tf[(16 + kx) * kTP + 16 + n]; }, lane);
+                float *Rb = Rw + bi * 256;
+                block_store(acc2, [&](int rr, int n, float x) { Rb[rr * 16 + n] = x; }, lane, 1.f);
+            }
+            asm volatile("bar.sync 3, 128;" ::: "memory");
+            // T_2j = -D_2 X_2j,  T_3j = -(T_32 X_2j + D_3 X_3j)
+            {
+                const float *X2 = Rw + jj * 256, *X3 = Rw + (2 + jj) * 256;
+                float acc3[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                if (ii == 2)
+                    block_mm<2>(acc3, [&](int rr, int kx) { return Tf[(32 + rr) * kTP + 32 + kx]; },
+                                [&](int kx, int n) { return X2[kx * 16 + n]; }, lane);
+                else
+                    block_mm<4>(acc3, [&](int rr, int kx) { return Tf[(48 + rr) * kTP + 32 + kx]; },
+                                [&](int kx, int n) { return kx < 16 ? X2[kx * 16 + n] : X3[(kx - 16) * 16 + n]; },
+                                lane);
+                block_store(acc3, [&](int rr, int n, float x) { Tf[(16 * ii + rr) * kTP + 16 * jj + n] = x; }, lane,
+                            -1.f);
+                emit(ii, jj);
+            }
+        }
+    } else {
+        const int t4 = tid - 128;
+        bool vok = true;
+        if (t4 == 0) vok = ctl.wait(VB_V, 0);
+        vok = __shfl_sync(0xffffffffu, vok ? 1 : 0, 0) != 0;   // warp 4 lane 0 polled
+        asm volatile("bar.sync 4, 128;" ::: "memory");
+        if (warp != 4) vok = !ctl.aborted();
+        if (vok) convert_tile_bf16_to_f16(smem + VP_V, 16384, t4, 128);
+        ok = ok && vok;
+    }
+    fence_proxy_async();
+    ok = !__syncthreads_or(!ok);
+
+    // ---- W^T = (K o exp(G))^T (T diag(beta))^T and U^T = V^T (T diag(beta))^T
+    const bool wu_issued = ok;
+    if (ok && tid == 0) {
+        tc_fence_after();
+        if (DELTA) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                mma_f16(tmem + TMV_W, sdesc_sw128(sb + VP_KG + kk * 2048, 8192, 1024),
+                        sdesc_sw128(sb + VP_T2 + kk * 32, 16, 1024), ID_WU, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+            mma_f16(tmem + TMV_U, sdesc_sw128(sb + VP_V + kk * 2048, 8192, 1024),
+                    sdesc_sw128(sb + VP_T2 + kk * 32, 16, 1024), ID_WU, kk > 0);
+        mma_commit(&bars[VB_WU]);
+    }
+    if (ok) ok = ctl.wait(VB_WU, 0);
+    tc_fence_after();
+    if (!__syncthreads_or(!ok)) {
+        // warps 0-3: -W^T rows j; warps 4-7: U^T rows v (one TMEM lane each)
+        if (warp >= 4 || DELTA) {
+            const int row = (warp >= 4 ? kRU : kRW) + R;
+            const float sg = warp >= 4 ? 1.f : -1.f;
+            uint8_t *dst = rec + static_cast<size_t>(row) * 128;
+            float x[64];
+            ld_cols<64>(trow + (warp >= 4 ? TMV_U : TMV_W), x);
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch)
+                *reinterpret_cast<uint4 *>(dst + 16 * ch) =
+                    make_uint4(pack_h2(sg * x[8 * ch], sg * x[8 * ch + 1]), pack_h2(sg * x[8 * ch + 2], sg * x[8 * ch + 3]),
+                               pack_h2(sg * x[8 * ch + 4], sg * x[8 * ch + 5]),
+                               pack_h2(sg * x[8 * ch + 6], sg * x[8 * ch + 7]));
+        }
+    }
+    // never leave a copy or a UMMA in flight past the end of the CTA
+    if (tid == 0) {
+        ctl.drain(VB_V, 0);
+        if (!allslow) ctl.drain(VB_G, 0);
+        if (wu_issued) ctl.drain(VB_WU, 0);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+// ================================================================== chain kernel
+constexpr int kVCThreads = 192;
+constexpr uint32_t VC_S = 2 * kRecBytes;        // S fp16 MN-major A: 2 x (128 key rows x 64 v)
+constexpr uint32_t VC_UB = VC_S + 32768;        // Ut fp16, K-major rows v
+constexpr uint32_t VC_XN = VC_UB + 16384;       // output-normalisation scratch (384 fp32)
+constexpr uint32_t VC_BAR = VC_XN + 1536;       // mbarriers, TMEM base, abort flag
+constexpr uint32_t kVCSmem = VC_BAR + 256;
+constexpr uint32_t kVCAlloc = kVCSmem + 1024;
+static_assert(kVCAlloc <= 232448, "shared memory budget");
+static_assert(VC_S % 1024 == 0 && VC_UB % 1024 == 0, "UMMA tiles need 1024-B alignment");
+constexpr uint32_t TMC_S = 0;      // state S: lane = key row j, 128 value columns
+constexpr uint32_t TMC_OU = 128;   // 2 x [O^T | U^T then Ut^T]: lane = value v
+constexpr uint32_t ID_SQW = idesc_f16(128, 128, true, true);   // [O^T | Ut^T] += S^T [Q'^T | -W^T]
+constexpr uint32_t ID_SQ = idesc_f16(128, 64, true, true);     // O^T += S^T Q'^T (linear attention)
+constexpr uint32_t ID_ST = idesc_f16(128, 128, false, false);  // S += Kd^T Ut
+constexpr uint32_t ID_O = idesc_f16(128, 64, false, false);    // O^T += Ut^T P^T
+constexpr int kBarS = 1;
+enum : int { CB_FULL = 0, CB_CDONE = 2, CB_SRDY = 4, CB_ADONE = 5, CB_URDY = 6, kVCBars = 7 };
+
+template <bool DELTA, bool OPTS>
+__global__ void __launch_bounds__(kVCThreads, 1)
+vg_chain_kernel(const __grid_constant__ CUtensorMap tm_rec, const float *__restrict__ egl, const OutArgs out,
+                const float *__restrict__ s0, float *__restrict__ s_final, int H, int L, int nch,
+                long long wait_limit, unsigned *__restrict__ err_word) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const uint32_t sb = smem_u32(smem);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + VC_BAR);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kVCBars);
+    int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
+    const Ctl ctl{bars, abort_flag, err_word, wait_limit};
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int bh = blockIdx.x;
+    const size_t row0 = static_cast<size_t>(bh) * L;
+    const long long rec0 = static_cast<long long>(bh) * nch;
+
+    if (tid == 0) {
+        for (int b = 0; b < kVCBars; ++b) mbar_init(&bars[b], 1);
+        abort_flag[0] = 0;
+        fence_mbar_init();
+        prefetch_tmap(&tm_rec);
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ================================================================ TMA producer
+        if (lane == 0) {
+            int last[2] = {-1, -1};
+            for (int c = 0; c < nch; ++c) {
+                const int s = c & 1;
+                if (c >= 2 && !ctl.wait_lazy(CB_CDONE + s, ((c - 2) >> 1) & 1)) break;
+                uint64_t *fb = &bars[CB_FULL + s];
+                mbar_arrive_expect_tx(fb, kRecBytes);
+                const int row = static_cast<int>((rec0 + c) * kRecRows);
+#pragma unroll
+                for (int b = 0; b < kRecRows / kBoxRows; ++b)
+                    tma_load_2d(smem + s * kRecBytes + b * kBoxRows * 128, &tm_rec, fb, 0, row + b * kBoxRows);
+                last[s] = c;
+            }
+            for (int s = 0; s < 2; ++s)
+                if (last[s] >= 0) ctl.drain(CB_FULL + s, (last[s] >> 1) & 1);
+        }
+    } else if (warp == 1) {
+        // ================================================================ chain UMMA issuer
+        if (lane == 0) {
+            int last_bar = -1, last_par = 0;
+            for (int c = 0; c < nch; ++c) {
+                const int s = c & 1;
+                const uint32_t stg = sb + s * kRecBytes;
+                if (!ctl.wait(CB_FULL + s, (c >> 1) & 1)) break;
+                if (!ctl.wait(CB_SRDY, c & 1)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_f16(tmem + TMC_OU + s * 128, sdesc_sw128(sb + VC_S + kk * 2048, 16384, 1024),
+                            sdesc_sw128(stg + kRQ * 128 + kk * 2048, (kRW - kRQ) * 128, 1024), DELTA ? ID_SQW : ID_SQ,
+                            1u);
+                mma_commit(&bars[CB_ADONE]);
+                last_bar = CB_ADONE;
+                last_par = c & 1;
+                if (!ctl.wait(CB_URDY, c & 1)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_f16(tmem + TMC_S, sdesc_sw128(stg + kRKD * 128 + kk * 32, 16, 1024),
+                            sdesc_sw128(sb + VC_UB + kk * 32, 16, 1024), ID_ST, 1u);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_f16(tmem + TMC_OU + s * 128, sdesc_sw128(sb + VC_UB + kk * 32, 16, 1024),
+                            sdesc_sw128(stg + kRP * 128 + kk * 32, 16, 1024), ID_O, 1u);
+                mma_commit(&bars[CB_CDONE + s]);
+                last_bar = CB_CDONE + s;
+                last_par = (c >> 1) & 1;
+            }
+            if (last_bar >= 0) ctl.drain(last_bar, last_par);
+        }
+    } else {
+        // ================================================================ state group (warps 2-5)
+        const int j = (warp & 3) * 32 + lane;              // TMEM lane: key row j / value column v
+        const bool lead = (j == 0);
+        const int head = bh % H;
+        float *xn = reinterpret_cast<float *>(smem + VC_XN);
+        const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+        {
+            const float *src = s0 ? s0 + (static_cast<size_t>(bh) * kD + j) * kD : nullptr;
+#pragma unroll 1
+            for (int cc = 0; cc < 8; ++cc) {
+                float rr[16];
+#pragma unroll
+                for (int e = 0; e < 16; e += 4) {
+                    const float4 x = src ? *reinterpret_cast<const float4 *>(src + cc * 16 + e)
+                                         : make_float4(0.f, 0.f, 0.f, 0.f);
+                    rr[e] = x.x; rr[e + 1] = x.y; rr[e + 2] = x.z; rr[e + 3] = x.w;
+                }
+                tmem_st16(trow + TMC_S + cc * 16, rr);
+            }
+            float z[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) z[e] = 0.f;
+#pragma unroll 1
+            for (int cc = 0; cc < 8; ++cc) tmem_st16(trow + TMC_OU + (cc >> 2) * 128 + (cc & 3) * 16, z);
+            tmem_wait_st();
+        }
+        const float *egl_h = egl + static_cast<size_t>(rec0) * kD;
+        float e_next = nch > 0 ? egl_h[j] : 1.f;
+        int done = 0;
+        float nf = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < nch; ++c) {
+            const int s = c & 1;
+            const uint8_t *stg = smem + s * kRecBytes;
+            const float e_cur = e_next;
+            if (c + 1 < nch) e_next = egl_h[static_cast<size_t>(c + 1) * kD + j];
+            // S(c) complete (state update of c-1 done) and this chunk's record landed
+            if (!ctl.group_wait_all({c >= 1 ? CB_CDONE + ((c - 1) & 1) : -1, CB_FULL + s},
+                                    {static_cast<uint32_t>((c - 1) >> 1) & 1u, static_cast<uint32_t>(c >> 1) & 1u},
+                                    kBarS, lead))
+                break;
+            tc_fence_after();
+            // ---- S row j -> fp16 MN-major operand; S <- exp(GL[j]) S (ahead of the update)
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc) {
+                float sv[16];
+                tmem_ld16(trow + TMC_S + cc * 16, sv);
+                tmem_wait_ld();
+                st_row16_h(sb + VC_S + (cc >> 2) * 16384u, j, (cc & 3) * 2, sv);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) sv[e] *= e_cur;
+                tmem_st16(trow + TMC_S + cc * 16, sv);
+            }
+            // ---- U^T row v -> the Ut^T columns of this chunk's tile
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                const uint4 a = *reinterpret_cast<const uint4 *>(stg + sw128(kRU + j, 2 * cc));
+                const uint4 b = *reinterpret_cast<const uint4 *>(stg + sw128(kRU + j, 2 * cc + 1));
+                const float u[16] = {h_lo(a.x), h_hi(a.x), h_lo(a.y), h_hi(a.y), h_lo(a.z), h_hi(a.z),
+                                     h_lo(a.w), h_hi(a.w), h_lo(b.x), h_hi(b.x), h_lo(b.y), h_hi(b.y),
+                                     h_lo(b.z), h_hi(b.z), h_lo(b.w), h_hi(b.w)};
+                tmem_st16(trow + TMC_OU + s * 128 + 64 + cc * 16, u);
+            }
+            tmem_wait_st();
+            fence_proxy_async();
+            tc_fence_before();
+            named_bar(kBarS, 128);
+            if (lead) mbar_arrive(&bars[CB_SRDY]);
+            // ---- output of the previous chunk (its O tile is complete)
+            if (c >= 1) {
+                const int cp = c - 1;
+                store_out_col<OPTS>(trow + TMC_OU + (cp & 1) * 128, out, (row0 + static_cast<size_t>(cp) * kC) * kD + j,
+                                    kC, head, j, kBarS, xn, false, nf);
+                float z[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) z[e] = 0.f;
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) tmem_st16(trow + TMC_OU + (cp & 1) * 128 + cc * 16, z);
+                tmem_wait_st();
+                done = c;
+            }
+            // ---- Ut^T row v -> Ut operand (K-major, rows v)
+            if (!ctl.group_wait(CB_ADONE, c & 1, kBarS, lead)) break;
+            tc_fence_after();
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                float u[16];
+                tmem_ld16(trow + TMC_OU + s * 128 + 64 + cc * 16, u);
+                tmem_wait_ld();
+                st_row16_h(sb + VC_UB, j, 2 * cc, u);
+            }
+            fence_proxy_async();
+            tc_fence_before();
+            named_bar(kBarS, 128);
+            if (lead) mbar_arrive(&bars[CB_URDY]);
+        }
+        // ---- last output tile and the final state
+        if (nch > 0 && done == nch - 1) {
+            const int cp = nch - 1;
+            if (ctl.group_wait(CB_CDONE + (cp & 1), (cp >> 1) & 1, kBarS, lead)) {
+                tc_fence_after();
+                store_out_col<OPTS>(trow + TMC_OU + (cp & 1) * 128, out, (row0 + static_cast<size_t>(cp) * kC) * kD + j,
+                                    L - cp * kC, head, j, kBarS, xn, true, nf);
+                done = nch;
+            }
+        }
+        if (s_final && done == nch) {
+            float *dst = s_final + (static_cast<size_t>(bh) * kD + j) * kD;
+#pragma unroll 1
+            for (int cc = 0; cc < 8; ++cc) {
+                float sv[16];
+                tmem_ld16(trow + TMC_S + cc * 16, sv);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 16; e += 4) {
+                    probe_finite(nf, sv[e] + sv[e + 1] + sv[e + 2] + sv[e + 3]);
+                    *reinterpret_cast<float4 *>(dst + cc * 16 + e) = make_float4(sv[e], sv[e + 1], sv[e + 2], sv[e + 3]);
+                }
+            }
+        }
+        report_nonfinite(ctl.aborted() ? 0.f : nf, err_word);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------- host side
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_fn();
+
+namespace {
+
+// (rows, 64) fp16 record rows -> 2-D map, 64 x 192 boxes, 128-byte swizzle.
+bool make_rec_map(CUtensorMap *m, void *ptr, unsigned long long rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {64, static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {128};
+    const cuuint32_t box[2] = {64, kBoxRows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, ptr, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// One stream-ordered memory pool per device for the per-chunk records; it keeps what it
+// has reserved (release threshold: never), so repeated calls of one size allocate once.
+cudaMemPool_t record_pool(int dev) {
+    static std::mutex mu;
+    static cudaMemPool_t pools[64] = {};
+    if (dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!pools[dev]) {
+        cudaMemPoolProps props = {};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        cudaMemPool_t p = nullptr;
+        if (cudaMemPoolCreate(&p, &props) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        cuuint64_t keep = ~0ull;
+        cudaMemPoolSetAttribute(p, cudaMemPoolAttrReleaseThreshold, &keep);
+        pools[dev] = p;
+    }
+    return pools[dev];
+}
+
+template <bool DELTA, bool OPTS>
+gdn_status_t launch_vg_t(const CUtensorMap &mv, const CUtensorMap &mrec, const void *q, const void *k,
+                         const float *beta, const float *g, uint8_t *recs, float *egl, const OutArgs &out,
+                         const float *s0, float *s_final, int BH, int H, int L, int nch, float scale,
+                         cudaStream_t stream) {
+    auto kp = vg_prep_kernel<DELTA>;
+    auto kc = vg_chain_kernel<DELTA, OPTS>;
+    if (!ensure_smem_limit(reinterpret_cast<const void *>(kp), kVPAlloc) ||
+        !ensure_smem_limit(reinterpret_cast<const void *>(kc), kVCAlloc))
+        return GDN_ERR_CUDA;
+    unsigned *err = device_error_word();
+    if (!err) return GDN_ERR_CUDA;
+    const long long nrec = static_cast<long long>(BH) * nch;
+    kp<<<static_cast<unsigned>(nrec), kVPThreads, kVPAlloc, stream>>>(
+        mv, static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k), beta, g, recs, egl, L, nch,
+        scale, wait_limit_cycles(), err);
+    if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+    kc<<<BH, kVCThreads, kVCAlloc, stream>>>(mrec, egl, out, s0, s_final, H, L, nch, wait_limit_cycles(), err);
+    return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+}  // namespace
+
+size_t tc_vg_workspace_bytes(int B, int H, int L) {
+    const long long nch = (static_cast<long long>(L) + kC - 1) / kC;
+    return static_cast<size_t>(B) * H * nch * (kRecBytes + kD * sizeof(float));
+}
+
+gdn_status_t launch_tc_vg(bool delta, const void *q, const void *k, const void *v, const float *beta, const float *g,
+                          void *o, const float *s0, float *s_final, int B, int H, int L, float scale, FwdOpts oo,
+                          cudaStream_t stream, bool *fallback) {
+    *fallback = false;
+    const int BH = B * H;
+    const int nch = (L + kC - 1) / kC;
+    const long long nrec = static_cast<long long>(BH) * nch;
+    if (nrec * kRecRows > 2147483647LL) {   // TMA row coordinates are int32
+        *fallback = true;
+        return GDN_ERR_UNSUPPORTED;
+    }
+    if (reinterpret_cast<uintptr_t>(g) % 8 != 0) {   // the prep kernel reads g two floats at a time
+        *fallback = true;
+        return GDN_ERR_UNSUPPORTED;
+    }
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GDN_ERR_CUDA;
+    cudaMemPool_t pool = record_pool(dev);
+    void *ws = nullptr;
+    if (!pool || cudaMallocFromPoolAsync(&ws, tc_vg_workspace_bytes(B, H, L), pool, stream) != cudaSuccess) {
+        cudaGetLastError();
+        *fallback = true;   // the caller takes the kernel that needs no workspace
+        return GDN_ERR_CUDA;
+    }
+    uint8_t *recs = static_cast<uint8_t *>(ws);
+    float *egl = reinterpret_cast<float *>(recs + static_cast<size_t>(nrec) * kRecBytes);
+    CUtensorMap mv, mrec;
+    gdn_status_t st = GDN_ERR_CUDA;
+    if (make_qkv_map(&mv, v, L, BH) && make_rec_map(&mrec, recs, static_cast<unsigned long long>(nrec) * kRecRows)) {
+        const OutArgs out = make_out_args(o, v, oo);
+        const bool opts = oo.bf16 || oo.dskip != nullptr || oo.xnorm != kXNormNone;
+        if (delta)
+            st = opts ? launch_vg_t<true, true>(mv, mrec, q, k, beta, g, recs, egl, out, s0, s_final, BH, H, L, nch, scale, stream)
+                      : launch_vg_t<true, false>(mv, mrec, q, k, beta, g, recs, egl, out, s0, s_final, BH, H, L, nch, scale, stream);
+        else
+            st = opts ? launch_vg_t<false, true>(mv, mrec, q, k, beta, g, recs, egl, out, s0, s_final, BH, H, L, nch, scale, stream)
+                      : launch_vg_t<false, false>(mv, mrec, q, k, beta, g, recs, egl, out, s0, s_final, BH, H, L, nch, scale, stream);
+    }
+    // stream-ordered: the records are released once both kernels have run
+    if (cudaFreeAsync(ws, stream) != cudaSuccess && st == GDN_OK) st = GDN_ERR_CUDA;
+    return st;
+}
+
+}  // namespace gdn

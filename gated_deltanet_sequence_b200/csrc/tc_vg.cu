@@ -23,7 +23,7 @@
 //                    Q'^T = (scale Q o exp(G))^T, -W^T, Kd^T = (K o exp(GL - G))^T, U^T and P
 //                    (fp16, 128-byte rows), plus exp(GL) (fp32).
 //   vg_chain_kernel  one CTA per (sequence, head): the fp32 state lives in tensor memory; per
-//                    chunk the record arrives by TMA and the chain takes three products,
+//                    chunk the record arrives by bulk copies and the chain takes three products,
 //                    [O^T | Ut^T] += S^T [Q'^T | -W^T] (Ut^T preloaded with U^T),
 //                    S <- exp(GL) o S + Kd^T Ut and O^T += Ut^T P^T.
 //
@@ -44,20 +44,15 @@ namespace {
 using namespace ptx;
 using namespace tcgdn;
 
-__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
-        : "memory");
-}
 __device__ __forceinline__ void st_shared_b32(uint32_t addr, uint32_t a) {
     asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(a) : "memory");
 }
 __device__ __forceinline__ float h_lo(uint32_t w) { return __low2float(*reinterpret_cast<const __half2 *>(&w)); }
 __device__ __forceinline__ float h_hi(uint32_t w) { return __high2float(*reinterpret_cast<const __half2 *>(&w)); }
 
-// ---- the per-chunk record (fp16, rows of 64 values = 128 bytes)
+// ---- the per-chunk record: fp16 tiles of 128-byte rows, stored as the image of a shared-memory
+//      tile in the 128-byte swizzled layout (16-byte chunk c of row R at chunk c ^ (R mod 8)),
+//      so that a plain bulk copy into a 1024-aligned buffer yields the UMMA operand layout
 constexpr int kRQ = 0;        // Q'^T: row j holds scale q_r[j] exp(G_r[j]), r = 0..63
 constexpr int kRW = 128;      // -W^T: row j holds -W[r][j]
 constexpr int kRKD = 256;     // Kd^T: row j holds k_r[j] exp(GL[j] - G_r[j])
@@ -65,27 +60,41 @@ constexpr int kRU = 384;      // U^T: row v holds U[r][v]
 constexpr int kRP = 512;      // P: row r holds P[r][s], s = 0..63
 constexpr int kRecRows = 576;
 constexpr uint32_t kRecBytes = kRecRows * 128u;   // 73728 (a multiple of 1024)
-constexpr int kBoxRows = 192;                     // TMA box: 192 rows x 64 values, three per record
+constexpr uint32_t kRecPiece = kRecBytes / 3;     // one record arrives as three bulk copies
 constexpr float kSpanFast = 12.f;                 // coordinate's range of G within a chunk, factored Gram
 constexpr int kSlowCap = 32;                      // at most this many exact coordinates next to the UMMA Gram
 
+__device__ __forceinline__ void bulk_s2g(void *gdst, uint32_t ssrc, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(ssrc), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_g2s(uint32_t sdst, const void *gsrc, uint32_t bytes, uint64_t *bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(sdst),
+                 "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
 // ================================================================== prep kernel
 constexpr int kVPThreads = 256;
-// shared memory (byte offsets from a 1024-aligned base)
-constexpr uint32_t VP_KA = 0;          // per key half h at h * 16384: [K o e rows 0-63 | Q o e rows 0-63]
-constexpr uint32_t VP_KB = 32768;      // K o (1/e), per key half at h * 8192
-constexpr uint32_t VP_AT = 49152;      // A^T fp32 64 x 64; before it the gate sums, then exact-coordinate data
-constexpr uint32_t VP_TF = 0;          // T fp32 64 x 68 (once the Gram operands are dead)
+// shared memory (byte offsets from a 1024-aligned base); regions and their successive uses
+constexpr uint32_t X0 = 0;        // per key half h at h * 16384: [K o e^(G-c) rows | Q o e^(G-c) rows];
+                                  // the K rows stay (A operand of W^T); the Q rows then hold V (TMA)
+constexpr uint32_t X1 = 32768;    // K o e^(c-G), per key half at h * 8192; then T diag(beta) (8 KB);
+                                  // then -W^T (16 KB)
+constexpr uint32_t X2 = 49152;    // gate sums, exact-coordinate data (up to 32), A^T fp32; then U^T
+constexpr uint32_t X3 = 65536;    // Q'^T and Kd^T (32 KB); then T fp32 (pitch 68), the solve's block
+                                  // scratch and P (8 KB)
+constexpr uint32_t XS = X1;       // every coordinate exact: G fp32 32 KB, k and q bf16 16 KB each (X1-X3)
+constexpr uint32_t VP_TF = X3, VP_RS = X3 + 17408, VP_P = X3 + 22528;
 constexpr int kTP = 68;
-constexpr uint32_t VP_RS = 17408;      // 4 x 16 x 16 fp32 block scratch of the solve
-constexpr uint32_t VP_KG = 65536;      // K o exp(G), per key half at h * 8192 (rows r; MN-major A of W^T)
-constexpr uint32_t VP_V = 81920;       // V, per value half at h * 8192 (TMA, bf16 -> fp16 in place)
-constexpr uint32_t VP_T2 = 98304;      // T diag(beta) fp16, K-major 64 x 64
-constexpr uint32_t VP_VEC = 106496;    // beta[64] | slot u8[128] | count | bars | tmem | abort
+constexpr uint32_t VP_VEC = 98304;   // beta[64] | c[128] | slot u8[128] | count | bars | tmem | abort
 constexpr uint32_t kVPSmem = VP_VEC + 1024;
 constexpr uint32_t kVPAlloc = kVPSmem + 1024;
 static_assert(kVPAlloc * 2 + 2048 <= 233472, "two prep CTAs per SM");
-constexpr uint32_t V_BETA = 0, V_SLOT = 256, V_NSLOW = 384, V_BARS = 448, V_TMEM = 480, V_ABORT = 484;
+static_assert(VP_P + 8192 <= X3 + 32768, "P after T and the block scratch");
+constexpr uint32_t V_BETA = 0, V_C = 256, V_SLOT = 768, V_NSLOW = 896, V_BARS = 928, V_TMEM = 960, V_ABORT = 964;
 // tensor memory (256 columns)
 constexpr uint32_t TMV_G = 0, TMV_W = 64, TMV_U = 128;
 constexpr uint32_t ID_G16 = idesc_f16(128, 64, false, false);   // Gram: both K-major, fp16
@@ -107,6 +116,7 @@ vg_prep_kernel(const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__
     int *abort_flag = reinterpret_cast<int *>(vec + V_ABORT);
     const Ctl ctl{bars, abort_flag, err_word, wait_limit};
     float *betav = reinterpret_cast<float *>(vec + V_BETA);
+    float *cv = reinterpret_cast<float *>(vec + V_C);
     uint8_t *slot = vec + V_SLOT;
     int *nslow_p = reinterpret_cast<int *>(vec + V_NSLOW);
 
@@ -122,14 +132,9 @@ vg_prep_kernel(const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__
         *abort_flag = 0;
         *nslow_p = 0;
         fence_mbar_init();
-        // V of this chunk (two value halves; rows past L read as zeros)
-        mbar_arrive_expect_tx(&bars[VB_V], 16384);
-        tma_load_3d(smem + VP_V, &tm_v, &bars[VB_V], 0, c * kC, bh);
-        tma_load_3d(smem + VP_V + 8192, &tm_v, &bars[VB_V], 64, c * kC, bh);
+        prefetch_tmap(&tm_v);
     }
     if (tid < kC) betav[tid] = (DELTA && tid < nvalid) ? beta[row0 + tid] : 0.f;
-    for (int i = tid; i < 8192 / 16; i += kVPThreads)      // T2: upper blocks stay zero
-        *reinterpret_cast<uint4 *>(smem + VP_T2 + i * 16) = make_uint4(0u, 0u, 0u, 0u);
     if (warp == 0) {
         tmem_alloc(tmem_slot, 256);
         tmem_relinquish();
@@ -161,7 +166,7 @@ vg_prep_kernel(const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__
         G0[i] += G0[i - 1];
         G1[i] += G1[i - 1];
     }
-    float *tot = reinterpret_cast<float *>(smem + VP_AT);   // [4][128] quarter sums, then min, max
+    float *tot = reinterpret_cast<float *>(smem + X2);   // [4][128] quarter sums, then min, max
     tot[h * 128 + j0] = G0[15];
     tot[h * 128 + j0 + 1] = G1[15];
     tc_fence_before();
@@ -204,31 +209,31 @@ vg_prep_kernel(const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__
     }
     const bool f0 = hi0 - lo0 <= kSpanFast, f1 = hi1 - lo1 <= kSpanFast;   // false for NaN ranges
     if (h == 0) {
-        if (!f0) {
-            const int f = atomicAdd(nslow_p, 1);
-            slot[j0] = static_cast<uint8_t>(f);
-        }
-        if (!f1) {
-            const int f = atomicAdd(nslow_p, 1);
-            slot[j0 + 1] = static_cast<uint8_t>(f);
-        }
+        if (!f0) slot[j0] = static_cast<uint8_t>(atomicAdd(nslow_p, 1));
+        if (!f1) slot[j0 + 1] = static_cast<uint8_t>(atomicAdd(nslow_p, 1));
         egl[static_cast<size_t>(rec_id) * kD + j0] = __expf(gl0);
         egl[static_cast<size_t>(rec_id) * kD + j0 + 1] = __expf(gl1);
     }
-    __syncthreads();   // gate sums read; the slow list is complete
+    __syncthreads();   // gate sums read; the exact-coordinate slots are assigned
     const int nslow = *nslow_p;
     const bool allslow = nslow > kSlowCap;
     const bool fa0 = f0 && !allslow, fa1 = f1 && !allslow;
-    const float c0 = 0.5f * (lo0 + hi0), c1 = 0.5f * (lo1 + hi1);
+    // reference c of the factors: the midpoint of the range for factored coordinates, else 0
+    const float c0 = fa0 ? 0.5f * (lo0 + hi0) : 0.f, c1 = fa1 ? 0.5f * (lo1 + hi1) : 0.f;
+    if (h == 0) {
+        cv[j0] = c0;
+        cv[j0 + 1] = c1;
+    }
     const float ec0 = fa0 ? __expf(c0) : 0.f, ec1 = fa1 ? __expf(c1) : 0.f;
     const float edc0 = fa0 ? __expf(gl0 - c0) : 0.f, edc1 = fa1 ? __expf(gl1 - c1) : 0.f;
-    uint32_t qT0[8], qT1[8], dT0[8], dT1[8];   // fp16 pairs along r for the transposed record rows
+    uint32_t qT0[8], qT1[8], dT0[8], dT1[8];   // fp16 pairs along r for the transposed rows
     float pq0 = 0.f, pq1 = 0.f, pd0 = 0.f, pd1 = 0.f;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
         const int r = r0 + i;
         const float k0 = bf_lo(kw[i]), k1 = bf_hi(kw[i]), q0 = bf_lo(qw[i]), q1 = bf_hi(qw[i]);
-        float ka0 = 0.f, qa0 = 0.f, kb0 = 0.f, eg0, ed0, ka1 = 0.f, qa1 = 0.f, kb1 = 0.f, eg1, ed1;
+        // K o e^(G-c) (Gram A rows, and W's operand), Q o e^(G-c), K o e^(c-G) (Gram B rows)
+        float ka0, qa0 = 0.f, kb0 = 0.f, eg0, ed0, ka1, qa1 = 0.f, kb1 = 0.f, eg1, ed1;
         if (fa0) {
             const float e1 = __expf(G0[i] - c0), e2 = __expf(c0 - G0[i]);
             ka0 = k0 * e1;
@@ -239,6 +244,7 @@ vg_prep_kernel(const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__
         } else {
             eg0 = __expf(G0[i]);
             ed0 = __expf(gl0 - G0[i]);
+            ka0 = k0 * eg0;
         }
         if (fa1) {
             const float e1 = __expf(G1[i] - c1), e2 = __expf(c1 - G1[i]);
@@ -250,14 +256,14 @@ vg_prep_kernel(const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__
         } else {
             eg1 = __expf(G1[i]);
             ed1 = __expf(gl1 - G1[i]);
+            ka1 = k1 * eg1;
         }
         const uint32_t sw = sw128(r, jc >> 3) + (jc & 7) * 2;
+        st_shared_b32(sb + X0 + kh * 16384 + sw, pack_h2(ka0, ka1));
         if (!allslow) {
-            st_shared_b32(sb + VP_KA + kh * 16384 + sw, pack_h2(ka0, ka1));
-            st_shared_b32(sb + VP_KA + kh * 16384 + 8192 + sw, pack_h2(qa0, qa1));
-            st_shared_b32(sb + VP_KB + kh * 8192 + sw, pack_h2(kb0, kb1));
+            st_shared_b32(sb + X0 + kh * 16384 + 8192 + sw, pack_h2(qa0, qa1));
+            st_shared_b32(sb + X1 + kh * 8192 + sw, pack_h2(kb0, kb1));
         }
-        st_shared_b32(sb + VP_KG + kh * 8192 + sw, pack_h2(k0 * eg0, k1 * eg1));
         const float qp0 = scale * q0 * eg0, qp1 = scale * q1 * eg1, kd0 = k0 * ed0, kd1 = k1 * ed1;
         if (i & 1) {
             qT0[i >> 1] = pack_h2(pq0, qp0);
@@ -271,74 +277,94 @@ vg_prep_kernel(const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__
             pd1 = kd1;
         }
         if ((i & 7) == 7) {
-            // rows j0, j0+1 of Q'^T and Kd^T: the 8 values r = r0 + i - 7 .. r0 + i
-            const int b = (i >> 3) * 4, off = 32 * h + 16 * (i >> 3);
-            uint8_t *rq = rec + static_cast<size_t>(kRQ + j0) * 128 + off;
-            uint8_t *rd = rec + static_cast<size_t>(kRKD + j0) * 128 + off;
-            *reinterpret_cast<uint4 *>(rq) = make_uint4(qT0[b], qT0[b + 1], qT0[b + 2], qT0[b + 3]);
-            *reinterpret_cast<uint4 *>(rq + 128) = make_uint4(qT1[b], qT1[b + 1], qT1[b + 2], qT1[b + 3]);
-            *reinterpret_cast<uint4 *>(rd) = make_uint4(dT0[b], dT0[b + 1], dT0[b + 2], dT0[b + 3]);
-            *reinterpret_cast<uint4 *>(rd + 128) = make_uint4(dT1[b], dT1[b + 1], dT1[b + 2], dT1[b + 3]);
+            // rows j0, j0+1 of Q'^T and Kd^T: the 8 values r = r0 + i - 7 .. r0 + i (one chunk)
+            const int b = (i >> 3) * 4;
+            const uint32_t ch = 2 * h + (i >> 3);
+            st_shared_v4(sb + X3 + sw128(kRQ + j0, ch), qT0[b], qT0[b + 1], qT0[b + 2], qT0[b + 3]);
+            st_shared_v4(sb + X3 + sw128(kRQ + j0 + 1, ch), qT1[b], qT1[b + 1], qT1[b + 2], qT1[b + 3]);
+            st_shared_v4(sb + X3 + 16384 + sw128(j0, ch), dT0[b], dT0[b + 1], dT0[b + 2], dT0[b + 3]);
+            st_shared_v4(sb + X3 + 16384 + sw128(j0 + 1, ch), dT1[b], dT1[b + 1], dT1[b + 2], dT1[b + 3]);
         }
     }
-    // exact coordinates: G (fp32), k and q (bf16) by coordinate slot, rows contiguous
-    const int NF = allslow ? kD : kSlowCap;
-    const uint32_t sbase = allslow ? 0u : VP_AT;
+    // exact coordinates next to the UMMA Gram: G (fp32), k and q (bf16) by slot, rows contiguous
+    auto put_exact = [&](uint32_t base, int NF) {
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-        const bool ex = allslow || !(e ? f1 : f0);
-        if (!ex) continue;
-        const int j = j0 + e;
-        const int f = allslow ? j : slot[j];
-        const float *Gv = e ? G1 : G0;
-        float *sg = reinterpret_cast<float *>(smem + sbase) + f * 64 + r0;
+        for (int e = 0; e < 2; ++e) {
+            if (!allslow && (e ? f1 : f0)) continue;
+            const int j = j0 + e;
+            const int f = allslow ? j : slot[j];
+            const float *Gv = e ? G1 : G0;
+            float *sg = reinterpret_cast<float *>(smem + base) + f * 64 + r0;
 #pragma unroll
-        for (int i = 0; i < 16; i += 4)
-            *reinterpret_cast<float4 *>(sg + i) = make_float4(Gv[i], Gv[i + 1], Gv[i + 2], Gv[i + 3]);
-        uint32_t kk[8], qq[8];
+            for (int i = 0; i < 16; i += 4)
+                *reinterpret_cast<float4 *>(sg + i) = make_float4(Gv[i], Gv[i + 1], Gv[i + 2], Gv[i + 3]);
+            uint32_t kk[8], qq[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const uint32_t a = kw[2 * i], b = kw[2 * i + 1], x = qw[2 * i], y = qw[2 * i + 1];
-            kk[i] = e ? ((a >> 16) | (b & 0xFFFF0000u)) : ((a & 0xFFFFu) | (b << 16));
-            qq[i] = e ? ((x >> 16) | (y & 0xFFFF0000u)) : ((x & 0xFFFFu) | (y << 16));
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t a = kw[2 * i], b = kw[2 * i + 1], x = qw[2 * i], y = qw[2 * i + 1];
+                kk[i] = e ? ((a >> 16) | (b & 0xFFFF0000u)) : ((a & 0xFFFFu) | (b << 16));
+                qq[i] = e ? ((x >> 16) | (y & 0xFFFF0000u)) : ((x & 0xFFFFu) | (y << 16));
+            }
+            uint8_t *sk = smem + base + NF * 256 + f * 128 + r0 * 2;
+            uint8_t *sq = smem + base + NF * 384 + f * 128 + r0 * 2;
+            *reinterpret_cast<uint4 *>(sk) = make_uint4(kk[0], kk[1], kk[2], kk[3]);
+            *reinterpret_cast<uint4 *>(sk + 16) = make_uint4(kk[4], kk[5], kk[6], kk[7]);
+            *reinterpret_cast<uint4 *>(sq) = make_uint4(qq[0], qq[1], qq[2], qq[3]);
+            *reinterpret_cast<uint4 *>(sq + 16) = make_uint4(qq[4], qq[5], qq[6], qq[7]);
         }
-        uint8_t *sk = smem + sbase + NF * 256 + f * 128 + r0 * 2;
-        uint8_t *sq = smem + sbase + NF * 384 + f * 128 + r0 * 2;
-        *reinterpret_cast<uint4 *>(sk) = make_uint4(kk[0], kk[1], kk[2], kk[3]);
-        *reinterpret_cast<uint4 *>(sk + 16) = make_uint4(kk[4], kk[5], kk[6], kk[7]);
-        *reinterpret_cast<uint4 *>(sq) = make_uint4(qq[0], qq[1], qq[2], qq[3]);
-        *reinterpret_cast<uint4 *>(sq + 16) = make_uint4(qq[4], qq[5], qq[6], qq[7]);
-    }
+    };
+    if (!allslow && nslow > 0) put_exact(X2, kSlowCap);
     fence_proxy_async();
     __syncthreads();
-
-    // ---- decay-weighted Gram [K o e; Q o e] (K o 1/e)^T: rows 0-63 -> A, 64-127 -> P
-    bool ok = true;
-    if (!allslow) {
-        if (tid == 0) {
+    // Q'^T and Kd^T go out; the Gram starts; V is fetched into the Q rows once the Gram has read them
+    bool ok = true, issued_v = false;   // issued_v: thread 0's own record of the V copy
+    if (tid == 0) {
+        bulk_s2g(rec + kRQ * 128, sb + X3, 16384);
+        bulk_s2g(rec + kRKD * 128, sb + X3 + 16384, 16384);
+        bulk_commit();
+        if (!allslow) {
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-                mma_f16(tmem + TMV_G, sdesc_sw128(sb + VP_KA + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                        sdesc_sw128(sb + VP_KB + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), ID_G16, kk > 0);
+                mma_f16(tmem + TMV_G, sdesc_sw128(sb + X0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                        sdesc_sw128(sb + X1 + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), ID_G16, kk > 0);
             mma_commit(&bars[VB_G]);
+            ok = ctl.wait(VB_G, 0);
+        } else {
+            bulk_wait_read();   // X3 takes the exact-coordinate data next
         }
+        if (ok) {
+            mbar_arrive_expect_tx(&bars[VB_V], 16384);
+            tma_load_3d(smem + X0 + 8192, &tm_v, &bars[VB_V], 0, c * kC, bh);
+            tma_load_3d(smem + X0 + 24576, &tm_v, &bars[VB_V], 64, c * kC, bh);
+            issued_v = true;
+        }
+    }
+    if (allslow) {
+        __syncthreads();
+        put_exact(XS, kD);
+        __syncthreads();
+    } else {
         ok = ctl.wait(VB_G, 0);
         tc_fence_after();
     }
+    const bool v_issued = !__syncthreads_or(!ok);   // thread 0 issued V iff every wait so far held
+    ok = v_issued;
     const int sub = warp & 3, hh = warp >> 2, R = sub * 32 + lane;
     const int r = R & 63;
     const bool isP = R >= 64;
     const uint32_t trow = tmem + (static_cast<uint32_t>(sub * 32) << 16);
     float v[32];
-    if (!allslow && !__syncthreads_or(!ok)) {
+    if (!allslow && ok) {
         ld_cols<32>(trow + TMV_G + 32 * hh, v);
     } else {
 #pragma unroll
         for (int e = 0; e < 32; ++e) v[e] = 0.f;
     }
-    if (nslow > 0 && r >= 32 * hh && (DELTA || isP)) {
+    if (ok && nslow > 0 && r >= 32 * hh && (DELTA || isP)) {
         // exact terms of the coordinates left out of the factored Gram
+        const uint32_t sbase = allslow ? XS : X2;
+        const int NF = allslow ? kD : kSlowCap;
         const float *SG = reinterpret_cast<const float *>(smem + sbase);
         const __nv_bfloat16 *SK = reinterpret_cast<const __nv_bfloat16 *>(smem + sbase + NF * 256);
         const __nv_bfloat16 *SX = reinterpret_cast<const __nv_bfloat16 *>(smem + sbase + NF * (isP ? 384 : 256));
@@ -354,38 +380,46 @@ vg_prep_kernel(const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__
             }
         }
     }
+    if (tid == 0) bulk_wait_read();   // Q'^T / Kd^T have left X3 (P and T go there)
     tc_fence_before();
-    ok = !__syncthreads_or(!ok);   // Gram and exact-coordinate data read: A^T may overwrite them
+    __syncthreads();   // Gram and exact-coordinate data read: A^T and P may overwrite them
     if (!isP) {
         if (DELTA) {
-            float *At = reinterpret_cast<float *>(smem + VP_AT);   // At[s * 64 + r] = A[r][s]
+            float *At = reinterpret_cast<float *>(smem + X2);   // At[s * 64 + r] = A[r][s]
             const float br = betav[r];
 #pragma unroll
             for (int e = 0; e < 32; ++e) At[(32 * hh + e) * 64 + r] = (32 * hh + e < r) ? br * v[e] : 0.f;
         }
     } else {
-        uint8_t *prow = rec + static_cast<size_t>(kRP + r) * 128 + 64 * hh;
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
             float pv[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) pv[e] = (32 * hh + 8 * ch + e <= r) ? scale * v[8 * ch + e] : 0.f;
-            *reinterpret_cast<uint4 *>(prow + 16 * ch) =
-                make_uint4(pack_h2(pv[0], pv[1]), pack_h2(pv[2], pv[3]), pack_h2(pv[4], pv[5]), pack_h2(pv[6], pv[7]));
+            st_shared_v4(sb + VP_P + sw128(r, 4 * hh + ch), pack_h2(pv[0], pv[1]), pack_h2(pv[2], pv[3]),
+                         pack_h2(pv[4], pv[5]), pack_h2(pv[6], pv[7]));
         }
     }
-    __syncthreads();   // A^T complete
+    fence_proxy_async();
+    __syncthreads();   // A^T and P complete
+    if (tid == 0) {
+        bulk_s2g(rec + kRP * 128, sb + VP_P, 8192);
+        bulk_commit();
+    }
 
     // ---- UT solve (warps 0-3) while warps 4-7 convert V to fp16
     if (warp < 4) {
-        const float *At = reinterpret_cast<const float *>(smem + VP_AT);
+        const float *At = reinterpret_cast<const float *>(smem + X2);
         float *Tf = reinterpret_cast<float *>(smem + VP_TF);    // Tf[r * kTP + c] = T[r][c]
+        for (int i = tid; i < 8192 / 16; i += 128)              // T diag(beta): upper blocks stay zero
+            *reinterpret_cast<uint4 *>(smem + X1 + i * 16) = make_uint4(0u, 0u, 0u, 0u);
         if (!DELTA) {
             // linear attention: T = I, so T diag(beta) is the identity (U = V)
+            asm volatile("bar.sync 3, 128;" ::: "memory");
             if (tid < 64)
-                *reinterpret_cast<__half *>(smem + VP_T2 + sw128(tid, tid >> 3) + (tid & 7) * 2) = __float2half_rn(1.f);
+                *reinterpret_cast<__half *>(smem + X1 + sw128(tid, tid >> 3) + (tid & 7) * 2) = __float2half_rn(1.f);
         } else {
-            // one 16 x 16 block (bi, bj) of Tf -> T2 = T diag(beta) (K-major rows r)
+            // one 16 x 16 block (bi, bj) of Tf -> T diag(beta) (K-major rows r)
             auto emit = [&](int bi2, int bj2) {
                 __syncwarp();
                 const int rr = 16 * bi2 + (lane >> 1), cc0 = 16 * bj2 + 8 * (lane & 1);
@@ -393,12 +427,12 @@ vg_prep_kernel(const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__
                 const float4 b1 = *reinterpret_cast<const float4 *>(betav + cc0 + 4);
                 const float4 t0 = *reinterpret_cast<const float4 *>(Tf + rr * kTP + cc0);
                 const float4 t1 = *reinterpret_cast<const float4 *>(Tf + rr * kTP + cc0 + 4);
-                st_shared_v4(sb + VP_T2 + sw128(rr, cc0 >> 3), pack_h2(t0.x * b0.x, t0.y * b0.y),
+                st_shared_v4(sb + X1 + sw128(rr, cc0 >> 3), pack_h2(t0.x * b0.x, t0.y * b0.y),
                              pack_h2(t0.z * b0.z, t0.w * b0.w), pack_h2(t1.x * b1.x, t1.y * b1.y),
                              pack_h2(t1.z * b1.z, t1.w * b1.w));
             };
             const int bi = warp, cl = lane & 15;
-            {
+            if (ok) {
                 // diagonal block D_i = (I + A_ii)^-1 by right-looking substitution (lane = column)
                 float acc[16];
 #pragma unroll
@@ -423,10 +457,10 @@ vg_prep_kernel(const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__
                 }
             }
             asm volatile("bar.sync 3, 128;" ::: "memory");
-            emit(bi, bi);
+            if (ok) emit(bi, bi);
             float *Rw = reinterpret_cast<float *>(smem + VP_RS);
             // T_10 = -D_1 (A_10 D_0), T_32 = -D_3 (A_32 D_2)
-            if (bi < 2) {
+            if (ok && bi < 2) {
                 const int i = 2 * bi + 1, j = 2 * bi;
                 float *Rb = Rw + bi * 256;
                 float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
@@ -444,7 +478,7 @@ vg_prep_kernel(const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__
             asm volatile("bar.sync 3, 128;" ::: "memory");
             // X_ij = A_{i,0..1} T_{0..1,j} for (i, j) = (2 + w / 2, w % 2)
             const int ii = 2 + (bi >> 1), jj = bi & 1;
-            {
+            if (ok) {
                 float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
                 if (jj == 0)
                     block_mm<4>(acc2, [&](int rr, int kx) { return At[kx * 64 + 16 * ii + rr]; },
@@ -457,71 +491,80 @@ vg_prep_kernel(const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__
             }
             asm volatile("bar.sync 3, 128;" ::: "memory");
             // T_2j = -D_2 X_2j,  T_3j = -(T_32 X_2j + D_3 X_3j)
-            {
-                const float *X2 = Rw + jj * 256, *X3 = Rw + (2 + jj) * 256;
+            if (ok) {
+                const float *X2p = Rw + jj * 256, *X3p = Rw + (2 + jj) * 256;
                 float acc3[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
                 if (ii == 2)
                     block_mm<2>(acc3, [&](int rr, int kx) { return Tf[(32 + rr) * kTP + 32 + kx]; },
-                                [&](int kx, int n) { return X2[kx * 16 + n]; }, lane);
+                                [&](int kx, int n) { return X2p[kx * 16 + n]; }, lane);
                 else
                     block_mm<4>(acc3, [&](int rr, int kx) { return Tf[(48 + rr) * kTP + 32 + kx]; },
-                                [&](int kx, int n) { return kx < 16 ? X2[kx * 16 + n] : X3[(kx - 16) * 16 + n]; },
+                                [&](int kx, int n) { return kx < 16 ? X2p[kx * 16 + n] : X3p[(kx - 16) * 16 + n]; },
                                 lane);
                 block_store(acc3, [&](int rr, int n, float x) { Tf[(16 * ii + rr) * kTP + 16 * jj + n] = x; }, lane,
                             -1.f);
                 emit(ii, jj);
             }
         }
-    } else {
+    } else if (ok) {
         const int t4 = tid - 128;
         bool vok = true;
         if (t4 == 0) vok = ctl.wait(VB_V, 0);
-        vok = __shfl_sync(0xffffffffu, vok ? 1 : 0, 0) != 0;   // warp 4 lane 0 polled
         asm volatile("bar.sync 4, 128;" ::: "memory");
-        if (warp != 4) vok = !ctl.aborted();
-        if (vok) convert_tile_bf16_to_f16(smem + VP_V, 16384, t4, 128);
-        ok = ok && vok;
+        vok = !ctl.aborted();   // the wait that gave up set the abort flag
+        if (vok) {
+            convert_tile_bf16_to_f16(smem + X0 + 8192, 8192, t4, 128);
+            convert_tile_bf16_to_f16(smem + X0 + 24576, 8192, t4, 128);
+        }
+        ok = vok;
     }
     fence_proxy_async();
     ok = !__syncthreads_or(!ok);
 
-    // ---- W^T = (K o exp(G))^T (T diag(beta))^T and U^T = V^T (T diag(beta))^T
+    // ---- W^T = diag(e^c) (K o e^(G-c))^T (T diag(beta))^T and U^T = V^T (T diag(beta))^T
     const bool wu_issued = ok;
     if (ok && tid == 0) {
         tc_fence_after();
         if (DELTA) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                mma_f16(tmem + TMV_W, sdesc_sw128(sb + VP_KG + kk * 2048, 8192, 1024),
-                        sdesc_sw128(sb + VP_T2 + kk * 32, 16, 1024), ID_WU, kk > 0);
+                mma_f16(tmem + TMV_W, sdesc_sw128(sb + X0 + kk * 2048, 16384, 1024),
+                        sdesc_sw128(sb + X1 + kk * 32, 16, 1024), ID_WU, kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-            mma_f16(tmem + TMV_U, sdesc_sw128(sb + VP_V + kk * 2048, 8192, 1024),
-                    sdesc_sw128(sb + VP_T2 + kk * 32, 16, 1024), ID_WU, kk > 0);
+            mma_f16(tmem + TMV_U, sdesc_sw128(sb + X0 + 8192 + kk * 2048, 16384, 1024),
+                    sdesc_sw128(sb + X1 + kk * 32, 16, 1024), ID_WU, kk > 0);
         mma_commit(&bars[VB_WU]);
     }
     if (ok) ok = ctl.wait(VB_WU, 0);
     tc_fence_after();
     if (!__syncthreads_or(!ok)) {
-        // warps 0-3: -W^T rows j; warps 4-7: U^T rows v (one TMEM lane each)
+        // warps 0-3: -W^T rows j (times e^(c_j)) into X1; warps 4-7: U^T rows v into X2
         if (warp >= 4 || DELTA) {
-            const int row = (warp >= 4 ? kRU : kRW) + R;
-            const float sg = warp >= 4 ? 1.f : -1.f;
-            uint8_t *dst = rec + static_cast<size_t>(row) * 128;
+            const float sg = warp >= 4 ? 1.f : -__expf(cv[R]);
+            const uint32_t dst = sb + (warp >= 4 ? X2 : X1);
             float x[64];
             ld_cols<64>(trow + (warp >= 4 ? TMV_U : TMV_W), x);
 #pragma unroll
             for (int ch = 0; ch < 8; ++ch)
-                *reinterpret_cast<uint4 *>(dst + 16 * ch) =
-                    make_uint4(pack_h2(sg * x[8 * ch], sg * x[8 * ch + 1]), pack_h2(sg * x[8 * ch + 2], sg * x[8 * ch + 3]),
-                               pack_h2(sg * x[8 * ch + 4], sg * x[8 * ch + 5]),
-                               pack_h2(sg * x[8 * ch + 6], sg * x[8 * ch + 7]));
+                st_shared_v4(dst + sw128(R, ch), pack_h2(sg * x[8 * ch], sg * x[8 * ch + 1]),
+                             pack_h2(sg * x[8 * ch + 2], sg * x[8 * ch + 3]), pack_h2(sg * x[8 * ch + 4], sg * x[8 * ch + 5]),
+                             pack_h2(sg * x[8 * ch + 6], sg * x[8 * ch + 7]));
+        }
+        fence_proxy_async();
+        __syncthreads();
+        if (tid == 0) {
+            if (DELTA) bulk_s2g(rec + kRW * 128, sb + X1, 16384);
+            bulk_s2g(rec + kRU * 128, sb + X2, 16384);
+            bulk_commit();
         }
     }
-    // never leave a copy or a UMMA in flight past the end of the CTA
+    // never leave a copy or a UMMA in flight past the end of the CTA (the shared memory the
+    // bulk stores read stays until they have read it)
     if (tid == 0) {
-        ctl.drain(VB_V, 0);
+        bulk_wait_read();
+        if (issued_v) ctl.drain(VB_V, 0);
         if (!allslow) ctl.drain(VB_G, 0);
         if (wu_issued) ctl.drain(VB_WU, 0);
     }
@@ -554,7 +597,7 @@ enum : int { CB_FULL = 0, CB_CDONE = 2, CB_SRDY = 4, CB_ADONE = 5, CB_URDY = 6, 
 
 template <bool DELTA, bool OPTS>
 __global__ void __launch_bounds__(kVCThreads, 1)
-vg_chain_kernel(const __grid_constant__ CUtensorMap tm_rec, const float *__restrict__ egl, const OutArgs out,
+vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl, const OutArgs out,
                 const float *__restrict__ s0, float *__restrict__ s_final, int H, int L, int nch,
                 long long wait_limit, unsigned *__restrict__ err_word) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -574,7 +617,6 @@ vg_chain_kernel(const __grid_constant__ CUtensorMap tm_rec, const float *__restr
         for (int b = 0; b < kVCBars; ++b) mbar_init(&bars[b], 1);
         abort_flag[0] = 0;
         fence_mbar_init();
-        prefetch_tmap(&tm_rec);
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, 512);
@@ -594,10 +636,9 @@ vg_chain_kernel(const __grid_constant__ CUtensorMap tm_rec, const float *__restr
                 if (c >= 2 && !ctl.wait_lazy(CB_CDONE + s, ((c - 2) >> 1) & 1)) break;
                 uint64_t *fb = &bars[CB_FULL + s];
                 mbar_arrive_expect_tx(fb, kRecBytes);
-                const int row = static_cast<int>((rec0 + c) * kRecRows);
+                const uint8_t *src = recs + static_cast<size_t>(rec0 + c) * kRecBytes;
 #pragma unroll
-                for (int b = 0; b < kRecRows / kBoxRows; ++b)
-                    tma_load_2d(smem + s * kRecBytes + b * kBoxRows * 128, &tm_rec, fb, 0, row + b * kBoxRows);
+                for (int b = 0; b < 3; ++b) bulk_g2s(sb + s * kRecBytes + b * kRecPiece, src + b * kRecPiece, kRecPiece, fb);
                 last[s] = c;
             }
             for (int s = 0; s < 2; ++s)
@@ -772,25 +813,8 @@ vg_chain_kernel(const __grid_constant__ CUtensorMap tm_rec, const float *__restr
 }  // namespace
 
 // ---------------------------------------------------------------- host side
-using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-EncodeTiledFn encode_fn();
 
 namespace {
-
-// (rows, 64) fp16 record rows -> 2-D map, 64 x 192 boxes, 128-byte swizzle.
-bool make_rec_map(CUtensorMap *m, void *ptr, unsigned long long rows) {
-    EncodeTiledFn enc = encode_fn();
-    if (!enc) return false;
-    const cuuint64_t dims[2] = {64, static_cast<cuuint64_t>(rows)};
-    const cuuint64_t strides[1] = {128};
-    const cuuint32_t box[2] = {64, kBoxRows};
-    const cuuint32_t estr[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, ptr, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 // One stream-ordered memory pool per device for the per-chunk records; it keeps what it
 // has reserved (release threshold: never), so repeated calls of one size allocate once.
@@ -817,7 +841,7 @@ cudaMemPool_t record_pool(int dev) {
 }
 
 template <bool DELTA, bool OPTS>
-gdn_status_t launch_vg_t(const CUtensorMap &mv, const CUtensorMap &mrec, const void *q, const void *k,
+gdn_status_t launch_vg_t(const CUtensorMap &mv, const void *q, const void *k,
                          const float *beta, const float *g, uint8_t *recs, float *egl, const OutArgs &out,
                          const float *s0, float *s_final, int BH, int H, int L, int nch, float scale,
                          cudaStream_t stream) {
@@ -833,7 +857,7 @@ gdn_status_t launch_vg_t(const CUtensorMap &mv, const CUtensorMap &mrec, const v
         mv, static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k), beta, g, recs, egl, L, nch,
         scale, wait_limit_cycles(), err);
     if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
-    kc<<<BH, kVCThreads, kVCAlloc, stream>>>(mrec, egl, out, s0, s_final, H, L, nch, wait_limit_cycles(), err);
+    kc<<<BH, kVCThreads, kVCAlloc, stream>>>(recs, egl, out, s0, s_final, H, L, nch, wait_limit_cycles(), err);
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
@@ -851,7 +875,7 @@ gdn_status_t launch_tc_vg(bool delta, const void *q, const void *k, const void *
     const int BH = B * H;
     const int nch = (L + kC - 1) / kC;
     const long long nrec = static_cast<long long>(BH) * nch;
-    if (nrec * kRecRows > 2147483647LL) {   // TMA row coordinates are int32
+    if (nrec > 2147483647LL) {   // one prep CTA per chunk
         *fallback = true;
         return GDN_ERR_UNSUPPORTED;
     }
@@ -870,17 +894,17 @@ gdn_status_t launch_tc_vg(bool delta, const void *q, const void *k, const void *
     }
     uint8_t *recs = static_cast<uint8_t *>(ws);
     float *egl = reinterpret_cast<float *>(recs + static_cast<size_t>(nrec) * kRecBytes);
-    CUtensorMap mv, mrec;
+    CUtensorMap mv;
     gdn_status_t st = GDN_ERR_CUDA;
-    if (make_qkv_map(&mv, v, L, BH) && make_rec_map(&mrec, recs, static_cast<unsigned long long>(nrec) * kRecRows)) {
+    if (make_qkv_map(&mv, v, L, BH)) {
         const OutArgs out = make_out_args(o, v, oo);
         const bool opts = oo.bf16 || oo.dskip != nullptr || oo.xnorm != kXNormNone;
         if (delta)
-            st = opts ? launch_vg_t<true, true>(mv, mrec, q, k, beta, g, recs, egl, out, s0, s_final, BH, H, L, nch, scale, stream)
-                      : launch_vg_t<true, false>(mv, mrec, q, k, beta, g, recs, egl, out, s0, s_final, BH, H, L, nch, scale, stream);
+            st = opts ? launch_vg_t<true, true>(mv, q, k, beta, g, recs, egl, out, s0, s_final, BH, H, L, nch, scale, stream)
+                      : launch_vg_t<true, false>(mv, q, k, beta, g, recs, egl, out, s0, s_final, BH, H, L, nch, scale, stream);
         else
-            st = opts ? launch_vg_t<false, true>(mv, mrec, q, k, beta, g, recs, egl, out, s0, s_final, BH, H, L, nch, scale, stream)
-                      : launch_vg_t<false, false>(mv, mrec, q, k, beta, g, recs, egl, out, s0, s_final, BH, H, L, nch, scale, stream);
+            st = opts ? launch_vg_t<false, true>(mv, q, k, beta, g, recs, egl, out, s0, s_final, BH, H, L, nch, scale, stream)
+                      : launch_vg_t<false, false>(mv, q, k, beta, g, recs, egl, out, s0, s_final, BH, H, L, nch, scale, stream);
     }
     // stream-ordered: the records are released once both kernels have run
     if (cudaFreeAsync(ws, stream) != cudaSuccess && st == GDN_OK) st = GDN_ERR_CUDA;

@@ -348,23 +348,16 @@ def measure_rows(gdn, peaks, peak_src, args):
     fl = flops_per_head_token("gdn", w.dk, w.dv, w.chunk) * w.B * w.H * w.L
     rows["gdn_prefill_bf16_out_skip"] = _row(w, ms, nb, fl, peaks, peak_src, "hbm", w.B * w.L)
     del ob
-    # the same workload with vector-valued gates (one log-decay per token and key coordinate),
-    # which run on the fp32 CUDA-core chunk kernel
+    # the same workload with vector-valued gates (one log-decay per token and key coordinate): a
+    # per-chunk prep kernel on every SM and a per-head chain kernel, through a chunk-record
+    # workspace (the call's algorithmic bytes count g in fp32 per key coordinate)
     gv = W.make_gate_per_key((w.B, w.H), w.L, w.dk, seed=W.SEED_BASE + 7, device="cuda")
     o = torch.empty(w.B, w.H, w.L, w.dv, device="cuda")
     fn = lambda: gdn.gdn_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["beta"], gv, o=o, s_final=sf, chunk=w.chunk)
-    ms = timed(fn, max(3, args.steps // 6), 2)
+    ms = timed(fn, max(5, args.steps), 3)
     nb = prefill_bytes(w.B, w.H, w.L, w.dk, w.dv, 2, True, False, False, True) + w.B * w.H * w.L * w.dk * 4
     row = _row(w, ms, nb, fl, peaks, peak_src, "hbm", w.B * w.L)
-    row["path"] = "fp32 chunk kernel (CUDA cores)"
-    # fp32 CUDA-core arithmetic bounds this path: peak = SMs x 128 fp32 lanes x 2 FLOP x max SM clock
-    sms = torch.cuda.get_device_properties(0).multi_processor_count
-    peak_f32 = sms * 128 * 2 * FP32_CLOCK_GHZ / 1e3
-    tf32 = fl / (ms * 1e-3) / 1e12
-    row["roofline"] = {"bound": "alu", "achieved": round(tf32, 2), "peak": round(peak_f32, 1), "unit": "TFLOP/s",
-                       "frac": round(tf32 / peak_f32, 4), "traffic": None,
-                       "peak_source": f"derived: {sms} SMs x 128 fp32 lanes x 2 FLOP x {FP32_CLOCK_GHZ} GHz",
-                       "algorithmic_flop_per_launch": fl}
+    row["path"] = "tensor cores: vg_prep_kernel (one CTA per chunk) + vg_chain_kernel (one CTA per head)"
     rows["gdn_prefill_vector_gate"] = row
     del inp, o, sf, gv
     # backward pass (gradients of the prefill) on the headline shape: fp32 CUDA-core kernel whose
@@ -556,7 +549,7 @@ def run_profile(spec: str):
     spec: gdn[:B] (GDN bf16, B x 16 x 4096 x 128), la[:B] (plain LA, B x 16 x 4096 x 128),
     decode[:N] (N x 32 heads, 3 steps), gdn_long (1 x 32 x 65536), gdnh[:H[:L]] (1 x H x L,
     the cluster form when 3 H fits the SM count), gdnvec[:B[:L]] (vector-valued gates, B x 16 x L,
-    the fp32 chunk kernel)."""
+    bf16: the prep and chain kernels), gdnvec32[:B[:L]] (the same in fp32: the fp32 chunk kernel)."""
     from gated_deltanet_sequence_b200 import _lib as gdn
     kind, _, arg = spec.partition(":")
     torch.cuda.set_device(0)
@@ -582,11 +575,13 @@ def run_profile(spec: str):
         sf = torch.empty(1, H, 128, 128, device="cuda")
         for _ in range(2):
             gdn.gdn_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["g"], o=o, s0=inp["s0"], s_final=sf)
-    elif kind == "gdnvec":
-        # vector-valued gates (fp32 chunk kernel): B x 16 heads x L tokens, d = 128, bf16 inputs
+    elif kind in ("gdnvec", "gdnvec32"):
+        # vector-valued gates: B x 16 heads x L tokens, d = 128; bf16 inputs take the tensor-core
+        # prep and chain kernels, fp32 inputs the fp32 chunk kernel
         B, _, L = arg.partition(":")
         B, L = int(B or 1), int(L or 1024)
-        inp = W.make_prefill_inputs(B, 16, L, 128, 128, mode="gdn", in_dtype=torch.bfloat16,
+        inp = W.make_prefill_inputs(B, 16, L, 128, 128, mode="gdn",
+                                    in_dtype=torch.bfloat16 if kind == "gdnvec" else torch.float32,
                                     seed=W.SEED_BASE + 7, device="cuda")
         gv = W.make_gate_per_key((B, 16), L, 128, seed=W.SEED_BASE + 7, device="cuda")
         o = torch.empty(B, 16, L, 128, device="cuda")

@@ -145,8 +145,13 @@ gdn_status_t gdn_chunk_fwd_varlen(const void *q, const void *k, const void *v, c
  *             decays by exp(g_t[j]):  S_t = (I - beta_t k_t k_t^T) diag(exp(g_t)) S_{t-1}
  *             + beta_t k_t v_t^T (without beta: S_t = diag(exp(g_t)) S_{t-1} + k_t v_t^T),
  *             the per-coordinate form of the scalar gate (GLA-style gates, next to the
- *             scalar gate of page "混合注意力学习(1)", section "Gated DeltaNet"). These
- *             calls run on the fp32 chunk kernel. Any other value: GDN_ERR_INVALID_ARG.
+ *             scalar gate of page "混合注意力学习(1)", section "Gated DeltaNet"). Dense
+ *             bf16 calls with dk = dv = 128 and chunk 64 run on the tensor cores as two
+ *             kernels (a per-chunk prep kernel, then a per-head chain kernel) and take a
+ *             stream-ordered workspace of 74 240 bytes per chunk of 64 tokens from a memory
+ *             pool the library owns (reserved memory stays in the pool for later calls); if
+ *             that workspace cannot be had, and for every other dtype, size or layout, the
+ *             call runs on the fp32 chunk kernel. Any other value: GDN_ERR_INVALID_ARG.
  *  xnorm      output normalisation (page "LinearAttention 概述", section "The Devil in Linear
  *             Transformer": the normaliser's denominator is dropped and the output is
  *             normalised instead, O = XNorm(Q (K^T V))). GDN_XNORM_NONE (0, default),

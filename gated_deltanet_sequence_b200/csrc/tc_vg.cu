@@ -577,7 +577,7 @@ vg_prep_kernel(const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__
 }
 
 // ================================================================== chain kernel
-constexpr int kVCThreads = 192;
+constexpr int kVCThreads = 320;   // TMA warp, issuer warp, 8 state warps (two per TMEM lane quarter)
 constexpr uint32_t VC_S = 2 * kRecBytes;        // S fp16 MN-major A: 2 x (128 key rows x 64 v)
 constexpr uint32_t VC_UB = VC_S + 32768;        // Ut fp16, K-major rows v
 constexpr uint32_t VC_XN = VC_UB + 16384;       // output-normalisation scratch (384 fp32)
@@ -592,8 +592,11 @@ constexpr uint32_t ID_SQW = idesc_f16(128, 128, true, true);   // [O^T | Ut^T] +
 constexpr uint32_t ID_SQ = idesc_f16(128, 64, true, true);     // O^T += S^T Q'^T (linear attention)
 constexpr uint32_t ID_ST = idesc_f16(128, 128, false, false);  // S += Kd^T Ut
 constexpr uint32_t ID_O = idesc_f16(128, 64, false, false);    // O^T += Ut^T P^T
-constexpr int kBarS = 1;
-enum : int { CB_FULL = 0, CB_CDONE = 2, CB_SRDY = 4, CB_ADONE = 5, CB_URDY = 6, kVCBars = 7 };
+constexpr int kBarS = 1;   // the 8 state warps
+constexpr int kBarO = 2;   // the 4 state warps that store the output
+// mbarriers: FULL / ODONE per stage parity (the TMA ring and the output tile of that parity);
+// SDONE: the state update of the last chunk is done (the next chunk may read S)
+enum : int { CB_FULL = 0, CB_ODONE = 2, CB_SRDY = 4, CB_ADONE = 5, CB_URDY = 6, CB_SDONE = 7, kVCBars = 8 };
 
 template <bool DELTA, bool OPTS>
 __global__ void __launch_bounds__(kVCThreads, 1)
@@ -628,12 +631,12 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        // ================================================================ TMA producer
+        // ================================================================ record loads
         if (lane == 0) {
             int last[2] = {-1, -1};
             for (int c = 0; c < nch; ++c) {
                 const int s = c & 1;
-                if (c >= 2 && !ctl.wait_lazy(CB_CDONE + s, ((c - 2) >> 1) & 1)) break;
+                if (c >= 2 && !ctl.wait_lazy(CB_ODONE + s, ((c - 2) >> 1) & 1)) break;
                 uint64_t *fb = &bars[CB_FULL + s];
                 mbar_arrive_expect_tx(fb, kRecBytes);
                 const uint8_t *src = recs + static_cast<size_t>(rec0 + c) * kRecBytes;
@@ -668,27 +671,31 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
                 for (int kk = 0; kk < 4; ++kk)
                     mma_f16(tmem + TMC_S, sdesc_sw128(stg + kRKD * 128 + kk * 32, 16, 1024),
                             sdesc_sw128(sb + VC_UB + kk * 32, 16, 1024), ID_ST, 1u);
+                mma_commit(&bars[CB_SDONE]);   // the next chunk's state copy need not wait for O
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     mma_f16(tmem + TMC_OU + s * 128, sdesc_sw128(sb + VC_UB + kk * 32, 16, 1024),
                             sdesc_sw128(stg + kRP * 128 + kk * 32, 16, 1024), ID_O, 1u);
-                mma_commit(&bars[CB_CDONE + s]);
-                last_bar = CB_CDONE + s;
+                mma_commit(&bars[CB_ODONE + s]);
+                last_bar = CB_ODONE + s;
                 last_par = (c >> 1) & 1;
             }
             if (last_bar >= 0) ctl.drain(last_bar, last_par);
         }
     } else {
-        // ================================================================ state group (warps 2-5)
-        const int j = (warp & 3) * 32 + lane;              // TMEM lane: key row j / value column v
-        const bool lead = (j == 0);
+        // ================================================================ state group (warps 2-9)
+        // thread (j, half): TMEM lane j (key row j of S, value column v = j of O and Ut), and
+        // the half of S's value columns (64 * half ..) and of Ut's columns (32 * half ..) it copies
+        const int half = (warp - 2) >> 2;
+        const int j = (warp & 3) * 32 + lane;
+        const bool lead = (j == 0 && half == 0);
         const int head = bh % H;
         float *xn = reinterpret_cast<float *>(smem + VC_XN);
         const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
         {
-            const float *src = s0 ? s0 + (static_cast<size_t>(bh) * kD + j) * kD : nullptr;
+            const float *src = s0 ? s0 + (static_cast<size_t>(bh) * kD + j) * kD + 64 * half : nullptr;
 #pragma unroll 1
-            for (int cc = 0; cc < 8; ++cc) {
+            for (int cc = 0; cc < 4; ++cc) {
                 float rr[16];
 #pragma unroll
                 for (int e = 0; e < 16; e += 4) {
@@ -696,13 +703,14 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
                                          : make_float4(0.f, 0.f, 0.f, 0.f);
                     rr[e] = x.x; rr[e + 1] = x.y; rr[e + 2] = x.z; rr[e + 3] = x.w;
                 }
-                tmem_st16(trow + TMC_S + cc * 16, rr);
+                tmem_st16(trow + TMC_S + 64 * half + cc * 16, rr);
             }
+            // the O^T tile of parity `half` starts at zero
             float z[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) z[e] = 0.f;
 #pragma unroll 1
-            for (int cc = 0; cc < 8; ++cc) tmem_st16(trow + TMC_OU + (cc >> 2) * 128 + (cc & 3) * 16, z);
+            for (int cc = 0; cc < 4; ++cc) tmem_st16(trow + TMC_OU + half * 128 + cc * 16, z);
             tmem_wait_st();
         }
         const float *egl_h = egl + static_cast<size_t>(rec0) * kD;
@@ -716,42 +724,49 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
             const float e_cur = e_next;
             if (c + 1 < nch) e_next = egl_h[static_cast<size_t>(c + 1) * kD + j];
             // S(c) complete (state update of c-1 done) and this chunk's record landed
-            if (!ctl.group_wait_all({c >= 1 ? CB_CDONE + ((c - 1) & 1) : -1, CB_FULL + s},
-                                    {static_cast<uint32_t>((c - 1) >> 1) & 1u, static_cast<uint32_t>(c >> 1) & 1u},
-                                    kBarS, lead))
+            if (!ctl.group_wait_all({c >= 1 ? CB_SDONE : -1, CB_FULL + s},
+                                    {static_cast<uint32_t>(c - 1) & 1u, static_cast<uint32_t>(c >> 1) & 1u},
+                                    kBarS, lead, 256))
                 break;
             tc_fence_after();
-            // ---- S row j -> fp16 MN-major operand; S <- exp(GL[j]) S (ahead of the update)
-#pragma unroll
-            for (int cc = 0; cc < 8; ++cc) {
-                float sv[16];
-                tmem_ld16(trow + TMC_S + cc * 16, sv);
-                tmem_wait_ld();
-                st_row16_h(sb + VC_S + (cc >> 2) * 16384u, j, (cc & 3) * 2, sv);
-#pragma unroll
-                for (int e = 0; e < 16; ++e) sv[e] *= e_cur;
-                tmem_st16(trow + TMC_S + cc * 16, sv);
-            }
-            // ---- U^T row v -> the Ut^T columns of this chunk's tile
+            // ---- this thread's half of S row j -> fp16 MN-major operand; S <- exp(GL[j]) S
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
-                const uint4 a = *reinterpret_cast<const uint4 *>(stg + sw128(kRU + j, 2 * cc));
-                const uint4 b = *reinterpret_cast<const uint4 *>(stg + sw128(kRU + j, 2 * cc + 1));
+                float sv[16];
+                tmem_ld16(trow + TMC_S + 64 * half + cc * 16, sv);
+                tmem_wait_ld();
+                st_row16_h(sb + VC_S + half * 16384u, j, cc * 2, sv);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) sv[e] *= e_cur;
+                tmem_st16(trow + TMC_S + 64 * half + cc * 16, sv);
+            }
+            // ---- U^T row v, this thread's 32 columns -> the Ut^T columns of this chunk's tile
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+                const uint4 a = *reinterpret_cast<const uint4 *>(stg + sw128(kRU + j, 4 * half + 2 * cc));
+                const uint4 b = *reinterpret_cast<const uint4 *>(stg + sw128(kRU + j, 4 * half + 2 * cc + 1));
                 const float u[16] = {h_lo(a.x), h_hi(a.x), h_lo(a.y), h_hi(a.y), h_lo(a.z), h_hi(a.z),
                                      h_lo(a.w), h_hi(a.w), h_lo(b.x), h_hi(b.x), h_lo(b.y), h_hi(b.y),
                                      h_lo(b.z), h_hi(b.z), h_lo(b.w), h_hi(b.w)};
-                tmem_st16(trow + TMC_OU + s * 128 + 64 + cc * 16, u);
+                tmem_st16(trow + TMC_OU + s * 128 + 64 + 32 * half + cc * 16, u);
             }
             tmem_wait_st();
             fence_proxy_async();
             tc_fence_before();
-            named_bar(kBarS, 128);
+            named_bar(kBarS, 256);
             if (lead) mbar_arrive(&bars[CB_SRDY]);
-            // ---- output of the previous chunk (its O tile is complete)
-            if (c >= 1) {
+            // ---- output of the previous chunk (warps of half 0), once its O tile is complete
+            if (c >= 1 && half == 0) {
                 const int cp = c - 1;
+                if (!ctl.group_wait(CB_ODONE + (cp & 1), (cp >> 1) & 1, kBarO, lead, 128)) {
+                    named_bar_any(kBarS, 256, true);   // meet the other half at its Ut barrier, then stop
+                    break;
+                }
+                tc_fence_after();
                 store_out_col<OPTS>(trow + TMC_OU + (cp & 1) * 128, out, (row0 + static_cast<size_t>(cp) * kC) * kD + j,
-                                    kC, head, j, kBarS, xn, false, nf);
+                                    kC, head, j, kBarO, xn, false, nf);
+                // chunk c + 1 accumulates onto this tile: zero it (ordered before that chunk's
+                // product by the state-ready hand-off, which this half joins)
                 float z[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) z[e] = 0.f;
@@ -760,37 +775,39 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
                 tmem_wait_st();
                 done = c;
             }
-            // ---- Ut^T row v -> Ut operand (K-major, rows v)
-            if (!ctl.group_wait(CB_ADONE, c & 1, kBarS, lead)) break;
+            // ---- Ut^T row v, this thread's 32 columns -> Ut operand (K-major, rows v)
+            if (!ctl.group_wait(CB_ADONE, c & 1, kBarS, lead, 256)) break;
             tc_fence_after();
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
+            for (int cc = 0; cc < 2; ++cc) {
                 float u[16];
-                tmem_ld16(trow + TMC_OU + s * 128 + 64 + cc * 16, u);
+                tmem_ld16(trow + TMC_OU + s * 128 + 64 + 32 * half + cc * 16, u);
                 tmem_wait_ld();
-                st_row16_h(sb + VC_UB, j, 2 * cc, u);
+                st_row16_h(sb + VC_UB, j, 4 * half + 2 * cc, u);
             }
             fence_proxy_async();
             tc_fence_before();
-            named_bar(kBarS, 128);
+            named_bar(kBarS, 256);
             if (lead) mbar_arrive(&bars[CB_URDY]);
         }
-        // ---- last output tile and the final state
-        if (nch > 0 && done == nch - 1) {
-            const int cp = nch - 1;
-            if (ctl.group_wait(CB_CDONE + (cp & 1), (cp >> 1) & 1, kBarS, lead)) {
+        // ---- last output tile (half 0) and the final state (both halves)
+        const int cp = nch - 1;
+        if (half == 0 && nch > 0 && done == cp) {
+            if (ctl.group_wait(CB_ODONE + (cp & 1), (cp >> 1) & 1, kBarO, lead, 128)) {
                 tc_fence_after();
                 store_out_col<OPTS>(trow + TMC_OU + (cp & 1) * 128, out, (row0 + static_cast<size_t>(cp) * kC) * kD + j,
-                                    L - cp * kC, head, j, kBarS, xn, true, nf);
+                                    L - cp * kC, head, j, kBarO, xn, true, nf);
                 done = nch;
             }
         }
-        if (s_final && done == nch) {
-            float *dst = s_final + (static_cast<size_t>(bh) * kD + j) * kD;
+        if (s_final && nch > 0 && ctl.group_wait(CB_SDONE, static_cast<uint32_t>(cp) & 1u, kBarS, lead, 256) &&
+            !named_bar_any(kBarS, 256, half == 0 && done != nch)) {
+            tc_fence_after();
+            float *dst = s_final + (static_cast<size_t>(bh) * kD + j) * kD + 64 * half;
 #pragma unroll 1
-            for (int cc = 0; cc < 8; ++cc) {
+            for (int cc = 0; cc < 4; ++cc) {
                 float sv[16];
-                tmem_ld16(trow + TMC_S + cc * 16, sv);
+                tmem_ld16(trow + TMC_S + 64 * half + cc * 16, sv);
                 tmem_wait_ld();
 #pragma unroll
                 for (int e = 0; e < 16; e += 4) {

@@ -593,7 +593,8 @@ constexpr uint32_t ID_SQ = idesc_f16(128, 64, true, true);     // O^T += S^T Q'^
 constexpr uint32_t ID_ST = idesc_f16(128, 128, false, false);  // S += Kd^T Ut
 constexpr uint32_t ID_O = idesc_f16(128, 64, false, false);    // O^T += Ut^T P^T
 constexpr int kBarS = 1;   // the 8 state warps
-constexpr int kBarO = 2;   // the 4 state warps that store the output
+constexpr int kBarO = 2;   // the 4 state warps that store the output (half 0)
+constexpr int kBarU = 3;   // the 4 state warps of the Ut epilogue (half 1)
 // mbarriers: FULL / ODONE per stage parity (the TMA ring and the output tile of that parity);
 // SDONE: the state update of the last chunk is done (the next chunk may read S)
 enum : int { CB_FULL = 0, CB_ODONE = 2, CB_SRDY = 4, CB_ADONE = 5, CB_URDY = 6, CB_SDONE = 7, kVCBars = 8 };
@@ -684,11 +685,14 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
         }
     } else {
         // ================================================================ state group (warps 2-9)
-        // thread (j, half): TMEM lane j (key row j of S, value column v = j of O and Ut), and
-        // the half of S's value columns (64 * half ..) and of Ut's columns (32 * half ..) it copies
+        // thread (j, half): TMEM lane j (key row j of S, value column v = j of O and Ut). Both
+        // halves copy S (value columns 64 * half ..); then half 0 stores the previous chunk's
+        // output while half 1 takes the Ut epilogue of this chunk, so the output stores stay
+        // off the state chain.
         const int half = (warp - 2) >> 2;
         const int j = (warp & 3) * 32 + lane;
-        const bool lead = (j == 0 && half == 0);
+        const bool lead = (j == 0 && half == 0);    // polls for the whole group and for half 0
+        const bool lead1 = (j == 0 && half == 1);   // polls for half 1
         const int head = bh % H;
         float *xn = reinterpret_cast<float *>(smem + VC_XN);
         const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
@@ -717,6 +721,7 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
         float e_next = nch > 0 ? egl_h[j] : 1.f;
         int done = 0;
         float nf = 0.f;
+        bool stop = false;   // this half gave up waiting; the group stops at its next meeting
 #pragma unroll 1
         for (int c = 0; c < nch; ++c) {
             const int s = c & 1;
@@ -724,75 +729,101 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
             const float e_cur = e_next;
             if (c + 1 < nch) e_next = egl_h[static_cast<size_t>(c + 1) * kD + j];
             // S(c) complete (state update of c-1 done) and this chunk's record landed
-            if (!ctl.group_wait_all({c >= 1 ? CB_SDONE : -1, CB_FULL + s},
-                                    {static_cast<uint32_t>(c - 1) & 1u, static_cast<uint32_t>(c >> 1) & 1u},
-                                    kBarS, lead, 256))
-                break;
+            {
+                bool fail = stop;
+                if (lead && !fail) fail = (c >= 1 && !ctl.wait(CB_SDONE, static_cast<uint32_t>(c - 1) & 1u)) ||
+                                          !ctl.wait(CB_FULL + s, static_cast<uint32_t>(c >> 1) & 1u);
+                if (named_bar_any(kBarS, 256, fail)) break;
+            }
             tc_fence_after();
             // ---- this thread's half of S row j -> fp16 MN-major operand; S <- exp(GL[j]) S
+            {
+                float sv[64];
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                float sv[16];
-                tmem_ld16(trow + TMC_S + 64 * half + cc * 16, sv);
+                for (int cc = 0; cc < 4; ++cc) {
+                    float t[16];
+                    tmem_ld16(trow + TMC_S + 64 * half + cc * 16, t);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) sv[16 * cc + e] = t[e];
+                }
                 tmem_wait_ld();
-                st_row16_h(sb + VC_S + half * 16384u, j, cc * 2, sv);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) sv[e] *= e_cur;
-                tmem_st16(trow + TMC_S + 64 * half + cc * 16, sv);
+                for (int cc = 0; cc < 4; ++cc) {
+                    st_row16_h(sb + VC_S + half * 16384u, j, cc * 2, sv + 16 * cc);
+                    float t[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) t[e] = sv[16 * cc + e] * e_cur;
+                    tmem_st16(trow + TMC_S + 64 * half + cc * 16, t);
+                }
             }
-            // ---- U^T row v, this thread's 32 columns -> the Ut^T columns of this chunk's tile
+            if (half == 1) {
+                // ---- U^T row v -> the Ut^T columns of this chunk's tile
 #pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-                const uint4 a = *reinterpret_cast<const uint4 *>(stg + sw128(kRU + j, 4 * half + 2 * cc));
-                const uint4 b = *reinterpret_cast<const uint4 *>(stg + sw128(kRU + j, 4 * half + 2 * cc + 1));
-                const float u[16] = {h_lo(a.x), h_hi(a.x), h_lo(a.y), h_hi(a.y), h_lo(a.z), h_hi(a.z),
-                                     h_lo(a.w), h_hi(a.w), h_lo(b.x), h_hi(b.x), h_lo(b.y), h_hi(b.y),
-                                     h_lo(b.z), h_hi(b.z), h_lo(b.w), h_hi(b.w)};
-                tmem_st16(trow + TMC_OU + s * 128 + 64 + 32 * half + cc * 16, u);
+                for (int cc = 0; cc < 4; ++cc) {
+                    const uint4 a = *reinterpret_cast<const uint4 *>(stg + sw128(kRU + j, 2 * cc));
+                    const uint4 b = *reinterpret_cast<const uint4 *>(stg + sw128(kRU + j, 2 * cc + 1));
+                    const float u[16] = {h_lo(a.x), h_hi(a.x), h_lo(a.y), h_hi(a.y), h_lo(a.z), h_hi(a.z),
+                                         h_lo(a.w), h_hi(a.w), h_lo(b.x), h_hi(b.x), h_lo(b.y), h_hi(b.y),
+                                         h_lo(b.z), h_hi(b.z), h_lo(b.w), h_hi(b.w)};
+                    tmem_st16(trow + TMC_OU + s * 128 + 64 + cc * 16, u);
+                }
             }
             tmem_wait_st();
             fence_proxy_async();
             tc_fence_before();
             named_bar(kBarS, 256);
             if (lead) mbar_arrive(&bars[CB_SRDY]);
-            // ---- output of the previous chunk (warps of half 0), once its O tile is complete
-            if (c >= 1 && half == 0) {
-                const int cp = c - 1;
-                if (!ctl.group_wait(CB_ODONE + (cp & 1), (cp >> 1) & 1, kBarO, lead, 128)) {
-                    named_bar_any(kBarS, 256, true);   // meet the other half at its Ut barrier, then stop
-                    break;
+            if (half == 0) {
+                // ---- output of the previous chunk, once its O tile is complete
+                if (c >= 1) {
+                    const int cp = c - 1;
+                    if (!ctl.group_wait(CB_ODONE + (cp & 1), (cp >> 1) & 1, kBarO, lead, 128)) {
+                        stop = true;
+                        continue;
+                    }
+                    tc_fence_after();
+                    store_out_col<OPTS>(trow + TMC_OU + (cp & 1) * 128, out,
+                                        (row0 + static_cast<size_t>(cp) * kC) * kD + j, kC, head, j, kBarO, xn, false,
+                                        nf);
+                    // chunk c + 1 accumulates onto this tile: zero it (ordered before that chunk's
+                    // product by its state-ready hand-off, which this half joins)
+                    float z[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) z[e] = 0.f;
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc) tmem_st16(trow + TMC_OU + (cp & 1) * 128 + cc * 16, z);
+                    tmem_wait_st();
+                    done = c;
+                }
+            } else {
+                // ---- Ut^T row v -> Ut operand (K-major, rows v)
+                if (!ctl.group_wait(CB_ADONE, c & 1, kBarU, lead1, 128)) {
+                    stop = true;
+                    continue;
                 }
                 tc_fence_after();
-                store_out_col<OPTS>(trow + TMC_OU + (cp & 1) * 128, out, (row0 + static_cast<size_t>(cp) * kC) * kD + j,
-                                    kC, head, j, kBarO, xn, false, nf);
-                // chunk c + 1 accumulates onto this tile: zero it (ordered before that chunk's
-                // product by the state-ready hand-off, which this half joins)
-                float z[16];
+                {
+                    float u[64];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) z[e] = 0.f;
+                    for (int cc = 0; cc < 4; ++cc) {
+                        float t[16];
+                        tmem_ld16(trow + TMC_OU + s * 128 + 64 + cc * 16, t);
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) tmem_st16(trow + TMC_OU + (cp & 1) * 128 + cc * 16, z);
-                tmem_wait_st();
-                done = c;
+                        for (int e = 0; e < 16; ++e) u[16 * cc + e] = t[e];
+                    }
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc) st_row16_h(sb + VC_UB, j, 2 * cc, u + 16 * cc);
+                }
+                fence_proxy_async();
+                tc_fence_before();
+                named_bar(kBarU, 128);
+                if (lead1) mbar_arrive(&bars[CB_URDY]);
             }
-            // ---- Ut^T row v, this thread's 32 columns -> Ut operand (K-major, rows v)
-            if (!ctl.group_wait(CB_ADONE, c & 1, kBarS, lead, 256)) break;
-            tc_fence_after();
-#pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-                float u[16];
-                tmem_ld16(trow + TMC_OU + s * 128 + 64 + 32 * half + cc * 16, u);
-                tmem_wait_ld();
-                st_row16_h(sb + VC_UB, j, 4 * half + 2 * cc, u);
-            }
-            fence_proxy_async();
-            tc_fence_before();
-            named_bar(kBarS, 256);
-            if (lead) mbar_arrive(&bars[CB_URDY]);
         }
         // ---- last output tile (half 0) and the final state (both halves)
         const int cp = nch - 1;
-        if (half == 0 && nch > 0 && done == cp) {
+        if (half == 0 && !stop && nch > 0 && done == cp) {
             if (ctl.group_wait(CB_ODONE + (cp & 1), (cp >> 1) & 1, kBarO, lead, 128)) {
                 tc_fence_after();
                 store_out_col<OPTS>(trow + TMC_OU + (cp & 1) * 128, out, (row0 + static_cast<size_t>(cp) * kC) * kD + j,
@@ -800,19 +831,23 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
                 done = nch;
             }
         }
-        if (s_final && nch > 0 && ctl.group_wait(CB_SDONE, static_cast<uint32_t>(cp) & 1u, kBarS, lead, 256) &&
-            !named_bar_any(kBarS, 256, half == 0 && done != nch)) {
-            tc_fence_after();
-            float *dst = s_final + (static_cast<size_t>(bh) * kD + j) * kD + 64 * half;
+        {
+            // the final state once the last update is done, if every output tile was stored
+            bool fail = half == 0 && done != nch;
+            if (lead && !fail && nch > 0) fail = !ctl.wait(CB_SDONE, static_cast<uint32_t>(cp) & 1u);
+            if (!named_bar_any(kBarS, 256, fail || !s_final || nch == 0)) {
+                tc_fence_after();
+                float *dst = s_final + (static_cast<size_t>(bh) * kD + j) * kD + 64 * half;
 #pragma unroll 1
-            for (int cc = 0; cc < 4; ++cc) {
-                float sv[16];
-                tmem_ld16(trow + TMC_S + 64 * half + cc * 16, sv);
-                tmem_wait_ld();
+                for (int cc = 0; cc < 4; ++cc) {
+                    float sv[16];
+                    tmem_ld16(trow + TMC_S + 64 * half + cc * 16, sv);
+                    tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 16; e += 4) {
-                    probe_finite(nf, sv[e] + sv[e + 1] + sv[e + 2] + sv[e + 3]);
-                    *reinterpret_cast<float4 *>(dst + cc * 16 + e) = make_float4(sv[e], sv[e + 1], sv[e + 2], sv[e + 3]);
+                    for (int e = 0; e < 16; e += 4) {
+                        probe_finite(nf, sv[e] + sv[e + 1] + sv[e + 2] + sv[e + 3]);
+                        *reinterpret_cast<float4 *>(dst + cc * 16 + e) = make_float4(sv[e], sv[e + 1], sv[e + 2], sv[e + 3]);
+                    }
                 }
             }
         }

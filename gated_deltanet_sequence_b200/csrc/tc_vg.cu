@@ -577,25 +577,30 @@ vg_prep_kernel(const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__
 }
 
 // ================================================================== chain kernel
-constexpr int kVCThreads = 320;   // TMA warp, issuer warp, 8 state warps (two per TMEM lane quarter)
-constexpr uint32_t VC_S = 2 * kRecBytes;        // S fp16 MN-major A: 2 x (128 key rows x 64 v)
-constexpr uint32_t VC_UB = VC_S + 32768;        // Ut fp16, K-major rows v
-constexpr uint32_t VC_XN = VC_UB + 16384;       // output-normalisation scratch (384 fp32)
+// The state is kept transposed, S^T (TMEM lane = value column v, one column per key row j), so
+// that both state-side products take their A operand from tensor memory: the fp16 copy of S^T
+// for [O^T | Ut^T] += S^T [Q'^T | -W^T], and the fp16 copy of Ut^T for S^T += Ut^T Kd and
+// O^T += Ut^T P^T. Only the record tiles (the B operands) are read from shared memory; at N = 128
+// a UMMA with both operands in shared memory reads about as many bytes per cycle as shared
+// memory delivers, so every other access there slowed the chain.
+constexpr int kVCThreads = 320;   // record-load warp, issuer warp, 8 state warps (two per TMEM lane quarter)
+constexpr uint32_t VC_EGL = 2 * kRecBytes;      // exp(GL) of each stage's chunk (2 x 128 fp32)
+constexpr uint32_t VC_XN = VC_EGL + 1024;       // output-normalisation scratch (384 fp32)
 constexpr uint32_t VC_BAR = VC_XN + 1536;       // mbarriers, TMEM base, abort flag
 constexpr uint32_t kVCSmem = VC_BAR + 256;
 constexpr uint32_t kVCAlloc = kVCSmem + 1024;
 static_assert(kVCAlloc <= 232448, "shared memory budget");
-static_assert(VC_S % 1024 == 0 && VC_UB % 1024 == 0, "UMMA tiles need 1024-B alignment");
-constexpr uint32_t TMC_S = 0;      // state S: lane = key row j, 128 value columns
-constexpr uint32_t TMC_OU = 128;   // 2 x [O^T | U^T then Ut^T]: lane = value v
-constexpr uint32_t ID_SQW = idesc_f16(128, 128, true, true);   // [O^T | Ut^T] += S^T [Q'^T | -W^T]
-constexpr uint32_t ID_SQ = idesc_f16(128, 64, true, true);     // O^T += S^T Q'^T (linear attention)
-constexpr uint32_t ID_ST = idesc_f16(128, 128, false, false);  // S += Kd^T Ut
+constexpr uint32_t TMC_S = 0;      // S^T fp32: lane = v, 128 columns j
+constexpr uint32_t TMC_SH = 128;   // S^T fp16 (A operand): 64 columns of key pairs
+constexpr uint32_t TMC_OU = 192;   // 2 x [O^T | U^T, then Ut^T; its first 32 columns then Ut^T fp16]
+constexpr uint32_t ID_SQW = idesc_f16(128, 128, false, true);  // [O^T | Ut^T] += S^T [Q'^T | -W^T]
+constexpr uint32_t ID_SQ = idesc_f16(128, 64, false, true);    // O^T += S^T Q'^T (linear attention)
+constexpr uint32_t ID_ST = idesc_f16(128, 128, false, false);  // S^T += Ut^T Kd
 constexpr uint32_t ID_O = idesc_f16(128, 64, false, false);    // O^T += Ut^T P^T
 constexpr int kBarS = 1;   // the 8 state warps
 constexpr int kBarO = 2;   // the 4 state warps that store the output (half 0)
 constexpr int kBarU = 3;   // the 4 state warps of the Ut epilogue (half 1)
-// mbarriers: FULL / ODONE per stage parity (the TMA ring and the output tile of that parity);
+// mbarriers: FULL / ODONE per stage parity (the record ring and the output tile of that parity);
 // SDONE: the state update of the last chunk is done (the next chunk may read S)
 enum : int { CB_FULL = 0, CB_ODONE = 2, CB_SRDY = 4, CB_ADONE = 5, CB_URDY = 6, CB_SDONE = 7, kVCBars = 8 };
 
@@ -639,10 +644,11 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
                 const int s = c & 1;
                 if (c >= 2 && !ctl.wait_lazy(CB_ODONE + s, ((c - 2) >> 1) & 1)) break;
                 uint64_t *fb = &bars[CB_FULL + s];
-                mbar_arrive_expect_tx(fb, kRecBytes);
+                mbar_arrive_expect_tx(fb, kRecBytes + kD * 4);
                 const uint8_t *src = recs + static_cast<size_t>(rec0 + c) * kRecBytes;
 #pragma unroll
                 for (int b = 0; b < 3; ++b) bulk_g2s(sb + s * kRecBytes + b * kRecPiece, src + b * kRecPiece, kRecPiece, fb);
+                bulk_g2s(sb + VC_EGL + s * 512, egl + static_cast<size_t>(rec0 + c) * kD, kD * 4, fb);
                 last[s] = c;
             }
             for (int s = 0; s < 2; ++s)
@@ -655,14 +661,15 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
             for (int c = 0; c < nch; ++c) {
                 const int s = c & 1;
                 const uint32_t stg = sb + s * kRecBytes;
+                const uint32_t uh = tmem + TMC_OU + s * 128 + 64;   // Ut^T fp16 of this chunk
                 if (!ctl.wait(CB_FULL + s, (c >> 1) & 1)) break;
                 if (!ctl.wait(CB_SRDY, c & 1)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_f16(tmem + TMC_OU + s * 128, sdesc_sw128(sb + VC_S + kk * 2048, 16384, 1024),
-                            sdesc_sw128(stg + kRQ * 128 + kk * 2048, (kRW - kRQ) * 128, 1024), DELTA ? ID_SQW : ID_SQ,
-                            1u);
+                    mma_f16_ts(tmem + TMC_OU + s * 128, tmem + TMC_SH + kk * 8,
+                               sdesc_sw128(stg + kRQ * 128 + kk * 2048, (kRW - kRQ) * 128, 1024), DELTA ? ID_SQW : ID_SQ,
+                               1u);
                 mma_commit(&bars[CB_ADONE]);
                 last_bar = CB_ADONE;
                 last_par = c & 1;
@@ -670,13 +677,12 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_f16(tmem + TMC_S, sdesc_sw128(stg + kRKD * 128 + kk * 32, 16, 1024),
-                            sdesc_sw128(sb + VC_UB + kk * 32, 16, 1024), ID_ST, 1u);
+                    mma_f16_ts(tmem + TMC_S, uh + kk * 8, sdesc_sw128(stg + kRKD * 128 + kk * 32, 16, 1024), ID_ST, 1u);
                 mma_commit(&bars[CB_SDONE]);   // the next chunk's state copy need not wait for O
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_f16(tmem + TMC_OU + s * 128, sdesc_sw128(sb + VC_UB + kk * 32, 16, 1024),
-                            sdesc_sw128(stg + kRP * 128 + kk * 32, 16, 1024), ID_O, 1u);
+                    mma_f16_ts(tmem + TMC_OU + s * 128, uh + kk * 8, sdesc_sw128(stg + kRP * 128 + kk * 32, 16, 1024),
+                               ID_O, 1u);
                 mma_commit(&bars[CB_ODONE + s]);
                 last_bar = CB_ODONE + s;
                 last_par = (c >> 1) & 1;
@@ -685,28 +691,25 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
         }
     } else {
         // ================================================================ state group (warps 2-9)
-        // thread (j, half): TMEM lane j (key row j of S, value column v = j of O and Ut). Both
-        // halves copy S (value columns 64 * half ..); then half 0 stores the previous chunk's
-        // output while half 1 takes the Ut epilogue of this chunk, so the output stores stay
-        // off the state chain.
+        // thread (v, half): TMEM lane v (value column v of S^T, O and Ut). Both halves copy
+        // S^T (key columns 64 * half ..); then half 0 stores the previous chunk's output while
+        // half 1 takes the Ut epilogue of this chunk, so the output stores stay off the chain.
         const int half = (warp - 2) >> 2;
-        const int j = (warp & 3) * 32 + lane;
-        const bool lead = (j == 0 && half == 0);    // polls for the whole group and for half 0
-        const bool lead1 = (j == 0 && half == 1);   // polls for half 1
+        const int v = (warp & 3) * 32 + lane;
+        const bool lead = (v == 0 && half == 0);    // polls for the whole group and for half 0
+        const bool lead1 = (v == 0 && half == 1);   // polls for half 1
         const int head = bh % H;
         float *xn = reinterpret_cast<float *>(smem + VC_XN);
         const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
         {
-            const float *src = s0 ? s0 + (static_cast<size_t>(bh) * kD + j) * kD + 64 * half : nullptr;
+            // S^T[v][j] = S0[j][v] for this thread's 64 key rows j (a warp reads 128 bytes per j)
+            const float *src = s0 ? s0 + static_cast<size_t>(bh) * kD * kD + static_cast<size_t>(64 * half) * kD + v
+                                  : nullptr;
 #pragma unroll 1
             for (int cc = 0; cc < 4; ++cc) {
                 float rr[16];
 #pragma unroll
-                for (int e = 0; e < 16; e += 4) {
-                    const float4 x = src ? *reinterpret_cast<const float4 *>(src + cc * 16 + e)
-                                         : make_float4(0.f, 0.f, 0.f, 0.f);
-                    rr[e] = x.x; rr[e + 1] = x.y; rr[e + 2] = x.z; rr[e + 3] = x.w;
-                }
+                for (int e = 0; e < 16; ++e) rr[e] = src ? src[static_cast<size_t>(cc * 16 + e) * kD] : 0.f;
                 tmem_st16(trow + TMC_S + 64 * half + cc * 16, rr);
             }
             // the O^T tile of parity `half` starts at zero
@@ -717,8 +720,6 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
             for (int cc = 0; cc < 4; ++cc) tmem_st16(trow + TMC_OU + half * 128 + cc * 16, z);
             tmem_wait_st();
         }
-        const float *egl_h = egl + static_cast<size_t>(rec0) * kD;
-        float e_next = nch > 0 ? egl_h[j] : 1.f;
         int done = 0;
         float nf = 0.f;
         bool stop = false;   // this half gave up waiting; the group stops at its next meeting
@@ -726,8 +727,6 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
         for (int c = 0; c < nch; ++c) {
             const int s = c & 1;
             const uint8_t *stg = smem + s * kRecBytes;
-            const float e_cur = e_next;
-            if (c + 1 < nch) e_next = egl_h[static_cast<size_t>(c + 1) * kD + j];
             // S(c) complete (state update of c-1 done) and this chunk's record landed
             {
                 bool fail = stop;
@@ -736,7 +735,7 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
                 if (named_bar_any(kBarS, 256, fail)) break;
             }
             tc_fence_after();
-            // ---- this thread's half of S row j -> fp16 MN-major operand; S <- exp(GL[j]) S
+            // ---- this thread's 64 columns of S^T -> fp16 operand; S^T <- S^T diag(exp(GL))
             {
                 float sv[64];
 #pragma unroll
@@ -748,11 +747,24 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
                 }
                 tmem_wait_ld();
 #pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    float hv[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) hv[e] = __uint_as_float(pack_h2(sv[32 * cc + 2 * e], sv[32 * cc + 2 * e + 1]));
+                    tmem_st16(trow + TMC_SH + 32 * half + 16 * cc, hv);
+                }
+                const float *eg = reinterpret_cast<const float *>(smem + VC_EGL + s * 512) + 64 * half;
+#pragma unroll
                 for (int cc = 0; cc < 4; ++cc) {
-                    st_row16_h(sb + VC_S + half * 16384u, j, cc * 2, sv + 16 * cc);
                     float t[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) t[e] = sv[16 * cc + e] * e_cur;
+                    for (int e = 0; e < 16; e += 4) {
+                        const float4 f = *reinterpret_cast<const float4 *>(eg + 16 * cc + e);
+                        t[e] = sv[16 * cc + e] * f.x;
+                        t[e + 1] = sv[16 * cc + e + 1] * f.y;
+                        t[e + 2] = sv[16 * cc + e + 2] * f.z;
+                        t[e + 3] = sv[16 * cc + e + 3] * f.w;
+                    }
                     tmem_st16(trow + TMC_S + 64 * half + cc * 16, t);
                 }
             }
@@ -760,8 +772,8 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
                 // ---- U^T row v -> the Ut^T columns of this chunk's tile
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) {
-                    const uint4 a = *reinterpret_cast<const uint4 *>(stg + sw128(kRU + j, 2 * cc));
-                    const uint4 b = *reinterpret_cast<const uint4 *>(stg + sw128(kRU + j, 2 * cc + 1));
+                    const uint4 a = *reinterpret_cast<const uint4 *>(stg + sw128(kRU + v, 2 * cc));
+                    const uint4 b = *reinterpret_cast<const uint4 *>(stg + sw128(kRU + v, 2 * cc + 1));
                     const float u[16] = {h_lo(a.x), h_hi(a.x), h_lo(a.y), h_hi(a.y), h_lo(a.z), h_hi(a.z),
                                          h_lo(a.w), h_hi(a.w), h_lo(b.x), h_hi(b.x), h_lo(b.y), h_hi(b.y),
                                          h_lo(b.z), h_hi(b.z), h_lo(b.w), h_hi(b.w)};
@@ -769,7 +781,6 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
                 }
             }
             tmem_wait_st();
-            fence_proxy_async();
             tc_fence_before();
             named_bar(kBarS, 256);
             if (lead) mbar_arrive(&bars[CB_SRDY]);
@@ -783,7 +794,7 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
                     }
                     tc_fence_after();
                     store_out_col<OPTS>(trow + TMC_OU + (cp & 1) * 128, out,
-                                        (row0 + static_cast<size_t>(cp) * kC) * kD + j, kC, head, j, kBarO, xn, false,
+                                        (row0 + static_cast<size_t>(cp) * kC) * kD + v, kC, head, v, kBarO, xn, false,
                                         nf);
                     // chunk c + 1 accumulates onto this tile: zero it (ordered before that chunk's
                     // product by its state-ready hand-off, which this half joins)
@@ -796,7 +807,8 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
                     done = c;
                 }
             } else {
-                // ---- Ut^T row v -> Ut operand (K-major, rows v)
+                // ---- Ut^T row v -> fp16 pairs over its first 32 columns (A operand of the
+                //      state update and of the output product)
                 if (!ctl.group_wait(CB_ADONE, c & 1, kBarU, lead1, 128)) {
                     stop = true;
                     continue;
@@ -813,9 +825,14 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
                     }
                     tmem_wait_ld();
 #pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) st_row16_h(sb + VC_UB, j, 2 * cc, u + 16 * cc);
+                    for (int cc = 0; cc < 2; ++cc) {
+                        float hv[16];
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) hv[e] = __uint_as_float(pack_h2(u[32 * cc + 2 * e], u[32 * cc + 2 * e + 1]));
+                        tmem_st16(trow + TMC_OU + s * 128 + 64 + 16 * cc, hv);
+                    }
+                    tmem_wait_st();
                 }
-                fence_proxy_async();
                 tc_fence_before();
                 named_bar(kBarU, 128);
                 if (lead1) mbar_arrive(&bars[CB_URDY]);
@@ -826,8 +843,8 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
         if (half == 0 && !stop && nch > 0 && done == cp) {
             if (ctl.group_wait(CB_ODONE + (cp & 1), (cp >> 1) & 1, kBarO, lead, 128)) {
                 tc_fence_after();
-                store_out_col<OPTS>(trow + TMC_OU + (cp & 1) * 128, out, (row0 + static_cast<size_t>(cp) * kC) * kD + j,
-                                    L - cp * kC, head, j, kBarO, xn, true, nf);
+                store_out_col<OPTS>(trow + TMC_OU + (cp & 1) * 128, out, (row0 + static_cast<size_t>(cp) * kC) * kD + v,
+                                    L - cp * kC, head, v, kBarO, xn, true, nf);
                 done = nch;
             }
         }
@@ -837,16 +854,16 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
             if (lead && !fail && nch > 0) fail = !ctl.wait(CB_SDONE, static_cast<uint32_t>(cp) & 1u);
             if (!named_bar_any(kBarS, 256, fail || !s_final || nch == 0)) {
                 tc_fence_after();
-                float *dst = s_final + (static_cast<size_t>(bh) * kD + j) * kD + 64 * half;
+                float *dst = s_final + static_cast<size_t>(bh) * kD * kD + static_cast<size_t>(64 * half) * kD + v;
 #pragma unroll 1
                 for (int cc = 0; cc < 4; ++cc) {
                     float sv[16];
                     tmem_ld16(trow + TMC_S + 64 * half + cc * 16, sv);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 16; e += 4) {
-                        probe_finite(nf, sv[e] + sv[e + 1] + sv[e + 2] + sv[e + 3]);
-                        *reinterpret_cast<float4 *>(dst + cc * 16 + e) = make_float4(sv[e], sv[e + 1], sv[e + 2], sv[e + 3]);
+                    for (int e = 0; e < 16; ++e) {
+                        probe_finite(nf, sv[e]);
+                        dst[static_cast<size_t>(cc * 16 + e) * kD] = sv[e];
                     }
                 }
             }

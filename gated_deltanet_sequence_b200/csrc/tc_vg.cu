@@ -584,8 +584,9 @@ vg_prep_kernel(const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__
 // a UMMA with both operands in shared memory reads about as many bytes per cycle as shared
 // memory delivers, so every other access there slowed the chain.
 constexpr int kVCThreads = 320;   // record-load warp, issuer warp, 8 state warps (two per TMEM lane quarter)
-constexpr uint32_t VC_EGL = 2 * kRecBytes;      // exp(GL) of each stage's chunk (2 x 128 fp32)
-constexpr uint32_t VC_XN = VC_EGL + 1024;       // output-normalisation scratch (384 fp32)
+constexpr int kVCStages = 3;      // records in flight: one SM's bulk loads take about a chunk's time each
+constexpr uint32_t VC_EGL = kVCStages * kRecBytes;   // exp(GL) of each stage's chunk (128 fp32 each)
+constexpr uint32_t VC_XN = VC_EGL + 512 * kVCStages;  // output-normalisation scratch (384 fp32)
 constexpr uint32_t VC_BAR = VC_XN + 1536;       // mbarriers, TMEM base, abort flag
 constexpr uint32_t kVCSmem = VC_BAR + 256;
 constexpr uint32_t kVCAlloc = kVCSmem + 1024;
@@ -600,9 +601,11 @@ constexpr uint32_t ID_O = idesc_f16(128, 64, false, false);    // O^T += Ut^T P^
 constexpr int kBarS = 1;   // the 8 state warps
 constexpr int kBarO = 2;   // the 4 state warps that store the output (half 0)
 constexpr int kBarU = 3;   // the 4 state warps of the Ut epilogue (half 1)
-// mbarriers: FULL / ODONE per stage parity (the record ring and the output tile of that parity);
-// SDONE: the state update of the last chunk is done (the next chunk may read S)
-enum : int { CB_FULL = 0, CB_ODONE = 2, CB_SRDY = 4, CB_ADONE = 5, CB_URDY = 6, CB_SDONE = 7, kVCBars = 8 };
+// mbarriers: FULL / ODONE per record stage (chunk c takes stage c % 3; ODONE also marks its
+// output tile, parity c & 1, complete); SDONE: the state update of the last chunk is done (the
+// next chunk may read S, and every UMMA issued before it, such as the output product of the
+// chunk before, is complete)
+enum : int { CB_FULL = 0, CB_ODONE = 3, CB_SRDY = 6, CB_ADONE = 7, CB_URDY = 8, CB_SDONE = 9, kVCBars = 10 };
 
 template <bool DELTA, bool OPTS>
 __global__ void __launch_bounds__(kVCThreads, 1)
@@ -639,30 +642,30 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
     if (warp == 0) {
         // ================================================================ record loads
         if (lane == 0) {
-            int last[2] = {-1, -1};
+            int last[kVCStages] = {-1, -1, -1};
             for (int c = 0; c < nch; ++c) {
-                const int s = c & 1;
-                if (c >= 2 && !ctl.wait_lazy(CB_ODONE + s, ((c - 2) >> 1) & 1)) break;
-                uint64_t *fb = &bars[CB_FULL + s];
+                const int st = c % kVCStages;
+                if (c >= kVCStages && !ctl.wait_lazy(CB_ODONE + st, ((c - kVCStages) / kVCStages) & 1)) break;
+                uint64_t *fb = &bars[CB_FULL + st];
                 mbar_arrive_expect_tx(fb, kRecBytes + kD * 4);
                 const uint8_t *src = recs + static_cast<size_t>(rec0 + c) * kRecBytes;
 #pragma unroll
-                for (int b = 0; b < 3; ++b) bulk_g2s(sb + s * kRecBytes + b * kRecPiece, src + b * kRecPiece, kRecPiece, fb);
-                bulk_g2s(sb + VC_EGL + s * 512, egl + static_cast<size_t>(rec0 + c) * kD, kD * 4, fb);
-                last[s] = c;
+                for (int b = 0; b < 3; ++b) bulk_g2s(sb + st * kRecBytes + b * kRecPiece, src + b * kRecPiece, kRecPiece, fb);
+                bulk_g2s(sb + VC_EGL + st * 512, egl + static_cast<size_t>(rec0 + c) * kD, kD * 4, fb);
+                last[st] = c;
             }
-            for (int s = 0; s < 2; ++s)
-                if (last[s] >= 0) ctl.drain(CB_FULL + s, (last[s] >> 1) & 1);
+            for (int st = 0; st < kVCStages; ++st)
+                if (last[st] >= 0) ctl.drain(CB_FULL + st, (last[st] / kVCStages) & 1);
         }
     } else if (warp == 1) {
         // ================================================================ chain UMMA issuer
         if (lane == 0) {
             int last_bar = -1, last_par = 0;
             for (int c = 0; c < nch; ++c) {
-                const int s = c & 1;
-                const uint32_t stg = sb + s * kRecBytes;
+                const int s = c & 1, st = c % kVCStages;
+                const uint32_t stg = sb + st * kRecBytes;
                 const uint32_t uh = tmem + TMC_OU + s * 128 + 64;   // Ut^T fp16 of this chunk
-                if (!ctl.wait(CB_FULL + s, (c >> 1) & 1)) break;
+                if (!ctl.wait(CB_FULL + st, (c / kVCStages) & 1)) break;
                 if (!ctl.wait(CB_SRDY, c & 1)) break;
                 tc_fence_after();
 #pragma unroll
@@ -683,9 +686,9 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
                 for (int kk = 0; kk < 4; ++kk)
                     mma_f16_ts(tmem + TMC_OU + s * 128, uh + kk * 8, sdesc_sw128(stg + kRP * 128 + kk * 32, 16, 1024),
                                ID_O, 1u);
-                mma_commit(&bars[CB_ODONE + s]);
-                last_bar = CB_ODONE + s;
-                last_par = (c >> 1) & 1;
+                mma_commit(&bars[CB_ODONE + st]);
+                last_bar = CB_ODONE + st;
+                last_par = (c / kVCStages) & 1;
             }
             if (last_bar >= 0) ctl.drain(last_bar, last_par);
         }
@@ -725,13 +728,13 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
         bool stop = false;   // this half gave up waiting; the group stops at its next meeting
 #pragma unroll 1
         for (int c = 0; c < nch; ++c) {
-            const int s = c & 1;
-            const uint8_t *stg = smem + s * kRecBytes;
+            const int s = c & 1, st = c % kVCStages;
+            const uint8_t *stg = smem + st * kRecBytes;
             // S(c) complete (state update of c-1 done) and this chunk's record landed
             {
                 bool fail = stop;
                 if (lead && !fail) fail = (c >= 1 && !ctl.wait(CB_SDONE, static_cast<uint32_t>(c - 1) & 1u)) ||
-                                          !ctl.wait(CB_FULL + s, static_cast<uint32_t>(c >> 1) & 1u);
+                                          !ctl.wait(CB_FULL + st, static_cast<uint32_t>(c / kVCStages) & 1u);
                 if (named_bar_any(kBarS, 256, fail)) break;
             }
             tc_fence_after();
@@ -753,7 +756,7 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
                     for (int e = 0; e < 16; ++e) hv[e] = __uint_as_float(pack_h2(sv[32 * cc + 2 * e], sv[32 * cc + 2 * e + 1]));
                     tmem_st16(trow + TMC_SH + 32 * half + 16 * cc, hv);
                 }
-                const float *eg = reinterpret_cast<const float *>(smem + VC_EGL + s * 512) + 64 * half;
+                const float *eg = reinterpret_cast<const float *>(smem + VC_EGL + st * 512) + 64 * half;
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) {
                     float t[16];
@@ -788,7 +791,7 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
                 // ---- output of the previous chunk, once its O tile is complete
                 if (c >= 1) {
                     const int cp = c - 1;
-                    if (!ctl.group_wait(CB_ODONE + (cp & 1), (cp >> 1) & 1, kBarO, lead, 128)) {
+                    if (!ctl.group_wait(CB_ODONE + cp % kVCStages, (cp / kVCStages) & 1, kBarO, lead, 128)) {
                         stop = true;
                         continue;
                     }
@@ -841,7 +844,7 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
         // ---- last output tile (half 0) and the final state (both halves)
         const int cp = nch - 1;
         if (half == 0 && !stop && nch > 0 && done == cp) {
-            if (ctl.group_wait(CB_ODONE + (cp & 1), (cp >> 1) & 1, kBarO, lead, 128)) {
+            if (ctl.group_wait(CB_ODONE + cp % kVCStages, (cp / kVCStages) & 1, kBarO, lead, 128)) {
                 tc_fence_after();
                 store_out_col<OPTS>(trow + TMC_OU + (cp & 1) * 128, out, (row0 + static_cast<size_t>(cp) * kC) * kD + v,
                                     L - cp * kC, head, v, kBarO, xn, true, nf);

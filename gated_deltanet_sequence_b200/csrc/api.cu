@@ -48,12 +48,15 @@ gdn_status_t check_prefill(const void *q, const void *k, const void *v, const fl
 }  // namespace
 
 namespace gdn {
-// Vector-valued gates on the tensor cores (dense batches; tc_vg.cu): a per-chunk prep kernel
-// and a per-head chain kernel with a stream-ordered workspace. *fallback is set when the call
-// cannot run there (no workspace, or too many chunks); nothing has been launched then.
-gdn_status_t launch_tc_vg(bool delta, const void *q, const void *k, const void *v, const float *beta, const float *g,
-                          void *o, const float *s0, float *s_final, int B, int H, int L, float scale, FwdOpts oo,
-                          cudaStream_t stream, bool *fallback);
+// The per-chunk prep kernel and the per-head chain kernel (tc_vg.cu), dense bf16 batches at
+// dk = dv = 128, C = 64, with a stream-ordered workspace: vector-valued gates (per_key), and
+// scalar gates for few heads with long sequences (tc_vg_takes_scalar), whose sequences are then
+// cut into segments whose prep overlaps the chain of the segment before. *fallback is set when
+// the call cannot run there (no workspace, or too many chunks); nothing has been launched then.
+gdn_status_t launch_tc_vg(bool delta, bool per_key, const void *q, const void *k, const void *v, const float *beta,
+                          const float *g, void *o, const float *s0, float *s_final, int B, int H, int L, float scale,
+                          FwdOpts oo, cudaStream_t stream, bool *fallback);
+bool tc_vg_takes_scalar(int B, int H, int L);
 }  // namespace gdn
 
 extern "C" {
@@ -94,6 +97,13 @@ gdn_status_t gdn_chunk_fwd(const void *q, const void *k, const void *v, const fl
     if (L > 0 && !beta) return GDN_ERR_INVALID_ARG;
     if (!opt_aligned4(beta)) return GDN_ERR_INVALID_ARG;
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+    if (gdn::tc_supported(in_dtype, dk, dv, chunk) && L > 0 && gdn::tc_vg_takes_scalar(B, H, L)) {
+        // few heads, long sequences: prep on every SM, overlapped with the per-head chain
+        bool fallback = false;
+        const gdn_status_t vs = gdn::launch_tc_vg(true, false, q, k, v, beta, g, o, s0, s_final, B, H, L, scale,
+                                                  kDefaultOut, stream, &fallback);
+        if (!fallback) return vs;
+    }
     if (gdn::tc_supported(in_dtype, dk, dv, chunk) && L > 0)
         return gdn::launch_tc_gdn(q, k, v, beta, g, o, s0, s_final, nullptr, B, H, L, scale, kDefaultOut, stream);
     // with L == 0 beta may be NULL: the kernel then only writes s0 (or zeros) to s_final
@@ -164,7 +174,13 @@ static gdn_status_t prefill_ex(bool delta, const void *q, const void *k, const v
     // C = 64; the fp32 chunk kernel for every other input dtype, size and layout
     if (gdn::tc_supported(in_dtype, dk, dv, chunk) && L > 0 && oo.gate_per_key && !cu_seqlens) {
         bool fallback = false;
-        const gdn_status_t vs = gdn::launch_tc_vg(delta, q, k, v, beta, g, o, s0, s_final, B, H, L, scale, oo,
+        const gdn_status_t vs = gdn::launch_tc_vg(delta, true, q, k, v, beta, g, o, s0, s_final, B, H, L, scale, oo,
+                                                  stream, &fallback);
+        if (!fallback) return vs;
+    }
+    if (delta && gdn::tc_supported(in_dtype, dk, dv, chunk) && L > 0 && !cu_seqlens && gdn::tc_vg_takes_scalar(B, H, L)) {
+        bool fallback = false;
+        const gdn_status_t vs = gdn::launch_tc_vg(true, false, q, k, v, beta, g, o, s0, s_final, B, H, L, scale, oo,
                                                   stream, &fallback);
         if (!fallback) return vs;
     }

@@ -34,7 +34,9 @@
 // one exp per element, are added on the CUDA cores; when more than 32 coordinates of a chunk
 // are such, the whole Gram of that chunk is formed that way. Every other factor (exp(G),
 // exp(GL - G), exp(GL)) is at most 1 for non-positive log-decays and is formed directly.
+#include <algorithm>
 #include <mutex>
+#include <vector>
 
 #include "tc_gdn_parts.cuh"
 
@@ -89,23 +91,29 @@ constexpr uint32_t X3 = 65536;    // Q'^T and Kd^T (32 KB); then T fp32 (pitch 6
 constexpr uint32_t XS = X1;       // every coordinate exact: G fp32 32 KB, k and q bf16 16 KB each (X1-X3)
 constexpr uint32_t VP_TF = X3, VP_RS = X3 + 17408, VP_P = X3 + 22528;
 constexpr int kTP = 68;
-constexpr uint32_t VP_VEC = 98304;   // beta[64] | c[128] | slot u8[128] | count | bars | tmem | abort
-constexpr uint32_t kVPSmem = VP_VEC + 1024;
+constexpr uint32_t VP_VEC = 98304;   // beta[64] | c[128] | slot u8[128] | count | bars | tmem | abort |
+                                     // scalar gate: G[64], exp(G)[64], exp(-G)[64], factored flag
+constexpr uint32_t kVPSmem = VP_VEC + 2048;
 constexpr uint32_t kVPAlloc = kVPSmem + 1024;
 static_assert(kVPAlloc * 2 + 2048 <= 233472, "two prep CTAs per SM");
 static_assert(VP_P + 8192 <= X3 + 32768, "P after T and the block scratch");
 constexpr uint32_t V_BETA = 0, V_C = 256, V_SLOT = 768, V_NSLOW = 896, V_BARS = 928, V_TMEM = 960, V_ABORT = 964;
+constexpr uint32_t V_GROW = 1024, V_GAM = 1280, V_IG = 1536, V_FACT = 1792;
+constexpr float kFastDecayLimit = -60.f;   // scalar gate, G_last >= this: exp(G_r - G_s) = exp(G_r) exp(-G_s)
 // tensor memory (256 columns)
 constexpr uint32_t TMV_G = 0, TMV_W = 64, TMV_U = 128;
 constexpr uint32_t ID_G16 = idesc_f16(128, 64, false, false);   // Gram: both K-major, fp16
 constexpr uint32_t ID_WU = idesc_f16(128, 64, true, false);     // W^T, U^T: A MN-major
 enum : int { VB_V = 0, VB_G = 1, VB_WU = 2, kVPBars = 3 };
 
-template <bool DELTA>
+// SCALAR: g holds one log-decay per token (or is null); the Gram then runs on the plain tiles and
+// the masks take exp(G_r - G_s) per element. CTA i takes chunk cbase + i % nseg of head i / nseg
+// and writes record i.
+template <bool DELTA, bool SCALAR>
 __global__ void __launch_bounds__(kVPThreads, 2)
 vg_prep_kernel(const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__restrict__ q,
                const __nv_bfloat16 *__restrict__ k, const float *__restrict__ beta, const float *__restrict__ g,
-               uint8_t *__restrict__ recs, float *__restrict__ egl, int L, int nch, float scale,
+               uint8_t *__restrict__ recs, float *__restrict__ egl, int L, int cbase, int nseg, float scale,
                long long wait_limit, unsigned *__restrict__ err_word) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -122,7 +130,8 @@ vg_prep_kernel(const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const long long rec_id = blockIdx.x;
-    const int bh = static_cast<int>(rec_id / nch), c = static_cast<int>(rec_id - static_cast<long long>(bh) * nch);
+    const int bh = static_cast<int>(rec_id / nseg);
+    const int c = cbase + static_cast<int>(rec_id - static_cast<long long>(bh) * nseg);
     const int nvalid = min(kC, L - c * kC);
     const size_t row0 = static_cast<size_t>(bh) * L + static_cast<size_t>(c) * kC;
     uint8_t *rec = recs + static_cast<size_t>(rec_id) * kRecBytes;
@@ -151,9 +160,13 @@ vg_prep_kernel(const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__
         const int r = r0 + i;
         if (r < nvalid) {
             const size_t e = (row0 + r) * kD + j0;
-            const float2 gg = *reinterpret_cast<const float2 *>(g + e);
-            G0[i] = gg.x;
-            G1[i] = gg.y;
+            if constexpr (SCALAR) {
+                G0[i] = G1[i] = g ? g[row0 + r] : 0.f;
+            } else {
+                const float2 gg = *reinterpret_cast<const float2 *>(g + e);
+                G0[i] = gg.x;
+                G1[i] = gg.y;
+            }
             kw[i] = *reinterpret_cast<const uint32_t *>(k + e);
             qw[i] = *reinterpret_cast<const uint32_t *>(q + e);
         } else {
@@ -207,7 +220,8 @@ vg_prep_kernel(const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__
         hi0 = fmaxf(hi0, tot[1024 + hh * 128 + j0]);
         hi1 = fmaxf(hi1, tot[1024 + hh * 128 + j0 + 1]);
     }
-    const bool f0 = hi0 - lo0 <= kSpanFast, f1 = hi1 - lo1 <= kSpanFast;   // false for NaN ranges
+    // factored Gram coordinates (false for NaN ranges); the scalar gate takes the plain tiles
+    const bool f0 = SCALAR || hi0 - lo0 <= kSpanFast, f1 = SCALAR || hi1 - lo1 <= kSpanFast;
     if (h == 0) {
         if (!f0) slot[j0] = static_cast<uint8_t>(atomicAdd(nslow_p, 1));
         if (!f1) slot[j0 + 1] = static_cast<uint8_t>(atomicAdd(nslow_p, 1));
@@ -217,13 +231,14 @@ vg_prep_kernel(const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__
     __syncthreads();   // gate sums read; the exact-coordinate slots are assigned
     const int nslow = *nslow_p;
     const bool allslow = nslow > kSlowCap;
-    const bool fa0 = f0 && !allslow, fa1 = f1 && !allslow;
+    const bool fa0 = !SCALAR && f0 && !allslow, fa1 = !SCALAR && f1 && !allslow;
     // reference c of the factors: the midpoint of the range for factored coordinates, else 0
     const float c0 = fa0 ? 0.5f * (lo0 + hi0) : 0.f, c1 = fa1 ? 0.5f * (lo1 + hi1) : 0.f;
     if (h == 0) {
         cv[j0] = c0;
         cv[j0 + 1] = c1;
     }
+    if (SCALAR && tid == 0) *reinterpret_cast<int *>(vec + V_FACT) = gl0 >= kFastDecayLimit ? 1 : 0;
     const float ec0 = fa0 ? __expf(c0) : 0.f, ec1 = fa1 ? __expf(c1) : 0.f;
     const float edc0 = fa0 ? __expf(gl0 - c0) : 0.f, edc1 = fa1 ? __expf(gl1 - c1) : 0.f;
     uint32_t qT0[8], qT1[8], dT0[8], dT1[8];   // fp16 pairs along r for the transposed rows
@@ -234,7 +249,20 @@ vg_prep_kernel(const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__
         const float k0 = bf_lo(kw[i]), k1 = bf_hi(kw[i]), q0 = bf_lo(qw[i]), q1 = bf_hi(qw[i]);
         // K o e^(G-c) (Gram A rows, and W's operand), Q o e^(G-c), K o e^(c-G) (Gram B rows)
         float ka0, qa0 = 0.f, kb0 = 0.f, eg0, ed0, ka1, qa1 = 0.f, kb1 = 0.f, eg1, ed1;
-        if (fa0) {
+        if constexpr (SCALAR) {
+            // plain tiles; exp(G_r) and exp(GL - G_r) once per row
+            eg0 = eg1 = __expf(G0[i]);
+            ed0 = ed1 = __expf(gl0 - G0[i]);
+            ka0 = kb0 = k0;
+            ka1 = kb1 = k1;
+            qa0 = q0;
+            qa1 = q1;
+            if (p == 0) {
+                reinterpret_cast<float *>(vec + V_GROW)[r] = G0[i];
+                reinterpret_cast<float *>(vec + V_GAM)[r] = eg0;
+                reinterpret_cast<float *>(vec + V_IG)[r] = gl0 >= kFastDecayLimit ? __expf(-G0[i]) : 0.f;
+            }
+        } else if (fa0) {
             const float e1 = __expf(G0[i] - c0), e2 = __expf(c0 - G0[i]);
             ka0 = k0 * e1;
             qa0 = q0 * e1;
@@ -246,7 +274,8 @@ vg_prep_kernel(const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__
             ed0 = __expf(gl0 - G0[i]);
             ka0 = k0 * eg0;
         }
-        if (fa1) {
+        if (SCALAR) {
+        } else if (fa1) {
             const float e1 = __expf(G1[i] - c1), e2 = __expf(c1 - G1[i]);
             ka1 = k1 * e1;
             qa1 = q1 * e1;
@@ -383,6 +412,19 @@ vg_prep_kernel(const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__
     if (tid == 0) bulk_wait_read();   // Q'^T / Kd^T have left X3 (P and T go there)
     tc_fence_before();
     __syncthreads();   // Gram and exact-coordinate data read: A^T and P may overwrite them
+    if constexpr (SCALAR) {
+        // the decay of the plain Gram: Gamma_rs = exp(G_r - G_s), factored when G_last >= -60
+        const float *Gw = reinterpret_cast<const float *>(vec + V_GROW);
+        const float *gam = reinterpret_cast<const float *>(vec + V_GAM);
+        const float *ig = reinterpret_cast<const float *>(vec + V_IG);
+        const bool fact = *reinterpret_cast<const int *>(vec + V_FACT) != 0;
+        const float gr = gam[r], Gr = Gw[r];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+            const int s2 = 32 * hh + e;
+            v[e] *= fact ? gr * ig[s2] : (s2 <= r ? __expf(Gr - Gw[s2]) : 0.f);
+        }
+    }
     if (!isP) {
         if (DELTA) {
             float *At = reinterpret_cast<float *>(smem + X2);   // At[s * 64 + r] = A[r][s]
@@ -411,7 +453,7 @@ vg_prep_kernel(const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__
     if (warp < 4) {
         const float *At = reinterpret_cast<const float *>(smem + X2);
         float *Tf = reinterpret_cast<float *>(smem + VP_TF);    // Tf[r * kTP + c] = T[r][c]
-        for (int i = tid; i < 8192 / 16; i += 128)              // T diag(beta): upper blocks stay zero
+        for (int i = tid; i < (SCALAR ? 16384 : 8192) / 16; i += 128)   // T factors: upper blocks stay zero
             *reinterpret_cast<uint4 *>(smem + X1 + i * 16) = make_uint4(0u, 0u, 0u, 0u);
         if (!DELTA) {
             // linear attention: T = I, so T diag(beta) is the identity (U = V)
@@ -430,6 +472,14 @@ vg_prep_kernel(const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__
                 st_shared_v4(sb + X1 + sw128(rr, cc0 >> 3), pack_h2(t0.x * b0.x, t0.y * b0.y),
                              pack_h2(t0.z * b0.z, t0.w * b0.w), pack_h2(t1.x * b1.x, t1.y * b1.y),
                              pack_h2(t1.z * b1.z, t1.w * b1.w));
+                if constexpr (SCALAR) {
+                    // T diag(beta gamma) for W = T diag(beta gamma) K (the plain K tile)
+                    const float *gm = reinterpret_cast<const float *>(vec + V_GAM) + cc0;
+                    st_shared_v4(sb + X1 + 8192 + sw128(rr, cc0 >> 3), pack_h2(t0.x * b0.x * gm[0], t0.y * b0.y * gm[1]),
+                                 pack_h2(t0.z * b0.z * gm[2], t0.w * b0.w * gm[3]),
+                                 pack_h2(t1.x * b1.x * gm[4], t1.y * b1.y * gm[5]),
+                                 pack_h2(t1.z * b1.z * gm[6], t1.w * b1.w * gm[7]));
+                }
             };
             const int bi = warp, cl = lane & 15;
             if (ok) {
@@ -529,7 +579,7 @@ vg_prep_kernel(const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
                 mma_f16(tmem + TMV_W, sdesc_sw128(sb + X0 + kk * 2048, 16384, 1024),
-                        sdesc_sw128(sb + X1 + kk * 32, 16, 1024), ID_WU, kk > 0);
+                        sdesc_sw128(sb + X1 + (SCALAR ? 8192u : 0u) + kk * 32, 16, 1024), ID_WU, kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
@@ -610,7 +660,7 @@ enum : int { CB_FULL = 0, CB_ODONE = 3, CB_SRDY = 6, CB_ADONE = 7, CB_URDY = 8, 
 template <bool DELTA, bool OPTS>
 __global__ void __launch_bounds__(kVCThreads, 1)
 vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl, const OutArgs out,
-                const float *__restrict__ s0, float *__restrict__ s_final, int H, int L, int nch,
+                const float *__restrict__ s0, float *__restrict__ s_final, int H, int L, int cbase, int nch,
                 long long wait_limit, unsigned *__restrict__ err_word) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -622,7 +672,11 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int bh = blockIdx.x;
-    const size_t row0 = static_cast<size_t>(bh) * L;
+    // this launch takes chunks cbase .. cbase + nch - 1 of the head (records bh * nch ..); rows of
+    // the chunk with index c of the launch start at row0 + c * C
+    const size_t row0 = static_cast<size_t>(bh) * L + static_cast<size_t>(cbase) * kC;
+    const int Lrem = L - cbase * kC;                     // tokens from the launch's first chunk on
+    const bool seq_end = cbase + nch == (L + kC - 1) / kC;   // the launch ends the sequence
     const long long rec0 = static_cast<long long>(bh) * nch;
 
     if (tid == 0) {
@@ -847,7 +901,7 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
             if (ctl.group_wait(CB_ODONE + cp % kVCStages, (cp / kVCStages) & 1, kBarO, lead, 128)) {
                 tc_fence_after();
                 store_out_col<OPTS>(trow + TMC_OU + (cp & 1) * 128, out, (row0 + static_cast<size_t>(cp) * kC) * kD + v,
-                                    L - cp * kC, head, v, kBarO, xn, true, nf);
+                                    min(kC, Lrem - cp * kC), head, v, kBarO, xn, seq_end, nf);
                 done = nch;
             }
         }
@@ -912,75 +966,160 @@ cudaMemPool_t record_pool(int dev) {
     return pools[dev];
 }
 
-template <bool DELTA, bool OPTS>
-gdn_status_t launch_vg_t(const CUtensorMap &mv, const void *q, const void *k,
-                         const float *beta, const float *g, uint8_t *recs, float *egl, const OutArgs &out,
-                         const float *s0, float *s_final, int BH, int H, int L, int nch, float scale,
-                         cudaStream_t stream) {
-    auto kp = vg_prep_kernel<DELTA>;
-    auto kc = vg_chain_kernel<DELTA, OPTS>;
-    if (!ensure_smem_limit(reinterpret_cast<const void *>(kp), kVPAlloc) ||
-        !ensure_smem_limit(reinterpret_cast<const void *>(kc), kVCAlloc))
-        return GDN_ERR_CUDA;
+template <bool DELTA, bool SCALAR>
+bool launch_prep(const CUtensorMap &mv, const void *q, const void *k, const void *v, const float *beta,
+                 const float *g, uint8_t *recs, float *egl, int BH, int L, int cbase, int nseg, float scale,
+                 cudaStream_t stream) {
+    auto kp = vg_prep_kernel<DELTA, SCALAR>;
+    if (!ensure_smem_limit(reinterpret_cast<const void *>(kp), kVPAlloc)) return false;
     unsigned *err = device_error_word();
-    if (!err) return GDN_ERR_CUDA;
-    const long long nrec = static_cast<long long>(BH) * nch;
-    kp<<<static_cast<unsigned>(nrec), kVPThreads, kVPAlloc, stream>>>(
-        mv, static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k), beta, g, recs, egl, L, nch,
-        scale, wait_limit_cycles(), err);
-    if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
-    kc<<<BH, kVCThreads, kVCAlloc, stream>>>(recs, egl, out, s0, s_final, H, L, nch, wait_limit_cycles(), err);
-    return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+    if (!err) return false;
+    kp<<<static_cast<unsigned>(static_cast<long long>(BH) * nseg), kVPThreads, kVPAlloc, stream>>>(
+        mv, static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k), beta, g, recs, egl, L,
+        cbase, nseg, scale, wait_limit_cycles(), err);
+    return cudaGetLastError() == cudaSuccess;
+}
+
+template <bool DELTA, bool OPTS>
+bool launch_chain(const uint8_t *recs, const float *egl, const OutArgs &out, const float *s0, float *s_final, int BH,
+                  int H, int L, int cbase, int nseg, cudaStream_t stream) {
+    auto kc = vg_chain_kernel<DELTA, OPTS>;
+    if (!ensure_smem_limit(reinterpret_cast<const void *>(kc), kVCAlloc)) return false;
+    unsigned *err = device_error_word();
+    if (!err) return false;
+    kc<<<BH, kVCThreads, kVCAlloc, stream>>>(recs, egl, out, s0, s_final, H, L, cbase, nseg, wait_limit_cycles(),
+                                             err);
+    return cudaGetLastError() == cudaSuccess;
+}
+
+bool prep_any(bool delta, bool scalar, const CUtensorMap &mv, const void *q, const void *k, const void *v,
+              const float *beta, const float *g, uint8_t *recs, float *egl, int BH, int L, int cbase, int nseg,
+              float scale, cudaStream_t stream) {
+    if (delta)
+        return scalar ? launch_prep<true, true>(mv, q, k, v, beta, g, recs, egl, BH, L, cbase, nseg, scale, stream)
+                      : launch_prep<true, false>(mv, q, k, v, beta, g, recs, egl, BH, L, cbase, nseg, scale, stream);
+    return scalar ? launch_prep<false, true>(mv, q, k, v, beta, g, recs, egl, BH, L, cbase, nseg, scale, stream)
+                  : launch_prep<false, false>(mv, q, k, v, beta, g, recs, egl, BH, L, cbase, nseg, scale, stream);
+}
+
+bool chain_any(bool delta, bool opts, const uint8_t *recs, const float *egl, const OutArgs &out, const float *s0,
+               float *s_final, int BH, int H, int L, int cbase, int nseg, cudaStream_t stream) {
+    if (delta)
+        return opts ? launch_chain<true, true>(recs, egl, out, s0, s_final, BH, H, L, cbase, nseg, stream)
+                    : launch_chain<true, false>(recs, egl, out, s0, s_final, BH, H, L, cbase, nseg, stream);
+    return opts ? launch_chain<false, true>(recs, egl, out, s0, s_final, BH, H, L, cbase, nseg, stream)
+                : launch_chain<false, false>(recs, egl, out, s0, s_final, BH, H, L, cbase, nseg, stream);
+}
+
+// A second stream per device (created once) on which the prep kernel of the next segment of a
+// long sequence runs while the chain kernel of the current one runs on the caller's stream.
+cudaStream_t side_stream(int dev) {
+    static std::mutex mu;
+    static cudaStream_t streams[64] = {};
+    if (dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!streams[dev] && cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess) {
+        cudaGetLastError();
+        streams[dev] = nullptr;
+    }
+    return streams[dev];
+}
+
+constexpr int kSegChunks = 64;   // chunks of each head per segment when a call is split
+
+// Few heads with long sequences: the chain kernel runs on as many SMs as there are heads,
+// so the sequence is cut into segments and the prep of segment i + 1 runs on the other SMs
+// while the chain takes segment i.
+bool split_in_segments(int BH, int nch) {
+    const int sms = sm_count();
+    return sms > 0 && 3LL * BH <= sms && nch >= 2 * kSegChunks;
 }
 
 }  // namespace
 
 size_t tc_vg_workspace_bytes(int B, int H, int L) {
     const long long nch = (static_cast<long long>(L) + kC - 1) / kC;
-    return static_cast<size_t>(B) * H * nch * (kRecBytes + kD * sizeof(float));
+    const long long BH = static_cast<long long>(B) * H;
+    const size_t per_chunk = kRecBytes + kD * sizeof(float);
+    if (split_in_segments(static_cast<int>(BH), static_cast<int>(nch)))
+        return 2 * static_cast<size_t>(BH) * kSegChunks * per_chunk + static_cast<size_t>(BH) * kD * kD * sizeof(float);
+    return static_cast<size_t>(BH) * nch * per_chunk;
 }
 
-gdn_status_t launch_tc_vg(bool delta, const void *q, const void *k, const void *v, const float *beta, const float *g,
-                          void *o, const float *s0, float *s_final, int B, int H, int L, float scale, FwdOpts oo,
-                          cudaStream_t stream, bool *fallback) {
+bool tc_vg_takes_scalar(int B, int H, int L) {
+    return split_in_segments(B * H, (L + kC - 1) / kC);
+}
+
+gdn_status_t launch_tc_vg(bool delta, bool per_key, const void *q, const void *k, const void *v, const float *beta,
+                          const float *g, void *o, const float *s0, float *s_final, int B, int H, int L, float scale,
+                          FwdOpts oo, cudaStream_t stream, bool *fallback) {
     *fallback = false;
     const int BH = B * H;
     const int nch = (L + kC - 1) / kC;
-    const long long nrec = static_cast<long long>(BH) * nch;
-    if (nrec > 2147483647LL) {   // one prep CTA per chunk
-        *fallback = true;
-        return GDN_ERR_UNSUPPORTED;
-    }
-    if (reinterpret_cast<uintptr_t>(g) % 8 != 0) {   // the prep kernel reads g two floats at a time
+    const bool split = split_in_segments(BH, nch);
+    const int seg = split ? kSegChunks : nch;
+    const long long nrec = static_cast<long long>(BH) * seg;   // records of one segment
+    if (nrec > 2147483647LL || (per_key && reinterpret_cast<uintptr_t>(g) % 8 != 0)) {
+        // one prep CTA per record; the vector-gate prep reads g two floats at a time
         *fallback = true;
         return GDN_ERR_UNSUPPORTED;
     }
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return GDN_ERR_CUDA;
     cudaMemPool_t pool = record_pool(dev);
+    cudaStream_t side = split ? side_stream(dev) : nullptr;
     void *ws = nullptr;
-    if (!pool || cudaMallocFromPoolAsync(&ws, tc_vg_workspace_bytes(B, H, L), pool, stream) != cudaSuccess) {
+    if (!pool || (split && !side) ||
+        cudaMallocFromPoolAsync(&ws, tc_vg_workspace_bytes(B, H, L), pool, stream) != cudaSuccess) {
         cudaGetLastError();
         *fallback = true;   // the caller takes the kernel that needs no workspace
         return GDN_ERR_CUDA;
     }
-    uint8_t *recs = static_cast<uint8_t *>(ws);
-    float *egl = reinterpret_cast<float *>(recs + static_cast<size_t>(nrec) * kRecBytes);
+    const size_t slot_bytes = static_cast<size_t>(nrec) * (kRecBytes + kD * sizeof(float));
+    auto recs_of = [&](int slot) { return static_cast<uint8_t *>(ws) + slot * slot_bytes; };
+    auto egl_of = [&](int slot) { return reinterpret_cast<float *>(recs_of(slot) + static_cast<size_t>(nrec) * kRecBytes); };
     CUtensorMap mv;
-    gdn_status_t st = GDN_ERR_CUDA;
-    if (make_qkv_map(&mv, v, L, BH)) {
-        const OutArgs out = make_out_args(o, v, oo);
-        const bool opts = oo.bf16 || oo.dskip != nullptr || oo.xnorm != kXNormNone;
-        if (delta)
-            st = opts ? launch_vg_t<true, true>(mv, q, k, beta, g, recs, egl, out, s0, s_final, BH, H, L, nch, scale, stream)
-                      : launch_vg_t<true, false>(mv, q, k, beta, g, recs, egl, out, s0, s_final, BH, H, L, nch, scale, stream);
-        else
-            st = opts ? launch_vg_t<false, true>(mv, q, k, beta, g, recs, egl, out, s0, s_final, BH, H, L, nch, scale, stream)
-                      : launch_vg_t<false, false>(mv, q, k, beta, g, recs, egl, out, s0, s_final, BH, H, L, nch, scale, stream);
+    const OutArgs out = make_out_args(o, v, oo);
+    const bool opts = oo.bf16 || oo.dskip != nullptr || oo.xnorm != kXNormNone;
+    const bool scalar = !per_key;
+    bool ok = make_qkv_map(&mv, v, L, BH);
+    if (ok && !split) {
+        ok = prep_any(delta, scalar, mv, q, k, v, beta, g, recs_of(0), egl_of(0), BH, L, 0, nch, scale, stream) &&
+             chain_any(delta, opts, recs_of(0), egl_of(0), out, s0, s_final, BH, H, L, 0, nch, stream);
+    } else if (ok) {
+        // segments of kSegChunks chunks; records in two slots; the state between segments in a
+        // (BH, dk, dv) buffer after the slots
+        float *state = reinterpret_cast<float *>(recs_of(2));
+        const int nsegs = (nch + seg - 1) / seg;
+        std::vector<cudaEvent_t> evs;
+        auto event = [&]() -> cudaEvent_t {
+            cudaEvent_t e = nullptr;
+            if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return nullptr;
+            evs.push_back(e);
+            return e;
+        };
+        cudaEvent_t start = event();
+        ok = start && cudaEventRecord(start, stream) == cudaSuccess && cudaStreamWaitEvent(side, start, 0) == cudaSuccess;
+        std::vector<cudaEvent_t> chain_done(nsegs, nullptr);
+        for (int i = 0; ok && i < nsegs; ++i) {
+            const int cb = i * seg, n = std::min(seg, nch - cb), sl = i & 1;
+            if (i >= 2) ok = cudaStreamWaitEvent(side, chain_done[i - 2], 0) == cudaSuccess;   // slot reuse
+            cudaEvent_t prepped = ok ? event() : nullptr;
+            ok = ok && prepped && prep_any(delta, scalar, mv, q, k, v, beta, g, recs_of(sl), egl_of(sl), BH, L, cb, n, scale, side) &&
+                 cudaEventRecord(prepped, side) == cudaSuccess && cudaStreamWaitEvent(stream, prepped, 0) == cudaSuccess;
+            chain_done[i] = ok ? event() : nullptr;
+            ok = ok && chain_done[i] &&
+                 chain_any(delta, opts, recs_of(sl), egl_of(sl), out, i == 0 ? s0 : state,
+                           i == nsegs - 1 ? s_final : state, BH, H, L, cb, n, stream) &&
+                 cudaEventRecord(chain_done[i], stream) == cudaSuccess;
+        }
+        if (!ok) cudaStreamSynchronize(side);   // leave nothing of this call running on the side stream
+        for (cudaEvent_t e : evs) cudaEventDestroy(e);   // released once their work is done
     }
-    // stream-ordered: the records are released once both kernels have run
-    if (cudaFreeAsync(ws, stream) != cudaSuccess && st == GDN_OK) st = GDN_ERR_CUDA;
-    return st;
+    // stream-ordered: the workspace is released once every kernel of the call has run (the side
+    // stream's work all precedes events the caller's stream waited for)
+    const bool freed = cudaFreeAsync(ws, stream) == cudaSuccess;
+    return ok && freed ? GDN_OK : GDN_ERR_CUDA;
 }
 
 }  // namespace gdn

@@ -1011,18 +1011,28 @@ bool chain_any(bool delta, bool opts, const uint8_t *recs, const float *egl, con
                 : launch_chain<false, false>(recs, egl, out, s0, s_final, BH, H, L, cbase, nseg, stream);
 }
 
-// A second stream per device (created once) on which the prep kernel of the next segment of a
-// long sequence runs while the chain kernel of the current one runs on the caller's stream.
-cudaStream_t side_stream(int dev) {
+// Two streams per device (created once) for a long sequence cut into segments: the prep
+// kernels on one with the lowest priority, the chain kernels on one with the highest, so that
+// as the prep CTAs of segment i + 1 retire, the SMs they free go to the chain of segment i.
+struct SegStreams {
+    cudaStream_t prep = nullptr, chain = nullptr;
+};
+SegStreams seg_streams(int dev) {
     static std::mutex mu;
-    static cudaStream_t streams[64] = {};
-    if (dev < 0 || dev >= 64) return nullptr;
+    static SegStreams streams[64];
+    if (dev < 0 || dev >= 64) return SegStreams{};
     std::lock_guard<std::mutex> lock(mu);
-    if (!streams[dev] && cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess) {
-        cudaGetLastError();
-        streams[dev] = nullptr;
+    SegStreams &s = streams[dev];
+    if (!s.prep || !s.chain) {
+        int least = 0, greatest = 0;
+        if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess ||
+            (!s.prep && cudaStreamCreateWithPriority(&s.prep, cudaStreamNonBlocking, least) != cudaSuccess) ||
+            (!s.chain && cudaStreamCreateWithPriority(&s.chain, cudaStreamNonBlocking, greatest) != cudaSuccess)) {
+            cudaGetLastError();
+            return SegStreams{};
+        }
     }
-    return streams[dev];
+    return s;
 }
 
 constexpr int kSegChunks = 64;   // chunks of each head per segment when a call is split
@@ -1067,9 +1077,9 @@ gdn_status_t launch_tc_vg(bool delta, bool per_key, const void *q, const void *k
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return GDN_ERR_CUDA;
     cudaMemPool_t pool = record_pool(dev);
-    cudaStream_t side = split ? side_stream(dev) : nullptr;
+    const SegStreams ss = split ? seg_streams(dev) : SegStreams{};
     void *ws = nullptr;
-    if (!pool || (split && !side) ||
+    if (!pool || (split && (!ss.prep || !ss.chain)) ||
         cudaMallocFromPoolAsync(&ws, tc_vg_workspace_bytes(B, H, L), pool, stream) != cudaSuccess) {
         cudaGetLastError();
         *fallback = true;   // the caller takes the kernel that needs no workspace
@@ -1099,21 +1109,30 @@ gdn_status_t launch_tc_vg(bool delta, bool per_key, const void *q, const void *k
             return e;
         };
         cudaEvent_t start = event();
-        ok = start && cudaEventRecord(start, stream) == cudaSuccess && cudaStreamWaitEvent(side, start, 0) == cudaSuccess;
+        ok = start && cudaEventRecord(start, stream) == cudaSuccess && cudaStreamWaitEvent(ss.prep, start, 0) == cudaSuccess &&
+             cudaStreamWaitEvent(ss.chain, start, 0) == cudaSuccess;
         std::vector<cudaEvent_t> chain_done(nsegs, nullptr);
         for (int i = 0; ok && i < nsegs; ++i) {
             const int cb = i * seg, n = std::min(seg, nch - cb), sl = i & 1;
-            if (i >= 2) ok = cudaStreamWaitEvent(side, chain_done[i - 2], 0) == cudaSuccess;   // slot reuse
+            if (i >= 2) ok = cudaStreamWaitEvent(ss.prep, chain_done[i - 2], 0) == cudaSuccess;   // slot reuse
             cudaEvent_t prepped = ok ? event() : nullptr;
-            ok = ok && prepped && prep_any(delta, scalar, mv, q, k, v, beta, g, recs_of(sl), egl_of(sl), BH, L, cb, n, scale, side) &&
-                 cudaEventRecord(prepped, side) == cudaSuccess && cudaStreamWaitEvent(stream, prepped, 0) == cudaSuccess;
+            ok = ok && prepped &&
+                 prep_any(delta, scalar, mv, q, k, v, beta, g, recs_of(sl), egl_of(sl), BH, L, cb, n, scale, ss.prep) &&
+                 cudaEventRecord(prepped, ss.prep) == cudaSuccess && cudaStreamWaitEvent(ss.chain, prepped, 0) == cudaSuccess;
             chain_done[i] = ok ? event() : nullptr;
             ok = ok && chain_done[i] &&
                  chain_any(delta, opts, recs_of(sl), egl_of(sl), out, i == 0 ? s0 : state,
-                           i == nsegs - 1 ? s_final : state, BH, H, L, cb, n, stream) &&
-                 cudaEventRecord(chain_done[i], stream) == cudaSuccess;
+                           i == nsegs - 1 ? s_final : state, BH, H, L, cb, n, ss.chain) &&
+                 cudaEventRecord(chain_done[i], ss.chain) == cudaSuccess;
         }
-        if (!ok) cudaStreamSynchronize(side);   // leave nothing of this call running on the side stream
+        // the caller's stream continues once the last chain kernel is done (it follows every
+        // kernel of the call)
+        ok = ok && cudaStreamWaitEvent(stream, chain_done[nsegs - 1], 0) == cudaSuccess;
+        if (!ok) {
+            // leave nothing of this call running behind the caller's back
+            cudaStreamSynchronize(ss.prep);
+            cudaStreamSynchronize(ss.chain);
+        }
         for (cudaEvent_t e : evs) cudaEventDestroy(e);   // released once their work is done
     }
     // stream-ordered: the workspace is released once every kernel of the call has run (the side

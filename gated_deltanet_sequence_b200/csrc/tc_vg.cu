@@ -633,7 +633,7 @@ vg_prep_kernel(const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__
 // O^T += Ut^T P^T. Only the record tiles (the B operands) are read from shared memory; at N = 128
 // a UMMA with both operands in shared memory reads about as many bytes per cycle as shared
 // memory delivers, so every other access there slowed the chain.
-constexpr int kVCThreads = 320;   // record-load warp, issuer warp, 8 state warps (two per TMEM lane quarter)
+constexpr int kVCThreads = 320;   // record-load warp, an idle warp, 8 state warps (two per TMEM lane quarter)
 constexpr int kVCStages = 3;      // records in flight: one SM's bulk loads take about a chunk's time each
 constexpr uint32_t VC_EGL = kVCStages * kRecBytes;   // exp(GL) of each stage's chunk (128 fp32 each)
 constexpr uint32_t VC_XN = VC_EGL + 512 * kVCStages;  // output-normalisation scratch (384 fp32)
@@ -643,7 +643,7 @@ constexpr uint32_t kVCAlloc = kVCSmem + 1024;
 static_assert(kVCAlloc <= 232448, "shared memory budget");
 constexpr uint32_t TMC_S = 0;      // S^T fp32: lane = v, 128 columns j
 constexpr uint32_t TMC_SH = 128;   // S^T fp16 (A operand): 64 columns of key pairs
-constexpr uint32_t TMC_OU = 192;   // 2 x [O^T | U^T, then Ut^T; its first 32 columns then Ut^T fp16]
+constexpr uint32_t TMC_OU = 192;   // 2 x [O^T | -(W S)^T; its first 32 columns then Ut^T fp16]
 constexpr uint32_t ID_SQW = idesc_f16(128, 128, false, true);  // [O^T | Ut^T] += S^T [Q'^T | -W^T]
 constexpr uint32_t ID_SQ = idesc_f16(128, 64, false, true);    // O^T += S^T Q'^T (linear attention)
 constexpr uint32_t ID_ST = idesc_f16(128, 128, false, false);  // S^T += Ut^T Kd
@@ -652,10 +652,10 @@ constexpr int kBarS = 1;   // the 8 state warps
 constexpr int kBarO = 2;   // the 4 state warps that store the output (half 0)
 constexpr int kBarU = 3;   // the 4 state warps of the Ut epilogue (half 1)
 // mbarriers: FULL / ODONE per record stage (chunk c takes stage c % 3; ODONE also marks its
-// output tile, parity c & 1, complete); SDONE: the state update of the last chunk is done (the
-// next chunk may read S, and every UMMA issued before it, such as the output product of the
-// chunk before, is complete)
-enum : int { CB_FULL = 0, CB_ODONE = 3, CB_SRDY = 6, CB_ADONE = 7, CB_URDY = 8, CB_SDONE = 9, kVCBars = 10 };
+// output tile, parity c & 1, complete); ADONE: the [O^T | Ut^T] product is done; DEC: half 0
+// has written its decayed half of S^T; SDONE: the state update of the last chunk is done (the
+// next chunk may read S, and every UMMA lead1 issued before it is complete)
+enum : int { CB_FULL = 0, CB_ODONE = 3, CB_ADONE = 6, CB_DEC = 7, CB_SDONE = 8, kVCBars = 9 };
 
 template <bool DELTA, bool OPTS>
 __global__ void __launch_bounds__(kVCThreads, 1)
@@ -675,7 +675,7 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
     // this launch takes chunks cbase .. cbase + nch - 1 of the head (records bh * nch ..); rows of
     // the chunk with index c of the launch start at row0 + c * C
     const size_t row0 = static_cast<size_t>(bh) * L + static_cast<size_t>(cbase) * kC;
-    const int Lrem = L - cbase * kC;                     // tokens from the launch's first chunk on
+    const int Lrem = L - cbase * kC;                         // tokens from the launch's first chunk on
     const bool seq_end = cbase + nch == (L + kC - 1) / kC;   // the launch ends the sequence
     const long long rec0 = static_cast<long long>(bh) * nch;
 
@@ -711,46 +711,14 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
             for (int st = 0; st < kVCStages; ++st)
                 if (last[st] >= 0) ctl.drain(CB_FULL + st, (last[st] / kVCStages) & 1);
         }
-    } else if (warp == 1) {
-        // ================================================================ chain UMMA issuer
-        if (lane == 0) {
-            int last_bar = -1, last_par = 0;
-            for (int c = 0; c < nch; ++c) {
-                const int s = c & 1, st = c % kVCStages;
-                const uint32_t stg = sb + st * kRecBytes;
-                const uint32_t uh = tmem + TMC_OU + s * 128 + 64;   // Ut^T fp16 of this chunk
-                if (!ctl.wait(CB_FULL + st, (c / kVCStages) & 1)) break;
-                if (!ctl.wait(CB_SRDY, c & 1)) break;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_f16_ts(tmem + TMC_OU + s * 128, tmem + TMC_SH + kk * 8,
-                               sdesc_sw128(stg + kRQ * 128 + kk * 2048, (kRW - kRQ) * 128, 1024), DELTA ? ID_SQW : ID_SQ,
-                               1u);
-                mma_commit(&bars[CB_ADONE]);
-                last_bar = CB_ADONE;
-                last_par = c & 1;
-                if (!ctl.wait(CB_URDY, c & 1)) break;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_f16_ts(tmem + TMC_S, uh + kk * 8, sdesc_sw128(stg + kRKD * 128 + kk * 32, 16, 1024), ID_ST, 1u);
-                mma_commit(&bars[CB_SDONE]);   // the next chunk's state copy need not wait for O
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_f16_ts(tmem + TMC_OU + s * 128, uh + kk * 8, sdesc_sw128(stg + kRP * 128 + kk * 32, 16, 1024),
-                               ID_O, 1u);
-                mma_commit(&bars[CB_ODONE + st]);
-                last_bar = CB_ODONE + st;
-                last_par = (c / kVCStages) & 1;
-            }
-            if (last_bar >= 0) ctl.drain(last_bar, last_par);
-        }
-    } else {
+    } else if (warp >= 2) {
         // ================================================================ state group (warps 2-9)
         // thread (v, half): TMEM lane v (value column v of S^T, O and Ut). Both halves copy
         // S^T (key columns 64 * half ..); then half 0 stores the previous chunk's output while
         // half 1 takes the Ut epilogue of this chunk, so the output stores stay off the chain.
+        // The group issues the chain's UMMAs itself: thread `lead` the [O^T | Ut^T] product once
+        // the fp16 copy of S^T is complete, thread `lead1` the state update and the output
+        // product once the fp16 copy of Ut^T is complete.
         const int half = (warp - 2) >> 2;
         const int v = (warp & 3) * 32 + lane;
         const bool lead = (v == 0 && half == 0);    // polls for the whole group and for half 0
@@ -769,21 +737,17 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
                 for (int e = 0; e < 16; ++e) rr[e] = src ? src[static_cast<size_t>(cc * 16 + e) * kD] : 0.f;
                 tmem_st16(trow + TMC_S + 64 * half + cc * 16, rr);
             }
-            // the O^T tile of parity `half` starts at zero
-            float z[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) z[e] = 0.f;
-#pragma unroll 1
-            for (int cc = 0; cc < 4; ++cc) tmem_st16(trow + TMC_OU + half * 128 + cc * 16, z);
             tmem_wait_st();
         }
         int done = 0;
+        int issued_a = -1, issued_o = -1;   // last chunk whose products lead / lead1 committed
         float nf = 0.f;
         bool stop = false;   // this half gave up waiting; the group stops at its next meeting
 #pragma unroll 1
         for (int c = 0; c < nch; ++c) {
             const int s = c & 1, st = c % kVCStages;
             const uint8_t *stg = smem + st * kRecBytes;
+            const uint32_t stg_a = sb + st * kRecBytes;
             // S(c) complete (state update of c-1 done) and this chunk's record landed
             {
                 bool fail = stop;
@@ -792,24 +756,40 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
                 if (named_bar_any(kBarS, 256, fail)) break;
             }
             tc_fence_after();
-            // ---- this thread's 64 columns of S^T -> fp16 operand; S^T <- S^T diag(exp(GL))
+            // ---- this thread's 64 columns of S^T -> fp16 operand (the critical path), then
+            //      S^T <- S^T diag(exp(GL)) while the product runs
+            float sv[64];
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                float t[16];
+                tmem_ld16(trow + TMC_S + 64 * half + cc * 16, t);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) sv[16 * cc + e] = t[e];
+            }
+            tmem_wait_ld();
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+                float hv[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) hv[e] = __uint_as_float(pack_h2(sv[32 * cc + 2 * e], sv[32 * cc + 2 * e + 1]));
+                tmem_st16(trow + TMC_SH + 32 * half + 16 * cc, hv);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            named_bar(kBarS, 256);
+            if (lead) {
+                // [O^T | -(W S)^T] = S^T [Q'^T | -W^T] into a fresh tile (U^T is added by the Ut
+                // epilogue; linear attention: O^T = S^T Q'^T, Ut = U)
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_f16_ts(tmem + TMC_OU + s * 128, tmem + TMC_SH + kk * 8,
+                               sdesc_sw128(stg_a + kRQ * 128 + kk * 2048, (kRW - kRQ) * 128, 1024),
+                               DELTA ? ID_SQW : ID_SQ, kk > 0 ? 1u : 0u);
+                mma_commit(&bars[CB_ADONE]);
+                issued_a = c;
+            }
             {
-                float sv[64];
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    float t[16];
-                    tmem_ld16(trow + TMC_S + 64 * half + cc * 16, t);
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) sv[16 * cc + e] = t[e];
-                }
-                tmem_wait_ld();
-#pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    float hv[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) hv[e] = __uint_as_float(pack_h2(sv[32 * cc + 2 * e], sv[32 * cc + 2 * e + 1]));
-                    tmem_st16(trow + TMC_SH + 32 * half + 16 * cc, hv);
-                }
                 const float *eg = reinterpret_cast<const float *>(smem + VC_EGL + st * 512) + 64 * half;
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) {
@@ -824,24 +804,13 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
                     }
                     tmem_st16(trow + TMC_S + 64 * half + cc * 16, t);
                 }
+                tmem_wait_st();
             }
-            if (half == 1) {
-                // ---- U^T row v -> the Ut^T columns of this chunk's tile
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    const uint4 a = *reinterpret_cast<const uint4 *>(stg + sw128(kRU + v, 2 * cc));
-                    const uint4 b = *reinterpret_cast<const uint4 *>(stg + sw128(kRU + v, 2 * cc + 1));
-                    const float u[16] = {h_lo(a.x), h_hi(a.x), h_lo(a.y), h_hi(a.y), h_lo(a.z), h_hi(a.z),
-                                         h_lo(a.w), h_hi(a.w), h_lo(b.x), h_hi(b.x), h_lo(b.y), h_hi(b.y),
-                                         h_lo(b.z), h_hi(b.z), h_lo(b.w), h_hi(b.w)};
-                    tmem_st16(trow + TMC_OU + s * 128 + 64 + cc * 16, u);
-                }
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            named_bar(kBarS, 256);
-            if (lead) mbar_arrive(&bars[CB_SRDY]);
             if (half == 0) {
+                // the decayed half of S^T is in place: hand it to the state update
+                tc_fence_before();
+                named_bar(kBarO, 128);
+                if (lead) mbar_arrive(&bars[CB_DEC]);
                 // ---- output of the previous chunk, once its O tile is complete
                 if (c >= 1) {
                     const int cp = c - 1;
@@ -853,14 +822,6 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
                     store_out_col<OPTS>(trow + TMC_OU + (cp & 1) * 128, out,
                                         (row0 + static_cast<size_t>(cp) * kC) * kD + v, kC, head, v, kBarO, xn, false,
                                         nf);
-                    // chunk c + 1 accumulates onto this tile: zero it (ordered before that chunk's
-                    // product by its state-ready hand-off, which this half joins)
-                    float z[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) z[e] = 0.f;
-#pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) tmem_st16(trow + TMC_OU + (cp & 1) * 128 + cc * 16, z);
-                    tmem_wait_st();
                     done = c;
                 }
             } else {
@@ -872,15 +833,34 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
                 }
                 tc_fence_after();
                 {
+                    // Ut^T = U^T - (W S)^T: U^T row v from the record (GDN); linear attention
+                    // has no W, so Ut^T = U^T
                     float u[64];
+                    if (DELTA) {
 #pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) {
-                        float t[16];
-                        tmem_ld16(trow + TMC_OU + s * 128 + 64 + cc * 16, t);
+                        for (int cc = 0; cc < 4; ++cc) {
+                            float t[16];
+                            tmem_ld16(trow + TMC_OU + s * 128 + 64 + cc * 16, t);
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) u[16 * cc + e] = t[e];
+                            for (int e = 0; e < 16; ++e) u[16 * cc + e] = t[e];
+                        }
+                        tmem_wait_ld();
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 64; ++e) u[e] = 0.f;
                     }
-                    tmem_wait_ld();
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) {
+                        const uint4 a = *reinterpret_cast<const uint4 *>(stg + sw128(kRU + v, ch));
+                        u[8 * ch] += h_lo(a.x);
+                        u[8 * ch + 1] += h_hi(a.x);
+                        u[8 * ch + 2] += h_lo(a.y);
+                        u[8 * ch + 3] += h_hi(a.y);
+                        u[8 * ch + 4] += h_lo(a.z);
+                        u[8 * ch + 5] += h_hi(a.z);
+                        u[8 * ch + 6] += h_lo(a.w);
+                        u[8 * ch + 7] += h_hi(a.w);
+                    }
 #pragma unroll
                     for (int cc = 0; cc < 2; ++cc) {
                         float hv[16];
@@ -891,10 +871,32 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
                     tmem_wait_st();
                 }
                 tc_fence_before();
-                named_bar(kBarU, 128);
-                if (lead1) mbar_arrive(&bars[CB_URDY]);
+                const bool fail = lead1 && !ctl.wait(CB_DEC, static_cast<uint32_t>(c) & 1u);
+                if (named_bar_any(kBarU, 128, fail)) {
+                    stop = true;
+                    continue;
+                }
+                if (lead1) {
+                    // S^T += Ut^T Kd ; O^T += Ut^T P^T
+                    const uint32_t uh = tmem + TMC_OU + s * 128 + 64;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_f16_ts(tmem + TMC_S, uh + kk * 8, sdesc_sw128(stg_a + kRKD * 128 + kk * 32, 16, 1024), ID_ST,
+                                   1u);
+                    mma_commit(&bars[CB_SDONE]);   // the next chunk's state copy need not wait for O
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_f16_ts(tmem + TMC_OU + s * 128, uh + kk * 8, sdesc_sw128(stg_a + kRP * 128 + kk * 32, 16, 1024),
+                                   ID_O, 1u);
+                    mma_commit(&bars[CB_ODONE + st]);
+                    issued_o = c;
+                }
             }
         }
+        // UMMAs complete in issue order: each issuing thread waits for its last commit
+        if (lead && issued_a >= 0) ctl.drain(CB_ADONE, static_cast<uint32_t>(issued_a) & 1u);
+        if (lead1 && issued_o >= 0) ctl.drain(CB_ODONE + issued_o % kVCStages, (issued_o / kVCStages) & 1);
         // ---- last output tile (half 0) and the final state (both halves)
         const int cp = nch - 1;
         if (half == 0 && !stop && nch > 0 && done == cp) {
@@ -914,13 +916,13 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
                 float *dst = s_final + static_cast<size_t>(bh) * kD * kD + static_cast<size_t>(64 * half) * kD + v;
 #pragma unroll 1
                 for (int cc = 0; cc < 4; ++cc) {
-                    float sv[16];
-                    tmem_ld16(trow + TMC_S + 64 * half + cc * 16, sv);
+                    float t[16];
+                    tmem_ld16(trow + TMC_S + 64 * half + cc * 16, t);
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
-                        probe_finite(nf, sv[e]);
-                        dst[static_cast<size_t>(cc * 16 + e) * kD] = sv[e];
+                        probe_finite(nf, t[e]);
+                        dst[static_cast<size_t>(cc * 16 + e) * kD] = t[e];
                     }
                 }
             }

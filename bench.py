@@ -381,7 +381,10 @@ def measure_rows(gdn, peaks, peak_src, args):
     ms = timed(fn, max(3, args.steps // 4), 2)
     nb = prefill_bytes(w.B, w.H, w.L, w.dk, w.dv, 2, True, True, True, True)
     fl = flops_per_head_token("gdn", w.dk, w.dv, w.chunk) * w.B * w.H * w.L
-    rows["gdn_prefill_long"] = _row(w, ms, nb, fl, peaks, peak_src, "hbm", w.B * w.L, "gdn_prefill_cluster")
+    row = _row(w, ms, nb, fl, peaks, peak_src, "hbm", w.B * w.L, "gdn_prefill_long")
+    row["path"] = ("vg_prep_kernel (all SMs) + vg_chain_kernel (one CTA per head) in 16 segments of 64 chunks; "
+                   "the prep of segment i+1 overlaps the chain of segment i (two library streams)")
+    rows["gdn_prefill_long"] = row
     # the same workload as a sequence split into 3 segments on this one device: segments 0-1
     # (from s0 / from 0) with segment 1 from lambda I alongside (96 one-CTA sequences, one
     # wave on 148 SMs), the composition, then segments 1-2 again from their incoming states;

@@ -18,16 +18,25 @@
  *
  * Conventions for every entry point
  *  - Ownership: the caller allocates and owns every buffer (device memory unless
- *    stated). The library allocates no memory and keeps no per-call state; its only
- *    state is per device: the condition word that gdn_sync_status reads, cached
- *    kernel attributes, and the wait limit of gdn_set_wait_limit_for_testing.
+ *    stated). Two prefill forms take a stream-ordered workspace from a memory pool the
+ *    library creates per device, and release it on the stream once their kernels have
+ *    run (the pool keeps what it reserved for later calls): vector-valued gates on the
+ *    tensor cores, and Gated DeltaNet over few heads with long sequences (dense bf16
+ *    calls at dk = dv = 128, chunk 64, with at most a third of the SM count of (sequence,
+ *    head) pairs and at least 128 chunks); if that memory cannot be had they run on
+ *    kernels that need none. Otherwise the library allocates no memory and keeps no
+ *    per-call state; its only state is per device: the condition word that
+ *    gdn_sync_status reads, cached kernel attributes, the wait limit of
+ *    gdn_set_wait_limit_for_testing, the workspace pool and the two streams below.
  *  - Layout: dense, contiguous, row-major, as annotated. Device pointers must be
  *    16-byte aligned, except beta and g, which need 4-byte alignment.
  *  - Asynchrony: work is enqueued on `cuda_stream` (a cudaStream_t; NULL = the
  *    legacy default stream) and the call returns without synchronising. The
  *    return value reports argument validation and launch errors only; a kernel
  *    that gave up on a bounded wait records it in a device-side word that
- *    gdn_sync_status() reads.
+ *    gdn_sync_status() reads. The long-sequence form runs its kernels on two streams
+ *    of the library's (after the work already on `cuda_stream`) and makes `cuda_stream`
+ *    wait for the last of them, so later work on `cuda_stream` sees the results.
  *  - Errors: on any non-OK return nothing was enqueued (validation) or the
  *    launch failed (GDN_ERR_CUDA). No exceptions cross this boundary.
  *  - Aliasing: s_final may alias s0. q, k, v, beta, g must not alias o.
@@ -89,7 +98,10 @@ gdn_status_t lin_attn_chunk_fwd(const void *q, const void *k, const void *v, con
  * "HouseHolder变换和WY表示"; page "LinearAttention 概述" section "FLASH".
  *
  *  beta     (B, H, L) fp32, required (the delta term's learning rate)
- *  other arguments as for lin_attn_chunk_fwd.
+ *  other arguments as for lin_attn_chunk_fwd. Few (sequence, head) pairs with long
+ *  sequences (see Ownership above) run as a per-chunk prep kernel on every SM and a
+ *  per-head chain kernel, in segments of 64 chunks whose prep overlaps the chain of the
+ *  segment before; the same result within the tolerance of the tensor-core kernels.
  */
 gdn_status_t gdn_chunk_fwd(const void *q, const void *k, const void *v, const float *beta,
                            const float *g, float *o, const float *s0, float *s_final,

@@ -7,7 +7,8 @@ purpose and nothing hangs: the kernel stops issuing, drains the copies and tenso
 products it has issued, frees its tensor memory and returns; gdn_sync_status reports
 GDN_ERR_TIMEOUT. The next call with the default limit must then be clean and match the
 oracle (the context stays usable). Covers the one-CTA and cluster forms of the Gated
-DeltaNet kernel and the linear-attention kernel.
+DeltaNet kernel, the linear-attention kernel, and the prep and chain kernels (vector-valued
+gates; and a long sequence over few heads, where they run in segments on two streams).
 """
 import pytest
 import torch
@@ -27,9 +28,12 @@ def lib():
     _lib.gdn_set_wait_limit_for_testing(0)
 
 
-# (entry, B, H): 4 x 16 heads take the one-CTA form (3 x 64 CTAs exceed the SM count),
-# 1 x 2 heads the cluster form
-CASES = {"gdn_one_cta": ("gdn", 4, 16), "gdn_cluster": ("gdn", 1, 2), "lin_attn": ("la", 1, 2)}
+# (entry, B, H, L, vector gates): 4 x 16 heads take the one-CTA form (3 x 64 CTAs exceed the
+# SM count), 1 x 2 heads the cluster form; vector gates the prep and chain kernels; 130 chunks
+# over 2 heads the segmented prep and chain kernels
+CASES = {"gdn_one_cta": ("gdn", 4, 16, 200, False), "gdn_cluster": ("gdn", 1, 2, 200, False),
+         "lin_attn": ("la", 1, 2, 200, False), "gdn_vector_gate": ("gdn", 1, 2, 200, True),
+         "gdn_long_segments": ("gdn", 1, 2, 64 * 130, False)}
 
 
 def _run(lib, entry, inp, o, sf):
@@ -42,9 +46,11 @@ def _run(lib, entry, inp, o, sf):
 
 @pytest.mark.parametrize("case", list(CASES))
 def test_wait_gives_up_then_next_call_is_clean(lib, case):
-    entry, B, H = CASES[case]
-    L, d = 200, 128
+    entry, B, H, L, vector = CASES[case]
+    d = 128
     inp = W.make_prefill_inputs(B, H, L, d, d, mode="gdn", in_dtype=torch.bfloat16, seed=606)
+    if vector:
+        inp["g"] = W.make_gate_per_key((B, H), L, d, seed=607)
     o = torch.empty(B, H, L, d, device="cuda")
     sf = torch.empty(B, H, d, d, device="cuda")
     for _ in range(3):                          # nothing pending from earlier tests

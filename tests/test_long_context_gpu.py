@@ -92,3 +92,25 @@ def test_segments_agree_with_the_one_cta_kernel(lib):
     o1, s1 = _run(lib, small, small["g"], True)
     o2, s2 = _run(lib, big, big["g"], True)
     assert _err(o1, o2[:, :3].double().numpy()) <= TOL and _err(s1, s2[:, :3].double().numpy()) <= TOL
+
+
+@pytest.mark.parametrize("L,B,H,with_s0", [(128 * 64, 1, 2, True), (128 * 64 + 1, 2, 3, False),
+                                           (192 * 64 - 5, 1, 4, True)])
+def test_segment_boundaries(lib, L, B, H, with_s0):
+    # exactly two segments; one token past them (a one-token third segment) over two sequences;
+    # a ragged third segment
+    inp = W.make_prefill_inputs(B, H, L, 128, 128, mode="gdn", in_dtype=torch.bfloat16, s0=with_s0,
+                                seed=640 + L % 97)
+    o, sf = _run(lib, inp, inp["g"], True)
+    o_ref, s_ref = oracle.recurrent_fwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["g"], inp["s0"])
+    eo, es = _err(o, o_ref), _err(sf, s_ref)
+    assert eo <= TOL and es <= TOL, f"L={L}: o {eo:.3e}  S {es:.3e}"
+
+
+def test_segmented_vector_gates_without_initial_state(lib):
+    L = 128 * 64 + 33
+    inp = W.make_prefill_inputs(1, 2, L, 128, 128, mode="gdn", in_dtype=torch.bfloat16, s0=False, seed=650)
+    g = W.make_gate_per_key((1, 2), L, 128, seed=651, g_low=-0.3)
+    o, sf = _run(lib, inp, g, True)
+    o_ref, s_ref = oracle.recurrent_fwd(inp["q"], inp["k"], inp["v"], inp["beta"], g, None)
+    assert _err(o, o_ref) <= TOL and _err(sf, s_ref) <= TOL

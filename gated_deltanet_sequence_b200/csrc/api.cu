@@ -12,6 +12,8 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 bool opt_aligned16(const void *p) { return p == nullptr || aligned16(p); }
 bool opt_aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 bool head_dim_ok(int d) { return d == 64 || d == 128; }
+// token rows of a call (the padded copies index them with an int)
+bool rows_fit_int(const int *cu, int B, int H, int L) { return (double)(cu ? 1 : B) * H * L < 1073741824.0; }
 constexpr gdn::FwdOpts kDefaultOut{false, nullptr, false, gdn::kXNormNone, nullptr, 0.f};   // fp32 o, no options
 
 // The output-normalisation fields of the options: a known kind, a positive finite eps
@@ -57,9 +59,82 @@ gdn_status_t launch_tc_vg(bool delta, bool per_key, const void *q, const void *k
                           const float *g, void *o, const float *s0, float *s_final, int B, int H, int L, float scale,
                           FwdOpts oo, cudaStream_t stream, bool *fallback);
 bool tc_vg_takes_scalar(int B, int H, int L);
+// Zero-padded copies for head sizes of 64 (pad.cu): dst[o][r][c] from src with zero fill (or a
+// crop when the source is the larger), rows given in bytes; and the copies' workspace.
+bool pad_copy(void *dst, const void *src, long long n_outer, int rows_dst, int cols_dst_bytes, int rows_src,
+              int cols_src_bytes, cudaStream_t stream);
+bool pad_alloc(void **p, size_t bytes, cudaStream_t stream);
 }  // namespace gdn
 
 extern "C" {
+
+static gdn_status_t prefill_ex(bool delta, const void *q, const void *k, const void *v, const float *beta,
+                               const float *g, void *o, const float *s0, float *s_final, const int *cu_seqlens,
+                               int B, int H, int L, int dk, int dv, int chunk, float scale, gdn_dtype_t in_dtype,
+                               const gdn_fwd_opts_t *opts, void *cuda_stream);
+
+// bf16 calls at chunk 64 with dk or dv = 64 run on the tensor-core kernels through copies padded
+// to 128 (pad.cu); not with the output normalisation, which reduces over the value width
+static bool pad_applies(gdn_dtype_t in_dtype, int dk, int dv, int chunk, int L) {
+    return in_dtype == GDN_BF16 && chunk == 64 && L > 0 && (dk != 128 || dv != 128);
+}
+
+// The padded call: q, k (dk -> 128), v (dv -> 128), a vector gate (dk -> 128, log-decay 0), the
+// skip weights (dv -> 128) and S0 (dk x dv -> 128 x 128) are copied with zero fill into a
+// stream-ordered workspace, the call runs at 128 x 128, and o and S_final are cropped back.
+// Rows of the padded state and output beyond dk / dv stay zero (zero keys and values), so the
+// first dk x dv entries are the results of the unpadded call. *fallback: no workspace.
+static gdn_status_t padded_prefill(bool delta, const void *q, const void *k, const void *v, const float *beta,
+                                   const float *g, void *o, const float *s0, float *s_final, const int *cu_seqlens,
+                                   int B, int H, int L, int dk, int dv, float scale, const gdn::FwdOpts &oo,
+                                   cudaStream_t stream, bool *fallback) {
+    *fallback = false;
+    const long long rows = static_cast<long long>(cu_seqlens ? 1 : B) * H * L;   // token rows
+    const long long nstate = static_cast<long long>(B) * H;
+    const int ob = oo.bf16 ? 2 : 4;
+    const bool vec = oo.gate_per_key;
+    auto up = [](long long x) { return static_cast<size_t>((x + 255) / 256 * 256); };
+    size_t off = 0;
+    const size_t o_q = off; off += up(rows * 256);
+    const size_t o_k = off; off += up(rows * 256);
+    const size_t o_v = off; off += up(rows * 256);
+    const size_t o_o = off; off += up(rows * 128 * ob);
+    const size_t o_g = off; if (vec) off += up(rows * 512);
+    const size_t o_s0 = off; if (s0) off += up(nstate * 65536);
+    const size_t o_sf = off; if (s_final) off += up(nstate * 65536);
+    const size_t o_d = off; if (oo.dskip) off += up(static_cast<long long>(H) * 512);
+    void *ws = nullptr;
+    if (!gdn::pad_alloc(&ws, off, stream)) {
+        *fallback = true;
+        return GDN_ERR_CUDA;
+    }
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    bool ok = gdn::pad_copy(w + o_q, q, 1, static_cast<int>(rows), 256, static_cast<int>(rows), dk * 2, stream) &&
+              gdn::pad_copy(w + o_k, k, 1, static_cast<int>(rows), 256, static_cast<int>(rows), dk * 2, stream) &&
+              gdn::pad_copy(w + o_v, v, 1, static_cast<int>(rows), 256, static_cast<int>(rows), dv * 2, stream);
+    if (vec) ok = ok && gdn::pad_copy(w + o_g, g, 1, static_cast<int>(rows), 512, static_cast<int>(rows), dk * 4, stream);
+    if (s0) ok = ok && gdn::pad_copy(w + o_s0, s0, nstate, 128, 512, dk, dv * 4, stream);
+    if (oo.dskip) ok = ok && gdn::pad_copy(w + o_d, oo.dskip, 1, H, 512, H, dv * 4, stream);
+    gdn_status_t st = GDN_ERR_CUDA;
+    if (ok) {
+        gdn_fwd_opts_t po = {};
+        po.out_dtype = oo.bf16 ? GDN_BF16 : GDN_F32;
+        po.d_skip = oo.dskip ? reinterpret_cast<const float *>(w + o_d) : nullptr;
+        po.g_per_key = vec ? 1 : 0;
+        po.xnorm = GDN_XNORM_NONE;
+        st = prefill_ex(delta, w + o_q, w + o_k, w + o_v, beta, vec ? reinterpret_cast<const float *>(w + o_g) : g,
+                        w + o_o, s0 ? reinterpret_cast<const float *>(w + o_s0) : nullptr,
+                        s_final ? reinterpret_cast<float *>(w + o_sf) : nullptr, cu_seqlens, B, H, L, 128, 128, 64,
+                        scale, GDN_BF16, &po, stream);
+        if (st == GDN_OK) {
+            ok = gdn::pad_copy(o, w + o_o, 1, static_cast<int>(rows), dv * ob, static_cast<int>(rows), 128 * ob, stream);
+            if (s_final) ok = ok && gdn::pad_copy(s_final, w + o_sf, nstate, dk, dv * 4, 128, 512, stream);
+            if (!ok) st = GDN_ERR_CUDA;
+        }
+    }
+    if (cudaFreeAsync(ws, stream) != cudaSuccess && st == GDN_OK) st = GDN_ERR_CUDA;
+    return st;
+}
 
 const char *gdn_status_str(gdn_status_t s) {
     switch (s) {
@@ -81,6 +156,9 @@ gdn_status_t lin_attn_chunk_fwd(const void *q, const void *k, const void *v, con
                                 void *cuda_stream) {
     gdn_status_t st = check_prefill(q, k, v, g, o, s0, s_final, B, H, L, dk, dv, chunk, scale, in_dtype);
     if (st != GDN_OK) return st;
+    if (pad_applies(in_dtype, dk, dv, chunk, L))
+        return prefill_ex(false, q, k, v, nullptr, g, o, s0, s_final, nullptr, B, H, L, dk, dv, chunk, scale, in_dtype,
+                          nullptr, cuda_stream);
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
     if (gdn::tc_supported(in_dtype, dk, dv, chunk) && L > 0)
         return gdn::launch_tc_la(q, k, v, g, o, s0, s_final, nullptr, B, H, L, scale, kDefaultOut, stream);
@@ -96,6 +174,9 @@ gdn_status_t gdn_chunk_fwd(const void *q, const void *k, const void *v, const fl
     if (st != GDN_OK) return st;
     if (L > 0 && !beta) return GDN_ERR_INVALID_ARG;
     if (!opt_aligned4(beta)) return GDN_ERR_INVALID_ARG;
+    if (pad_applies(in_dtype, dk, dv, chunk, L))
+        return prefill_ex(true, q, k, v, beta, g, o, s0, s_final, nullptr, B, H, L, dk, dv, chunk, scale, in_dtype,
+                          nullptr, cuda_stream);
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
     if (gdn::tc_supported(in_dtype, dk, dv, chunk) && L > 0 && gdn::tc_vg_takes_scalar(B, H, L)) {
         // few heads, long sequences: prep on every SM, overlapped with the per-head chain
@@ -120,6 +201,9 @@ gdn_status_t lin_attn_chunk_fwd_varlen(const void *q, const void *k, const void 
     gdn_status_t st = check_prefill(q, k, v, g, o, s0, s_final, 1, H, T, dk, dv, chunk, scale, in_dtype);
     if (st != GDN_OK) return st;
     if ((double)N * H > 2147483647.0) return GDN_ERR_INVALID_ARG;
+    if (pad_applies(in_dtype, dk, dv, chunk, T))
+        return prefill_ex(false, q, k, v, nullptr, g, o, s0, s_final, cu_seqlens, N, H, T, dk, dv, chunk, scale,
+                          in_dtype, nullptr, cuda_stream);
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
     if (gdn::tc_supported(in_dtype, dk, dv, chunk) && T > 0)
         return gdn::launch_tc_la(q, k, v, g, o, s0, s_final, cu_seqlens, N, H, T, scale, kDefaultOut, stream);
@@ -137,6 +221,9 @@ gdn_status_t gdn_chunk_fwd_varlen(const void *q, const void *k, const void *v, c
     if ((double)N * H > 2147483647.0) return GDN_ERR_INVALID_ARG;
     if (T > 0 && !beta) return GDN_ERR_INVALID_ARG;
     if (!opt_aligned4(beta)) return GDN_ERR_INVALID_ARG;
+    if (pad_applies(in_dtype, dk, dv, chunk, T))
+        return prefill_ex(true, q, k, v, beta, g, o, s0, s_final, cu_seqlens, N, H, T, dk, dv, chunk, scale,
+                          in_dtype, nullptr, cuda_stream);
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
     if (gdn::tc_supported(in_dtype, dk, dv, chunk) && T > 0)
         return gdn::launch_tc_gdn(q, k, v, beta, g, o, s0, s_final, cu_seqlens, N, H, T, scale, kDefaultOut, stream);
@@ -170,6 +257,12 @@ static gdn_status_t prefill_ex(bool delta, const void *q, const void *k, const v
     if (!opt_aligned4(beta)) return GDN_ERR_INVALID_ARG;
     if ((double)B * H * (double)L * dk > 9.0e18) return GDN_ERR_INVALID_ARG;   // g of (rows, dk)
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+    if (pad_applies(in_dtype, dk, dv, chunk, L) && oo.xnorm == gdn::kXNormNone && rows_fit_int(cu_seqlens, B, H, L)) {
+        bool fallback = false;
+        const gdn_status_t ps = padded_prefill(delta, q, k, v, beta, g, o, s0, s_final, cu_seqlens, B, H, L, dk, dv,
+                                               scale, oo, stream, &fallback);
+        if (!fallback) return ps;
+    }
     // vector-valued gates: the two tensor-core kernels for dense bf16 batches at dk = dv = 128,
     // C = 64; the fp32 chunk kernel for every other input dtype, size and layout
     if (gdn::tc_supported(in_dtype, dk, dv, chunk) && L > 0 && oo.gate_per_key && !cu_seqlens) {

@@ -18,13 +18,13 @@
  *
  * Conventions for every entry point
  *  - Ownership: the caller allocates and owns every buffer (device memory unless
- *    stated). Two prefill forms take a stream-ordered workspace from a memory pool the
+ *    stated). Three prefill forms take a stream-ordered workspace from a memory pool the
  *    library creates per device, and release it on the stream once their kernels have
  *    run (the pool keeps what it reserved for later calls): vector-valued gates on the
- *    tensor cores, and Gated DeltaNet over few heads with long sequences (dense bf16
- *    calls at dk = dv = 128, chunk 64, with at most a third of the SM count of (sequence,
- *    head) pairs and at least 128 chunks); if that memory cannot be had they run on
- *    kernels that need none. Otherwise the library allocates no memory and keeps no
+ *    tensor cores, Gated DeltaNet over few heads with long sequences (dense bf16 calls at
+ *    dk = dv = 128, chunk 64, with at most a third of the SM count of (sequence, head)
+ *    pairs and at least 128 chunks), and bf16 calls with dk or dv = 64 (zero-padded
+ *    copies); if that memory cannot be had they run on kernels that need none. Otherwise the library allocates no memory and keeps no
  *    per-call state; its only state is per device: the condition word that
  *    gdn_sync_status reads, cached kernel attributes, the wait limit of
  *    gdn_set_wait_limit_for_testing, the workspace pool and the two streams below.
@@ -77,9 +77,13 @@ typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype_t;
  *  s0       (B, H, dk, dv) fp32 initial state, nullable (zero state)
  *  s_final  (B, H, dk, dv) fp32 final state,   nullable (not written)
  *  B, H >= 1; L >= 0 (L == 0: only s_final is written, = s0 or 0)
- *  dk, dv in {64, 128}; chunk: 1..64. bf16 inputs with dk = dv = 128 and chunk 64 run on
- *  the tensor-core kernels; every other combination runs on the fp32 chunk kernel (the
- *  same result within its tolerance, at CUDA-core speed).
+ *  dk, dv in {64, 128}; chunk: 1..64. bf16 inputs with chunk 64 run on the tensor-core
+ *  kernels: at dk = dv = 128 directly, with dk or dv = 64 through copies of the operands
+ *  zero-padded to 128 (the padded results, cropped, are the call's: zero key coordinates
+ *  and value columns leave the other entries unchanged; a stream-ordered workspace from the
+ *  library's pool, see Ownership; not with the output normalisation). Every other
+ *  combination runs on the fp32 chunk kernel (the same result within its tolerance, at
+ *  CUDA-core speed).
  *  scale multiplies q.  in_dtype: GDN_BF16 or GDN_F32 (q, k, v share it).
  */
 gdn_status_t lin_attn_chunk_fwd(const void *q, const void *k, const void *v, const float *g,

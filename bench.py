@@ -359,6 +359,22 @@ def measure_rows(gdn, peaks, peak_src, args):
     row = _row(w, ms, nb, fl, peaks, peak_src, "hbm", w.B * w.L)
     row["path"] = "tensor cores: vg_prep_kernel (one CTA per chunk) + vg_chain_kernel (one CTA per head)"
     rows["gdn_prefill_vector_gate"] = row
+    # the same shape at head size 64 (dk = dv = 64): the tensor-core kernels through copies
+    # zero-padded to 128 (bytes and FLOP counted at d = 64, the call's own work)
+    inp64 = W.make_prefill_inputs(w.B, w.H, w.L, 64, 64, mode="gdn", in_dtype=torch.bfloat16,
+                                  seed=W.SEED_BASE + 8, device="cuda")
+    o64 = torch.empty(w.B, w.H, w.L, 64, device="cuda")
+    sf64 = torch.empty(w.B, w.H, 64, 64, device="cuda")
+    fn = lambda: gdn.gdn_chunk_fwd(inp64["q"], inp64["k"], inp64["v"], inp64["beta"], inp64["g"], o=o64,
+                                   s_final=sf64, chunk=w.chunk)
+    ms = timed(fn, max(5, args.steps), 3)
+    nb64 = prefill_bytes(w.B, w.H, w.L, 64, 64, 2, True, True, False, True)
+    fl64 = flops_per_head_token("gdn", 64, 64, w.chunk) * w.B * w.H * w.L
+    row = _row(w, ms, nb64, fl64, peaks, peak_src, "hbm", w.B * w.L)
+    row["workload"] = "gdn_bf16_B8_H16_L4096_d64"
+    row["path"] = "tc_gdn_kernel at 128 x 128 on zero-padded copies, cropped (pad_copy_kernel)"
+    rows["gdn_prefill_d64"] = row
+    del inp64, o64, sf64
     del inp, o, sf, gv
     # backward pass (gradients of the prefill) on the headline shape: fp32 CUDA-core kernel whose
     # per-token state traffic goes through the caller's workspace (checkpoints + chunk slab)

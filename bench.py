@@ -356,7 +356,7 @@ def measure_rows(gdn, peaks, peak_src, args):
     fn = lambda: gdn.gdn_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["beta"], gv, o=o, s_final=sf, chunk=w.chunk)
     ms = timed(fn, max(5, args.steps), 3)
     nb = prefill_bytes(w.B, w.H, w.L, w.dk, w.dv, 2, True, False, False, True) + w.B * w.H * w.L * w.dk * 4
-    row = _row(w, ms, nb, fl, peaks, peak_src, "hbm", w.B * w.L)
+    row = _row(w, ms, nb, fl, peaks, peak_src, "hbm", w.B * w.L, "gdn_prefill_vector_gate")
     row["path"] = "tensor cores: vg_prep_kernel (one CTA per chunk) + vg_chain_kernel (one CTA per head)"
     rows["gdn_prefill_vector_gate"] = row
     # the same shape at head size 64 (dk = dv = 64): the tensor-core kernels through copies

@@ -566,8 +566,9 @@ def run_reference(args, rank, world):
 def run_profile(spec: str):
     """Run one kernel a few times on one case (for an ncu capture; prints nothing timed).
     spec: gdn[:B] (GDN bf16, B x 16 x 4096 x 128), la[:B] (plain LA, B x 16 x 4096 x 128),
-    decode[:N] (N x 32 heads, 3 steps), gdn_long (1 x 32 x 65536), gdnh[:H[:L]] (1 x H x L,
-    the cluster form when 3 H fits the SM count), gdnvec[:B[:L]] (vector-valued gates, B x 16 x L,
+    decode[:N] (N x 32 heads, 3 steps), gdn_long (1 x 32 x 65536), gdnh[:H[:L]] (1 x H x L, S0 != 0:
+    with 3 H within the SM count, the segmented prep + chain kernels from 128 chunks on, the
+    cluster form below that), gdnvec[:B[:L]] (vector-valued gates, B x 16 x L,
     bf16: the prep and chain kernels), gdnvec32[:B[:L]] (the same in fp32: the fp32 chunk kernel)."""
     from gated_deltanet_sequence_b200 import _lib as gdn
     kind, _, arg = spec.partition(":")
@@ -585,7 +586,8 @@ def run_profile(spec: str):
             else:
                 gdn.lin_attn_chunk_fwd(inp["q"], inp["k"], inp["v"], None, o=o, s_final=sf)
     elif kind == "gdnh":
-        # B=1, H heads of L tokens (few heads: the cluster form), S0 != 0
+        # B=1, H heads of L tokens, S0 != 0 (few heads: the segmented form, or the cluster form
+        # below 128 chunks)
         H, _, L = arg.partition(":")
         H, L = int(H or 32), int(L or 8192)
         inp = W.make_prefill_inputs(1, H, L, 128, 128, mode="gdn", in_dtype=torch.bfloat16, s0=True,

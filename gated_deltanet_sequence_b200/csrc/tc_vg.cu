@@ -633,7 +633,8 @@ vg_prep_kernel(const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__
 // O^T += Ut^T P^T. Only the record tiles (the B operands) are read from shared memory; at N = 128
 // a UMMA with both operands in shared memory reads about as many bytes per cycle as shared
 // memory delivers, so every other access there slowed the chain.
-constexpr int kVCThreads = 320;   // record-load warp, an idle warp, 8 state warps (two per TMEM lane quarter)
+constexpr int kVCThreads = 448;   // record-load warp, an idle warp, 8 state warps (two per TMEM lane quarter),
+                                  // 4 output warps
 constexpr int kVCStages = 3;      // records in flight: one SM's bulk loads take about a chunk's time each
 constexpr uint32_t VC_EGL = kVCStages * kRecBytes;   // exp(GL) of each stage's chunk (128 fp32 each)
 constexpr uint32_t VC_XN = VC_EGL + 512 * kVCStages;  // output-normalisation scratch (384 fp32)
@@ -649,13 +650,15 @@ constexpr uint32_t ID_SQ = idesc_f16(128, 64, false, true);    // O^T += S^T Q'^
 constexpr uint32_t ID_ST = idesc_f16(128, 128, false, false);  // S^T += Ut^T Kd
 constexpr uint32_t ID_O = idesc_f16(128, 64, false, false);    // O^T += Ut^T P^T
 constexpr int kBarS = 1;   // the 8 state warps
-constexpr int kBarO = 2;   // the 4 state warps that store the output (half 0)
+constexpr int kBarO = 2;   // the 4 output warps
 constexpr int kBarU = 3;   // the 4 state warps of the Ut epilogue (half 1)
+constexpr int kBarH = 4;   // the 4 state warps that write back the decayed half of S^T first (half 0)
 // mbarriers: FULL / ODONE per record stage (chunk c takes stage c % 3; ODONE also marks its
 // output tile, parity c & 1, complete); ADONE: the [O^T | Ut^T] product is done; DEC: half 0
 // has written its decayed half of S^T; SDONE: the state update of the last chunk is done (the
-// next chunk may read S, and every UMMA lead1 issued before it is complete)
-enum : int { CB_FULL = 0, CB_ODONE = 3, CB_ADONE = 6, CB_DEC = 7, CB_SDONE = 8, kVCBars = 9 };
+// next chunk may read S, and every UMMA lead1 issued before it is complete); OFREE per output
+// tile: the output warps have read it (the product of chunk c + 2 may write it)
+enum : int { CB_FULL = 0, CB_ODONE = 3, CB_ADONE = 6, CB_DEC = 7, CB_SDONE = 8, CB_OFREE = 9, kVCBars = 11 };
 
 template <bool DELTA, bool OPTS>
 __global__ void __launch_bounds__(kVCThreads, 1)
@@ -711,20 +714,19 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
             for (int st = 0; st < kVCStages; ++st)
                 if (last[st] >= 0) ctl.drain(CB_FULL + st, (last[st] / kVCStages) & 1);
         }
-    } else if (warp >= 2) {
+    } else if (warp >= 2 && warp < 10) {
         // ================================================================ state group (warps 2-9)
         // thread (v, half): TMEM lane v (value column v of S^T, O and Ut). Both halves copy
-        // S^T (key columns 64 * half ..); then half 0 stores the previous chunk's output while
-        // half 1 takes the Ut epilogue of this chunk, so the output stores stay off the chain.
-        // The group issues the chain's UMMAs itself: thread `lead` the [O^T | Ut^T] product once
-        // the fp16 copy of S^T is complete, thread `lead1` the state update and the output
-        // product once the fp16 copy of Ut^T is complete.
+        // S^T (key columns 64 * half ..) and write back its decayed half; half 1 then takes the
+        // Ut epilogue of this chunk. The output warps store the output tiles, so the chain
+        // carries no output stores. The group issues the chain's UMMAs itself: thread `lead`
+        // the [O^T | Ut^T] product once the fp16 copy of S^T is complete (and the output tile
+        // it writes has been read), thread `lead1` the state update and the output product once
+        // the fp16 copy of Ut^T is complete.
         const int half = (warp - 2) >> 2;
         const int v = (warp & 3) * 32 + lane;
         const bool lead = (v == 0 && half == 0);    // polls for the whole group and for half 0
         const bool lead1 = (v == 0 && half == 1);   // polls for half 1
-        const int head = bh % H;
-        float *xn = reinterpret_cast<float *>(smem + VC_XN);
         const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
         {
             // S^T[v][j] = S0[j][v] for this thread's 64 key rows j (a warp reads 128 bytes per j)
@@ -739,7 +741,6 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
             }
             tmem_wait_st();
         }
-        int done = 0;
         int issued_a = -1, issued_o = -1;   // last chunk whose products lead / lead1 committed
         float nf = 0.f;
         bool stop = false;   // this half gave up waiting; the group stops at its next meeting
@@ -748,11 +749,13 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
             const int s = c & 1, st = c % kVCStages;
             const uint8_t *stg = smem + st * kRecBytes;
             const uint32_t stg_a = sb + st * kRecBytes;
-            // S(c) complete (state update of c-1 done) and this chunk's record landed
+            // S(c) complete (state update of c-1 done), this chunk's record landed and the output
+            // tile of chunk c - 2 read (this chunk's product writes it)
             {
                 bool fail = stop;
                 if (lead && !fail) fail = (c >= 1 && !ctl.wait(CB_SDONE, static_cast<uint32_t>(c - 1) & 1u)) ||
-                                          !ctl.wait(CB_FULL + st, static_cast<uint32_t>(c / kVCStages) & 1u);
+                                          !ctl.wait(CB_FULL + st, static_cast<uint32_t>(c / kVCStages) & 1u) ||
+                                          (c >= 2 && !ctl.wait(CB_OFREE + s, static_cast<uint32_t>((c - 2) >> 1) & 1u));
                 if (named_bar_any(kBarS, 256, fail)) break;
             }
             tc_fence_after();
@@ -809,21 +812,8 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
             if (half == 0) {
                 // the decayed half of S^T is in place: hand it to the state update
                 tc_fence_before();
-                named_bar(kBarO, 128);
+                named_bar(kBarH, 128);
                 if (lead) mbar_arrive(&bars[CB_DEC]);
-                // ---- output of the previous chunk, once its O tile is complete
-                if (c >= 1) {
-                    const int cp = c - 1;
-                    if (!ctl.group_wait(CB_ODONE + cp % kVCStages, (cp / kVCStages) & 1, kBarO, lead, 128)) {
-                        stop = true;
-                        continue;
-                    }
-                    tc_fence_after();
-                    store_out_col<OPTS>(trow + TMC_OU + (cp & 1) * 128, out,
-                                        (row0 + static_cast<size_t>(cp) * kC) * kD + v, kC, head, v, kBarO, xn, false,
-                                        nf);
-                    done = c;
-                }
             } else {
                 // ---- Ut^T row v -> fp16 pairs over its first 32 columns (A operand of the
                 //      state update and of the output product)
@@ -897,19 +887,11 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
         // UMMAs complete in issue order: each issuing thread waits for its last commit
         if (lead && issued_a >= 0) ctl.drain(CB_ADONE, static_cast<uint32_t>(issued_a) & 1u);
         if (lead1 && issued_o >= 0) ctl.drain(CB_ODONE + issued_o % kVCStages, (issued_o / kVCStages) & 1);
-        // ---- last output tile (half 0) and the final state (both halves)
+        // ---- the final state (both halves)
         const int cp = nch - 1;
-        if (half == 0 && !stop && nch > 0 && done == cp) {
-            if (ctl.group_wait(CB_ODONE + cp % kVCStages, (cp / kVCStages) & 1, kBarO, lead, 128)) {
-                tc_fence_after();
-                store_out_col<OPTS>(trow + TMC_OU + (cp & 1) * 128, out, (row0 + static_cast<size_t>(cp) * kC) * kD + v,
-                                    min(kC, Lrem - cp * kC), head, v, kBarO, xn, seq_end, nf);
-                done = nch;
-            }
-        }
         {
-            // the final state once the last update is done, if every output tile was stored
-            bool fail = half == 0 && done != nch;
+            // the final state once the last update is done, unless the group stopped
+            bool fail = stop;
             if (lead && !fail && nch > 0) fail = !ctl.wait(CB_SDONE, static_cast<uint32_t>(cp) & 1u);
             if (!named_bar_any(kBarS, 256, fail || !s_final || nch == 0)) {
                 tc_fence_after();
@@ -925,6 +907,39 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
                         dst[static_cast<size_t>(cc * 16 + e) * kD] = t[e];
                     }
                 }
+            }
+        }
+        report_nonfinite(ctl.aborted() ? 0.f : nf, err_word);
+    } else if (warp >= 10) {
+        // ================================================================ output warps (10-13)
+        // thread v: TMEM lane v. Each chunk's output tile, once complete, is read, handed back
+        // (OFREE) and stored; the last tile holds the sequence's ragged tail.
+        const int v = (warp & 3) * 32 + lane;
+        const bool olead = v == 0;
+        const int head = bh % H;
+        float *xn = reinterpret_cast<float *>(smem + VC_XN);
+        const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+        float nf = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < nch; ++c) {
+            if (!ctl.group_wait(CB_ODONE + c % kVCStages, (c / kVCStages) & 1, kBarO, olead, 128)) break;
+            tc_fence_after();
+            float ov[64];
+            ld_cols<64>(trow + TMC_OU + (c & 1) * 128, ov);
+            tc_fence_before();
+            named_bar(kBarO, 128);
+            if (olead) mbar_arrive(&bars[CB_OFREE + (c & 1)]);
+            const bool last = c == nch - 1;
+            const int n = last ? min(kC, Lrem - c * kC) : kC;
+            const size_t elem0 = (row0 + static_cast<size_t>(c) * kC) * kD + v;
+            if constexpr (OPTS) {
+                store_out_rows_group(ov, out, elem0, n, head, v, kBarO, xn, xn + 256, last && seq_end, nf);
+            } else {
+                float *ocol = static_cast<float *>(out.o) + elem0;
+#pragma unroll
+                for (int r = 0; r < 64; ++r)
+                    if (r < n) ocol[static_cast<size_t>(r) * kD] = ov[r];
+                if (last && seq_end) probe_tile(nf, ov, n);
             }
         }
         report_nonfinite(ctl.aborted() ? 0.f : nf, err_word);

@@ -126,6 +126,31 @@ enum : int {
     kNumBars = 20
 };
 
+// Packed batches of at most this many sequences start their longest sequences first.
+constexpr int kLongestFirstMax = 256;
+
+// Block bid of a packed batch of nseq sequences -> state index n * H + h of the (sequence,
+// head) pair it takes: blocks r * H .. r * H + H - 1 take the sequence of rank r by length
+// (longest first, ties by index). Blocks start in index order as SMs free up, so the longest
+// sequences start first and the call ends about when its longest sequence does. A malformed
+// offset array still gives a permutation (the chosen sequence's offsets are checked after).
+__device__ __forceinline__ int longest_first(const int *__restrict__ cu, int bid, int H, int nseq) {
+    __shared__ int len[kLongestFirstMax];
+    __shared__ int pick;
+    if (nseq > kLongestFirstMax) return bid;
+    const int r = bid / H, h = bid - r * H;
+    for (int i = threadIdx.x; i < nseq; i += blockDim.x) len[i] = cu[i + 1] - cu[i];
+    __syncthreads();
+    for (int i = threadIdx.x; i < nseq; i += blockDim.x) {
+        const int li = len[i];
+        int rank = 0;
+        for (int k = 0; k < nseq; ++k) rank += (len[k] > li || (len[k] == li && k < i)) ? 1 : 0;
+        if (rank == r) pick = i;
+    }
+    __syncthreads();
+    return pick * H + h;
+}
+
 template <bool GATED, bool OPTS>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -144,7 +169,8 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const Ctl ctl{bars, abort_flag, err_word, wait_limit};
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int bh = blockIdx.x;                          // (sequence, head): state index
+    // (sequence, head): state index; packed batches take their sequences longest first
+    const int bh = cu ? longest_first(cu, blockIdx.x, H, gridDim.x / H) : blockIdx.x;
     const SeqSpan sp = seq_span(cu, bh, H, Lrow, err_word);
     const int L = sp.len;                               // tokens of this sequence
     const int zc = sp.head_row, ty0 = sp.t0;            // TMA head and first-token coordinates

@@ -156,8 +156,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ beta,
               const float *__restrict__ g, const OutArgs out, const float *__restrict__ s0,
-              float *__restrict__ s_final, const int *__restrict__ cu, int H, int Lrow, float scale,
-              long long wait_limit, unsigned *__restrict__ err_word) {
+              float *__restrict__ s_final, const int *__restrict__ cu, int H, int Lrow, float scale, int dk_in,
+              int dv_in, long long wait_limit, unsigned *__restrict__ err_word) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned base derived by pointer arithmetic on the shared array, so the
     // compiler keeps every access below in the shared address space (LDS/STS)
@@ -313,14 +313,15 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         float *xn = reinterpret_cast<float *>(smem + OFF_XN);
         const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
         {
-            const float *src = s0 ? s0 + (static_cast<size_t>(bh) * kD + j) * kD : nullptr;
+            // row j of S0 (dk_in x dv_in; rows and columns beyond them are zero)
+            const float *src = s0 && j < dk_in ? s0 + (static_cast<size_t>(bh) * dk_in + j) * dv_in : nullptr;
 #pragma unroll 1
             for (int cc = 0; cc < 8; ++cc) {
                 float r[16];
 #pragma unroll
                 for (int e = 0; e < 16; e += 4) {
-                    const float4 x = src ? *reinterpret_cast<const float4 *>(src + cc * 16 + e)
-                                         : make_float4(0.f, 0.f, 0.f, 0.f);
+                    const float4 x = src && cc * 16 < dv_in ? *reinterpret_cast<const float4 *>(src + cc * 16 + e)
+                                                            : make_float4(0.f, 0.f, 0.f, 0.f);
                     r[e] = x.x; r[e + 1] = x.y; r[e + 2] = x.z; r[e + 3] = x.w;
                 }
                 tmem_st16(trow + TM_S + cc * 16, r);
@@ -335,6 +336,23 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
         int done = 0;   // chunks whose output tile has been stored
         float nf = 0.f;  // non-finite probe over sampled output tiles and the final state
+        // output tile of chunk cp (n rows): the general epilogue (dv = 128) with the output
+        // options, else fp32 rows of dv_in columns (lanes j >= dv_in are whole warps: no store)
+        auto store_tile = [&](int cp, int n, bool probe) {
+            const uint32_t taddr = trow + TM_OU + (cp & 1) * 128;
+            if constexpr (OPTS) {
+                store_out_col<OPTS>(taddr, out, (row0 + static_cast<size_t>(cp) * kC) * kD + j, n, head, j, kBarS, xn,
+                                    probe, nf);
+            } else if (j < dv_in) {
+                float ov[64];
+                ld_cols<64>(taddr, ov);
+                float *ocol = static_cast<float *>(out.o) + (row0 + static_cast<size_t>(cp) * kC) * dv_in + j;
+#pragma unroll
+                for (int r = 0; r < 64; ++r)
+                    if (r < n) ocol[static_cast<size_t>(r) * dv_in] = ov[r];
+                if (probe) probe_tile(nf, ov, n);
+            }
+        };
 #pragma unroll 1
         for (int c = 0; c < nchunks; ++c) {
             const int s = c & 1;
@@ -408,8 +426,7 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             // ---- output of the previous chunk (its O tile is complete)
             if (c >= 1) {
                 const int cp = c - 1;
-                store_out_col<OPTS>(trow + TM_OU + (cp & 1) * 128, out, (row0 + static_cast<size_t>(cp) * kC) * kD + j, kC, head, j, kBarS, xn,
-                                    false, nf);   // the last tile is stored (and probed) after the loop
+                store_tile(cp, kC, false);   // the last tile is stored (and probed) after the loop
                 // chunk c + 1 accumulates onto this tile: zero it (ordered before that chunk's
                 // product by this group's state-ready hand-off)
                 float z[16];
@@ -440,15 +457,15 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             const int cp = nchunks - 1;
             if (ctl.group_wait(B_CDONE + (cp & 1), (cp >> 1) & 1, kBarS, lead)) {
                 tc_fence_after();
-                store_out_col<OPTS>(trow + TM_OU + (cp & 1) * 128, out, (row0 + static_cast<size_t>(cp) * kC) * kD + j,
-                              L - cp * kC, head, j, kBarS, xn, true, nf);
+                store_tile(cp, L - cp * kC, true);
                 done = nchunks;
             }
         }
-        if (s_final && done == nchunks) {
-            float *dst = s_final + (static_cast<size_t>(bh) * kD + j) * kD;
+        if (s_final && done == nchunks && j < dk_in) {
+            // row j of the dk_in x dv_in final state (lanes j >= dk_in are whole warps)
+            float *dst = s_final + (static_cast<size_t>(bh) * dk_in + j) * dv_in;
 #pragma unroll 1
-            for (int cc = 0; cc < 8; ++cc) {
+            for (int cc = 0; cc < dv_in / 16; ++cc) {
                 float sv[16];
                 tmem_ld16(trow + TM_S + cc * 16, sv);
                 tmem_wait_ld();
@@ -803,29 +820,36 @@ EncodeTiledFn encode_fn() {
 }
 
 // (BH, L, 128) bf16 -> 3-D map, 64 x 64 boxes, 128-byte swizzle, zero fill out of range.
-bool make_qkv_map(CUtensorMap *m, const void *ptr, int L, int BH) {
+namespace {
+// (BH, L, width) bf16 rows, width 64 or 128, in 64 x 64 boxes: a box past the width (x = 64 of a
+// 64-wide tensor) loads as zeros
+bool make_rows_map(CUtensorMap *m, const void *ptr, int L, int BH, int width) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
-    const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(BH)};
-    const cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(L) * 256};
+    const cuuint64_t row_bytes = static_cast<cuuint64_t>(width) * 2;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(width), static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(BH)};
+    const cuuint64_t strides[2] = {row_bytes, static_cast<cuuint64_t>(L) * row_bytes};
     const cuuint32_t box[3] = {64, 64, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+}  // namespace
+
+bool make_qkv_map(CUtensorMap *m, const void *ptr, int L, int BH) { return make_rows_map(m, ptr, L, BH, 128); }
 
 namespace {
 
 template <bool GATED, bool OPTS>
 gdn_status_t launch_gdn_t(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const float *beta,
                           const float *g, const OutArgs &out, const float *s0, float *s_final, const int *cu,
-                          int nctas, int H, int L, float scale, cudaStream_t stream) {
+                          int nctas, int H, int L, float scale, cudaStream_t stream, int dk = kD, int dv = kD) {
     auto kern = tc_gdn_kernel<GATED, OPTS>;
     if (!ensure_smem_limit(reinterpret_cast<const void *>(kern), kSmemAlloc)) return GDN_ERR_CUDA;
     unsigned *err = device_error_word();
     if (!err) return GDN_ERR_CUDA;
-    kern<<<nctas, kThreads, kSmemAlloc, stream>>>(mq, mk, mv, beta, g, out, s0, s_final, cu, H, L, scale,
+    kern<<<nctas, kThreads, kSmemAlloc, stream>>>(mq, mk, mv, beta, g, out, s0, s_final, cu, H, L, scale, dk, dv,
                                                   wait_limit_cycles(), err);
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
@@ -853,6 +877,23 @@ gdn_status_t launch_tc_gdn(const void *q, const void *k, const void *v, const fl
                        : launch_gdn_t<true, false>(mq, mk, mv, beta, g, out, s0, s_final, cu, nctas, H, L, scale, stream);
     return opts ? launch_gdn_t<false, true>(mq, mk, mv, beta, g, out, s0, s_final, cu, nctas, H, L, scale, stream)
                 : launch_gdn_t<false, false>(mq, mk, mv, beta, g, out, s0, s_final, cu, nctas, H, L, scale, stream);
+}
+
+bool tc_gdn_takes_narrow(int nctas) { return encode_fn() != nullptr && nctas > 0 && !tc_gdn_cluster_fits(nctas); }
+
+gdn_status_t launch_tc_gdn_narrow(const void *q, const void *k, const void *v, const float *beta, const float *g,
+                                  float *o, const float *s0, float *s_final, const int *cu, int B, int H, int L,
+                                  int dk, int dv, float scale, cudaStream_t stream) {
+    const int nctas = B * H;
+    const int rows = cu ? H : B * H;
+    const FwdOpts plain{false, nullptr, false, kXNormNone, nullptr, 0.f};
+    const OutArgs out = make_out_args(o, v, plain);
+    CUtensorMap mq, mk, mv;
+    if (!make_rows_map(&mq, q, L, rows, dk) || !make_rows_map(&mk, k, L, rows, dk) ||
+        !make_rows_map(&mv, v, L, rows, dv))
+        return GDN_ERR_CUDA;
+    return g ? launch_gdn_t<true, false>(mq, mk, mv, beta, g, out, s0, s_final, cu, nctas, H, L, scale, stream, dk, dv)
+             : launch_gdn_t<false, false>(mq, mk, mv, beta, g, out, s0, s_final, cu, nctas, H, L, scale, stream, dk, dv);
 }
 
 }  // namespace gdn

@@ -2,10 +2,14 @@
 oracle, through the C ABI. Such calls run on the tensor-core kernels through copies of the
 operands zero-padded to 128: zero key coordinates and zero value columns change no product the
 first dk x dv entries depend on, so the padded call's output and final state, cropped, are the
-results of the call. Cases: Gated DeltaNet and linear attention at 64 x 64, 64 x 128 and
+results of the call. Gated DeltaNet with the plain fp32 output and a scalar gate, on batches of
+enough (sequence, head) pairs for the one-CTA kernel, skips the copies: that kernel reads the
+64-wide tiles directly and stores only dk x dv states and dv output columns, and must give the
+padded call's bits. Cases: Gated DeltaNet and linear attention at 64 x 64, 64 x 128 and
 128 x 64, with and without S0, ragged and one-token lengths; the packed layout; vector-valued
 gates; bf16 output with the skip term; S_final written in place over S0; the output
-normalisation (which runs on the fp32 chunk kernel). Bound 2e-3 (bf16 output: + 2^-8)."""
+normalisation (which runs on the fp32 chunk kernel); the direct form against the oracle and
+against the padded form, packed, and at the benchmark's size. Bound 2e-3 (bf16 output: + 2^-8)."""
 import pytest
 import torch
 
@@ -98,3 +102,59 @@ def test_output_normalisation_at_dv64(lib):
     assert lib.gdn_sync_status() == 0
     o_plain, _ = oracle.recurrent_fwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["g"], inp["s0"])
     assert _err(o.cpu(), oracle.xnorm(o_plain, "rms")) <= TOL
+
+
+# ---- the direct (copy-free) form: Gated DeltaNet, fp32 output, at least 50 (sequence, head) pairs
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (64, 128), (128, 64)])
+@pytest.mark.parametrize("L,with_s0,gated", [(130, True, True), (1, True, True), (257, False, False)])
+def test_direct_head_sizes(lib, dk, dv, L, with_s0, gated):
+    B, H = 4, 16
+    inp = W.make_prefill_inputs(B, H, L, dk, dv, mode="gdn", in_dtype=torch.bfloat16, s0=with_s0,
+                                seed=860 + L + dk + dv)
+    g = inp["g"] if gated else None
+    q, k, v, beta = (inp[n].cuda() for n in ("q", "k", "v", "beta"))
+    s0 = inp["s0"].cuda() if with_s0 else None
+    sf = torch.full((B, H, dk, dv), float("nan"), device="cuda")
+    o, sf = lib.gdn_chunk_fwd(q, k, v, beta, None if g is None else g.cuda(), s0=s0, s_final=sf, scale=0.9)
+    # the padded form of the same call (a zero skip term adds nothing but takes the copies)
+    zero = torch.zeros(H, dv, device="cuda")
+    sfp = torch.full((B, H, dk, dv), float("nan"), device="cuda")
+    op, sfp = lib.gdn_chunk_fwd(q, k, v, beta, None if g is None else g.cuda(), s0=s0, s_final=sfp, scale=0.9,
+                                d_skip=zero)
+    assert lib.gdn_sync_status() == 0
+    assert torch.equal(o, op) and torch.equal(sf, sfp), "direct and padded forms differ"
+    o_ref, s_ref = oracle.recurrent_fwd(inp["q"], inp["k"], inp["v"], inp["beta"], g, inp["s0"], scale=0.9)
+    assert _err(o.cpu(), o_ref) <= TOL and _err(sf.cpu(), s_ref) <= TOL
+
+
+def test_direct_packed_batch(lib):
+    lens = [0, 1, 64, 65, 130, 300, 7, 191]
+    H = 8
+    inp = W.make_varlen_inputs(lens, H, 64, 64, mode="gdn", in_dtype=torch.bfloat16, s0=True, seed=870)
+    dev = {n: inp[n].cuda() for n in ("q", "k", "v", "beta", "g", "s0", "cu_seqlens")}
+    sf = torch.full((len(lens), H, 64, 64), float("nan"), device="cuda")
+    o, sf = lib.gdn_chunk_fwd_varlen(dev["q"], dev["k"], dev["v"], dev["beta"], dev["cu_seqlens"], dev["g"],
+                                     s0=dev["s0"], s_final=sf)
+    assert lib.gdn_sync_status() == 0
+    o_ref, s_ref = oracle.recurrent_fwd_varlen(inp["q"], inp["k"], inp["v"], inp["cu_seqlens"], beta=inp["beta"],
+                                               g=inp["g"], s0=inp["s0"])
+    assert _err(o.cpu(), o_ref) <= TOL and _err(sf.cpu(), s_ref) <= TOL
+
+
+def test_direct_full_size_sampled_heads(lib):
+    # the benchmark's head-size-64 row: 8 x 16 heads x 4096 tokens, compared on four heads
+    B, H, L = 8, 16, 4096
+    inp = W.make_prefill_inputs(B, H, L, 64, 64, mode="gdn", in_dtype=torch.bfloat16, seed=W.SEED_BASE + 8)
+    dev = {n: inp[n].cuda() for n in ("q", "k", "v", "beta", "g")}
+    o = torch.empty(B, H, L, 64, device="cuda")
+    sf = torch.empty(B, H, 64, 64, device="cuda")
+    lib.gdn_chunk_fwd(dev["q"], dev["k"], dev["v"], dev["beta"], dev["g"], o=o, s_final=sf)
+    assert lib.gdn_sync_status() == 0
+    o, sf = o.cpu(), sf.cpu()
+    for b, h in [(0, 0), (2, 9), (5, 3), (7, 15)]:
+        sl = lambda x: x[b:b + 1, h:h + 1]
+        o_ref, s_ref = oracle.recurrent_fwd(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]), sl(inp["beta"]), sl(inp["g"]))
+        assert _err(sl(o), o_ref) <= TOL, f"o head ({b},{h})"
+        assert _err(sl(sf), s_ref) <= TOL, f"S head ({b},{h})"

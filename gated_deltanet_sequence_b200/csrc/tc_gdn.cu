@@ -151,13 +151,17 @@ __device__ __forceinline__ int longest_first(const int *__restrict__ cu, int bid
     return pick * H + h;
 }
 
-template <bool GATED, bool OPTS>
+// NARROW: head sizes dk_in, dv_in of 64 or 128 (tiles past them load as zeros; plain fp32
+// output only); otherwise both are 128 and the arguments are ignored.
+template <bool GATED, bool OPTS, bool NARROW>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ beta,
               const float *__restrict__ g, const OutArgs out, const float *__restrict__ s0,
-              float *__restrict__ s_final, const int *__restrict__ cu, int H, int Lrow, float scale, int dk_in,
-              int dv_in, long long wait_limit, unsigned *__restrict__ err_word) {
+              float *__restrict__ s_final, const int *__restrict__ cu, int H, int Lrow, float scale, int dk_arg,
+              int dv_arg, long long wait_limit, unsigned *__restrict__ err_word) {
+    static_assert(!(NARROW && OPTS), "the output options need dv = 128");
+    const int dk_in = NARROW ? dk_arg : kD, dv_in = NARROW ? dv_arg : kD;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned base derived by pointer arithmetic on the shared array, so the
     // compiler keeps every access below in the shared address space (LDS/STS)
@@ -841,11 +845,11 @@ bool make_qkv_map(CUtensorMap *m, const void *ptr, int L, int BH) { return make_
 
 namespace {
 
-template <bool GATED, bool OPTS>
+template <bool GATED, bool OPTS, bool NARROW = false>
 gdn_status_t launch_gdn_t(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const float *beta,
                           const float *g, const OutArgs &out, const float *s0, float *s_final, const int *cu,
                           int nctas, int H, int L, float scale, cudaStream_t stream, int dk = kD, int dv = kD) {
-    auto kern = tc_gdn_kernel<GATED, OPTS>;
+    auto kern = tc_gdn_kernel<GATED, OPTS, NARROW>;
     if (!ensure_smem_limit(reinterpret_cast<const void *>(kern), kSmemAlloc)) return GDN_ERR_CUDA;
     unsigned *err = device_error_word();
     if (!err) return GDN_ERR_CUDA;
@@ -892,8 +896,10 @@ gdn_status_t launch_tc_gdn_narrow(const void *q, const void *k, const void *v, c
     if (!make_rows_map(&mq, q, L, rows, dk) || !make_rows_map(&mk, k, L, rows, dk) ||
         !make_rows_map(&mv, v, L, rows, dv))
         return GDN_ERR_CUDA;
-    return g ? launch_gdn_t<true, false>(mq, mk, mv, beta, g, out, s0, s_final, cu, nctas, H, L, scale, stream, dk, dv)
-             : launch_gdn_t<false, false>(mq, mk, mv, beta, g, out, s0, s_final, cu, nctas, H, L, scale, stream, dk, dv);
+    return g ? launch_gdn_t<true, false, true>(mq, mk, mv, beta, g, out, s0, s_final, cu, nctas, H, L, scale, stream,
+                                               dk, dv)
+             : launch_gdn_t<false, false, true>(mq, mk, mv, beta, g, out, s0, s_final, cu, nctas, H, L, scale, stream,
+                                                dk, dv);
 }
 
 }  // namespace gdn

@@ -359,8 +359,8 @@ def measure_rows(gdn, peaks, peak_src, args):
     row = _row(w, ms, nb, fl, peaks, peak_src, "hbm", w.B * w.L, "gdn_prefill_vector_gate")
     row["path"] = "tensor cores: vg_prep_kernel (one CTA per chunk) + vg_chain_kernel (one CTA per head)"
     rows["gdn_prefill_vector_gate"] = row
-    # the same shape at head size 64 (dk = dv = 64): the tensor-core kernels through copies
-    # zero-padded to 128 (bytes and FLOP counted at d = 64, the call's own work)
+    # the same shape at head size 64 (dk = dv = 64): the one-CTA tensor-core kernel reading the
+    # 64-wide tiles directly (bytes and FLOP counted at d = 64, the call's own work)
     inp64 = W.make_prefill_inputs(w.B, w.H, w.L, 64, 64, mode="gdn", in_dtype=torch.bfloat16,
                                   seed=W.SEED_BASE + 8, device="cuda")
     o64 = torch.empty(w.B, w.H, w.L, 64, device="cuda")
@@ -372,7 +372,7 @@ def measure_rows(gdn, peaks, peak_src, args):
     fl64 = flops_per_head_token("gdn", 64, 64, w.chunk) * w.B * w.H * w.L
     row = _row(w, ms, nb64, fl64, peaks, peak_src, "hbm", w.B * w.L)
     row["workload"] = "gdn_bf16_B8_H16_L4096_d64"
-    row["path"] = "tc_gdn_kernel at 128 x 128 on zero-padded copies, cropped (pad_copy_kernel)"
+    row["path"] = "tc_gdn_kernel, narrow instantiation (64-wide tensor maps; the far tile halves load as zeros)"
     rows["gdn_prefill_d64"] = row
     del inp64, o64, sf64
     del inp, o, sf, gv

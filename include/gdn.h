@@ -23,8 +23,8 @@
  *    run (the pool keeps what it reserved for later calls): vector-valued gates on the
  *    tensor cores, Gated DeltaNet over few heads with long sequences (dense bf16 calls at
  *    dk = dv = 128, chunk 64, with at most a third of the SM count of (sequence, head)
- *    pairs and at least 128 chunks), and bf16 calls with dk or dv = 64 (zero-padded
- *    copies); if that memory cannot be had they run on kernels that need none. Otherwise the library allocates no memory and keeps no
+ *    pairs and at least 128 chunks), and bf16 calls with dk or dv = 64 that take
+ *    zero-padded copies (below); if that memory cannot be had they run on kernels that need none. Otherwise the library allocates no memory and keeps no
  *    per-call state; its only state is per device: the condition word that
  *    gdn_sync_status reads, cached kernel attributes, the wait limit of
  *    gdn_set_wait_limit_for_testing, the workspace pool and the two streams below.
@@ -81,7 +81,10 @@ typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype_t;
  *  kernels: at dk = dv = 128 directly, with dk or dv = 64 through copies of the operands
  *  zero-padded to 128 (the padded results, cropped, are the call's: zero key coordinates
  *  and value columns leave the other entries unchanged; a stream-ordered workspace from the
- *  library's pool, see Ownership; not with the output normalisation). Every other
+ *  library's pool, see Ownership; not with the output normalisation). Gated DeltaNet with
+ *  the plain fp32 output and a scalar gate (or none), on batches of enough (sequence, head)
+ *  pairs for the one-CTA kernel (more than a third of the SM count), reads the 64-wide
+ *  operands directly instead: the same bits, no copies and no workspace. Every other
  *  combination runs on the fp32 chunk kernel (the same result within its tolerance, at
  *  CUDA-core speed).
  *  scale multiplies q.  in_dtype: GDN_BF16 or GDN_F32 (q, k, v share it).

@@ -158,3 +158,16 @@ def test_direct_full_size_sampled_heads(lib):
         o_ref, s_ref = oracle.recurrent_fwd(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]), sl(inp["beta"]), sl(inp["g"]))
         assert _err(sl(o), o_ref) <= TOL, f"o head ({b},{h})"
         assert _err(sl(sf), s_ref) <= TOL, f"S head ({b},{h})"
+
+
+def test_direct_in_place_state(lib):
+    # S_final written over S0 (the same buffer) on the direct form: the kernel reads S0 before
+    # any chunk and writes S_final after the last
+    B, H, L = 4, 16, 100
+    inp = W.make_prefill_inputs(B, H, L, 64, 128, mode="gdn", in_dtype=torch.bfloat16, s0=True, seed=880)
+    q, k, v, beta, g = (inp[n].cuda() for n in ("q", "k", "v", "beta", "g"))
+    state = inp["s0"].cuda().clone()
+    o, sf = lib.gdn_chunk_fwd(q, k, v, beta, g, s0=state, s_final=state)
+    assert lib.gdn_sync_status() == 0
+    o_ref, s_ref = oracle.recurrent_fwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["g"], inp["s0"])
+    assert _err(o.cpu(), o_ref) <= TOL and _err(state.cpu(), s_ref) <= TOL

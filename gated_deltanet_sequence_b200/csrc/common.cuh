@@ -69,6 +69,31 @@ __device__ __forceinline__ SeqSpan seq_span(const int *cu, int bid, int H, int L
     return SeqSpan{h, a, b - a};
 }
 
+// Packed batches of at most this many sequences start their longest sequences first.
+constexpr int kLongestFirstMax = 256;
+
+// Block bid of a packed batch of nseq sequences -> state index n * H + h of the (sequence,
+// head) pair it takes: blocks r * H .. r * H + H - 1 take the sequence of rank r by length
+// (longest first, ties by index). Blocks start in index order as SMs free up, so the longest
+// sequences start first and the call ends about when its longest sequence does. A malformed
+// offset array still gives a permutation (the chosen sequence's offsets are checked after).
+__device__ __forceinline__ int longest_first(const int *__restrict__ cu, int bid, int H, int nseq) {
+    __shared__ int len[kLongestFirstMax];
+    __shared__ int pick;
+    if (nseq > kLongestFirstMax) return bid;
+    const int r = bid / H, h = bid - r * H;
+    for (int i = threadIdx.x; i < nseq; i += blockDim.x) len[i] = cu[i + 1] - cu[i];
+    __syncthreads();
+    for (int i = threadIdx.x; i < nseq; i += blockDim.x) {
+        const int li = len[i];
+        int rank = 0;
+        for (int k = 0; k < nseq; ++k) rank += (len[k] > li || (len[k] == li && k < i)) ? 1 : 0;
+        if (rank == r) pick = i;
+    }
+    __syncthreads();
+    return pick * H + h;
+}
+
 template <typename T> __device__ __forceinline__ float ld_in(const T *p);
 template <> __device__ __forceinline__ float ld_in<float>(const float *p) { return *p; }
 template <> __device__ __forceinline__ float ld_in<__nv_bfloat16>(const __nv_bfloat16 *p) {

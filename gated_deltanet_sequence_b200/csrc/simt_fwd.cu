@@ -88,9 +88,11 @@ simt_chunk_fwd_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const 
     Sm &sm = *reinterpret_cast<Sm *>(smem_raw);
     constexpr int KP = Sm::KP, CP = Sm::CP;
     const int tid = threadIdx.x;
-    const long bh = blockIdx.x;                  // (sequence, head): state index
+    // (sequence, head): state index; packed batches take their sequences longest first
+    const long bh = cu ? longest_first(cu, static_cast<int>(blockIdx.x), H, static_cast<int>(gridDim.x) / H)
+                       : static_cast<long>(blockIdx.x);
     const int c0 = blockIdx.y * kDvs;            // first value column of this CTA
-    const SeqSpan sp = seq_span(cu, blockIdx.x, H, Lrow, err);
+    const SeqSpan sp = seq_span(cu, static_cast<int>(bh), H, Lrow, err);
     const int L = sp.len;                        // tokens of this sequence
     const long r0 = (long)sp.head_row * Lrow + sp.t0;   // its first row in the token grid
 

@@ -126,31 +126,6 @@ enum : int {
     kNumBars = 20
 };
 
-// Packed batches of at most this many sequences start their longest sequences first.
-constexpr int kLongestFirstMax = 256;
-
-// Block bid of a packed batch of nseq sequences -> state index n * H + h of the (sequence,
-// head) pair it takes: blocks r * H .. r * H + H - 1 take the sequence of rank r by length
-// (longest first, ties by index). Blocks start in index order as SMs free up, so the longest
-// sequences start first and the call ends about when its longest sequence does. A malformed
-// offset array still gives a permutation (the chosen sequence's offsets are checked after).
-__device__ __forceinline__ int longest_first(const int *__restrict__ cu, int bid, int H, int nseq) {
-    __shared__ int len[kLongestFirstMax];
-    __shared__ int pick;
-    if (nseq > kLongestFirstMax) return bid;
-    const int r = bid / H, h = bid - r * H;
-    for (int i = threadIdx.x; i < nseq; i += blockDim.x) len[i] = cu[i + 1] - cu[i];
-    __syncthreads();
-    for (int i = threadIdx.x; i < nseq; i += blockDim.x) {
-        const int li = len[i];
-        int rank = 0;
-        for (int k = 0; k < nseq; ++k) rank += (len[k] > li || (len[k] == li && k < i)) ? 1 : 0;
-        if (rank == r) pick = i;
-    }
-    __syncthreads();
-    return pick * H + h;
-}
-
 // NARROW: head sizes dk_in, dv_in of 64 or 128 (tiles past them load as zeros; plain fp32
 // output only); otherwise both are 128 and the arguments are ignored.
 template <bool GATED, bool OPTS, bool NARROW>

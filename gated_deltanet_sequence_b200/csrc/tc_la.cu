@@ -133,7 +133,8 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     const Ctl ctl{bars, abort_flag, err_word, wait_limit};
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int bh = blockIdx.x;                          // (sequence, head): state index
+    // (sequence, head): state index; packed batches take their sequences longest first
+    const int bh = cu ? longest_first(cu, blockIdx.x, H, gridDim.x / H) : blockIdx.x;
     const SeqSpan sp = seq_span(cu, bh, H, Lrow, err_word);
     const int L = sp.len;                               // tokens of this sequence
     const int zc = sp.head_row, ty0 = sp.t0;            // TMA head and first-token coordinates

@@ -394,7 +394,7 @@ def measure_rows(gdn, peaks, peak_src, args):
     sf = torch.empty(w.B, w.H, w.dk, w.dv, device="cuda")
     fn = lambda: gdn.gdn_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["g"], o=o,
                                    s0=inp["s0"], s_final=sf, chunk=w.chunk)
-    ms = timed(fn, max(3, args.steps // 4), 2)
+    ms = timed(fn, max(10, args.steps // 2), 3)
     nb = prefill_bytes(w.B, w.H, w.L, w.dk, w.dv, 2, True, True, True, True)
     fl = flops_per_head_token("gdn", w.dk, w.dv, w.chunk) * w.B * w.H * w.L
     row = _row(w, ms, nb, fl, peaks, peak_src, "hbm", w.B * w.L, "gdn_prefill_long")

@@ -70,6 +70,10 @@ bool tc_gdn_takes_narrow(int nctas);
 gdn_status_t launch_tc_gdn_narrow(const void *q, const void *k, const void *v, const float *beta, const float *g,
                                   float *o, const float *s0, float *s_final, const int *cu, int B, int H, int L,
                                   int dk, int dv, float scale, cudaStream_t stream);
+// The same for linear attention on its kernel (tc_la.cu), which takes every batch.
+gdn_status_t launch_tc_la_narrow(const void *q, const void *k, const void *v, const float *g, float *o,
+                                 const float *s0, float *s_final, const int *cu, int B, int H, int L, int dk, int dv,
+                                 float scale, cudaStream_t stream);
 }  // namespace gdn
 
 extern "C" {
@@ -263,13 +267,18 @@ static gdn_status_t prefill_ex(bool delta, const void *q, const void *k, const v
     if (!opt_aligned4(beta)) return GDN_ERR_INVALID_ARG;
     if ((double)B * H * (double)L * dk > 9.0e18) return GDN_ERR_INVALID_ARG;   // g of (rows, dk)
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
-    // Gated DeltaNet at head size 64 with the plain fp32 output and a scalar gate, on batches the
-    // one-CTA tensor-core kernel takes: that kernel reads the 64-wide tiles directly (their
-    // halves past dk or dv load as zeros) and writes only dk x dv states and dv output columns,
-    // which gives the results of the zero-padded call below without its copies
-    if (delta && pad_applies(in_dtype, dk, dv, chunk, L) && (dk == 64 || dk == 128) && (dv == 64 || dv == 128) &&
-        !oo.bf16 && !oo.dskip && oo.xnorm == gdn::kXNormNone && !oo.gate_per_key && aligned16(q) && aligned16(k) && aligned16(v) &&
-        gdn::tc_gdn_takes_narrow(B * H) && (cu_seqlens || !gdn::tc_vg_takes_scalar(B, H, L)))
+    // Head size 64 with the plain fp32 output and a scalar gate, for linear attention and for
+    // Gated DeltaNet on batches its one-CTA tensor-core kernel takes: the kernel reads the
+    // 64-wide tiles directly (their halves past dk or dv load as zeros) and writes only dk x dv
+    // states and dv output columns, which gives the results of the zero-padded call below
+    // without its copies
+    const bool narrow = pad_applies(in_dtype, dk, dv, chunk, L) && (dk == 64 || dk == 128) &&
+                        (dv == 64 || dv == 128) && !oo.bf16 && !oo.dskip && oo.xnorm == gdn::kXNormNone &&
+                        !oo.gate_per_key && aligned16(q) && aligned16(k) && aligned16(v);
+    if (narrow && !delta)
+        return gdn::launch_tc_la_narrow(q, k, v, g, static_cast<float *>(o), s0, s_final, cu_seqlens, B, H, L, dk, dv,
+                                        scale, stream);
+    if (narrow && gdn::tc_gdn_takes_narrow(B * H) && (cu_seqlens || !gdn::tc_vg_takes_scalar(B, H, L)))
         return gdn::launch_tc_gdn_narrow(q, k, v, beta, g, static_cast<float *>(o), s0, s_final, cu_seqlens, B, H, L,
                                          dk, dv, scale, stream);
     if (pad_applies(in_dtype, dk, dv, chunk, L) && oo.xnorm == gdn::kXNormNone && rows_fit_int(cu_seqlens, B, H, L)) {

@@ -799,9 +799,8 @@ EncodeTiledFn encode_fn() {
 }
 
 // (BH, L, 128) bf16 -> 3-D map, 64 x 64 boxes, 128-byte swizzle, zero fill out of range.
-namespace {
 // (BH, L, width) bf16 rows, width 64 or 128, in 64 x 64 boxes: a box past the width (x = 64 of a
-// 64-wide tensor) loads as zeros
+// 64-wide tensor) loads as zeros (also used by the linear-attention kernel's narrow launch)
 bool make_rows_map(CUtensorMap *m, const void *ptr, int L, int BH, int width) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
@@ -814,7 +813,6 @@ bool make_rows_map(CUtensorMap *m, const void *ptr, int L, int BH, int width) {
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
-}  // namespace
 
 bool make_qkv_map(CUtensorMap *m, const void *ptr, int L, int BH) { return make_rows_map(m, ptr, L, BH, 128); }
 

@@ -116,12 +116,16 @@ __device__ __forceinline__ uint4 scale_chunk(uint4 x, float f) {
     return x;
 }
 
-template <bool GATED, bool OPTS>
+// NARROW: head sizes dk_arg, dv_arg of 64 or 128 (tiles past them load as zeros; plain fp32
+// output only); otherwise both are 128 and the arguments are ignored.
+template <bool GATED, bool OPTS, bool NARROW>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
              const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ g, const OutArgs out,
              const float *__restrict__ s0, float *__restrict__ s_final, const int *__restrict__ cu, int H,
-             int Lrow, float scale, long long wait_limit, unsigned *__restrict__ err_word) {
+             int Lrow, float scale, int dk_arg, int dv_arg, long long wait_limit, unsigned *__restrict__ err_word) {
+    static_assert(!(NARROW && OPTS), "the output options need dv = 128");
+    const int dk_in = NARROW ? dk_arg : kD, dv_in = NARROW ? dv_arg : kD;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned base derived by pointer arithmetic on the shared array, so the
     // compiler keeps every access below in the shared address space (LDS/STS)
@@ -316,13 +320,15 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
         float nf = 0.f;   // non-finite probe over the final state
         {
-            // S^T row v = column v of the initial state (a warp reads 32 consecutive floats)
-            const float *src = s0 ? s0 + static_cast<size_t>(bh) * kD * kD + v : nullptr;
+            // S^T row v = column v of the dk_in x dv_in initial state (a warp reads 32 consecutive
+            // floats; rows and columns beyond it are zero)
+            const float *src = s0 && v < dv_in ? s0 + static_cast<size_t>(bh) * dk_in * dv_in + v : nullptr;
 #pragma unroll 1
             for (int cc = 0; cc < 8; ++cc) {
                 float r[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) r[e] = src ? src[static_cast<size_t>(cc * 16 + e) * kD] : 0.f;
+                for (int e = 0; e < 16; ++e)
+                    r[e] = src && cc * 16 < dk_in ? src[static_cast<size_t>(cc * 16 + e) * dv_in] : 0.f;
                 tmem_st16(trow + TM_S + cc * 16, r);
             }
             tmem_wait_st();
@@ -358,31 +364,36 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             if (lead) mbar_arrive(&bars[B_SRDY]);
             done = c;
         }
+        // column v of the dk_in x dv_in final state (a warp writes 32 consecutive floats; lanes
+        // v >= dv_in are whole warps and store nothing)
         if (s_final && nchunks == 0) {
             // empty sequence: the final state is the initial one (TMEM holds it)
-            float *dst = s_final + static_cast<size_t>(bh) * kD * kD + v;
+            if (v < dv_in) {
+                float *dst = s_final + static_cast<size_t>(bh) * dk_in * dv_in + v;
 #pragma unroll 1
-            for (int cc = 0; cc < 8; ++cc) {
-                float sv[16];
-                tmem_ld16(trow + TM_S + cc * 16, sv);
-                tmem_wait_ld();
+                for (int cc = 0; cc < dk_in / 16; ++cc) {
+                    float sv[16];
+                    tmem_ld16(trow + TM_S + cc * 16, sv);
+                    tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 16; ++e) dst[static_cast<size_t>(cc * 16 + e) * kD] = sv[e];
+                    for (int e = 0; e < 16; ++e) dst[static_cast<size_t>(cc * 16 + e) * dv_in] = sv[e];
+                }
             }
         } else if (s_final && nchunks > 0 && done == nchunks - 1 &&
             ctl.group_wait(B_SDONE, (nchunks - 1) & 1, kBarState, lead, 128)) {
             tc_fence_after();
-            // column v of the final state (a warp writes 32 consecutive floats)
-            float *dst = s_final + static_cast<size_t>(bh) * kD * kD + v;
+            if (v < dv_in) {
+                float *dst = s_final + static_cast<size_t>(bh) * dk_in * dv_in + v;
 #pragma unroll 1
-            for (int cc = 0; cc < 8; ++cc) {
-                float sv[16];
-                tmem_ld16(trow + TM_S + cc * 16, sv);
-                tmem_wait_ld();
+                for (int cc = 0; cc < dk_in / 16; ++cc) {
+                    float sv[16];
+                    tmem_ld16(trow + TM_S + cc * 16, sv);
+                    tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    probe_finite(nf, sv[e]);
-                    dst[static_cast<size_t>(cc * 16 + e) * kD] = sv[e];
+                    for (int e = 0; e < 16; ++e) {
+                        probe_finite(nf, sv[e]);
+                        dst[static_cast<size_t>(cc * 16 + e) * dv_in] = sv[e];
+                    }
                 }
             }
         }
@@ -409,11 +420,11 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             if constexpr (OPTS) {
                 store_out_rows_group(ov, out, (row0 + static_cast<size_t>(c) * kC) * kD + v, n, head, v, kBarOut, xn,
                                      xn + 256, probe_chunk(c, nchunks), nf);
-            } else {
-                float *ocol = static_cast<float *>(out.o) + (row0 + static_cast<size_t>(c) * kC) * kD + v;
+            } else if (v < dv_in) {
+                float *ocol = static_cast<float *>(out.o) + (row0 + static_cast<size_t>(c) * kC) * dv_in + v;
 #pragma unroll
                 for (int r = 0; r < 64; ++r)
-                    if (r < n) ocol[static_cast<size_t>(r) * kD] = ov[r];
+                    if (r < n) ocol[static_cast<size_t>(r) * dv_in] = ov[r];
                 if (probe_chunk(c, nchunks)) probe_tile(nf, ov, n);
             }
         }
@@ -543,15 +554,15 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     }
 }
 
-template <bool GATED, bool OPTS>
+template <bool GATED, bool OPTS, bool NARROW = false>
 gdn_status_t launch_la_t(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const float *g,
                          const OutArgs &out, const float *s0, float *s_final, const int *cu, int nctas, int H,
-                         int L, float scale, cudaStream_t stream) {
-    auto kern = tc_la_kernel<GATED, OPTS>;
+                         int L, float scale, cudaStream_t stream, int dk = kD, int dv = kD) {
+    auto kern = tc_la_kernel<GATED, OPTS, NARROW>;
     if (!ensure_smem_limit(reinterpret_cast<const void *>(kern), kSmemAlloc)) return GDN_ERR_CUDA;
     unsigned *err = device_error_word();
     if (!err) return GDN_ERR_CUDA;
-    kern<<<nctas, kThreads, kSmemAlloc, stream>>>(mq, mk, mv, g, out, s0, s_final, cu, H, L, scale,
+    kern<<<nctas, kThreads, kSmemAlloc, stream>>>(mq, mk, mv, g, out, s0, s_final, cu, H, L, scale, dk, dv,
                                                   wait_limit_cycles(), err);
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
@@ -572,6 +583,27 @@ gdn_status_t launch_tc_la(const void *q, const void *k, const void *v, const flo
                        : launch_la_t<true, false>(mq, mk, mv, g, out, s0, s_final, cu, nctas, H, L, scale, stream);
     return opts ? launch_la_t<false, true>(mq, mk, mv, g, out, s0, s_final, cu, nctas, H, L, scale, stream)
                 : launch_la_t<false, false>(mq, mk, mv, g, out, s0, s_final, cu, nctas, H, L, scale, stream);
+}
+
+// 64- or 128-wide bf16 row tensor maps (tc_gdn.cu)
+bool make_rows_map(CUtensorMap *m, const void *ptr, int L, int BH, int width);
+
+// Head sizes of 64 (dk or dv; the other 64 or 128) with the plain fp32 output: 64-wide tensor
+// maps whose second 64-column box loads as zeros, so the kernel computes the zero-padded call
+// and stores only dk x dv states and dv output columns.
+gdn_status_t launch_tc_la_narrow(const void *q, const void *k, const void *v, const float *g, float *o,
+                                 const float *s0, float *s_final, const int *cu, int B, int H, int L, int dk, int dv,
+                                 float scale, cudaStream_t stream) {
+    const int nctas = B * H;
+    const FwdOpts plain{false, nullptr, false, kXNormNone, nullptr, 0.f};
+    const OutArgs out = make_out_args(o, v, plain);
+    const int rows = cu ? H : B * H;
+    CUtensorMap mq, mk, mv;
+    if (!make_rows_map(&mq, q, L, rows, dk) || !make_rows_map(&mk, k, L, rows, dk) ||
+        !make_rows_map(&mv, v, L, rows, dv))
+        return GDN_ERR_CUDA;
+    return g ? launch_la_t<true, false, true>(mq, mk, mv, g, out, s0, s_final, cu, nctas, H, L, scale, stream, dk, dv)
+             : launch_la_t<false, false, true>(mq, mk, mv, g, out, s0, s_final, cu, nctas, H, L, scale, stream, dk, dv);
 }
 
 }  // namespace gdn

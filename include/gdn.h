@@ -81,10 +81,11 @@ typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype_t;
  *  kernels: at dk = dv = 128 directly, with dk or dv = 64 through copies of the operands
  *  zero-padded to 128 (the padded results, cropped, are the call's: zero key coordinates
  *  and value columns leave the other entries unchanged; a stream-ordered workspace from the
- *  library's pool, see Ownership; not with the output normalisation). Gated DeltaNet with
- *  the plain fp32 output and a scalar gate (or none), on batches of enough (sequence, head)
- *  pairs for the one-CTA kernel (more than a third of the SM count), reads the 64-wide
- *  operands directly instead: the same bits, no copies and no workspace. Every other
+ *  library's pool, see Ownership; not with the output normalisation). Calls with the plain
+ *  fp32 output and a scalar gate (or none) read the 64-wide operands directly instead (the
+ *  same bits, no copies and no workspace): linear attention always, Gated DeltaNet on
+ *  batches of enough (sequence, head) pairs for its one-CTA kernel (more than a third of the
+ *  SM count). Every other
  *  combination runs on the fp32 chunk kernel (the same result within its tolerance, at
  *  CUDA-core speed).
  *  scale multiplies q.  in_dtype: GDN_BF16 or GDN_F32 (q, k, v share it).

@@ -171,3 +171,22 @@ def test_direct_in_place_state(lib):
     assert lib.gdn_sync_status() == 0
     o_ref, s_ref = oracle.recurrent_fwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["g"], inp["s0"])
     assert _err(o.cpu(), o_ref) <= TOL and _err(state.cpu(), s_ref) <= TOL
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (64, 128), (128, 64)])
+@pytest.mark.parametrize("gated", [True, False])
+def test_direct_linear_attention_matches_padded(lib, dk, dv, gated):
+    # linear attention with the plain fp32 output reads the 64-wide tiles directly on any batch;
+    # a zero skip term takes the padded copies: both must give the same bits
+    B, H, L = 2, 3, 200
+    inp = W.make_prefill_inputs(B, H, L, dk, dv, mode="la", in_dtype=torch.bfloat16, s0=True, seed=890 + dk + dv,
+                                gated=gated)
+    q, k, v, s0 = (inp[n].cuda() for n in ("q", "k", "v", "s0"))
+    g = inp["g"].cuda() if gated else None
+    o, sf = lib.lin_attn_chunk_fwd(q, k, v, g, s0=s0, s_final=torch.empty(B, H, dk, dv, device="cuda"))
+    op, sfp = lib.lin_attn_chunk_fwd(q, k, v, g, s0=s0, s_final=torch.empty(B, H, dk, dv, device="cuda"),
+                                     d_skip=torch.zeros(H, dv, device="cuda"))
+    assert lib.gdn_sync_status() == 0
+    assert torch.equal(o, op) and torch.equal(sf, sfp), "direct and padded forms differ"
+    o_ref, s_ref = oracle.recurrent_fwd(inp["q"], inp["k"], inp["v"], None, inp["g"] if gated else None, inp["s0"])
+    assert _err(o.cpu(), o_ref) <= TOL and _err(sf.cpu(), s_ref) <= TOL

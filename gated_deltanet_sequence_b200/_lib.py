@@ -5,7 +5,8 @@ contiguity, their data pointers and sizes are passed to the C entry points, and 
 non-OK status raises. Every step of the computation runs in the library's CUDA
 kernels; there is no other code path. The library must be built
 (``python -m gated_deltanet_sequence_b200.build``); if it is missing, importing this
-module raises ImportError.
+module raises ImportError. With GDN_LIBRARY=debug in the environment the bounds-checked
+build (libgdn_debug.so, ``build --debug-bounds``) is loaded instead.
 """
 from __future__ import annotations
 
@@ -16,9 +17,9 @@ from typing import Optional
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libgdn.so")
+LIB_PATH = os.path.join(_HERE, "libgdn_debug.so" if os.environ.get("GDN_LIBRARY") == "debug" else "libgdn.so")
 
-GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_TIMEOUT, GDN_ERR_NONFINITE = range(6)
+GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_TIMEOUT, GDN_ERR_NONFINITE, GDN_ERR_BOUNDS = range(7)
 GDN_F32, GDN_BF16 = 0, 1
 
 EXPORTS = ("lin_attn_chunk_fwd", "gdn_chunk_fwd", "lin_attn_chunk_fwd_varlen", "gdn_chunk_fwd_varlen",
@@ -47,7 +48,7 @@ class GdnError(RuntimeError):
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"libgdn.so is not built ({LIB_PATH}); run "
+        raise ImportError(f"{os.path.basename(LIB_PATH)} is not built ({LIB_PATH}); run "
                           "`python -m gated_deltanet_sequence_b200.build`")
     lib = ctypes.CDLL(LIB_PATH)
     P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float

@@ -154,6 +154,7 @@ const char *gdn_status_str(gdn_status_t s) {
         case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
         case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT";
         case GDN_ERR_NONFINITE: return "GDN_ERR_NONFINITE";
+        case GDN_ERR_BOUNDS: return "GDN_ERR_BOUNDS";
     }
     return "GDN_ERR_UNKNOWN";
 }

@@ -9,9 +9,23 @@
 namespace gdn {
 
 // Codes a kernel ORs into the device-side error word (the word lives in the
-// tensor-core translation unit): a bounded wait gave up, or a packed batch's
-// sequence offsets were not a non-decreasing list inside [0, T].
-enum : unsigned { kErrWaitTimeout = 1u, kErrBadSeqlens = 2u, kErrNonFinite = 4u };
+// tensor-core translation unit): a bounded wait gave up, a packed batch's sequence offsets
+// were not a non-decreasing list inside [0, T], a stored result was not finite, or (debug
+// builds) an access index fell outside the extent its launch implies.
+enum : unsigned { kErrWaitTimeout = 1u, kErrBadSeqlens = 2u, kErrNonFinite = 4u, kErrBounds = 8u };
+
+// Bounds checks of the debug build (-DGDN_DEBUG_BOUNDS): in_bounds(i, n, err) is true for
+// 0 <= i < n; otherwise it sets kErrBounds in the error word and the caller skips the access
+// (nothing traps). Release builds compile every check to true.
+#ifdef GDN_DEBUG_BOUNDS
+__device__ __forceinline__ bool in_bounds(long long i, long long n, unsigned *err) {
+    if (i >= 0 && i < n) return true;
+    if (err) atomicOr(err, kErrBounds);
+    return false;
+}
+#else
+__device__ __forceinline__ bool in_bounds(long long, long long, unsigned *) { return true; }
+#endif
 
 // Non-finite detector for stored results: nf <- nf + 0 * x keeps nf at 0 for finite x and
 // turns it into NaN for an infinite or NaN x (0 * inf = NaN), one FMA per value (IEEE

@@ -21,12 +21,14 @@ namespace {
 std::atomic<long long> g_wait_limit{kWaitLimitCycles};
 
 // Reports one condition and clears only that bit, atomically: a malformed sequence-offset
-// list first, then a bounded wait that gave up, then a non-finite stored result. Bits set
-// meanwhile by kernels on other streams stay in the word.
+// list first, then a bounded wait that gave up, then (debug builds) an access out of its
+// extent, then a non-finite stored result. Bits set meanwhile by kernels on other streams
+// stay in the word.
 __global__ void take_error_kernel(unsigned *word, unsigned *taken) {
     const unsigned now = atomicOr(word, 0u);
     const unsigned bit = (now & kErrBadSeqlens)    ? kErrBadSeqlens
                          : (now & kErrWaitTimeout) ? kErrWaitTimeout
+                         : (now & kErrBounds)      ? kErrBounds
                                                    : (now & kErrNonFinite);
     if (bit) atomicAnd(word, ~bit);
     *taken = bit;
@@ -100,6 +102,7 @@ gdn_status_t gdn_sync_status(void *cuda_stream) {
     if (!gdn::take_device_error(stream, &err)) return GDN_ERR_CUDA;
     if (err & gdn::kErrBadSeqlens) return GDN_ERR_INVALID_ARG;
     if (err & gdn::kErrWaitTimeout) return GDN_ERR_TIMEOUT;
+    if (err & gdn::kErrBounds) return GDN_ERR_BOUNDS;
     return err ? GDN_ERR_NONFINITE : GDN_OK;
 }
 

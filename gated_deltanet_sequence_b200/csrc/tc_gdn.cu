@@ -155,6 +155,10 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const int zc = sp.head_row, ty0 = sp.t0;            // TMA head and first-token coordinates
     const int nchunks = (L + kC - 1) / kC;
     const size_t row0 = static_cast<size_t>(zc) * Lrow + ty0;   // first token row in the grid
+    // extents the launch implies (bounds checks of the debug build): token rows of the grid, and
+    // state elements
+    const long long n_rows = static_cast<long long>(cu ? H : gridDim.x) * Lrow;
+    const long long n_state = static_cast<long long>(gridDim.x) * dk_in * dv_in;
 
     if (tid == 0) {
         for (int b = 0; b < kNumBars; ++b) mbar_init(&bars[b], 1);
@@ -299,8 +303,11 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 float r[16];
 #pragma unroll
                 for (int e = 0; e < 16; e += 4) {
-                    const float4 x = src && cc * 16 < dv_in ? *reinterpret_cast<const float4 *>(src + cc * 16 + e)
-                                                            : make_float4(0.f, 0.f, 0.f, 0.f);
+                    const bool in = src && cc * 16 < dv_in &&
+                                    in_bounds((static_cast<long long>(bh) * dk_in + j) * dv_in + cc * 16 + e + 3, n_state,
+                                              err_word);
+                    const float4 x = in ? *reinterpret_cast<const float4 *>(src + cc * 16 + e)
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
                     r[e] = x.x; r[e + 1] = x.y; r[e + 2] = x.z; r[e + 3] = x.w;
                 }
                 tmem_st16(trow + TM_S + cc * 16, r);
@@ -328,7 +335,9 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 float *ocol = static_cast<float *>(out.o) + (row0 + static_cast<size_t>(cp) * kC) * dv_in + j;
 #pragma unroll
                 for (int r = 0; r < 64; ++r)
-                    if (r < n) ocol[static_cast<size_t>(r) * dv_in] = ov[r];
+                    if (r < n && in_bounds((static_cast<long long>(row0) + cp * kC + r) * dv_in + j, n_rows * dv_in,
+                                           err_word))
+                        ocol[static_cast<size_t>(r) * dv_in] = ov[r];
                 if (probe) probe_tile(nf, ov, n);
             }
         };
@@ -451,7 +460,8 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
                 for (int e = 0; e < 16; e += 4) {
                     probe_finite(nf, sv[e] + sv[e + 1] + sv[e + 2] + sv[e + 3]);
-                    *reinterpret_cast<float4 *>(dst + cc * 16 + e) = make_float4(sv[e], sv[e + 1], sv[e + 2], sv[e + 3]);
+                    if (in_bounds((static_cast<long long>(bh) * dk_in + j) * dv_in + cc * 16 + e + 3, n_state, err_word))
+                        *reinterpret_cast<float4 *>(dst + cc * 16 + e) = make_float4(sv[e], sv[e + 1], sv[e + 2], sv[e + 3]);
                 }
             }
         }
@@ -718,7 +728,7 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
             const int t = 2 * lane + e;
-            if (t < L) {
+            if (t < L && in_bounds(static_cast<long long>(row0) + t, n_rows, err_word)) {
                 if (GATED) g_nx[e] = g[row0 + t];
                 b_nx[e] = beta[row0 + t];
             }
@@ -739,8 +749,9 @@ tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 const int t = (c + 1) * kC + 2 * lane + e;
-                g_nx[e] = (GATED && c + 1 < nchunks && t < L) ? g[row0 + t] : 0.f;
-                b_nx[e] = (c + 1 < nchunks && t < L) ? beta[row0 + t] : 0.f;
+                const bool in = c + 1 < nchunks && t < L && in_bounds(static_cast<long long>(row0) + t, n_rows, err_word);
+                g_nx[e] = (GATED && in) ? g[row0 + t] : 0.f;
+                b_nx[e] = in ? beta[row0 + t] : 0.f;
             }
             // inclusive scan of the 64 log-decays (pairs, then a warp scan of pair sums)
             float x = g0 + g1;

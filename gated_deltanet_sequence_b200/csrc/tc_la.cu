@@ -144,6 +144,10 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     const int zc = sp.head_row, ty0 = sp.t0;            // TMA head and first-token coordinates
     const int nchunks = (L + kC - 1) / kC;
     const size_t row0 = static_cast<size_t>(zc) * Lrow + ty0;   // first token row in the grid
+    // extents the launch implies (bounds checks of the debug build): token rows of the grid, and
+    // state elements
+    const long long n_rows = static_cast<long long>(cu ? H : gridDim.x) * Lrow;
+    const long long n_state = static_cast<long long>(gridDim.x) * dk_in * dv_in;
 
     if (tid == 0) {
         for (int b = 0; b < kNumBars; ++b) mbar_init(&bars[b], 1);
@@ -225,7 +229,8 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             float g_nx[2] = {0.f, 0.f};
 #pragma unroll
             for (int e = 0; e < 2; ++e)
-                if (2 * lane + e < L) g_nx[e] = g[row0 + 2 * lane + e];
+                if (2 * lane + e < L && in_bounds(static_cast<long long>(row0) + 2 * lane + e, n_rows, err_word))
+                    g_nx[e] = g[row0 + 2 * lane + e];
 #pragma unroll 1
             for (int c = 0; c < nchunks; ++c) {
                 const int p = c & 1;
@@ -240,7 +245,8 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     const int t = (c + 1) * kC + 2 * lane + e;
-                    g_nx[e] = (c + 1 < nchunks && t < L) ? g[row0 + t] : 0.f;
+                    g_nx[e] = (c + 1 < nchunks && t < L && in_bounds(static_cast<long long>(row0) + t, n_rows, err_word))
+                                  ? g[row0 + t] : 0.f;
                 }
                 float x = g0 + g1;
 #pragma unroll
@@ -328,7 +334,10 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 float r[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
-                    r[e] = src && cc * 16 < dk_in ? src[static_cast<size_t>(cc * 16 + e) * dv_in] : 0.f;
+                    r[e] = src && cc * 16 < dk_in &&
+                                   in_bounds(static_cast<long long>(bh) * dk_in * dv_in + static_cast<long long>(cc * 16 + e) * dv_in + v,
+                                             n_state, err_word)
+                               ? src[static_cast<size_t>(cc * 16 + e) * dv_in] : 0.f;
                 tmem_st16(trow + TM_S + cc * 16, r);
             }
             tmem_wait_st();
@@ -376,7 +385,10 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     tmem_ld16(trow + TM_S + cc * 16, sv);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) dst[static_cast<size_t>(cc * 16 + e) * dv_in] = sv[e];
+                    for (int e = 0; e < 16; ++e)
+                        if (in_bounds(static_cast<long long>(bh) * dk_in * dv_in + static_cast<long long>(cc * 16 + e) * dv_in + v,
+                                      n_state, err_word))
+                            dst[static_cast<size_t>(cc * 16 + e) * dv_in] = sv[e];
                 }
             }
         } else if (s_final && nchunks > 0 && done == nchunks - 1 &&
@@ -392,7 +404,9 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
                         probe_finite(nf, sv[e]);
-                        dst[static_cast<size_t>(cc * 16 + e) * dv_in] = sv[e];
+                        if (in_bounds(static_cast<long long>(bh) * dk_in * dv_in + static_cast<long long>(cc * 16 + e) * dv_in + v,
+                                      n_state, err_word))
+                            dst[static_cast<size_t>(cc * 16 + e) * dv_in] = sv[e];
                     }
                 }
             }
@@ -424,7 +438,8 @@ tc_la_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 float *ocol = static_cast<float *>(out.o) + (row0 + static_cast<size_t>(c) * kC) * dv_in + v;
 #pragma unroll
                 for (int r = 0; r < 64; ++r)
-                    if (r < n) ocol[static_cast<size_t>(r) * dv_in] = ov[r];
+                    if (r < n && in_bounds((static_cast<long long>(row0) + c * kC + r) * dv_in + v, n_rows * dv_in, err_word))
+                        ocol[static_cast<size_t>(r) * dv_in] = ov[r];
                 if (probe_chunk(c, nchunks)) probe_tile(nf, ov, n);
             }
         }

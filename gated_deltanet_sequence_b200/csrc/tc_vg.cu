@@ -679,6 +679,9 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
     // the chunk with index c of the launch start at row0 + c * C
     const size_t row0 = static_cast<size_t>(bh) * L + static_cast<size_t>(cbase) * kC;
     const int Lrem = L - cbase * kC;                         // tokens from the launch's first chunk on
+    // extents the launch implies (bounds checks of the debug build): output and state elements
+    const long long n_out = static_cast<long long>(gridDim.x) * L * kD;
+    const long long n_state = static_cast<long long>(gridDim.x) * kD * kD;
     const bool seq_end = cbase + nch == (L + kC - 1) / kC;   // the launch ends the sequence
     const long long rec0 = static_cast<long long>(bh) * nch;
 
@@ -736,7 +739,10 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
             for (int cc = 0; cc < 4; ++cc) {
                 float rr[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) rr[e] = src ? src[static_cast<size_t>(cc * 16 + e) * kD] : 0.f;
+                for (int e = 0; e < 16; ++e)
+                    rr[e] = src && in_bounds((static_cast<long long>(bh) * kD + 64 * half + cc * 16 + e) * kD + v, n_state,
+                                             err_word)
+                                ? src[static_cast<size_t>(cc * 16 + e) * kD] : 0.f;
                 tmem_st16(trow + TMC_S + 64 * half + cc * 16, rr);
             }
             tmem_wait_st();
@@ -904,7 +910,8 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
                         probe_finite(nf, t[e]);
-                        dst[static_cast<size_t>(cc * 16 + e) * kD] = t[e];
+                        if (in_bounds((static_cast<long long>(bh) * kD + 64 * half + cc * 16 + e) * kD + v, n_state, err_word))
+                            dst[static_cast<size_t>(cc * 16 + e) * kD] = t[e];
                     }
                 }
             }
@@ -938,7 +945,8 @@ vg_chain_kernel(const uint8_t *__restrict__ recs, const float *__restrict__ egl,
                 float *ocol = static_cast<float *>(out.o) + elem0;
 #pragma unroll
                 for (int r = 0; r < 64; ++r)
-                    if (r < n) ocol[static_cast<size_t>(r) * kD] = ov[r];
+                    if (r < n && in_bounds(static_cast<long long>(elem0) + static_cast<long long>(r) * kD, n_out, err_word))
+                        ocol[static_cast<size_t>(r) * kD] = ov[r];
                 if (last && seq_end) probe_tile(nf, ov, n);
             }
         }

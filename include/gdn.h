@@ -56,8 +56,10 @@ typedef enum {
     GDN_ERR_UNSUPPORTED = 2,   /* valid but not implemented (head dim, chunk, dtype)  */
     GDN_ERR_CUDA = 3,          /* a CUDA runtime/driver call or launch failed          */
     GDN_ERR_TIMEOUT = 4,       /* a kernel gave up on a bounded wait (see sync_status) */
-    GDN_ERR_NONFINITE = 5      /* a tensor-core prefill stored inf / NaN in o or S_final
+    GDN_ERR_NONFINITE = 5,     /* a tensor-core prefill stored inf / NaN in o or S_final
                                   (checked on a sample, see sync_status)               */
+    GDN_ERR_BOUNDS = 6         /* bounds-checked debug build only: a kernel index fell
+                                  outside its extent; the access was skipped            */
 } gdn_status_t;
 
 typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype_t;
@@ -368,7 +370,9 @@ const char *gdn_status_str(gdn_status_t status);
  * gdn_sync_status — synchronise `cuda_stream`, then report and clear one device-side
  * condition met by a kernel of this library on the current device since it was last
  * reported, in this order: GDN_ERR_INVALID_ARG for a malformed cu_seqlens list,
- * GDN_ERR_TIMEOUT for a bounded wait that gave up, GDN_ERR_NONFINITE when a tensor-core
+ * GDN_ERR_TIMEOUT for a bounded wait that gave up, GDN_ERR_BOUNDS (only in the library built
+ * with -DGDN_DEBUG_BOUNDS, libgdn_debug.so) when a kernel's global access index fell outside
+ * the extent its launch implies, GDN_ERR_NONFINITE when a tensor-core
  * prefill kernel found inf or NaN among the results it stored (non-finite inputs, or an
  * intermediate beyond the fp16 operand range, |x| > 65504, of those kernels). The kernels
  * check the last 64-token output tile of each sequence and its final state: a non-finite

@@ -40,10 +40,24 @@ def test_library_exports_every_declared_symbol(lib):
         assert hasattr(raw, name), f"libgdn.so does not export {name}"
 
 
+def test_debug_library_exports_the_same_symbols(lib):
+    # the bounds-checked build (python -m gated_deltanet_sequence_b200.build --debug-bounds)
+    path = os.path.join(os.path.dirname(lib.LIB_PATH), "libgdn_debug.so")
+    if not os.path.exists(path):
+        pytest.skip("libgdn_debug.so is not built")
+    raw = ctypes.CDLL(path)
+    for name in lib.EXPORTS:
+        assert hasattr(raw, name), f"libgdn_debug.so does not export {name}"
+    raw.gdn_status_str.argtypes = [ctypes.c_int]
+    raw.gdn_status_str.restype = ctypes.c_char_p
+    assert raw.gdn_status_str(6) == b"GDN_ERR_BOUNDS"
+
+
 def test_status_strings_and_version(lib):
     assert lib.status_str(0) == "GDN_OK"
     assert lib.status_str(4) == "GDN_ERR_TIMEOUT"
     assert lib.status_str(5) == "GDN_ERR_NONFINITE"
+    assert lib.status_str(6) == "GDN_ERR_BOUNDS"
     assert lib.status_str(99) == "GDN_ERR_UNKNOWN"
     assert lib.gdn_version() >= 100
 

@@ -1,0 +1,70 @@
+"""The bounds-checked debug build (libgdn_debug.so, -DGDN_DEBUG_BOUNDS): its kernels check the
+index of each thread-side global access of inputs, outputs and states against the extent the
+launch implies and report GDN_ERR_BOUNDS instead of making an out-of-range access. On valid
+calls it must report nothing and give the release build's results bit for bit: the tensor-core
+prefill kernels (one-CTA Gated DeltaNet dense and packed, the head-size-64 direct form, linear
+attention, the vector-gate prep and chain kernels, the segmented long-sequence path) run once in
+a child process on the debug library and once here on the release library."""
+import os
+import subprocess
+import sys
+
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+CHILD = r'''
+import sys, torch
+sys.path.insert(0, sys.argv[1])
+from gated_deltanet_sequence_b200 import _lib as gdn, workloads as W
+out = {}
+torch.cuda.set_device(0)
+inp = W.make_prefill_inputs(4, 16, 200, 128, 128, mode="gdn", in_dtype=torch.bfloat16, s0=True, seed=901, device="cuda")
+out["gdn"] = gdn.gdn_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["g"], s0=inp["s0"],
+                              s_final=torch.empty_like(inp["s0"]))
+out["la"] = gdn.lin_attn_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["g"], s0=inp["s0"],
+                                   s_final=torch.empty_like(inp["s0"]))
+gv = W.make_gate_per_key((4, 16), 200, 128, seed=902, device="cuda")
+out["vec"] = gdn.gdn_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["beta"], gv, s0=inp["s0"],
+                               s_final=torch.empty_like(inp["s0"]))
+d64 = W.make_prefill_inputs(4, 16, 130, 64, 64, mode="gdn", in_dtype=torch.bfloat16, s0=True, seed=903, device="cuda")
+out["d64"] = gdn.gdn_chunk_fwd(d64["q"], d64["k"], d64["v"], d64["beta"], d64["g"], s0=d64["s0"],
+                               s_final=torch.empty_like(d64["s0"]))
+lens = [0, 1, 64, 65, 130, 300, 7, 191]
+vl = W.make_varlen_inputs(lens, 8, 128, 128, mode="gdn", in_dtype=torch.bfloat16, s0=True, seed=904, device="cuda")
+out["varlen"] = gdn.gdn_chunk_fwd_varlen(vl["q"], vl["k"], vl["v"], vl["beta"], vl["cu_seqlens"], vl["g"],
+                                         s0=vl["s0"], s_final=torch.empty_like(vl["s0"]))
+lg = W.make_prefill_inputs(1, 2, 64 * 130 + 17, 128, 128, mode="gdn", in_dtype=torch.bfloat16, s0=True, seed=905,
+                           device="cuda")
+out["long"] = gdn.gdn_chunk_fwd(lg["q"], lg["k"], lg["v"], lg["beta"], lg["g"], s0=lg["s0"],
+                                s_final=torch.empty_like(lg["s0"]))
+status = gdn.gdn_sync_status()
+torch.save({"status": status, "lib": gdn.LIB_PATH,
+            "out": {k: tuple(t.cpu() for t in v) for k, v in out.items()}}, sys.argv[2])
+'''
+
+
+def _run(tmp_path, debug):
+    env = dict(os.environ)
+    if debug:
+        env["GDN_LIBRARY"] = "debug"
+    else:
+        env.pop("GDN_LIBRARY", None)
+    path = str(tmp_path / ("debug.pt" if debug else "release.pt"))
+    subprocess.run([sys.executable, "-c", CHILD, ROOT, path], env=env, check=True, timeout=600)
+    return torch.load(path)
+
+
+def test_debug_build_reports_nothing_and_matches_release(tmp_path):
+    if not os.path.exists(os.path.join(ROOT, "gated_deltanet_sequence_b200", "libgdn_debug.so")):
+        pytest.fail("libgdn_debug.so is not built (python -m gated_deltanet_sequence_b200.build --debug-bounds)")
+    dbg = _run(tmp_path, True)
+    rel = _run(tmp_path, False)
+    assert dbg["lib"].endswith("libgdn_debug.so") and rel["lib"].endswith("libgdn.so")
+    assert dbg["status"] == 0, f"debug build reported status {dbg['status']}"
+    assert rel["status"] == 0
+    for k in rel["out"]:
+        for a, b in zip(dbg["out"][k], rel["out"][k]):
+            assert torch.equal(a, b), f"{k}: debug and release builds differ"

@@ -17,6 +17,7 @@
 // columns (float4) of RPT rows strided by the number of row groups, so every
 // warp-wide access is a contiguous 256-512 B run of one or two state rows.
 #include "common.cuh"
+#include "tc_kernels.cuh"
 
 namespace gdn {
 namespace {
@@ -30,7 +31,7 @@ decode_step_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
                    const float *__restrict__ beta, const float *__restrict__ g,
                    float *__restrict__ state, void *__restrict__ o, float scale, int H, int vec,
                    int out_bf16, const float *__restrict__ dskip, int xnorm, const float *__restrict__ xw,
-                   float xeps) {
+                   float xeps, unsigned *__restrict__ err) {
     constexpr int CG = DV / 4;               // float4 column groups
     constexpr int RG = kDecThreads / CG;     // row groups
     constexpr int RPT = DK / RG;             // rows per thread
@@ -46,21 +47,28 @@ decode_step_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
     const int tid = threadIdx.x;
     const int cg = tid % CG, rg = tid / CG;
     float *S = state + head * (long)DK * DV;
+    // extents the launch implies (bounds checks of the debug build)
+    const long long nh = gridDim.x;
 
     // stream the state rows into registers first (independent 16 B loads)
     float4 sreg[RPT];
 #pragma unroll
-    for (int i = 0; i < RPT; ++i) sreg[i] = ld_global4(S + (long)(rg + RG * i) * DV + 4 * cg);
+    for (int i = 0; i < RPT; ++i)
+        sreg[i] = in_bounds((head * DK + rg + RG * i) * (long long)DV + 4 * cg + 3, nh * DK * DV, err)
+                      ? ld_global4(S + (long)(rg + RG * i) * DV + 4 * cg) : make_float4(0.f, 0.f, 0.f, 0.f);
 
     for (int i = tid; i < DK; i += kDecThreads) {
-        s_k[i] = ld_in(k + head * DK + i);
-        s_q[i] = scale * ld_in(q + head * DK + i);
+        const bool in = in_bounds(head * DK + i, nh * DK, err);
+        s_k[i] = in ? ld_in(k + head * DK + i) : 0.f;
+        s_q[i] = in ? scale * ld_in(q + head * DK + i) : 0.f;
     }
-    for (int i = tid; i < DV; i += kDecThreads) s_v[i] = ld_in(v + head * DV + i);
+    for (int i = tid; i < DV; i += kDecThreads) s_v[i] = in_bounds(head * DV + i, nh * DV, err) ? ld_in(v + head * DV + i) : 0.f;
     if (vg)
-        for (int i = tid; i < DK; i += kDecThreads) s_a[i] = g ? expf(g[head * DK + i]) : 1.f;
-    const float alpha = (g && !vg) ? expf(g[head]) : 1.f;
-    const float bt = DELTA ? beta[head] : 0.f;
+        for (int i = tid; i < DK; i += kDecThreads)
+            s_a[i] = g && in_bounds(head * DK + i, nh * DK, err) ? expf(g[head * DK + i]) : 1.f;
+    const bool head_in = in_bounds(head, nh, err);
+    const float alpha = (g && !vg && head_in) ? expf(g[head]) : 1.f;
+    const float bt = DELTA && head_in ? beta[head] : 0.f;
     __syncthreads();
 
     // partial S^T k and S^T q' over this thread's rows
@@ -114,8 +122,9 @@ decode_step_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
         ov.y = fmaf(alpha, sq[1], qk * u[1]);
         ov.z = fmaf(alpha, sq[2], qk * u[2]);
         ov.w = fmaf(alpha, sq[3], qk * u[3]);
+        const bool o_in = in_bounds(head * DV + 4 * cg + 3, nh * DV, err);
         if (!OPT) {
-            st_global4(static_cast<float *>(o) + head * DV + 4 * cg, ov);
+            if (o_in) st_global4(static_cast<float *>(o) + head * DV + 4 * cg, ov);
         } else {
             if (dskip) {        // skip term D_h v (head = sequence * H + h)
                 const float *dh = dskip + (head % H) * DV + 4 * cg;
@@ -145,13 +154,13 @@ decode_step_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
                 ov.z *= rs * (wh ? wh[2] : 1.f);
                 ov.w *= rs * (wh ? wh[3] : 1.f);
             }
-            if (out_bf16) {
+            if (o_in && out_bf16) {
                 __nv_bfloat16 *ob = static_cast<__nv_bfloat16 *>(o) + head * DV + 4 * cg;
                 ob[0] = __float2bfloat16_rn(ov.x);
                 ob[1] = __float2bfloat16_rn(ov.y);
                 ob[2] = __float2bfloat16_rn(ov.z);
                 ob[3] = __float2bfloat16_rn(ov.w);
-            } else {
+            } else if (o_in) {
                 st_global4(static_cast<float *>(o) + head * DV + 4 * cg, ov);
             }
         }
@@ -166,7 +175,7 @@ decode_step_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const IT 
         s.y = fmaf(aj, s.y, kj * u[1]);
         s.z = fmaf(aj, s.z, kj * u[2]);
         s.w = fmaf(aj, s.w, kj * u[3]);
-        st_global4(S + (long)j * DV + 4 * cg, s);
+        if (in_bounds((head * DK + j) * (long long)DV + 4 * cg + 3, nh * DK * DV, err)) st_global4(S + (long)j * DV + 4 * cg, s);
     }
 }
 
@@ -175,14 +184,16 @@ gdn_status_t launch_dec_t(const void *q, const void *k, const void *v, const flo
                           const float *g, float *state, void *o, long NH, int H, float scale, const FwdOpts &oo,
                           cudaStream_t stream) {
     const int vec = oo.gate_per_key ? 1 : 0, ob = oo.bf16 ? 1 : 0;
+    unsigned *err = device_error_word();
+    if (!err) return GDN_ERR_CUDA;
     if (beta)
         decode_step_kernel<DK, DV, IT, true, OPT><<<(unsigned)NH, kDecThreads, 0, stream>>>(
             (const IT *)q, (const IT *)k, (const IT *)v, beta, g, state, o, scale, H, vec, ob, oo.dskip, oo.xnorm,
-            oo.xw, oo.xeps);
+            oo.xw, oo.xeps, err);
     else
         decode_step_kernel<DK, DV, IT, false, OPT><<<(unsigned)NH, kDecThreads, 0, stream>>>(
             (const IT *)q, (const IT *)k, (const IT *)v, beta, g, state, o, scale, H, vec, ob, oo.dskip, oo.xnorm,
-            oo.xw, oo.xeps);
+            oo.xw, oo.xeps, err);
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 

@@ -3,8 +3,8 @@ index of each thread-side global access of inputs, outputs and states against th
 launch implies and report GDN_ERR_BOUNDS instead of making an out-of-range access. On valid
 calls it must report nothing and give the release build's results bit for bit: the tensor-core
 prefill kernels (one-CTA Gated DeltaNet dense and packed, the head-size-64 direct form, linear
-attention, the vector-gate prep and chain kernels, the segmented long-sequence path) run once in
-a child process on the debug library and once here on the release library."""
+attention, the vector-gate prep and chain kernels, the segmented long-sequence path) and three
+decode steps run in a child process on each library."""
 import os
 import subprocess
 import sys
@@ -40,6 +40,12 @@ lg = W.make_prefill_inputs(1, 2, 64 * 130 + 17, 128, 128, mode="gdn", in_dtype=t
                            device="cuda")
 out["long"] = gdn.gdn_chunk_fwd(lg["q"], lg["k"], lg["v"], lg["beta"], lg["g"], s0=lg["s0"],
                                 s_final=torch.empty_like(lg["s0"]))
+dec = W.make_decode_inputs(16, 8, 128, 128, 3, seed=906, device="cuda")
+state = dec["state"].clone()
+outs = []
+for t in range(3):
+    outs.append(gdn.gdn_decode_step(dec["q"][t], dec["k"][t], dec["v"][t], dec["beta"][t], dec["g"][t], state))
+out["decode"] = (torch.stack(outs), state)
 status = gdn.gdn_sync_status()
 torch.save({"status": status, "lib": gdn.LIB_PATH,
             "out": {k: tuple(t.cpu() for t in v) for k, v in out.items()}}, sys.argv[2])

@@ -103,11 +103,15 @@ simt_chunk_fwd_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const 
     const float *bh_g = (g && !VEC) ? g + r0 : nullptr;
     const float *bh_gv = (g && VEC) ? g + r0 * DK : nullptr;   // (L, DK) log-decays per key
     const long o0 = r0 * dv;                     // first output element of the sequence
+    // extents the launch implies (bounds checks of the debug build): token rows of the grid, and
+    // state elements
+    const long long n_rows = static_cast<long long>(cu ? H : gridDim.x) * Lrow;
+    const long long n_state = static_cast<long long>(gridDim.x) * DK * dv;
     const float *dsk = dskip ? dskip + static_cast<long>(sp.head_row % H) * dv + c0 : nullptr;
 
     for (int i = tid; i < DK * kDvs; i += kSimtThreads) {
         const int j = i / kDvs, c = i % kDvs;
-        sm.S[i] = s0 ? s0[(bh * DK + j) * dv + c0 + c] : 0.f;
+        sm.S[i] = s0 && in_bounds((bh * DK + j) * dv + c0 + c, n_state, err) ? s0[(bh * DK + j) * dv + c0 + c] : 0.f;
     }
 
     int round = 0;   // reduction rounds across the cluster (output normalisation)
@@ -117,12 +121,13 @@ simt_chunk_fwd_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const 
         // ---- load the chunk ------------------------------------------------
         for (int i = tid; i < n * DK; i += kSimtThreads) {
             const int r = i / DK, j = i % DK;
-            sm.K[r * KP + j] = ld_in(kh + (long)(t0 + r) * DK + j);
-            sm.Q[r * KP + j] = scale * ld_in(qh + (long)(t0 + r) * DK + j);
+            const bool in = in_bounds((r0 + t0 + r) * DK + j, n_rows * DK, err);
+            sm.K[r * KP + j] = in ? ld_in(kh + (long)(t0 + r) * DK + j) : 0.f;
+            sm.Q[r * KP + j] = in ? scale * ld_in(qh + (long)(t0 + r) * DK + j) : 0.f;
         }
         for (int i = tid; i < n * kDvs; i += kSimtThreads) {
             const int r = i / kDvs, c = i % kDvs;
-            sm.V[i] = ld_in(vh + (long)(t0 + r) * dv + c0 + c);
+            sm.V[i] = in_bounds((r0 + t0 + r) * dv + c0 + c, n_rows * dv, err) ? ld_in(vh + (long)(t0 + r) * dv + c0 + c) : 0.f;
         }
         int wide = 0;   // a cumulative log-decay of this chunk is outside [-60, 60]
         if (VEC) {
@@ -130,7 +135,8 @@ simt_chunk_fwd_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const 
             // inclusive within-chunk cumulative sum of g[:, j], in place
             for (int i = tid; i < n * DK; i += kSimtThreads) {
                 const int r = i / DK, j = i % DK;
-                sm.GV[r * KP + j] = bh_gv ? bh_gv[(long)(t0 + r) * DK + j] : 0.f;
+                sm.GV[r * KP + j] = bh_gv && in_bounds((r0 + t0 + r) * DK + j, n_rows * DK, err)
+                                        ? bh_gv[(long)(t0 + r) * DK + j] : 0.f;
             }
             __syncthreads();
             if (tid < DK) {
@@ -147,7 +153,7 @@ simt_chunk_fwd_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const 
             float carry = 0.f;
             for (int base = 0; base < n; base += 32) {
                 const int r = base + tid;
-                float x = (bh_g && r < n) ? bh_g[t0 + r] : 0.f;
+                float x = (bh_g && r < n && in_bounds(r0 + t0 + r, n_rows, err)) ? bh_g[t0 + r] : 0.f;
                 for (int off = 1; off < 32; off <<= 1) {
                     const float y = __shfl_up_sync(0xffffffffu, x, off);
                     if (tid >= off) x += y;
@@ -157,7 +163,7 @@ simt_chunk_fwd_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const 
             }
         } else if (DELTA && tid >= 64 && tid < 64 + kCmax) {
             const int r = tid - 64;
-            if (r < n) sm.bt[r] = bh_beta[t0 + r];
+            if (r < n) sm.bt[r] = in_bounds(r0 + t0 + r, n_rows, err) ? bh_beta[t0 + r] : 0.f;
         }
         const bool direct = VEC && __syncthreads_or(wide);   // VEC: direct exp per decay factor
         if (!VEC) __syncthreads();
@@ -289,7 +295,8 @@ simt_chunk_fwd_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const 
                 continue;
             }
             const long oi = o0 + (long)(t0 + r) * dv + c0 + c;
-            if (out_bf16) static_cast<__nv_bfloat16 *>(o)[oi] = __float2bfloat16_rn(ov);
+            if (!in_bounds(oi, n_rows * dv, err)) {
+            } else if (out_bf16) static_cast<__nv_bfloat16 *>(o)[oi] = __float2bfloat16_rn(ov);
             else static_cast<float *>(o)[oi] = ov;
         }
         __syncthreads();
@@ -319,7 +326,8 @@ simt_chunk_fwd_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const 
                 const float y = x * rsqrtf(ms + xeps) * wc;
                 if (r < n) {
                     const long oi = o0 + (long)(t0 + r) * dv + c0 + lane;
-                    if (out_bf16) static_cast<__nv_bfloat16 *>(o)[oi] = __float2bfloat16_rn(y);
+                    if (!in_bounds(oi, n_rows * dv, err)) {
+                    } else if (out_bf16) static_cast<__nv_bfloat16 *>(o)[oi] = __float2bfloat16_rn(y);
                     else static_cast<float *>(o)[oi] = y;
                 }
             }
@@ -348,7 +356,7 @@ simt_chunk_fwd_kernel(const IT *__restrict__ q, const IT *__restrict__ k, const 
     if (s_final) {
         for (int i = tid; i < DK * kDvs; i += kSimtThreads) {
             const int j = i / kDvs, c = i % kDvs;
-            s_final[(bh * DK + j) * dv + c0 + c] = sm.S[i];
+            if (in_bounds((bh * DK + j) * dv + c0 + c, n_state, err)) s_final[(bh * DK + j) * dv + c0 + c] = sm.S[i];
         }
     }
 }

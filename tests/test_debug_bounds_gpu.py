@@ -3,8 +3,9 @@ index of each thread-side global access of inputs, outputs and states against th
 launch implies and report GDN_ERR_BOUNDS instead of making an out-of-range access. On valid
 calls it must report nothing and give the release build's results bit for bit: the tensor-core
 prefill kernels (one-CTA Gated DeltaNet dense and packed, the head-size-64 direct form, linear
-attention, the vector-gate prep and chain kernels, the segmented long-sequence path) and three
-decode steps run in a child process on each library."""
+attention, the vector-gate prep and chain kernels, the segmented long-sequence path), the fp32
+chunk kernel (dense, vector gates, packed) and three decode steps run in a child process on each
+library."""
 import os
 import subprocess
 import sys
@@ -40,6 +41,16 @@ lg = W.make_prefill_inputs(1, 2, 64 * 130 + 17, 128, 128, mode="gdn", in_dtype=t
                            device="cuda")
 out["long"] = gdn.gdn_chunk_fwd(lg["q"], lg["k"], lg["v"], lg["beta"], lg["g"], s0=lg["s0"],
                                 s_final=torch.empty_like(lg["s0"]))
+f32 = W.make_prefill_inputs(2, 3, 150, 128, 64, mode="gdn", in_dtype=torch.float32, s0=True, seed=907, device="cuda")
+out["f32"] = gdn.gdn_chunk_fwd(f32["q"], f32["k"], f32["v"], f32["beta"], f32["g"], s0=f32["s0"],
+                               s_final=torch.empty_like(f32["s0"]))
+gv32 = W.make_gate_per_key((2, 3), 150, 128, seed=908, device="cuda")
+out["f32vec"] = gdn.gdn_chunk_fwd(f32["q"], f32["k"], f32["v"], f32["beta"], gv32, s0=f32["s0"],
+                                  s_final=torch.empty_like(f32["s0"]))
+vl32 = W.make_varlen_inputs([5, 70, 0, 140], 2, 64, 64, mode="gdn", in_dtype=torch.float32, s0=True, seed=909,
+                            device="cuda")
+out["f32varlen"] = gdn.gdn_chunk_fwd_varlen(vl32["q"], vl32["k"], vl32["v"], vl32["beta"], vl32["cu_seqlens"],
+                                            vl32["g"], s0=vl32["s0"], s_final=torch.empty_like(vl32["s0"]))
 dec = W.make_decode_inputs(16, 8, 128, 128, 3, seed=906, device="cuda")
 state = dec["state"].clone()
 outs = []
